@@ -1,0 +1,506 @@
+#!/usr/bin/env python
+"""Benchmark of the paged KV-cache hot path on B200.
+
+One step = one pass of the hot path over one batch of the 4k-token decode
+workload (batch 16 x 4096 tokens, 32 q / 8 KV heads, head_dim 128, block 16,
+bf16): copy-on-write block copy (none are due in this workload: no block is
+shared), the KV-cache append of the batch's 16 new tokens, then paged decode
+attention over all 4096 tokens of every request.  Inputs are synthetic
+(seeded N(0,1) values, randomly permuted block pool) and resident in HBM
+before the timed region.  Each step uses the next of 4 layer pools (268 MB of
+K+V each, 1.07 GB in all), so every step reads KV that is not in the 126 MB L2.
+
+Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle (the
+only other implementation of the path) on a bounded sample instead.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU: launched by torchrun, one rank per GPU; every rank runs its own
+replica (independent requests, no data-path collective), timing is the max
+over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "paged decode attention KV GB/s (fraction of HBM peak) and tokens/s at 1 B200"
+UNIT = "GB/s"
+WORKLOAD = "gqa_4k: batch 16 x 4096 tokens, 32 q / 8 KV heads, head_dim 128, block 16, bf16"
+FALLBACK_HBM_GBS = 6650.0
+N_LAYERS = 4
+DECODE_SRC = os.path.join(ROOT, "paged_kv_cache_412_b200", "csrc", "decode_simt.cu")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_gqa_4k_traffic.txt")
+
+
+# ---------------------------------------------------------------------------
+# byte model of one step (the decode's algorithmic bytes; the append's bytes
+# are reported beside it)
+# ---------------------------------------------------------------------------
+
+def decode_bytes(B, L, Hq, Hkv, d, e_kv=2, e_q=2, e_out=2):
+    """K and V of every token once per kv head, plus q and out."""
+    return 2 * B * L * Hkv * d * e_kv + B * Hq * d * (e_q + e_out)
+
+
+def write_bytes(T, Hkv, d, e=2):
+    """Read the new K and V rows, write them into the cache."""
+    return 2 * 2 * T * Hkv * d * e
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def traffic_per_launch():
+    """DRAM bytes per decode launch from the committed ncu summary, or None if
+    the summary is missing or was taken on a different kernel source."""
+    try:
+        src_hash = hashlib.sha256(open(DECODE_SRC, "rb").read()).hexdigest()[:16]
+        vals = {}
+        for line in open(TRAFFIC_FILE):
+            if "=" in line and not line.lstrip().startswith("#"):
+                k, v = line.split("=", 1)
+                vals[k.strip()] = v.split("#")[0].strip()
+        if vals.get("decode_source_sha256_16") != src_hash:
+            return None
+        return int(float(vals["dram_bytes_per_launch"]))
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (only for --gpus > 1 under torchrun)
+# ---------------------------------------------------------------------------
+
+def dist_setup(n_gpus: int):
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def dist_max(value: float, world: int) -> float:
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def dist_barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def dist_done(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------------
+# CPU baseline: the oracle, as it stands, on a bounded sample
+# ---------------------------------------------------------------------------
+
+def cpu_baseline(budget_s: float = 12.0, per_call_cap_s: float | None = None) -> dict:
+    """Time the oracle (write + decode) on whole requests of the same workload
+    until about ``budget_s`` seconds of CPU work; report KV GB/s by the same
+    byte formula as the GPU line."""
+    import oracle
+    import workloads
+    w = workloads.gqa_4k(poison=False, seed=2002, batch=4)
+    lib = oracle.load()
+    threads = oracle.max_threads(lib)
+    total_bytes = 0
+    calls = 0
+    reqs = 0
+    t_all = 0.0
+    while t_all < budget_s:
+        b = calls % w.B
+        sl = slice(b, b + 1)
+        kc, vc = w.k_cache, w.v_cache
+        t0 = time.perf_counter()
+        oracle.kv_cache_write(w.k_new[sl], w.v_new[sl], w.slot_mapping[sl], kc, vc, lib=lib)
+        oracle.decode(w.q[sl], kc, vc, w.block_tables[sl], w.seq_lens[sl], w.scale, lib=lib)
+        t_all += time.perf_counter() - t0
+        total_bytes += decode_bytes(1, 4096, 32, 8, 128)
+        calls += 1
+        reqs += 1
+        if per_call_cap_s is not None and t_all > per_call_cap_s:
+            break
+    gbs = total_bytes / t_all / 1e9
+    return {"value": round(gbs, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{reqs} whole requests of the 4k workload (4096 tokens x 32 q / 8 KV "
+                      f"heads each), fp64 C oracle with OpenMP over (request, head), "
+                      f"{t_all:.1f} s of CPU time",
+            "seconds": round(t_all, 3)}
+
+
+def run_reference(args, rank: int, world: int):
+    """--impl reference: the CPU oracle on a bounded sample per step."""
+    if rank != 0:
+        return
+    import oracle
+    import workloads
+    w = workloads.gqa_4k(poison=False, seed=2002, batch=4)
+    lib = oracle.load()
+    threads = oracle.max_threads(lib)
+    budget_total = 150.0
+    per_step = max(budget_total / max(args.steps + args.warmup, 1), 0.0)
+    # calibrate the sample: whole requests if affordable, else the first
+    # kv-head group(s) of one request (all 4096 tokens)
+    b = 0
+    sl = slice(0, 1)
+    t0 = time.perf_counter()
+    oracle.decode(w.q[sl], w.k_cache, w.v_cache, w.block_tables[sl], w.seq_lens[sl], w.scale,
+                  lib=lib)
+    t_req = time.perf_counter() - t0
+    G = w.Hq // w.Hkv
+    if per_step >= t_req:
+        nreq = max(1, min(w.B, int(per_step // t_req)))
+        groups = w.Hkv
+    else:
+        nreq = 1
+        groups = max(1, min(w.Hkv, int(per_step / (t_req / w.Hkv))))
+    # sub-problem for `groups` kv heads: slice the cache's kv-head axis once
+    kc = np.ascontiguousarray(w.k_cache[:, :groups])
+    vc = np.ascontiguousarray(w.v_cache[:, :groups])
+    q = np.ascontiguousarray(w.q[:nreq, : groups * G])
+    knew = np.ascontiguousarray(w.k_new[:nreq, :groups])
+    vnew = np.ascontiguousarray(w.v_new[:nreq, :groups])
+    bt, sls, sm = w.block_tables[:nreq], w.seq_lens[:nreq], w.slot_mapping[:nreq]
+
+    def step():
+        oracle.kv_cache_write(knew, vnew, sm, kc, vc, lib=lib)
+        oracle.decode(q, kc, vc, bt, sls, w.scale, lib=lib)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    step_bytes = decode_bytes(nreq, 4096, groups * G, groups, 128)
+    value = step_bytes * args.steps / dt / 1e9
+    sample = (f"{nreq} request(s) x {groups} of 8 kv-head groups ({groups * G} q heads) x "
+              f"4096 tokens per step")
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": UNIT,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "sample": sample, "l2": "n/a (host)"},
+            "cpu_baseline": {"value": round(value, 4), "unit": UNIT, "cores": threads,
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 4), "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0},
+            "tokens_per_s": round(nreq * args.steps / dt, 3)}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# our implementation
+# ---------------------------------------------------------------------------
+
+def run_ours(args, rank: int, world: int, local: int):
+    import torch
+    import paged_kv_cache_412_b200 as pkv
+    import workloads
+
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    B, L, Hq, Hkv, d, bs = 16, 4096, 32, 8, 128, 16
+
+    # --- inputs resident in HBM: N_LAYERS layer pools of the same workload ---
+    layers = []
+    for li in range(N_LAYERS):
+        w = workloads.gqa_4k(poison=False, seed=1002 + 100 * rank + li)
+        t = {}
+        t["q"] = torch.from_numpy(w.q.view(np.int16)).to(dev).view(torch.bfloat16)
+        t["kc"] = torch.from_numpy(w.k_cache.view(np.int16)).to(dev).view(torch.bfloat16)
+        t["vc"] = torch.from_numpy(w.v_cache.view(np.int16)).to(dev).view(torch.bfloat16)
+        t["bt"] = torch.from_numpy(w.block_tables).to(dev)
+        t["sl"] = torch.from_numpy(w.seq_lens).to(dev)
+        t["kn"] = torch.from_numpy(w.k_new.view(np.int16)).to(dev).view(torch.bfloat16)
+        t["vn"] = torch.from_numpy(w.v_new.view(np.int16)).to(dev).view(torch.bfloat16)
+        t["sm"] = torch.from_numpy(w.slot_mapping).to(dev)
+        t["host"] = w
+        layers.append(t)
+        del w
+    out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev)
+    ws_bytes = pkv.decode_workspace_bytes(B, Hq, Hkv, d, bs, L, 0)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    no_pairs = torch.empty((0, 2), dtype=torch.int64, device=dev)
+    scale = 1.0 / math.sqrt(d)
+
+    def step(i, ev=None):
+        t = layers[i % N_LAYERS]
+        pkv.copy_blocks(t["kc"], t["vc"], no_pairs)  # no shared block to fork here
+        pkv.kv_cache_write(t["kn"], t["vn"], t["sm"], t["kc"], t["vc"])
+        if ev is not None:
+            ev[0].record()
+        pkv.paged_attention_decode(t["q"], t["kc"], t["vc"], t["bt"], t["sl"], bs, scale, out,
+                                   max_seq_len=L, workspace=ws)
+        if ev is not None:
+            ev[1].record()
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert pkv.get_device_error() == 0
+
+    # --- timed region: K steps, device-timed ---
+    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler.start()
+    time.sleep(0.3)
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    start.record()
+    for i in range(args.steps):
+        step(i, evs[i])
+    stop.record()
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    clocks = sampler.stop()
+    ms_total = start.elapsed_time(stop)
+    decode_ms = [a.elapsed_time(b) for a, b in evs]
+    ms_total_max = dist_max(ms_total, world)
+    ms_step = ms_total_max / args.steps
+
+    dbytes = decode_bytes(B, L, Hq, Hkv, d)
+    wbytes = write_bytes(B, Hkv, d)
+    value = dbytes * args.steps * world / (ms_total_max / 1e3) / 1e9
+    dec_avg_ms = statistics.fmean(decode_ms)
+    dec_med_ms = statistics.median(decode_ms)
+    peak, peak_kind = measured_peak()
+    achieved = dbytes / (dec_avg_ms / 1e3) / 1e9
+
+    # --- e2e: host inputs -> device, the step, result -> host, per step ---
+    t0l = layers[0]
+    hw = t0l["host"]
+    pin = lambda a: torch.from_numpy(a).pin_memory()
+    h_q = pin(hw.q.view(np.int16))
+    h_kn = pin(hw.k_new.view(np.int16))
+    h_vn = pin(hw.v_new.view(np.int16))
+    h_sm = pin(hw.slot_mapping)
+    h_bt = pin(hw.block_tables)
+    h_sl = pin(hw.seq_lens)
+    h_out = torch.empty((B, Hq, d), dtype=torch.int16).pin_memory()
+    d_q = torch.empty_like(t0l["q"]).view(torch.int16)
+    d_kn = torch.empty_like(t0l["kn"]).view(torch.int16)
+    d_vn = torch.empty_like(t0l["vn"]).view(torch.int16)
+    d_sm = torch.empty_like(t0l["sm"])
+    d_bt = torch.empty_like(t0l["bt"])
+    d_sl = torch.empty_like(t0l["sl"])
+    h2d = sum(x.numel() * x.element_size() for x in (h_q, h_kn, h_vn, h_sm, h_bt, h_sl))
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step(li):
+        t = layers[li % N_LAYERS]
+        d_q.copy_(h_q, non_blocking=True)
+        d_kn.copy_(h_kn, non_blocking=True)
+        d_vn.copy_(h_vn, non_blocking=True)
+        d_sm.copy_(h_sm, non_blocking=True)
+        d_bt.copy_(h_bt, non_blocking=True)
+        d_sl.copy_(h_sl, non_blocking=True)
+        pkv.copy_blocks(t["kc"], t["vc"], no_pairs)
+        pkv.kv_cache_write(d_kn.view(torch.bfloat16), d_vn.view(torch.bfloat16), d_sm, t["kc"],
+                           t["vc"])
+        pkv.paged_attention_decode(d_q.view(torch.bfloat16), t["kc"], t["vc"], d_bt, d_sl, bs,
+                                   scale, out, max_seq_len=L, workspace=ws)
+        h_out.copy_(out.view(torch.int16), non_blocking=True)
+        torch.cuda.current_stream().synchronize()
+
+    e2e_steps = max(10, min(args.steps, 2000))
+    for i in range(5):
+        e2e_step(i)
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(e2e_steps):
+        e2e_step(i)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = dist_max(e0.elapsed_time(e1), world)
+    e2e_value = dbytes * e2e_steps * world / (e2e_ms / 1e3) / 1e9
+    assert pkv.get_device_error() == 0
+
+    # --- one parity spot check of the timed path against the oracle ---
+    parity = None
+    if rank == 0 and not args.no_check:
+        parity = spot_check(pkv, layers[0], out, ws, scale)
+
+    result = None
+    if rank == 0:
+        cpu = cpu_baseline() if (world == 1 and not args.no_cpu_baseline) else None
+        result = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "config": {"workload": WORKLOAD, "global_batch": B * world, "seq_len": L,
+                       "num_q_heads": Hq, "num_kv_heads": Hkv, "head_dim": d, "block_size": bs,
+                       "layers_rotated": N_LAYERS,
+                       "l2": f"inputs larger than L2: {N_LAYERS} layer pools of "
+                             f"{2 * B * L * Hkv * d * 2 / 1e6:.0f} MB K+V rotated per step",
+                       "parallelism": f"replica x{world}" if world > 1 else "single GPU",
+                       "step": "copy_blocks (0 pairs) + kv_cache_write (16 tokens) + "
+                               "paged_attention_decode"},
+            "tokens_per_s": round(B * world * args.steps / (ms_total_max / 1e3), 1),
+            "context_tokens_per_s": round(B * L * world * args.steps / (ms_total_max / 1e3), 1),
+            "fraction_of_hbm_peak": round(value / peak, 4),
+            "decode_ms_avg": round(dec_avg_ms, 5), "decode_ms_median": round(dec_med_ms, 5),
+            "write_and_launch_ms_per_step": round(ms_step - dec_avg_ms, 5),
+            "bytes_per_step": {"decode_algorithmic": dbytes, "write": wbytes},
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
+                         "unit": "GB/s", "frac": round(achieved / peak, 4),
+                         "traffic": traffic_per_launch(),
+                         "kernel": "paged_attention_decode (split kernel + merge kernel)",
+                         "peak_kind": f"{peak_kind} HBM copy bandwidth"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                    "ms_per_step": round(e2e_ms / e2e_steps, 5),
+                    "note": "pinned host inputs copied in and output copied out every step, "
+                            "with a stream synchronize per step"},
+            "gpu_launches": 3 * args.steps,
+            "clocks": clocks,
+            "parity_spot_check": parity,
+        }
+        print(json.dumps(result), flush=True)
+    dist_barrier(world)
+    return result
+
+
+def spot_check(pkv, t, out, ws, scale):
+    """Compare a few outputs of the timed configuration with the oracle."""
+    import torch
+    import oracle
+    w = t["host"]
+    kc, vc = w.k_cache.copy(), w.v_cache.copy()
+    oracle.kv_cache_write(w.k_new, w.v_new, w.slot_mapping, kc, vc)
+    rows = [0, 7, 15]
+    ref = oracle.decode(w.q[rows], kc, vc, w.block_tables[rows], w.seq_lens[rows], w.scale)
+    pkv.kv_cache_write(t["kn"], t["vn"], t["sm"], t["kc"], t["vc"])
+    pkv.paged_attention_decode(t["q"], t["kc"], t["vc"], t["bt"], t["sl"], 16, scale, out,
+                               max_seq_len=4096, workspace=ws)
+    got = out.float().cpu().numpy()[rows].astype(np.float64)
+    err = np.abs(got - ref)
+    ok = bool(np.all(err <= 2e-3 + 1e-2 * np.abs(ref)))
+    return {"requests": rows, "max_abs": float(err.max()), "pass": ok}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-check", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        # The oracle runs on the host of rank 0 only; other ranks have no work
+        # and leave without joining a process group.
+        if int(os.environ.get("RANK", "0")) == 0:
+            run_reference(args, 0, int(os.environ.get("WORLD_SIZE", "1")))
+        return
+    rank, world, local = dist_setup(args.gpus)
+    try:
+        run_ours(args, rank, world, local)
+    finally:
+        dist_barrier(world)
+        dist_done(world)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,192 @@
+/*
+ * pkv.h -- C ABI of the B200 paged KV-cache library (sm_100a).
+ *
+ * The library implements the data-parallel hot path of PagedAttention:
+ *   - pkv_kv_cache_write          scatter each new token's K/V into its slot;
+ *   - pkv_paged_attention_decode  single-query decode attention over a cache
+ *                                 held in fixed-size physical blocks reached
+ *                                 through a per-request block table;
+ *   - pkv_copy_blocks             copy-on-write copy of shared blocks.
+ *
+ * Sources (web pages on the subject; cited by title and section):
+ *   [KVOPT]  "KV Cache Optimization and PagedAttention" (intro prose).
+ *   [PAMEM]  "PagedAttention: Optimizing KV Cache Utilization in Large Language
+ *            Models": "The Mechanics of PagedAttention", "The Math: Block
+ *            Attention Calculation", "Serving Advantages", "Conclusion".
+ *   [KVMGMT] "KV Cache Management": "The Solution: PagedAttention (vLLM)",
+ *            "The Bonus: Zero-Copy Sharing", "Watch Out For".
+ *
+ * Conventions shared by every call
+ *   - Pointers are DEVICE pointers of the current CUDA device unless a comment
+ *     says "host".  The caller owns and allocates all memory; the library
+ *     allocates nothing (decode scratch is a caller-provided workspace).
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream).  The returned status reports host-side validation and
+ *     launch errors only.
+ *   - Cache layout: k_cache / v_cache are [num_blocks, num_kv_heads,
+ *     block_size, head_dim], row-major, so each (block, kv head) is one
+ *     contiguous block_size*head_dim run.  The token at logical position t of a
+ *     request lives in physical block block_tables[b][t / block_size] at offset
+ *     t % block_size; a slot id is physical_block * block_size + offset.
+ *   - Query head h reads kv head h / (num_q_heads / num_kv_heads).
+ *   - Indices the device finds out of range (a slot, a block id, a sequence
+ *     longer than its block table) are skipped and raise a bit in a per-device
+ *     error word; pkv_get_device_error reads and clears it.  Kernels never trap.
+ *   - Supported: head_dim 64 or 128; block_size a power of two in [1, 256];
+ *     element types PKV_F32 and PKV_BF16 (decode, write, copy) and
+ *     PKV_FP8_E4M3 caches (see the fp8 calls).
+ */
+#ifndef PKV_H_
+#define PKV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t, spelled without the CUDA headers. */
+typedef struct CUstream_st* pkv_stream_t;
+
+typedef enum pkv_status {
+    PKV_OK = 0,
+    PKV_ERR_INVALID_ARG = 1,   /* null pointer, bad size, inconsistent dims      */
+    PKV_ERR_UNSUPPORTED = 2,   /* valid but not implemented (dtype, head_dim...) */
+    PKV_ERR_WORKSPACE = 3,     /* workspace null or smaller than required        */
+    PKV_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed           */
+    PKV_ERR_DEVICE_INDEX = 5   /* pkv_get_device_error found a device-side flag  */
+} pkv_status;
+
+typedef enum pkv_dtype {
+    PKV_F32 = 0,
+    PKV_BF16 = 1,
+    PKV_FP8_E4M3 = 2
+} pkv_dtype;
+
+/* Bits of the device error word (pkv_get_device_error). */
+#define PKV_DEVERR_BAD_SLOT 0x1u       /* write: slot >= num_blocks*block_size      */
+#define PKV_DEVERR_BAD_BLOCK 0x2u      /* decode: table entry outside [0,num_blocks) */
+#define PKV_DEVERR_BAD_SEQ_LEN 0x4u    /* decode: seq_len < 0 or > max_blocks*bs    */
+#define PKV_DEVERR_BAD_PAIR 0x8u       /* copy/swap: block id out of range          */
+#define PKV_DEVERR_TIMEOUT 0x10u       /* a bounded in-kernel wait gave up          */
+
+/* Human-readable name of a status code (static string). */
+const char* pkv_status_string(pkv_status status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int pkv_version(void);
+
+/*
+ * pkv_kv_cache_write -- append new tokens' K and V to the paged cache.
+ *
+ * [PAMEM] "The Mechanics of PagedAttention": as tokens are generated, their K
+ * and V vectors are written into the request's allocated physical blocks,
+ * wherever those blocks sit in memory.
+ *
+ *   k, v          [num_tokens, num_kv_heads, head_dim], element type dtype.
+ *   slot_mapping  [num_tokens] int64; token t goes to block slot/block_size at
+ *                 offset slot%block_size.  slot < 0 marks padding: skipped.
+ *                 slot >= num_blocks*block_size: skipped, PKV_DEVERR_BAD_SLOT.
+ *                 Slots must be distinct within one call (else the result of
+ *                 the colliding tokens is unspecified).
+ *   k_cache, v_cache  [num_blocks, num_kv_heads, block_size, head_dim].
+ * The copy is bit-exact.  num_tokens == 0 launches nothing and returns PKV_OK.
+ */
+pkv_status pkv_kv_cache_write(const void* k, const void* v, const int64_t* slot_mapping,
+                              void* k_cache, void* v_cache, int32_t num_tokens,
+                              int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                              int32_t num_blocks, pkv_dtype dtype, pkv_stream_t stream);
+
+/*
+ * pkv_decode_workspace_bytes -- bytes of device scratch that
+ * pkv_paged_attention_decode needs for these sizes on the CURRENT device.
+ * max_seq_len bounds every seq_lens entry of the calls that will use it;
+ * partition_size as in the decode call (0 = automatic).  Returns 0 for
+ * invalid sizes.
+ */
+size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
+                                  int32_t num_kv_heads, int32_t head_dim,
+                                  int32_t block_size, int32_t max_seq_len,
+                                  int32_t partition_size);
+
+/*
+ * pkv_paged_attention_decode -- one decode step of attention for a batch.
+ *
+ * [PAMEM] "The Math: Block Attention Calculation": for query q_i the page
+ * table gives the physical location of every key K_j and the scores are
+ * Softmax(q_i K^T / sqrt(d_k)).  The printed per-block softmax is read as the
+ * block's slice of ONE softmax over all of the request's tokens; the output
+ * is that softmax applied to the V rows:
+ *     out[b,h,:] = sum_t softmax_t(scale * q[b,h,:] . K_t) V_t
+ * over the seq_lens[b] tokens of request b (seq_lens counts the token
+ * appended this step).  seq_lens[b] == 0 gives an all-zero row.
+ *
+ *   q             [num_seqs, num_q_heads, head_dim], element type q_dtype
+ *                 (PKV_F32 with an fp32 cache, PKV_BF16 with bf16/fp8 caches).
+ *   k_cache, v_cache  cache layout above, element type kv_dtype.
+ *   block_tables  [num_seqs, max_blocks_per_seq] int32; entries past
+ *                 ceil(seq_len/block_size) are never read.
+ *   seq_lens      [num_seqs] int32.
+ *   out           [num_seqs, num_q_heads, head_dim], element type out_dtype
+ *                 (PKV_F32 or PKV_BF16; round to nearest even).
+ *   k_scale, v_scale  [num_kv_heads] fp32 dequantisation scales for an fp8
+ *                 cache (value = code * scale); NULL otherwise.
+ *   scale         softmax scale (1/sqrt(head_dim) for standard attention).
+ *   max_seq_len   an upper bound of seq_lens (sizes the workspace check).
+ *   partition_size  0 = automatic split of the whole batch's KV into equal
+ *                 shares, one per resident CTA; else tokens per split unit
+ *                 (a multiple of 32).
+ *   workspace     device scratch of at least pkv_decode_workspace_bytes(...)
+ *                 bytes, 256-byte aligned.  Calls that overlap in time need
+ *                 distinct workspaces.
+ * Accumulation is fp32.  Out-of-range table entries are skipped (their tokens
+ * do not take part) and flag PKV_DEVERR_BAD_BLOCK; seq_lens outside
+ * [0, max_blocks_per_seq*block_size] are clamped and flag
+ * PKV_DEVERR_BAD_SEQ_LEN.
+ */
+pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache,
+                                      const void* v_cache, const int32_t* block_tables,
+                                      const int32_t* seq_lens, int32_t block_size,
+                                      float scale, void* out, int32_t num_seqs,
+                                      int32_t num_q_heads, int32_t num_kv_heads,
+                                      int32_t head_dim, int32_t max_blocks_per_seq,
+                                      int32_t num_blocks, int32_t max_seq_len,
+                                      pkv_dtype q_dtype, pkv_dtype kv_dtype,
+                                      pkv_dtype out_dtype, const float* k_scale,
+                                      const float* v_scale, int32_t partition_size,
+                                      void* workspace, size_t workspace_bytes,
+                                      pkv_stream_t stream);
+
+/*
+ * pkv_copy_blocks -- copy whole physical blocks (copy-on-write fork).
+ *
+ * [KVOPT] intro and [KVMGMT] "The Bonus: Zero-Copy Sharing": requests with a
+ * common prefix point their block tables at the same physical blocks; before
+ * a request appends into a shared, partially filled block it takes a private
+ * copy of it.  For every pair: k_cache[dst] = k_cache[src] and
+ * v_cache[dst] = v_cache[src] (all kv heads, all slots), bit-exact.
+ *
+ *   block_mapping [num_pairs, 2] int64 (src, dst).  dst ids must be distinct
+ *                 and no dst may also be a src in the same call.  Out-of-range
+ *                 ids: pair skipped, PKV_DEVERR_BAD_PAIR.
+ *   elem_bytes of dtype: 4 (F32), 2 (BF16), 1 (FP8_E4M3).
+ */
+pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping,
+                           int32_t num_pairs, int32_t num_kv_heads, int32_t head_dim,
+                           int32_t block_size, int32_t num_blocks, pkv_dtype dtype,
+                           pkv_stream_t stream);
+
+/*
+ * pkv_get_device_error -- synchronise `stream`, then read and clear the error
+ * word of the current device into *flags (PKV_DEVERR_* bits; 0 = clean).
+ * Returns PKV_ERR_DEVICE_INDEX if any bit was set, PKV_OK if none.  The word
+ * is shared by every stream of the device.
+ */
+pkv_status pkv_get_device_error(pkv_stream_t stream, uint32_t* flags /* host */);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PKV_H_ */

@@ -1,0 +1,229 @@
+"""B200 paged KV-cache library -- Python binding.
+
+Argument marshalling only: every call goes straight to the C ABI in
+``libpkv.so`` (declared in ``include/pkv.h``) with raw device pointers taken
+from torch tensors and the current torch CUDA stream.  There is no CPU or
+eager-torch fallback: if the library is not built, importing this package
+raises ImportError.
+
+Calls (names follow the C ABI):
+
+* :func:`kv_cache_write` -- scatter new tokens' K/V into their cache slots.
+* :func:`paged_attention_decode` -- one decode step of attention over the
+  block-paged cache.
+* :func:`copy_blocks` -- copy-on-write copy of physical blocks.
+* :func:`decode_workspace_bytes`, :func:`get_device_error`.
+
+Cache layout: ``[num_blocks, num_kv_heads, block_size, head_dim]``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+__all__ = [
+    "PkvError", "LIB_PATH", "lib", "kv_cache_write", "paged_attention_decode", "copy_blocks",
+    "decode_workspace_bytes", "get_device_error", "status_string", "DEVERR",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpkv.so")
+
+PKV_OK = 0
+STATUS_NAMES = {0: "PKV_OK", 1: "PKV_ERR_INVALID_ARG", 2: "PKV_ERR_UNSUPPORTED",
+                3: "PKV_ERR_WORKSPACE", 4: "PKV_ERR_CUDA", 5: "PKV_ERR_DEVICE_INDEX"}
+DEVERR = {"BAD_SLOT": 0x1, "BAD_BLOCK": 0x2, "BAD_SEQ_LEN": 0x4, "BAD_PAIR": 0x8,
+          "TIMEOUT": 0x10}
+
+_F32, _BF16, _FP8 = 0, 1, 2
+
+
+class PkvError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn}: {status_string(status)}")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is not built; run `python -m paged_kv_cache_412_b200.build` "
+            "(the library has no fallback path)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                             ctypes.c_size_t)
+    L.pkv_status_string.argtypes = [ctypes.c_int]
+    L.pkv_status_string.restype = ctypes.c_char_p
+    L.pkv_version.argtypes = []
+    L.pkv_version.restype = ctypes.c_int
+    L.pkv_kv_cache_write.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, ctypes.c_int, vp]
+    L.pkv_kv_cache_write.restype = ctypes.c_int
+    L.pkv_decode_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32]
+    L.pkv_decode_workspace_bytes.restype = sz
+    L.pkv_paged_attention_decode.argtypes = [vp, vp, vp, vp, vp, i32, f32, vp, i32, i32, i32,
+                                             i32, i32, i32, i32, ctypes.c_int, ctypes.c_int,
+                                             ctypes.c_int, vp, vp, i32, vp, sz, vp]
+    L.pkv_paged_attention_decode.restype = ctypes.c_int
+    L.pkv_copy_blocks.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, ctypes.c_int, vp]
+    L.pkv_copy_blocks.restype = ctypes.c_int
+    L.pkv_get_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
+    L.pkv_get_device_error.restype = ctypes.c_int
+    return L
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.pkv_status_string(int(status)).decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != PKV_OK:
+        raise PkvError(fn, status)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return _F32
+    if t.dtype == torch.bfloat16:
+        return _BF16
+    if t.dtype in (torch.float8_e4m3fn, torch.uint8):
+        return _FP8
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need_cuda(*ts: torch.Tensor) -> torch.device:
+    dev = None
+    for t in ts:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("all tensors must be CUDA tensors")
+        if not t.is_contiguous():
+            raise ValueError("all tensors must be contiguous")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError("all tensors must be on one device")
+    return dev
+
+
+def kv_cache_write(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor,
+                   k_cache: torch.Tensor, v_cache: torch.Tensor) -> None:
+    """k, v [T, Hkv, d]; slot_mapping [T] int64; caches [NB, Hkv, bs, d]."""
+    dev = _need_cuda(k, v, slot_mapping, k_cache, v_cache)
+    if slot_mapping.dtype != torch.int64:
+        raise TypeError("slot_mapping must be int64")
+    if k.dtype != k_cache.dtype or v.dtype != v_cache.dtype or k.dtype != v.dtype:
+        raise TypeError("k, v and the caches must share one dtype")
+    T, Hkv, d = k.shape
+    NB, Hkv2, bs, d2 = k_cache.shape
+    if (Hkv, d) != (Hkv2, d2) or v.shape != k.shape or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    with torch.cuda.device(dev):
+        st = lib.pkv_kv_cache_write(_ptr(k), _ptr(v), _ptr(slot_mapping), _ptr(k_cache),
+                                    _ptr(v_cache), T, Hkv, d, bs, NB, _dtype_code(k_cache),
+                                    _stream(dev))
+    _check("pkv_kv_cache_write", st)
+
+
+def decode_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                           block_size: int, max_seq_len: int, partition_size: int = 0) -> int:
+    return int(lib.pkv_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim,
+                                              block_size, max_seq_len, partition_size))
+
+
+_ws_lock = threading.Lock()
+_ws_cache: dict = {}
+
+
+def _workspace(dev: torch.device, nbytes: int) -> torch.Tensor:
+    """A per-(device, stream) scratch buffer, grown on demand (caller-side
+    allocation through torch; the library itself allocates nothing)."""
+    key = (dev.index, torch.cuda.current_stream(dev).cuda_stream)
+    with _ws_lock:
+        buf = _ws_cache.get(key)
+        if buf is None or buf.numel() < nbytes:
+            buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+            _ws_cache[key] = buf
+        return buf
+
+
+def paged_attention_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                           block_tables: torch.Tensor, seq_lens: torch.Tensor,
+                           block_size: int | None = None, scale: float | None = None,
+                           out: torch.Tensor | None = None, *, max_seq_len: int | None = None,
+                           partition_size: int = 0, out_dtype: torch.dtype | None = None,
+                           k_scale: torch.Tensor | None = None,
+                           v_scale: torch.Tensor | None = None,
+                           workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """out[b, h] = softmax(scale * q[b, h] . K^T) V over request b's tokens.
+
+    q [B, Hq, d]; caches [NB, Hkv, bs, d]; block_tables [B, max_blocks] int32;
+    seq_lens [B] int32.  ``max_seq_len`` defaults to the block tables' capacity.
+    """
+    dev = _need_cuda(q, k_cache, v_cache, block_tables, seq_lens, out, k_scale, v_scale,
+                     workspace)
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise TypeError("block_tables and seq_lens must be int32")
+    B, Hq, d = q.shape
+    NB, Hkv, bs, d2 = k_cache.shape
+    if block_size is None:
+        block_size = bs
+    if block_size != bs or d2 != d or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    if scale is None:
+        scale = d ** -0.5
+    max_blocks = block_tables.shape[1]
+    if max_seq_len is None:
+        max_seq_len = max_blocks * bs
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=out_dtype or q.dtype, device=dev)
+    need = decode_workspace_bytes(B, Hq, Hkv, d, bs, max_seq_len, partition_size)
+    with torch.cuda.device(dev):
+        ws = workspace if workspace is not None else _workspace(dev, need)
+        st = lib.pkv_paged_attention_decode(
+            _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(seq_lens),
+            bs, float(scale), _ptr(out), B, Hq, Hkv, d, max_blocks, NB, int(max_seq_len),
+            _dtype_code(q), _dtype_code(k_cache), _dtype_code(out), _ptr(k_scale),
+            _ptr(v_scale), int(partition_size), _ptr(ws), ws.numel() * ws.element_size(),
+            _stream(dev))
+    _check("pkv_paged_attention_decode", st)
+    return out
+
+
+def copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, block_mapping: torch.Tensor) -> None:
+    """block_mapping [n, 2] int64 (src, dst): cache[dst] = cache[src] for K and V."""
+    dev = _need_cuda(k_cache, v_cache, block_mapping)
+    if block_mapping.dtype != torch.int64:
+        raise TypeError("block_mapping must be int64")
+    n = block_mapping.numel() // 2
+    NB, Hkv, bs, d = k_cache.shape
+    with torch.cuda.device(dev):
+        st = lib.pkv_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(block_mapping), n, Hkv, d,
+                                 bs, NB, _dtype_code(k_cache), _stream(dev))
+    _check("pkv_copy_blocks", st)
+
+
+def get_device_error(device: torch.device | int | None = None) -> int:
+    """Synchronise the current stream, then read and clear the device error
+    word (PKV_DEVERR_* bits, see ``DEVERR``)."""
+    dev = torch.device("cuda", torch.cuda.current_device() if device is None else
+                       (device if isinstance(device, int) else device.index))
+    flags = ctypes.c_uint32(0)
+    with torch.cuda.device(dev):
+        st = lib.pkv_get_device_error(_stream(dev), ctypes.byref(flags))
+    if st not in (PKV_OK, 5):
+        raise PkvError("pkv_get_device_error", st)
+    return int(flags.value)

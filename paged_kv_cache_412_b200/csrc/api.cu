@@ -1,0 +1,273 @@
+// api.cu -- the extern "C" entry points declared in include/pkv.h: host-side
+// validation, workspace planning, per-device state and the error word.
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "pkv_device.cuh"
+#include "pkv_internal.h"
+
+namespace pkv {
+
+// The per-device error word (PKV_DEVERR_* bits).  Kernels receive its address
+// as an argument; pkv_get_device_error reads and clears it.
+__device__ unsigned g_error_word = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kChunkTokens = 32;  // tokens per decode pipeline stage
+constexpr int kMaxCtasPerSm = 4;  // cap of resident decode CTAs per SM
+
+bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
+
+int log2_int(int x) {
+    int r = 0;
+    while ((1 << r) < x) ++r;
+    return r;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int elem_size(pkv_dtype t) {
+    switch (t) {
+        case PKV_F32: return 4;
+        case PKV_BF16: return 2;
+        case PKV_FP8_E4M3: return 1;
+        default: return 0;
+    }
+}
+
+int group_pad_of(int group) {
+    if (group >= 8) return 8;
+    int g = 1;
+    while (g < group) g <<= 1;
+    return g;
+}
+
+}  // namespace
+
+const DeviceInfo* current_device_info() {
+    static std::mutex mu;
+    static DeviceInfo infos[kMaxDevices];
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    DeviceInfo& di = infos[dev];
+    if (di.device == dev) return &di;
+    DeviceInfo tmp;
+    tmp.device = dev;
+    if (cudaDeviceGetAttribute(&tmp.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return nullptr;
+    if (cudaDeviceGetAttribute(&tmp.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) !=
+        cudaSuccess)
+        return nullptr;
+    void* addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_error_word) != cudaSuccess) return nullptr;
+    tmp.error_word = static_cast<unsigned*>(addr);
+    di = tmp;
+    return &di;
+}
+
+bool make_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                      int block_size, int max_seq_len, int partition_size, int ctas_per_sm,
+                      DecodePlan* plan) {
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        block_size <= 0 || max_seq_len < 0 || partition_size < 0)
+        return false;
+    if (num_q_heads % num_kv_heads) return false;
+    if (partition_size % kChunkTokens) return false;
+    const DeviceInfo* di = current_device_info();
+    if (!di) return false;
+    const int group = num_q_heads / num_kv_heads;
+    DecodePlan pl{};
+    pl.group_pad = group_pad_of(group);
+    pl.num_sub = (group + 7) / 8;
+    pl.num_hg = num_kv_heads * pl.num_sub;
+    pl.chunk_tokens = kChunkTokens;
+    pl.fixed_units = partition_size / kChunkTokens;
+    pl.grid = di->num_sms * ctas_per_sm;
+    const size_t n_bg = (size_t)num_seqs * pl.num_hg;
+    const size_t max_chunks = (size_t)((max_seq_len + kChunkTokens - 1) / kChunkTokens);
+    const size_t total_max = n_bg * max_chunks;
+    size_t units = (size_t)pl.grid;
+    if (pl.fixed_units > 0) units = std::max(units, total_max / pl.fixed_units + 1);
+    pl.units_max = units;
+    pl.records = n_bg + units;
+    const size_t acc_bytes = pl.records * pl.group_pad * head_dim * sizeof(float);
+    const size_t ml_bytes = pl.records * pl.group_pad * 2 * sizeof(float);
+    const size_t meta_bytes = n_bg * 2 * sizeof(int32_t);
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    pl.bytes = up(acc_bytes) + up(ml_bytes) + up(meta_bytes);
+    *plan = pl;
+    return true;
+}
+
+}  // namespace pkv
+
+using namespace pkv;
+
+extern "C" {
+
+const char* pkv_status_string(pkv_status status) {
+    switch (status) {
+        case PKV_OK: return "PKV_OK";
+        case PKV_ERR_INVALID_ARG: return "PKV_ERR_INVALID_ARG: invalid argument";
+        case PKV_ERR_UNSUPPORTED: return "PKV_ERR_UNSUPPORTED: unsupported configuration";
+        case PKV_ERR_WORKSPACE: return "PKV_ERR_WORKSPACE: workspace missing or too small";
+        case PKV_ERR_CUDA: return "PKV_ERR_CUDA: CUDA runtime or launch failure";
+        case PKV_ERR_DEVICE_INDEX: return "PKV_ERR_DEVICE_INDEX: device reported a bad index";
+        default: return "PKV_ERR_UNKNOWN";
+    }
+}
+
+int pkv_version(void) { return 100; }
+
+pkv_status pkv_kv_cache_write(const void* k, const void* v, const int64_t* slot_mapping,
+                              void* k_cache, void* v_cache, int32_t num_tokens,
+                              int32_t num_kv_heads, int32_t head_dim, int32_t block_size,
+                              int32_t num_blocks, pkv_dtype dtype, pkv_stream_t stream) {
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0 ||
+        !is_pow2(block_size) || block_size > 256)
+        return PKV_ERR_INVALID_ARG;
+    const int es = elem_size(dtype);
+    if (es == 0) return PKV_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return PKV_OK;
+    if (!k || !v || !slot_mapping || !k_cache || !v_cache) return PKV_ERR_INVALID_ARG;
+    if (!aligned(k, 16) || !aligned(v, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(slot_mapping, 8))
+        return PKV_ERR_INVALID_ARG;
+    const DeviceInfo* di = current_device_info();
+    if (!di) return PKV_ERR_CUDA;
+    return launch_kv_cache_write(k, v, slot_mapping, k_cache, v_cache, num_tokens, num_kv_heads,
+                                 head_dim, block_size, num_blocks, es, di->error_word,
+                                 reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                  int32_t head_dim, int32_t block_size, int32_t max_seq_len,
+                                  int32_t partition_size) {
+    if (!is_pow2(block_size) || block_size > 256) return 0;
+    DecodePlan pl;
+    if (!make_decode_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len,
+                          partition_size, kMaxCtasPerSm, &pl))
+        return 0;
+    return pl.bytes;
+}
+
+pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const void* v_cache,
+                                      const int32_t* block_tables, const int32_t* seq_lens,
+                                      int32_t block_size, float scale, void* out,
+                                      int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                      int32_t head_dim, int32_t max_blocks_per_seq,
+                                      int32_t num_blocks, int32_t max_seq_len, pkv_dtype q_dtype,
+                                      pkv_dtype kv_dtype, pkv_dtype out_dtype,
+                                      const float* k_scale, const float* v_scale,
+                                      int32_t partition_size, void* workspace,
+                                      size_t workspace_bytes, pkv_stream_t stream) {
+    if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
+        max_blocks_per_seq <= 0 || num_blocks <= 0 || max_seq_len < 0 || partition_size < 0)
+        return PKV_ERR_INVALID_ARG;
+    if (num_q_heads % num_kv_heads) return PKV_ERR_INVALID_ARG;
+    if (!is_pow2(block_size) || block_size > 256) return PKV_ERR_INVALID_ARG;
+    if (partition_size % kChunkTokens) return PKV_ERR_INVALID_ARG;
+    if (!std::isfinite(scale)) return PKV_ERR_INVALID_ARG;
+    if (elem_size(q_dtype) == 0 || elem_size(kv_dtype) == 0 || elem_size(out_dtype) == 0)
+        return PKV_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
+    if (out_dtype == PKV_FP8_E4M3) return PKV_ERR_UNSUPPORTED;
+    const bool f32_pair = q_dtype == PKV_F32 && kv_dtype == PKV_F32;
+    const bool bf16_pair = q_dtype == PKV_BF16 && kv_dtype == PKV_BF16;
+    if (kv_dtype == PKV_FP8_E4M3) return PKV_ERR_UNSUPPORTED;
+    if (!f32_pair && !bf16_pair) return PKV_ERR_INVALID_ARG;
+    if ((long long)max_blocks_per_seq * block_size > 0x7fffffffLL) return PKV_ERR_INVALID_ARG;
+    if (num_seqs == 0) return PKV_OK;
+    if (!q || !k_cache || !v_cache || !block_tables || !seq_lens || !out)
+        return PKV_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(block_tables, 4) || !aligned(seq_lens, 4) || !aligned(out, elem_size(out_dtype)))
+        return PKV_ERR_INVALID_ARG;
+    DecodePlan pl;
+    if (!make_decode_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len,
+                          partition_size, kMaxCtasPerSm, &pl))
+        return PKV_ERR_CUDA;
+    if (!workspace || workspace_bytes < pl.bytes || !aligned(workspace, 256))
+        return PKV_ERR_WORKSPACE;
+    const DeviceInfo* di = current_device_info();
+    if (!di) return PKV_ERR_CUDA;
+
+    const size_t n_bg = (size_t)num_seqs * pl.num_hg;
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    DecodeParams p{};
+    p.q = q;
+    p.k_cache = k_cache;
+    p.v_cache = v_cache;
+    p.block_tables = block_tables;
+    p.seq_lens = seq_lens;
+    p.out = out;
+    p.k_scale = k_scale;
+    p.v_scale = v_scale;
+    p.rec_acc = reinterpret_cast<float*>(ws);
+    p.rec_ml = reinterpret_cast<float*>(ws + up(pl.records * pl.group_pad * head_dim * 4));
+    p.meta = reinterpret_cast<int32_t*>(ws + up(pl.records * pl.group_pad * head_dim * 4) +
+                                        up(pl.records * pl.group_pad * 2 * 4));
+    (void)n_bg;
+    p.err = di->error_word;
+    p.num_seqs = num_seqs;
+    p.num_q_heads = num_q_heads;
+    p.num_kv_heads = num_kv_heads;
+    p.group = num_q_heads / num_kv_heads;
+    p.num_sub = pl.num_sub;
+    p.num_hg = pl.num_hg;
+    p.block_size = block_size;
+    p.log2_bs = log2_int(block_size);
+    p.max_blocks = max_blocks_per_seq;
+    p.num_blocks = num_blocks;
+    p.fixed_units = pl.fixed_units;
+    p.rec_cap = (long long)pl.records;
+    p.out_dtype = out_dtype;
+    p.scale_log2 = scale * 1.4426950408889634f;
+    return launch_decode_simt(p, head_dim, kv_dtype, pl.group_pad,
+                              reinterpret_cast<cudaStream_t>(stream), nullptr);
+}
+
+pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping,
+                           int32_t num_pairs, int32_t num_kv_heads, int32_t head_dim,
+                           int32_t block_size, int32_t num_blocks, pkv_dtype dtype,
+                           pkv_stream_t stream) {
+    if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0 ||
+        !is_pow2(block_size) || block_size > 256)
+        return PKV_ERR_INVALID_ARG;
+    const int es = elem_size(dtype);
+    if (es == 0) return PKV_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
+    if (num_pairs == 0) return PKV_OK;
+    if (!k_cache || !v_cache || !block_mapping) return PKV_ERR_INVALID_ARG;
+    if (!aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(block_mapping, 8))
+        return PKV_ERR_INVALID_ARG;
+    const DeviceInfo* di = current_device_info();
+    if (!di) return PKV_ERR_CUDA;
+    const size_t block_bytes = (size_t)num_kv_heads * block_size * head_dim * es;
+    return launch_copy_blocks(k_cache, v_cache, block_mapping, num_pairs, block_bytes, num_blocks,
+                              di->error_word, reinterpret_cast<cudaStream_t>(stream));
+}
+
+pkv_status pkv_get_device_error(pkv_stream_t stream, uint32_t* flags) {
+    if (!flags) return PKV_ERR_INVALID_ARG;
+    *flags = 0;
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return PKV_ERR_CUDA;
+    unsigned v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_error_word, sizeof v) != cudaSuccess) return PKV_ERR_CUDA;
+    if (v) {
+        const unsigned zero = 0;
+        if (cudaMemcpyToSymbol(g_error_word, &zero, sizeof zero) != cudaSuccess)
+            return PKV_ERR_CUDA;
+    }
+    *flags = v;
+    return v ? PKV_ERR_DEVICE_INDEX : PKV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,104 @@
+// cache_ops.cu -- the cache-mutating kernels: KV append (scatter into slots)
+// and copy-on-write block copy.  Both are pure byte movement, done in 16-byte
+// vectors with coalesced loads and stores; both are bit-exact.
+//
+// kv_cache_write: "PagedAttention: Optimizing KV Cache Utilization in Large
+// Language Models", "The Mechanics of PagedAttention" -- new tokens' K and V
+// vectors are written into their allocated blocks, wherever those sit.
+// copy_blocks: "KV Cache Optimization and PagedAttention" (intro) and "KV Cache
+// Management", "The Bonus: Zero-Copy Sharing" -- shared prefix blocks are
+// stored once; a request privately copies a shared block before appending.
+#include <algorithm>
+
+#include "pkv_device.cuh"
+#include "pkv_internal.h"
+
+namespace pkv {
+namespace {
+
+// One thread per 16-byte vector of one (token, kv head) row, K and V together.
+// Row r = t * Hkv + h of k/v goes to cache row ((blk * Hkv + h) * bs + off).
+__global__ void kv_cache_write_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
+                                      const int64_t* __restrict__ slots, uint4* __restrict__ kc,
+                                      uint4* __restrict__ vc, long long total_vecs,
+                                      int vecs_per_row, int num_kv_heads, int block_size,
+                                      int num_blocks, unsigned* err) {
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total_vecs; i += stride) {
+        const long long row = i / vecs_per_row;
+        const int vec = (int)(i - row * vecs_per_row);
+        const long long t = row / num_kv_heads;
+        const int h = (int)(row - t * num_kv_heads);
+        const int64_t slot = __ldg(slots + t);
+        if (slot < 0) continue;  // padding token
+        if (slot >= (int64_t)num_blocks * block_size) {
+            if (h == 0 && vec == 0) raise_error(err, PKV_DEVERR_BAD_SLOT);
+            continue;
+        }
+        const int64_t blk = slot / block_size;
+        const int off = (int)(slot - blk * block_size);
+        const size_t dst = (((size_t)blk * num_kv_heads + h) * block_size + off) * vecs_per_row + vec;
+        const uint4 kv = __ldg(k + i);
+        const uint4 vv = __ldg(v + i);
+        kc[dst] = kv;
+        vc[dst] = vv;
+    }
+}
+
+// grid.x = pair, grid.y = 0 (K) / 1 (V), grid.z = slice of the block.
+__global__ void copy_blocks_kernel(uint4* __restrict__ kc, uint4* __restrict__ vc,
+                                   const int64_t* __restrict__ pairs, long long vecs_per_block,
+                                   int slice_vecs, int num_blocks, unsigned* err) {
+    const int64_t src = __ldg(pairs + 2 * blockIdx.x);
+    const int64_t dst = __ldg(pairs + 2 * blockIdx.x + 1);
+    if (src < 0 || dst < 0 || src >= num_blocks || dst >= num_blocks) {
+        if (threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+            raise_error(err, PKV_DEVERR_BAD_PAIR);
+        return;
+    }
+    uint4* base = blockIdx.y == 0 ? kc : vc;
+    const uint4* s = base + src * vecs_per_block;
+    uint4* d = base + dst * vecs_per_block;
+    const long long lo = (long long)blockIdx.z * slice_vecs;
+    const long long hi = min(lo + slice_vecs, vecs_per_block);
+    for (long long i = lo + threadIdx.x; i < hi; i += blockDim.x) d[i] = s[i];
+}
+
+}  // namespace
+
+pkv_status launch_kv_cache_write(const void* k, const void* v, const int64_t* slots,
+                                 void* k_cache, void* v_cache, int num_tokens, int num_kv_heads,
+                                 int head_dim, int block_size, int num_blocks, int elem_bytes,
+                                 unsigned* err, cudaStream_t stream) {
+    const DeviceInfo* di = current_device_info();
+    if (!di) return PKV_ERR_CUDA;
+    const int vecs_per_row = head_dim * elem_bytes / 16;
+    const long long total = (long long)num_tokens * num_kv_heads * vecs_per_row;
+    if (total == 0) return PKV_OK;
+    const int threads = 256;
+    const long long want = (total + threads - 1) / threads;
+    const int grid = (int)std::min<long long>(want, (long long)di->num_sms * 8);
+    kv_cache_write_kernel<<<grid, threads, 0, stream>>>(
+        static_cast<const uint4*>(k), static_cast<const uint4*>(v), slots,
+        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), total, vecs_per_row,
+        num_kv_heads, block_size, num_blocks, err);
+    return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+pkv_status launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int num_pairs,
+                              size_t block_bytes, int num_blocks, unsigned* err,
+                              cudaStream_t stream) {
+    if (num_pairs == 0) return PKV_OK;
+    const long long vecs = (long long)(block_bytes / 16);
+    const int threads = 256;
+    const int slice = threads * 4;  // 16 KB per CTA
+    const long long slices = (vecs + slice - 1) / slice;
+    if (slices > 65535 || num_pairs > 2147483647) return PKV_ERR_UNSUPPORTED;
+    dim3 grid(num_pairs, 2, (unsigned)slices);
+    copy_blocks_kernel<<<grid, threads, 0, stream>>>(static_cast<uint4*>(k_cache),
+                                                      static_cast<uint4*>(v_cache), pairs, vecs,
+                                                      slice, num_blocks, err);
+    return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+}  // namespace pkv

@@ -1,0 +1,137 @@
+"""C-ABI library: it loads, exports every symbol the public header declares,
+and rejects bad arguments on the host before touching a device (no GPU)."""
+from __future__ import annotations
+
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+LIB = os.path.join(ROOT, "paged_kv_cache_412_b200", "libpkv.so")
+
+
+def _declared_functions():
+    names = set()
+    for hdr in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(hdr).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^[A-Za-z_][\w\s\*]*?\b(pkv_\w+)\s*\(", text, flags=re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(LIB):
+        from paged_kv_cache_412_b200 import build
+        build.build()
+    return ctypes.CDLL(LIB)
+
+
+def test_header_declares_the_hot_path_calls():
+    names = _declared_functions()
+    for n in ("pkv_kv_cache_write", "pkv_paged_attention_decode", "pkv_copy_blocks",
+              "pkv_decode_workspace_bytes", "pkv_get_device_error", "pkv_status_string"):
+        assert n in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    missing = [n for n in _declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings(lib):
+    lib.pkv_status_string.restype = ctypes.c_char_p
+    assert lib.pkv_status_string(0) == b"PKV_OK"
+    assert b"WORKSPACE" in lib.pkv_status_string(3)
+    assert b"UNKNOWN" in lib.pkv_status_string(99)
+    assert lib.pkv_version() >= 100
+
+
+def test_binding_imports_and_names_match(lib):
+    import paged_kv_cache_412_b200 as pkv
+    assert os.path.samefile(pkv.LIB_PATH, LIB)
+    for fn in ("kv_cache_write", "paged_attention_decode", "copy_blocks"):
+        assert callable(getattr(pkv, fn))
+
+
+# Host validation paths that return before any CUDA call.
+V = ctypes.c_void_p
+DUMMY = V(0x10000)
+
+
+def _write(lib, **kw):
+    a = dict(k=DUMMY, v=DUMMY, slots=DUMMY, kc=DUMMY, vc=DUMMY, T=4, Hkv=2, d=64, bs=16, NB=8,
+             dt=1)
+    a.update(kw)
+    f = lib.pkv_kv_cache_write
+    f.argtypes = [V, V, V, V, V, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                  ctypes.c_int32, ctypes.c_int, V]
+    return f(a["k"], a["v"], a["slots"], a["kc"], a["vc"], a["T"], a["Hkv"], a["d"], a["bs"],
+             a["NB"], a["dt"], None)
+
+
+def test_write_rejects_bad_args(lib):
+    assert _write(lib, T=-1) == 1
+    assert _write(lib, bs=12) == 1          # not a power of two
+    assert _write(lib, bs=512) == 1         # too large
+    assert _write(lib, dt=7) == 1           # unknown dtype
+    assert _write(lib, d=96) == 2           # unsupported head_dim
+    assert _write(lib, T=0) == 0            # nothing to do
+    assert _write(lib, k=None) == 1         # null pointer
+    assert _write(lib, kc=V(0x10004)) == 1  # misaligned cache
+
+
+def _decode(lib, **kw):
+    a = dict(q=DUMMY, kc=DUMMY, vc=DUMMY, bt=DUMMY, sl=DUMMY, bs=16, scale=0.125, out=DUMMY,
+             B=2, Hq=8, Hkv=2, d=128, maxb=4, NB=8, maxL=64, qdt=1, kvdt=1, odt=1, ks=None,
+             vs=None, P=0, ws=DUMMY, wsb=1 << 20)
+    a.update(kw)
+    f = lib.pkv_paged_attention_decode
+    i32 = ctypes.c_int32
+    f.argtypes = [V, V, V, V, V, i32, ctypes.c_float, V, i32, i32, i32, i32, i32, i32, i32,
+                  ctypes.c_int, ctypes.c_int, ctypes.c_int, V, V, i32, V, ctypes.c_size_t, V]
+    return f(a["q"], a["kc"], a["vc"], a["bt"], a["sl"], a["bs"], a["scale"], a["out"], a["B"],
+             a["Hq"], a["Hkv"], a["d"], a["maxb"], a["NB"], a["maxL"], a["qdt"], a["kvdt"],
+             a["odt"], a["ks"], a["vs"], a["P"], a["ws"], a["wsb"], None)
+
+
+def test_decode_rejects_bad_args(lib):
+    assert _decode(lib, Hq=6, Hkv=4) == 1       # Hq % Hkv != 0
+    assert _decode(lib, bs=24) == 1             # not a power of two
+    assert _decode(lib, d=80) == 2              # unsupported head_dim
+    assert _decode(lib, qdt=0, kvdt=1) == 1     # dtype mismatch
+    assert _decode(lib, odt=2) == 2             # fp8 output not supported
+    assert _decode(lib, P=48) == 1              # partition not a multiple of 32
+    assert _decode(lib, scale=float("nan")) == 1
+    assert _decode(lib, B=-1) == 1
+    assert _decode(lib, B=0) == 0               # empty batch: nothing to do
+    assert _decode(lib, q=None) == 1
+    assert _decode(lib, maxb=0) == 1
+
+
+def _copy(lib, **kw):
+    a = dict(kc=DUMMY, vc=DUMMY, bm=DUMMY, n=3, Hkv=2, d=64, bs=16, NB=8, dt=1)
+    a.update(kw)
+    f = lib.pkv_copy_blocks
+    i32 = ctypes.c_int32
+    f.argtypes = [V, V, V, i32, i32, i32, i32, i32, ctypes.c_int, V]
+    return f(a["kc"], a["vc"], a["bm"], a["n"], a["Hkv"], a["d"], a["bs"], a["NB"], a["dt"], None)
+
+
+def test_copy_rejects_bad_args(lib):
+    assert _copy(lib, n=-2) == 1
+    assert _copy(lib, bs=3) == 1
+    assert _copy(lib, d=32) == 2
+    assert _copy(lib, n=0) == 0
+    assert _copy(lib, bm=None) == 1
+    assert _copy(lib, bm=V(0x10004)) == 1
+
+
+def test_get_device_error_needs_output_pointer(lib):
+    f = lib.pkv_get_device_error
+    f.argtypes = [V, V]
+    assert f(None, None) == 1

@@ -1,0 +1,102 @@
+"""Device-detected faults and host validation that needs a device.
+
+Bad indices are planted on the HOST in the inputs (a slot past the pool, a
+block id past the pool, a sequence longer than its table, a copy pair out of
+range).  The kernels must skip the bad item, raise a bit in the error word and
+carry on -- no trap, no assert, no hang.  Nothing here faults the GPU."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+from _helpers import DevWorkload, assert_decode_close, host_step, to_dev, to_host_f64
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def pkv():
+    import paged_kv_cache_412_b200 as m
+    m.get_device_error()  # start clean
+    return m
+
+
+def test_bad_slot_is_skipped_and_flagged(pkv):
+    w = workloads.make_paged([10, 20, 30], Hq=4, Hkv=2, d=64, bs=16, dtype="bf16", seed=1)
+    dw = DevWorkload(w)
+    slots = dw.slot_mapping.clone()
+    slots[1] = w.num_blocks * w.bs + 5
+    before = dw.k_cache.clone()
+    pkv.kv_cache_write(dw.k_new, dw.v_new, slots, dw.k_cache, dw.v_cache)
+    assert pkv.get_device_error() & pkv.DEVERR["BAD_SLOT"]
+    assert pkv.get_device_error() == 0  # read-and-clear
+    # the two good tokens landed, nothing else changed
+    kc_ref = w.k_cache.copy()
+    vc_ref = w.v_cache.copy()
+    good = np.array([0, 2])
+    oracle.kv_cache_write(w.k_new[good], w.v_new[good], w.slot_mapping[good], kc_ref, vc_ref)
+    got = dw.k_cache.cpu().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, kc_ref)
+
+
+def test_bad_block_id_is_skipped_and_flagged(pkv):
+    w = workloads.make_paged([100, 64, 50], Hq=8, Hkv=2, d=128, bs=16, dtype="bf16", seed=2,
+                             append_last=False)
+    bt = w.block_tables.copy()
+    bt[1, 2] = w.num_blocks + 7  # request 1's third block is out of range
+    dw = DevWorkload(w)
+    out = pkv.paged_attention_decode(dw.q, dw.k_cache, dw.v_cache, to_dev(bt), dw.seq_lens,
+                                     w.bs, w.scale)
+    assert pkv.get_device_error() & pkv.DEVERR["BAD_BLOCK"]
+    ref = oracle.decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale)
+    got = to_host_f64(out)
+    for b in (0, 2):  # the other requests are untouched
+        assert_decode_close(got[b], ref[b], "bf16", "bf16", what=f"req {b}")
+    assert np.all(np.isfinite(got[1]))
+
+
+def test_seq_len_past_table_is_clamped_and_flagged(pkv):
+    w = workloads.make_paged([40, 16], Hq=4, Hkv=4, d=64, bs=16, dtype="f32", seed=3,
+                             append_last=False)
+    sl = w.seq_lens.copy()
+    sl[1] = 10_000  # table holds 3 blocks (48 tokens) for this batch
+    dw = DevWorkload(w)
+    pkv.paged_attention_decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, to_dev(sl),
+                               w.bs, w.scale)
+    assert pkv.get_device_error() & pkv.DEVERR["BAD_SEQ_LEN"]
+
+
+def test_bad_copy_pair_is_skipped_and_flagged(pkv):
+    w = workloads.make_paged([40, 40], Hq=4, Hkv=2, d=64, bs=16, dtype="bf16", seed=4,
+                             extra_blocks=4, append_last=False)
+    pairs = np.array([[int(w.block_tables[0, 0]), w.num_blocks - 1], [0, w.num_blocks + 3]],
+                     np.int64)
+    dw = DevWorkload(w)
+    pkv.copy_blocks(dw.k_cache, dw.v_cache, to_dev(pairs))
+    assert pkv.get_device_error() & pkv.DEVERR["BAD_PAIR"]
+    kc_ref, vc_ref = w.k_cache.copy(), w.v_cache.copy()
+    oracle.copy_blocks(kc_ref, vc_ref, pairs[:1])
+    got = dw.k_cache.cpu().view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(got, kc_ref)
+
+
+def test_workspace_too_small_is_rejected(pkv):
+    w = workloads.make_paged([40], Hq=4, Hkv=2, d=64, bs=16, dtype="bf16", seed=5)
+    dw = DevWorkload(w)
+    tiny = torch.empty(256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(pkv.PkvError) as ei:
+        pkv.paged_attention_decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens,
+                                   w.bs, w.scale, workspace=tiny)
+    assert ei.value.status == 3
+
+
+def test_clean_run_leaves_no_flag(pkv):
+    w = workloads.make_paged([40, 7], Hq=4, Hkv=2, d=64, bs=16, dtype="bf16", seed=6)
+    dw = DevWorkload(w)
+    pkv.kv_cache_write(dw.k_new, dw.v_new, dw.slot_mapping, dw.k_cache, dw.v_cache)
+    pkv.paged_attention_decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens,
+                               w.bs, w.scale)
+    assert pkv.get_device_error() == 0

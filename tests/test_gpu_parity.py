@@ -1,0 +1,212 @@
+"""GPU parity: the CUDA library against the fp64 CPU oracle, element by element.
+
+Every call goes through the C ABI (via the thin binding).  Cache writes and
+block copies must be bit-exact (including the NaN-poisoned slots nobody owns,
+which must stay untouched); decode must meet the tolerances in _helpers.py.
+
+Small cases span several pipeline stages and ragged tails; the five named
+workloads run at full size in the launch configuration the bench uses, with
+the oracle on all outputs (or a sample of requests where the oracle would take
+too long)."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+import workloads
+from _helpers import (DevWorkload, assert_decode_close, host_step, to_dev, to_host_bits,
+                      to_host_f64)
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def pkv():
+    import paged_kv_cache_412_b200 as m
+    return m
+
+
+def run_step(pkv, dw, out_dtype=None, partition_size=0):
+    """copy_blocks -> kv_cache_write -> paged_attention_decode on the device."""
+    w = dw.w
+    if w.copy_pairs.shape[0]:
+        pkv.copy_blocks(dw.k_cache, dw.v_cache, dw.copy_pairs)
+    if w.slot_mapping.shape[0]:
+        pkv.kv_cache_write(dw.k_new, dw.v_new, dw.slot_mapping, dw.k_cache, dw.v_cache)
+    out = pkv.paged_attention_decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens,
+                                     w.bs, w.scale, out_dtype=out_dtype,
+                                     partition_size=partition_size)
+    torch.cuda.synchronize()
+    return out
+
+
+def _bits(a):
+    return a.view(np.uint32) if a.dtype == np.float32 else a
+
+
+def check_caches(dw, kc_ref, vc_ref):
+    """Bit-exact, NaN payloads included."""
+    assert np.array_equal(_bits(to_host_bits(dw.k_cache)), _bits(kc_ref)), "k_cache differs"
+    assert np.array_equal(_bits(to_host_bits(dw.v_cache)), _bits(vc_ref)), "v_cache differs"
+
+
+# ---------------------------------------------------------------------------
+# small randomized cases
+# ---------------------------------------------------------------------------
+
+SMALL = [
+    # lens, Hq, Hkv, d, bs, dtype
+    ([1, 17, 100, 200], 4, 2, 64, 16, "f32"),
+    ([33, 64, 65, 7, 1, 300], 8, 8, 128, 16, "bf16"),
+    ([129, 31, 512], 32, 8, 128, 16, "bf16"),
+    ([250, 3, 40], 16, 2, 128, 8, "bf16"),       # G = 8
+    ([77, 160], 12, 4, 64, 32, "bf16"),          # G = 3 (padded to 4)
+    ([90, 45], 16, 1, 128, 16, "bf16"),          # G = 16 (two head groups per kv head)
+    ([70, 200, 5], 6, 3, 64, 1, "f32"),          # block size 1
+    ([70, 200, 5], 10, 2, 128, 4, "bf16"),       # G = 5
+    ([300, 129], 8, 2, 128, 64, "bf16"),         # block larger than a stage
+    ([513, 20], 8, 4, 64, 256, "f32"),           # block size 256
+    ([0, 40, 0, 1], 4, 2, 128, 16, "bf16"),      # empty requests
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: f"L{len(c[0])}_G{c[1]//c[2]}_d{c[3]}_bs{c[4]}_{c[5]}")
+def test_small_step_parity(pkv, case):
+    lens, Hq, Hkv, d, bs, dt = case
+    w = workloads.make_paged(lens, Hq=Hq, Hkv=Hkv, d=d, bs=bs, dtype=dt,
+                             seed=1000 + sum(lens) + bs, pool_factor=1.3, extra_blocks=3,
+                             table_pad=1)
+    kc_ref, vc_ref = host_step(w)
+    ref = oracle.decode(w.q, kc_ref, vc_ref, w.block_tables, w.seq_lens, w.scale)
+    for out_dtype in ([None] if dt == "f32" else [None, torch.float32]):
+        dw = DevWorkload(w)
+        out = run_step(pkv, dw, out_dtype=out_dtype)
+        check_caches(dw, kc_ref, vc_ref)
+        od = "f32" if (dt == "f32" or out_dtype == torch.float32) else "bf16"
+        assert_decode_close(to_host_f64(out), ref, dt, od, what=f"{case} out={od}")
+
+
+@pytest.mark.parametrize("P", [32, 64, 96, 512])
+def test_fixed_partition_sizes(pkv, P):
+    w = workloads.make_paged([1000, 33, 400, 1], Hq=8, Hkv=2, d=128, bs=16, dtype="bf16",
+                             seed=77)
+    kc, vc = host_step(w)
+    ref = oracle.decode(w.q, kc, vc, w.block_tables, w.seq_lens, w.scale)
+    dw = DevWorkload(w)
+    out = run_step(pkv, dw, partition_size=P)
+    assert_decode_close(to_host_f64(out), ref, "bf16", "bf16", what=f"P={P}")
+
+
+def test_length_one_returns_v_row(pkv):
+    w = workloads.make_paged([1, 1, 1], Hq=8, Hkv=2, d=128, bs=16, dtype="bf16", seed=5)
+    dw = DevWorkload(w)
+    out = run_step(pkv, dw, out_dtype=torch.float32)
+    got = to_host_f64(out)
+    vnew = workloads.bf16_bits_to_f32(w.v_new).astype(np.float64)
+    for b in range(3):
+        for h in range(8):
+            np.testing.assert_array_equal(got[b, h], vnew[b, h // 4])
+
+
+def test_deterministic_repeat(pkv):
+    w = workloads.make_paged([3000, 100, 2000], Hq=32, Hkv=8, d=128, bs=16, dtype="bf16",
+                             seed=9, append_last=False)
+    dw = DevWorkload(w)
+    a = run_step(pkv, dw)
+    b = run_step(pkv, dw)
+    assert torch.equal(a.view(torch.int16), b.view(torch.int16))
+
+
+def test_identity_and_permuted_tables_agree(pkv):
+    lens = [700, 300]
+    w1 = workloads.make_paged(lens, Hq=8, Hkv=2, d=128, bs=16, dtype="bf16", seed=3,
+                              permute=False, append_last=False)
+    w2 = workloads.make_paged(lens, Hq=8, Hkv=2, d=128, bs=16, dtype="bf16", seed=3,
+                              permute=True, append_last=False)
+    # same logical content, different placement (the generator draws the
+    # permutation before the values, so redo the placement from w1's data)
+    kc = np.full_like(w1.k_cache, workloads.BF16_NAN)
+    vc = np.full_like(w1.v_cache, workloads.BF16_NAN)
+    for b, L in enumerate(lens):
+        for j in range(-(-L // 16)):
+            kc[w2.block_tables[b, j]] = w1.k_cache[w1.block_tables[b, j]]
+            vc[w2.block_tables[b, j]] = w1.v_cache[w1.block_tables[b, j]]
+    w2.k_cache, w2.v_cache, w2.q = kc, vc, w1.q
+    o1 = run_step(pkv, DevWorkload(w1))
+    o2 = run_step(pkv, DevWorkload(w2))
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+
+
+# ---------------------------------------------------------------------------
+# the five workloads at full size
+# ---------------------------------------------------------------------------
+
+def _full_check(pkv, w, sample=None, partition_size=0, out_f32=True):
+    kc_ref, vc_ref = host_step(w)
+    dw = DevWorkload(w)
+    out = run_step(pkv, dw, partition_size=partition_size)
+    check_caches(dw, kc_ref, vc_ref)
+    got = to_host_f64(out)
+    rows = range(w.B) if sample is None else sample
+    ref = _oracle_rows(w, kc_ref, vc_ref, rows)
+    od = "f32" if w.dtype == "f32" else "bf16"
+    stats = assert_decode_close(got[list(rows)], ref, w.dtype, od, what=w.name)
+    if out_f32 and w.dtype == "bf16":
+        out32 = pkv.paged_attention_decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables,
+                                           dw.seq_lens, w.bs, w.scale, out_dtype=torch.float32,
+                                           partition_size=partition_size)
+        torch.cuda.synchronize()
+        assert_decode_close(to_host_f64(out32)[list(rows)], ref, "bf16", "f32",
+                            what=w.name + " fp32-out")
+    assert pkv.get_device_error() == 0
+    return stats
+
+
+def _oracle_rows(w, kc, vc, rows):
+    rows = list(rows)
+    return oracle.decode(w.q[rows], kc, vc, w.block_tables[rows], w.seq_lens[rows], w.scale)
+
+
+def test_workload_tiny_f32(pkv):
+    _full_check(pkv, workloads.tiny_f32())
+
+
+def test_workload_gqa_4k(pkv):
+    _full_check(pkv, workloads.gqa_4k())
+
+
+def test_workload_mixed(pkv):
+    w = workloads.mixed()
+    rng = np.random.default_rng(0)
+    sample = sorted(set(rng.choice(w.B, size=48, replace=False).tolist()) |
+                    {int(np.argmax(w.seq_lens)), int(np.argmin(w.seq_lens))})
+    _full_check(pkv, w, sample=sample)
+
+
+def test_workload_prefix(pkv):
+    w = workloads.prefix_shared()
+    _full_check(pkv, w)
+
+
+@pytest.mark.parametrize("bs", [8, 16, 32])
+def test_workload_long_ctx(pkv, bs):
+    w = workloads.long_ctx(bs=bs)
+    kc_ref, vc_ref = host_step(w)
+    ref = _oracle_rows(w, kc_ref, vc_ref, [0, 1])
+    dw = DevWorkload(w)
+    first = True
+    for P in (0, 512, 1024, 2048, 4096):
+        if first:
+            out = run_step(pkv, dw, partition_size=P)
+            check_caches(dw, kc_ref, vc_ref)
+            first = False
+        else:
+            out = pkv.paged_attention_decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables,
+                                             dw.seq_lens, w.bs, w.scale, partition_size=P)
+            torch.cuda.synchronize()
+        assert_decode_close(to_host_f64(out), ref, "bf16", "bf16", what=f"long bs{bs} P{P}")
+    assert pkv.get_device_error() == 0
