@@ -40,7 +40,7 @@ UNIT = "GB/s"
 WORKLOAD = "gqa_4k: batch 16 x 4096 tokens, 32 q / 8 KV heads, head_dim 128, block 16, bf16"
 FALLBACK_HBM_GBS = 6650.0
 N_LAYERS = 4
-DECODE_SRC = os.path.join(ROOT, "paged_kv_cache_412_b200", "csrc", "decode_simt.cu")
+DECODE_SRC = os.path.join(ROOT, "paged_kv_cache_412_b200", "csrc", "decode_mma.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_gqa_4k_traffic.txt")
 
 
@@ -312,7 +312,7 @@ def run_ours(args, rank: int, world: int, local: int):
         del w
     out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev)
     ws_bytes = pkv.decode_workspace_bytes(B, Hq, Hkv, d, bs, L, 0)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    ws = pkv.new_workspace(ws_bytes, dev)
     no_pairs = torch.empty((0, 2), dtype=torch.int64, device=dev)
     scale = 1.0 / math.sqrt(d)
 
@@ -442,7 +442,7 @@ def run_ours(args, rank: int, world: int, local: int):
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "traffic": traffic_per_launch(),
-                         "kernel": "paged_attention_decode (split kernel + merge kernel)",
+                         "kernel": "decode_mma_kernel (split decode with in-kernel merge)",
                          "peak_kind": f"{peak_kind} HBM copy bandwidth"},
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
@@ -450,7 +450,7 @@ def run_ours(args, rank: int, world: int, local: int):
                     "ms_per_step": round(e2e_ms / e2e_steps, 5),
                     "note": "pinned host inputs copied in and output copied out every step, "
                             "with a stream synchronize per step"},
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": 2 * args.steps,
             "clocks": clocks,
             "parity_spot_check": parity,
         }

@@ -111,6 +111,16 @@ size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
                                   int32_t partition_size);
 
 /*
+ * pkv_decode_workspace_init -- zero a decode workspace (asynchronous on
+ * `stream`).  Call once after allocating a workspace, before its first decode.
+ * Decode calls leave the workspace ready for the next call (the per-group
+ * arrival counters they use return to zero), so re-initialising is needed only
+ * if a call reported PKV_DEVERR_TIMEOUT.
+ */
+pkv_status pkv_decode_workspace_init(void* workspace, size_t workspace_bytes,
+                                     pkv_stream_t stream);
+
+/*
  * pkv_paged_attention_decode -- one decode step of attention for a batch.
  *
  * [PAMEM] "The Math: Block Attention Calculation": for query q_i the page
@@ -138,7 +148,8 @@ size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
  *                 shares, one per resident CTA; else tokens per split unit
  *                 (a multiple of 32).
  *   workspace     device scratch of at least pkv_decode_workspace_bytes(...)
- *                 bytes, 256-byte aligned.  Calls that overlap in time need
+ *                 bytes, 256-byte aligned, zeroed once by
+ *                 pkv_decode_workspace_init.  Calls that overlap in time need
  *                 distinct workspaces.
  * Accumulation is fp32.  Out-of-range table entries are skipped (their tokens
  * do not take part) and flag PKV_DEVERR_BAD_BLOCK; seq_lens outside

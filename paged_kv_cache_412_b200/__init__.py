@@ -3,8 +3,9 @@
 Argument marshalling only: every call goes straight to the C ABI in
 ``libpkv.so`` (declared in ``include/pkv.h``) with raw device pointers taken
 from torch tensors and the current torch CUDA stream.  There is no CPU or
-eager-torch fallback: if the library is not built, importing this package
-raises ImportError.
+eager-torch fallback: the library is loaded on first use, and if it is not
+built every call raises ImportError (build it with
+``python -m paged_kv_cache_412_b200.build``).
 
 Calls (names follow the C ABI):
 
@@ -26,7 +27,7 @@ import torch
 
 __all__ = [
     "PkvError", "LIB_PATH", "lib", "kv_cache_write", "paged_attention_decode", "copy_blocks",
-    "decode_workspace_bytes", "get_device_error", "status_string", "DEVERR",
+    "decode_workspace_bytes", "new_workspace", "get_device_error", "status_string", "DEVERR",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpkv.so")
@@ -62,6 +63,8 @@ def _load() -> ctypes.CDLL:
     L.pkv_kv_cache_write.restype = ctypes.c_int
     L.pkv_decode_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32, i32]
     L.pkv_decode_workspace_bytes.restype = sz
+    L.pkv_decode_workspace_init.argtypes = [vp, sz, vp]
+    L.pkv_decode_workspace_init.restype = ctypes.c_int
     L.pkv_paged_attention_decode.argtypes = [vp, vp, vp, vp, vp, i32, f32, vp, i32, i32, i32,
                                              i32, i32, i32, i32, ctypes.c_int, ctypes.c_int,
                                              ctypes.c_int, vp, vp, i32, vp, sz, vp]
@@ -73,11 +76,27 @@ def _load() -> ctypes.CDLL:
     return L
 
 
-lib = _load()
+_lib = None
+_lib_lock = threading.Lock()
+
+
+def _get_lib() -> ctypes.CDLL:
+    global _lib
+    if _lib is None:
+        with _lib_lock:
+            if _lib is None:
+                _lib = _load()
+    return _lib
+
+
+def __getattr__(name):
+    if name == "lib":
+        return _get_lib()
+    raise AttributeError(name)
 
 
 def status_string(status: int) -> str:
-    return lib.pkv_status_string(int(status)).decode()
+    return _get_lib().pkv_status_string(int(status)).decode()
 
 
 def _check(fn: str, status: int) -> None:
@@ -132,7 +151,7 @@ def kv_cache_write(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor,
     if (Hkv, d) != (Hkv2, d2) or v.shape != k.shape or v_cache.shape != k_cache.shape:
         raise ValueError("shape mismatch")
     with torch.cuda.device(dev):
-        st = lib.pkv_kv_cache_write(_ptr(k), _ptr(v), _ptr(slot_mapping), _ptr(k_cache),
+        st = _get_lib().pkv_kv_cache_write(_ptr(k), _ptr(v), _ptr(slot_mapping), _ptr(k_cache),
                                     _ptr(v_cache), T, Hkv, d, bs, NB, _dtype_code(k_cache),
                                     _stream(dev))
     _check("pkv_kv_cache_write", st)
@@ -140,12 +159,22 @@ def kv_cache_write(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor,
 
 def decode_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
                            block_size: int, max_seq_len: int, partition_size: int = 0) -> int:
-    return int(lib.pkv_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim,
+    return int(_get_lib().pkv_decode_workspace_bytes(num_seqs, num_q_heads, num_kv_heads, head_dim,
                                               block_size, max_seq_len, partition_size))
 
 
 _ws_lock = threading.Lock()
 _ws_cache: dict = {}
+
+
+def new_workspace(nbytes: int, device: torch.device | None = None) -> torch.Tensor:
+    """Allocate (through torch) and initialise a decode workspace of nbytes."""
+    dev = device or torch.device("cuda", torch.cuda.current_device())
+    buf = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        _check("pkv_decode_workspace_init",
+               _get_lib().pkv_decode_workspace_init(_ptr(buf), buf.numel(), _stream(dev)))
+    return buf
 
 
 def _workspace(dev: torch.device, nbytes: int) -> torch.Tensor:
@@ -155,7 +184,7 @@ def _workspace(dev: torch.device, nbytes: int) -> torch.Tensor:
     with _ws_lock:
         buf = _ws_cache.get(key)
         if buf is None or buf.numel() < nbytes:
-            buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=dev)
+            buf = new_workspace(nbytes, dev)
             _ws_cache[key] = buf
         return buf
 
@@ -193,7 +222,7 @@ def paged_attention_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torc
     need = decode_workspace_bytes(B, Hq, Hkv, d, bs, max_seq_len, partition_size)
     with torch.cuda.device(dev):
         ws = workspace if workspace is not None else _workspace(dev, need)
-        st = lib.pkv_paged_attention_decode(
+        st = _get_lib().pkv_paged_attention_decode(
             _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(seq_lens),
             bs, float(scale), _ptr(out), B, Hq, Hkv, d, max_blocks, NB, int(max_seq_len),
             _dtype_code(q), _dtype_code(k_cache), _dtype_code(out), _ptr(k_scale),
@@ -211,7 +240,7 @@ def copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, block_mapping: tor
     n = block_mapping.numel() // 2
     NB, Hkv, bs, d = k_cache.shape
     with torch.cuda.device(dev):
-        st = lib.pkv_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(block_mapping), n, Hkv, d,
+        st = _get_lib().pkv_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(block_mapping), n, Hkv, d,
                                  bs, NB, _dtype_code(k_cache), _stream(dev))
     _check("pkv_copy_blocks", st)
 
@@ -223,7 +252,7 @@ def get_device_error(device: torch.device | int | None = None) -> int:
                        (device if isinstance(device, int) else device.index))
     flags = ctypes.c_uint32(0)
     with torch.cuda.device(dev):
-        st = lib.pkv_get_device_error(_stream(dev), ctypes.byref(flags))
+        st = _get_lib().pkv_get_device_error(_stream(dev), ctypes.byref(flags))
     if st not in (PKV_OK, 5):
         raise PkvError("pkv_get_device_error", st)
     return int(flags.value)

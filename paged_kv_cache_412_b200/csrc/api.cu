@@ -1,5 +1,6 @@
 // api.cu -- the extern "C" entry points declared in include/pkv.h: host-side
 // validation, workspace planning, per-device state and the error word.
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -70,8 +71,7 @@ const DeviceInfo* current_device_info() {
 }
 
 bool make_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
-                      int block_size, int max_seq_len, int partition_size, int ctas_per_sm,
-                      DecodePlan* plan) {
+                      int block_size, int max_seq_len, int partition_size, DecodePlan* plan) {
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
         block_size <= 0 || max_seq_len < 0 || partition_size < 0)
         return false;
@@ -81,24 +81,29 @@ bool make_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_
     if (!di) return false;
     const int group = num_q_heads / num_kv_heads;
     DecodePlan pl{};
-    pl.group_pad = group_pad_of(group);
-    pl.num_sub = (group + 7) / 8;
-    pl.num_hg = num_kv_heads * pl.num_sub;
-    pl.chunk_tokens = kChunkTokens;
-    pl.fixed_units = partition_size / kChunkTokens;
-    pl.grid = di->num_sms * ctas_per_sm;
-    const size_t n_bg = (size_t)num_seqs * pl.num_hg;
-    const size_t max_chunks = (size_t)((max_seq_len + kChunkTokens - 1) / kChunkTokens);
-    const size_t total_max = n_bg * max_chunks;
-    size_t units = (size_t)pl.grid;
-    if (pl.fixed_units > 0) units = std::max(units, total_max / pl.fixed_units + 1);
+    // CUDA-core path: groups of <= 8 query heads; tensor-core path: <= 16.
+    pl.rec_gp = group > 8 ? 16 : 8;
+    pl.n_bg_max = (size_t)num_seqs * num_kv_heads * ((group + 7) / 8);
+    size_t units = (size_t)di->num_sms * kMaxCtasPerSm;
+    if (partition_size > 0) {
+        // fixed split units: W = partition / stage tokens (32 or 64), at least 1
+        for (int ch : {32, 64}) {
+            const size_t w = std::max(1, partition_size / ch);
+            const size_t chunks = (size_t)((max_seq_len + ch - 1) / ch);
+            units = std::max(units, pl.n_bg_max * chunks / w + 1);
+        }
+    }
     pl.units_max = units;
-    pl.records = n_bg + units;
-    const size_t acc_bytes = pl.records * pl.group_pad * head_dim * sizeof(float);
-    const size_t ml_bytes = pl.records * pl.group_pad * 2 * sizeof(float);
-    const size_t meta_bytes = n_bg * 2 * sizeof(int32_t);
+    pl.records = pl.n_bg_max + units;
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
-    pl.bytes = up(acc_bytes) + up(ml_bytes) + up(meta_bytes);
+    const size_t acc_bytes = pl.records * pl.rec_gp * head_dim * sizeof(float);
+    const size_t ml_bytes = pl.records * pl.rec_gp * 2 * sizeof(float);
+    const size_t meta_bytes = pl.n_bg_max * 2 * sizeof(int32_t);
+    const size_t cnt_bytes = pl.n_bg_max * sizeof(uint32_t);
+    pl.off_ml = up(acc_bytes);
+    pl.off_meta = pl.off_ml + up(ml_bytes);
+    pl.off_cnt = pl.off_meta + up(meta_bytes);
+    pl.bytes = pl.off_cnt + up(cnt_bytes);
     *plan = pl;
     return true;
 }
@@ -151,9 +156,18 @@ size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t
     if (!is_pow2(block_size) || block_size > 256) return 0;
     DecodePlan pl;
     if (!make_decode_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len,
-                          partition_size, kMaxCtasPerSm, &pl))
+                          partition_size, &pl))
         return 0;
     return pl.bytes;
+}
+
+pkv_status pkv_decode_workspace_init(void* workspace, size_t workspace_bytes,
+                                     pkv_stream_t stream) {
+    if (!workspace || workspace_bytes == 0) return PKV_ERR_INVALID_ARG;
+    return cudaMemsetAsync(workspace, 0, workspace_bytes, reinterpret_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? PKV_OK
+               : PKV_ERR_CUDA;
 }
 
 pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const void* v_cache,
@@ -190,15 +204,22 @@ pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const 
         return PKV_ERR_INVALID_ARG;
     DecodePlan pl;
     if (!make_decode_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len,
-                          partition_size, kMaxCtasPerSm, &pl))
+                          partition_size, &pl))
         return PKV_ERR_CUDA;
     if (!workspace || workspace_bytes < pl.bytes || !aligned(workspace, 256))
         return PKV_ERR_WORKSPACE;
+    if ((long long)num_blocks * num_kv_heads * block_size > 0x7fffffffLL)
+        return PKV_ERR_UNSUPPORTED;  // cache rows must fit the 32-bit TMA row coordinate
     const DeviceInfo* di = current_device_info();
     if (!di) return PKV_ERR_CUDA;
 
-    const size_t n_bg = (size_t)num_seqs * pl.num_hg;
-    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    const int group = num_q_heads / num_kv_heads;
+    const bool mma = decode_mma_supported(head_dim, block_size, q_dtype, kv_dtype);
+    // heads per kv-head pass: 8 or 16 on the tensor-core path, 1/2/4/8 otherwise
+    const int group_pad = mma ? (group > 8 ? 16 : 8) : group_pad_of(group);
+    const int per_pass = mma ? (group > 8 ? 16 : 8) : 8;
+    const int num_sub = (group + per_pass - 1) / per_pass;
+
     unsigned char* ws = static_cast<unsigned char*>(workspace);
     DecodeParams p{};
     p.q = q;
@@ -210,27 +231,27 @@ pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const 
     p.k_scale = k_scale;
     p.v_scale = v_scale;
     p.rec_acc = reinterpret_cast<float*>(ws);
-    p.rec_ml = reinterpret_cast<float*>(ws + up(pl.records * pl.group_pad * head_dim * 4));
-    p.meta = reinterpret_cast<int32_t*>(ws + up(pl.records * pl.group_pad * head_dim * 4) +
-                                        up(pl.records * pl.group_pad * 2 * 4));
-    (void)n_bg;
+    p.rec_ml = reinterpret_cast<float*>(ws + pl.off_ml);
+    p.meta = reinterpret_cast<int32_t*>(ws + pl.off_meta);
+    p.counters = reinterpret_cast<unsigned*>(ws + pl.off_cnt);
     p.err = di->error_word;
     p.num_seqs = num_seqs;
     p.num_q_heads = num_q_heads;
     p.num_kv_heads = num_kv_heads;
-    p.group = num_q_heads / num_kv_heads;
-    p.num_sub = pl.num_sub;
-    p.num_hg = pl.num_hg;
+    p.group = group;
+    p.num_sub = num_sub;
+    p.num_hg = num_kv_heads * num_sub;
     p.block_size = block_size;
     p.log2_bs = log2_int(block_size);
     p.max_blocks = max_blocks_per_seq;
     p.num_blocks = num_blocks;
-    p.fixed_units = pl.fixed_units;
+    p.fixed_units = partition_size > 0 ? std::max(1, partition_size / (mma ? 64 : 32)) : 0;
     p.rec_cap = (long long)pl.records;
     p.out_dtype = out_dtype;
     p.scale_log2 = scale * 1.4426950408889634f;
-    return launch_decode_simt(p, head_dim, kv_dtype, pl.group_pad,
-                              reinterpret_cast<cudaStream_t>(stream), nullptr);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (mma) return launch_decode_mma(p, head_dim, group_pad, st, nullptr);
+    return launch_decode_simt(p, head_dim, kv_dtype, group_pad, st, nullptr);
 }
 
 pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping,

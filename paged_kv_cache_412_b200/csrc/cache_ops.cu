@@ -23,6 +23,9 @@ __global__ void kv_cache_write_kernel(const uint4* __restrict__ k, const uint4* 
                                       uint4* __restrict__ vc, long long total_vecs,
                                       int vecs_per_row, int num_kv_heads, int block_size,
                                       int num_blocks, unsigned* err) {
+    // The previous kernel (a decode reading this cache) must be done first.
+    griddep_wait();
+    griddep_launch_dependents();
     const long long stride = (long long)gridDim.x * blockDim.x;
     for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total_vecs; i += stride) {
         const long long row = i / vecs_per_row;
@@ -78,11 +81,12 @@ pkv_status launch_kv_cache_write(const void* k, const void* v, const int64_t* sl
     const int threads = 256;
     const long long want = (total + threads - 1) / threads;
     const int grid = (int)std::min<long long>(want, (long long)di->num_sms * 8);
-    kv_cache_write_kernel<<<grid, threads, 0, stream>>>(
-        static_cast<const uint4*>(k), static_cast<const uint4*>(v), slots,
-        static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), total, vecs_per_row,
+    PdlLaunch L(dim3(grid), dim3(threads), 0, stream);
+    const cudaError_t e = cudaLaunchKernelEx(
+        &L.cfg, kv_cache_write_kernel, static_cast<const uint4*>(k), static_cast<const uint4*>(v),
+        slots, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), total, vecs_per_row,
         num_kv_heads, block_size, num_blocks, err);
-    return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 
 pkv_status launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int num_pairs,

@@ -1,0 +1,695 @@
+// decode_mma.cu -- paged decode attention with the q.K^T and P.V contractions
+// on the tensor cores (bf16 operands, fp32 accumulation), for bf16 caches with
+// block_size >= 8.
+//
+// What it computes ("PagedAttention: Optimizing KV Cache Utilization in Large
+// Language Models", "The Math: Block Attention Calculation", read as one
+// softmax over the whole request): for request b and query head h,
+//     out[b,h,:] = sum_t softmax_t(scale * q[b,h,:] . K_t) V_t,
+// with K_t / V_t located through the request's block table ("The Mechanics of
+// PagedAttention").
+//
+// Why tensor cores on an HBM-bound path: the CUDA-core version executes ~0.17
+// instructions per DRAM byte, which would need ~97 % of the SM issue ceiling at
+// the HBM copy peak.  Here a 16-token tile costs ~50 warp instructions.
+//
+// Shapes per 16-token tile (tokens are the MMA M dimension, the query heads of
+// the group -- padded to 8 per n-tile -- are N, so one K/V read serves the whole
+// group):
+//   S^T[16 x 8]  = K[16 x d] . Q^T[d x 8]        (d/16 mma.m16n8k16, A = K via ldmatrix)
+//   O^T[d x 8]  += V^T[d x 16] . P^T[16 x 8]     (d/16 mma per split, A = V^T via ldmatrix.trans)
+// P^T comes from the S^T accumulator: exp2 in fp32, packed to bf16 and moved
+// into the B-operand layout with movmatrix.trans.  P is split into bf16 hi + lo
+// parts (two MMAs) so the weights keep ~16 mantissa bits.
+//
+// Data movement: one producer warp walks the block table (32 entries per
+// coalesced load, next window prefetched, next segment's first window too) and
+// issues TMA tensor copies (2-D tensor map over the cache rows, 128-byte
+// swizzle, no multicast) of each physical block's K and V rows into a ring of
+// shared-memory stages with mbarrier completion.  One consumer warp per CTA
+// does the math, so no cross-warp reduction is needed; several CTAs share an
+// SM.  A request's (head group) split over several units is merged in-kernel by
+// the last unit to finish (per-group arrival counter in the workspace, reset by
+// the merger): out = sum_u 2^(m_u - M) acc_u / sum_u 2^(m_u - M) l_u.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <mutex>
+
+#include "decode_common.cuh"
+
+namespace pkv {
+namespace {
+
+constexpr int kCH = 64;         // tokens per stage
+constexpr int kMT = kCH / 16;   // 16-token MMA tiles per stage
+constexpr int kThreads = 64;    // producer warp + consumer warp
+constexpr int kRingBudget = 98304;
+
+constexpr int cmin(int a, int b) { return a < b ? a : b; }
+constexpr int cmax(int a, int b) { return a > b ? a : b; }
+
+template <int D, int NT>
+struct MmaCfg {
+    static constexpr int NHALF = D / 64;            // 128-byte column halves of a row
+    static constexpr int KS = D / 16;               // k-steps of q.K^T, m-tiles of P.V
+    static constexpr int HALF_BYTES = kCH * 128;    // one swizzled half region
+    static constexpr int KV_BYTES = NHALF * HALF_BYTES;
+    static constexpr int STAGE_BYTES = 2 * KV_BYTES;
+    static constexpr int NSTAGE = cmax(2, cmin(8, kRingBudget / STAGE_BYTES));
+    static constexpr int GP = 8 * NT;               // query heads per head group (padded)
+    static constexpr int OFF_BAR = NSTAGE * STAGE_BYTES;
+    static constexpr int OFF_META = OFF_BAR + 2 * NSTAGE * 8;
+    static constexpr int OFF_SCR = (OFF_META + 2 * NSTAGE * 4 + 15) / 16 * 16;
+    static constexpr int OFF_CTRL = OFF_SCR + 4 * 8;
+    static constexpr int SMEM = OFF_CTRL + 16 + 1024;  // + alignment slack
+};
+
+// ---- PTX wrappers -----------------------------------------------------------
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+
+__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float bf16_round(float x) {
+    return __bfloat162float(__float2bfloat16_rn(x));
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ float ld_cg(const float* p) { return __ldcg(p); }
+
+// ---- producer ------------------------------------------------------------------
+
+template <int D, int NT>
+struct Producer {
+    using C = MmaCfg<D, NT>;
+
+    const DecodeParams& p;
+    const CUtensorMap* tmk;
+    const CUtensorMap* tmv;
+    unsigned char* smem;
+    uint64_t* full;
+    uint64_t* empty;
+    int* st_ntok;
+    unsigned* st_bad;
+    volatile int* ctrl;
+    int lane;
+    uint64_t policy;
+    Ring ring;
+    int issued = 0;
+
+    __device__ int load_window(const Cursor& cur, int wbase) const {
+        const int nblk = (cur.L + p.block_size - 1) >> p.log2_bs;
+        const int j = wbase + lane;
+        return j < nblk ? __ldg(p.block_tables + (size_t)cur.b * p.max_blocks + j) : -1;
+    }
+
+    static __device__ __forceinline__ int first_block(int c0, int log2_bs) {
+        return (c0 * kCH) >> log2_bs;
+    }
+
+    // Returns false when the CTA must stop (a wait gave up).
+    __device__ bool run_segment(const Segment& sg, int tab_first) {
+        const Cursor& cur = sg.cur;
+        const int kvh = cur.hg / p.num_sub;
+        const int nblk = (cur.L + p.block_size - 1) >> p.log2_bs;
+        const int rb = min(p.block_size, kCH);  // rows per TMA box
+        int wbase = first_block(sg.c0, p.log2_bs) & ~31;
+        int tab = tab_first;
+        int tab_next = (wbase + 32 < nblk) ? load_window(cur, wbase + 32) : -1;
+        for (int c = sg.c0; c < sg.c1; ++c) {
+            const int t0 = c * kCH;
+            const int ntok = min(kCH, cur.L - t0);
+            const int ja = t0 >> p.log2_bs;
+            const int jb = (t0 + ntok - 1) >> p.log2_bs;
+            if (ja >= wbase + 32) {
+                wbase += 32;
+                tab = tab_next;
+                tab_next = (wbase + 32 < nblk) ? load_window(cur, wbase + 32) : -1;
+            }
+            int ok = 1;
+            if (lane == 0) ok = !ctrl[0] && mbar_wait(&empty[ring.stage], ring.phase ^ 1u);
+            ok = __shfl_sync(FULL_MASK, ok, 0);
+            if (!ok) {
+                if (lane == 0) {
+                    ctrl[0] = 1;
+                    raise_error(p.err, PKV_DEVERR_TIMEOUT);
+                }
+                return false;
+            }
+            uint32_t nvalid = 0, bad = 0;
+            for (int j = ja; j <= jb; ++j) {
+                const int phys = __shfl_sync(FULL_MASK, tab, j - wbase);
+                if (phys < 0 || phys >= p.num_blocks)
+                    bad |= 1u << (j - ja);
+                else
+                    ++nvalid;
+            }
+            unsigned char* sk = smem + ring.stage * C::STAGE_BYTES;
+            unsigned char* sv = sk + C::KV_BYTES;
+            if (lane == 0) {
+                st_ntok[ring.stage] = ntok;
+                st_bad[ring.stage] = bad;
+                if (bad) raise_error(p.err, PKV_DEVERR_BAD_BLOCK);
+                mbar_arrive_expect_tx(&full[ring.stage], nvalid * 2u * C::NHALF * rb * 128u);
+            }
+            for (int j = ja; j <= jb; ++j) {
+                const int phys = __shfl_sync(FULL_MASK, tab, j - wbase);
+                if (lane == 0 && phys >= 0 && phys < p.num_blocks) {
+                    // rows of this block in the stage, and where they start in the cache
+                    const int srow = (j << p.log2_bs) - t0 > 0 ? (j << p.log2_bs) - t0 : 0;
+                    const int boff = t0 - (j << p.log2_bs) > 0 ? t0 - (j << p.log2_bs) : 0;
+                    const int grow = (phys * p.num_kv_heads + kvh) * p.block_size + boff;
+#pragma unroll
+                    for (int h = 0; h < C::NHALF; ++h) {
+                        tma_load_2d(sk + h * C::HALF_BYTES + srow * 128, tmk, h * 64, grow,
+                                    &full[ring.stage], policy);
+                        tma_load_2d(sv + h * C::HALF_BYTES + srow * 128, tmv, h * 64, grow,
+                                    &full[ring.stage], policy);
+                    }
+                }
+            }
+            ++issued;
+            ring.advance(C::NSTAGE);
+        }
+        return true;
+    }
+
+    __device__ void run(SegIter<kCH>& it) {
+        int tab_first = -1;
+        if (it.valid) {
+            const Segment sg = it.current();
+            tab_first = load_window(sg.cur, first_block(sg.c0, p.log2_bs) & ~31);
+        }
+        while (it.valid) {
+            const Segment sg = it.current();
+            it.advance(p, lane);
+            // prefetch the next segment's first table window before streaming this one
+            int tab_after = -1;
+            if (it.valid) {
+                const Segment nx = it.current();
+                tab_after = load_window(nx.cur, first_block(nx.c0, p.log2_bs) & ~31);
+            }
+            if (!run_segment(sg, tab_first)) break;
+            tab_first = tab_after;
+        }
+        if (ctrl[0] && lane == 0) {
+            // A wait gave up somewhere in the CTA: before this warp exits, wait
+            // (bounded) for the stages it issued last, so no copy lands in
+            // shared memory after the CTA has gone.
+            const int n = min(issued, C::NSTAGE);
+            Ring r = ring;
+            for (int i = 0; i < n; ++i) {
+                if (r.stage == 0) {
+                    r.stage = C::NSTAGE - 1;
+                    r.phase ^= 1u;
+                } else {
+                    --r.stage;
+                }
+                mbar_wait(&full[r.stage], r.phase);
+            }
+        }
+    }
+};
+
+// ---- consumer ----------------------------------------------------------------
+
+template <int D, int NT>
+__device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
+                                        unsigned char* smem, uint64_t* full, uint64_t* empty,
+                                        const int* st_ntok, const unsigned* st_bad,
+                                        volatile int* ctrl, int lane) {
+    using C = MmaCfg<D, NT>;
+    constexpr int GP = C::GP;
+    const int grp = lane >> 2, tig = lane & 3;
+    const int mi = lane >> 3, r8 = lane & 7;
+    // ldmatrix row/chunk components that depend only on the lane
+    const int k_row = r8 + 8 * (mi & 1), k_cx = mi >> 1;  // K (A operand)
+    const int v_row = r8 + 8 * (mi >> 1), v_cx = mi & 1;  // V^T (A operand, transposed load)
+    Ring ring;
+
+    while (it.valid) {
+        const Segment sg = it.current();
+        it.advance(p, lane);
+        const Cursor& cur = sg.cur;
+        const long long u_first = sg.gstart / it.W;
+        const long long u_last = (sg.gstart + cur.nch - 1) / it.W;
+        const int nseg = (int)(u_last - u_first + 1);
+        const int kvh = cur.hg / p.num_sub, sub = cur.hg % p.num_sub;
+        const int hq0 = kvh * p.group + sub * GP;
+        const int gv = min(GP, p.group - sub * GP);
+        const size_t bg = (size_t)cur.b * p.num_hg + cur.hg;
+
+        // Q^T B-fragments: head nt*8+grp, dims ks*16 + 2*tig (+1) and +8 (+9).
+        uint32_t qb[NT][C::KS][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int h = nt * 8 + grp;
+            const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
+                static_cast<const __nv_bfloat16*>(p.q) +
+                ((size_t)cur.b * p.num_q_heads + hq0 + (h < gv ? h : 0)) * D);
+#pragma unroll
+            for (int ks = 0; ks < C::KS; ++ks) {
+                qb[nt][ks][0] = h < gv ? __ldg(qrow + ks * 8 + tig) : 0u;
+                qb[nt][ks][1] = h < gv ? __ldg(qrow + ks * 8 + 4 + tig) : 0u;
+            }
+        }
+        float m[NT][2], l[NT][2], acc[C::KS][NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            m[nt][0] = m[nt][1] = -INFINITY;
+            l[nt][0] = l[nt][1] = 0.f;
+#pragma unroll
+            for (int dt = 0; dt < C::KS; ++dt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[dt][nt][i] = 0.f;
+        }
+
+        for (int c = sg.c0; c < sg.c1; ++c) {
+            if (ctrl[0] || !mbar_wait(&full[ring.stage], ring.phase)) {
+                if (lane == 0 && !ctrl[0]) {
+                    ctrl[0] = 1;
+                    raise_error(p.err, PKV_DEVERR_TIMEOUT);
+                }
+                return;
+            }
+            const int ntok = st_ntok[ring.stage];
+            const unsigned bad = st_bad[ring.stage];
+            const bool whole = ntok == kCH && bad == 0;
+            unsigned char* sk = smem + ring.stage * C::STAGE_BYTES;
+            unsigned char* sv = sk + C::KV_BYTES;
+            const uint32_t skb = smem_addr(sk), svb = smem_addr(sv);
+
+            if (!whole) {
+                // Rows of tokens that do not take part (past the end, or in a
+                // block the table got wrong) may hold stale or poisoned data:
+                // zero their V rows so 0-weight x NaN cannot reach the sum.
+                for (int idx = lane; idx < kCH * C::NHALF * 8; idx += 32) {
+                    const int row = idx / (C::NHALF * 8);
+                    const int rest = idx % (C::NHALF * 8);
+                    const int jrel = ((c * kCH + row) >> p.log2_bs) - ((c * kCH) >> p.log2_bs);
+                    const bool valid = row < ntok && !((bad >> jrel) & 1u);
+                    if (!valid)
+                        *reinterpret_cast<uint4*>(sv + (rest >> 3) * C::HALF_BYTES + row * 128 +
+                                                  (rest & 7) * 16) = make_uint4(0, 0, 0, 0);
+                }
+                __syncwarp();
+            }
+
+            // ---- S^T = K . Q^T for the stage's 4 token tiles ----
+            float s[kMT][NT][4];
+#pragma unroll
+            for (int mt = 0; mt < kMT; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) s[mt][nt][i] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < C::KS; ++ks) {
+                const int half = ks >> 2;
+                const int chunk = (2 * (ks & 3) + k_cx) ^ r8;
+#pragma unroll
+                for (int mt = 0; mt < kMT; ++mt) {
+                    uint32_t a[4];
+                    ldsm_x4(skb + half * C::HALF_BYTES + (mt * 16 + k_row) * 128 + (chunk << 4), a);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) mma_bf16(s[mt][nt], a, qb[nt][ks][0], qb[nt][ks][1]);
+                }
+            }
+
+            // ---- scale, mask, online softmax (base 2) ----
+            bool grew = false;
+            float alpha[NT][2];
+#pragma unroll
+            for (int mt = 0; mt < kMT; ++mt) {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) s[mt][nt][i] *= p.scale_log2;
+                if (!whole) {
+#pragma unroll
+                    for (int hi = 0; hi < 2; ++hi) {
+                        const int row = mt * 16 + grp + 8 * hi;
+                        const int jrel = ((c * kCH + row) >> p.log2_bs) - ((c * kCH) >> p.log2_bs);
+                        const bool valid = row < ntok && !((bad >> jrel) & 1u);
+                        if (!valid) {
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt) {
+                                s[mt][nt][2 * hi] = -INFINITY;
+                                s[mt][nt][2 * hi + 1] = -INFINITY;
+                            }
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    float mx = fmaxf(s[0][nt][j], s[0][nt][j + 2]);
+#pragma unroll
+                    for (int mt = 1; mt < kMT; ++mt) mx = fmaxf(mx, fmaxf(s[mt][nt][j], s[mt][nt][j + 2]));
+                    mx = fmaxf(mx, __shfl_xor_sync(FULL_MASK, mx, 4));
+                    mx = fmaxf(mx, __shfl_xor_sync(FULL_MASK, mx, 8));
+                    mx = fmaxf(mx, __shfl_xor_sync(FULL_MASK, mx, 16));
+                    const float mnew = fmaxf(m[nt][j], mx);
+                    const float mref = mnew == -INFINITY ? 0.f : mnew;
+                    grew |= mnew > m[nt][j];
+                    alpha[nt][j] = exp2f(m[nt][j] - mref);
+                    m[nt][j] = mnew;
+                    float ps = 0.f;
+#pragma unroll
+                    for (int mt = 0; mt < kMT; ++mt) {
+                        s[mt][nt][j] = exp2f(s[mt][nt][j] - mref);
+                        s[mt][nt][j + 2] = exp2f(s[mt][nt][j + 2] - mref);
+                        ps += s[mt][nt][j] + s[mt][nt][j + 2];
+                    }
+                    l[nt][j] = fmaf(l[nt][j], alpha[nt][j], ps);
+                }
+            }
+            if (__any_sync(FULL_MASK, grew)) {
+#pragma unroll
+                for (int dt = 0; dt < C::KS; ++dt)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        acc[dt][nt][0] *= alpha[nt][0];
+                        acc[dt][nt][1] *= alpha[nt][1];
+                        acc[dt][nt][2] *= alpha[nt][0];
+                        acc[dt][nt][3] *= alpha[nt][1];
+                    }
+            }
+
+            // ---- O^T += V^T . P^T, P split into bf16 hi + lo ----
+#pragma unroll
+            for (int mt = 0; mt < kMT; ++mt) {
+                uint32_t bh[NT][2], bl[NT][2];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+                    for (int hi = 0; hi < 2; ++hi) {
+                        const float p0 = s[mt][nt][2 * hi], p1 = s[mt][nt][2 * hi + 1];
+                        const float h0 = bf16_round(p0), h1 = bf16_round(p1);
+                        bh[nt][hi] = movmatrix_t(pack_bf16(h0, h1));
+                        bl[nt][hi] = movmatrix_t(pack_bf16(p0 - h0, p1 - h1));
+                    }
+                }
+#pragma unroll
+                for (int dt = 0; dt < C::KS; ++dt) {
+                    const int half = dt >> 2;
+                    const int chunk = (2 * (dt & 3) + v_cx) ^ r8;
+                    uint32_t a[4];
+                    ldsm_x4_t(svb + half * C::HALF_BYTES + (mt * 16 + v_row) * 128 + (chunk << 4), a);
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        mma_bf16(acc[dt][nt], a, bh[nt][0], bh[nt][1]);
+                        mma_bf16(acc[dt][nt], a, bl[nt][0], bl[nt][1]);
+                    }
+                }
+            }
+            if (!whole) fence_proxy_async_smem();  // our zero-fill before the next TMA write
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[ring.stage]);
+            ring.advance(C::NSTAGE);
+        }
+
+        // ---- segment end: finish the normaliser, then output or record ----
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                l[nt][j] += __shfl_xor_sync(FULL_MASK, l[nt][j], 4);
+                l[nt][j] += __shfl_xor_sync(FULL_MASK, l[nt][j], 8);
+                l[nt][j] += __shfl_xor_sync(FULL_MASK, l[nt][j], 16);
+            }
+        if (nseg == 1) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int h = nt * 8 + 2 * tig + j;
+                    if (h >= gv) continue;
+                    const float inv = l[nt][j] > 0.f ? 1.f / l[nt][j] : 0.f;
+                    const size_t orow = ((size_t)cur.b * p.num_q_heads + hq0 + h) * D;
+#pragma unroll
+                    for (int dt = 0; dt < C::KS; ++dt) {
+                        store_out(p.out, orow + dt * 16 + grp, acc[dt][nt][j] * inv, p.out_dtype);
+                        store_out(p.out, orow + dt * 16 + grp + 8, acc[dt][nt][j + 2] * inv,
+                                  p.out_dtype);
+                    }
+                }
+            continue;
+        }
+        const long long rec = (long long)bg + sg.u;
+        if (bg + u_last >= (size_t)p.rec_cap) {
+            if (lane == 0) raise_error(p.err, PKV_DEVERR_BAD_SEQ_LEN);
+            continue;
+        }
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int h = nt * 8 + 2 * tig + j;
+                float* ra = p.rec_acc + ((size_t)rec * GP + h) * D;
+#pragma unroll
+                for (int dt = 0; dt < C::KS; ++dt) {
+                    ra[dt * 16 + grp] = acc[dt][nt][j];
+                    ra[dt * 16 + grp + 8] = acc[dt][nt][j + 2];
+                }
+                if (grp == 0) {
+                    p.rec_ml[((size_t)rec * GP + h) * 2] = m[nt][j];
+                    p.rec_ml[((size_t)rec * GP + h) * 2 + 1] = l[nt][j];
+                }
+            }
+        __threadfence();
+        __syncwarp();
+        unsigned arrived = 0;
+        if (lane == 0) arrived = atomicAdd(reinterpret_cast<unsigned*>(p.counters) + bg, 1u);
+        arrived = __shfl_sync(FULL_MASK, arrived, 0);
+        if (arrived != (unsigned)(nseg - 1)) continue;
+        // Last unit of this (request, head group) to finish: merge all records.
+        __threadfence();
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int h = nt * 8 + 2 * tig + j;
+                float M = -INFINITY;
+                for (long long uu = u_first; uu <= u_last; ++uu)
+                    M = fmaxf(M, ld_cg(p.rec_ml + (((size_t)bg + uu) * GP + h) * 2));
+                const float mref = M == -INFINITY ? 0.f : M;
+                float S = 0.f;
+                float A[C::KS][2];
+#pragma unroll
+                for (int dt = 0; dt < C::KS; ++dt) A[dt][0] = A[dt][1] = 0.f;
+                for (long long uu = u_first; uu <= u_last; ++uu) {
+                    const size_t rr = ((size_t)bg + uu) * GP + h;
+                    const float f = exp2f(ld_cg(p.rec_ml + rr * 2) - mref);
+                    S = fmaf(ld_cg(p.rec_ml + rr * 2 + 1), f, S);
+                    const float* ra = p.rec_acc + rr * D;
+#pragma unroll
+                    for (int dt = 0; dt < C::KS; ++dt) {
+                        A[dt][0] = fmaf(ld_cg(ra + dt * 16 + grp), f, A[dt][0]);
+                        A[dt][1] = fmaf(ld_cg(ra + dt * 16 + grp + 8), f, A[dt][1]);
+                    }
+                }
+                if (h >= gv) continue;
+                const float inv = S > 0.f ? 1.f / S : 0.f;
+                const size_t orow = ((size_t)cur.b * p.num_q_heads + hq0 + h) * D;
+#pragma unroll
+                for (int dt = 0; dt < C::KS; ++dt) {
+                    store_out(p.out, orow + dt * 16 + grp, A[dt][0] * inv, p.out_dtype);
+                    store_out(p.out, orow + dt * 16 + grp + 8, A[dt][1] * inv, p.out_dtype);
+                }
+            }
+        if (lane == 0) reinterpret_cast<unsigned*>(p.counters)[bg] = 0u;  // ready for the next call
+    }
+}
+
+template <int D, int NT>
+__global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_constant__ DecodeParams p,
+                                                             const __grid_constant__ CUtensorMap tmk,
+                                                             const __grid_constant__ CUtensorMap tmv) {
+    using C = MmaCfg<D, NT>;
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* empty = full + C::NSTAGE;
+    int* st_ntok = reinterpret_cast<int*>(smem + C::OFF_META);
+    unsigned* st_bad = reinterpret_cast<unsigned*>(st_ntok + C::NSTAGE);
+    long long* scratch = reinterpret_cast<long long*>(smem + C::OFF_SCR);
+    volatile int* ctrl = reinterpret_cast<volatile int*>(smem + C::OFF_CTRL);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        ctrl[0] = 0;
+        for (int s = 0; s < C::NSTAGE; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        fence_mbar_init();
+        prefetch_tensormap(&tmk);
+        prefetch_tensormap(&tmv);
+    }
+    // Everything above overlaps the previous kernel in the stream; from here
+    // on we read memory it may have written.
+    griddep_wait();
+    griddep_launch_dependents();
+
+    const long long total = total_chunks<kCH>(p, scratch, blockIdx.x == 0);
+    if (warp == 1) {
+        // empty requests: all-zero rows (softmax of an empty set)
+        for (int b = blockIdx.x; b < p.num_seqs; b += gridDim.x) {
+            if (clamp_len(p, b, false) != 0) continue;
+            for (int i = lane; i < p.num_q_heads * D; i += 32)
+                store_out(p.out, (size_t)b * p.num_q_heads * D + i, 0.f, p.out_dtype);
+        }
+    }
+    if (total == 0) return;
+    long long W = p.fixed_units > 0 ? p.fixed_units : (total + gridDim.x - 1) / gridDim.x;
+    if (W < 1) W = 1;
+    SegIter<kCH> it;
+    it.init(p, total, W, lane);
+
+    if (warp == 0) {
+        Producer<D, NT> pr{p, &tmk, &tmv, smem, full, empty, st_ntok, st_bad, ctrl, lane,
+                           l2_policy_evict_first()};
+        pr.run(it);
+    } else {
+        consume<D, NT>(p, it, smem, full, empty, st_ntok, st_bad, ctrl, lane);
+    }
+}
+
+// ---- host side ---------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// 2-D view of a cache: rows = num_blocks*Hkv*block_size, columns = head_dim
+// bf16; boxes of 64 columns x min(block_size, 64) rows, 128-byte swizzle.
+bool encode_cache_map(CUtensorMap* map, const void* base, long long rows, int head_dim,
+                      int box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t gdim[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
+    cuuint64_t gstride[1] = {(cuuint64_t)head_dim * 2};
+    cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+    cuuint32_t estride[2] = {1u, 1u};
+    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim,
+                           gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int D, int NT>
+pkv_status launch_impl(const DecodeParams& p, cudaStream_t stream, int* grid_out) {
+    using C = MmaCfg<D, NT>;
+    const DeviceInfo* di = current_device_info();
+    if (!di) return PKV_ERR_CUDA;
+    static std::mutex mu;
+    static int occupancy[64] = {0};
+    auto kern = decode_mma_kernel<D, NT>;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (di->device >= 64) return PKV_ERR_UNSUPPORTED;
+        if (occupancy[di->device] == 0) {
+            if (C::SMEM > di->max_smem_optin) return PKV_ERR_UNSUPPORTED;
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+                cudaSuccess)
+                return PKV_ERR_CUDA;
+            int occ = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, C::SMEM) !=
+                    cudaSuccess ||
+                occ < 1)
+                return PKV_ERR_CUDA;
+            occupancy[di->device] = occ;
+        }
+    }
+    const long long rows = (long long)p.num_blocks * p.num_kv_heads * p.block_size;
+    const int box_rows = std::min(p.block_size, kCH);
+    CUtensorMap tmk, tmv;
+    if (!encode_cache_map(&tmk, p.k_cache, rows, D, box_rows) ||
+        !encode_cache_map(&tmv, p.v_cache, rows, D, box_rows))
+        return PKV_ERR_CUDA;
+    const int grid = di->num_sms * std::min(occupancy[di->device], 4);
+
+    PdlLaunch L(dim3(grid), dim3(kThreads), C::SMEM, stream);
+    if (cudaLaunchKernelEx(&L.cfg, kern, p, tmk, tmv) != cudaSuccess) return PKV_ERR_CUDA;
+    if (grid_out) *grid_out = grid;
+    return PKV_OK;
+}
+
+}  // namespace
+
+bool decode_mma_supported(int head_dim, int block_size, pkv_dtype q_dtype, pkv_dtype kv_dtype) {
+    return q_dtype == PKV_BF16 && kv_dtype == PKV_BF16 && (head_dim == 64 || head_dim == 128) &&
+           block_size >= 8;
+}
+
+pkv_status launch_decode_mma(const DecodeParams& p, int head_dim, int group_pad,
+                             cudaStream_t stream, int* grid_out) {
+    const int nt = group_pad > 8 ? 2 : 1;
+    if (head_dim == 128) return nt == 1 ? launch_impl<128, 1>(p, stream, grid_out)
+                                        : launch_impl<128, 2>(p, stream, grid_out);
+    if (head_dim == 64) return nt == 1 ? launch_impl<64, 1>(p, stream, grid_out)
+                                       : launch_impl<64, 2>(p, stream, grid_out);
+    return PKV_ERR_UNSUPPORTED;
+}
+
+}  // namespace pkv

@@ -34,8 +34,7 @@
 #include <algorithm>
 #include <mutex>
 
-#include "pkv_device.cuh"
-#include "pkv_internal.h"
+#include "decode_common.cuh"
 
 namespace pkv {
 namespace {
@@ -75,85 +74,15 @@ struct SimtCfg {
     static_assert(ROW_BYTES % 16 == 0, "rows must be whole 16-byte vectors");
 };
 
-__device__ __forceinline__ int clamp_len(const DecodeParams& p, int b, bool flag) {
-    int L = __ldg(p.seq_lens + b);
-    const int cap = p.max_blocks * p.block_size;
-    if (L < 0 || L > cap) {
-        if (flag) raise_error(p.err, PKV_DEVERR_BAD_SEQ_LEN);
-        L = L < 0 ? 0 : cap;
-    }
-    return L;
+__device__ __forceinline__ int chunks_of_len(int L) { return chunks_of<kChunk>(L); }
+
+__device__ __forceinline__ Cursor locate(const DecodeParams& p, long long s, int lane) {
+    return pkv::locate<kChunk>(p, s, lane);
 }
 
-__device__ __forceinline__ int chunks_of_len(int L) { return (L + kChunk - 1) / kChunk; }
-
-// Position in the flattened (request, head group, chunk) list.
-struct Cursor {
-    int b, hg, c, nch, L;
-};
-
-// Warp-cooperative search for global chunk index s.
-__device__ Cursor locate(const DecodeParams& p, long long s, int lane) {
-    Cursor cur{p.num_seqs, 0, 0, 0, 0};
-    long long base = 0;
-    for (int b0 = 0; b0 < p.num_seqs; b0 += 32) {
-        const int b = b0 + lane;
-        const int L = b < p.num_seqs ? clamp_len(p, b, false) : 0;
-        const long long n = (long long)chunks_of_len(L) * p.num_hg;
-        long long incl = n;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const long long t = __shfl_up_sync(FULL_MASK, incl, off);
-            if (lane >= off) incl += t;
-        }
-        const long long excl = incl - n;
-        const unsigned hit =
-            __ballot_sync(FULL_MASK, n > 0 && base + excl <= s && s < base + incl);
-        if (hit) {
-            const int src = __ffs(hit) - 1;
-            const int Lb = __shfl_sync(FULL_MASK, L, src);
-            const long long ex = __shfl_sync(FULL_MASK, excl, src);
-            const long long off = s - (base + ex);
-            const int nch = chunks_of_len(Lb);
-            cur.b = b0 + src;
-            cur.L = Lb;
-            cur.nch = nch;
-            cur.hg = (int)(off / nch);
-            cur.c = (int)(off % nch);
-            return cur;
-        }
-        base += __shfl_sync(FULL_MASK, incl, 31);
-    }
-    return cur;
-}
-
-// Move to chunk 0 of the next non-empty (request, head group).
 __device__ __forceinline__ void next_group(const DecodeParams& p, Cursor& cur) {
-    cur.c = 0;
-    if (++cur.hg < p.num_hg) return;
-    cur.hg = 0;
-    for (;;) {
-        if (++cur.b >= p.num_seqs) {
-            cur.nch = 0;
-            return;
-        }
-        cur.L = clamp_len(p, cur.b, false);
-        cur.nch = chunks_of_len(cur.L);
-        if (cur.nch > 0) return;
-    }
+    pkv::next_group<kChunk>(p, cur);
 }
-
-// Shared pipeline position (producer and consumers advance identically).
-struct Ring {
-    int stage = 0;
-    uint32_t phase = 0;
-    __device__ __forceinline__ void advance(int nstage) {
-        if (++stage == nstage) {
-            stage = 0;
-            phase ^= 1u;
-        }
-    }
-};
 
 template <typename KV, int D, int GP>
 __device__ __forceinline__ void produce_segment(const DecodeParams& p, const Cursor& cur, int c0,

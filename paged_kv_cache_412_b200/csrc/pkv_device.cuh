@@ -96,6 +96,17 @@ __device__ __forceinline__ void bulk_load(void* dst_smem, const void* src_gmem, 
         : "memory");
 }
 
+// ---- programmatic dependent launch ------------------------------------------
+
+// Wait until the previous kernel in the stream has completed and its writes are
+// visible (no-op when the kernel was not launched as a dependent).
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Let the next kernel in the stream begin launching.
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ---- named barriers ---------------------------------------------------------
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {

@@ -21,24 +21,21 @@ struct DeviceInfo {
 // Info for the current device (thread-safe, cached).  nullptr on failure.
 const DeviceInfo* current_device_info();
 
-// Decomposition of one decode call, shared by the workspace sizing and the
-// launch so both agree.
+// Workspace bound of one decode call.  It covers both decode kernels (the
+// tensor-core one groups up to 16 query heads per kv-head pass, the CUDA-core
+// one up to 8), so one size fits whichever path the call takes.
 struct DecodePlan {
-    int group_pad;     // query heads per head group, padded to 1/2/4/8
-    int num_sub;       // head groups per kv head (ceil(G / 8) when G > 8)
-    int num_hg;        // head groups per request = num_kv_heads * num_sub
-    int chunk_tokens;  // tokens per pipeline stage
-    int fixed_units;   // chunks per split unit when partition_size > 0, else 0
-    int grid;          // persistent CTAs
+    int rec_gp;        // floats per record row = largest query-head group of either path
+    size_t n_bg_max;   // (request, head group) pairs, largest over the paths
     size_t units_max;  // upper bound of split units
     size_t records;    // partial-result records
+    size_t off_ml, off_meta, off_cnt;  // byte offsets of the workspace regions
     size_t bytes;      // workspace bytes
 };
 
 // Fill a plan for these sizes on the current device (false if invalid).
 bool make_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
-                      int block_size, int max_seq_len, int partition_size, int ctas_per_sm,
-                      DecodePlan* plan);
+                      int block_size, int max_seq_len, int partition_size, DecodePlan* plan);
 
 // Kernel arguments of the decode path (plain values, passed by value).
 struct DecodeParams {
@@ -53,6 +50,7 @@ struct DecodeParams {
     float* rec_acc;   // [records][group_pad][head_dim]
     float* rec_ml;    // [records][group_pad][2]  (running max in log2 units, sum)
     int32_t* meta;    // [num_seqs * num_hg][2]   (first unit, number of units)
+    unsigned* counters;  // [num_seqs * num_hg] arrivals per split group (zero between calls)
     unsigned* err;
     int num_seqs, num_q_heads, num_kv_heads, group, num_sub, num_hg;
     int block_size, log2_bs, max_blocks, num_blocks;
@@ -64,6 +62,29 @@ struct DecodeParams {
 
 pkv_status launch_decode_simt(const DecodeParams& p, int head_dim, pkv_dtype kv_dtype,
                               int group_pad, cudaStream_t stream, int* grid_out);
+
+bool decode_mma_supported(int head_dim, int block_size, pkv_dtype q_dtype, pkv_dtype kv_dtype);
+
+pkv_status launch_decode_mma(const DecodeParams& p, int head_dim, int group_pad,
+                             cudaStream_t stream, int* grid_out);
+
+// Launch config with programmatic dependent launch: the kernel may start while
+// the previous kernel in the stream drains; it waits (griddepcontrol.wait)
+// before touching memory.
+struct PdlLaunch {
+    cudaLaunchConfig_t cfg{};
+    cudaLaunchAttribute attr[1];
+    PdlLaunch(dim3 grid, dim3 block, size_t smem, cudaStream_t s) {
+        cfg.gridDim = grid;
+        cfg.blockDim = block;
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = s;
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+    }
+};
 
 pkv_status launch_kv_cache_write(const void* k, const void* v, const int64_t* slots,
                                  void* k_cache, void* v_cache, int num_tokens, int num_kv_heads,

@@ -71,6 +71,10 @@ SMALL = [
     ([300, 129], 8, 2, 128, 64, "bf16"),         # block larger than a stage
     ([513, 20], 8, 4, 64, 256, "f32"),           # block size 256
     ([0, 40, 0, 1], 4, 2, 128, 16, "bf16"),      # empty requests
+    ([513, 20, 300], 8, 4, 64, 256, "bf16"),     # tensor-core path, block 256 > stage
+    ([700, 129], 32, 8, 128, 128, "bf16"),       # tensor-core path, block 128
+    ([100, 260], 32, 1, 128, 16, "bf16"),        # G = 32: two 16-head passes per kv head
+    ([64, 65, 63, 128], 8, 2, 64, 8, "bf16"),    # stage-boundary lengths, d 64
 ]
 
 
