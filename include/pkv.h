@@ -147,6 +147,14 @@ pkv_status pkv_decode_workspace_init(void* workspace, size_t workspace_bytes,
  *   partition_size  0 = automatic split of the whole batch's KV into equal
  *                 shares, one per resident CTA; else tokens per split unit
  *                 (a multiple of 32).
+ *   Ordering: the kernel is launched as a programmatic dependent of the
+ *                 previous kernel in the stream and reads seq_lens and
+ *                 block_tables while that kernel drains; it waits for it before
+ *                 touching q, the caches, out or the workspace.  So seq_lens and
+ *                 block_tables must not be written by the kernel immediately
+ *                 before this call if that kernel releases its dependents early
+ *                 (griddepcontrol.launch_dependents); host copies and ordinary
+ *                 kernels are fine, and so is pkv_kv_cache_write.
  *   workspace     device scratch of at least pkv_decode_workspace_bytes(...)
  *                 bytes, 256-byte aligned, zeroed once by
  *                 pkv_decode_workspace_init.  Calls that overlap in time need

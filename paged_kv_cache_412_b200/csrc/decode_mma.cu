@@ -44,8 +44,8 @@ namespace {
 
 constexpr int kCH = 64;         // tokens per stage
 constexpr int kMT = kCH / 16;   // 16-token MMA tiles per stage
-constexpr int kThreads = 64;    // producer warp + consumer warp
-constexpr int kRingBudget = 98304;
+constexpr int kThreads = 96;    // producer, tensor-core consumer, epilogue
+constexpr int kRingBudget = 104448;  // 3 stages of K+V+q at head_dim 128
 
 constexpr int cmin(int a, int b) { return a < b ? a : b; }
 constexpr int cmax(int a, int b) { return a > b ? a : b; }
@@ -56,14 +56,11 @@ struct MmaCfg {
     static constexpr int KS = D / 16;               // k-steps of q.K^T, m-tiles of P.V
     static constexpr int HALF_BYTES = kCH * 128;    // one swizzled half region
     static constexpr int KV_BYTES = NHALF * HALF_BYTES;
-    static constexpr int STAGE_BYTES = 2 * KV_BYTES;
-    static constexpr int NSTAGE = cmax(2, cmin(8, kRingBudget / STAGE_BYTES));
     static constexpr int GP = 8 * NT;               // query heads per head group (padded)
-    static constexpr int OFF_BAR = NSTAGE * STAGE_BYTES;
-    static constexpr int OFF_META = OFF_BAR + 2 * NSTAGE * 8;
-    static constexpr int OFF_SCR = (OFF_META + 2 * NSTAGE * 4 + 15) / 16 * 16;
-    static constexpr int OFF_CTRL = OFF_SCR + 4 * 8;
-    static constexpr int SMEM = OFF_CTRL + 16 + 1024;  // + alignment slack
+    static constexpr int Q_BYTES = GP * D * 2;      // the group's q rows (first stage of a segment)
+    // K | V | q, rounded to the 1 KB the 128-byte swizzle pattern repeats on
+    static constexpr int STAGE_BYTES = (2 * KV_BYTES + Q_BYTES + 1023) / 1024 * 1024;
+    static constexpr int NSTAGE = cmax(2, cmin(8, kRingBudget / STAGE_BYTES));
 };
 
 // ---- PTX wrappers -----------------------------------------------------------
@@ -123,6 +120,22 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 
 __device__ __forceinline__ float ld_cg(const float* p) { return __ldcg(p); }
 
+// ---- shared-memory layout ------------------------------------------------------
+
+template <int D, int NT>
+struct Smem {
+    using C = MmaCfg<D, NT>;
+    static constexpr int NDUMP = 2;                       // consumer -> epilogue hand-off slots
+    static constexpr int DUMP_ACC = C::KS * NT * 4;       // acc registers per lane
+    static constexpr int DUMP_ML = NT * 4;                // m[2], l[2] per n-tile per lane
+    static constexpr int DUMP_BYTES = (DUMP_ACC + DUMP_ML) * 32 * 4;
+    static constexpr int OFF_DUMP = C::NSTAGE * C::STAGE_BYTES;
+    static constexpr int OFF_BAR = OFF_DUMP + NDUMP * DUMP_BYTES;
+    static constexpr int OFF_META = OFF_BAR + (2 * C::NSTAGE + 2 * NDUMP) * 8;
+    static constexpr int OFF_CTRL = OFF_META + 2 * C::NSTAGE * 4;
+    static constexpr int BYTES = OFF_CTRL + 16 + 1024;   // + alignment slack
+};
+
 // ---- producer ------------------------------------------------------------------
 
 template <int D, int NT>
@@ -142,6 +155,7 @@ struct Producer {
     uint64_t policy;
     Ring ring;
     int issued = 0;
+    bool waited = false;
 
     __device__ int load_window(const Cursor& cur, int wbase) const {
         const int nblk = (cur.L + p.block_size - 1) >> p.log2_bs;
@@ -156,7 +170,9 @@ struct Producer {
     // Returns false when the CTA must stop (a wait gave up).
     __device__ bool run_segment(const Segment& sg, int tab_first) {
         const Cursor& cur = sg.cur;
-        const int kvh = cur.hg / p.num_sub;
+        const int kvh = cur.hg / p.num_sub, sub = cur.hg % p.num_sub;
+        const int hq0 = kvh * p.group + sub * C::GP;
+        const int gv = min(C::GP, p.group - sub * C::GP);
         const int nblk = (cur.L + p.block_size - 1) >> p.log2_bs;
         const int rb = min(p.block_size, kCH);  // rows per TMA box
         int wbase = first_block(sg.c0, p.log2_bs) & ~31;
@@ -182,6 +198,11 @@ struct Producer {
                 }
                 return false;
             }
+            if (!waited) {
+                // K/V and q may come from the previous kernel in the stream.
+                griddep_wait();
+                waited = true;
+            }
             uint32_t nvalid = 0, bad = 0;
             for (int j = ja; j <= jb; ++j) {
                 const int phys = __shfl_sync(FULL_MASK, tab, j - wbase);
@@ -192,11 +213,18 @@ struct Producer {
             }
             unsigned char* sk = smem + ring.stage * C::STAGE_BYTES;
             unsigned char* sv = sk + C::KV_BYTES;
+            unsigned char* sq = sv + C::KV_BYTES;
             if (lane == 0) {
                 st_ntok[ring.stage] = ntok;
                 st_bad[ring.stage] = bad;
                 if (bad) raise_error(p.err, PKV_DEVERR_BAD_BLOCK);
-                mbar_arrive_expect_tx(&full[ring.stage], nvalid * 2u * C::NHALF * rb * 128u);
+                const uint32_t qbytes = c == sg.c0 ? (uint32_t)gv * D * 2u : 0u;
+                mbar_arrive_expect_tx(&full[ring.stage],
+                                      nvalid * 2u * C::NHALF * rb * 128u + qbytes);
+                if (qbytes)  // the group's q rows ride with the segment's first stage
+                    bulk_load(sq, static_cast<const __nv_bfloat16*>(p.q) +
+                                      ((size_t)cur.b * p.num_q_heads + hq0) * D,
+                              qbytes, &full[ring.stage], policy);
             }
             for (int j = ja; j <= jb; ++j) {
                 const int phys = __shfl_sync(FULL_MASK, tab, j - wbase);
@@ -257,48 +285,51 @@ struct Producer {
     }
 };
 
-// ---- consumer ----------------------------------------------------------------
+// Per-segment facts every role derives the same way.
+struct SegInfo {
+    long long u, u_first, u_last;
+    int nseg, hq0, gv, b;
+    size_t bg;
+};
+
+template <int GP>
+__device__ __forceinline__ SegInfo seg_info(const DecodeParams& p, const Segment& sg, long long W) {
+    SegInfo si;
+    si.u = sg.u;
+    si.u_first = sg.gstart / W;
+    si.u_last = (sg.gstart + sg.cur.nch - 1) / W;
+    si.nseg = (int)(si.u_last - si.u_first + 1);
+    const int kvh = sg.cur.hg / p.num_sub, sub = sg.cur.hg % p.num_sub;
+    si.hq0 = kvh * p.group + sub * GP;
+    si.gv = min(GP, p.group - sub * GP);
+    si.b = sg.cur.b;
+    si.bg = (size_t)sg.cur.b * p.num_hg + sg.cur.hg;
+    return si;
+}
+
+// ---- consumer (tensor-core math) ----------------------------------------------
 
 template <int D, int NT>
 __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                                         unsigned char* smem, uint64_t* full, uint64_t* empty,
-                                        const int* st_ntok, const unsigned* st_bad,
-                                        volatile int* ctrl, int lane) {
+                                        uint64_t* dfull, uint64_t* dempty, const int* st_ntok,
+                                        const unsigned* st_bad, volatile int* ctrl, int lane) {
     using C = MmaCfg<D, NT>;
+    using S = Smem<D, NT>;
     constexpr int GP = C::GP;
     const int grp = lane >> 2, tig = lane & 3;
     const int mi = lane >> 3, r8 = lane & 7;
     // ldmatrix row/chunk components that depend only on the lane
     const int k_row = r8 + 8 * (mi & 1), k_cx = mi >> 1;  // K (A operand)
     const int v_row = r8 + 8 * (mi >> 1), v_cx = mi & 1;  // V^T (A operand, transposed load)
-    Ring ring;
+    Ring ring, dring;
 
     while (it.valid) {
         const Segment sg = it.current();
         it.advance(p, lane);
-        const Cursor& cur = sg.cur;
-        const long long u_first = sg.gstart / it.W;
-        const long long u_last = (sg.gstart + cur.nch - 1) / it.W;
-        const int nseg = (int)(u_last - u_first + 1);
-        const int kvh = cur.hg / p.num_sub, sub = cur.hg % p.num_sub;
-        const int hq0 = kvh * p.group + sub * GP;
-        const int gv = min(GP, p.group - sub * GP);
-        const size_t bg = (size_t)cur.b * p.num_hg + cur.hg;
+        const SegInfo si = seg_info<GP>(p, sg, it.W);
 
-        // Q^T B-fragments: head nt*8+grp, dims ks*16 + 2*tig (+1) and +8 (+9).
         uint32_t qb[NT][C::KS][2];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const int h = nt * 8 + grp;
-            const uint32_t* qrow = reinterpret_cast<const uint32_t*>(
-                static_cast<const __nv_bfloat16*>(p.q) +
-                ((size_t)cur.b * p.num_q_heads + hq0 + (h < gv ? h : 0)) * D);
-#pragma unroll
-            for (int ks = 0; ks < C::KS; ++ks) {
-                qb[nt][ks][0] = h < gv ? __ldg(qrow + ks * 8 + tig) : 0u;
-                qb[nt][ks][1] = h < gv ? __ldg(qrow + ks * 8 + 4 + tig) : 0u;
-            }
-        }
         float m[NT][2], l[NT][2], acc[C::KS][NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) {
@@ -324,6 +355,20 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
             unsigned char* sk = smem + ring.stage * C::STAGE_BYTES;
             unsigned char* sv = sk + C::KV_BYTES;
             const uint32_t skb = smem_addr(sk), svb = smem_addr(sv);
+
+            if (c == sg.c0) {
+                // Q^T B-fragments: head nt*8+grp, dims ks*16 + 2*tig (+1) and +8 (+9).
+                const uint32_t* sq = reinterpret_cast<const uint32_t*>(sv + C::KV_BYTES);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const int h = nt * 8 + grp;
+#pragma unroll
+                    for (int ks = 0; ks < C::KS; ++ks) {
+                        qb[nt][ks][0] = h < si.gv ? sq[h * (D / 2) + ks * 8 + tig] : 0u;
+                        qb[nt][ks][1] = h < si.gv ? sq[h * (D / 2) + ks * 8 + 4 + tig] : 0u;
+                    }
+                }
+            }
 
             if (!whole) {
                 // Rows of tokens that do not take part (past the end, or in a
@@ -457,7 +502,84 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
             ring.advance(C::NSTAGE);
         }
 
-        // ---- segment end: finish the normaliser, then output or record ----
+        // ---- hand the segment's state to the epilogue warp ----
+        if (!mbar_wait(&dempty[dring.stage], dring.phase ^ 1u)) {
+            if (lane == 0) {
+                ctrl[0] = 1;
+                raise_error(p.err, PKV_DEVERR_TIMEOUT);
+            }
+            return;
+        }
+        float* dump = reinterpret_cast<float*>(smem + S::OFF_DUMP + dring.stage * S::DUMP_BYTES);
+#pragma unroll
+        for (int dt = 0; dt < C::KS; ++dt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) dump[((dt * NT + nt) * 4 + i) * 32 + lane] = acc[dt][nt][i];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                dump[(S::DUMP_ACC + nt * 4 + j) * 32 + lane] = m[nt][j];
+                dump[(S::DUMP_ACC + nt * 4 + 2 + j) * 32 + lane] = l[nt][j];
+            }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&dfull[dring.stage]);
+        dring.advance(S::NDUMP);
+    }
+}
+
+// ---- epilogue: normalise, or write a partial record and merge the group ----
+
+template <int D, int NT>
+__device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it,
+                                         unsigned char* smem, uint64_t* dfull, uint64_t* dempty,
+                                         volatile int* ctrl, int lane) {
+    using C = MmaCfg<D, NT>;
+    using S = Smem<D, NT>;
+    constexpr int GP = C::GP;
+    const int grp = lane >> 2, tig = lane & 3;
+    Ring dring;
+    griddep_wait();  // `out` and the workspace may be in use by the previous kernel
+    // empty requests: all-zero rows (softmax of an empty set)
+    for (int b = blockIdx.x; b < p.num_seqs; b += gridDim.x) {
+        if (clamp_len(p, b, false) != 0) continue;
+        for (int i = lane; i < p.num_q_heads * D; i += 32)
+            store_out(p.out, (size_t)b * p.num_q_heads * D + i, 0.f, p.out_dtype);
+    }
+    while (it.valid) {
+        const Segment sg = it.current();
+        it.advance(p, lane);
+        const SegInfo si = seg_info<GP>(p, sg, it.W);
+        if (ctrl[0] || !mbar_wait(&dfull[dring.stage], dring.phase)) {
+            if (lane == 0 && !ctrl[0]) {
+                ctrl[0] = 1;
+                raise_error(p.err, PKV_DEVERR_TIMEOUT);
+            }
+            return;
+        }
+        const float* dump =
+            reinterpret_cast<const float*>(smem + S::OFF_DUMP + dring.stage * S::DUMP_BYTES);
+        float acc[C::KS][NT][4], m[NT][2], l[NT][2];
+#pragma unroll
+        for (int dt = 0; dt < C::KS; ++dt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) acc[dt][nt][i] = dump[((dt * NT + nt) * 4 + i) * 32 + lane];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                m[nt][j] = dump[(S::DUMP_ACC + nt * 4 + j) * 32 + lane];
+                l[nt][j] = dump[(S::DUMP_ACC + nt * 4 + 2 + j) * 32 + lane];
+            }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&dempty[dring.stage]);
+        dring.advance(S::NDUMP);
+
+        // the normaliser: sum the per-lane partials over the lanes sharing a head
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -466,15 +588,15 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                 l[nt][j] += __shfl_xor_sync(FULL_MASK, l[nt][j], 8);
                 l[nt][j] += __shfl_xor_sync(FULL_MASK, l[nt][j], 16);
             }
-        if (nseg == 1) {
+        if (si.nseg == 1) {
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     const int h = nt * 8 + 2 * tig + j;
-                    if (h >= gv) continue;
+                    if (h >= si.gv) continue;
                     const float inv = l[nt][j] > 0.f ? 1.f / l[nt][j] : 0.f;
-                    const size_t orow = ((size_t)cur.b * p.num_q_heads + hq0 + h) * D;
+                    const size_t orow = ((size_t)si.b * p.num_q_heads + si.hq0 + h) * D;
 #pragma unroll
                     for (int dt = 0; dt < C::KS; ++dt) {
                         store_out(p.out, orow + dt * 16 + grp, acc[dt][nt][j] * inv, p.out_dtype);
@@ -484,33 +606,34 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                 }
             continue;
         }
-        const long long rec = (long long)bg + sg.u;
-        if (bg + u_last >= (size_t)p.rec_cap) {
+        if (si.bg + si.u_last >= (size_t)p.rec_cap) {
             if (lane == 0) raise_error(p.err, PKV_DEVERR_BAD_SEQ_LEN);
             continue;
         }
+        const size_t rec = si.bg + si.u;
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 const int h = nt * 8 + 2 * tig + j;
-                float* ra = p.rec_acc + ((size_t)rec * GP + h) * D;
+                float* ra = p.rec_acc + (rec * GP + h) * D;
 #pragma unroll
                 for (int dt = 0; dt < C::KS; ++dt) {
                     ra[dt * 16 + grp] = acc[dt][nt][j];
                     ra[dt * 16 + grp + 8] = acc[dt][nt][j + 2];
                 }
                 if (grp == 0) {
-                    p.rec_ml[((size_t)rec * GP + h) * 2] = m[nt][j];
-                    p.rec_ml[((size_t)rec * GP + h) * 2 + 1] = l[nt][j];
+                    p.rec_ml[(rec * GP + h) * 2] = m[nt][j];
+                    p.rec_ml[(rec * GP + h) * 2 + 1] = l[nt][j];
                 }
             }
         __threadfence();
         __syncwarp();
         unsigned arrived = 0;
-        if (lane == 0) arrived = atomicAdd(reinterpret_cast<unsigned*>(p.counters) + bg, 1u);
+        if (lane == 0) arrived = atomicAdd(p.counters + si.bg, 1u);
         arrived = __shfl_sync(FULL_MASK, arrived, 0);
-        if (arrived != (unsigned)(nseg - 1)) continue;
+        if (arrived != (unsigned)(si.nseg - 1)) continue;
+
         // Last unit of this (request, head group) to finish: merge all records.
         __threadfence();
 #pragma unroll
@@ -519,15 +642,17 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
             for (int j = 0; j < 2; ++j) {
                 const int h = nt * 8 + 2 * tig + j;
                 float M = -INFINITY;
-                for (long long uu = u_first; uu <= u_last; ++uu)
-                    M = fmaxf(M, ld_cg(p.rec_ml + (((size_t)bg + uu) * GP + h) * 2));
+#pragma unroll 4
+                for (long long uu = si.u_first; uu <= si.u_last; ++uu)
+                    M = fmaxf(M, ld_cg(p.rec_ml + ((si.bg + uu) * GP + h) * 2));
                 const float mref = M == -INFINITY ? 0.f : M;
                 float S = 0.f;
                 float A[C::KS][2];
 #pragma unroll
                 for (int dt = 0; dt < C::KS; ++dt) A[dt][0] = A[dt][1] = 0.f;
-                for (long long uu = u_first; uu <= u_last; ++uu) {
-                    const size_t rr = ((size_t)bg + uu) * GP + h;
+#pragma unroll 2
+                for (long long uu = si.u_first; uu <= si.u_last; ++uu) {
+                    const size_t rr = (si.bg + uu) * GP + h;
                     const float f = exp2f(ld_cg(p.rec_ml + rr * 2) - mref);
                     S = fmaf(ld_cg(p.rec_ml + rr * 2 + 1), f, S);
                     const float* ra = p.rec_acc + rr * D;
@@ -537,17 +662,48 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                         A[dt][1] = fmaf(ld_cg(ra + dt * 16 + grp + 8), f, A[dt][1]);
                     }
                 }
-                if (h >= gv) continue;
+                if (h >= si.gv) continue;
                 const float inv = S > 0.f ? 1.f / S : 0.f;
-                const size_t orow = ((size_t)cur.b * p.num_q_heads + hq0 + h) * D;
+                const size_t orow = ((size_t)si.b * p.num_q_heads + si.hq0 + h) * D;
 #pragma unroll
                 for (int dt = 0; dt < C::KS; ++dt) {
                     store_out(p.out, orow + dt * 16 + grp, A[dt][0] * inv, p.out_dtype);
                     store_out(p.out, orow + dt * 16 + grp + 8, A[dt][1] * inv, p.out_dtype);
                 }
             }
-        if (lane == 0) reinterpret_cast<unsigned*>(p.counters)[bg] = 0u;  // ready for the next call
+        // Return every workspace word this group used to zero, so the next call
+        // (whatever its sizes, hence its layout) starts from a zeroed workspace.
+        __syncwarp();
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int h = nt * 8 + 2 * tig + j;
+                for (long long uu = si.u_first; uu <= si.u_last; ++uu) {
+                    const size_t rr = (si.bg + uu) * GP + h;
+                    float* ra = p.rec_acc + rr * D;
+#pragma unroll
+                    for (int dt = 0; dt < C::KS; ++dt) {
+                        ra[dt * 16 + grp] = 0.f;
+                        ra[dt * 16 + grp + 8] = 0.f;
+                    }
+                    if (grp == 0) {
+                        p.rec_ml[rr * 2] = 0.f;
+                        p.rec_ml[rr * 2 + 1] = 0.f;
+                    }
+                }
+            }
+        if (lane == 0) p.counters[si.bg] = 0u;  // ready for the next call
     }
+}
+
+// Total chunk count, computed by one warp (same value in every warp and CTA).
+__device__ __forceinline__ long long total_chunks_warp(const DecodeParams& p, int lane, bool flag) {
+    long long t = 0;
+    for (int b = lane; b < p.num_seqs; b += 32) t += chunks_of<kCH>(clamp_len(p, b, flag));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(FULL_MASK, t, off);
+    return t * p.num_hg;
 }
 
 template <int D, int NT>
@@ -555,14 +711,16 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                                                              const __grid_constant__ CUtensorMap tmk,
                                                              const __grid_constant__ CUtensorMap tmv) {
     using C = MmaCfg<D, NT>;
+    using S = Smem<D, NT>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
     uint64_t* empty = full + C::NSTAGE;
-    int* st_ntok = reinterpret_cast<int*>(smem + C::OFF_META);
+    uint64_t* dfull = empty + C::NSTAGE;
+    uint64_t* dempty = dfull + S::NDUMP;
+    int* st_ntok = reinterpret_cast<int*>(smem + S::OFF_META);
     unsigned* st_bad = reinterpret_cast<unsigned*>(st_ntok + C::NSTAGE);
-    long long* scratch = reinterpret_cast<long long*>(smem + C::OFF_SCR);
-    volatile int* ctrl = reinterpret_cast<volatile int*>(smem + C::OFF_CTRL);
+    volatile int* ctrl = reinterpret_cast<volatile int*>(smem + S::OFF_CTRL);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
@@ -571,25 +729,30 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], 1);
         }
+        for (int s = 0; s < S::NDUMP; ++s) {
+            mbar_init(&dfull[s], 1);
+            mbar_init(&dempty[s], 1);
+        }
         fence_mbar_init();
         prefetch_tensormap(&tmk);
         prefetch_tensormap(&tmv);
     }
-    // Everything above overlaps the previous kernel in the stream; from here
-    // on we read memory it may have written.
-    griddep_wait();
+    __syncthreads();
     griddep_launch_dependents();
 
-    const long long total = total_chunks<kCH>(p, scratch, blockIdx.x == 0);
-    if (warp == 1) {
-        // empty requests: all-zero rows (softmax of an empty set)
-        for (int b = blockIdx.x; b < p.num_seqs; b += gridDim.x) {
-            if (clamp_len(p, b, false) != 0) continue;
-            for (int i = lane; i < p.num_q_heads * D; i += 32)
-                store_out(p.out, (size_t)b * p.num_q_heads * D + i, 0.f, p.out_dtype);
+    // Planning reads only seq_lens and the block tables, which the caller
+    // guarantees are not produced by the kernel right before this one; so it
+    // overlaps that kernel's tail.  Each role waits on the grid dependency
+    // before touching K/V, q, out or the workspace.
+    const long long total = total_chunks_warp(p, lane, blockIdx.x == 0 && warp == 0);
+    if (total == 0) {
+        if (warp == 2) {
+            SegIter<kCH> none;
+            none.valid = false;
+            epilogue<D, NT>(p, none, smem, dfull, dempty, ctrl, lane);
         }
+        return;
     }
-    if (total == 0) return;
     long long W = p.fixed_units > 0 ? p.fixed_units : (total + gridDim.x - 1) / gridDim.x;
     if (W < 1) W = 1;
     SegIter<kCH> it;
@@ -599,8 +762,11 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
         Producer<D, NT> pr{p, &tmk, &tmv, smem, full, empty, st_ntok, st_bad, ctrl, lane,
                            l2_policy_evict_first()};
         pr.run(it);
+        if (!pr.waited) griddep_wait();
+    } else if (warp == 1) {
+        consume<D, NT>(p, it, smem, full, empty, dfull, dempty, st_ntok, st_bad, ctrl, lane);
     } else {
-        consume<D, NT>(p, it, smem, full, empty, st_ntok, st_bad, ctrl, lane);
+        epilogue<D, NT>(p, it, smem, dfull, dempty, ctrl, lane);
     }
 }
 
@@ -639,7 +805,7 @@ bool encode_cache_map(CUtensorMap* map, const void* base, long long rows, int he
 
 template <int D, int NT>
 pkv_status launch_impl(const DecodeParams& p, cudaStream_t stream, int* grid_out) {
-    using C = MmaCfg<D, NT>;
+    using S = Smem<D, NT>;
     const DeviceInfo* di = current_device_info();
     if (!di) return PKV_ERR_CUDA;
     static std::mutex mu;
@@ -649,12 +815,12 @@ pkv_status launch_impl(const DecodeParams& p, cudaStream_t stream, int* grid_out
         std::lock_guard<std::mutex> lock(mu);
         if (di->device >= 64) return PKV_ERR_UNSUPPORTED;
         if (occupancy[di->device] == 0) {
-            if (C::SMEM > di->max_smem_optin) return PKV_ERR_UNSUPPORTED;
-            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM) !=
+            if (S::BYTES > di->max_smem_optin) return PKV_ERR_UNSUPPORTED;
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::BYTES) !=
                 cudaSuccess)
                 return PKV_ERR_CUDA;
             int occ = 0;
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, C::SMEM) !=
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, S::BYTES) !=
                     cudaSuccess ||
                 occ < 1)
                 return PKV_ERR_CUDA;
@@ -669,7 +835,7 @@ pkv_status launch_impl(const DecodeParams& p, cudaStream_t stream, int* grid_out
         return PKV_ERR_CUDA;
     const int grid = di->num_sms * std::min(occupancy[di->device], 4);
 
-    PdlLaunch L(dim3(grid), dim3(kThreads), C::SMEM, stream);
+    PdlLaunch L(dim3(grid), dim3(kThreads), S::BYTES, stream);
     if (cudaLaunchKernelEx(&L.cfg, kern, p, tmk, tmv) != cudaSuccess) return PKV_ERR_CUDA;
     if (grid_out) *grid_out = grid;
     return PKV_OK;

@@ -495,24 +495,43 @@ __global__ void decode_merge_kernel(const __grid_constant__ DecodeParams p, int 
     }
     const int u0 = p.meta[2 * (size_t)bg];
     const int nseg = p.meta[2 * (size_t)bg + 1];
-    if (nseg <= 1) return;
-    for (int idx = threadIdx.x; idx < gv * D; idx += blockDim.x) {
-        const int h = idx / D, k = idx % D;
-        float M = -INFINITY;
-        for (int r = 0; r < nseg; ++r) {
-            const size_t rec = (size_t)bg + u0 + r;
-            M = fmaxf(M, p.rec_ml[(rec * GP + h) * 2]);
+    if (nseg > 1) {
+        for (int idx = threadIdx.x; idx < gv * D; idx += blockDim.x) {
+            const int h = idx / D, k = idx % D;
+            float M = -INFINITY;
+            for (int r = 0; r < nseg; ++r) {
+                const size_t rec = (size_t)bg + u0 + r;
+                M = fmaxf(M, p.rec_ml[(rec * GP + h) * 2]);
+            }
+            const float mref = M == -INFINITY ? 0.f : M;
+            float S = 0.f, A = 0.f;
+            for (int r = 0; r < nseg; ++r) {
+                const size_t rec = (size_t)bg + u0 + r;
+                const float f = exp2f(p.rec_ml[(rec * GP + h) * 2] - mref);
+                S = fmaf(p.rec_ml[(rec * GP + h) * 2 + 1], f, S);
+                A = fmaf(p.rec_acc[(rec * GP + h) * D + k], f, A);
+            }
+            store_out(p.out, ((size_t)b * p.num_q_heads + hq0 + h) * D + k, S > 0.f ? A / S : 0.f,
+                      p.out_dtype);
         }
-        const float mref = M == -INFINITY ? 0.f : M;
-        float S = 0.f, A = 0.f;
-        for (int r = 0; r < nseg; ++r) {
-            const size_t rec = (size_t)bg + u0 + r;
-            const float f = exp2f(p.rec_ml[(rec * GP + h) * 2] - mref);
-            S = fmaf(p.rec_ml[(rec * GP + h) * 2 + 1], f, S);
-            A = fmaf(p.rec_acc[(rec * GP + h) * D + k], f, A);
+        // Return the records and the group's meta words to zero, so the next
+        // call (whatever its sizes, hence its layout) starts from a zeroed workspace.
+        __syncthreads();
+        for (int idx = threadIdx.x; idx < gv * D; idx += blockDim.x) {
+            const int h = idx / D, k = idx % D;
+            for (int r = 0; r < nseg; ++r) {
+                const size_t rec = (size_t)bg + u0 + r;
+                p.rec_acc[(rec * GP + h) * D + k] = 0.f;
+                if (k == 0) {
+                    p.rec_ml[(rec * GP + h) * 2] = 0.f;
+                    p.rec_ml[(rec * GP + h) * 2 + 1] = 0.f;
+                }
+            }
         }
-        store_out(p.out, ((size_t)b * p.num_q_heads + hq0 + h) * D + k, S > 0.f ? A / S : 0.f,
-                  p.out_dtype);
+    }
+    if (threadIdx.x == 0) {
+        p.meta[2 * (size_t)bg] = 0;
+        p.meta[2 * (size_t)bg + 1] = 0;
     }
 }
 
