@@ -178,6 +178,44 @@ pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache,
                                       pkv_stream_t stream);
 
 /*
+ * pkv_paged_attention_decode_noalloc -- pkv_paged_attention_decode for callers
+ * that cannot allocate device memory.
+ *
+ * The pages have no counterpart of this call; it exists for integration.  A
+ * serving engine that reserves nearly all device memory for its KV pool up
+ * front may not let an extension allocate, and on a latency-critical path the
+ * device-wide synchronisation of cudaMalloc may not be acceptable.  This
+ * variant takes the same arguments minus the workspace and runs the same
+ * decode with its scratch in a fixed array inside the library's device image
+ * (pkv_decode_noalloc_scratch_bytes() bytes, held by every device that loads
+ * the library until the process exits).  It allocates nothing.
+ *   - Sizes whose scratch (pkv_decode_workspace_bytes) exceeds that maximum are
+ *     refused with PKV_ERR_WORKSPACE; nothing is launched.
+ *   - The first call on a device finds the array's device address (with that
+ *     device current) and zeroes it on `stream`; make that first call before
+ *     any stream capture.
+ *   - Each call clears, on `stream`, the part of the array that must start at
+ *     zero; the rest keeps the previous call's contents.
+ *   - All calls on a device share the array: calls that overlap on the GPU
+ *     (other streams, other host threads) race.  Order them.
+ */
+pkv_status pkv_paged_attention_decode_noalloc(const void* q, const void* k_cache,
+                                              const void* v_cache,
+                                              const int32_t* block_tables,
+                                              const int32_t* seq_lens, int32_t block_size,
+                                              float scale, void* out, int32_t num_seqs,
+                                              int32_t num_q_heads, int32_t num_kv_heads,
+                                              int32_t head_dim, int32_t max_blocks_per_seq,
+                                              int32_t num_blocks, int32_t max_seq_len,
+                                              pkv_dtype q_dtype, pkv_dtype kv_dtype,
+                                              pkv_dtype out_dtype, const float* k_scale,
+                                              const float* v_scale, int32_t partition_size,
+                                              pkv_stream_t stream);
+
+/* Size in bytes of the fixed scratch array pkv_paged_attention_decode_noalloc uses. */
+size_t pkv_decode_noalloc_scratch_bytes(void);
+
+/*
  * pkv_copy_blocks -- copy whole physical blocks (copy-on-write fork).
  *
  * [KVOPT] intro and [KVMGMT] "The Bonus: Zero-Copy Sharing": requests with a

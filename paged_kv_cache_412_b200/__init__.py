@@ -232,6 +232,58 @@ def paged_attention_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torc
     return out
 
 
+_noalloc_declared = False
+
+
+def paged_attention_decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                                   block_tables: torch.Tensor, seq_lens: torch.Tensor,
+                                   block_size: int | None = None, scale: float | None = None,
+                                   out: torch.Tensor | None = None, *,
+                                   max_seq_len: int | None = None, partition_size: int = 0,
+                                   out_dtype: torch.dtype | None = None) -> torch.Tensor:
+    """The same decode through ``pkv_paged_attention_decode_noalloc``: no
+    workspace argument, the library's fixed device scratch array is used.
+
+    For callers that may not allocate device memory (see the C header).  Calls
+    on one device share that array and must not overlap on the GPU.
+    """
+    global _noalloc_declared
+    L = _get_lib()
+    if not _noalloc_declared:
+        vp, i32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+        L.pkv_paged_attention_decode_noalloc.argtypes = [
+            vp, vp, vp, vp, vp, i32, ctypes.c_float, vp, i32, i32, i32, i32, i32, i32, i32,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, i32, vp]
+        L.pkv_paged_attention_decode_noalloc.restype = ctypes.c_int
+        L.pkv_decode_noalloc_scratch_bytes.argtypes = []
+        L.pkv_decode_noalloc_scratch_bytes.restype = sz
+        _noalloc_declared = True
+    dev = _need_cuda(q, k_cache, v_cache, block_tables, seq_lens, out)
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise TypeError("block_tables and seq_lens must be int32")
+    B, Hq, d = q.shape
+    NB, Hkv, bs, d2 = k_cache.shape
+    if block_size is None:
+        block_size = bs
+    if block_size != bs or d2 != d or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    if scale is None:
+        scale = d ** -0.5
+    max_blocks = block_tables.shape[1]
+    if max_seq_len is None:
+        max_seq_len = max_blocks * bs
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=out_dtype or q.dtype, device=dev)
+    with torch.cuda.device(dev):
+        st = L.pkv_paged_attention_decode_noalloc(
+            _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(seq_lens), bs,
+            float(scale), _ptr(out), B, Hq, Hkv, d, max_blocks, NB, int(max_seq_len),
+            _dtype_code(q), _dtype_code(k_cache), _dtype_code(out), None, None,
+            int(partition_size), _stream(dev))
+    _check("pkv_paged_attention_decode_noalloc", st)
+    return out
+
+
 def copy_blocks(k_cache: torch.Tensor, v_cache: torch.Tensor, block_mapping: torch.Tensor) -> None:
     """block_mapping [n, 2] int64 (src, dst): cache[dst] = cache[src] for K and V."""
     dev = _need_cuda(k_cache, v_cache, block_mapping)
