@@ -55,7 +55,8 @@ typedef enum pkv_status {
     PKV_ERR_UNSUPPORTED = 2,   /* valid but not implemented (dtype, head_dim...) */
     PKV_ERR_WORKSPACE = 3,     /* workspace null or smaller than required        */
     PKV_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed           */
-    PKV_ERR_DEVICE_INDEX = 5   /* pkv_get_device_error found a device-side flag  */
+    PKV_ERR_DEVICE_INDEX = 5,  /* pkv_get_device_error found a device-side flag  */
+    PKV_ERR_OUT_OF_BLOCKS = 6  /* block allocator: not enough free blocks        */
 } pkv_status;
 
 typedef enum pkv_dtype {
@@ -241,6 +242,85 @@ pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_ma
  * is shared by every stream of the device.
  */
 pkv_status pkv_get_device_error(pkv_stream_t stream, uint32_t* flags /* host */);
+
+/* ==========================================================================
+ * Host-side block manager (no GPU work; all pointers below are HOST pointers)
+ *
+ * "KV Cache Optimization and PagedAttention" (intro), "PagedAttention:
+ * Optimizing KV Cache Utilization in Large Language Models" ("The Mechanics of
+ * PagedAttention") and "KV Cache Management" ("The Solution: PagedAttention
+ * (vLLM)", "The Bonus: Zero-Copy Sharing"): physical blocks are handed out on
+ * demand as a request's tokens arrive; a per-request block table maps logical
+ * to physical blocks; requests with a common prefix share physical blocks, each
+ * carrying a reference count, and a request that must write into a shared,
+ * partially filled block first gets a private copy (copy-on-write).
+ * Not thread-safe: one allocator per host thread, or external locking.
+ * ========================================================================== */
+
+typedef struct pkv_allocator pkv_allocator;
+
+typedef struct pkv_allocator_stats {
+    int32_t num_blocks;      /* pool size                                   */
+    int32_t free_blocks;     /* on the free list                            */
+    int32_t used_blocks;     /* referenced by at least one sequence         */
+    int32_t shared_blocks;   /* referenced by more than one sequence        */
+    int32_t num_seqs;
+    int64_t stored_tokens;   /* valid slots in used blocks (shared counted once) */
+    int64_t logical_tokens;  /* sum of the sequences' lengths               */
+    int64_t unused_slots;    /* empty slots in used blocks (internal waste)  */
+} pkv_allocator_stats;
+
+/* Pool of num_blocks blocks of block_size slots (power of two <= 256). */
+pkv_status pkv_allocator_create(int32_t num_blocks, int32_t block_size, pkv_allocator** out);
+void pkv_allocator_destroy(pkv_allocator* allocator);
+
+/* Register an empty sequence (seq_id must be new). */
+pkv_status pkv_allocator_add_seq(pkv_allocator* allocator, int64_t seq_id);
+
+/* New sequence `child` sharing every block of `parent` (reference counts + 1). */
+pkv_status pkv_allocator_fork(pkv_allocator* allocator, int64_t parent, int64_t child);
+
+/*
+ * Append num_tokens tokens to seq_id.  Writes their slot ids to slots[0..n)
+ * (for pkv_kv_cache_write).  If the sequence's last block is shared and only
+ * partially filled, it is first replaced by a private copy: *num_cow = 1 and
+ * cow_pair = {src, dst} (run pkv_copy_blocks on it before writing); else
+ * *num_cow = 0.  PKV_ERR_OUT_OF_BLOCKS (nothing changed) if the pool cannot
+ * supply the blocks needed.
+ */
+pkv_status pkv_allocator_append(pkv_allocator* allocator, int64_t seq_id, int32_t num_tokens,
+                                int64_t* slots, int64_t* cow_pair, int32_t* num_cow);
+
+/* Drop a sequence; blocks whose reference count reaches 0 return to the pool. */
+pkv_status pkv_allocator_free_seq(pkv_allocator* allocator, int64_t seq_id);
+
+/* Copy the sequence's block table into table[0..capacity); report its size. */
+pkv_status pkv_allocator_block_table(const pkv_allocator* allocator, int64_t seq_id,
+                                     int32_t* table, int32_t capacity, int32_t* num_blocks,
+                                     int64_t* num_tokens);
+
+pkv_status pkv_allocator_get_stats(const pkv_allocator* allocator, pkv_allocator_stats* out);
+
+/* Reference count of a physical block (-1 for an invalid id). */
+int32_t pkv_allocator_refcount(const pkv_allocator* allocator, int32_t block);
+
+/*
+ * Waste of the two reservation schemes the pages contrast ("KV Cache
+ * Optimization and PagedAttention", intro and its waste example): a
+ * contiguous region of reserve_len slots per request versus whole blocks of
+ * block_size slots.  Also how many of the requests, taken in order, fit at
+ * once in a pool of pool_slots slots under each scheme.
+ */
+typedef struct pkv_waste_report {
+    int64_t used_slots;           /* sum of the lengths                       */
+    int64_t contiguous_reserved;  /* n * reserve_len                          */
+    int64_t paged_reserved;       /* sum of ceil(L / block_size) * block_size */
+    int32_t contiguous_admitted;
+    int32_t paged_admitted;
+} pkv_waste_report;
+
+pkv_status pkv_waste_compare(const int32_t* lengths, int32_t n, int32_t reserve_len,
+                             int32_t block_size, int64_t pool_slots, pkv_waste_report* out);
 
 #ifdef __cplusplus
 }

@@ -28,6 +28,7 @@ import torch
 __all__ = [
     "PkvError", "LIB_PATH", "lib", "kv_cache_write", "paged_attention_decode", "copy_blocks",
     "decode_workspace_bytes", "new_workspace", "get_device_error", "status_string", "DEVERR",
+    "paged_attention_decode_noalloc", "BlockAllocator", "waste_compare",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpkv.so")
@@ -308,3 +309,125 @@ def get_device_error(device: torch.device | int | None = None) -> int:
     if st not in (PKV_OK, 5):
         raise PkvError("pkv_get_device_error", st)
     return int(flags.value)
+
+
+# ---------------------------------------------------------------------------
+# host-side block manager (C++ in libpkv.so; no GPU work)
+# ---------------------------------------------------------------------------
+
+class _AllocStats(ctypes.Structure):
+    _fields_ = [("num_blocks", ctypes.c_int32), ("free_blocks", ctypes.c_int32),
+                ("used_blocks", ctypes.c_int32), ("shared_blocks", ctypes.c_int32),
+                ("num_seqs", ctypes.c_int32), ("stored_tokens", ctypes.c_int64),
+                ("logical_tokens", ctypes.c_int64), ("unused_slots", ctypes.c_int64)]
+
+
+class _WasteReport(ctypes.Structure):
+    _fields_ = [("used_slots", ctypes.c_int64), ("contiguous_reserved", ctypes.c_int64),
+                ("paged_reserved", ctypes.c_int64), ("contiguous_admitted", ctypes.c_int32),
+                ("paged_admitted", ctypes.c_int32)]
+
+
+_alloc_declared = False
+
+
+def _alloc_lib():
+    global _alloc_declared
+    L = _get_lib()
+    if not _alloc_declared:
+        vp, i32, i64 = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64
+        P = ctypes.POINTER
+        L.pkv_allocator_create.argtypes = [i32, i32, P(vp)]
+        L.pkv_allocator_destroy.argtypes = [vp]
+        L.pkv_allocator_destroy.restype = None
+        L.pkv_allocator_add_seq.argtypes = [vp, i64]
+        L.pkv_allocator_fork.argtypes = [vp, i64, i64]
+        L.pkv_allocator_append.argtypes = [vp, i64, i32, P(i64), P(i64), P(i32)]
+        L.pkv_allocator_free_seq.argtypes = [vp, i64]
+        L.pkv_allocator_block_table.argtypes = [vp, i64, P(i32), i32, P(i32), P(i64)]
+        L.pkv_allocator_get_stats.argtypes = [vp, P(_AllocStats)]
+        L.pkv_allocator_refcount.argtypes = [vp, i32]
+        L.pkv_allocator_refcount.restype = i32
+        L.pkv_waste_compare.argtypes = [P(i32), i32, i32, i32, i64, P(_WasteReport)]
+        for f in ("pkv_allocator_create", "pkv_allocator_add_seq", "pkv_allocator_fork",
+                  "pkv_allocator_append", "pkv_allocator_free_seq", "pkv_allocator_block_table",
+                  "pkv_allocator_get_stats", "pkv_waste_compare"):
+            getattr(L, f).restype = ctypes.c_int
+        _alloc_declared = True
+    return L
+
+
+class BlockAllocator:
+    """Physical-block pool with per-sequence block tables, reference-counted
+    sharing (fork) and copy-on-write on append.  Host memory only."""
+
+    def __init__(self, num_blocks: int, block_size: int):
+        import numpy as np  # noqa: F401  (numpy arrays are returned)
+        self._L = _alloc_lib()
+        h = ctypes.c_void_p()
+        _check("pkv_allocator_create", self._L.pkv_allocator_create(num_blocks, block_size,
+                                                                    ctypes.byref(h)))
+        self._h = h
+        self.num_blocks, self.block_size = num_blocks, block_size
+
+    def close(self) -> None:
+        if getattr(self, "_h", None):
+            self._L.pkv_allocator_destroy(self._h)
+            self._h = None
+
+    __del__ = close
+
+    def add_seq(self, seq_id: int) -> None:
+        _check("pkv_allocator_add_seq", self._L.pkv_allocator_add_seq(self._h, seq_id))
+
+    def fork(self, parent: int, child: int) -> None:
+        _check("pkv_allocator_fork", self._L.pkv_allocator_fork(self._h, parent, child))
+
+    def append(self, seq_id: int, num_tokens: int):
+        """Returns (slots int64[num_tokens], copy-on-write pair (src, dst) or None)."""
+        import numpy as np
+        slots = np.zeros(max(num_tokens, 1), dtype=np.int64)
+        pair = (ctypes.c_int64 * 2)()
+        ncow = ctypes.c_int32(0)
+        st = self._L.pkv_allocator_append(self._h, seq_id, num_tokens,
+                                          slots.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                                          pair, ctypes.byref(ncow))
+        _check("pkv_allocator_append", st)
+        return slots[:num_tokens], ((int(pair[0]), int(pair[1])) if ncow.value else None)
+
+    def free_seq(self, seq_id: int) -> None:
+        _check("pkv_allocator_free_seq", self._L.pkv_allocator_free_seq(self._h, seq_id))
+
+    def block_table(self, seq_id: int):
+        """Returns (int32 block ids, number of tokens)."""
+        import numpy as np
+        nb, nt = ctypes.c_int32(0), ctypes.c_int64(0)
+        self._L.pkv_allocator_block_table(self._h, seq_id, None, 0, ctypes.byref(nb),
+                                          ctypes.byref(nt))
+        table = np.zeros(max(nb.value, 1), dtype=np.int32)
+        _check("pkv_allocator_block_table", self._L.pkv_allocator_block_table(
+            self._h, seq_id, table.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), table.size,
+            ctypes.byref(nb), ctypes.byref(nt)))
+        return table[:nb.value], int(nt.value)
+
+    def stats(self) -> dict:
+        s = _AllocStats()
+        _check("pkv_allocator_get_stats", self._L.pkv_allocator_get_stats(self._h,
+                                                                          ctypes.byref(s)))
+        return {k: getattr(s, k) for k, _ in _AllocStats._fields_}
+
+    def refcount(self, block: int) -> int:
+        return int(self._L.pkv_allocator_refcount(self._h, block))
+
+
+def waste_compare(lengths, reserve_len: int, block_size: int, pool_slots: int) -> dict:
+    """Contiguous (reserve_len per request) vs paged (whole blocks) reservation:
+    slots used/reserved and how many requests fit at once in pool_slots."""
+    import numpy as np
+    L = _alloc_lib()
+    arr = np.ascontiguousarray(lengths, dtype=np.int32)
+    r = _WasteReport()
+    _check("pkv_waste_compare", L.pkv_waste_compare(
+        arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), arr.size, reserve_len, block_size,
+        pool_slots, ctypes.byref(r)))
+    return {k: getattr(r, k) for k, _ in _WasteReport._fields_}

@@ -43,13 +43,13 @@ def build(verbose: bool = False, ptxas_info: bool = False, force: bool = False,
           jobs: int = 8) -> str:
     nvcc = _nvcc()
     os.makedirs(BUILD, exist_ok=True)
-    sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    sources = sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
     headers = sorted(glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) +
                      glob.glob(os.path.join(ROOT, "include", "*.h")))
     extra = ["-Xptxas", "-v"] if ptxas_info else []
 
     def compile_one(src: str) -> str:
-        obj = os.path.join(BUILD, os.path.basename(src)[:-3] + ".o")
+        obj = os.path.join(BUILD, os.path.splitext(os.path.basename(src))[0] + ".o")
         if force or ptxas_info or _stale(obj, [src] + headers):
             cmd = [nvcc, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
             if verbose:

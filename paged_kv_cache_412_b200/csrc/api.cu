@@ -99,11 +99,15 @@ bool make_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_
     const size_t acc_bytes = pl.records * pl.rec_gp * head_dim * sizeof(float);
     const size_t ml_bytes = pl.records * pl.rec_gp * 2 * sizeof(float);
     const size_t meta_bytes = pl.n_bg_max * 2 * sizeof(int32_t);
-    const size_t cnt_bytes = pl.n_bg_max * sizeof(uint32_t);
     pl.off_ml = up(acc_bytes);
     pl.off_meta = pl.off_ml + up(ml_bytes);
-    pl.off_cnt = pl.off_meta + up(meta_bytes);
-    pl.bytes = pl.off_cnt + up(cnt_bytes);
+    pl.rec_bytes = pl.off_meta + up(meta_bytes);
+    // smallest B with counter region(B) + records <= B and room for every counter
+    size_t b = up(pl.rec_bytes + pl.n_bg_max * sizeof(uint32_t));
+    while (counter_region_bytes(b) + pl.rec_bytes > b ||
+           counter_region_bytes(b) < pl.n_bg_max * sizeof(uint32_t))
+        b += 256;
+    pl.bytes = b;
     *plan = pl;
     return true;
 }
@@ -122,6 +126,7 @@ const char* pkv_status_string(pkv_status status) {
         case PKV_ERR_WORKSPACE: return "PKV_ERR_WORKSPACE: workspace missing or too small";
         case PKV_ERR_CUDA: return "PKV_ERR_CUDA: CUDA runtime or launch failure";
         case PKV_ERR_DEVICE_INDEX: return "PKV_ERR_DEVICE_INDEX: device reported a bad index";
+        case PKV_ERR_OUT_OF_BLOCKS: return "PKV_ERR_OUT_OF_BLOCKS: not enough free blocks";
         default: return "PKV_ERR_UNKNOWN";
     }
 }
@@ -230,10 +235,14 @@ pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const 
     p.out = out;
     p.k_scale = k_scale;
     p.v_scale = v_scale;
-    p.rec_acc = reinterpret_cast<float*>(ws);
-    p.rec_ml = reinterpret_cast<float*>(ws + pl.off_ml);
-    p.meta = reinterpret_cast<int32_t*>(ws + pl.off_meta);
-    p.counters = reinterpret_cast<unsigned*>(ws + pl.off_cnt);
+    const size_t cnt_region = counter_region_bytes(workspace_bytes);
+    if (cnt_region + pl.rec_bytes > workspace_bytes ||
+        cnt_region < pl.n_bg_max * sizeof(uint32_t))
+        return PKV_ERR_WORKSPACE;
+    p.counters = reinterpret_cast<unsigned*>(ws);
+    p.rec_acc = reinterpret_cast<float*>(ws + cnt_region);
+    p.rec_ml = reinterpret_cast<float*>(ws + cnt_region + pl.off_ml);
+    p.meta = reinterpret_cast<int32_t*>(ws + cnt_region + pl.off_meta);
     p.err = di->error_word;
     p.num_seqs = num_seqs;
     p.num_q_heads = num_q_heads;

@@ -634,24 +634,30 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
         arrived = __shfl_sync(FULL_MASK, arrived, 0);
         if (arrived != (unsigned)(si.nseg - 1)) continue;
 
-        // Last unit of this (request, head group) to finish: merge all records.
+        // Last unit of this (request, head group) to finish: merge all records
+        // (its own from registers, the others from L2).
         __threadfence();
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 const int h = nt * 8 + 2 * tig + j;
-                float M = -INFINITY;
+                float M = m[nt][j];
 #pragma unroll 4
                 for (long long uu = si.u_first; uu <= si.u_last; ++uu)
-                    M = fmaxf(M, ld_cg(p.rec_ml + ((si.bg + uu) * GP + h) * 2));
+                    if (uu != si.u) M = fmaxf(M, ld_cg(p.rec_ml + ((si.bg + uu) * GP + h) * 2));
                 const float mref = M == -INFINITY ? 0.f : M;
-                float S = 0.f;
+                const float fo = exp2f(m[nt][j] - mref);
+                float S = l[nt][j] * fo;
                 float A[C::KS][2];
 #pragma unroll
-                for (int dt = 0; dt < C::KS; ++dt) A[dt][0] = A[dt][1] = 0.f;
+                for (int dt = 0; dt < C::KS; ++dt) {
+                    A[dt][0] = acc[dt][nt][j] * fo;
+                    A[dt][1] = acc[dt][nt][j + 2] * fo;
+                }
 #pragma unroll 2
                 for (long long uu = si.u_first; uu <= si.u_last; ++uu) {
+                    if (uu == si.u) continue;
                     const size_t rr = (si.bg + uu) * GP + h;
                     const float f = exp2f(ld_cg(p.rec_ml + rr * 2) - mref);
                     S = fmaf(ld_cg(p.rec_ml + rr * 2 + 1), f, S);
@@ -669,28 +675,6 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
                 for (int dt = 0; dt < C::KS; ++dt) {
                     store_out(p.out, orow + dt * 16 + grp, A[dt][0] * inv, p.out_dtype);
                     store_out(p.out, orow + dt * 16 + grp + 8, A[dt][1] * inv, p.out_dtype);
-                }
-            }
-        // Return every workspace word this group used to zero, so the next call
-        // (whatever its sizes, hence its layout) starts from a zeroed workspace.
-        __syncwarp();
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int h = nt * 8 + 2 * tig + j;
-                for (long long uu = si.u_first; uu <= si.u_last; ++uu) {
-                    const size_t rr = (si.bg + uu) * GP + h;
-                    float* ra = p.rec_acc + rr * D;
-#pragma unroll
-                    for (int dt = 0; dt < C::KS; ++dt) {
-                        ra[dt * 16 + grp] = 0.f;
-                        ra[dt * 16 + grp + 8] = 0.f;
-                    }
-                    if (grp == 0) {
-                        p.rec_ml[rr * 2] = 0.f;
-                        p.rec_ml[rr * 2 + 1] = 0.f;
-                    }
                 }
             }
         if (lane == 0) p.counters[si.bg] = 0u;  // ready for the next call

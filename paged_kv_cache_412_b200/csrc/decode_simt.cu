@@ -514,24 +514,6 @@ __global__ void decode_merge_kernel(const __grid_constant__ DecodeParams p, int 
             store_out(p.out, ((size_t)b * p.num_q_heads + hq0 + h) * D + k, S > 0.f ? A / S : 0.f,
                       p.out_dtype);
         }
-        // Return the records and the group's meta words to zero, so the next
-        // call (whatever its sizes, hence its layout) starts from a zeroed workspace.
-        __syncthreads();
-        for (int idx = threadIdx.x; idx < gv * D; idx += blockDim.x) {
-            const int h = idx / D, k = idx % D;
-            for (int r = 0; r < nseg; ++r) {
-                const size_t rec = (size_t)bg + u0 + r;
-                p.rec_acc[(rec * GP + h) * D + k] = 0.f;
-                if (k == 0) {
-                    p.rec_ml[(rec * GP + h) * 2] = 0.f;
-                    p.rec_ml[(rec * GP + h) * 2 + 1] = 0.f;
-                }
-            }
-        }
-    }
-    if (threadIdx.x == 0) {
-        p.meta[2 * (size_t)bg] = 0;
-        p.meta[2 * (size_t)bg + 1] = 0;
     }
 }
 

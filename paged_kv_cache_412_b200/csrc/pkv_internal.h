@@ -24,14 +24,26 @@ const DeviceInfo* current_device_info();
 // Workspace bound of one decode call.  It covers both decode kernels (the
 // tensor-core one groups up to 16 query heads per kv-head pass, the CUDA-core
 // one up to 8), so one size fits whichever path the call takes.
+//
+// Layout of a workspace of B bytes: arrival counters first, in a region whose
+// size depends only on B (counter_region_bytes(B)), then the partial records.
+// A given buffer therefore always keeps its counters in the same words, which
+// every call returns to zero; records are always written before they are read
+// in the same call and need no clearing, whatever the sizes of the next call.
 struct DecodePlan {
     int rec_gp;        // floats per record row = largest query-head group of either path
     size_t n_bg_max;   // (request, head group) pairs, largest over the paths
     size_t units_max;  // upper bound of split units
     size_t records;    // partial-result records
-    size_t off_ml, off_meta, off_cnt;  // byte offsets of the workspace regions
-    size_t bytes;      // workspace bytes
+    size_t rec_bytes;  // records + their (max, sum) pairs + per-group meta
+    size_t off_ml, off_meta;  // offsets inside the record region
+    size_t bytes;      // smallest workspace that fits
 };
+
+// Bytes at the start of a B-byte workspace reserved for arrival counters.
+inline size_t counter_region_bytes(size_t workspace_bytes) {
+    return (workspace_bytes / 128 + 255) / 256 * 256;
+}
 
 // Fill a plan for these sizes on the current device (false if invalid).
 bool make_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
