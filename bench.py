@@ -142,6 +142,12 @@ class ClockSampler:
 # distributed plumbing (only for --gpus > 1 under torchrun)
 # ---------------------------------------------------------------------------
 
+def replica_seed(rank: int, layer: int) -> int:
+    """Seed of a rank's replica of one layer pool: every rank decodes its own
+    independent batch (weak scaling, no data exchanged between ranks)."""
+    return 1002 + 100 * rank + layer
+
+
 def dist_setup(n_gpus: int):
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -297,7 +303,7 @@ def run_ours(args, rank: int, world: int, local: int):
     # --- inputs resident in HBM: N_LAYERS layer pools of the same workload ---
     layers = []
     for li in range(N_LAYERS):
-        w = workloads.gqa_4k(poison=False, seed=1002 + 100 * rank + li)
+        w = workloads.gqa_4k(poison=False, seed=replica_seed(rank, li))
         t = {}
         t["q"] = torch.from_numpy(w.q.view(np.int16)).to(dev).view(torch.bfloat16)
         t["kc"] = torch.from_numpy(w.k_cache.view(np.int16)).to(dev).view(torch.bfloat16)

@@ -100,6 +100,25 @@ pkv_status pkv_kv_cache_write(const void* k, const void* v, const int64_t* slot_
                               int32_t num_blocks, pkv_dtype dtype, pkv_stream_t stream);
 
 /*
+ * pkv_kv_cache_write_fp8 -- append new tokens to an fp8 (e4m3) cache.
+ *
+ * "KV Cache Management", "Watch Out For" and "What to Read Next": long
+ * contexts call for quantising the KV cache to 8 bits.  Each value is stored
+ * as the e4m3 code of x / scale[h] (one fp32 scale per kv head, the quotient
+ * rounded as an IEEE fp32 division, then rounded to nearest even and saturated
+ * at +-448), and read back as code * scale[h].
+ *   k, v          [num_tokens, num_kv_heads, head_dim] bf16.
+ *   k_cache, v_cache  [num_blocks, num_kv_heads, block_size, head_dim] uint8 codes.
+ *   k_scale, v_scale  [num_kv_heads] fp32 (device).
+ * Slots as in pkv_kv_cache_write.
+ */
+pkv_status pkv_kv_cache_write_fp8(const void* k, const void* v, const int64_t* slot_mapping,
+                                  void* k_cache, void* v_cache, const float* k_scale,
+                                  const float* v_scale, int32_t num_tokens, int32_t num_kv_heads,
+                                  int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                                  pkv_stream_t stream);
+
+/*
  * pkv_decode_workspace_bytes -- bytes of device scratch that
  * pkv_paged_attention_decode needs for these sizes on the CURRENT device.
  * max_seq_len bounds every seq_lens entry of the calls that will use it;
@@ -233,6 +252,30 @@ size_t pkv_decode_noalloc_scratch_bytes(void);
 pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping,
                            int32_t num_pairs, int32_t num_kv_heads, int32_t head_dim,
                            int32_t block_size, int32_t num_blocks, pkv_dtype dtype,
+                           pkv_stream_t stream);
+
+/*
+ * pkv_swap_blocks -- copy whole blocks between two pools, e.g. the device cache
+ * and a host pool, for preemption.
+ *
+ * "PagedAttention: Optimizing KV Cache Utilization in Large Language Models",
+ * "Conclusion": when generation runs out of physical blocks, requests are
+ * preempted and their KV cache recomputed or swapped out, then swapped back in.
+ * For every pair: dst_k_cache[dst] = src_k_cache[src] (same for V), all kv
+ * heads and slots, bit-exact.  Pools have the cache layout above with
+ * src_num_blocks / dst_num_blocks blocks.
+ *
+ *   All five pointers must be reachable from the current device: device
+ *   memory, or pinned host memory mapped into its address space (cudaHostAlloc /
+ *   torch pin_memory).  Anything else (pageable host memory, another device's
+ *   memory) is refused with PKV_ERR_INVALID_ARG before any launch.
+ *   block_mapping [num_pairs, 2] int64 (src, dst); out-of-range ids: pair
+ *   skipped, PKV_DEVERR_BAD_PAIR.  dst ids distinct.
+ */
+pkv_status pkv_swap_blocks(const void* src_k_cache, const void* src_v_cache, void* dst_k_cache,
+                           void* dst_v_cache, const int64_t* block_mapping, int32_t num_pairs,
+                           int32_t src_num_blocks, int32_t dst_num_blocks, int32_t num_kv_heads,
+                           int32_t head_dim, int32_t block_size, pkv_dtype dtype,
                            pkv_stream_t stream);
 
 /*

@@ -28,7 +28,8 @@ import torch
 __all__ = [
     "PkvError", "LIB_PATH", "lib", "kv_cache_write", "paged_attention_decode", "copy_blocks",
     "decode_workspace_bytes", "new_workspace", "get_device_error", "status_string", "DEVERR",
-    "paged_attention_decode_noalloc", "BlockAllocator", "waste_compare",
+    "paged_attention_decode_noalloc", "BlockAllocator", "waste_compare", "swap_blocks",
+    "kv_cache_write_fp8",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpkv.so")
@@ -231,6 +232,81 @@ def paged_attention_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torc
             _stream(dev))
     _check("pkv_paged_attention_decode", st)
     return out
+
+
+_fp8w_declared = False
+
+
+def kv_cache_write_fp8(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor,
+                       k_cache: torch.Tensor, v_cache: torch.Tensor, k_scale: torch.Tensor,
+                       v_scale: torch.Tensor) -> None:
+    """Quantising append: k, v [T, Hkv, d] bf16 -> e4m3 codes (uint8 caches
+    [NB, Hkv, bs, d]) of x / scale[h]; k_scale, v_scale [Hkv] fp32 on device."""
+    global _fp8w_declared
+    L = _get_lib()
+    if not _fp8w_declared:
+        vp, i32 = ctypes.c_void_p, ctypes.c_int32
+        L.pkv_kv_cache_write_fp8.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32,
+                                             vp]
+        L.pkv_kv_cache_write_fp8.restype = ctypes.c_int
+        _fp8w_declared = True
+    dev = _need_cuda(k, v, slot_mapping, k_cache, v_cache, k_scale, v_scale)
+    if k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
+        raise TypeError("k and v must be bf16")
+    if k_cache.dtype not in (torch.uint8, torch.float8_e4m3fn) or v_cache.dtype != k_cache.dtype:
+        raise TypeError("fp8 caches must be uint8 or float8_e4m3fn")
+    if k_scale.dtype != torch.float32 or v_scale.dtype != torch.float32:
+        raise TypeError("scales must be float32")
+    T, Hkv, d = k.shape
+    NB, _, bs, _ = k_cache.shape
+    with torch.cuda.device(dev):
+        st = L.pkv_kv_cache_write_fp8(_ptr(k), _ptr(v), _ptr(slot_mapping), _ptr(k_cache),
+                                      _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), T, Hkv, d, bs,
+                                      NB, _stream(dev))
+    _check("pkv_kv_cache_write_fp8", st)
+
+
+_swap_declared = False
+
+
+def swap_blocks(src_k: torch.Tensor, src_v: torch.Tensor, dst_k: torch.Tensor,
+                dst_v: torch.Tensor, block_mapping: torch.Tensor,
+                device: torch.device | int | None = None) -> None:
+    """dst pools[dst] = src pools[src] for each (src, dst) row of block_mapping.
+
+    Pools are [num_blocks, Hkv, bs, d]; each may be a CUDA tensor or a pinned
+    CPU tensor (``pin_memory()``); block_mapping likewise.  The copy runs on the
+    current stream of ``device`` (default: the CUDA tensor's device, else the
+    current device)."""
+    global _swap_declared
+    L = _get_lib()
+    if not _swap_declared:
+        vp, i32 = ctypes.c_void_p, ctypes.c_int32
+        L.pkv_swap_blocks.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, i32,
+                                      ctypes.c_int, vp]
+        L.pkv_swap_blocks.restype = ctypes.c_int
+        _swap_declared = True
+    ts = (src_k, src_v, dst_k, dst_v, block_mapping)
+    for t in ts:
+        if not t.is_contiguous():
+            raise ValueError("all tensors must be contiguous")
+        if not t.is_cuda and not t.is_pinned():
+            raise ValueError("CPU tensors must be pinned (pin_memory())")
+    if device is None:
+        cuda = [t.device for t in ts if t.is_cuda]
+        device = cuda[0] if cuda else torch.device("cuda", torch.cuda.current_device())
+    dev = torch.device("cuda", device) if isinstance(device, int) else device
+    if block_mapping.dtype != torch.int64:
+        raise TypeError("block_mapping must be int64")
+    if src_k.dtype != dst_k.dtype or src_k.shape[1:] != dst_k.shape[1:]:
+        raise ValueError("pools must share dtype and block shape")
+    n = block_mapping.numel() // 2
+    NBs, Hkv, bs, d = src_k.shape
+    with torch.cuda.device(dev):
+        st = L.pkv_swap_blocks(_ptr(src_k), _ptr(src_v), _ptr(dst_k), _ptr(dst_v),
+                               _ptr(block_mapping), n, NBs, dst_k.shape[0], Hkv, d, bs,
+                               _dtype_code(src_k), _stream(dev))
+    _check("pkv_swap_blocks", st)
 
 
 _noalloc_declared = False

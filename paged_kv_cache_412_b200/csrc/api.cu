@@ -103,9 +103,10 @@ bool make_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_
     pl.off_meta = pl.off_ml + up(ml_bytes);
     pl.rec_bytes = pl.off_meta + up(meta_bytes);
     // smallest B with counter region(B) + records <= B and room for every counter
-    size_t b = up(pl.rec_bytes + pl.n_bg_max * sizeof(uint32_t));
+    const size_t sync_words = std::max(pl.n_bg_max, pl.records);
+    size_t b = up(pl.rec_bytes + 2 * sync_words * sizeof(uint32_t));
     while (counter_region_bytes(b) + pl.rec_bytes > b ||
-           counter_region_bytes(b) < pl.n_bg_max * sizeof(uint32_t))
+           ready_flags_offset(b) < sync_words * sizeof(uint32_t))
         b += 256;
     pl.bytes = b;
     *plan = pl;
@@ -155,6 +156,28 @@ pkv_status pkv_kv_cache_write(const void* k, const void* v, const int64_t* slot_
                                  reinterpret_cast<cudaStream_t>(stream));
 }
 
+pkv_status pkv_kv_cache_write_fp8(const void* k, const void* v, const int64_t* slot_mapping,
+                                  void* k_cache, void* v_cache, const float* k_scale,
+                                  const float* v_scale, int32_t num_tokens, int32_t num_kv_heads,
+                                  int32_t head_dim, int32_t block_size, int32_t num_blocks,
+                                  pkv_stream_t stream) {
+    if (num_tokens < 0 || num_kv_heads <= 0 || head_dim <= 0 || num_blocks <= 0 ||
+        !is_pow2(block_size) || block_size > 256)
+        return PKV_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
+    if (num_tokens == 0) return PKV_OK;
+    if (!k || !v || !slot_mapping || !k_cache || !v_cache || !k_scale || !v_scale)
+        return PKV_ERR_INVALID_ARG;
+    if (!aligned(k, 16) || !aligned(v, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
+        !aligned(slot_mapping, 8) || !aligned(k_scale, 4) || !aligned(v_scale, 4))
+        return PKV_ERR_INVALID_ARG;
+    const DeviceInfo* di = current_device_info();
+    if (!di) return PKV_ERR_CUDA;
+    return launch_kv_cache_write_fp8(k, v, slot_mapping, k_cache, v_cache, k_scale, v_scale,
+                                     num_tokens, num_kv_heads, head_dim, block_size, num_blocks,
+                                     di->error_word, reinterpret_cast<cudaStream_t>(stream));
+}
+
 size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
                                   int32_t head_dim, int32_t block_size, int32_t max_seq_len,
                                   int32_t partition_size) {
@@ -198,8 +221,10 @@ pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const 
     if (out_dtype == PKV_FP8_E4M3) return PKV_ERR_UNSUPPORTED;
     const bool f32_pair = q_dtype == PKV_F32 && kv_dtype == PKV_F32;
     const bool bf16_pair = q_dtype == PKV_BF16 && kv_dtype == PKV_BF16;
-    if (kv_dtype == PKV_FP8_E4M3) return PKV_ERR_UNSUPPORTED;
-    if (!f32_pair && !bf16_pair) return PKV_ERR_INVALID_ARG;
+    const bool fp8_cache = q_dtype == PKV_BF16 && kv_dtype == PKV_FP8_E4M3;
+    if (!f32_pair && !bf16_pair && !fp8_cache) return PKV_ERR_INVALID_ARG;
+    if (fp8_cache && block_size < 8) return PKV_ERR_UNSUPPORTED;  // tensor-core path only
+    if (fp8_cache && (!k_scale || !v_scale)) return PKV_ERR_INVALID_ARG;
     if ((long long)max_blocks_per_seq * block_size > 0x7fffffffLL) return PKV_ERR_INVALID_ARG;
     if (num_seqs == 0) return PKV_OK;
     if (!q || !k_cache || !v_cache || !block_tables || !seq_lens || !out)
@@ -237,9 +262,10 @@ pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const 
     p.v_scale = v_scale;
     const size_t cnt_region = counter_region_bytes(workspace_bytes);
     if (cnt_region + pl.rec_bytes > workspace_bytes ||
-        cnt_region < pl.n_bg_max * sizeof(uint32_t))
+        ready_flags_offset(workspace_bytes) < std::max(pl.n_bg_max, pl.records) * sizeof(uint32_t))
         return PKV_ERR_WORKSPACE;
     p.counters = reinterpret_cast<unsigned*>(ws);
+    p.ready = reinterpret_cast<unsigned*>(ws + ready_flags_offset(workspace_bytes));
     p.rec_acc = reinterpret_cast<float*>(ws + cnt_region);
     p.rec_ml = reinterpret_cast<float*>(ws + cnt_region + pl.off_ml);
     p.meta = reinterpret_cast<int32_t*>(ws + cnt_region + pl.off_meta);
@@ -259,7 +285,8 @@ pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const 
     p.out_dtype = out_dtype;
     p.scale_log2 = scale * 1.4426950408889634f;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    if (mma) return launch_decode_mma(p, head_dim, group_pad, st, nullptr);
+    if (mma)
+        return launch_decode_mma(p, head_dim, group_pad, kv_dtype == PKV_FP8_E4M3, st, nullptr);
     return launch_decode_simt(p, head_dim, kv_dtype, group_pad, st, nullptr);
 }
 
@@ -282,6 +309,58 @@ pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_ma
     const size_t block_bytes = (size_t)num_kv_heads * block_size * head_dim * es;
     return launch_copy_blocks(k_cache, v_cache, block_mapping, num_pairs, block_bytes, num_blocks,
                               di->error_word, reinterpret_cast<cudaStream_t>(stream));
+}
+
+namespace {
+
+// Device address of p if the current device can dereference it (device or
+// managed memory, or pinned host memory mapped into the device's address
+// space); nullptr otherwise (pageable host memory, another device's memory).
+void* device_view(const void* p) {
+    cudaPointerAttributes a{};
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();  // clear the sticky-free error of an unknown pointer
+        return nullptr;
+    }
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+    if (a.type == cudaMemoryTypeDevice) return a.device == dev ? a.devicePointer : nullptr;
+    if (a.type == cudaMemoryTypeManaged || a.type == cudaMemoryTypeHost) return a.devicePointer;
+    return nullptr;
+}
+
+}  // namespace
+
+pkv_status pkv_swap_blocks(const void* src_k_cache, const void* src_v_cache, void* dst_k_cache,
+                           void* dst_v_cache, const int64_t* block_mapping, int32_t num_pairs,
+                           int32_t src_num_blocks, int32_t dst_num_blocks, int32_t num_kv_heads,
+                           int32_t head_dim, int32_t block_size, pkv_dtype dtype,
+                           pkv_stream_t stream) {
+    if (num_pairs < 0 || num_kv_heads <= 0 || head_dim <= 0 || src_num_blocks <= 0 ||
+        dst_num_blocks <= 0 || !is_pow2(block_size) || block_size > 256)
+        return PKV_ERR_INVALID_ARG;
+    const int es = elem_size(dtype);
+    if (es == 0) return PKV_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return PKV_ERR_UNSUPPORTED;
+    if (num_pairs == 0) return PKV_OK;
+    if (!src_k_cache || !src_v_cache || !dst_k_cache || !dst_v_cache || !block_mapping)
+        return PKV_ERR_INVALID_ARG;
+    const DeviceInfo* di = current_device_info();
+    if (!di) return PKV_ERR_CUDA;
+    // every pointer must be reachable from the device: refuse rather than fault
+    void* sk = device_view(src_k_cache);
+    void* sv = device_view(src_v_cache);
+    void* dk = device_view(dst_k_cache);
+    void* dv = device_view(dst_v_cache);
+    void* bm = device_view(block_mapping);
+    if (!sk || !sv || !dk || !dv || !bm) return PKV_ERR_INVALID_ARG;
+    if (!aligned(sk, 16) || !aligned(sv, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+        !aligned(bm, 8))
+        return PKV_ERR_INVALID_ARG;
+    const size_t block_bytes = (size_t)num_kv_heads * block_size * head_dim * es;
+    return launch_swap_blocks(sk, sv, dk, dv, static_cast<const int64_t*>(bm), num_pairs,
+                              block_bytes, src_num_blocks, dst_num_blocks, di->error_word,
+                              reinterpret_cast<cudaStream_t>(stream));
 }
 
 pkv_status pkv_get_device_error(pkv_stream_t stream, uint32_t* flags) {

@@ -8,6 +8,8 @@
 // copy_blocks: "KV Cache Optimization and PagedAttention" (intro) and "KV Cache
 // Management", "The Bonus: Zero-Copy Sharing" -- shared prefix blocks are
 // stored once; a request privately copies a shared block before appending.
+#include <cuda_fp8.h>
+
 #include <algorithm>
 
 #include "pkv_device.cuh"
@@ -48,6 +50,60 @@ __global__ void kv_cache_write_kernel(const uint4* __restrict__ k, const uint4* 
     }
 }
 
+// fp8 append: one thread per 16 output bytes (16 elements) of one (token, kv
+// head) row, K and V together.  code = e4m3(x / scale[h]): the quotient is the
+// correctly rounded fp32 division, the conversion rounds to nearest even and
+// saturates at +-448 ("KV Cache Management", "Watch Out For": compress the KV
+// cache to 8-bit floats to fit long contexts).
+__global__ void kv_cache_write_fp8_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
+                                          const int64_t* __restrict__ slots,
+                                          uint4* __restrict__ kc, uint4* __restrict__ vc,
+                                          const float* __restrict__ k_scale,
+                                          const float* __restrict__ v_scale, long long total_vecs,
+                                          int vecs_per_row, int num_kv_heads, int block_size,
+                                          int num_blocks, unsigned* err) {
+    griddep_wait();
+    griddep_launch_dependents();
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total_vecs; i += stride) {
+        const long long row = i / vecs_per_row;
+        const int vec = (int)(i - row * vecs_per_row);
+        const long long t = row / num_kv_heads;
+        const int h = (int)(row - t * num_kv_heads);
+        const int64_t slot = __ldg(slots + t);
+        if (slot < 0) continue;
+        if (slot >= (int64_t)num_blocks * block_size) {
+            if (h == 0 && vec == 0) raise_error(err, PKV_DEVERR_BAD_SLOT);
+            continue;
+        }
+        const int64_t blk = slot / block_size;
+        const int off = (int)(slot - blk * block_size);
+        const size_t dst = (((size_t)blk * num_kv_heads + h) * block_size + off) * vecs_per_row + vec;
+        const float ks = __ldg(k_scale + h), vs = __ldg(v_scale + h);
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+            const uint4* src = (which == 0 ? k : v) + 2 * i;  // 16 bf16 = 32 bytes
+            const float sc = which == 0 ? ks : vs;
+            const uint4 a = __ldg(src), b = __ldg(src + 1);
+            float f[16];
+            bf16x8_to_f32(a, f);
+            bf16x8_to_f32(b, f + 8);
+            uint32_t w[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const __nv_fp8x2_storage_t lo = __nv_cvt_float2_to_fp8x2(
+                    make_float2(__fdiv_rn(f[4 * q], sc), __fdiv_rn(f[4 * q + 1], sc)),
+                    __NV_SATFINITE, __NV_E4M3);
+                const __nv_fp8x2_storage_t hi = __nv_cvt_float2_to_fp8x2(
+                    make_float2(__fdiv_rn(f[4 * q + 2], sc), __fdiv_rn(f[4 * q + 3], sc)),
+                    __NV_SATFINITE, __NV_E4M3);
+                w[q] = (uint32_t)lo | ((uint32_t)hi << 16);
+            }
+            (which == 0 ? kc : vc)[dst] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+    }
+}
+
 // grid.x = pair, grid.y = 0 (K) / 1 (V), grid.z = slice of the block.
 __global__ void copy_blocks_kernel(uint4* __restrict__ kc, uint4* __restrict__ vc,
                                    const int64_t* __restrict__ pairs, long long vecs_per_block,
@@ -67,7 +123,45 @@ __global__ void copy_blocks_kernel(uint4* __restrict__ kc, uint4* __restrict__ v
     for (long long i = lo + threadIdx.x; i < hi; i += blockDim.x) d[i] = s[i];
 }
 
+// Block copy between two pools (either may be pinned host memory reached over
+// the bus): grid.x = pair, grid.y = 0 (K) / 1 (V), grid.z = slice of the block.
+__global__ void swap_blocks_kernel(const uint4* __restrict__ sk, const uint4* __restrict__ sv,
+                                   uint4* __restrict__ dk, uint4* __restrict__ dv,
+                                   const int64_t* __restrict__ pairs, long long vecs_per_block,
+                                   int slice_vecs, int src_blocks, int dst_blocks, unsigned* err) {
+    const int64_t src = pairs[2 * blockIdx.x];
+    const int64_t dst = pairs[2 * blockIdx.x + 1];
+    if (src < 0 || dst < 0 || src >= src_blocks || dst >= dst_blocks) {
+        if (threadIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0)
+            raise_error(err, PKV_DEVERR_BAD_PAIR);
+        return;
+    }
+    const uint4* s = (blockIdx.y == 0 ? sk : sv) + src * vecs_per_block;
+    uint4* d = (blockIdx.y == 0 ? dk : dv) + dst * vecs_per_block;
+    const long long lo = (long long)blockIdx.z * slice_vecs;
+    const long long hi = min(lo + slice_vecs, vecs_per_block);
+    for (long long i = lo + threadIdx.x; i < hi; i += blockDim.x) d[i] = s[i];
+}
+
 }  // namespace
+
+pkv_status launch_swap_blocks(const void* src_k, const void* src_v, void* dst_k, void* dst_v,
+                              const int64_t* pairs, int num_pairs, size_t block_bytes,
+                              int src_blocks, int dst_blocks, unsigned* err,
+                              cudaStream_t stream) {
+    if (num_pairs == 0) return PKV_OK;
+    const long long vecs = (long long)(block_bytes / 16);
+    const int threads = 256;
+    const int slice = threads * 4;
+    const long long slices = (vecs + slice - 1) / slice;
+    if (slices > 65535) return PKV_ERR_UNSUPPORTED;
+    dim3 grid(num_pairs, 2, (unsigned)slices);
+    swap_blocks_kernel<<<grid, threads, 0, stream>>>(
+        static_cast<const uint4*>(src_k), static_cast<const uint4*>(src_v),
+        static_cast<uint4*>(dst_k), static_cast<uint4*>(dst_v), pairs, vecs, slice, src_blocks,
+        dst_blocks, err);
+    return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
 
 pkv_status launch_kv_cache_write(const void* k, const void* v, const int64_t* slots,
                                  void* k_cache, void* v_cache, int num_tokens, int num_kv_heads,
@@ -86,6 +180,28 @@ pkv_status launch_kv_cache_write(const void* k, const void* v, const int64_t* sl
         &L.cfg, kv_cache_write_kernel, static_cast<const uint4*>(k), static_cast<const uint4*>(v),
         slots, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), total, vecs_per_row,
         num_kv_heads, block_size, num_blocks, err);
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+pkv_status launch_kv_cache_write_fp8(const void* k, const void* v, const int64_t* slots,
+                                     void* k_cache, void* v_cache, const float* k_scale,
+                                     const float* v_scale, int num_tokens, int num_kv_heads,
+                                     int head_dim, int block_size, int num_blocks, unsigned* err,
+                                     cudaStream_t stream) {
+    const DeviceInfo* di = current_device_info();
+    if (!di) return PKV_ERR_CUDA;
+    const int vecs_per_row = head_dim / 16;  // 16-byte vectors of fp8 codes
+    const long long total = (long long)num_tokens * num_kv_heads * vecs_per_row;
+    if (total == 0) return PKV_OK;
+    const int threads = 256;
+    const long long want = (total + threads - 1) / threads;
+    const int grid = (int)std::min<long long>(want, (long long)di->num_sms * 8);
+    PdlLaunch L(dim3(grid), dim3(threads), 0, stream);
+    const cudaError_t e = cudaLaunchKernelEx(
+        &L.cfg, kv_cache_write_fp8_kernel, static_cast<const uint4*>(k),
+        static_cast<const uint4*>(v), slots, static_cast<uint4*>(k_cache),
+        static_cast<uint4*>(v_cache), k_scale, v_scale, total, vecs_per_row, num_kv_heads,
+        block_size, num_blocks, err);
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 

@@ -34,13 +34,16 @@ struct Cursor {
 };
 
 // Warp-cooperative search for global chunk index s (all lanes get the result).
+// L_first, if >= 0, is this lane's (clamped) length of request `lane`, already
+// loaded by the caller; it saves a dependent global load on the first pass.
 template <int CH>
-__device__ Cursor locate(const DecodeParams& p, long long s, int lane) {
+__device__ Cursor locate(const DecodeParams& p, long long s, int lane, int L_first = -1) {
     Cursor cur{p.num_seqs, 0, 0, 0, 0};
     long long base = 0;
     for (int b0 = 0; b0 < p.num_seqs; b0 += 32) {
         const int b = b0 + lane;
-        const int L = b < p.num_seqs ? clamp_len(p, b, false) : 0;
+        const int L = b < p.num_seqs ? ((b0 == 0 && L_first >= 0) ? L_first : clamp_len(p, b, false))
+                                     : 0;
         const long long n = (long long)chunks_of<CH>(L) * p.num_hg;
         long long incl = n;
 #pragma unroll
@@ -116,6 +119,7 @@ struct SegIter {
     long long u, s1, g;
     Cursor cur;
     bool valid;
+    int L_first = -1;  // this lane's length of request `lane` (first 32 requests)
 
     __device__ void start_unit(const DecodeParams& p, int lane) {
         valid = u < nunits;
@@ -123,15 +127,17 @@ struct SegIter {
         const long long s0 = u * W;
         s1 = min(s0 + W, total);
         g = s0;
-        cur = locate<CH>(p, s0, lane);
+        cur = locate<CH>(p, s0, lane, L_first);
         valid = cur.nch > 0;
     }
 
-    __device__ void init(const DecodeParams& p, long long total_, long long W_, int lane) {
+    __device__ void init(const DecodeParams& p, long long total_, long long W_, int lane,
+                         int L_first_ = -1) {
         total = total_;
         W = W_;
         nunits = (total + W - 1) / W;
         u = blockIdx.x;
+        L_first = L_first_;
         start_unit(p, lane);
     }
 

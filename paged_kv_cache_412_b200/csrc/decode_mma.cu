@@ -33,6 +33,8 @@
 // the merger): out = sum_u 2^(m_u - M) acc_u / sum_u 2^(m_u - M) l_u.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
 
 #include <algorithm>
 #include <mutex>
@@ -50,17 +52,22 @@ constexpr int kRingBudget = 104448;  // 3 stages of K+V+q at head_dim 128
 constexpr int cmin(int a, int b) { return a < b ? a : b; }
 constexpr int cmax(int a, int b) { return a > b ? a : b; }
 
-template <int D, int NT>
+// F8 = false: bf16 cache, tiles land swizzled and feed bf16 MMAs directly.
+// F8 = true : fp8 (e4m3) cache, tiles land as plain rows of head_dim bytes and
+//             the consumer widens them (exactly) to f16 in a swizzled staging
+//             tile before f16 MMAs; q is widened to f16 likewise.
+template <int D, int NT, bool F8>
 struct MmaCfg {
-    static constexpr int NHALF = D / 64;            // 128-byte column halves of a row
+    static constexpr int NHALF = D / 64;            // 128-byte column halves of a 16-bit row
     static constexpr int KS = D / 16;               // k-steps of q.K^T, m-tiles of P.V
-    static constexpr int HALF_BYTES = kCH * 128;    // one swizzled half region
-    static constexpr int KV_BYTES = NHALF * HALF_BYTES;
+    static constexpr int HALF_BYTES = kCH * 128;    // one swizzled half region (16-bit data)
+    static constexpr int KV_BYTES = F8 ? kCH * D : NHALF * HALF_BYTES;  // K (or V) of a stage
+    static constexpr int STG_BYTES = F8 ? 2 * NHALF * HALF_BYTES : 0;  // f16 K+V staging
     static constexpr int GP = 8 * NT;               // query heads per head group (padded)
     static constexpr int Q_BYTES = GP * D * 2;      // the group's q rows (first stage of a segment)
     // K | V | q, rounded to the 1 KB the 128-byte swizzle pattern repeats on
     static constexpr int STAGE_BYTES = (2 * KV_BYTES + Q_BYTES + 1023) / 1024 * 1024;
-    static constexpr int NSTAGE = cmax(2, cmin(8, kRingBudget / STAGE_BYTES));
+    static constexpr int NSTAGE = cmax(2, cmin(8, (kRingBudget - STG_BYTES) / STAGE_BYTES));
 };
 
 // ---- PTX wrappers -----------------------------------------------------------
@@ -99,6 +106,43 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+__device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                        uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+template <bool F8>
+__device__ __forceinline__ void mma16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    if constexpr (F8)
+        mma_f16(c, a, b0, b1);
+    else
+        mma_bf16(c, a, b0, b1);
+}
+
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+    const __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+__device__ __forceinline__ float f16_round(float x) { return __half2float(__float2half_rn(x)); }
+
+// two bf16 (one 32-bit word) -> two f16, exact inside the f16 range
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+    return pack_f16(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// four e4m3 codes (one 32-bit word) -> four f16 (two 32-bit words), exact
+__device__ __forceinline__ void e4m3x4_to_f16(uint32_t w, uint32_t& lo, uint32_t& hi) {
+    const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xffffu), __NV_E4M3);
+    const __half2_raw b = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w >> 16), __NV_E4M3);
+    lo = (uint32_t)a.x | ((uint32_t)a.y << 16);
+    hi = (uint32_t)b.x | ((uint32_t)b.y << 16);
+}
+
 __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
     uint32_t y;
     asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
@@ -122,14 +166,15 @@ __device__ __forceinline__ float ld_cg(const float* p) { return __ldcg(p); }
 
 // ---- shared-memory layout ------------------------------------------------------
 
-template <int D, int NT>
+template <int D, int NT, bool F8>
 struct Smem {
-    using C = MmaCfg<D, NT>;
+    using C = MmaCfg<D, NT, F8>;
     static constexpr int NDUMP = 2;                       // consumer -> epilogue hand-off slots
     static constexpr int DUMP_ACC = C::KS * NT * 4;       // acc registers per lane
     static constexpr int DUMP_ML = NT * 4;                // m[2], l[2] per n-tile per lane
     static constexpr int DUMP_BYTES = (DUMP_ACC + DUMP_ML) * 32 * 4;
-    static constexpr int OFF_DUMP = C::NSTAGE * C::STAGE_BYTES;
+    static constexpr int OFF_STG = C::NSTAGE * C::STAGE_BYTES;
+    static constexpr int OFF_DUMP = OFF_STG + C::STG_BYTES;
     static constexpr int OFF_BAR = OFF_DUMP + NDUMP * DUMP_BYTES;
     static constexpr int OFF_META = OFF_BAR + (2 * C::NSTAGE + 2 * NDUMP) * 8;
     static constexpr int OFF_CTRL = OFF_META + 2 * C::NSTAGE * 4;
@@ -138,9 +183,9 @@ struct Smem {
 
 // ---- producer ------------------------------------------------------------------
 
-template <int D, int NT>
+template <int D, int NT, bool F8>
 struct Producer {
-    using C = MmaCfg<D, NT>;
+    using C = MmaCfg<D, NT, F8>;
 
     const DecodeParams& p;
     const CUtensorMap* tmk;
@@ -219,8 +264,8 @@ struct Producer {
                 st_bad[ring.stage] = bad;
                 if (bad) raise_error(p.err, PKV_DEVERR_BAD_BLOCK);
                 const uint32_t qbytes = c == sg.c0 ? (uint32_t)gv * D * 2u : 0u;
-                mbar_arrive_expect_tx(&full[ring.stage],
-                                      nvalid * 2u * C::NHALF * rb * 128u + qbytes);
+                const uint32_t row_bytes = F8 ? (uint32_t)D : (uint32_t)C::NHALF * 128u;
+                mbar_arrive_expect_tx(&full[ring.stage], nvalid * 2u * rb * row_bytes + qbytes);
                 if (qbytes)  // the group's q rows ride with the segment's first stage
                     bulk_load(sq, static_cast<const __nv_bfloat16*>(p.q) +
                                       ((size_t)cur.b * p.num_q_heads + hq0) * D,
@@ -233,12 +278,17 @@ struct Producer {
                     const int srow = (j << p.log2_bs) - t0 > 0 ? (j << p.log2_bs) - t0 : 0;
                     const int boff = t0 - (j << p.log2_bs) > 0 ? t0 - (j << p.log2_bs) : 0;
                     const int grow = (phys * p.num_kv_heads + kvh) * p.block_size + boff;
+                    if constexpr (F8) {
+                        tma_load_2d(sk + srow * D, tmk, 0, grow, &full[ring.stage], policy);
+                        tma_load_2d(sv + srow * D, tmv, 0, grow, &full[ring.stage], policy);
+                    } else {
 #pragma unroll
-                    for (int h = 0; h < C::NHALF; ++h) {
-                        tma_load_2d(sk + h * C::HALF_BYTES + srow * 128, tmk, h * 64, grow,
-                                    &full[ring.stage], policy);
-                        tma_load_2d(sv + h * C::HALF_BYTES + srow * 128, tmv, h * 64, grow,
-                                    &full[ring.stage], policy);
+                        for (int h = 0; h < C::NHALF; ++h) {
+                            tma_load_2d(sk + h * C::HALF_BYTES + srow * 128, tmk, h * 64, grow,
+                                        &full[ring.stage], policy);
+                            tma_load_2d(sv + h * C::HALF_BYTES + srow * 128, tmv, h * 64, grow,
+                                        &full[ring.stage], policy);
+                        }
                     }
                 }
             }
@@ -288,7 +338,7 @@ struct Producer {
 // Per-segment facts every role derives the same way.
 struct SegInfo {
     long long u, u_first, u_last;
-    int nseg, hq0, gv, b;
+    int nseg, hq0, gv, b, kvh;
     size_t bg;
 };
 
@@ -303,22 +353,24 @@ __device__ __forceinline__ SegInfo seg_info(const DecodeParams& p, const Segment
     si.hq0 = kvh * p.group + sub * GP;
     si.gv = min(GP, p.group - sub * GP);
     si.b = sg.cur.b;
+    si.kvh = kvh;
     si.bg = (size_t)sg.cur.b * p.num_hg + sg.cur.hg;
     return si;
 }
 
 // ---- consumer (tensor-core math) ----------------------------------------------
 
-template <int D, int NT>
+template <int D, int NT, bool F8>
 __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                                         unsigned char* smem, uint64_t* full, uint64_t* empty,
                                         uint64_t* dfull, uint64_t* dempty, const int* st_ntok,
                                         const unsigned* st_bad, volatile int* ctrl, int lane) {
-    using C = MmaCfg<D, NT>;
-    using S = Smem<D, NT>;
+    using C = MmaCfg<D, NT, F8>;
+    using S = Smem<D, NT, F8>;
     constexpr int GP = C::GP;
     const int grp = lane >> 2, tig = lane & 3;
     const int mi = lane >> 3, r8 = lane & 7;
+    unsigned char* stg = smem + S::OFF_STG;  // f16 staging (fp8 caches only)
     // ldmatrix row/chunk components that depend only on the lane
     const int k_row = r8 + 8 * (mi & 1), k_cx = mi >> 1;  // K (A operand)
     const int v_row = r8 + 8 * (mi >> 1), v_cx = mi & 1;  // V^T (A operand, transposed load)
@@ -328,6 +380,8 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
         const Segment sg = it.current();
         it.advance(p, lane);
         const SegInfo si = seg_info<GP>(p, sg, it.W);
+        // softmax scale in log2 units, times the K dequantisation scale for fp8
+        const float s_log2 = F8 ? p.scale_log2 * __ldg(p.k_scale + si.kvh) : p.scale_log2;
 
         uint32_t qb[NT][C::KS][2];
         float m[NT][2], l[NT][2], acc[C::KS][NT][4];
@@ -354,7 +408,6 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
             const bool whole = ntok == kCH && bad == 0;
             unsigned char* sk = smem + ring.stage * C::STAGE_BYTES;
             unsigned char* sv = sk + C::KV_BYTES;
-            const uint32_t skb = smem_addr(sk), svb = smem_addr(sv);
 
             if (c == sg.c0) {
                 // Q^T B-fragments: head nt*8+grp, dims ks*16 + 2*tig (+1) and +8 (+9).
@@ -364,13 +417,55 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                     const int h = nt * 8 + grp;
 #pragma unroll
                     for (int ks = 0; ks < C::KS; ++ks) {
-                        qb[nt][ks][0] = h < si.gv ? sq[h * (D / 2) + ks * 8 + tig] : 0u;
-                        qb[nt][ks][1] = h < si.gv ? sq[h * (D / 2) + ks * 8 + 4 + tig] : 0u;
+                        uint32_t w0 = h < si.gv ? sq[h * (D / 2) + ks * 8 + tig] : 0u;
+                        uint32_t w1 = h < si.gv ? sq[h * (D / 2) + ks * 8 + 4 + tig] : 0u;
+                        if constexpr (F8) {
+                            w0 = bf16x2_to_f16x2(w0);
+                            w1 = bf16x2_to_f16x2(w1);
+                        }
+                        qb[nt][ks][0] = w0;
+                        qb[nt][ks][1] = w1;
                     }
                 }
             }
 
-            if (!whole) {
+            if constexpr (F8) {
+                // Widen the stage's e4m3 K and V rows to f16 in the swizzled
+                // staging tile; tokens that do not take part become zero rows.
+                // The fp8 stage is then free for the next copy.
+#pragma unroll 4
+                for (int idx = lane; idx < 2 * kCH * (D / 16); idx += 32) {
+                    const int part = idx / (kCH * (D / 16));
+                    const int rest = idx % (kCH * (D / 16));
+                    const int row = rest / (D / 16), c16 = rest % (D / 16);
+                    bool valid = whole;
+                    if (!whole) {
+                        const int jrel = ((c * kCH + row) >> p.log2_bs) - ((c * kCH) >> p.log2_bs);
+                        valid = row < ntok && !((bad >> jrel) & 1u);
+                    }
+                    uint4 o0 = make_uint4(0, 0, 0, 0), o1 = make_uint4(0, 0, 0, 0);
+                    if (valid) {
+                        const uint4 raw = *reinterpret_cast<const uint4*>(
+                            (part ? sv : sk) + row * D + c16 * 16);
+                        e4m3x4_to_f16(raw.x, o0.x, o0.y);
+                        e4m3x4_to_f16(raw.y, o0.z, o0.w);
+                        e4m3x4_to_f16(raw.z, o1.x, o1.y);
+                        e4m3x4_to_f16(raw.w, o1.z, o1.w);
+                    }
+                    const int half = (c16 * 16) >> 6, cc = ((c16 * 16) & 63) >> 3;
+                    unsigned char* dst = stg + part * C::NHALF * C::HALF_BYTES +
+                                         half * C::HALF_BYTES + row * 128;
+                    *reinterpret_cast<uint4*>(dst + ((cc ^ (row & 7)) << 4)) = o0;
+                    *reinterpret_cast<uint4*>(dst + (((cc + 1) ^ (row & 7)) << 4)) = o1;
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[ring.stage]);
+                sk = stg;
+                sv = stg + C::NHALF * C::HALF_BYTES;
+            }
+            const uint32_t skb = smem_addr(sk), svb = smem_addr(sv);
+
+            if (!F8 && !whole) {
                 // Rows of tokens that do not take part (past the end, or in a
                 // block the table got wrong) may hold stale or poisoned data:
                 // zero their V rows so 0-weight x NaN cannot reach the sum.
@@ -403,7 +498,7 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                     uint32_t a[4];
                     ldsm_x4(skb + half * C::HALF_BYTES + (mt * 16 + k_row) * 128 + (chunk << 4), a);
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) mma_bf16(s[mt][nt], a, qb[nt][ks][0], qb[nt][ks][1]);
+                    for (int nt = 0; nt < NT; ++nt) mma16<F8>(s[mt][nt], a, qb[nt][ks][0], qb[nt][ks][1]);
                 }
             }
 
@@ -415,7 +510,7 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) s[mt][nt][i] *= p.scale_log2;
+                    for (int i = 0; i < 4; ++i) s[mt][nt][i] *= s_log2;
                 if (!whole) {
 #pragma unroll
                     for (int hi = 0; hi < 2; ++hi) {
@@ -478,9 +573,15 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
 #pragma unroll
                     for (int hi = 0; hi < 2; ++hi) {
                         const float p0 = s[mt][nt][2 * hi], p1 = s[mt][nt][2 * hi + 1];
-                        const float h0 = bf16_round(p0), h1 = bf16_round(p1);
-                        bh[nt][hi] = movmatrix_t(pack_bf16(h0, h1));
-                        bl[nt][hi] = movmatrix_t(pack_bf16(p0 - h0, p1 - h1));
+                        if constexpr (F8) {
+                            const float h0 = f16_round(p0), h1 = f16_round(p1);
+                            bh[nt][hi] = movmatrix_t(pack_f16(h0, h1));
+                            bl[nt][hi] = movmatrix_t(pack_f16(p0 - h0, p1 - h1));
+                        } else {
+                            const float h0 = bf16_round(p0), h1 = bf16_round(p1);
+                            bh[nt][hi] = movmatrix_t(pack_bf16(h0, h1));
+                            bl[nt][hi] = movmatrix_t(pack_bf16(p0 - h0, p1 - h1));
+                        }
                     }
                 }
 #pragma unroll
@@ -491,14 +592,18 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                     ldsm_x4_t(svb + half * C::HALF_BYTES + (mt * 16 + v_row) * 128 + (chunk << 4), a);
 #pragma unroll
                     for (int nt = 0; nt < NT; ++nt) {
-                        mma_bf16(acc[dt][nt], a, bh[nt][0], bh[nt][1]);
-                        mma_bf16(acc[dt][nt], a, bl[nt][0], bl[nt][1]);
+                        mma16<F8>(acc[dt][nt], a, bh[nt][0], bh[nt][1]);
+                        mma16<F8>(acc[dt][nt], a, bl[nt][0], bl[nt][1]);
                     }
                 }
             }
-            if (!whole) fence_proxy_async_smem();  // our zero-fill before the next TMA write
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[ring.stage]);
+            if constexpr (!F8) {
+                if (!whole) fence_proxy_async_smem();  // our zero-fill before the next TMA write
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[ring.stage]);
+            } else {
+                __syncwarp();  // staging tile reads done before the next widening
+            }
             ring.advance(C::NSTAGE);
         }
 
@@ -532,12 +637,12 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
 
 // ---- epilogue: normalise, or write a partial record and merge the group ----
 
-template <int D, int NT>
+template <int D, int NT, bool F8>
 __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it,
                                          unsigned char* smem, uint64_t* dfull, uint64_t* dempty,
                                          volatile int* ctrl, int lane) {
-    using C = MmaCfg<D, NT>;
-    using S = Smem<D, NT>;
+    using C = MmaCfg<D, NT, F8>;
+    using S = Smem<D, NT, F8>;
     constexpr int GP = C::GP;
     const int grp = lane >> 2, tig = lane & 3;
     Ring dring;
@@ -552,6 +657,7 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
         const Segment sg = it.current();
         it.advance(p, lane);
         const SegInfo si = seg_info<GP>(p, sg, it.W);
+        const float vsc = F8 ? __ldg(p.v_scale + si.kvh) : 1.f;  // V dequantisation scale
         if (ctrl[0] || !mbar_wait(&dfull[dring.stage], dring.phase)) {
             if (lane == 0 && !ctrl[0]) {
                 ctrl[0] = 1;
@@ -595,7 +701,7 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
                 for (int j = 0; j < 2; ++j) {
                     const int h = nt * 8 + 2 * tig + j;
                     if (h >= si.gv) continue;
-                    const float inv = l[nt][j] > 0.f ? 1.f / l[nt][j] : 0.f;
+                    const float inv = l[nt][j] > 0.f ? vsc / l[nt][j] : 0.f;
                     const size_t orow = ((size_t)si.b * p.num_q_heads + si.hq0 + h) * D;
 #pragma unroll
                     for (int dt = 0; dt < C::KS; ++dt) {
@@ -610,92 +716,158 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
             if (lane == 0) raise_error(p.err, PKV_DEVERR_BAD_SEQ_LEN);
             continue;
         }
-        const size_t rec = si.bg + si.u;
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int h = nt * 8 + 2 * tig + j;
-                float* ra = p.rec_acc + (rec * GP + h) * D;
-#pragma unroll
-                for (int dt = 0; dt < C::KS; ++dt) {
-                    ra[dt * 16 + grp] = acc[dt][nt][j];
-                    ra[dt * 16 + grp + 8] = acc[dt][nt][j + 2];
-                }
-                if (grp == 0) {
-                    p.rec_ml[(rec * GP + h) * 2] = m[nt][j];
-                    p.rec_ml[(rec * GP + h) * 2 + 1] = l[nt][j];
-                }
-            }
-        __threadfence();
-        __syncwarp();
+        // Arrive first.  Only a part that is not the last of its group to
+        // finish publishes its partial result (record, then a ready flag); the
+        // last one keeps its own in registers and merges the others'.
         unsigned arrived = 0;
         if (lane == 0) arrived = atomicAdd(p.counters + si.bg, 1u);
         arrived = __shfl_sync(FULL_MASK, arrived, 0);
-        if (arrived != (unsigned)(si.nseg - 1)) continue;
+        const size_t rec = si.bg + si.u;
+        if (arrived != (unsigned)(si.nseg - 1)) {
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int h = nt * 8 + 2 * tig + j;
+                    float* ra = p.rec_acc + (rec * GP + h) * D;
+#pragma unroll
+                    for (int dt = 0; dt < C::KS; ++dt) {
+                        ra[dt * 16 + grp] = acc[dt][nt][j];
+                        ra[dt * 16 + grp + 8] = acc[dt][nt][j + 2];
+                    }
+                    if (grp == 0) {
+                        p.rec_ml[(rec * GP + h) * 2] = m[nt][j];
+                        p.rec_ml[(rec * GP + h) * 2 + 1] = l[nt][j];
+                    }
+                }
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) atomicExch(p.ready + rec, 1u);
+            continue;
+        }
 
-        // Last unit of this (request, head group) to finish: merge all records
-        // (its own from registers, the others from L2).
+        // Last part: wait (bounded) until every other part's record is out.
+        int ok = 1;
+        if (lane == 0) {
+            const uint64_t t0 = global_timer_ns();
+            for (long long uu = si.u_first; uu <= si.u_last && ok; ++uu) {
+                if (uu == si.u) continue;
+                volatile unsigned* f = p.ready + si.bg + uu;
+                for (uint32_t it = 0; *f == 0u; ++it) {
+                    if ((it & 63u) == 63u && global_timer_ns() - t0 > kWaitLimitNs) {
+                        ok = 0;
+                        break;
+                    }
+                }
+            }
+            if (!ok) raise_error(p.err, PKV_DEVERR_TIMEOUT);
+        }
+        ok = __shfl_sync(FULL_MASK, ok, 0);
+        if (!ok) continue;
         __threadfence();
+        // Online merge, records in order: M = max m, S = sum 2^(m-M) l,
+        // A = sum 2^(m-M) acc, out = A / S.  The other records are fetched two
+        // at a time with every load of the pair in flight before any math.
+        float Mc[NT][2], Sc[NT][2], A[C::KS][NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                Mc[nt][j] = m[nt][j];
+                Sc[nt][j] = l[nt][j];
+            }
+#pragma unroll
+        for (int dt = 0; dt < C::KS; ++dt)
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int i = 0; i < 4; ++i) A[dt][nt][i] = acc[dt][nt][i];
+        for (long long uu0 = si.u_first; uu0 <= si.u_last; uu0 += 2) {
+            float mr[2][NT][2], lr[2][NT][2], ar[2][C::KS][NT][4];
+            bool use[2];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                const long long uu = uu0 + k;
+                use[k] = uu <= si.u_last && uu != si.u;
+                if (!use[k]) continue;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const size_t rr = (si.bg + uu) * GP + nt * 8 + 2 * tig + j;
+                        mr[k][nt][j] = ld_cg(p.rec_ml + rr * 2);
+                        lr[k][nt][j] = ld_cg(p.rec_ml + rr * 2 + 1);
+                        const float* ra = p.rec_acc + rr * D;
+#pragma unroll
+                        for (int dt = 0; dt < C::KS; ++dt) {
+                            ar[k][dt][nt][j] = ld_cg(ra + dt * 16 + grp);
+                            ar[k][dt][nt][j + 2] = ld_cg(ra + dt * 16 + grp + 8);
+                        }
+                    }
+            }
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+                if (!use[k]) continue;
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const float M = fmaxf(Mc[nt][j], mr[k][nt][j]);
+                        const float mref = M == -INFINITY ? 0.f : M;
+                        const float fa = exp2f(Mc[nt][j] - mref), fb = exp2f(mr[k][nt][j] - mref);
+                        Sc[nt][j] = Sc[nt][j] * fa + lr[k][nt][j] * fb;
+#pragma unroll
+                        for (int dt = 0; dt < C::KS; ++dt) {
+                            A[dt][nt][j] = A[dt][nt][j] * fa + ar[k][dt][nt][j] * fb;
+                            A[dt][nt][j + 2] = A[dt][nt][j + 2] * fa + ar[k][dt][nt][j + 2] * fb;
+                        }
+                        Mc[nt][j] = M;
+                    }
+            }
+        }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 const int h = nt * 8 + 2 * tig + j;
-                float M = m[nt][j];
-#pragma unroll 4
-                for (long long uu = si.u_first; uu <= si.u_last; ++uu)
-                    if (uu != si.u) M = fmaxf(M, ld_cg(p.rec_ml + ((si.bg + uu) * GP + h) * 2));
-                const float mref = M == -INFINITY ? 0.f : M;
-                const float fo = exp2f(m[nt][j] - mref);
-                float S = l[nt][j] * fo;
-                float A[C::KS][2];
-#pragma unroll
-                for (int dt = 0; dt < C::KS; ++dt) {
-                    A[dt][0] = acc[dt][nt][j] * fo;
-                    A[dt][1] = acc[dt][nt][j + 2] * fo;
-                }
-#pragma unroll 2
-                for (long long uu = si.u_first; uu <= si.u_last; ++uu) {
-                    if (uu == si.u) continue;
-                    const size_t rr = (si.bg + uu) * GP + h;
-                    const float f = exp2f(ld_cg(p.rec_ml + rr * 2) - mref);
-                    S = fmaf(ld_cg(p.rec_ml + rr * 2 + 1), f, S);
-                    const float* ra = p.rec_acc + rr * D;
-#pragma unroll
-                    for (int dt = 0; dt < C::KS; ++dt) {
-                        A[dt][0] = fmaf(ld_cg(ra + dt * 16 + grp), f, A[dt][0]);
-                        A[dt][1] = fmaf(ld_cg(ra + dt * 16 + grp + 8), f, A[dt][1]);
-                    }
-                }
                 if (h >= si.gv) continue;
-                const float inv = S > 0.f ? 1.f / S : 0.f;
+                const float inv = Sc[nt][j] > 0.f ? vsc / Sc[nt][j] : 0.f;
                 const size_t orow = ((size_t)si.b * p.num_q_heads + si.hq0 + h) * D;
 #pragma unroll
                 for (int dt = 0; dt < C::KS; ++dt) {
-                    store_out(p.out, orow + dt * 16 + grp, A[dt][0] * inv, p.out_dtype);
-                    store_out(p.out, orow + dt * 16 + grp + 8, A[dt][1] * inv, p.out_dtype);
+                    store_out(p.out, orow + dt * 16 + grp, A[dt][nt][j] * inv, p.out_dtype);
+                    store_out(p.out, orow + dt * 16 + grp + 8, A[dt][nt][j + 2] * inv, p.out_dtype);
                 }
             }
+        __syncwarp();
+        if (lane == 0)  // ready for the next call
+            for (long long uu = si.u_first; uu <= si.u_last; ++uu) p.ready[si.bg + uu] = 0u;
         if (lane == 0) p.counters[si.bg] = 0u;  // ready for the next call
     }
 }
 
 // Total chunk count, computed by one warp (same value in every warp and CTA).
-__device__ __forceinline__ long long total_chunks_warp(const DecodeParams& p, int lane, bool flag) {
+// *L_first receives this lane's length of request `lane` (or 0).
+__device__ __forceinline__ long long total_chunks_warp(const DecodeParams& p, int lane, bool flag,
+                                                       int* L_first) {
     long long t = 0;
-    for (int b = lane; b < p.num_seqs; b += 32) t += chunks_of<kCH>(clamp_len(p, b, flag));
+    *L_first = 0;
+    for (int b = lane; b < p.num_seqs; b += 32) {
+        const int L = clamp_len(p, b, flag);
+        if (b == lane) *L_first = L;
+        t += chunks_of<kCH>(L);
+    }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(FULL_MASK, t, off);
     return t * p.num_hg;
 }
 
-template <int D, int NT>
+template <int D, int NT, bool F8>
 __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_constant__ DecodeParams p,
                                                              const __grid_constant__ CUtensorMap tmk,
                                                              const __grid_constant__ CUtensorMap tmv) {
-    using C = MmaCfg<D, NT>;
-    using S = Smem<D, NT>;
+    using C = MmaCfg<D, NT, F8>;
+    using S = Smem<D, NT, F8>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
@@ -728,29 +900,30 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
     // guarantees are not produced by the kernel right before this one; so it
     // overlaps that kernel's tail.  Each role waits on the grid dependency
     // before touching K/V, q, out or the workspace.
-    const long long total = total_chunks_warp(p, lane, blockIdx.x == 0 && warp == 0);
+    int L_first = 0;
+    const long long total = total_chunks_warp(p, lane, blockIdx.x == 0 && warp == 0, &L_first);
     if (total == 0) {
         if (warp == 2) {
             SegIter<kCH> none;
             none.valid = false;
-            epilogue<D, NT>(p, none, smem, dfull, dempty, ctrl, lane);
+            epilogue<D, NT, F8>(p, none, smem, dfull, dempty, ctrl, lane);
         }
         return;
     }
     long long W = p.fixed_units > 0 ? p.fixed_units : (total + gridDim.x - 1) / gridDim.x;
     if (W < 1) W = 1;
     SegIter<kCH> it;
-    it.init(p, total, W, lane);
+    it.init(p, total, W, lane, L_first);
 
     if (warp == 0) {
-        Producer<D, NT> pr{p, &tmk, &tmv, smem, full, empty, st_ntok, st_bad, ctrl, lane,
+        Producer<D, NT, F8> pr{p, &tmk, &tmv, smem, full, empty, st_ntok, st_bad, ctrl, lane,
                            l2_policy_evict_first()};
         pr.run(it);
         if (!pr.waited) griddep_wait();
     } else if (warp == 1) {
-        consume<D, NT>(p, it, smem, full, empty, dfull, dempty, st_ntok, st_bad, ctrl, lane);
+        consume<D, NT, F8>(p, it, smem, full, empty, dfull, dempty, st_ntok, st_bad, ctrl, lane);
     } else {
-        epilogue<D, NT>(p, it, smem, dfull, dempty, ctrl, lane);
+        epilogue<D, NT, F8>(p, it, smem, dfull, dempty, ctrl, lane);
     }
 }
 
@@ -772,29 +945,32 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // 2-D view of a cache: rows = num_blocks*Hkv*block_size, columns = head_dim
 // bf16; boxes of 64 columns x min(block_size, 64) rows, 128-byte swizzle.
+// fp8: rows of head_dim one-byte codes, whole-row boxes, no swizzle (the
+// consumer reads them linearly while widening them).
 bool encode_cache_map(CUtensorMap* map, const void* base, long long rows, int head_dim,
-                      int box_rows) {
+                      int box_rows, bool fp8) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint64_t gdim[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
-    cuuint64_t gstride[1] = {(cuuint64_t)head_dim * 2};
-    cuuint32_t box[2] = {64u, (cuuint32_t)box_rows};
+    cuuint64_t gstride[1] = {(cuuint64_t)head_dim * (fp8 ? 1 : 2)};
+    cuuint32_t box[2] = {fp8 ? (cuuint32_t)head_dim : 64u, (cuuint32_t)box_rows};
     cuuint32_t estride[2] = {1u, 1u};
-    const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), gdim,
-                           gstride, box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    const CUresult r = enc(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                           2, const_cast<void*>(base), gdim, gstride, box, estride,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           fp8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
-template <int D, int NT>
+template <int D, int NT, bool F8>
 pkv_status launch_impl(const DecodeParams& p, cudaStream_t stream, int* grid_out) {
-    using S = Smem<D, NT>;
+    using S = Smem<D, NT, F8>;
     const DeviceInfo* di = current_device_info();
     if (!di) return PKV_ERR_CUDA;
     static std::mutex mu;
     static int occupancy[64] = {0};
-    auto kern = decode_mma_kernel<D, NT>;
+    auto kern = decode_mma_kernel<D, NT, F8>;
     {
         std::lock_guard<std::mutex> lock(mu);
         if (di->device >= 64) return PKV_ERR_UNSUPPORTED;
@@ -814,8 +990,8 @@ pkv_status launch_impl(const DecodeParams& p, cudaStream_t stream, int* grid_out
     const long long rows = (long long)p.num_blocks * p.num_kv_heads * p.block_size;
     const int box_rows = std::min(p.block_size, kCH);
     CUtensorMap tmk, tmv;
-    if (!encode_cache_map(&tmk, p.k_cache, rows, D, box_rows) ||
-        !encode_cache_map(&tmv, p.v_cache, rows, D, box_rows))
+    if (!encode_cache_map(&tmk, p.k_cache, rows, D, box_rows, F8) ||
+        !encode_cache_map(&tmv, p.v_cache, rows, D, box_rows, F8))
         return PKV_ERR_CUDA;
     const int grid = di->num_sms * std::min(occupancy[di->device], 4);
 
@@ -828,17 +1004,24 @@ pkv_status launch_impl(const DecodeParams& p, cudaStream_t stream, int* grid_out
 }  // namespace
 
 bool decode_mma_supported(int head_dim, int block_size, pkv_dtype q_dtype, pkv_dtype kv_dtype) {
-    return q_dtype == PKV_BF16 && kv_dtype == PKV_BF16 && (head_dim == 64 || head_dim == 128) &&
-           block_size >= 8;
+    return q_dtype == PKV_BF16 && (kv_dtype == PKV_BF16 || kv_dtype == PKV_FP8_E4M3) &&
+           (head_dim == 64 || head_dim == 128) && block_size >= 8;
 }
 
-pkv_status launch_decode_mma(const DecodeParams& p, int head_dim, int group_pad,
+pkv_status launch_decode_mma(const DecodeParams& p, int head_dim, int group_pad, bool fp8,
                              cudaStream_t stream, int* grid_out) {
     const int nt = group_pad > 8 ? 2 : 1;
-    if (head_dim == 128) return nt == 1 ? launch_impl<128, 1>(p, stream, grid_out)
-                                        : launch_impl<128, 2>(p, stream, grid_out);
-    if (head_dim == 64) return nt == 1 ? launch_impl<64, 1>(p, stream, grid_out)
-                                       : launch_impl<64, 2>(p, stream, grid_out);
+    if (fp8) {
+        if (head_dim == 128) return nt == 1 ? launch_impl<128, 1, true>(p, stream, grid_out)
+                                            : launch_impl<128, 2, true>(p, stream, grid_out);
+        if (head_dim == 64) return nt == 1 ? launch_impl<64, 1, true>(p, stream, grid_out)
+                                           : launch_impl<64, 2, true>(p, stream, grid_out);
+    } else {
+        if (head_dim == 128) return nt == 1 ? launch_impl<128, 1, false>(p, stream, grid_out)
+                                            : launch_impl<128, 2, false>(p, stream, grid_out);
+        if (head_dim == 64) return nt == 1 ? launch_impl<64, 1, false>(p, stream, grid_out)
+                                           : launch_impl<64, 2, false>(p, stream, grid_out);
+    }
     return PKV_ERR_UNSUPPORTED;
 }
 

@@ -40,9 +40,15 @@ struct DecodePlan {
     size_t bytes;      // smallest workspace that fits
 };
 
-// Bytes at the start of a B-byte workspace reserved for arrival counters.
+// Bytes at the start of a B-byte workspace reserved for the merge's
+// synchronisation words: per-group arrival counters in its first half, one
+// ready flag per partial record in its second half.  Both return to zero at
+// the end of every call.
 inline size_t counter_region_bytes(size_t workspace_bytes) {
     return (workspace_bytes / 128 + 255) / 256 * 256;
+}
+inline size_t ready_flags_offset(size_t workspace_bytes) {
+    return counter_region_bytes(workspace_bytes) / 2;
 }
 
 // Fill a plan for these sizes on the current device (false if invalid).
@@ -63,6 +69,7 @@ struct DecodeParams {
     float* rec_ml;    // [records][group_pad][2]  (running max in log2 units, sum)
     int32_t* meta;    // [num_seqs * num_hg][2]   (first unit, number of units)
     unsigned* counters;  // [num_seqs * num_hg] arrivals per split group (zero between calls)
+    unsigned* ready;     // [records] 1 once a partial record is written (zero between calls)
     unsigned* err;
     int num_seqs, num_q_heads, num_kv_heads, group, num_sub, num_hg;
     int block_size, log2_bs, max_blocks, num_blocks;
@@ -77,7 +84,7 @@ pkv_status launch_decode_simt(const DecodeParams& p, int head_dim, pkv_dtype kv_
 
 bool decode_mma_supported(int head_dim, int block_size, pkv_dtype q_dtype, pkv_dtype kv_dtype);
 
-pkv_status launch_decode_mma(const DecodeParams& p, int head_dim, int group_pad,
+pkv_status launch_decode_mma(const DecodeParams& p, int head_dim, int group_pad, bool fp8,
                              cudaStream_t stream, int* grid_out);
 
 // Launch config with programmatic dependent launch: the kernel may start while
@@ -102,6 +109,17 @@ pkv_status launch_kv_cache_write(const void* k, const void* v, const int64_t* sl
                                  void* k_cache, void* v_cache, int num_tokens, int num_kv_heads,
                                  int head_dim, int block_size, int num_blocks, int elem_bytes,
                                  unsigned* err, cudaStream_t stream);
+
+pkv_status launch_kv_cache_write_fp8(const void* k, const void* v, const int64_t* slots,
+                                     void* k_cache, void* v_cache, const float* k_scale,
+                                     const float* v_scale, int num_tokens, int num_kv_heads,
+                                     int head_dim, int block_size, int num_blocks, unsigned* err,
+                                     cudaStream_t stream);
+
+pkv_status launch_swap_blocks(const void* src_k, const void* src_v, void* dst_k, void* dst_v,
+                              const int64_t* pairs, int num_pairs, size_t block_bytes,
+                              int src_blocks, int dst_blocks, unsigned* err,
+                              cudaStream_t stream);
 
 pkv_status launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs, int num_pairs,
                               size_t block_bytes, int num_blocks, unsigned* err,

@@ -79,7 +79,19 @@ class DevWorkload:
         self.v_new = to_dev(w.v_new, device)
         self.slot_mapping = to_dev(w.slot_mapping.astype(np.int64), device)
         self.copy_pairs = to_dev(w.copy_pairs.astype(np.int64), device)
+        self.k_scale = None if w.k_scale is None else to_dev(w.k_scale, device)
+        self.v_scale = None if w.v_scale is None else to_dev(w.v_scale, device)
         self.torch = torch
+
+
+def quantize_tokens(x_bits: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """Oracle e4m3 codes of bf16 tokens [T, Hkv, d] with one scale per kv head."""
+    import oracle
+    x = (x_bits.astype(np.uint32) << 16).view(np.float32)
+    out = np.zeros(x.shape, np.uint8)
+    for h in range(x.shape[1]):
+        out[:, h, :] = oracle.quantize_e4m3(np.ascontiguousarray(x[:, h, :]), float(scale[h]))
+    return out
 
 
 def host_step(w):
@@ -90,5 +102,8 @@ def host_step(w):
     if w.copy_pairs.shape[0]:
         assert oracle.copy_blocks(kc, vc, w.copy_pairs) == 0
     if w.slot_mapping.shape[0]:
-        assert oracle.kv_cache_write(w.k_new, w.v_new, w.slot_mapping, kc, vc) == 0
+        k, v = w.k_new, w.v_new
+        if w.dtype == "fp8":
+            k, v = quantize_tokens(k, w.k_scale), quantize_tokens(v, w.v_scale)
+        assert oracle.kv_cache_write(k, v, w.slot_mapping, kc, vc) == 0
     return kc, vc

@@ -40,6 +40,7 @@ from dataclasses import dataclass, field
 import numpy as np
 
 BF16_NAN = np.uint16(0x7FC0)
+E4M3_NAN = np.uint8(0x7F)
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -74,6 +75,8 @@ class Workload:
     slot_mapping: np.ndarray        # [T] int64
     copy_pairs: np.ndarray = field(default_factory=lambda: np.zeros((0, 2), np.int64))
     info: dict = field(default_factory=dict)
+    k_scale: np.ndarray | None = None  # [Hkv] fp32, fp8 caches only
+    v_scale: np.ndarray | None = None
 
     @property
     def max_blocks(self) -> int:
@@ -81,7 +84,7 @@ class Workload:
 
     @property
     def elem_bytes(self) -> int:
-        return 4 if self.dtype == "f32" else 2
+        return {"f32": 4, "bf16": 2, "fp8": 1}[self.dtype]
 
 
 def _normal(rng: np.random.Generator, shape, dtype: str) -> np.ndarray:
@@ -89,9 +92,25 @@ def _normal(rng: np.random.Generator, shape, dtype: str) -> np.ndarray:
     return x if dtype == "f32" else f32_to_bf16_bits(x)
 
 
+def e4m3_codes(rng: np.random.Generator, shape) -> np.ndarray:
+    """Random fp8 e4m3 codes (uint8): random sign, exponent field 0..10 (so
+    magnitudes up to 15, subnormals included), random mantissa; never NaN."""
+    sign = rng.integers(0, 2, size=shape, dtype=np.uint8) << 7
+    exp = rng.integers(0, 11, size=shape, dtype=np.uint8) << 3
+    man = rng.integers(0, 8, size=shape, dtype=np.uint8)
+    return (sign | exp | man).astype(np.uint8)
+
+
+def _cache_values(rng, shape, dtype: str) -> np.ndarray:
+    """Stored cache contents: values for fp32/bf16 caches, codes for fp8."""
+    return e4m3_codes(rng, shape) if dtype == "fp8" else _normal(rng, shape, dtype)
+
+
 def _empty_cache(shape, dtype: str, poison: bool) -> np.ndarray:
     if dtype == "f32":
         return np.full(shape, np.nan if poison else 0.0, dtype=np.float32)
+    if dtype == "fp8":
+        return np.full(shape, E4M3_NAN if poison else 0, dtype=np.uint8)
     return np.full(shape, BF16_NAN if poison else 0, dtype=np.uint16)
 
 
@@ -100,8 +119,8 @@ def _fill_history(rng, k_cache, v_cache, table_row, n_tokens, bs, dtype):
     Hkv, d = k_cache.shape[1], k_cache.shape[3]
     if n_tokens <= 0:
         return
-    kh = _normal(rng, (n_tokens, Hkv, d), dtype)
-    vh = _normal(rng, (n_tokens, Hkv, d), dtype)
+    kh = _cache_values(rng, (n_tokens, Hkv, d), dtype)
+    vh = _cache_values(rng, (n_tokens, Hkv, d), dtype)
     nfull = n_tokens // bs
     if nfull:
         blocks = np.asarray(table_row[:nfull], dtype=np.int64)
@@ -126,6 +145,8 @@ def make_paged(seq_lens, *, Hq: int, Hkv: int, d: int, bs: int, dtype: str, seed
     rng = np.random.default_rng(seed)
     seq_lens = np.asarray(seq_lens, dtype=np.int32)
     B = int(seq_lens.shape[0])
+    # fp8 caches: q and the appended tokens are bf16, the cache holds e4m3 codes
+    qdt = "bf16" if dtype == "fp8" else dtype
     nblk = [-(-int(L) // bs) for L in seq_lens]
     need = int(sum(nblk))
     NB = max(int(math.ceil(need * pool_factor)) + int(extra_blocks), 1)
@@ -136,7 +157,7 @@ def make_paged(seq_lens, *, Hq: int, Hkv: int, d: int, bs: int, dtype: str, seed
     for b in range(B):
         tables[b, : nblk[b]] = pool[pos: pos + nblk[b]]
         pos += nblk[b]
-    q = _normal(rng, (B, Hq, d), dtype)
+    q = _normal(rng, (B, Hq, d), qdt)
     k_cache = _empty_cache((NB, Hkv, bs, d), dtype, poison)
     v_cache = _empty_cache((NB, Hkv, bs, d), dtype, poison)
     hist = [int(L) - 1 if (append_last and L > 0) else int(L) for L in seq_lens]
@@ -144,19 +165,23 @@ def make_paged(seq_lens, *, Hq: int, Hkv: int, d: int, bs: int, dtype: str, seed
         _fill_history(rng, k_cache, v_cache, tables[b], hist[b], bs, dtype)
     new_rows = [b for b in range(B) if append_last and seq_lens[b] > 0]
     T = len(new_rows)
-    k_new = _normal(rng, (T, Hkv, d), dtype)
-    v_new = _normal(rng, (T, Hkv, d), dtype)
+    k_new = _normal(rng, (T, Hkv, d), qdt)
+    v_new = _normal(rng, (T, Hkv, d), qdt)
     slots = np.zeros(T, dtype=np.int64)
     for i, b in enumerate(new_rows):
         t = int(seq_lens[b]) - 1
         slots[i] = int(tables[b, t // bs]) * bs + t % bs
     if scale is None:
         scale = 1.0 / math.sqrt(d)
+    ks = vs = None
+    if dtype == "fp8":  # per-kv-head dequantisation scales
+        ks = rng.uniform(0.05, 0.5, size=Hkv).astype(np.float32)
+        vs = rng.uniform(0.05, 0.5, size=Hkv).astype(np.float32)
     return Workload(name=name, B=B, Hq=Hq, Hkv=Hkv, d=d, bs=bs, num_blocks=NB,
                     dtype=dtype, scale=float(scale), q=q, k_cache=k_cache,
                     v_cache=v_cache, block_tables=tables, seq_lens=seq_lens,
                     k_new=k_new, v_new=v_new, slot_mapping=slots,
-                    info={"seed": seed, "blocks_used": need})
+                    info={"seed": seed, "blocks_used": need}, k_scale=ks, v_scale=vs)
 
 
 def tiny_f32(poison: bool = True, seed: int = 1001) -> Workload:
@@ -246,10 +271,19 @@ def long_ctx(bs: int = 16, poison: bool = True, seed: int = 1005, batch: int = 2
                       seed=seed + bs, poison=poison, name=f"long_ctx_bs{bs}")
 
 
+def gqa_4k_fp8(poison: bool = True, seed: int = 1006, batch: int = 16,
+               seq_len: int = 4096) -> Workload:
+    """The 4k-token decode workload with an fp8 (e4m3) cache: random codes with
+    per-kv-head scales; q and appended tokens bf16."""
+    return make_paged([seq_len] * batch, Hq=32, Hkv=8, d=128, bs=16, dtype="fp8",
+                      seed=seed, poison=poison, name="gqa_4k_fp8")
+
+
 WORKLOADS = {
     "tiny_f32": tiny_f32,
     "gqa_4k": gqa_4k,
     "mixed": mixed,
     "prefix": prefix_shared,
     "long_ctx": long_ctx,
+    "gqa_4k_fp8": gqa_4k_fp8,
 }
