@@ -488,6 +488,188 @@ def run_ours(args, rank: int, world: int, local: int):
     return result
 
 
+# ---------------------------------------------------------------------------
+# --suite: one JSON line per workload of the scope table (not the headline)
+# ---------------------------------------------------------------------------
+
+class _L2Flush:
+    """Writes a buffer twice the size of L2 between timed launches."""
+
+    def __init__(self, dev):
+        import torch
+        self.buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def __call__(self):
+        self.buf.zero_()
+
+
+def _time_graph(fn, iters, flush, warm=5):
+    """Mean / median device time (ms) of ``fn`` captured in a CUDA graph, L2
+    flushed before each launch, CUDA events around each launch."""
+    import torch
+    for _ in range(2):
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    for _ in range(warm):
+        flush()
+        g.replay()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(iters)]
+    for a, b in ev:
+        flush()
+        a.record()
+        g.replay()
+        b.record()
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in ev]
+    del g
+    return statistics.fmean(ms), statistics.median(ms)
+
+
+def _dev_workload(w, dev):
+    import torch
+
+    def t(a):
+        a = np.ascontiguousarray(a)
+        if a.dtype == np.uint16:
+            return torch.from_numpy(a.view(np.int16)).to(dev).view(torch.bfloat16)
+        return torch.from_numpy(a).to(dev)
+    d = {"q": t(w.q), "kc": t(w.k_cache), "vc": t(w.v_cache), "bt": t(w.block_tables),
+         "sl": t(w.seq_lens), "kn": t(w.k_new), "vn": t(w.v_new),
+         "sm": t(w.slot_mapping.astype(np.int64)),
+         "pairs": t(w.copy_pairs.astype(np.int64).reshape(-1, 2))}
+    d["ks"] = None if w.k_scale is None else t(w.k_scale)
+    d["vs"] = None if w.v_scale is None else t(w.v_scale)
+    return d
+
+
+def run_suite(args):
+    import torch
+    import paged_kv_cache_412_b200 as pkv
+    import workloads
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    peak, peak_kind = measured_peak()
+    flush = _L2Flush(dev)
+    iters = max(20, min(args.steps, 500))
+
+    def emit(name, ms, nbytes, extra):
+        mean, med = ms
+        gbs = nbytes / (mean / 1e3) / 1e9
+        line = {"suite": name, "unit": "GB/s", "value": round(gbs, 2),
+                "frac_of_hbm_peak": round(gbs / peak, 4), "peak": peak,
+                "peak_kind": f"{peak_kind} HBM copy bandwidth", "us_mean": round(mean * 1e3, 2),
+                "us_median": round(med * 1e3, 2), "bytes": int(nbytes), "launches_timed": iters,
+                "l2": "flushed (256 MB write) before every timed launch"}
+        line.update(extra)
+        print(json.dumps(line), flush=True)
+
+    def decode_case(name, w, partition_size=0, extra=None, fp8=False):
+        t = _dev_workload(w, dev)
+        L = int(w.seq_lens.max())
+        out = torch.empty((w.B, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+        ws = pkv.new_workspace(pkv.decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.d, w.bs, L,
+                                                          partition_size), dev)
+
+        def fn():
+            pkv.paged_attention_decode(t["q"], t["kc"], t["vc"], t["bt"], t["sl"], w.bs,
+                                       w.scale, out, max_seq_len=L, workspace=ws,
+                                       partition_size=partition_size, k_scale=t["ks"],
+                                       v_scale=t["vs"])
+        ms = _time_graph(fn, iters, flush)
+        assert pkv.get_device_error() == 0
+        e_kv = 1 if fp8 else 2
+        nbytes = (2 * int(w.seq_lens.astype(np.int64).sum()) * w.Hkv * w.d * e_kv
+                  + w.B * w.Hq * w.d * 4)
+        info = {"B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "block_size": w.bs,
+                "kv_dtype": "fp8_e4m3" if fp8 else "bf16", "partition_size": partition_size,
+                "context_tokens": int(w.seq_lens.astype(np.int64).sum())}
+        info.update(extra or {})
+        emit(name, ms, nbytes, info)
+        del t, ws, out
+        torch.cuda.empty_cache()
+
+    # the 4k workload: permuted pool (as benched) and identity tables (the
+    # indirection's cost is the difference)
+    decode_case("decode gqa_4k permuted pool", workloads.gqa_4k(poison=False))
+    w = workloads.make_paged([4096] * 16, Hq=32, Hkv=8, d=128, bs=16, dtype="bf16",
+                             seed=1002, poison=False, permute=False, name="gqa_4k_identity")
+    decode_case("decode gqa_4k identity tables", w)
+    decode_case("decode gqa_4k fp8 e4m3 cache", workloads.gqa_4k_fp8(poison=False), fp8=True)
+    decode_case("decode mixed (256 requests, log-uniform 16..8192)", workloads.mixed(poison=False))
+    for bs in (8, 16, 32):
+        wl = workloads.long_ctx(bs=bs, poison=False)
+        for P in (0, 512, 1024, 2048, 4096):
+            decode_case(f"decode long_ctx 2 x 131072 bs {bs} partition {P or 'auto'}", wl,
+                        partition_size=P)
+        del wl
+
+    # shared prefix: the step (fork copy + suffix append + decode)
+    w = workloads.prefix_shared(poison=False)
+    t = _dev_workload(w, dev)
+    L = int(w.seq_lens.max())
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
+    ws = pkv.new_workspace(pkv.decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.d, w.bs, L, 0), dev)
+    kc0, vc0 = t["kc"].clone(), t["vc"].clone()
+
+    def prefix_step():
+        pkv.copy_blocks(t["kc"], t["vc"], t["pairs"])
+        pkv.kv_cache_write(t["kn"], t["vn"], t["sm"], t["kc"], t["vc"])
+        pkv.paged_attention_decode(t["q"], t["kc"], t["vc"], t["bt"], t["sl"], w.bs, w.scale,
+                                   out, max_seq_len=L, workspace=ws)
+    ms = _time_graph(prefix_step, iters, flush)
+    logical = 2 * int(w.seq_lens.astype(np.int64).sum()) * w.Hkv * w.d * 2 + w.B * w.Hq * w.d * 4
+    unique_tok = w.info["prefix_tokens"] + sum(w.info["suffix"])
+    unique = 2 * unique_tok * w.Hkv * w.d * 2 + w.B * w.Hq * w.d * 4
+    emit("step prefix (64 requests sharing a 2040-token prefix)", ms, logical,
+         {"bytes_kind": "logical (prefix counted once per request)", "unique_bytes": unique,
+          "unique_GBps": round(unique / (ms[0] / 1e3) / 1e9, 2),
+          "step": "copy_blocks (64 forks) + kv_cache_write (suffixes) + decode"})
+    del t, ws, out, kc0, vc0
+    torch.cuda.empty_cache()
+
+    # cache operations alone
+    w = workloads.gqa_4k(poison=False)
+    t = _dev_workload(w, dev)
+    NB = w.num_blocks
+    blk_bytes = 2 * w.Hkv * w.bs * w.d * 2  # K + V of one block
+    T = 16384
+    rng = np.random.default_rng(7)
+    slots = torch.from_numpy(rng.permutation(NB * w.bs)[:T].astype(np.int64)).to(dev)
+    kn = torch.randn((T, w.Hkv, w.d), device=dev).to(torch.bfloat16)
+    vn = torch.randn((T, w.Hkv, w.d), device=dev).to(torch.bfloat16)
+    ms = _time_graph(lambda: pkv.kv_cache_write(kn, vn, slots, t["kc"], t["vc"]), iters, flush)
+    emit("kv_cache_write 16384 scattered tokens", ms, 2 * 2 * T * w.Hkv * w.d * 2,
+         {"bytes_kind": "read new K,V + write cache rows"})
+    ms = _time_graph(lambda: pkv.kv_cache_write(t["kn"], t["vn"], t["sm"], t["kc"], t["vc"]),
+                     iters, flush)
+    emit("kv_cache_write 16 tokens (one decode step)", ms, 2 * 2 * 16 * w.Hkv * w.d * 2,
+         {"bytes_kind": "read new K,V + write cache rows", "note": "launch-latency bound"})
+    perm = rng.permutation(NB)
+    pairs = torch.from_numpy(np.stack([perm[:1024], perm[1024:2048]], 1).astype(np.int64)).to(dev)
+    ms = _time_graph(lambda: pkv.copy_blocks(t["kc"], t["vc"], pairs), iters, flush)
+    emit("copy_blocks 1024 pairs", ms, 2 * 1024 * blk_bytes,
+         {"bytes_kind": "read + write K and V of each pair"})
+    nsw = 1024
+    hk = torch.empty((nsw, w.Hkv, w.bs, w.d), dtype=torch.bfloat16).pin_memory()
+    hv = torch.empty_like(hk).pin_memory()
+    out_pairs = torch.from_numpy(np.stack([perm[:nsw], np.arange(nsw)], 1).astype(np.int64)).to(dev)
+    in_pairs = torch.from_numpy(np.stack([np.arange(nsw), perm[2048:2048 + nsw]], 1)
+                                .astype(np.int64)).to(dev)
+    ms = _time_graph(lambda: pkv.swap_blocks(t["kc"], t["vc"], hk, hv, out_pairs), iters, flush)
+    emit("swap_blocks device -> pinned host, 1024 blocks", ms, nsw * blk_bytes,
+         {"bytes_kind": "K and V bytes moved", "note": "host link bound, not HBM"})
+    ms = _time_graph(lambda: pkv.swap_blocks(hk, hv, t["kc"], t["vc"], in_pairs), iters, flush)
+    emit("swap_blocks pinned host -> device, 1024 blocks", ms, nsw * blk_bytes,
+         {"bytes_kind": "K and V bytes moved", "note": "host link bound, not HBM"})
+    assert pkv.get_device_error() == 0
+
+
 def spot_check(pkv, t, out, ws, scale):
     """Compare a few outputs of the timed configuration with the oracle."""
     import torch
@@ -514,6 +696,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-check", action="store_true")
+    ap.add_argument("--suite", action="store_true",
+                    help="one line per workload of the scope table instead of the headline")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -522,6 +706,9 @@ def main():
         # and leave without joining a process group.
         if int(os.environ.get("RANK", "0")) == 0:
             run_reference(args, 0, int(os.environ.get("WORLD_SIZE", "1")))
+        return
+    if args.suite:
+        run_suite(args)
         return
     rank, world, local = dist_setup(args.gpus)
     try:
