@@ -6,7 +6,9 @@
  *   - pkv_paged_attention_decode  single-query decode attention over a cache
  *                                 held in fixed-size physical blocks reached
  *                                 through a per-request block table;
- *   - pkv_copy_blocks             copy-on-write copy of shared blocks.
+ *   - pkv_copy_blocks             copy-on-write copy of shared blocks;
+ *   - pkv_paged_attention_decode_prefix  the same decode with the blocks a
+ *                                 group of requests shares read once per group.
  *
  * Sources (web pages on the subject; cited by title and section):
  *   [KVOPT]  "KV Cache Optimization and PagedAttention" (intro prose).
@@ -71,6 +73,7 @@ typedef enum pkv_dtype {
 #define PKV_DEVERR_BAD_SEQ_LEN 0x4u    /* decode: seq_len < 0 or > max_blocks*bs    */
 #define PKV_DEVERR_BAD_PAIR 0x8u       /* copy/swap: block id out of range          */
 #define PKV_DEVERR_TIMEOUT 0x10u       /* a bounded in-kernel wait gave up          */
+#define PKV_DEVERR_PREFIX 0x20u        /* prefix decode: bad group id, length or size */
 
 /* Human-readable name of a status code (static string). */
 const char* pkv_status_string(pkv_status status);
@@ -196,6 +199,66 @@ pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache,
                                       const float* v_scale, int32_t partition_size,
                                       void* workspace, size_t workspace_bytes,
                                       pkv_stream_t stream);
+
+/*
+ * pkv_decode_prefix_workspace_bytes -- workspace bytes of
+ * pkv_paged_attention_decode_prefix for these sizes on the CURRENT device:
+ * the decode's own scratch plus one partial result per (split of the shared
+ * pass, request, query head).  max_prefix_members bounds the requests of any
+ * one group; max_prefix_len bounds every prefix_lens entry.  0 if invalid.
+ */
+size_t pkv_decode_prefix_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
+                                         int32_t num_kv_heads, int32_t head_dim,
+                                         int32_t block_size, int32_t max_seq_len,
+                                         int32_t num_prefixes, int32_t max_prefix_members,
+                                         int32_t max_prefix_len);
+
+/*
+ * pkv_paged_attention_decode_prefix -- pkv_paged_attention_decode for a batch
+ * in which groups of requests share the physical blocks of a common prefix.
+ *
+ * [KVMGMT] "The Bonus: Zero-Copy Sharing" and [KVOPT]: requests forked from
+ * one prompt point their block tables at the same physical blocks, stored
+ * once.  This call also READS them once per group: a shared pass streams the
+ * group's prefix blocks a single time for all of the group's query heads (a
+ * dense contraction over the group's q rows), leaving one partial softmax
+ * state per (request, query head); each request's own pass then covers only
+ * the tokens after the prefix and merges the two states.  The result is the
+ * same attention as pkv_paged_attention_decode over the full tables (up to
+ * fp32 rounding order); nothing about the output depends on the grouping.
+ *
+ *   prefix_of     [num_seqs] int32: the group of request b, or -1 for none.
+ *   prefix_lens   [num_prefixes] int32: tokens of group g's prefix, a multiple
+ *                 of block_size, <= max_prefix_len.  Contract: for every
+ *                 member b, block_tables[b][j] is the same physical block for
+ *                 all j < prefix_lens[g] / block_size (the shared blocks of a
+ *                 fork; the partly filled block a fork copies is not part of
+ *                 it).  A member shorter than the prefix attends to its own
+ *                 seq_lens[b] tokens only.  The shared pass reads the table of
+ *                 the group's longest member.
+ *   num_prefixes, max_prefix_members, max_prefix_len  as for
+ *                 pkv_decode_prefix_workspace_bytes; the workspace must be at
+ *                 least that size.
+ *   Other arguments as pkv_paged_attention_decode (partition_size automatic).
+ *   Supported: q and caches PKV_BF16, head_dim 64 or 128, block_size >= 8;
+ *   other configurations return PKV_ERR_UNSUPPORTED.
+ *   Ordering: two kernels on `stream`, the shared pass first; both read
+ *   seq_lens, block_tables, prefix_of and prefix_lens before waiting for the
+ *   previous kernel, with the same rule as pkv_paged_attention_decode.
+ *   Device checks: a group id >= num_prefixes, a prefix length that is not a
+ *   multiple of block_size or exceeds max_prefix_len (it is clamped and
+ *   rounded down), and a group with more than max_prefix_members requests
+ *   raise PKV_DEVERR_PREFIX; the outputs of members past that bound are
+ *   undefined.
+ */
+pkv_status pkv_paged_attention_decode_prefix(
+    const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+    const int32_t* seq_lens, int32_t block_size, float scale, void* out, int32_t num_seqs,
+    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t max_blocks_per_seq,
+    int32_t num_blocks, int32_t max_seq_len, pkv_dtype q_dtype, pkv_dtype kv_dtype,
+    pkv_dtype out_dtype, const int32_t* prefix_of, const int32_t* prefix_lens,
+    int32_t num_prefixes, int32_t max_prefix_members, int32_t max_prefix_len, void* workspace,
+    size_t workspace_bytes, pkv_stream_t stream);
 
 /*
  * pkv_paged_attention_decode_noalloc -- pkv_paged_attention_decode for callers

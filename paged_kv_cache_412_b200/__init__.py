@@ -38,7 +38,7 @@ PKV_OK = 0
 STATUS_NAMES = {0: "PKV_OK", 1: "PKV_ERR_INVALID_ARG", 2: "PKV_ERR_UNSUPPORTED",
                 3: "PKV_ERR_WORKSPACE", 4: "PKV_ERR_CUDA", 5: "PKV_ERR_DEVICE_INDEX"}
 DEVERR = {"BAD_SLOT": 0x1, "BAD_BLOCK": 0x2, "BAD_SEQ_LEN": 0x4, "BAD_PAIR": 0x8,
-          "TIMEOUT": 0x10}
+          "TIMEOUT": 0x10, "PREFIX": 0x20}
 
 _F32, _BF16, _FP8 = 0, 1, 2
 
@@ -71,6 +71,13 @@ def _load() -> ctypes.CDLL:
                                              i32, i32, i32, i32, ctypes.c_int, ctypes.c_int,
                                              ctypes.c_int, vp, vp, i32, vp, sz, vp]
     L.pkv_paged_attention_decode.restype = ctypes.c_int
+    L.pkv_decode_prefix_workspace_bytes.argtypes = [i32] * 9
+    L.pkv_decode_prefix_workspace_bytes.restype = sz
+    L.pkv_paged_attention_decode_prefix.argtypes = [vp, vp, vp, vp, vp, i32, f32, vp, i32, i32,
+                                                    i32, i32, i32, i32, i32, ctypes.c_int,
+                                                    ctypes.c_int, ctypes.c_int, vp, vp, i32, i32,
+                                                    i32, vp, sz, vp]
+    L.pkv_paged_attention_decode_prefix.restype = ctypes.c_int
     L.pkv_copy_blocks.argtypes = [vp, vp, vp, i32, i32, i32, i32, i32, ctypes.c_int, vp]
     L.pkv_copy_blocks.restype = ctypes.c_int
     L.pkv_get_device_error.argtypes = [vp, ctypes.POINTER(ctypes.c_uint32)]
@@ -231,6 +238,75 @@ def paged_attention_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torc
             _ptr(v_scale), int(partition_size), _ptr(ws), ws.numel() * ws.element_size(),
             _stream(dev))
     _check("pkv_paged_attention_decode", st)
+    return out
+
+
+def decode_prefix_workspace_bytes(num_seqs: int, num_q_heads: int, num_kv_heads: int,
+                                  head_dim: int, block_size: int, max_seq_len: int,
+                                  num_prefixes: int, max_prefix_members: int,
+                                  max_prefix_len: int) -> int:
+    return int(_get_lib().pkv_decode_prefix_workspace_bytes(
+        num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len, num_prefixes,
+        max_prefix_members, max_prefix_len))
+
+
+def paged_attention_decode_prefix(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor,
+                                  block_tables: torch.Tensor, seq_lens: torch.Tensor,
+                                  prefix_of: torch.Tensor, prefix_lens: torch.Tensor,
+                                  block_size: int | None = None, scale: float | None = None,
+                                  out: torch.Tensor | None = None, *,
+                                  max_seq_len: int | None = None,
+                                  max_prefix_members: int | None = None,
+                                  max_prefix_len: int | None = None,
+                                  out_dtype: torch.dtype | None = None,
+                                  workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """paged_attention_decode for requests that share prefix blocks.
+
+    prefix_of [B] int32: the group of each request (-1: none); prefix_lens [G]
+    int32: tokens of each group's shared prefix (a multiple of block_size).
+    The group's shared blocks are read once for all its members, then each
+    request's own tokens; the result equals paged_attention_decode.
+    ``max_prefix_members`` defaults to B and ``max_prefix_len`` to max_seq_len.
+    """
+    dev = _need_cuda(q, k_cache, v_cache, block_tables, seq_lens, prefix_of, prefix_lens, out,
+                     workspace)
+    for name, t in (("block_tables", block_tables), ("seq_lens", seq_lens),
+                    ("prefix_of", prefix_of), ("prefix_lens", prefix_lens)):
+        if t.dtype != torch.int32:
+            raise TypeError(f"{name} must be int32")
+    B, Hq, d = q.shape
+    NB, Hkv, bs, d2 = k_cache.shape
+    if block_size is None:
+        block_size = bs
+    if block_size != bs or d2 != d or v_cache.shape != k_cache.shape:
+        raise ValueError("shape mismatch")
+    if prefix_of.numel() != B:
+        raise ValueError("prefix_of must hold one entry per request")
+    if scale is None:
+        scale = d ** -0.5
+    max_blocks = block_tables.shape[1]
+    if max_seq_len is None:
+        max_seq_len = max_blocks * bs
+    if max_prefix_members is None:
+        max_prefix_members = max(B, 1)
+    if max_prefix_len is None:
+        max_prefix_len = max_seq_len
+    G = prefix_lens.numel()
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=out_dtype or q.dtype, device=dev)
+    need = decode_prefix_workspace_bytes(B, Hq, Hkv, d, bs, max_seq_len, G, max_prefix_members,
+                                         max_prefix_len)
+    if need == 0:
+        raise PkvError("pkv_decode_prefix_workspace_bytes", 1)
+    with torch.cuda.device(dev):
+        ws = workspace if workspace is not None else _workspace(dev, need)
+        st = _get_lib().pkv_paged_attention_decode_prefix(
+            _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(seq_lens), bs,
+            float(scale), _ptr(out), B, Hq, Hkv, d, max_blocks, NB, int(max_seq_len),
+            _dtype_code(q), _dtype_code(k_cache), _dtype_code(out), _ptr(prefix_of),
+            _ptr(prefix_lens), G, int(max_prefix_members), int(max_prefix_len), _ptr(ws),
+            ws.numel() * ws.element_size(), _stream(dev))
+    _check("pkv_paged_attention_decode_prefix", st)
     return out
 
 

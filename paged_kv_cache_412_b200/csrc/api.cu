@@ -39,6 +39,30 @@ int elem_size(pkv_dtype t) {
     }
 }
 
+// Splits of the shared prefix pass: enough (group, kv head, row tile, split)
+// CTAs for about two per SM, at most one per 64-token chunk of the longest
+// prefix.
+int prefix_splits_for(int num_sms, int num_prefixes, int num_kv_heads, int row_tiles,
+                      int max_prefix_len) {
+    const long long base = (long long)num_prefixes * num_kv_heads * row_tiles;
+    const long long nch = (max_prefix_len + 63) / 64;
+    if (base <= 0 || nch <= 0) return 1;
+    long long s = (2LL * num_sms + base - 1) / base;
+    s = std::min(s, nch);
+    s = std::min(s, 64LL);
+    return (int)std::max(s, 1LL);
+}
+
+int prefix_row_tiles(int max_members, int group) {
+    return (int)(((long long)max_members * group + kPrefixRows - 1) / kPrefixRows);
+}
+
+size_t prefix_record_bytes(int splits, int num_seqs, int num_q_heads, int head_dim) {
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    const size_t rows = (size_t)splits * num_seqs * num_q_heads;
+    return up(rows * head_dim * sizeof(float)) + up(rows * 2 * sizeof(float));
+}
+
 int group_pad_of(int group) {
     if (group >= 8) return 8;
     int g = 1;
@@ -71,7 +95,8 @@ const DeviceInfo* current_device_info() {
 }
 
 bool make_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
-                      int block_size, int max_seq_len, int partition_size, DecodePlan* plan) {
+                      int block_size, int max_seq_len, int partition_size, DecodePlan* plan,
+                      size_t extra_bytes) {
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
         block_size <= 0 || max_seq_len < 0 || partition_size < 0)
         return false;
@@ -101,7 +126,8 @@ bool make_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_
     const size_t meta_bytes = pl.n_bg_max * 2 * sizeof(int32_t);
     pl.off_ml = up(acc_bytes);
     pl.off_meta = pl.off_ml + up(ml_bytes);
-    pl.rec_bytes = pl.off_meta + up(meta_bytes);
+    pl.off_extra = pl.off_meta + up(meta_bytes);
+    pl.rec_bytes = pl.off_extra + up(extra_bytes);
     // smallest B with counter region(B) + records <= B and room for every counter
     const size_t sync_words = std::max(pl.n_bg_max, pl.records);
     size_t b = up(pl.rec_bytes + 2 * sync_words * sizeof(uint32_t));
@@ -198,16 +224,26 @@ pkv_status pkv_decode_workspace_init(void* workspace, size_t workspace_bytes,
                : PKV_ERR_CUDA;
 }
 
-pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const void* v_cache,
-                                      const int32_t* block_tables, const int32_t* seq_lens,
-                                      int32_t block_size, float scale, void* out,
-                                      int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
-                                      int32_t head_dim, int32_t max_blocks_per_seq,
-                                      int32_t num_blocks, int32_t max_seq_len, pkv_dtype q_dtype,
-                                      pkv_dtype kv_dtype, pkv_dtype out_dtype,
-                                      const float* k_scale, const float* v_scale,
-                                      int32_t partition_size, void* workspace,
-                                      size_t workspace_bytes, pkv_stream_t stream) {
+}  // extern "C"
+
+namespace pkv {
+namespace {
+
+// Shared-prefix arguments of pkv_paged_attention_decode_prefix.
+struct PrefixArgs {
+    const int32_t* prefix_of;
+    const int32_t* prefix_lens;
+    int num_prefixes, max_members, max_prefix_len;
+};
+
+pkv_status decode_entry(const void* q, const void* k_cache, const void* v_cache,
+                        const int32_t* block_tables, const int32_t* seq_lens, int32_t block_size,
+                        float scale, void* out, int32_t num_seqs, int32_t num_q_heads,
+                        int32_t num_kv_heads, int32_t head_dim, int32_t max_blocks_per_seq,
+                        int32_t num_blocks, int32_t max_seq_len, pkv_dtype q_dtype,
+                        pkv_dtype kv_dtype, pkv_dtype out_dtype, const float* k_scale,
+                        const float* v_scale, int32_t partition_size, void* workspace,
+                        size_t workspace_bytes, pkv_stream_t stream, const PrefixArgs* pa) {
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
         max_blocks_per_seq <= 0 || num_blocks <= 0 || max_seq_len < 0 || partition_size < 0)
         return PKV_ERR_INVALID_ARG;
@@ -232,9 +268,31 @@ pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const 
     if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
         !aligned(block_tables, 4) || !aligned(seq_lens, 4) || !aligned(out, elem_size(out_dtype)))
         return PKV_ERR_INVALID_ARG;
+    const DeviceInfo* di0 = current_device_info();
+    if (!di0) return PKV_ERR_CUDA;
+    const bool use_prefix = pa && pa->num_prefixes > 0;
+    int pfx_splits = 0, pfx_tiles = 0;
+    size_t pfx_bytes = 0;
+    if (pa) {
+        if (pa->num_prefixes < 0 || pa->max_members < 1 || pa->max_prefix_len < 0)
+            return PKV_ERR_INVALID_ARG;
+        if (partition_size != 0) return PKV_ERR_INVALID_ARG;
+        if (use_prefix) {
+            if (!pa->prefix_of || !pa->prefix_lens || !aligned(pa->prefix_of, 4) ||
+                !aligned(pa->prefix_lens, 4))
+                return PKV_ERR_INVALID_ARG;
+            if (!(q_dtype == PKV_BF16 && kv_dtype == PKV_BF16) ||
+                !decode_mma_supported(head_dim, block_size, q_dtype, kv_dtype))
+                return PKV_ERR_UNSUPPORTED;
+            pfx_tiles = prefix_row_tiles(pa->max_members, num_q_heads / num_kv_heads);
+            pfx_splits = prefix_splits_for(di0->num_sms, pa->num_prefixes, num_kv_heads,
+                                           pfx_tiles, pa->max_prefix_len);
+            pfx_bytes = prefix_record_bytes(pfx_splits, num_seqs, num_q_heads, head_dim);
+        }
+    }
     DecodePlan pl;
     if (!make_decode_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len,
-                          partition_size, &pl))
+                          partition_size, &pl, pfx_bytes))
         return PKV_ERR_CUDA;
     if (!workspace || workspace_bytes < pl.bytes || !aligned(workspace, 256))
         return PKV_ERR_WORKSPACE;
@@ -281,13 +339,116 @@ pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const 
     p.max_blocks = max_blocks_per_seq;
     p.num_blocks = num_blocks;
     p.fixed_units = partition_size > 0 ? std::max(1, partition_size / (mma ? 64 : 32)) : 0;
+    // Fixed partitions on the tensor-core path: merge in a separate kernel, so
+    // a group split into many parts is combined in parallel instead of by its
+    // last part alone (which would stall that part's CTA).
+    p.defer_merge = (mma && partition_size > 0) ? 1 : 0;
     p.rec_cap = (long long)pl.records;
     p.out_dtype = out_dtype;
     p.scale_log2 = scale * 1.4426950408889634f;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (use_prefix) {
+        const size_t rows = (size_t)pfx_splits * num_seqs * num_q_heads;
+        unsigned char* pfx = ws + cnt_region + pl.off_extra;
+        float* pfx_acc = reinterpret_cast<float*>(pfx);
+        float* pfx_ml = reinterpret_cast<float*>(pfx + (rows * head_dim * sizeof(float) + 255) /
+                                                           256 * 256);
+        p.prefix_of = pa->prefix_of;
+        p.prefix_lens = pa->prefix_lens;
+        p.num_prefixes = pa->num_prefixes;
+        p.max_prefix_len = pa->max_prefix_len;
+        p.pfx_acc = pfx_acc;
+        p.pfx_ml = pfx_ml;
+        p.pfx_splits = pfx_splits;
+        PrefixParams pp{};
+        pp.q = q;
+        pp.block_tables = block_tables;
+        pp.seq_lens = seq_lens;
+        pp.prefix_of = pa->prefix_of;
+        pp.prefix_lens = pa->prefix_lens;
+        pp.pfx_acc = pfx_acc;
+        pp.pfx_ml = pfx_ml;
+        pp.err = di->error_word;
+        pp.num_seqs = num_seqs;
+        pp.num_q_heads = num_q_heads;
+        pp.num_kv_heads = num_kv_heads;
+        pp.group = group;
+        pp.block_size = block_size;
+        pp.log2_bs = p.log2_bs;
+        pp.max_blocks = max_blocks_per_seq;
+        pp.num_blocks = num_blocks;
+        pp.num_prefixes = pa->num_prefixes;
+        pp.max_members = pa->max_members;
+        pp.max_prefix_len = pa->max_prefix_len;
+        pp.splits = pfx_splits;
+        pp.row_tiles = pfx_tiles;
+        pp.scale_log2 = p.scale_log2;
+        const pkv_status ps = launch_decode_prefix(pp, k_cache, v_cache, head_dim, st);
+        if (ps != PKV_OK) return ps;
+    }
     if (mma)
         return launch_decode_mma(p, head_dim, group_pad, kv_dtype == PKV_FP8_E4M3, st, nullptr);
     return launch_decode_simt(p, head_dim, kv_dtype, group_pad, st, nullptr);
+}
+
+}  // namespace
+}  // namespace pkv
+
+extern "C" {
+
+pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const void* v_cache,
+                                      const int32_t* block_tables, const int32_t* seq_lens,
+                                      int32_t block_size, float scale, void* out,
+                                      int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads,
+                                      int32_t head_dim, int32_t max_blocks_per_seq,
+                                      int32_t num_blocks, int32_t max_seq_len, pkv_dtype q_dtype,
+                                      pkv_dtype kv_dtype, pkv_dtype out_dtype,
+                                      const float* k_scale, const float* v_scale,
+                                      int32_t partition_size, void* workspace,
+                                      size_t workspace_bytes, pkv_stream_t stream) {
+    return decode_entry(q, k_cache, v_cache, block_tables, seq_lens, block_size, scale, out,
+                        num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                        num_blocks, max_seq_len, q_dtype, kv_dtype, out_dtype, k_scale, v_scale,
+                        partition_size, workspace, workspace_bytes, stream, nullptr);
+}
+
+size_t pkv_decode_prefix_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
+                                         int32_t num_kv_heads, int32_t head_dim,
+                                         int32_t block_size, int32_t max_seq_len,
+                                         int32_t num_prefixes, int32_t max_prefix_members,
+                                         int32_t max_prefix_len) {
+    if (!is_pow2(block_size) || block_size > 256) return 0;
+    if (num_prefixes < 0 || max_prefix_members < 1 || max_prefix_len < 0) return 0;
+    if (num_q_heads <= 0 || num_kv_heads <= 0 || num_q_heads % num_kv_heads) return 0;
+    const DeviceInfo* di = current_device_info();
+    if (!di) return 0;
+    size_t extra = 0;
+    if (num_prefixes > 0) {
+        const int tiles = prefix_row_tiles(max_prefix_members, num_q_heads / num_kv_heads);
+        const int splits = prefix_splits_for(di->num_sms, num_prefixes, num_kv_heads, tiles,
+                                             max_prefix_len);
+        extra = prefix_record_bytes(splits, num_seqs, num_q_heads, head_dim);
+    }
+    DecodePlan pl;
+    if (!make_decode_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len,
+                          0, &pl, extra))
+        return 0;
+    return pl.bytes;
+}
+
+pkv_status pkv_paged_attention_decode_prefix(
+    const void* q, const void* k_cache, const void* v_cache, const int32_t* block_tables,
+    const int32_t* seq_lens, int32_t block_size, float scale, void* out, int32_t num_seqs,
+    int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim, int32_t max_blocks_per_seq,
+    int32_t num_blocks, int32_t max_seq_len, pkv_dtype q_dtype, pkv_dtype kv_dtype,
+    pkv_dtype out_dtype, const int32_t* prefix_of, const int32_t* prefix_lens,
+    int32_t num_prefixes, int32_t max_prefix_members, int32_t max_prefix_len, void* workspace,
+    size_t workspace_bytes, pkv_stream_t stream) {
+    const PrefixArgs pa{prefix_of, prefix_lens, num_prefixes, max_prefix_members, max_prefix_len};
+    return decode_entry(q, k_cache, v_cache, block_tables, seq_lens, block_size, scale, out,
+                        num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                        num_blocks, max_seq_len, q_dtype, kv_dtype, out_dtype, nullptr, nullptr, 0,
+                        workspace, workspace_bytes, stream, &pa);
 }
 
 pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping,

@@ -28,23 +28,84 @@ __device__ __forceinline__ int chunks_of(int L) {
     return (L + CH - 1) / CH;
 }
 
+// ---- shared prefixes --------------------------------------------------------
+// A prefix group is a set of requests whose block tables name the same
+// physical blocks for their first prefix_lens[g] tokens (blocks a fork shares).
+// The shared pass reads those tokens once for the whole group and leaves
+// per-(request, query head) partial results; the per-request pass then starts
+// at the prefix's end and folds them in.
+
+constexpr int kPrefixCH = 64;  // tokens per chunk of the shared pass
+
+// Tokens the shared pass of group `g` covers: prefix_lens[g] clamped to
+// [0, min(max_prefix_len, cap)] and rounded down to whole blocks, so both
+// passes split every request at the same block boundary.  A length that needs
+// clamping or rounding raises PKV_DEVERR_PREFIX when `flag`.
+__device__ __forceinline__ int prefix_tokens(const int32_t* prefix_lens, int g, int max_prefix_len,
+                                             int cap, int log2_bs, unsigned* err, bool flag) {
+    const int raw = __ldg(prefix_lens + g);
+    int t = min(max(raw, 0), min(max_prefix_len, cap));
+    t = (t >> log2_bs) << log2_bs;
+    if (flag && t != raw) raise_error(err, PKV_DEVERR_PREFIX);
+    return t;
+}
+
+// The shared pass cuts a prefix of `ptok` tokens into splits of W chunks,
+// W = ceil(chunks / S) for the S splits the launch provides; returns the
+// number of splits that hold chunks (records the per-request pass folds in).
+__device__ __forceinline__ int prefix_chunk_span(int ptok, int S) {
+    const int nch = (ptok + kPrefixCH - 1) / kPrefixCH;
+    return nch == 0 ? 0 : (nch + S - 1) / S;
+}
+__device__ __forceinline__ int prefix_num_splits(int ptok, int S) {
+    const int nch = (ptok + kPrefixCH - 1) / kPrefixCH;
+    if (nch == 0) return 0;
+    const int w = (nch + S - 1) / S;
+    return (nch + w - 1) / w;
+}
+
+// First token of request b's own pass (0 without a prefix group): the
+// group's shared tokens, or all L of them if the request is shorter.
+__device__ __forceinline__ int seq_begin(const DecodeParams& p, int b, int L, bool flag = false) {
+    if (!p.prefix_of) return 0;
+    const int g = __ldg(p.prefix_of + b);
+    if (g < 0) return 0;
+    if (g >= p.num_prefixes) {
+        if (flag) raise_error(p.err, PKV_DEVERR_PREFIX);
+        return 0;
+    }
+    const int t = prefix_tokens(p.prefix_lens, g, p.max_prefix_len, p.max_blocks * p.block_size,
+                                p.log2_bs, p.err, flag);
+    return min(t, L);
+}
+
 // Position in the flattened (request, head group, chunk) list.
 struct Cursor {
     int b, hg, c, nch, L;
+    int t0;  // first token of the request's pass (its chunk c starts at t0 + c*CH)
 };
 
 // Warp-cooperative search for global chunk index s (all lanes get the result).
 // L_first, if >= 0, is this lane's (clamped) length of request `lane`, already
 // loaded by the caller; it saves a dependent global load on the first pass.
 template <int CH>
-__device__ Cursor locate(const DecodeParams& p, long long s, int lane, int L_first = -1) {
-    Cursor cur{p.num_seqs, 0, 0, 0, 0};
+__device__ Cursor locate(const DecodeParams& p, long long s, int lane, int L_first = -1,
+                         int T_first = 0) {
+    Cursor cur{p.num_seqs, 0, 0, 0, 0, 0};
     long long base = 0;
     for (int b0 = 0; b0 < p.num_seqs; b0 += 32) {
         const int b = b0 + lane;
-        const int L = b < p.num_seqs ? ((b0 == 0 && L_first >= 0) ? L_first : clamp_len(p, b, false))
-                                     : 0;
-        const long long n = (long long)chunks_of<CH>(L) * p.num_hg;
+        int L = 0, T = 0;
+        if (b < p.num_seqs) {
+            if (b0 == 0 && L_first >= 0) {
+                L = L_first;
+                T = T_first;
+            } else {
+                L = clamp_len(p, b, false);
+                T = seq_begin(p, b, L);
+            }
+        }
+        const long long n = (long long)chunks_of<CH>(L - T) * p.num_hg;
         long long incl = n;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -56,11 +117,13 @@ __device__ Cursor locate(const DecodeParams& p, long long s, int lane, int L_fir
         if (hit) {
             const int src = __ffs(hit) - 1;
             const int Lb = __shfl_sync(FULL_MASK, L, src);
+            const int Tb = __shfl_sync(FULL_MASK, T, src);
             const long long ex = __shfl_sync(FULL_MASK, excl, src);
             const long long off = s - (base + ex);
-            const int nch = chunks_of<CH>(Lb);
+            const int nch = chunks_of<CH>(Lb - Tb);
             cur.b = b0 + src;
             cur.L = Lb;
+            cur.t0 = Tb;
             cur.nch = nch;
             cur.hg = (int)(off / nch);
             cur.c = (int)(off % nch);
@@ -83,7 +146,8 @@ __device__ __forceinline__ void next_group(const DecodeParams& p, Cursor& cur) {
             return;
         }
         cur.L = clamp_len(p, cur.b, false);
-        cur.nch = chunks_of<CH>(cur.L);
+        cur.t0 = seq_begin(p, cur.b, cur.L);
+        cur.nch = chunks_of<CH>(cur.L - cur.t0);
         if (cur.nch > 0) return;
     }
 }
@@ -93,8 +157,10 @@ __device__ __forceinline__ void next_group(const DecodeParams& p, Cursor& cur) {
 template <int CH>
 __device__ long long total_chunks(const DecodeParams& p, long long* red, bool flag) {
     long long local = 0;
-    for (int b = threadIdx.x; b < p.num_seqs; b += blockDim.x)
-        local += chunks_of<CH>(clamp_len(p, b, flag));
+    for (int b = threadIdx.x; b < p.num_seqs; b += blockDim.x) {
+        const int L = clamp_len(p, b, flag);
+        local += chunks_of<CH>(L - seq_begin(p, b, L, flag));
+    }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) local += __shfl_xor_sync(FULL_MASK, local, off);
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = local;
@@ -120,6 +186,7 @@ struct SegIter {
     Cursor cur;
     bool valid;
     int L_first = -1;  // this lane's length of request `lane` (first 32 requests)
+    int T_first = 0;   // and the first token of its pass
 
     __device__ void start_unit(const DecodeParams& p, int lane) {
         valid = u < nunits;
@@ -127,17 +194,18 @@ struct SegIter {
         const long long s0 = u * W;
         s1 = min(s0 + W, total);
         g = s0;
-        cur = locate<CH>(p, s0, lane, L_first);
+        cur = locate<CH>(p, s0, lane, L_first, T_first);
         valid = cur.nch > 0;
     }
 
     __device__ void init(const DecodeParams& p, long long total_, long long W_, int lane,
-                         int L_first_ = -1) {
+                         int L_first_ = -1, int T_first_ = 0) {
         total = total_;
         W = W_;
         nunits = (total + W - 1) / W;
         u = blockIdx.x;
         L_first = L_first_;
+        T_first = T_first_;
         start_unit(p, lane);
     }
 

@@ -40,6 +40,7 @@
 #include <mutex>
 
 #include "decode_common.cuh"
+#include "mma_ptx.cuh"
 
 namespace pkv {
 namespace {
@@ -69,100 +70,6 @@ struct MmaCfg {
     static constexpr int STAGE_BYTES = (2 * KV_BYTES + Q_BYTES + 1023) / 1024 * 1024;
     static constexpr int NSTAGE = cmax(2, cmin(8, (kRingBudget - STG_BYTES) / STAGE_BYTES));
 };
-
-// ---- PTX wrappers -----------------------------------------------------------
-
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
-                                            uint64_t* bar, uint64_t policy) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        ".L2::cache_hint [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(policy)
-        : "memory");
-}
-
-__device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
-}
-
-__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
-}
-
-__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t (&r)[4]) {
-    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                 : "r"(addr));
-}
-
-__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                         uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
-        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ void mma_f16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                        uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, "
-        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-template <bool F8>
-__device__ __forceinline__ void mma16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    if constexpr (F8)
-        mma_f16(c, a, b0, b1);
-    else
-        mma_bf16(c, a, b0, b1);
-}
-
-__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
-    const __half2 v = __floats2half2_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t*>(&v);
-}
-
-__device__ __forceinline__ float f16_round(float x) { return __half2float(__float2half_rn(x)); }
-
-// two bf16 (one 32-bit word) -> two f16, exact inside the f16 range
-__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
-    return pack_f16(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
-}
-
-// four e4m3 codes (one 32-bit word) -> four f16 (two 32-bit words), exact
-__device__ __forceinline__ void e4m3x4_to_f16(uint32_t w, uint32_t& lo, uint32_t& hi) {
-    const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xffffu), __NV_E4M3);
-    const __half2_raw b = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w >> 16), __NV_E4M3);
-    lo = (uint32_t)a.x | ((uint32_t)a.y << 16);
-    hi = (uint32_t)b.x | ((uint32_t)b.y << 16);
-}
-
-__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
-    uint32_t y;
-    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
-    return y;
-}
-
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t*>(&v);
-}
-
-__device__ __forceinline__ float bf16_round(float x) {
-    return __bfloat162float(__float2bfloat16_rn(x));
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-__device__ __forceinline__ float ld_cg(const float* p) { return __ldcg(p); }
 
 // ---- shared-memory layout ------------------------------------------------------
 
@@ -208,8 +115,8 @@ struct Producer {
         return j < nblk ? __ldg(p.block_tables + (size_t)cur.b * p.max_blocks + j) : -1;
     }
 
-    static __device__ __forceinline__ int first_block(int c0, int log2_bs) {
-        return (c0 * kCH) >> log2_bs;
+    static __device__ __forceinline__ int first_block(const Cursor& cur, int c0, int log2_bs) {
+        return (cur.t0 + c0 * kCH) >> log2_bs;
     }
 
     // Returns false when the CTA must stop (a wait gave up).
@@ -220,11 +127,11 @@ struct Producer {
         const int gv = min(C::GP, p.group - sub * C::GP);
         const int nblk = (cur.L + p.block_size - 1) >> p.log2_bs;
         const int rb = min(p.block_size, kCH);  // rows per TMA box
-        int wbase = first_block(sg.c0, p.log2_bs) & ~31;
+        int wbase = first_block(cur, sg.c0, p.log2_bs) & ~31;
         int tab = tab_first;
         int tab_next = (wbase + 32 < nblk) ? load_window(cur, wbase + 32) : -1;
         for (int c = sg.c0; c < sg.c1; ++c) {
-            const int t0 = c * kCH;
+            const int t0 = cur.t0 + c * kCH;
             const int ntok = min(kCH, cur.L - t0);
             const int ja = t0 >> p.log2_bs;
             const int jb = (t0 + ntok - 1) >> p.log2_bs;
@@ -302,7 +209,7 @@ struct Producer {
         int tab_first = -1;
         if (it.valid) {
             const Segment sg = it.current();
-            tab_first = load_window(sg.cur, first_block(sg.c0, p.log2_bs) & ~31);
+            tab_first = load_window(sg.cur, first_block(sg.cur, sg.c0, p.log2_bs) & ~31);
         }
         while (it.valid) {
             const Segment sg = it.current();
@@ -311,7 +218,7 @@ struct Producer {
             int tab_after = -1;
             if (it.valid) {
                 const Segment nx = it.current();
-                tab_after = load_window(nx.cur, first_block(nx.c0, p.log2_bs) & ~31);
+                tab_after = load_window(nx.cur, first_block(nx.cur, nx.c0, p.log2_bs) & ~31);
             }
             if (!run_segment(sg, tab_first)) break;
             tab_first = tab_after;
@@ -635,6 +542,74 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
     }
 }
 
+// ---- shared-prefix results ------------------------------------------------------
+
+// Tokens of request b's prefix group that the shared pass covered (0: none).
+__device__ __forceinline__ int prefix_tokens_of(const DecodeParams& p, int b) {
+    if (!p.prefix_of) return 0;
+    const int g = __ldg(p.prefix_of + b);
+    if (g < 0 || g >= p.num_prefixes) return 0;
+    return prefix_tokens(p.prefix_lens, g, p.max_prefix_len, p.max_blocks * p.block_size,
+                         p.log2_bs, p.err, false);
+}
+
+// Fold the shared pass's partial results for request b, heads hq0 + h (this
+// lane's rows h = nt*8 + 2*tig + j, dims dt*16 + grp and + 8) into a running
+// (max M, sum S, unnormalised A) state in the same log2 units.
+template <int D, int NT>
+__device__ __forceinline__ void fold_prefix(const DecodeParams& p, int b, int hq0, int gv, int tig,
+                                            int grp, float (&M)[NT][2], float (&S)[NT][2],
+                                            float (&A)[D / 16][NT][4]) {
+    const int ptok = prefix_tokens_of(p, b);
+    const int ns = prefix_num_splits(ptok, p.pfx_splits);
+    for (int sp = 0; sp < ns; ++sp) {
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int h = nt * 8 + 2 * tig + j;
+                if (h >= gv) continue;
+                const size_t row = ((size_t)sp * p.num_seqs + b) * p.num_q_heads + hq0 + h;
+                const float mr = p.pfx_ml[row * 2], lr = p.pfx_ml[row * 2 + 1];
+                const float Mn = fmaxf(M[nt][j], mr);
+                const float mref = Mn == -INFINITY ? 0.f : Mn;
+                const float fa = exp2f(M[nt][j] - mref), fb = exp2f(mr - mref);
+                S[nt][j] = S[nt][j] * fa + lr * fb;
+                const float* ra = p.pfx_acc + row * D;
+#pragma unroll
+                for (int dt = 0; dt < D / 16; ++dt) {
+                    A[dt][nt][j] = A[dt][nt][j] * fa + ra[dt * 16 + grp] * fb;
+                    A[dt][nt][j + 2] = A[dt][nt][j + 2] * fa + ra[dt * 16 + grp + 8] * fb;
+                }
+                M[nt][j] = Mn;
+            }
+    }
+}
+
+// A part's partial result (unnormalised acc, max m, sum l) as record `rec`.
+template <int D, int NT>
+__device__ __forceinline__ void write_record(const DecodeParams& p, size_t rec, int tig, int grp,
+                                             const float (&acc)[D / 16][NT][4],
+                                             const float (&m)[NT][2], const float (&l)[NT][2]) {
+    constexpr int GP = 8 * NT;
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            const int h = nt * 8 + 2 * tig + j;
+            float* ra = p.rec_acc + (rec * GP + h) * D;
+#pragma unroll
+            for (int dt = 0; dt < D / 16; ++dt) {
+                ra[dt * 16 + grp] = acc[dt][nt][j];
+                ra[dt * 16 + grp + 8] = acc[dt][nt][j + 2];
+            }
+            if (grp == 0) {
+                p.rec_ml[(rec * GP + h) * 2] = m[nt][j];
+                p.rec_ml[(rec * GP + h) * 2 + 1] = l[nt][j];
+            }
+        }
+}
+
 // ---- epilogue: normalise, or write a partial record and merge the group ----
 
 template <int D, int NT, bool F8>
@@ -647,11 +622,33 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
     const int grp = lane >> 2, tig = lane & 3;
     Ring dring;
     griddep_wait();  // `out` and the workspace may be in use by the previous kernel
-    // empty requests: all-zero rows (softmax of an empty set)
+    // Requests with no token of their own pass: all-zero rows (softmax of an
+    // empty set), or, when the shared prefix covers the whole request, the
+    // merge of the shared pass's partial results.
     for (int b = blockIdx.x; b < p.num_seqs; b += gridDim.x) {
-        if (clamp_len(p, b, false) != 0) continue;
-        for (int i = lane; i < p.num_q_heads * D; i += 32)
-            store_out(p.out, (size_t)b * p.num_q_heads * D + i, 0.f, p.out_dtype);
+        const int L = clamp_len(p, b, false);
+        const int T = seq_begin(p, b, L);
+        if (L != T) continue;
+        const int ns = T > 0 ? prefix_num_splits(prefix_tokens_of(p, b), p.pfx_splits) : 0;
+        for (int i = lane; i < p.num_q_heads * D; i += 32) {
+            float v = 0.f;
+            if (ns > 0) {
+                const size_t hrow = (size_t)b * p.num_q_heads + i / D;
+                float Mx = -INFINITY;
+                for (int sp = 0; sp < ns; ++sp)
+                    Mx = fmaxf(Mx, p.pfx_ml[((size_t)sp * p.num_seqs * p.num_q_heads + hrow) * 2]);
+                const float mref = Mx == -INFINITY ? 0.f : Mx;
+                float Ssum = 0.f, Acc = 0.f;
+                for (int sp = 0; sp < ns; ++sp) {
+                    const size_t row = (size_t)sp * p.num_seqs * p.num_q_heads + hrow;
+                    const float f = exp2f(p.pfx_ml[row * 2] - mref);
+                    Ssum += p.pfx_ml[row * 2 + 1] * f;
+                    Acc += p.pfx_acc[row * D + i % D] * f;
+                }
+                v = Ssum > 0.f ? Acc / Ssum : 0.f;
+            }
+            store_out(p.out, (size_t)b * p.num_q_heads * D + i, v, p.out_dtype);
+        }
     }
     while (it.valid) {
         const Segment sg = it.current();
@@ -695,6 +692,7 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
                 l[nt][j] += __shfl_xor_sync(FULL_MASK, l[nt][j], 16);
             }
         if (si.nseg == 1) {
+            if (p.prefix_of) fold_prefix<D, NT>(p, si.b, si.hq0, si.gv, tig, grp, m, l, acc);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -716,6 +714,16 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
             if (lane == 0) raise_error(p.err, PKV_DEVERR_BAD_SEQ_LEN);
             continue;
         }
+        if (p.defer_merge) {
+            // Fixed partitions: every part publishes its record and the
+            // group's first unit / part count; the merge kernel combines them.
+            write_record<D, NT>(p, si.bg + si.u, tig, grp, acc, m, l);
+            if (si.u == si.u_first && lane == 0) {
+                p.meta[2 * si.bg] = (int32_t)si.u_first;
+                p.meta[2 * si.bg + 1] = si.nseg;
+            }
+            continue;
+        }
         // Arrive first.  Only a part that is not the last of its group to
         // finish publishes its partial result (record, then a ready flag); the
         // last one keeps its own in registers and merges the others'.
@@ -724,22 +732,7 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
         arrived = __shfl_sync(FULL_MASK, arrived, 0);
         const size_t rec = si.bg + si.u;
         if (arrived != (unsigned)(si.nseg - 1)) {
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const int h = nt * 8 + 2 * tig + j;
-                    float* ra = p.rec_acc + (rec * GP + h) * D;
-#pragma unroll
-                    for (int dt = 0; dt < C::KS; ++dt) {
-                        ra[dt * 16 + grp] = acc[dt][nt][j];
-                        ra[dt * 16 + grp + 8] = acc[dt][nt][j + 2];
-                    }
-                    if (grp == 0) {
-                        p.rec_ml[(rec * GP + h) * 2] = m[nt][j];
-                        p.rec_ml[(rec * GP + h) * 2 + 1] = l[nt][j];
-                    }
-                }
+            write_record<D, NT>(p, rec, tig, grp, acc, m, l);
             __threadfence();
             __syncwarp();
             if (lane == 0) atomicExch(p.ready + rec, 1u);
@@ -825,6 +818,7 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
                     }
             }
         }
+        if (p.prefix_of) fold_prefix<D, NT>(p, si.b, si.hq0, si.gv, tig, grp, Mc, Sc, A);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -847,15 +841,21 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
 }
 
 // Total chunk count, computed by one warp (same value in every warp and CTA).
-// *L_first receives this lane's length of request `lane` (or 0).
+// *L_first / *T_first receive this lane's length of request `lane` and the
+// first token of its pass (or 0).
 __device__ __forceinline__ long long total_chunks_warp(const DecodeParams& p, int lane, bool flag,
-                                                       int* L_first) {
+                                                       int* L_first, int* T_first) {
     long long t = 0;
     *L_first = 0;
+    *T_first = 0;
     for (int b = lane; b < p.num_seqs; b += 32) {
         const int L = clamp_len(p, b, flag);
-        if (b == lane) *L_first = L;
-        t += chunks_of<kCH>(L);
+        const int T = seq_begin(p, b, L, flag);
+        if (b == lane) {
+            *L_first = L;
+            *T_first = T;
+        }
+        t += chunks_of<kCH>(L - T);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(FULL_MASK, t, off);
@@ -900,8 +900,9 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
     // guarantees are not produced by the kernel right before this one; so it
     // overlaps that kernel's tail.  Each role waits on the grid dependency
     // before touching K/V, q, out or the workspace.
-    int L_first = 0;
-    const long long total = total_chunks_warp(p, lane, blockIdx.x == 0 && warp == 0, &L_first);
+    int L_first = 0, T_first = 0;
+    const long long total =
+        total_chunks_warp(p, lane, blockIdx.x == 0 && warp == 0, &L_first, &T_first);
     if (total == 0) {
         if (warp == 2) {
             SegIter<kCH> none;
@@ -913,7 +914,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
     long long W = p.fixed_units > 0 ? p.fixed_units : (total + gridDim.x - 1) / gridDim.x;
     if (W < 1) W = 1;
     SegIter<kCH> it;
-    it.init(p, total, W, lane, L_first);
+    it.init(p, total, W, lane, L_first, T_first);
 
     if (warp == 0) {
         Producer<D, NT, F8> pr{p, &tmk, &tmv, smem, full, empty, st_ntok, st_bad, ctrl, lane,
@@ -927,41 +928,66 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
     }
 }
 
+// ---- merge of fixed partitions --------------------------------------------------
+
+// CTA = (request, head group) x a 32-wide slice of head_dim; warp h merges
+// query head h of the group over all of its parts: lanes own one dimension
+// each, so every record read is one coalesced 128-byte row segment, eight
+// records in flight per lane.
+//   out = vscale * sum_r 2^(m_r - M) acc_r / sum_r 2^(m_r - M) l_r.
+template <int D, int GP>
+__global__ void __launch_bounds__(32 * GP) decode_mma_merge_kernel(const __grid_constant__ DecodeParams p) {
+    constexpr int NSL = D / 32;
+    const int bg = blockIdx.x / NSL, slice = blockIdx.x % NSL;
+    const int b = bg / p.num_hg, hg = bg % p.num_hg;
+    const int kvh = hg / p.num_sub, sub = hg % p.num_sub;
+    const int hq0 = kvh * p.group + sub * GP;
+    const int gv = min(GP, p.group - sub * GP);
+    const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int L = clamp_len(p, b, false);
+    const int T = seq_begin(p, b, L);
+    griddep_wait();  // the records and meta of the decode kernel
+    if (L == T || h >= gv) return;  // empty own pass: the decode kernel wrote it
+    const int u0 = p.meta[2 * (size_t)bg];
+    const int nseg = p.meta[2 * (size_t)bg + 1];
+    if (nseg <= 1) return;  // written by the decode kernel directly
+    const size_t rec0 = (size_t)bg + u0;
+    float M = -INFINITY;
+    for (int r = lane; r < nseg; r += 32) M = fmaxf(M, p.rec_ml[((rec0 + r) * GP + h) * 2]);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, off));
+    const float mref = M == -INFINITY ? 0.f : M;
+    float S = 0.f;
+    for (int r = lane; r < nseg; r += 32) {
+        const size_t row = (rec0 + r) * GP + h;
+        S += p.rec_ml[row * 2 + 1] * exp2f(p.rec_ml[row * 2] - mref);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) S += __shfl_xor_sync(FULL_MASK, S, off);
+    const int d = slice * 32 + lane;
+    float A = 0.f;
+    int r = 0;
+    for (; r + 8 <= nseg; r += 8) {
+        float a[8], w[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const size_t row = (rec0 + r + k) * GP + h;
+            a[k] = p.rec_acc[row * D + d];
+            w[k] = p.rec_ml[row * 2];
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) A = fmaf(a[k], exp2f(w[k] - mref), A);
+    }
+    for (; r < nseg; ++r) {
+        const size_t row = (rec0 + r) * GP + h;
+        A = fmaf(p.rec_acc[row * D + d], exp2f(p.rec_ml[row * 2] - mref), A);
+    }
+    const float vsc = p.v_scale ? __ldg(p.v_scale + kvh) : 1.f;
+    store_out(p.out, ((size_t)b * p.num_q_heads + hq0 + h) * D + d, S > 0.f ? A * vsc / S : 0.f,
+              p.out_dtype);
+}
+
 // ---- host side ---------------------------------------------------------------
-
-PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        void* ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    });
-    return fn;
-}
-
-// 2-D view of a cache: rows = num_blocks*Hkv*block_size, columns = head_dim
-// bf16; boxes of 64 columns x min(block_size, 64) rows, 128-byte swizzle.
-// fp8: rows of head_dim one-byte codes, whole-row boxes, no swizzle (the
-// consumer reads them linearly while widening them).
-bool encode_cache_map(CUtensorMap* map, const void* base, long long rows, int head_dim,
-                      int box_rows, bool fp8) {
-    auto enc = tensor_map_encoder();
-    if (!enc) return false;
-    cuuint64_t gdim[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
-    cuuint64_t gstride[1] = {(cuuint64_t)head_dim * (fp8 ? 1 : 2)};
-    cuuint32_t box[2] = {fp8 ? (cuuint32_t)head_dim : 64u, (cuuint32_t)box_rows};
-    cuuint32_t estride[2] = {1u, 1u};
-    const CUresult r = enc(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                           2, const_cast<void*>(base), gdim, gstride, box, estride,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE,
-                           fp8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
-                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
 
 template <int D, int NT, bool F8>
 pkv_status launch_impl(const DecodeParams& p, cudaStream_t stream, int* grid_out) {
@@ -997,11 +1023,53 @@ pkv_status launch_impl(const DecodeParams& p, cudaStream_t stream, int* grid_out
 
     PdlLaunch L(dim3(grid), dim3(kThreads), S::BYTES, stream);
     if (cudaLaunchKernelEx(&L.cfg, kern, p, tmk, tmv) != cudaSuccess) return PKV_ERR_CUDA;
+    if (p.defer_merge) {
+        constexpr int GP = MmaCfg<D, NT, F8>::GP;
+        const long long mgrid = (long long)p.num_seqs * p.num_hg * (D / 32);
+        if (mgrid > 0x7fffffffLL) return PKV_ERR_UNSUPPORTED;
+        PdlLaunch M(dim3((unsigned)mgrid), dim3(32 * GP), 0, stream);
+        if (cudaLaunchKernelEx(&M.cfg, decode_mma_merge_kernel<D, GP>, p) != cudaSuccess)
+            return PKV_ERR_CUDA;
+    }
     if (grid_out) *grid_out = grid;
     return PKV_OK;
 }
 
 }  // namespace
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
+
+// 2-D view of a cache: rows = num_blocks*Hkv*block_size, columns = head_dim
+// bf16; boxes of 64 columns x min(block_size, 64) rows, 128-byte swizzle.
+// fp8: rows of head_dim one-byte codes, whole-row boxes, no swizzle (the
+// consumer reads them linearly while widening them).
+bool encode_cache_map(CUtensorMap* map, const void* base, long long rows, int head_dim,
+                      int box_rows, bool fp8) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t gdim[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
+    cuuint64_t gstride[1] = {(cuuint64_t)head_dim * (fp8 ? 1 : 2)};
+    cuuint32_t box[2] = {fp8 ? (cuuint32_t)head_dim : 64u, (cuuint32_t)box_rows};
+    cuuint32_t estride[2] = {1u, 1u};
+    const CUresult r = enc(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                           2, const_cast<void*>(base), gdim, gstride, box, estride,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           fp8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
 
 bool decode_mma_supported(int head_dim, int block_size, pkv_dtype q_dtype, pkv_dtype kv_dtype) {
     return q_dtype == PKV_BF16 && (kv_dtype == PKV_BF16 || kv_dtype == PKV_FP8_E4M3) &&

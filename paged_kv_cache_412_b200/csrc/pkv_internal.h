@@ -2,6 +2,7 @@
 // units (launchers, per-device state).  Not part of the public ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -37,6 +38,7 @@ struct DecodePlan {
     size_t records;    // partial-result records
     size_t rec_bytes;  // records + their (max, sum) pairs + per-group meta
     size_t off_ml, off_meta;  // offsets inside the record region
+    size_t off_extra;         // caller-specific scratch after the records
     size_t bytes;      // smallest workspace that fits
 };
 
@@ -52,8 +54,10 @@ inline size_t ready_flags_offset(size_t workspace_bytes) {
 }
 
 // Fill a plan for these sizes on the current device (false if invalid).
+// extra_bytes: scratch placed after the records (no clearing needed).
 bool make_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
-                      int block_size, int max_seq_len, int partition_size, DecodePlan* plan);
+                      int block_size, int max_seq_len, int partition_size, DecodePlan* plan,
+                      size_t extra_bytes = 0);
 
 // Kernel arguments of the decode path (plain values, passed by value).
 struct DecodeParams {
@@ -74,10 +78,46 @@ struct DecodeParams {
     int num_seqs, num_q_heads, num_kv_heads, group, num_sub, num_hg;
     int block_size, log2_bs, max_blocks, num_blocks;
     int fixed_units;  // 0 = automatic
+    int defer_merge;  // 1: parts of a split group only publish records (+ meta);
+                      // a separate merge kernel combines them
     long long rec_cap;  // records the workspace holds
     int out_dtype;
     float scale_log2;  // softmax scale * log2(e)
+    // Shared prefixes (prefix_of == nullptr: none).  Request b's own pass
+    // starts at the end of its group's prefix and its output folds in the
+    // shared pass's partial results (pfx_*), one per split of that pass.
+    const int32_t* prefix_of;    // [num_seqs] group or -1
+    const int32_t* prefix_lens;  // [num_prefixes] tokens
+    const float* pfx_acc;        // [pfx_splits][num_seqs][num_q_heads][head_dim]
+    const float* pfx_ml;         // [pfx_splits][num_seqs][num_q_heads][2]
+    int num_prefixes, max_prefix_len, pfx_splits;
 };
+
+// Kernel arguments of the shared pass of pkv_paged_attention_decode_prefix.
+// CTA x handles split (x % splits) of row tile ((x / splits) % row_tiles) of
+// kv head ((x / splits / row_tiles) % num_kv_heads) of group
+// (x / splits / row_tiles / num_kv_heads); a row tile is 64 (member, query
+// head) rows of the group, members in request order.
+struct PrefixParams {
+    const void* q;
+    const int32_t* block_tables;
+    const int32_t* seq_lens;
+    const int32_t* prefix_of;
+    const int32_t* prefix_lens;
+    float* pfx_acc;  // as DecodeParams
+    float* pfx_ml;
+    unsigned* err;
+    int num_seqs, num_q_heads, num_kv_heads, group;
+    int block_size, log2_bs, max_blocks, num_blocks;
+    int num_prefixes, max_members, max_prefix_len, splits, row_tiles;
+    float scale_log2;
+};
+
+// Rows of (member, query head) pairs one CTA of the shared pass covers.
+constexpr int kPrefixRows = 64;
+
+pkv_status launch_decode_prefix(const PrefixParams& p, const void* k_cache, const void* v_cache,
+                                int head_dim, cudaStream_t stream);
 
 pkv_status launch_decode_simt(const DecodeParams& p, int head_dim, pkv_dtype kv_dtype,
                               int group_pad, cudaStream_t stream, int* grid_out);
@@ -86,6 +126,13 @@ bool decode_mma_supported(int head_dim, int block_size, pkv_dtype q_dtype, pkv_d
 
 pkv_status launch_decode_mma(const DecodeParams& p, int head_dim, int group_pad, bool fp8,
                              cudaStream_t stream, int* grid_out);
+
+// 2-D TMA view of a cache [num_blocks, Hkv, block_size, head_dim] as
+// rows x head_dim: bf16 boxes of 64 columns x box_rows rows with the 128-byte
+// swizzle; fp8 boxes of whole rows without swizzle.  False if the driver
+// entry point is missing or the encoder rejects the view.
+bool encode_cache_map(CUtensorMap* map, const void* base, long long rows, int head_dim,
+                      int box_rows, bool fp8);
 
 // Launch config with programmatic dependent launch: the kernel may start while
 // the previous kernel in the stream drains; it waits (griddepcontrol.wait)

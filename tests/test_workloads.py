@@ -85,3 +85,34 @@ def test_make_paged_tail_and_pool(permute):
     _check_consistent(w)
     assert w.block_tables.shape[1] == 5 + 2
     assert w.k_new.shape[0] == 2  # the empty request appends nothing
+
+
+def test_prefix_groups_share_blocks_and_fill_every_token():
+    """Members of a group name the same physical blocks for the prefix; after
+    the step (append of each request's last token) every token below a
+    request's length is a value, never the poison; appended slots lie in
+    blocks of the request's own."""
+    w = workloads.prefix_groups([(5, 64), (3, 128), (4, 0)], singles=3, bs=16, Hq=8, Hkv=2,
+                                d=64, short_members=1, seed=3)
+    po, pl = w.info["prefix_of"], w.info["prefix_lens"]
+    for g in range(len(pl)):
+        mem = np.where(po == g)[0]
+        nb = pl[g] // w.bs
+        longest = max(mem, key=lambda b: w.seq_lens[b])
+        for b in mem:
+            n = min(nb, -(-int(w.seq_lens[b]) // w.bs))
+            assert np.array_equal(w.block_tables[b, :n], w.block_tables[longest, :n])
+    kc, vc = w.k_cache.copy(), w.v_cache.copy()
+    for i, s in enumerate(w.slot_mapping):
+        kc[s // w.bs, :, s % w.bs] = w.k_new[i]
+        vc[s // w.bs, :, s % w.bs] = w.v_new[i]
+    shared = {int(x) for g in range(len(pl)) for x in
+              w.block_tables[np.where(po == g)[0][0], : pl[g] // w.bs]}
+    for s in w.slot_mapping:
+        assert int(s) // w.bs not in shared
+    for b in range(w.B):
+        for t in range(int(w.seq_lens[b])):
+            blk = w.block_tables[b, t // w.bs]
+            assert blk >= 0
+            assert not np.any(kc[blk, :, t % w.bs] == workloads.BF16_NAN)
+            assert not np.any(vc[blk, :, t % w.bs] == workloads.BF16_NAN)

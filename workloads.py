@@ -264,6 +264,99 @@ def prefix_shared(poison: bool = True, seed: int = 1004, batch: int = 64,
                           "suffix": suffix.tolist()})
 
 
+def prefix_groups(groups, singles: int = 0, *, seed: int = 1007, suffix_lo: int = 0,
+                  suffix_hi: int = 300, Hq: int = 32, Hkv: int = 8, d: int = 128, bs: int = 16,
+                  dtype: str = "bf16", poison: bool = True, short_members: int = 0,
+                  interleave: bool = True) -> Workload:
+    """Requests in groups that share the physical blocks of a prefix, plus
+    ungrouped requests.  ``groups`` lists (members, prefix_tokens) with
+    prefix_tokens a multiple of bs.  A member holds the group's shared blocks
+    for its first prefix_tokens tokens, then its own blocks for a suffix of
+    U{suffix_lo..suffix_hi} tokens; the first ``short_members`` members of each
+    group instead stop inside the prefix (length U{1..prefix_tokens}).  The
+    step appends each request's last token when it lies in a block of its own.
+    ``interleave`` spreads members of different groups across the batch.
+    info: prefix_of [B] int32 (-1 = none), prefix_lens [G] int32."""
+    rng = np.random.default_rng(seed)
+    reqs = []  # (group or -1, length)
+    for g, (n, ptok) in enumerate(groups):
+        assert ptok % bs == 0 and ptok >= 0
+        for i in range(n):
+            if i < short_members and ptok > 0:
+                L = int(rng.integers(1, ptok + 1))
+            else:
+                L = ptok + int(rng.integers(suffix_lo, suffix_hi + 1))
+            reqs.append((g, L))
+    for _ in range(singles):
+        reqs.append((-1, int(rng.integers(max(suffix_lo, 1), suffix_hi + 400))))
+    if interleave:
+        order = rng.permutation(len(reqs))
+        reqs = [reqs[i] for i in order]
+    B = len(reqs)
+    shared_nb = [ptok // bs for _, ptok in groups]
+    own_nb = []
+    for g, L in reqs:
+        nb = -(-L // bs)
+        own_nb.append(max(nb - (shared_nb[g] if g >= 0 else 0), 0))
+    NB = max(int(sum(shared_nb) + sum(own_nb)), 1)
+    pool = rng.permutation(NB)
+    pos = 0
+    shared = []
+    for nb in shared_nb:
+        shared.append([int(x) for x in pool[pos: pos + nb]])
+        pos += nb
+    max_blocks = max(max(-(-L // bs) for _, L in reqs), 1)
+    tables = np.full((B, max_blocks), -1, dtype=np.int32)
+    qdt = "bf16" if dtype == "fp8" else dtype
+    k_cache = _empty_cache((NB, Hkv, bs, d), dtype, poison)
+    v_cache = _empty_cache((NB, Hkv, bs, d), dtype, poison)
+    for g, ptok in enumerate(p for _, p in groups):
+        _fill_history(rng, k_cache, v_cache, np.asarray(shared[g], np.int64), ptok, bs, dtype)
+    slots = []
+    new_rows = []
+    for b, (g, L) in enumerate(reqs):
+        nb = -(-L // bs)
+        sh = shared[g] if g >= 0 else []
+        own = [int(x) for x in pool[pos: pos + own_nb[b]]]
+        pos += own_nb[b]
+        row = (sh + own)[:nb]
+        tables[b, : len(row)] = row
+        first_own = len(sh) * bs  # first token in an own block
+        last_in_own = L - 1 >= first_own
+        hist_end = L - 1 if last_in_own else L
+        # the request's own history tokens [first_own, hist_end)
+        if hist_end > first_own:
+            n_own = hist_end - first_own
+            kh = _cache_values(rng, (n_own, Hkv, d), dtype)
+            vh = _cache_values(rng, (n_own, Hkv, d), dtype)
+            for i in range(n_own):
+                t = first_own + i
+                blk, off = row[t // bs], t % bs
+                k_cache[blk, :, off, :] = kh[i]
+                v_cache[blk, :, off, :] = vh[i]
+        if last_in_own:
+            t = L - 1
+            slots.append(row[t // bs] * bs + t % bs)
+            new_rows.append(b)
+    T = len(slots)
+    k_new = _normal(rng, (T, Hkv, d), qdt)
+    v_new = _normal(rng, (T, Hkv, d), qdt)
+    q = _normal(rng, (B, Hq, d), qdt)
+    ks = vs = None
+    if dtype == "fp8":
+        ks = rng.uniform(0.05, 0.5, size=Hkv).astype(np.float32)
+        vs = rng.uniform(0.05, 0.5, size=Hkv).astype(np.float32)
+    return Workload(name="prefix_groups", B=B, Hq=Hq, Hkv=Hkv, d=d, bs=bs, num_blocks=NB,
+                    dtype=dtype, scale=1.0 / math.sqrt(d), q=q, k_cache=k_cache,
+                    v_cache=v_cache, block_tables=tables,
+                    seq_lens=np.asarray([L for _, L in reqs], np.int32), k_new=k_new,
+                    v_new=v_new, slot_mapping=np.asarray(slots, np.int64),
+                    info={"seed": seed,
+                          "prefix_of": np.asarray([g for g, _ in reqs], np.int32),
+                          "prefix_lens": np.asarray([p for _, p in groups], np.int32)},
+                    k_scale=ks, v_scale=vs)
+
+
 def long_ctx(bs: int = 16, poison: bool = True, seed: int = 1005, batch: int = 2,
              seq_len: int = 131072) -> Workload:
     """batch 2 x 131072 tokens, 64 q / 8 KV heads, d 128, block size bs, bf16."""
