@@ -630,6 +630,42 @@ def run_suite(args):
          {"bytes_kind": "logical (prefix counted once per request)", "unique_bytes": unique,
           "unique_GBps": round(unique / (ms[0] / 1e3) / 1e9, 2),
           "step": "copy_blocks (64 forks) + kv_cache_write (suffixes) + decode"})
+    # the same step with the shared blocks read once for the group
+    pfx_of = torch.zeros(w.B, dtype=torch.int32, device=dev)
+    pfx_len = torch.tensor([(w.info["prefix_tokens"] // w.bs) * w.bs], dtype=torch.int32,
+                           device=dev)
+    ws_p = pkv.new_workspace(pkv.decode_prefix_workspace_bytes(
+        w.B, w.Hq, w.Hkv, w.d, w.bs, L, 1, w.B, w.info["prefix_tokens"]), dev)
+
+    def prefix_decode():
+        pkv.paged_attention_decode_prefix(t["q"], t["kc"], t["vc"], t["bt"], t["sl"], pfx_of,
+                                          pfx_len, w.bs, w.scale, out, max_seq_len=L,
+                                          max_prefix_members=w.B,
+                                          max_prefix_len=w.info["prefix_tokens"],
+                                          workspace=ws_p)
+
+    def prefix_step_shared():
+        pkv.copy_blocks(t["kc"], t["vc"], t["pairs"])
+        pkv.kv_cache_write(t["kn"], t["vn"], t["sm"], t["kc"], t["vc"])
+        prefix_decode()
+    ms = _time_graph(prefix_step_shared, iters, flush)
+    emit("step prefix, prefix-aware decode (shared blocks read once per group)", ms, logical,
+         {"bytes_kind": "logical (prefix counted once per request)", "unique_bytes": unique,
+          "unique_GBps": round(unique / (ms[0] / 1e3) / 1e9, 2),
+          "step": "copy_blocks (64 forks) + kv_cache_write (suffixes) + "
+                  "paged_attention_decode_prefix"})
+    ms = _time_graph(lambda: pkv.paged_attention_decode(
+        t["q"], t["kc"], t["vc"], t["bt"], t["sl"], w.bs, w.scale, out, max_seq_len=L,
+        workspace=ws), iters, flush)
+    emit("decode prefix workload, per-request decode", ms, logical,
+         {"bytes_kind": "logical", "unique_bytes": unique,
+          "unique_GBps": round(unique / (ms[0] / 1e3) / 1e9, 2)})
+    ms = _time_graph(prefix_decode, iters, flush)
+    emit("decode prefix workload, prefix-aware decode", ms, logical,
+         {"bytes_kind": "logical", "unique_bytes": unique,
+          "unique_GBps": round(unique / (ms[0] / 1e3) / 1e9, 2)})
+    assert pkv.get_device_error() == 0
+    del ws_p
     del t, ws, out, kc0, vc0
     torch.cuda.empty_cache()
 

@@ -127,7 +127,11 @@ struct Producer {
         const int gv = min(C::GP, p.group - sub * C::GP);
         const int nblk = (cur.L + p.block_size - 1) >> p.log2_bs;
         const int rb = min(p.block_size, kCH);  // rows per TMA box
-        int wbase = first_block(cur, sg.c0, p.log2_bs) & ~31;
+        // Table windows start at the segment's first block and advance by 32
+        // blocks, a whole number of chunks (64 / block_size blocks each), so
+        // no chunk straddles two windows whatever block the request's pass
+        // starts at.
+        int wbase = first_block(cur, sg.c0, p.log2_bs);
         int tab = tab_first;
         int tab_next = (wbase + 32 < nblk) ? load_window(cur, wbase + 32) : -1;
         for (int c = sg.c0; c < sg.c1; ++c) {
@@ -209,7 +213,7 @@ struct Producer {
         int tab_first = -1;
         if (it.valid) {
             const Segment sg = it.current();
-            tab_first = load_window(sg.cur, first_block(sg.cur, sg.c0, p.log2_bs) & ~31);
+            tab_first = load_window(sg.cur, first_block(sg.cur, sg.c0, p.log2_bs));
         }
         while (it.valid) {
             const Segment sg = it.current();
@@ -218,7 +222,7 @@ struct Producer {
             int tab_after = -1;
             if (it.valid) {
                 const Segment nx = it.current();
-                tab_after = load_window(nx.cur, first_block(nx.cur, nx.c0, p.log2_bs) & ~31);
+                tab_after = load_window(nx.cur, first_block(nx.cur, nx.c0, p.log2_bs));
             }
             if (!run_segment(sg, tab_first)) break;
             tab_first = tab_after;
@@ -691,6 +695,15 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
                 l[nt][j] += __shfl_xor_sync(FULL_MASK, l[nt][j], 8);
                 l[nt][j] += __shfl_xor_sync(FULL_MASK, l[nt][j], 16);
             }
+        if (p.defer_merge && si.u == si.u_first && lane == 0) {
+            // The group's first part tells the merge kernel where its records
+            // are -- for every group with work, so no stale word is ever read;
+            // a group that does not fit the workspace is marked 0 (and flagged
+            // below) so the merge leaves it alone.
+            const bool fits = si.bg + si.u_last < (size_t)p.rec_cap;
+            p.meta[2 * si.bg] = (int32_t)si.u_first;
+            p.meta[2 * si.bg + 1] = fits ? si.nseg : 0;
+        }
         if (si.nseg == 1) {
             if (p.prefix_of) fold_prefix<D, NT>(p, si.b, si.hq0, si.gv, tig, grp, m, l, acc);
 #pragma unroll
@@ -715,13 +728,9 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
             continue;
         }
         if (p.defer_merge) {
-            // Fixed partitions: every part publishes its record and the
-            // group's first unit / part count; the merge kernel combines them.
+            // Fixed partitions: every part publishes its record; the merge
+            // kernel combines them.
             write_record<D, NT>(p, si.bg + si.u, tig, grp, acc, m, l);
-            if (si.u == si.u_first && lane == 0) {
-                p.meta[2 * si.bg] = (int32_t)si.u_first;
-                p.meta[2 * si.bg + 1] = si.nseg;
-            }
             continue;
         }
         // Arrive first.  Only a part that is not the last of its group to
@@ -951,6 +960,10 @@ __global__ void __launch_bounds__(32 * GP) decode_mma_merge_kernel(const __grid_
     const int u0 = p.meta[2 * (size_t)bg];
     const int nseg = p.meta[2 * (size_t)bg + 1];
     if (nseg <= 1) return;  // written by the decode kernel directly
+    if (u0 < 0 || (long long)bg + u0 + nseg > p.rec_cap) {  // never for a word this call wrote
+        if (threadIdx.x == 0) raise_error(p.err, PKV_DEVERR_BAD_SEQ_LEN);
+        return;
+    }
     const size_t rec0 = (size_t)bg + u0;
     float M = -INFINITY;
     for (int r = lane; r < nseg; r += 32) M = fmaxf(M, p.rec_ml[((rec0 + r) * GP + h) * 2]);

@@ -93,7 +93,12 @@ __global__ void __launch_bounds__(kThreadsP)
     const int ptok = prefix_tokens(p.prefix_lens, g, p.max_prefix_len, cap, p.log2_bs, p.err,
                                    leader && threadIdx.x == 0);
     const int nsplit = prefix_num_splits(ptok, p.splits);
-    if (sp >= nsplit) return;  // this split holds no chunk of the prefix
+    if (sp >= nsplit) {  // this split holds no chunk of the prefix
+        // still wait for the previous kernel, so that this grid's completion
+        // implies that kernel's (the decode pass after it relies on that)
+        griddep_wait();
+        return;
+    }
     const int span = prefix_chunk_span(ptok, p.splits);
     const int nch = chunks_of<kPrefixCH>(ptok);
     const int c0 = sp * span, c1 = min(c0 + span, nch);
@@ -160,7 +165,10 @@ __global__ void __launch_bounds__(kThreadsP)
     }
     __syncthreads();
     griddep_launch_dependents();
-    if (!ctrl[3]) return;
+    if (!ctrl[3]) {
+        griddep_wait();
+        return;
+    }
     const int b_src = ctrl[1];
     const int tl = ctrl[2];
     const int c_end = min(c1, chunks_of<kPrefixCH>(tl));
