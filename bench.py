@@ -558,6 +558,9 @@ def run_suite(args):
     flush = _L2Flush(dev)
     iters = max(20, min(args.steps, 500))
 
+    def want(section):
+        return not args.case or args.case in section
+
     def emit(name, ms, nbytes, extra):
         mean, med = ms
         gbs = nbytes / (mean / 1e3) / 1e9
@@ -596,18 +599,30 @@ def run_suite(args):
 
     # the 4k workload: permuted pool (as benched) and identity tables (the
     # indirection's cost is the difference)
-    decode_case("decode gqa_4k permuted pool", workloads.gqa_4k(poison=False))
-    w = workloads.make_paged([4096] * 16, Hq=32, Hkv=8, d=128, bs=16, dtype="bf16",
-                             seed=1002, poison=False, permute=False, name="gqa_4k_identity")
-    decode_case("decode gqa_4k identity tables", w)
-    decode_case("decode gqa_4k fp8 e4m3 cache", workloads.gqa_4k_fp8(poison=False), fp8=True)
-    decode_case("decode mixed (256 requests, log-uniform 16..8192)", workloads.mixed(poison=False))
-    for bs in (8, 16, 32):
-        wl = workloads.long_ctx(bs=bs, poison=False)
-        for P in (0, 512, 1024, 2048, 4096):
-            decode_case(f"decode long_ctx 2 x 131072 bs {bs} partition {P or 'auto'}", wl,
-                        partition_size=P)
-        del wl
+    if want("gqa_4k"):
+        decode_case("decode gqa_4k permuted pool", workloads.gqa_4k(poison=False))
+        w = workloads.make_paged([4096] * 16, Hq=32, Hkv=8, d=128, bs=16, dtype="bf16",
+                                 seed=1002, poison=False, permute=False, name="gqa_4k_identity")
+        decode_case("decode gqa_4k identity tables", w)
+    if want("fp8"):
+        decode_case("decode gqa_4k fp8 e4m3 cache", workloads.gqa_4k_fp8(poison=False), fp8=True)
+    if want("mixed"):
+        decode_case("decode mixed (256 requests, log-uniform 16..8192)",
+                    workloads.mixed(poison=False))
+    if want("long_ctx"):
+        for bs in (8, 16, 32):
+            wl = workloads.long_ctx(bs=bs, poison=False)
+            for P in (0, 512, 1024, 2048, 4096):
+                decode_case(f"decode long_ctx 2 x 131072 bs {bs} partition {P or 'auto'}", wl,
+                            partition_size=P)
+            del wl
+    if want("prefix"):
+        _suite_prefix(pkv, torch, workloads, dev, iters, flush, emit)
+    if want("cache_ops"):
+        _suite_cache_ops(pkv, torch, workloads, dev, iters, flush, emit)
+
+
+def _suite_prefix(pkv, torch, workloads, dev, iters, flush, emit):
 
     # shared prefix: the step (fork copy + suffix append + decode)
     w = workloads.prefix_shared(poison=False)
@@ -669,6 +684,8 @@ def run_suite(args):
     del t, ws, out, kc0, vc0
     torch.cuda.empty_cache()
 
+
+def _suite_cache_ops(pkv, torch, workloads, dev, iters, flush, emit):
     # cache operations alone
     w = workloads.gqa_4k(poison=False)
     t = _dev_workload(w, dev)
@@ -734,6 +751,9 @@ def main():
     ap.add_argument("--no-check", action="store_true")
     ap.add_argument("--suite", action="store_true",
                     help="one line per workload of the scope table instead of the headline")
+    ap.add_argument("--case", default="",
+                    help="with --suite: only the sections whose name contains this "
+                         "(gqa_4k, fp8, mixed, long_ctx, prefix, cache_ops)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

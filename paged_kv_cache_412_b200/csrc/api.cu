@@ -339,10 +339,11 @@ pkv_status decode_entry(const void* q, const void* k_cache, const void* v_cache,
     p.max_blocks = max_blocks_per_seq;
     p.num_blocks = num_blocks;
     p.fixed_units = partition_size > 0 ? std::max(1, partition_size / (mma ? 64 : 32)) : 0;
-    // Fixed partitions on the tensor-core path: merge in a separate kernel, so
-    // a group split into many parts is combined in parallel instead of by its
-    // last part alone (which would stall that part's CTA).
-    p.defer_merge = (mma && partition_size > 0) ? 1 : 0;
+    // Fixed partitions and prefix groups on the tensor-core path: merge in a
+    // separate kernel, so a group split into many parts (or folded with many
+    // splits of a shared prefix) is combined in parallel instead of by one
+    // warp of the decode kernel (which would stall that warp's CTA).
+    p.defer_merge = (mma && (partition_size > 0 || use_prefix)) ? 1 : 0;
     p.rec_cap = (long long)pl.records;
     p.out_dtype = out_dtype;
     p.scale_log2 = scale * 1.4426950408889634f;

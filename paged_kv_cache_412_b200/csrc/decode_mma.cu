@@ -557,39 +557,6 @@ __device__ __forceinline__ int prefix_tokens_of(const DecodeParams& p, int b) {
                          p.log2_bs, p.err, false);
 }
 
-// Fold the shared pass's partial results for request b, heads hq0 + h (this
-// lane's rows h = nt*8 + 2*tig + j, dims dt*16 + grp and + 8) into a running
-// (max M, sum S, unnormalised A) state in the same log2 units.
-template <int D, int NT>
-__device__ __forceinline__ void fold_prefix(const DecodeParams& p, int b, int hq0, int gv, int tig,
-                                            int grp, float (&M)[NT][2], float (&S)[NT][2],
-                                            float (&A)[D / 16][NT][4]) {
-    const int ptok = prefix_tokens_of(p, b);
-    const int ns = prefix_num_splits(ptok, p.pfx_splits);
-    for (int sp = 0; sp < ns; ++sp) {
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                const int h = nt * 8 + 2 * tig + j;
-                if (h >= gv) continue;
-                const size_t row = ((size_t)sp * p.num_seqs + b) * p.num_q_heads + hq0 + h;
-                const float mr = p.pfx_ml[row * 2], lr = p.pfx_ml[row * 2 + 1];
-                const float Mn = fmaxf(M[nt][j], mr);
-                const float mref = Mn == -INFINITY ? 0.f : Mn;
-                const float fa = exp2f(M[nt][j] - mref), fb = exp2f(mr - mref);
-                S[nt][j] = S[nt][j] * fa + lr * fb;
-                const float* ra = p.pfx_acc + row * D;
-#pragma unroll
-                for (int dt = 0; dt < D / 16; ++dt) {
-                    A[dt][nt][j] = A[dt][nt][j] * fa + ra[dt * 16 + grp] * fb;
-                    A[dt][nt][j + 2] = A[dt][nt][j + 2] * fa + ra[dt * 16 + grp + 8] * fb;
-                }
-                M[nt][j] = Mn;
-            }
-    }
-}
-
 // A part's partial result (unnormalised acc, max m, sum l) as record `rec`.
 template <int D, int NT>
 __device__ __forceinline__ void write_record(const DecodeParams& p, size_t rec, int tig, int grp,
@@ -626,33 +593,13 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
     const int grp = lane >> 2, tig = lane & 3;
     Ring dring;
     griddep_wait();  // `out` and the workspace may be in use by the previous kernel
-    // Requests with no token of their own pass: all-zero rows (softmax of an
-    // empty set), or, when the shared prefix covers the whole request, the
-    // merge of the shared pass's partial results.
+    // Requests with no token at all: all-zero rows (softmax of an empty set).
+    // (A request whose shared prefix covers all of it has no token of its own
+    // pass either; the merge kernel writes it from the shared pass's results.)
     for (int b = blockIdx.x; b < p.num_seqs; b += gridDim.x) {
-        const int L = clamp_len(p, b, false);
-        const int T = seq_begin(p, b, L);
-        if (L != T) continue;
-        const int ns = T > 0 ? prefix_num_splits(prefix_tokens_of(p, b), p.pfx_splits) : 0;
-        for (int i = lane; i < p.num_q_heads * D; i += 32) {
-            float v = 0.f;
-            if (ns > 0) {
-                const size_t hrow = (size_t)b * p.num_q_heads + i / D;
-                float Mx = -INFINITY;
-                for (int sp = 0; sp < ns; ++sp)
-                    Mx = fmaxf(Mx, p.pfx_ml[((size_t)sp * p.num_seqs * p.num_q_heads + hrow) * 2]);
-                const float mref = Mx == -INFINITY ? 0.f : Mx;
-                float Ssum = 0.f, Acc = 0.f;
-                for (int sp = 0; sp < ns; ++sp) {
-                    const size_t row = (size_t)sp * p.num_seqs * p.num_q_heads + hrow;
-                    const float f = exp2f(p.pfx_ml[row * 2] - mref);
-                    Ssum += p.pfx_ml[row * 2 + 1] * f;
-                    Acc += p.pfx_acc[row * D + i % D] * f;
-                }
-                v = Ssum > 0.f ? Acc / Ssum : 0.f;
-            }
-            store_out(p.out, (size_t)b * p.num_q_heads * D + i, v, p.out_dtype);
-        }
+        if (clamp_len(p, b, false) != 0) continue;
+        for (int i = lane; i < p.num_q_heads * D; i += 32)
+            store_out(p.out, (size_t)b * p.num_q_heads * D + i, 0.f, p.out_dtype);
     }
     while (it.valid) {
         const Segment sg = it.current();
@@ -695,17 +642,23 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
                 l[nt][j] += __shfl_xor_sync(FULL_MASK, l[nt][j], 8);
                 l[nt][j] += __shfl_xor_sync(FULL_MASK, l[nt][j], 16);
             }
-        if (p.defer_merge && si.u == si.u_first && lane == 0) {
-            // The group's first part tells the merge kernel where its records
-            // are -- for every group with work, so no stale word is ever read;
-            // a group that does not fit the workspace is marked 0 (and flagged
-            // below) so the merge leaves it alone.
+        if (p.defer_merge) {
+            // Fixed partitions and prefix groups: every part of every group
+            // publishes its record; the merge kernel combines them (with the
+            // shared pass's results) in parallel.  The group's first part
+            // tells it where the records are -- for every group with work, so
+            // no stale word is ever read; a group that does not fit the
+            // workspace is marked 0 and flagged, and the merge leaves it alone.
             const bool fits = si.bg + si.u_last < (size_t)p.rec_cap;
-            p.meta[2 * si.bg] = (int32_t)si.u_first;
-            p.meta[2 * si.bg + 1] = fits ? si.nseg : 0;
+            if (si.u == si.u_first && lane == 0) {
+                p.meta[2 * si.bg] = (int32_t)si.u_first;
+                p.meta[2 * si.bg + 1] = fits ? si.nseg : 0;
+                if (!fits) raise_error(p.err, PKV_DEVERR_BAD_SEQ_LEN);
+            }
+            if (fits) write_record<D, NT>(p, si.bg + si.u, tig, grp, acc, m, l);
+            continue;
         }
         if (si.nseg == 1) {
-            if (p.prefix_of) fold_prefix<D, NT>(p, si.b, si.hq0, si.gv, tig, grp, m, l, acc);
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -725,12 +678,6 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
         }
         if (si.bg + si.u_last >= (size_t)p.rec_cap) {
             if (lane == 0) raise_error(p.err, PKV_DEVERR_BAD_SEQ_LEN);
-            continue;
-        }
-        if (p.defer_merge) {
-            // Fixed partitions: every part publishes its record; the merge
-            // kernel combines them.
-            write_record<D, NT>(p, si.bg + si.u, tig, grp, acc, m, l);
             continue;
         }
         // Arrive first.  Only a part that is not the last of its group to
@@ -827,7 +774,6 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
                     }
             }
         }
-        if (p.prefix_of) fold_prefix<D, NT>(p, si.b, si.hq0, si.gv, tig, grp, Mc, Sc, A);
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
@@ -937,12 +883,13 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
     }
 }
 
-// ---- merge of fixed partitions --------------------------------------------------
+// ---- deferred merge (fixed partitions, prefix groups) ---------------------------
 
 // CTA = (request, head group) x a 32-wide slice of head_dim; warp h merges
-// query head h of the group over all of its parts: lanes own one dimension
-// each, so every record read is one coalesced 128-byte row segment, eight
-// records in flight per lane.
+// query head h of the group over the parts of its own pass (records of the
+// decode kernel) and the splits of its group's shared prefix pass: lanes own
+// one dimension each, so every record read is one coalesced 128-byte row
+// segment, eight records in flight per lane.
 //   out = vscale * sum_r 2^(m_r - M) acc_r / sum_r 2^(m_r - M) l_r.
 template <int D, int GP>
 __global__ void __launch_bounds__(32 * GP) decode_mma_merge_kernel(const __grid_constant__ DecodeParams p) {
@@ -955,46 +902,59 @@ __global__ void __launch_bounds__(32 * GP) decode_mma_merge_kernel(const __grid_
     const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int L = clamp_len(p, b, false);
     const int T = seq_begin(p, b, L);
-    griddep_wait();  // the records and meta of the decode kernel
-    if (L == T || h >= gv) return;  // empty own pass: the decode kernel wrote it
-    const int u0 = p.meta[2 * (size_t)bg];
-    const int nseg = p.meta[2 * (size_t)bg + 1];
-    if (nseg <= 1) return;  // written by the decode kernel directly
-    if (u0 < 0 || (long long)bg + u0 + nseg > p.rec_cap) {  // never for a word this call wrote
-        if (threadIdx.x == 0) raise_error(p.err, PKV_DEVERR_BAD_SEQ_LEN);
-        return;
+    const int ns = T > 0 ? prefix_num_splits(prefix_tokens_of(p, b), p.pfx_splits) : 0;
+    griddep_wait();  // the records and meta of the kernels before
+    if (h >= gv) return;
+    int u0 = 0, nseg = 0;
+    if (L > T) {
+        u0 = p.meta[2 * (size_t)bg];
+        nseg = p.meta[2 * (size_t)bg + 1];
+        if (nseg == 0) return;  // did not fit the workspace (flagged by the decode kernel)
+        if (u0 < 0 || (long long)bg + u0 + nseg > p.rec_cap) {  // never for a word this call wrote
+            if (threadIdx.x == 0) raise_error(p.err, PKV_DEVERR_BAD_SEQ_LEN);
+            return;
+        }
     }
+    if (nseg + ns == 0) return;  // an empty request: the decode kernel wrote zeros
     const size_t rec0 = (size_t)bg + u0;
+    // row r < nseg: own record; r >= nseg: split r - nseg of the shared pass
+    auto ml_of = [&](int r) -> const float* {
+        return r < nseg ? p.rec_ml + ((rec0 + r) * GP + h) * 2
+                        : p.pfx_ml + (((size_t)(r - nseg) * p.num_seqs + b) * p.num_q_heads +
+                                      hq0 + h) * 2;
+    };
+    auto acc_of = [&](int r) -> const float* {
+        return r < nseg ? p.rec_acc + ((rec0 + r) * GP + h) * D
+                        : p.pfx_acc + (((size_t)(r - nseg) * p.num_seqs + b) * p.num_q_heads +
+                                       hq0 + h) * D;
+    };
+    const int n = nseg + ns;
     float M = -INFINITY;
-    for (int r = lane; r < nseg; r += 32) M = fmaxf(M, p.rec_ml[((rec0 + r) * GP + h) * 2]);
+    for (int r = lane; r < n; r += 32) M = fmaxf(M, ml_of(r)[0]);
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, off));
     const float mref = M == -INFINITY ? 0.f : M;
     float S = 0.f;
-    for (int r = lane; r < nseg; r += 32) {
-        const size_t row = (rec0 + r) * GP + h;
-        S += p.rec_ml[row * 2 + 1] * exp2f(p.rec_ml[row * 2] - mref);
+    for (int r = lane; r < n; r += 32) {
+        const float* ml = ml_of(r);
+        S += ml[1] * exp2f(ml[0] - mref);
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) S += __shfl_xor_sync(FULL_MASK, S, off);
     const int d = slice * 32 + lane;
     float A = 0.f;
     int r = 0;
-    for (; r + 8 <= nseg; r += 8) {
+    for (; r + 8 <= n; r += 8) {
         float a[8], w[8];
 #pragma unroll
         for (int k = 0; k < 8; ++k) {
-            const size_t row = (rec0 + r + k) * GP + h;
-            a[k] = p.rec_acc[row * D + d];
-            w[k] = p.rec_ml[row * 2];
+            a[k] = acc_of(r + k)[d];
+            w[k] = ml_of(r + k)[0];
         }
 #pragma unroll
         for (int k = 0; k < 8; ++k) A = fmaf(a[k], exp2f(w[k] - mref), A);
     }
-    for (; r < nseg; ++r) {
-        const size_t row = (rec0 + r) * GP + h;
-        A = fmaf(p.rec_acc[row * D + d], exp2f(p.rec_ml[row * 2] - mref), A);
-    }
+    for (; r < n; ++r) A = fmaf(acc_of(r)[d], exp2f(ml_of(r)[0] - mref), A);
     const float vsc = p.v_scale ? __ldg(p.v_scale + kvh) : 1.f;
     store_out(p.out, ((size_t)b * p.num_q_heads + hq0 + h) * D + d, S > 0.f ? A * vsc / S : 0.f,
               p.out_dtype);

@@ -64,7 +64,7 @@ __device__ __forceinline__ uint32_t swz(uint32_t base, int row, int col, int hal
 }
 
 template <int D>
-__global__ void __launch_bounds__(kThreadsP)
+__global__ void __launch_bounds__(kThreadsP, 2)
     prefix_kernel(const __grid_constant__ PrefixParams p, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv) {
     using C = PCfg<D>;
@@ -314,111 +314,118 @@ __global__ void __launch_bounds__(kThreadsP)
         const uint32_t svb = skb + C::KV_BYTES;
         const int tbase = c * kPrefixCH;
 
-        // S = Q . K^T: 8 token tiles of 8; K rows (tokens) as the B operand
-        float sc[8][4];
+        // Two halves of 32 tokens, each a full online-softmax step: fewer
+        // live score registers keep two CTAs per SM within the register file.
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
+        for (int hf = 0; hf < 2; ++hf) {
+            // S = Q . K^T over 4 token tiles of 8; K rows (tokens) as the B operand
+            float sc[4][4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) sc[nt][i] = 0.f;
+            for (int nt = 0; nt < 4; ++nt) {
+                const int trow = (hf * 4 + nt) * 8;
 #pragma unroll
-            for (int k2 = 0; k2 < C::KS / 2; ++k2) {
-                uint32_t r[4];
-                ldsm_x4(swz(skb, nt * 8 + kr, k2 * 32 + kq * 8, C::HALF_BYTES), r);
-                mma_bf16(sc[nt], qa[2 * k2], r[0], r[1]);
-                mma_bf16(sc[nt], qa[2 * k2 + 1], r[2], r[3]);
-            }
-        }
-        // mask (chunk tail, bad blocks, each row's own length), scale to log2
-        // units, running max per row (the 4 lanes of a quad share a row)
-        float mxA = -INFINITY, mxB = -INFINITY;
+                for (int i = 0; i < 4; ++i) sc[nt][i] = 0.f;
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int tok = nt * 8 + 2 * tig + (e & 1);
-                bool ok = whole;
-                if (!whole) {
-                    const int jrel = ((tbase + tok) >> p.log2_bs) - (tbase >> p.log2_bs);
-                    ok = tok < ntok && !((bad >> jrel) & 1u);
+                for (int k2 = 0; k2 < C::KS / 2; ++k2) {
+                    uint32_t r[4];
+                    ldsm_x4(swz(skb, trow + kr, k2 * 32 + kq * 8, C::HALF_BYTES), r);
+                    mma_bf16(sc[nt], qa[2 * k2], r[0], r[1]);
+                    mma_bf16(sc[nt], qa[2 * k2 + 1], r[2], r[3]);
                 }
-                ok = ok && tbase + tok < (e < 2 ? LA : LB);
-                const float v = ok ? sc[nt][e] * sl2 : -INFINITY;
-                sc[nt][e] = v;
-                if (e < 2)
-                    mxA = fmaxf(mxA, v);
-                else
-                    mxB = fmaxf(mxB, v);
             }
-        mxA = fmaxf(mxA, __shfl_xor_sync(FULL_MASK, mxA, 1));
-        mxA = fmaxf(mxA, __shfl_xor_sync(FULL_MASK, mxA, 2));
-        mxB = fmaxf(mxB, __shfl_xor_sync(FULL_MASK, mxB, 1));
-        mxB = fmaxf(mxB, __shfl_xor_sync(FULL_MASK, mxB, 2));
-        const float nA = fmaxf(mA, mxA), nB = fmaxf(mB, mxB);
-        const float refA = nA == -INFINITY ? 0.f : nA, refB = nB == -INFINITY ? 0.f : nB;
-        const float alA = exp2f(mA - refA), alB = exp2f(mB - refB);
-        mA = nA;
-        mB = nB;
-        lA *= alA;
-        lB *= alB;
+            // mask (chunk tail, bad blocks, each row's own length), scale to
+            // log2 units, running max per row (the 4 lanes of a quad share a row)
+            float mxA = -INFINITY, mxB = -INFINITY;
 #pragma unroll
-        for (int dt = 0; dt < C::DT; ++dt) {
-            o[dt][0] *= alA;
-            o[dt][1] *= alA;
-            o[dt][2] *= alB;
-            o[dt][3] *= alB;
-        }
+            for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            sc[nt][0] = exp2f(sc[nt][0] - refA);
-            sc[nt][1] = exp2f(sc[nt][1] - refA);
-            sc[nt][2] = exp2f(sc[nt][2] - refB);
-            sc[nt][3] = exp2f(sc[nt][3] - refB);
-            lA += sc[nt][0] + sc[nt][1];
-            lB += sc[nt][2] + sc[nt][3];
-        }
+                for (int e = 0; e < 4; ++e) {
+                    const int tok = (hf * 4 + nt) * 8 + 2 * tig + (e & 1);
+                    bool ok = whole;
+                    if (!whole) {
+                        const int jrel = ((tbase + tok) >> p.log2_bs) - (tbase >> p.log2_bs);
+                        ok = tok < ntok && !((bad >> jrel) & 1u);
+                    }
+                    ok = ok && tbase + tok < (e < 2 ? LA : LB);
+                    const float v = ok ? sc[nt][e] * sl2 : -INFINITY;
+                    sc[nt][e] = v;
+                    if (e < 2)
+                        mxA = fmaxf(mxA, v);
+                    else
+                        mxB = fmaxf(mxB, v);
+                }
+            mxA = fmaxf(mxA, __shfl_xor_sync(FULL_MASK, mxA, 1));
+            mxA = fmaxf(mxA, __shfl_xor_sync(FULL_MASK, mxA, 2));
+            mxB = fmaxf(mxB, __shfl_xor_sync(FULL_MASK, mxB, 1));
+            mxB = fmaxf(mxB, __shfl_xor_sync(FULL_MASK, mxB, 2));
+            const float nA = fmaxf(mA, mxA), nB = fmaxf(mB, mxB);
+            const float refA = nA == -INFINITY ? 0.f : nA, refB = nB == -INFINITY ? 0.f : nB;
+            const float alA = exp2f(mA - refA), alB = exp2f(mB - refB);
+            mA = nA;
+            mB = nB;
+            lA *= alA;
+            lB *= alB;
+#pragma unroll
+            for (int dt = 0; dt < C::DT; ++dt) {
+                o[dt][0] *= alA;
+                o[dt][1] *= alA;
+                o[dt][2] *= alB;
+                o[dt][3] *= alB;
+            }
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                sc[nt][0] = exp2f(sc[nt][0] - refA);
+                sc[nt][1] = exp2f(sc[nt][1] - refA);
+                sc[nt][2] = exp2f(sc[nt][2] - refB);
+                sc[nt][3] = exp2f(sc[nt][3] - refB);
+                lA += sc[nt][0] + sc[nt][1];
+                lB += sc[nt][2] + sc[nt][3];
+            }
 
-        // O += P . V over 4 k-steps of 16 tokens; P from the S accumulator
-        // (token tiles 2kt, 2kt+1), split into bf16 hi + lo
+            // O += P . V over 2 k-steps of 16 tokens; P from the S accumulator
+            // (token tiles 2kt, 2kt+1 of this half), split into bf16 hi + lo
 #pragma unroll
-        for (int kt = 0; kt < 4; ++kt) {
-            uint32_t ph[4], pl[4];
-            {
-                const float* s0 = sc[2 * kt];
-                const float* s1 = sc[2 * kt + 1];
-                ph[0] = pack_bf16(s0[0], s0[1]);
-                ph[1] = pack_bf16(s0[2], s0[3]);
-                ph[2] = pack_bf16(s1[0], s1[1]);
-                ph[3] = pack_bf16(s1[2], s1[3]);
-                pl[0] = pack_bf16(s0[0] - bf16_round(s0[0]), s0[1] - bf16_round(s0[1]));
-                pl[1] = pack_bf16(s0[2] - bf16_round(s0[2]), s0[3] - bf16_round(s0[3]));
-                pl[2] = pack_bf16(s1[0] - bf16_round(s1[0]), s1[1] - bf16_round(s1[1]));
-                pl[3] = pack_bf16(s1[2] - bf16_round(s1[2]), s1[3] - bf16_round(s1[3]));
-            }
-            // V tokens this lane's B fragments carry: 16kt + 2tig (+1), and + 8
-            uint32_t keep0 = 0xffffffffu, keep1 = 0xffffffffu;
-            if (!whole) {
-                auto valid = [&](int tok) {
-                    const int jrel = ((tbase + tok) >> p.log2_bs) - (tbase >> p.log2_bs);
-                    return tok < ntok && !((bad >> jrel) & 1u);
-                };
-                const int t = kt * 16 + 2 * tig;
-                keep0 = (valid(t) ? 0x0000ffffu : 0u) | (valid(t + 1) ? 0xffff0000u : 0u);
-                keep1 = (valid(t + 8) ? 0x0000ffffu : 0u) | (valid(t + 9) ? 0xffff0000u : 0u);
-            }
+            for (int kt = 0; kt < 2; ++kt) {
+                const int t16 = hf * 32 + kt * 16;  // first token of the k-step
+                uint32_t ph[4], pl[4];
+                {
+                    const float* s0 = sc[2 * kt];
+                    const float* s1 = sc[2 * kt + 1];
+                    ph[0] = pack_bf16(s0[0], s0[1]);
+                    ph[1] = pack_bf16(s0[2], s0[3]);
+                    ph[2] = pack_bf16(s1[0], s1[1]);
+                    ph[3] = pack_bf16(s1[2], s1[3]);
+                    pl[0] = pack_bf16(s0[0] - bf16_round(s0[0]), s0[1] - bf16_round(s0[1]));
+                    pl[1] = pack_bf16(s0[2] - bf16_round(s0[2]), s0[3] - bf16_round(s0[3]));
+                    pl[2] = pack_bf16(s1[0] - bf16_round(s1[0]), s1[1] - bf16_round(s1[1]));
+                    pl[3] = pack_bf16(s1[2] - bf16_round(s1[2]), s1[3] - bf16_round(s1[3]));
+                }
+                // V tokens this lane's B fragments carry: t16 + 2tig (+1), and + 8
+                uint32_t keep0 = 0xffffffffu, keep1 = 0xffffffffu;
+                if (!whole) {
+                    auto valid = [&](int tok) {
+                        const int jrel = ((tbase + tok) >> p.log2_bs) - (tbase >> p.log2_bs);
+                        return tok < ntok && !((bad >> jrel) & 1u);
+                    };
+                    const int t = t16 + 2 * tig;
+                    keep0 = (valid(t) ? 0x0000ffffu : 0u) | (valid(t + 1) ? 0xffff0000u : 0u);
+                    keep1 = (valid(t + 8) ? 0x0000ffffu : 0u) | (valid(t + 9) ? 0xffff0000u : 0u);
+                }
 #pragma unroll
-            for (int d2 = 0; d2 < C::DT / 2; ++d2) {
-                uint32_t r[4];
-                ldsm_x4_t(swz(svb, kt * 16 + kr + 8 * (kq & 1), d2 * 16 + 8 * (kq >> 1),
-                              C::HALF_BYTES),
-                          r);
-                r[0] &= keep0;
-                r[1] &= keep1;
-                r[2] &= keep0;
-                r[3] &= keep1;
-                mma_bf16(o[2 * d2], ph, r[0], r[1]);
-                mma_bf16(o[2 * d2], pl, r[0], r[1]);
-                mma_bf16(o[2 * d2 + 1], ph, r[2], r[3]);
-                mma_bf16(o[2 * d2 + 1], pl, r[2], r[3]);
+                for (int d2 = 0; d2 < C::DT / 2; ++d2) {
+                    uint32_t r[4];
+                    ldsm_x4_t(swz(svb, t16 + kr + 8 * (kq & 1), d2 * 16 + 8 * (kq >> 1),
+                                  C::HALF_BYTES),
+                              r);
+                    r[0] &= keep0;
+                    r[1] &= keep1;
+                    r[2] &= keep0;
+                    r[3] &= keep1;
+                    mma_bf16(o[2 * d2], ph, r[0], r[1]);
+                    mma_bf16(o[2 * d2], pl, r[0], r[1]);
+                    mma_bf16(o[2 * d2 + 1], ph, r[2], r[3]);
+                    mma_bf16(o[2 * d2 + 1], pl, r[2], r[3]);
+                }
             }
         }
         __syncwarp();
