@@ -885,79 +885,127 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
 
 // ---- deferred merge (fixed partitions, prefix groups) ---------------------------
 
-// CTA = (request, head group) x a 32-wide slice of head_dim; warp h merges
-// query head h of the group over the parts of its own pass (records of the
-// decode kernel) and the splits of its group's shared prefix pass: lanes own
-// one dimension each, so every record read is one coalesced 128-byte row
-// segment, eight records in flight per lane.
+constexpr int kMergeWarps = 4;  // warps that share one output row
+
+// One CTA per output row (request b, query head): it merges the row over the
+// parts of its own pass (records of the decode kernel) and the splits of its
+// group's shared prefix pass.  The CTA finds the common max M first; then
+// warp w takes records w, w + 4, ... eight at a time (each record row read as
+// one coalesced run of float4 / float2, lane = head_dim/32 dims), and the
+// warps' sums meet in shared memory.
 //   out = vscale * sum_r 2^(m_r - M) acc_r / sum_r 2^(m_r - M) l_r.
 template <int D, int GP>
-__global__ void __launch_bounds__(32 * GP) decode_mma_merge_kernel(const __grid_constant__ DecodeParams p) {
-    constexpr int NSL = D / 32;
-    const int bg = blockIdx.x / NSL, slice = blockIdx.x % NSL;
-    const int b = bg / p.num_hg, hg = bg % p.num_hg;
-    const int kvh = hg / p.num_sub, sub = hg % p.num_sub;
-    const int hq0 = kvh * p.group + sub * GP;
-    const int gv = min(GP, p.group - sub * GP);
-    const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
+__global__ void __launch_bounds__(32 * kMergeWarps)
+    decode_mma_merge_kernel(const __grid_constant__ DecodeParams p) {
+    constexpr int PER = D / 32;  // dims per lane
+    constexpr int NB = 8;        // records in flight per warp
+    __shared__ float red_acc[kMergeWarps][D];
+    __shared__ float red_m[kMergeWarps], red_s[kMergeWarps];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int b = (int)(blockIdx.x / p.num_q_heads), hq = (int)(blockIdx.x % p.num_q_heads);
+    const int kvh = hq / p.group, jg = hq % p.group;
+    const int hg = kvh * p.num_sub + jg / GP, h = jg % GP;
+    const size_t bg = (size_t)b * p.num_hg + hg;
     const int L = clamp_len(p, b, false);
     const int T = seq_begin(p, b, L);
     const int ns = T > 0 ? prefix_num_splits(prefix_tokens_of(p, b), p.pfx_splits) : 0;
     griddep_wait();  // the records and meta of the kernels before
-    if (h >= gv) return;
+    // every condition below is the same in all threads of the CTA
     int u0 = 0, nseg = 0;
     if (L > T) {
-        u0 = p.meta[2 * (size_t)bg];
-        nseg = p.meta[2 * (size_t)bg + 1];
+        u0 = p.meta[2 * bg];
+        nseg = p.meta[2 * bg + 1];
         if (nseg == 0) return;  // did not fit the workspace (flagged by the decode kernel)
         if (u0 < 0 || (long long)bg + u0 + nseg > p.rec_cap) {  // never for a word this call wrote
             if (threadIdx.x == 0) raise_error(p.err, PKV_DEVERR_BAD_SEQ_LEN);
             return;
         }
     }
-    if (nseg + ns == 0) return;  // an empty request: the decode kernel wrote zeros
-    const size_t rec0 = (size_t)bg + u0;
-    // row r < nseg: own record; r >= nseg: split r - nseg of the shared pass
+    const int n = nseg + ns;
+    if (n == 0) return;  // an empty request: the decode kernel wrote zeros
+    const size_t rec0 = bg + u0;
+    // record r < nseg: own part r; r >= nseg: split r - nseg of the shared pass
     auto ml_of = [&](int r) -> const float* {
         return r < nseg ? p.rec_ml + ((rec0 + r) * GP + h) * 2
-                        : p.pfx_ml + (((size_t)(r - nseg) * p.num_seqs + b) * p.num_q_heads +
-                                      hq0 + h) * 2;
+                        : p.pfx_ml + (((size_t)(r - nseg) * p.num_seqs + b) * p.num_q_heads + hq) * 2;
     };
     auto acc_of = [&](int r) -> const float* {
         return r < nseg ? p.rec_acc + ((rec0 + r) * GP + h) * D
-                        : p.pfx_acc + (((size_t)(r - nseg) * p.num_seqs + b) * p.num_q_heads +
-                                       hq0 + h) * D;
+                        : p.pfx_acc + (((size_t)(r - nseg) * p.num_seqs + b) * p.num_q_heads + hq) * D;
     };
-    const int n = nseg + ns;
-    float M = -INFINITY;
-    for (int r = lane; r < n; r += 32) M = fmaxf(M, ml_of(r)[0]);
+    auto load_row = [&](const float* acc, float (&v)[PER]) {
+        if constexpr (PER == 4) {
+            const float4 t = *reinterpret_cast<const float4*>(acc + lane * 4);
+            v[0] = t.x;
+            v[1] = t.y;
+            v[2] = t.z;
+            v[3] = t.w;
+        } else {
+            const float2 t = *reinterpret_cast<const float2*>(acc + lane * 2);
+            v[0] = t.x;
+            v[1] = t.y;
+        }
+    };
+    // the common max
+    float m = -INFINITY;
+    for (int r = threadIdx.x; r < n; r += 32 * kMergeWarps) m = fmaxf(m, ml_of(r)[0]);
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL_MASK, M, off));
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL_MASK, m, off));
+    if (lane == 0) red_m[warp] = m;
+    __syncthreads();
+    float M = red_m[0];
+#pragma unroll
+    for (int w = 1; w < kMergeWarps; ++w) M = fmaxf(M, red_m[w]);
     const float mref = M == -INFINITY ? 0.f : M;
-    float S = 0.f;
-    for (int r = lane; r < n; r += 32) {
-        const float* ml = ml_of(r);
-        S += ml[1] * exp2f(ml[0] - mref);
-    }
+    // this warp's records
+    float A[PER], S = 0.f;
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) S += __shfl_xor_sync(FULL_MASK, S, off);
-    const int d = slice * 32 + lane;
-    float A = 0.f;
-    int r = 0;
-    for (; r + 8 <= n; r += 8) {
-        float a[8], w[8];
+    for (int i = 0; i < PER; ++i) A[i] = 0.f;
+    int r = warp;
+    for (; r + kMergeWarps * (NB - 1) < n; r += kMergeWarps * NB) {
+        float v[NB][PER], mm[NB], ll[NB];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            a[k] = acc_of(r + k)[d];
-            w[k] = ml_of(r + k)[0];
+        for (int q = 0; q < NB; ++q) {
+            const float* ml = ml_of(r + kMergeWarps * q);
+            mm[q] = ml[0];
+            ll[q] = ml[1];
+            load_row(acc_of(r + kMergeWarps * q), v[q]);
         }
 #pragma unroll
-        for (int k = 0; k < 8; ++k) A = fmaf(a[k], exp2f(w[k] - mref), A);
+        for (int q = 0; q < NB; ++q) {
+            const float wq = exp2f(mm[q] - mref);
+            S = fmaf(ll[q], wq, S);
+#pragma unroll
+            for (int i = 0; i < PER; ++i) A[i] = fmaf(v[q][i], wq, A[i]);
+        }
     }
-    for (; r < n; ++r) A = fmaf(acc_of(r)[d], exp2f(ml_of(r)[0] - mref), A);
+    for (; r < n; r += kMergeWarps) {
+        const float* ml = ml_of(r);
+        const float wq = exp2f(ml[0] - mref);
+        S = fmaf(ml[1], wq, S);
+        float v[PER];
+        load_row(acc_of(r), v);
+#pragma unroll
+        for (int i = 0; i < PER; ++i) A[i] = fmaf(v[i], wq, A[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < PER; ++i) red_acc[warp][lane * PER + i] = A[i];
+    if (lane == 0) red_s[warp] = S;
+    __syncthreads();
+    if (warp != 0) return;
+    float St = 0.f;
+#pragma unroll
+    for (int w = 0; w < kMergeWarps; ++w) St += red_s[w];
     const float vsc = p.v_scale ? __ldg(p.v_scale + kvh) : 1.f;
-    store_out(p.out, ((size_t)b * p.num_q_heads + hq0 + h) * D + d, S > 0.f ? A * vsc / S : 0.f,
-              p.out_dtype);
+    const float inv = St > 0.f ? vsc / St : 0.f;
+    const size_t orow = ((size_t)b * p.num_q_heads + hq) * D + lane * PER;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+        float t = 0.f;
+#pragma unroll
+        for (int w = 0; w < kMergeWarps; ++w) t += red_acc[w][lane * PER + i];
+        store_out(p.out, orow + i, t * inv, p.out_dtype);
+    }
 }
 
 // ---- host side ---------------------------------------------------------------
@@ -998,9 +1046,9 @@ pkv_status launch_impl(const DecodeParams& p, cudaStream_t stream, int* grid_out
     if (cudaLaunchKernelEx(&L.cfg, kern, p, tmk, tmv) != cudaSuccess) return PKV_ERR_CUDA;
     if (p.defer_merge) {
         constexpr int GP = MmaCfg<D, NT, F8>::GP;
-        const long long mgrid = (long long)p.num_seqs * p.num_hg * (D / 32);
+        const long long mgrid = (long long)p.num_seqs * p.num_q_heads;  // one CTA per output row
         if (mgrid > 0x7fffffffLL) return PKV_ERR_UNSUPPORTED;
-        PdlLaunch M(dim3((unsigned)mgrid), dim3(32 * GP), 0, stream);
+        PdlLaunch M(dim3((unsigned)mgrid), dim3(32 * kMergeWarps), 0, stream);
         if (cudaLaunchKernelEx(&M.cfg, decode_mma_merge_kernel<D, GP>, p) != cudaSuccess)
             return PKV_ERR_CUDA;
     }
