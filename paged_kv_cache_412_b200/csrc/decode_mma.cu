@@ -47,7 +47,6 @@ namespace {
 
 constexpr int kCH = 64;         // tokens per stage
 constexpr int kMT = kCH / 16;   // 16-token MMA tiles per stage
-constexpr int kThreads = 96;    // producer, tensor-core consumer, epilogue
 constexpr int kRingBudget = 104448;  // 3 stages of K+V+q at head_dim 128
 
 constexpr int cmin(int a, int b) { return a < b ? a : b; }
@@ -63,12 +62,23 @@ struct MmaCfg {
     static constexpr int KS = D / 16;               // k-steps of q.K^T, m-tiles of P.V
     static constexpr int HALF_BYTES = kCH * 128;    // one swizzled half region (16-bit data)
     static constexpr int KV_BYTES = F8 ? kCH * D : NHALF * HALF_BYTES;  // K (or V) of a stage
-    static constexpr int STG_BYTES = F8 ? 2 * NHALF * HALF_BYTES : 0;  // f16 K+V staging
     static constexpr int GP = 8 * NT;               // query heads per head group (padded)
-    static constexpr int Q_BYTES = GP * D * 2;      // the group's q rows (first stage of a segment)
+    static constexpr int Q_BYTES = GP * D * 2;      // the group's q rows (first stages of a segment)
     // K | V | q, rounded to the 1 KB the 128-byte swizzle pattern repeats on
     static constexpr int STAGE_BYTES = (2 * KV_BYTES + Q_BYTES + 1023) / 1024 * 1024;
-    static constexpr int NSTAGE = cmax(2, cmin(8, (kRingBudget - STG_BYTES) / STAGE_BYTES));
+    // bf16: one tensor-core consumer reads the TMA stages directly (two CTAs
+    // per SM).  fp8: NCONS consumers own one f16 staging slot each and take
+    // the CTA's chunks in turn (chunk n -> consumer n % NCONS), and NCV
+    // converter warps widen every fp8 stage into the slot of the consumer that
+    // takes it (one CTA per SM).  Each barrier then has one waiter stepping
+    // through its phases in order.
+    static constexpr int NCONS = F8 ? (NT == 1 ? 3 : 2) : 1;
+    static constexpr int NCV = F8 ? 4 : 0;
+    static constexpr int THREADS = 32 * (2 + NCONS + NCV);  // + producer, epilogue
+    static constexpr int QCH = NCONS;  // a segment's first QCH chunks carry the group's q
+    static constexpr int SLOT_BYTES = F8 ? (2 * NHALF * HALF_BYTES + Q_BYTES + 1023) / 1024 * 1024 : 0;
+    static constexpr int STG_BYTES = NCONS * SLOT_BYTES;   // f16 K | V | q per consumer
+    static constexpr int NSTAGE = F8 ? 4 : cmax(2, cmin(8, kRingBudget / STAGE_BYTES));
 };
 
 // ---- shared-memory layout ------------------------------------------------------
@@ -76,15 +86,19 @@ struct MmaCfg {
 template <int D, int NT, bool F8>
 struct Smem {
     using C = MmaCfg<D, NT, F8>;
-    static constexpr int NDUMP = 2;                       // consumer -> epilogue hand-off slots
+    // consumer -> epilogue hand-off slots per consumer
+    static constexpr int NDUMP = C::NCONS == 1 ? 2 : 1;
+    static constexpr int NSLOT = C::NCONS * NDUMP;
     static constexpr int DUMP_ACC = C::KS * NT * 4;       // acc registers per lane
     static constexpr int DUMP_ML = NT * 4;                // m[2], l[2] per n-tile per lane
     static constexpr int DUMP_BYTES = (DUMP_ACC + DUMP_ML) * 32 * 4;
     static constexpr int OFF_STG = C::NSTAGE * C::STAGE_BYTES;
     static constexpr int OFF_DUMP = OFF_STG + C::STG_BYTES;
-    static constexpr int OFF_BAR = OFF_DUMP + NDUMP * DUMP_BYTES;
-    static constexpr int OFF_META = OFF_BAR + (2 * C::NSTAGE + 2 * NDUMP) * 8;
-    static constexpr int OFF_CTRL = OFF_META + 2 * C::NSTAGE * 4;
+    static constexpr int OFF_BAR = OFF_DUMP + NSLOT * DUMP_BYTES;
+    // full/empty per stage, dfull/dempty per dump slot, sfull/sempty per staging slot
+    static constexpr int OFF_META = OFF_BAR + (2 * C::NSTAGE + 2 * NSLOT + 2 * C::NCONS) * 8;
+    // ntok/bad per stage, then per staging slot
+    static constexpr int OFF_CTRL = OFF_META + 2 * (C::NSTAGE + C::NCONS) * 4;
     static constexpr int BYTES = OFF_CTRL + 16 + 1024;   // + alignment slack
 };
 
@@ -174,17 +188,22 @@ struct Producer {
                 st_ntok[ring.stage] = ntok;
                 st_bad[ring.stage] = bad;
                 if (bad) raise_error(p.err, PKV_DEVERR_BAD_BLOCK);
-                const uint32_t qbytes = c == sg.c0 ? (uint32_t)gv * D * 2u : 0u;
+                const uint32_t qbytes = c - sg.c0 < C::QCH ? (uint32_t)gv * D * 2u : 0u;
                 const uint32_t row_bytes = F8 ? (uint32_t)D : (uint32_t)C::NHALF * 128u;
                 mbar_arrive_expect_tx(&full[ring.stage], nvalid * 2u * rb * row_bytes + qbytes);
-                if (qbytes)  // the group's q rows ride with the segment's first stage
+                if (qbytes)  // the group's q rows ride with the segment's first stage(s)
                     bulk_load(sq, static_cast<const __nv_bfloat16*>(p.q) +
                                       ((size_t)cur.b * p.num_q_heads + hq0) * D,
                               qbytes, &full[ring.stage], policy);
             }
-            for (int j = ja; j <= jb; ++j) {
-                const int phys = __shfl_sync(FULL_MASK, tab, j - wbase);
-                if (lane == 0 && phys >= 0 && phys < p.num_blocks) {
+            // One lane per block of the chunk issues that block's copies: a TMA
+            // issue costs the issuing thread ~0.1 us, so lane-parallel issue
+            // keeps the copies of a chunk from queueing behind each other.
+            __syncwarp();  // the expect-tx above comes first
+            {
+                const int j = ja + lane;
+                const int phys = __shfl_sync(FULL_MASK, tab, min(j, jb) - wbase);
+                if (j <= jb && phys >= 0 && phys < p.num_blocks) {
                     // rows of this block in the stage, and where they start in the cache
                     const int srow = (j << p.log2_bs) - t0 > 0 ? (j << p.log2_bs) - t0 : 0;
                     const int boff = t0 - (j << p.log2_bs) > 0 ? t0 - (j << p.log2_bs) : 0;
@@ -271,21 +290,29 @@ __device__ __forceinline__ SegInfo seg_info(const DecodeParams& p, const Segment
 
 // ---- consumer (tensor-core math) ----------------------------------------------
 
+// Consumer `me` (0 .. NCONS-1).  bf16: reads every TMA stage in turn.  fp8:
+// takes the CTA's chunks n with n % NCONS == me from its own f16 staging slot
+// (sfull/sempty), where the converter warps put K, V and, for a segment's
+// first chunks, q.
 template <int D, int NT, bool F8>
 __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                                         unsigned char* smem, uint64_t* full, uint64_t* empty,
-                                        uint64_t* dfull, uint64_t* dempty, const int* st_ntok,
-                                        const unsigned* st_bad, volatile int* ctrl, int lane) {
+                                        uint64_t* dfull, uint64_t* dempty, uint64_t* sfull,
+                                        uint64_t* sempty, const int* st_ntok,
+                                        const unsigned* st_bad, const int* sl_ntok,
+                                        const unsigned* sl_bad, volatile int* ctrl, int lane,
+                                        int me) {
     using C = MmaCfg<D, NT, F8>;
     using S = Smem<D, NT, F8>;
     constexpr int GP = C::GP;
     const int grp = lane >> 2, tig = lane & 3;
     const int mi = lane >> 3, r8 = lane & 7;
-    unsigned char* stg = smem + S::OFF_STG;  // f16 staging (fp8 caches only)
     // ldmatrix row/chunk components that depend only on the lane
     const int k_row = r8 + 8 * (mi & 1), k_cx = mi >> 1;  // K (A operand)
     const int v_row = r8 + 8 * (mi >> 1), v_cx = mi & 1;  // V^T (A operand, transposed load)
     Ring ring, dring;
+    uint32_t sphase = 0;   // fp8: phase of this consumer's staging slot
+    unsigned n_chunk = 0;  // fp8: chunks of the CTA so far
 
     while (it.valid) {
         const Segment sg = it.current();
@@ -306,23 +333,46 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                 for (int i = 0; i < 4; ++i) acc[dt][nt][i] = 0.f;
         }
 
+        bool have_q = false;
         for (int c = sg.c0; c < sg.c1; ++c) {
-            if (ctrl[0] || !mbar_wait(&full[ring.stage], ring.phase)) {
-                if (lane == 0 && !ctrl[0]) {
-                    ctrl[0] = 1;
-                    raise_error(p.err, PKV_DEVERR_TIMEOUT);
+            int ntok;
+            unsigned bad;
+            unsigned char* sk;
+            if constexpr (F8) {
+                const bool mine = (int)(n_chunk % C::NCONS) == me;
+                ++n_chunk;
+                if (!mine) continue;
+                if (ctrl[0] || !mbar_wait(&sfull[me], sphase)) {
+                    if (lane == 0 && !ctrl[0]) {
+                        ctrl[0] = 1;
+                        raise_error(p.err, PKV_DEVERR_TIMEOUT);
+                    }
+                    return;
                 }
-                return;
+                ntok = sl_ntok[me];
+                bad = sl_bad[me];
+                sk = smem + S::OFF_STG + me * C::SLOT_BYTES;
+            } else {
+                if (ctrl[0] || !mbar_wait(&full[ring.stage], ring.phase)) {
+                    if (lane == 0 && !ctrl[0]) {
+                        ctrl[0] = 1;
+                        raise_error(p.err, PKV_DEVERR_TIMEOUT);
+                    }
+                    return;
+                }
+                ntok = st_ntok[ring.stage];
+                bad = st_bad[ring.stage];
+                sk = smem + ring.stage * C::STAGE_BYTES;
             }
-            const int ntok = st_ntok[ring.stage];
-            const unsigned bad = st_bad[ring.stage];
             const bool whole = ntok == kCH && bad == 0;
-            unsigned char* sk = smem + ring.stage * C::STAGE_BYTES;
-            unsigned char* sv = sk + C::KV_BYTES;
+            // 16-bit K | V | q (a bf16 stage, or an fp8 chunk's f16 staging slot)
+            unsigned char* sv = sk + C::NHALF * C::HALF_BYTES;
 
-            if (c == sg.c0) {
+            if (!have_q) {
+                // This consumer's first chunk of the segment carries the group's q.
                 // Q^T B-fragments: head nt*8+grp, dims ks*16 + 2*tig (+1) and +8 (+9).
-                const uint32_t* sq = reinterpret_cast<const uint32_t*>(sv + C::KV_BYTES);
+                have_q = true;
+                const uint32_t* sq = reinterpret_cast<const uint32_t*>(sv + C::NHALF * C::HALF_BYTES);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     const int h = nt * 8 + grp;
@@ -340,40 +390,6 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                 }
             }
 
-            if constexpr (F8) {
-                // Widen the stage's e4m3 K and V rows to f16 in the swizzled
-                // staging tile; tokens that do not take part become zero rows.
-                // The fp8 stage is then free for the next copy.
-#pragma unroll 4
-                for (int idx = lane; idx < 2 * kCH * (D / 16); idx += 32) {
-                    const int part = idx / (kCH * (D / 16));
-                    const int rest = idx % (kCH * (D / 16));
-                    const int row = rest / (D / 16), c16 = rest % (D / 16);
-                    bool valid = whole;
-                    if (!whole) {
-                        const int jrel = ((c * kCH + row) >> p.log2_bs) - ((c * kCH) >> p.log2_bs);
-                        valid = row < ntok && !((bad >> jrel) & 1u);
-                    }
-                    uint4 o0 = make_uint4(0, 0, 0, 0), o1 = make_uint4(0, 0, 0, 0);
-                    if (valid) {
-                        const uint4 raw = *reinterpret_cast<const uint4*>(
-                            (part ? sv : sk) + row * D + c16 * 16);
-                        e4m3x4_to_f16(raw.x, o0.x, o0.y);
-                        e4m3x4_to_f16(raw.y, o0.z, o0.w);
-                        e4m3x4_to_f16(raw.z, o1.x, o1.y);
-                        e4m3x4_to_f16(raw.w, o1.z, o1.w);
-                    }
-                    const int half = (c16 * 16) >> 6, cc = ((c16 * 16) & 63) >> 3;
-                    unsigned char* dst = stg + part * C::NHALF * C::HALF_BYTES +
-                                         half * C::HALF_BYTES + row * 128;
-                    *reinterpret_cast<uint4*>(dst + ((cc ^ (row & 7)) << 4)) = o0;
-                    *reinterpret_cast<uint4*>(dst + (((cc + 1) ^ (row & 7)) << 4)) = o1;
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[ring.stage]);
-                sk = stg;
-                sv = stg + C::NHALF * C::HALF_BYTES;
-            }
             const uint32_t skb = smem_addr(sk), svb = smem_addr(sv);
 
             if (!F8 && !whole) {
@@ -512,21 +528,26 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                 if (!whole) fence_proxy_async_smem();  // our zero-fill before the next TMA write
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[ring.stage]);
+                ring.advance(C::NSTAGE);
             } else {
-                __syncwarp();  // staging tile reads done before the next widening
+                __syncwarp();  // slot reads done before the converters refill it
+                if (lane == 0) mbar_arrive(&sempty[me]);
+                sphase ^= 1u;
             }
-            ring.advance(C::NSTAGE);
         }
 
         // ---- hand the segment's state to the epilogue warp ----
-        if (!mbar_wait(&dempty[dring.stage], dring.phase ^ 1u)) {
+        // (an fp8 consumer that took no chunk of the segment hands over the
+        // empty state)
+        const int slot = me * S::NDUMP + dring.stage;
+        if (!mbar_wait(&dempty[slot], dring.phase ^ 1u)) {
             if (lane == 0) {
                 ctrl[0] = 1;
                 raise_error(p.err, PKV_DEVERR_TIMEOUT);
             }
             return;
         }
-        float* dump = reinterpret_cast<float*>(smem + S::OFF_DUMP + dring.stage * S::DUMP_BYTES);
+        float* dump = reinterpret_cast<float*>(smem + S::OFF_DUMP + slot * S::DUMP_BYTES);
 #pragma unroll
         for (int dt = 0; dt < C::KS; ++dt)
 #pragma unroll
@@ -541,8 +562,100 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                 dump[(S::DUMP_ACC + nt * 4 + 2 + j) * 32 + lane] = l[nt][j];
             }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&dfull[dring.stage]);
+        if (lane == 0) mbar_arrive(&dfull[slot]);
         dring.advance(S::NDUMP);
+    }
+}
+
+// ---- converters (fp8 caches) ----------------------------------------------------
+
+// Converter v (0 .. NCV-1) widens rows v*16 .. v*16+15 of every fp8 stage's K
+// and V (exactly, e4m3 -> f16) into the swizzled staging slot of the consumer
+// that takes the chunk; tokens that do not take part (past the end, or in a
+// block the table got wrong) become zero rows.  Converter 0 also copies the
+// group's q rows and the chunk's token count / bad-block mask into the slot.
+template <int D, int NT>
+__device__ __forceinline__ void convert(const DecodeParams& p, SegIter<kCH>& it,
+                                        unsigned char* smem, uint64_t* full, uint64_t* empty,
+                                        uint64_t* sfull, uint64_t* sempty, const int* st_ntok,
+                                        const unsigned* st_bad, int* sl_ntok, unsigned* sl_bad,
+                                        volatile int* ctrl, int lane, int v) {
+    using C = MmaCfg<D, NT, true>;
+    using S = Smem<D, NT, true>;
+    constexpr int RPW = kCH / C::NCV;              // rows of K (and of V) per converter
+    constexpr int C16 = D / 16;                    // 16-code groups per row
+    constexpr int PER_LANE = 2 * RPW * C16 / 32;
+    static_assert(2 * RPW * C16 % 32 == 0, "whole lanes");
+    Ring ring;
+    unsigned n_chunk = 0;
+    while (it.valid) {
+        const Segment sg = it.current();
+        it.advance(p, lane);
+        for (int c = sg.c0; c < sg.c1; ++c, ++n_chunk) {
+            const int slot = (int)(n_chunk % C::NCONS);
+            const uint32_t sph = (n_chunk / C::NCONS) & 1u;
+            if (ctrl[0] || !mbar_wait(&full[ring.stage], ring.phase) ||
+                !mbar_wait(&sempty[slot], sph ^ 1u)) {
+                if (lane == 0 && !ctrl[0]) {
+                    ctrl[0] = 1;
+                    raise_error(p.err, PKV_DEVERR_TIMEOUT);
+                }
+                return;
+            }
+            const int ntok = st_ntok[ring.stage];
+            const unsigned bad = st_bad[ring.stage];
+            const bool whole = ntok == kCH && bad == 0;
+            const unsigned char* sk = smem + ring.stage * C::STAGE_BYTES;  // e4m3 rows of D bytes
+            const unsigned char* sv = sk + C::KV_BYTES;
+            unsigned char* dst0 = smem + S::OFF_STG + slot * C::SLOT_BYTES;
+#pragma unroll
+            for (int i = 0; i < PER_LANE; ++i) {
+                const int idx = lane + 32 * i;
+                const int part = idx / (RPW * C16);
+                const int rest = idx % (RPW * C16);
+                const int row = v * RPW + rest / C16, c16 = rest % C16;
+                bool valid = whole;
+                if (!whole) {
+                    const int jrel = ((c * kCH + row) >> p.log2_bs) - ((c * kCH) >> p.log2_bs);
+                    valid = row < ntok && !((bad >> jrel) & 1u);
+                }
+                uint4 o0 = make_uint4(0, 0, 0, 0), o1 = make_uint4(0, 0, 0, 0);
+                if (valid) {
+                    // the code row is stored swizzled: 16-byte group c16 of row
+                    // r sits at c16 ^ (r % 8) (128-byte rows) or ^ (r / 2 % 4)
+                    // (64-byte rows)
+                    const int sw = D == 128 ? (row & 7) : ((row >> 1) & 3);
+                    const uint4 raw = *reinterpret_cast<const uint4*>((part ? sv : sk) + row * D +
+                                                                      ((c16 ^ sw) << 4));
+                    e4m3x4_to_f16(raw.x, o0.x, o0.y);
+                    e4m3x4_to_f16(raw.y, o0.z, o0.w);
+                    e4m3x4_to_f16(raw.z, o1.x, o1.y);
+                    e4m3x4_to_f16(raw.w, o1.z, o1.w);
+                }
+                const int half = (c16 * 16) >> 6, cc = ((c16 * 16) & 63) >> 3;
+                unsigned char* dst = dst0 + part * C::NHALF * C::HALF_BYTES +
+                                     half * C::HALF_BYTES + row * 128;
+                *reinterpret_cast<uint4*>(dst + ((cc ^ (row & 7)) << 4)) = o0;
+                *reinterpret_cast<uint4*>(dst + (((cc + 1) ^ (row & 7)) << 4)) = o1;
+            }
+            if (v == 0) {
+                if (c - sg.c0 < C::QCH) {
+                    const uint4* qs = reinterpret_cast<const uint4*>(sv + C::KV_BYTES);
+                    uint4* qd = reinterpret_cast<uint4*>(dst0 + 2 * C::NHALF * C::HALF_BYTES);
+                    for (int i = lane; i < C::Q_BYTES / 16; i += 32) qd[i] = qs[i];
+                }
+                if (lane == 0) {
+                    sl_ntok[slot] = ntok;
+                    sl_bad[slot] = bad;
+                }
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&empty[ring.stage]);
+                mbar_arrive(&sfull[slot]);
+            }
+            ring.advance(C::NSTAGE);
+        }
     }
 }
 
@@ -606,31 +719,62 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
         it.advance(p, lane);
         const SegInfo si = seg_info<GP>(p, sg, it.W);
         const float vsc = F8 ? __ldg(p.v_scale + si.kvh) : 1.f;  // V dequantisation scale
-        if (ctrl[0] || !mbar_wait(&dfull[dring.stage], dring.phase)) {
-            if (lane == 0 && !ctrl[0]) {
-                ctrl[0] = 1;
-                raise_error(p.err, PKV_DEVERR_TIMEOUT);
-            }
-            return;
-        }
-        const float* dump =
-            reinterpret_cast<const float*>(smem + S::OFF_DUMP + dring.stage * S::DUMP_BYTES);
+        // the segment's state: one consumer's, or the merge of NCONS consumers'
         float acc[C::KS][NT][4], m[NT][2], l[NT][2];
 #pragma unroll
-        for (int dt = 0; dt < C::KS; ++dt)
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) acc[dt][nt][i] = dump[((dt * NT + nt) * 4 + i) * 32 + lane];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                m[nt][j] = dump[(S::DUMP_ACC + nt * 4 + j) * 32 + lane];
-                l[nt][j] = dump[(S::DUMP_ACC + nt * 4 + 2 + j) * 32 + lane];
+        for (int k = 0; k < C::NCONS; ++k) {
+            const int slot = k * S::NDUMP + dring.stage;
+            if (ctrl[0] || !mbar_wait(&dfull[slot], dring.phase)) {
+                if (lane == 0 && !ctrl[0]) {
+                    ctrl[0] = 1;
+                    raise_error(p.err, PKV_DEVERR_TIMEOUT);
+                }
+                return;
             }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&dempty[dring.stage]);
+            const float* dump =
+                reinterpret_cast<const float*>(smem + S::OFF_DUMP + slot * S::DUMP_BYTES);
+            if (k == 0) {
+#pragma unroll
+                for (int dt = 0; dt < C::KS; ++dt)
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            acc[dt][nt][i] = dump[((dt * NT + nt) * 4 + i) * 32 + lane];
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        m[nt][j] = dump[(S::DUMP_ACC + nt * 4 + j) * 32 + lane];
+                        l[nt][j] = dump[(S::DUMP_ACC + nt * 4 + 2 + j) * 32 + lane];
+                    }
+            } else {
+                // combine with consumer k's state of the same segment (its
+                // running max is common to the lanes of a head, like ours)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                    for (int j = 0; j < 2; ++j) {
+                        const float mk = dump[(S::DUMP_ACC + nt * 4 + j) * 32 + lane];
+                        const float lk = dump[(S::DUMP_ACC + nt * 4 + 2 + j) * 32 + lane];
+                        const float M = fmaxf(m[nt][j], mk);
+                        const float mref = M == -INFINITY ? 0.f : M;
+                        const float fa = exp2f(m[nt][j] - mref), fb = exp2f(mk - mref);
+                        l[nt][j] = l[nt][j] * fa + lk * fb;
+#pragma unroll
+                        for (int dt = 0; dt < C::KS; ++dt) {
+                            acc[dt][nt][j] = acc[dt][nt][j] * fa +
+                                             dump[((dt * NT + nt) * 4 + j) * 32 + lane] * fb;
+                            acc[dt][nt][j + 2] =
+                                acc[dt][nt][j + 2] * fa +
+                                dump[((dt * NT + nt) * 4 + j + 2) * 32 + lane] * fb;
+                        }
+                        m[nt][j] = M;
+                    }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&dempty[slot]);
+        }
         dring.advance(S::NDUMP);
 
         // the normaliser: sum the per-lane partials over the lanes sharing a head
@@ -818,7 +962,8 @@ __device__ __forceinline__ long long total_chunks_warp(const DecodeParams& p, in
 }
 
 template <int D, int NT, bool F8>
-__global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_constant__ DecodeParams p,
+__global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
+    decode_mma_kernel(const __grid_constant__ DecodeParams p,
                                                              const __grid_constant__ CUtensorMap tmk,
                                                              const __grid_constant__ CUtensorMap tmv) {
     using C = MmaCfg<D, NT, F8>;
@@ -828,9 +973,13 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
     uint64_t* empty = full + C::NSTAGE;
     uint64_t* dfull = empty + C::NSTAGE;
-    uint64_t* dempty = dfull + S::NDUMP;
+    uint64_t* dempty = dfull + S::NSLOT;
+    uint64_t* sfull = dempty + S::NSLOT;  // fp8 staging slots
+    uint64_t* sempty = sfull + C::NCONS;
     int* st_ntok = reinterpret_cast<int*>(smem + S::OFF_META);
     unsigned* st_bad = reinterpret_cast<unsigned*>(st_ntok + C::NSTAGE);
+    int* sl_ntok = reinterpret_cast<int*>(st_bad + C::NSTAGE);
+    unsigned* sl_bad = reinterpret_cast<unsigned*>(sl_ntok + C::NCONS);
     volatile int* ctrl = reinterpret_cast<volatile int*>(smem + S::OFF_CTRL);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -838,11 +987,15 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
         ctrl[0] = 0;
         for (int s = 0; s < C::NSTAGE; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], F8 ? C::NCV : 1);  // released by the converters (fp8)
         }
-        for (int s = 0; s < S::NDUMP; ++s) {
+        for (int s = 0; s < S::NSLOT; ++s) {
             mbar_init(&dfull[s], 1);
             mbar_init(&dempty[s], 1);
+        }
+        for (int s = 0; s < C::NCONS; ++s) {
+            mbar_init(&sfull[s], C::NCV);
+            mbar_init(&sempty[s], 1);
         }
         fence_mbar_init();
         prefetch_tensormap(&tmk);
@@ -859,7 +1012,7 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
     const long long total =
         total_chunks_warp(p, lane, blockIdx.x == 0 && warp == 0, &L_first, &T_first);
     if (total == 0) {
-        if (warp == 2) {
+        if (warp == C::NCONS + 1) {
             SegIter<kCH> none;
             none.valid = false;
             epilogue<D, NT, F8>(p, none, smem, dfull, dempty, ctrl, lane);
@@ -876,10 +1029,15 @@ __global__ void __launch_bounds__(kThreads) decode_mma_kernel(const __grid_const
                            l2_policy_evict_first()};
         pr.run(it);
         if (!pr.waited) griddep_wait();
-    } else if (warp == 1) {
-        consume<D, NT, F8>(p, it, smem, full, empty, dfull, dempty, st_ntok, st_bad, ctrl, lane);
-    } else {
+    } else if (warp <= C::NCONS) {
+        consume<D, NT, F8>(p, it, smem, full, empty, dfull, dempty, sfull, sempty, st_ntok, st_bad,
+                           sl_ntok, sl_bad, ctrl, lane, warp - 1);
+    } else if (warp == C::NCONS + 1) {
         epilogue<D, NT, F8>(p, it, smem, dfull, dempty, ctrl, lane);
+    } else {
+        if constexpr (C::NCV > 0)
+            convert<D, NT>(p, it, smem, full, empty, sfull, sempty, st_ntok, st_bad, sl_ntok,
+                           sl_bad, ctrl, lane, warp - C::NCONS - 2);
     }
 }
 
@@ -1012,6 +1170,7 @@ __global__ void __launch_bounds__(32 * kMergeWarps)
 
 template <int D, int NT, bool F8>
 pkv_status launch_impl(const DecodeParams& p, cudaStream_t stream, int* grid_out) {
+    using C = MmaCfg<D, NT, F8>;
     using S = Smem<D, NT, F8>;
     const DeviceInfo* di = current_device_info();
     if (!di) return PKV_ERR_CUDA;
@@ -1027,7 +1186,7 @@ pkv_status launch_impl(const DecodeParams& p, cudaStream_t stream, int* grid_out
                 cudaSuccess)
                 return PKV_ERR_CUDA;
             int occ = 0;
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kThreads, S::BYTES) !=
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, C::THREADS, S::BYTES) !=
                     cudaSuccess ||
                 occ < 1)
                 return PKV_ERR_CUDA;
@@ -1042,7 +1201,7 @@ pkv_status launch_impl(const DecodeParams& p, cudaStream_t stream, int* grid_out
         return PKV_ERR_CUDA;
     const int grid = di->num_sms * std::min(occupancy[di->device], 4);
 
-    PdlLaunch L(dim3(grid), dim3(kThreads), S::BYTES, stream);
+    PdlLaunch L(dim3(grid), dim3(C::THREADS), S::BYTES, stream);
     if (cudaLaunchKernelEx(&L.cfg, kern, p, tmk, tmv) != cudaSuccess) return PKV_ERR_CUDA;
     if (p.defer_merge) {
         constexpr int GP = MmaCfg<D, NT, F8>::GP;
@@ -1074,8 +1233,8 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // 2-D view of a cache: rows = num_blocks*Hkv*block_size, columns = head_dim
 // bf16; boxes of 64 columns x min(block_size, 64) rows, 128-byte swizzle.
-// fp8: rows of head_dim one-byte codes, whole-row boxes, no swizzle (the
-// consumer reads them linearly while widening them).
+// fp8: rows of head_dim one-byte codes, whole-row boxes with the swizzle of
+// their width (128 bytes at head_dim 128, 64 at 64); the converters undo it.
 bool encode_cache_map(CUtensorMap* map, const void* base, long long rows, int head_dim,
                       int box_rows, bool fp8) {
     auto enc = tensor_map_encoder();
@@ -1087,7 +1246,8 @@ bool encode_cache_map(CUtensorMap* map, const void* base, long long rows, int he
     const CUresult r = enc(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                            2, const_cast<void*>(base), gdim, gstride, box, estride,
                            CU_TENSOR_MAP_INTERLEAVE_NONE,
-                           fp8 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+                           (fp8 && head_dim == 64) ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                   : CU_TENSOR_MAP_SWIZZLE_128B,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }

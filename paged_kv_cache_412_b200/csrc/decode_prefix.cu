@@ -225,9 +225,13 @@ __global__ void __launch_bounds__(kThreadsP, 2)
             }
             unsigned char* sk = smem + ring.stage * C::STAGE_BYTES;
             unsigned char* sv = sk + C::KV_BYTES;
-            for (int j = ja; j <= jb; ++j) {
-                const int phys = __shfl_sync(FULL_MASK, tab, j - ja);
-                if (lane == 0 && phys >= 0 && phys < p.num_blocks) {
+            // one lane per block issues that block's copies (a TMA issue costs
+            // the issuing thread ~0.1 us; lane-parallel issue overlaps them)
+            __syncwarp();  // the expect-tx above comes first
+            {
+                const int j = ja + lane;
+                const int phys = __shfl_sync(FULL_MASK, tab, min(j, jb) - ja);
+                if (j <= jb && phys >= 0 && phys < p.num_blocks) {
                     // t0 is a multiple of 64 and of block_size when block_size <= 64
                     const int srow = max((j << p.log2_bs) - t0, 0);
                     const int boff = max(t0 - (j << p.log2_bs), 0);

@@ -76,11 +76,17 @@ __device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
 }
 
 // four e4m3 codes (one 32-bit word) -> four f16 (two 32-bit words), exact
+// (byte k of w -> f16 k: lo = codes 0, 1; hi = codes 2, 3).  The hardware
+// conversion takes two codes per instruction and packs the f16 pair itself.
 __device__ __forceinline__ void e4m3x4_to_f16(uint32_t w, uint32_t& lo, uint32_t& hi) {
-    const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w & 0xffffu), __NV_E4M3);
-    const __half2_raw b = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(w >> 16), __NV_E4M3);
-    lo = (uint32_t)a.x | ((uint32_t)a.y << 16);
-    hi = (uint32_t)b.x | ((uint32_t)b.y << 16);
+    asm("{\n\t"
+        ".reg .b16 c01, c23;\n\t"
+        "mov.b32 {c01, c23}, %2;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %0, c01;\n\t"
+        "cvt.rn.f16x2.e4m3x2 %1, c23;\n\t"
+        "}"
+        : "=r"(lo), "=r"(hi)
+        : "r"(w));
 }
 
 __device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
