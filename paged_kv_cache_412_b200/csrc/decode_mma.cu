@@ -74,11 +74,18 @@ struct MmaCfg {
     // through its phases in order.
     static constexpr int NCONS = F8 ? (NT == 1 ? 3 : 2) : 1;
     static constexpr int NCV = F8 ? 4 : 0;
-    static constexpr int THREADS = 32 * (2 + NCONS + NCV);  // + producer, epilogue
+    // producer warps: a TMA issue holds the issuing warp ~0.1 us, and one fp8
+    // producer per SM cannot issue fast enough; two take alternate chunks
+    // (stage n % NSTAGE belongs to producer n % NPROD).  The 16-head fp8
+    // config keeps one (its consumers need all the registers).
+    static constexpr int NPROD = (F8 && NT == 1) ? 2 : 1;
+    static constexpr int THREADS = 32 * (NPROD + NCONS + NCV + 1);  // + the epilogue
     static constexpr int QCH = NCONS;  // a segment's first QCH chunks carry the group's q
     static constexpr int SLOT_BYTES = F8 ? (2 * NHALF * HALF_BYTES + Q_BYTES + 1023) / 1024 * 1024 : 0;
     static constexpr int STG_BYTES = NCONS * SLOT_BYTES;   // f16 K | V | q per consumer
-    static constexpr int NSTAGE = F8 ? 4 : cmax(2, cmin(8, kRingBudget / STAGE_BYTES));
+    // fp8 (one CTA per SM): six stages keep ~100 KB of codes in flight per SM
+    static constexpr int NSTAGE = F8 ? 6 : cmax(2, cmin(8, kRingBudget / STAGE_BYTES));
+    static_assert(NSTAGE % NPROD == 0, "each stage belongs to one producer");
 };
 
 // ---- shared-memory layout ------------------------------------------------------
@@ -100,6 +107,7 @@ struct Smem {
     // ntok/bad per stage, then per staging slot
     static constexpr int OFF_CTRL = OFF_META + 2 * (C::NSTAGE + C::NCONS) * 4;
     static constexpr int BYTES = OFF_CTRL + 16 + 1024;   // + alignment slack
+    static_assert(BYTES <= 227 * 1024, "within the opt-in shared memory of one CTA");
 };
 
 // ---- producer ------------------------------------------------------------------
@@ -119,7 +127,9 @@ struct Producer {
     volatile int* ctrl;
     int lane;
     uint64_t policy;
-    Ring ring;
+    int me = 0;              // this producer (chunks n with n % NPROD == me)
+    unsigned n_chunk = 0;    // chunks of the CTA so far (all producers')
+    unsigned last_n = 0;     // the last chunk this producer issued
     int issued = 0;
     bool waited = false;
 
@@ -158,8 +168,12 @@ struct Producer {
                 tab = tab_next;
                 tab_next = (wbase + 32 < nblk) ? load_window(cur, wbase + 32) : -1;
             }
+            const unsigned n = n_chunk++;
+            if (C::NPROD > 1 && (int)(n % C::NPROD) != me) continue;  // the other producer's
+            const int stage = (int)(n % C::NSTAGE);
+            const uint32_t phase = (n / C::NSTAGE) & 1u;
             int ok = 1;
-            if (lane == 0) ok = !ctrl[0] && mbar_wait(&empty[ring.stage], ring.phase ^ 1u);
+            if (lane == 0) ok = !ctrl[0] && mbar_wait(&empty[stage], phase ^ 1u);
             ok = __shfl_sync(FULL_MASK, ok, 0);
             if (!ok) {
                 if (lane == 0) {
@@ -181,20 +195,20 @@ struct Producer {
                 else
                     ++nvalid;
             }
-            unsigned char* sk = smem + ring.stage * C::STAGE_BYTES;
+            unsigned char* sk = smem + stage * C::STAGE_BYTES;
             unsigned char* sv = sk + C::KV_BYTES;
             unsigned char* sq = sv + C::KV_BYTES;
             if (lane == 0) {
-                st_ntok[ring.stage] = ntok;
-                st_bad[ring.stage] = bad;
+                st_ntok[stage] = ntok;
+                st_bad[stage] = bad;
                 if (bad) raise_error(p.err, PKV_DEVERR_BAD_BLOCK);
                 const uint32_t qbytes = c - sg.c0 < C::QCH ? (uint32_t)gv * D * 2u : 0u;
                 const uint32_t row_bytes = F8 ? (uint32_t)D : (uint32_t)C::NHALF * 128u;
-                mbar_arrive_expect_tx(&full[ring.stage], nvalid * 2u * rb * row_bytes + qbytes);
+                mbar_arrive_expect_tx(&full[stage], nvalid * 2u * rb * row_bytes + qbytes);
                 if (qbytes)  // the group's q rows ride with the segment's first stage(s)
                     bulk_load(sq, static_cast<const __nv_bfloat16*>(p.q) +
                                       ((size_t)cur.b * p.num_q_heads + hq0) * D,
-                              qbytes, &full[ring.stage], policy);
+                              qbytes, &full[stage], policy);
             }
             // One lane per block of the chunk issues that block's copies: a TMA
             // issue costs the issuing thread ~0.1 us, so lane-parallel issue
@@ -209,21 +223,21 @@ struct Producer {
                     const int boff = t0 - (j << p.log2_bs) > 0 ? t0 - (j << p.log2_bs) : 0;
                     const int grow = (phys * p.num_kv_heads + kvh) * p.block_size + boff;
                     if constexpr (F8) {
-                        tma_load_2d(sk + srow * D, tmk, 0, grow, &full[ring.stage], policy);
-                        tma_load_2d(sv + srow * D, tmv, 0, grow, &full[ring.stage], policy);
+                        tma_load_2d(sk + srow * D, tmk, 0, grow, &full[stage], policy);
+                        tma_load_2d(sv + srow * D, tmv, 0, grow, &full[stage], policy);
                     } else {
 #pragma unroll
                         for (int h = 0; h < C::NHALF; ++h) {
                             tma_load_2d(sk + h * C::HALF_BYTES + srow * 128, tmk, h * 64, grow,
-                                        &full[ring.stage], policy);
+                                        &full[stage], policy);
                             tma_load_2d(sv + h * C::HALF_BYTES + srow * 128, tmv, h * 64, grow,
-                                        &full[ring.stage], policy);
+                                        &full[stage], policy);
                         }
                     }
                 }
             }
             ++issued;
-            ring.advance(C::NSTAGE);
+            last_n = n;
         }
         return true;
     }
@@ -250,16 +264,10 @@ struct Producer {
             // A wait gave up somewhere in the CTA: before this warp exits, wait
             // (bounded) for the stages it issued last, so no copy lands in
             // shared memory after the CTA has gone.
-            const int n = min(issued, C::NSTAGE);
-            Ring r = ring;
-            for (int i = 0; i < n; ++i) {
-                if (r.stage == 0) {
-                    r.stage = C::NSTAGE - 1;
-                    r.phase ^= 1u;
-                } else {
-                    --r.stage;
-                }
-                mbar_wait(&full[r.stage], r.phase);
+            const int k_max = min(issued, C::NSTAGE / C::NPROD);
+            for (int k = 0; k < k_max; ++k) {
+                const unsigned nn = last_n - (unsigned)(k * C::NPROD);
+                mbar_wait(&full[nn % C::NSTAGE], (nn / C::NSTAGE) & 1u);
             }
         }
     }
@@ -608,6 +616,19 @@ __device__ __forceinline__ void convert(const DecodeParams& p, SegIter<kCH>& it,
             const unsigned char* sk = smem + ring.stage * C::STAGE_BYTES;  // e4m3 rows of D bytes
             const unsigned char* sv = sk + C::KV_BYTES;
             unsigned char* dst0 = smem + S::OFF_STG + slot * C::SLOT_BYTES;
+            // all of this lane's code groups in flight first, then widen them
+            uint4 raw[PER_LANE];
+#pragma unroll
+            for (int i = 0; i < PER_LANE; ++i) {
+                const int idx = lane + 32 * i;
+                const int part = idx / (RPW * C16);
+                const int rest = idx % (RPW * C16);
+                const int row = v * RPW + rest / C16, c16 = rest % C16;
+                // the code row is stored swizzled: 16-byte group c16 of row r
+                // sits at c16 ^ (r % 8) (128-byte rows) or ^ (r / 2 % 4) (64-byte rows)
+                const int sw = D == 128 ? (row & 7) : ((row >> 1) & 3);
+                raw[i] = *reinterpret_cast<const uint4*>((part ? sv : sk) + row * D + ((c16 ^ sw) << 4));
+            }
 #pragma unroll
             for (int i = 0; i < PER_LANE; ++i) {
                 const int idx = lane + 32 * i;
@@ -621,16 +642,10 @@ __device__ __forceinline__ void convert(const DecodeParams& p, SegIter<kCH>& it,
                 }
                 uint4 o0 = make_uint4(0, 0, 0, 0), o1 = make_uint4(0, 0, 0, 0);
                 if (valid) {
-                    // the code row is stored swizzled: 16-byte group c16 of row
-                    // r sits at c16 ^ (r % 8) (128-byte rows) or ^ (r / 2 % 4)
-                    // (64-byte rows)
-                    const int sw = D == 128 ? (row & 7) : ((row >> 1) & 3);
-                    const uint4 raw = *reinterpret_cast<const uint4*>((part ? sv : sk) + row * D +
-                                                                      ((c16 ^ sw) << 4));
-                    e4m3x4_to_f16(raw.x, o0.x, o0.y);
-                    e4m3x4_to_f16(raw.y, o0.z, o0.w);
-                    e4m3x4_to_f16(raw.z, o1.x, o1.y);
-                    e4m3x4_to_f16(raw.w, o1.z, o1.w);
+                    e4m3x4_to_f16(raw[i].x, o0.x, o0.y);
+                    e4m3x4_to_f16(raw[i].y, o0.z, o0.w);
+                    e4m3x4_to_f16(raw[i].z, o1.x, o1.y);
+                    e4m3x4_to_f16(raw[i].w, o1.z, o1.w);
                 }
                 const int half = (c16 * 16) >> 6, cc = ((c16 * 16) & 63) >> 3;
                 unsigned char* dst = dst0 + part * C::NHALF * C::HALF_BYTES +
@@ -1012,7 +1027,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
     const long long total =
         total_chunks_warp(p, lane, blockIdx.x == 0 && warp == 0, &L_first, &T_first);
     if (total == 0) {
-        if (warp == C::NCONS + 1) {
+        if (warp == C::NPROD + C::NCONS) {
             SegIter<kCH> none;
             none.valid = false;
             epilogue<D, NT, F8>(p, none, smem, dfull, dempty, ctrl, lane);
@@ -1024,20 +1039,22 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
     SegIter<kCH> it;
     it.init(p, total, W, lane, L_first, T_first);
 
-    if (warp == 0) {
+    // warps: producers | consumers | epilogue | converters (fp8)
+    if (warp < C::NPROD) {
         Producer<D, NT, F8> pr{p, &tmk, &tmv, smem, full, empty, st_ntok, st_bad, ctrl, lane,
                            l2_policy_evict_first()};
+        pr.me = warp;
         pr.run(it);
         if (!pr.waited) griddep_wait();
-    } else if (warp <= C::NCONS) {
+    } else if (warp < C::NPROD + C::NCONS) {
         consume<D, NT, F8>(p, it, smem, full, empty, dfull, dempty, sfull, sempty, st_ntok, st_bad,
-                           sl_ntok, sl_bad, ctrl, lane, warp - 1);
-    } else if (warp == C::NCONS + 1) {
+                           sl_ntok, sl_bad, ctrl, lane, warp - C::NPROD);
+    } else if (warp == C::NPROD + C::NCONS) {
         epilogue<D, NT, F8>(p, it, smem, dfull, dempty, ctrl, lane);
     } else {
         if constexpr (C::NCV > 0)
             convert<D, NT>(p, it, smem, full, empty, sfull, sempty, st_ntok, st_bad, sl_ntok,
-                           sl_bad, ctrl, lane, warp - C::NCONS - 2);
+                           sl_bad, ctrl, lane, warp - C::NPROD - C::NCONS - 1);
     }
 }
 
