@@ -18,8 +18,13 @@
 namespace pkv {
 namespace {
 
-// One thread per 16-byte vector of one (token, kv head) row, K and V together.
-// Row r = t * Hkv + h of k/v goes to cache row ((blk * Hkv + h) * bs + off).
+constexpr int kWriteVecs = 2;  // 16-byte vectors (of K and of V) per thread
+constexpr int kCopyVecs = 4;   // 16-byte vectors per thread of a block copy
+
+// Each thread moves kWriteVecs 16-byte vectors of K and of V (vector i of the
+// rows t * Hkv + h, i = base + j * blockDim.x, so a warp's accesses stay
+// contiguous), every load issued before any store.  Row r = t * Hkv + h of k/v
+// goes to cache row ((blk * Hkv + h) * bs + off).
 __global__ void kv_cache_write_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
                                       const int64_t* __restrict__ slots, uint4* __restrict__ kc,
                                       uint4* __restrict__ vc, long long total_vecs,
@@ -28,8 +33,15 @@ __global__ void kv_cache_write_kernel(const uint4* __restrict__ k, const uint4* 
     // The previous kernel (a decode reading this cache) must be done first.
     griddep_wait();
     griddep_launch_dependents();
-    const long long stride = (long long)gridDim.x * blockDim.x;
-    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < total_vecs; i += stride) {
+    const long long base = (long long)blockIdx.x * blockDim.x * kWriteVecs + threadIdx.x;
+    uint4 kv[kWriteVecs], vv[kWriteVecs];
+    size_t dst[kWriteVecs];
+    bool ok[kWriteVecs];
+#pragma unroll
+    for (int j = 0; j < kWriteVecs; ++j) {
+        const long long i = base + (long long)j * blockDim.x;
+        ok[j] = false;
+        if (i >= total_vecs) continue;
         const long long row = i / vecs_per_row;
         const int vec = (int)(i - row * vecs_per_row);
         const long long t = row / num_kv_heads;
@@ -42,11 +54,16 @@ __global__ void kv_cache_write_kernel(const uint4* __restrict__ k, const uint4* 
         }
         const int64_t blk = slot / block_size;
         const int off = (int)(slot - blk * block_size);
-        const size_t dst = (((size_t)blk * num_kv_heads + h) * block_size + off) * vecs_per_row + vec;
-        const uint4 kv = __ldg(k + i);
-        const uint4 vv = __ldg(v + i);
-        kc[dst] = kv;
-        vc[dst] = vv;
+        dst[j] = (((size_t)blk * num_kv_heads + h) * block_size + off) * vecs_per_row + vec;
+        kv[j] = __ldg(k + i);
+        vv[j] = __ldg(v + i);
+        ok[j] = true;
+    }
+#pragma unroll
+    for (int j = 0; j < kWriteVecs; ++j) {
+        if (!ok[j]) continue;
+        kc[dst[j]] = kv[j];
+        vc[dst[j]] = vv[j];
     }
 }
 
@@ -120,7 +137,18 @@ __global__ void copy_blocks_kernel(uint4* __restrict__ kc, uint4* __restrict__ v
     uint4* d = base + dst * vecs_per_block;
     const long long lo = (long long)blockIdx.z * slice_vecs;
     const long long hi = min(lo + slice_vecs, vecs_per_block);
-    for (long long i = lo + threadIdx.x; i < hi; i += blockDim.x) d[i] = s[i];
+    // slice_vecs = kCopyVecs * blockDim.x: all of a thread's loads, then its stores
+    uint4 x[kCopyVecs];
+#pragma unroll
+    for (int j = 0; j < kCopyVecs; ++j) {
+        const long long i = lo + threadIdx.x + (long long)j * blockDim.x;
+        if (i < hi) x[j] = s[i];
+    }
+#pragma unroll
+    for (int j = 0; j < kCopyVecs; ++j) {
+        const long long i = lo + threadIdx.x + (long long)j * blockDim.x;
+        if (i < hi) d[i] = x[j];
+    }
 }
 
 // Block copy between two pools (either may be pinned host memory reached over
@@ -140,7 +168,17 @@ __global__ void swap_blocks_kernel(const uint4* __restrict__ sk, const uint4* __
     uint4* d = (blockIdx.y == 0 ? dk : dv) + dst * vecs_per_block;
     const long long lo = (long long)blockIdx.z * slice_vecs;
     const long long hi = min(lo + slice_vecs, vecs_per_block);
-    for (long long i = lo + threadIdx.x; i < hi; i += blockDim.x) d[i] = s[i];
+    uint4 x[kCopyVecs];
+#pragma unroll
+    for (int j = 0; j < kCopyVecs; ++j) {
+        const long long i = lo + threadIdx.x + (long long)j * blockDim.x;
+        if (i < hi) x[j] = s[i];
+    }
+#pragma unroll
+    for (int j = 0; j < kCopyVecs; ++j) {
+        const long long i = lo + threadIdx.x + (long long)j * blockDim.x;
+        if (i < hi) d[i] = x[j];
+    }
 }
 
 }  // namespace
@@ -152,7 +190,7 @@ pkv_status launch_swap_blocks(const void* src_k, const void* src_v, void* dst_k,
     if (num_pairs == 0) return PKV_OK;
     const long long vecs = (long long)(block_bytes / 16);
     const int threads = 256;
-    const int slice = threads * 4;
+    const int slice = threads * kCopyVecs;
     const long long slices = (vecs + slice - 1) / slice;
     if (slices > 65535) return PKV_ERR_UNSUPPORTED;
     dim3 grid(num_pairs, 2, (unsigned)slices);
@@ -173,9 +211,9 @@ pkv_status launch_kv_cache_write(const void* k, const void* v, const int64_t* sl
     const long long total = (long long)num_tokens * num_kv_heads * vecs_per_row;
     if (total == 0) return PKV_OK;
     const int threads = 256;
-    const long long want = (total + threads - 1) / threads;
-    const int grid = (int)std::min<long long>(want, (long long)di->num_sms * 8);
-    PdlLaunch L(dim3(grid), dim3(threads), 0, stream);
+    const long long grid = (total + (long long)threads * kWriteVecs - 1) / ((long long)threads * kWriteVecs);
+    if (grid > 0x7fffffffLL) return PKV_ERR_UNSUPPORTED;
+    PdlLaunch L(dim3((unsigned)grid), dim3(threads), 0, stream);
     const cudaError_t e = cudaLaunchKernelEx(
         &L.cfg, kv_cache_write_kernel, static_cast<const uint4*>(k), static_cast<const uint4*>(v),
         slots, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), total, vecs_per_row,
@@ -211,7 +249,7 @@ pkv_status launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs
     if (num_pairs == 0) return PKV_OK;
     const long long vecs = (long long)(block_bytes / 16);
     const int threads = 256;
-    const int slice = threads * 4;  // 16 KB per CTA
+    const int slice = threads * kCopyVecs;  // 16 KB per CTA
     const long long slices = (vecs + slice - 1) / slice;
     if (slices > 65535 || num_pairs > 2147483647) return PKV_ERR_UNSUPPORTED;
     dim3 grid(num_pairs, 2, (unsigned)slices);
