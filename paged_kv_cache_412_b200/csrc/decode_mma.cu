@@ -22,15 +22,19 @@
 // into the B-operand layout with movmatrix.trans.  P is split into bf16 hi + lo
 // parts (two MMAs) so the weights keep ~16 mantissa bits.
 //
-// Data movement: one producer warp walks the block table (32 entries per
+// Data movement: a producer warp walks the block table (32 entries per
 // coalesced load, next window prefetched, next segment's first window too) and
 // issues TMA tensor copies (2-D tensor map over the cache rows, 128-byte
 // swizzle, no multicast) of each physical block's K and V rows into a ring of
-// shared-memory stages with mbarrier completion.  One consumer warp per CTA
-// does the math, so no cross-warp reduction is needed; several CTAs share an
-// SM.  A request's (head group) split over several units is merged in-kernel by
-// the last unit to finish (per-group arrival counter in the workspace, reset by
-// the merger): out = sum_u 2^(m_u - M) acc_u / sum_u 2^(m_u - M) l_u.
+// shared-memory stages with mbarrier completion, one lane per block.
+// bf16: one consumer warp does the math (no cross-warp reduction), two CTAs
+// share an SM.  fp8: one CTA per SM with two producers, four converter warps
+// that widen each stage to f16 and three consumers taking the chunks in turn.
+// An epilogue warp normalises; a request's (head group) split over several
+// units is merged in-kernel by the last unit to finish (per-group arrival
+// counter in the workspace, reset by the merger), or -- fixed partitions and
+// prefix groups -- by a separate merge kernel:
+//   out = sum_u 2^(m_u - M) acc_u / sum_u 2^(m_u - M) l_u.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_fp16.h>
