@@ -67,6 +67,12 @@ CASES = [
     ([90, 700], 32, 2, 128, 64),             # G = 16, block = stage
     ([300, 129, 2], 8, 4, 64, 32),           # d 64
     ([0, 40, 1], 4, 2, 128, 256),            # empty request, block > stage
+    ([50, 1, 333], 8, 8, 128, 16),           # G = 1
+    ([200, 77], 12, 4, 128, 16),             # G = 3 (padded to 8)
+    ([120, 260], 32, 1, 64, 16),             # G = 32 at d 64: two 16-head passes per kv head
+    ([1000, 3], 16, 1, 64, 128),             # G = 16, d 64, block 128
+    # 60 requests of 1..400 tokens: many segments per CTA, split across the consumers
+    ([int(x) for x in np.random.default_rng(77).integers(1, 401, size=60)], 32, 8, 128, 16),
 ]
 
 

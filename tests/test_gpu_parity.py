@@ -75,6 +75,9 @@ SMALL = [
     ([700, 129], 32, 8, 128, 128, "bf16"),       # tensor-core path, block 128
     ([100, 260], 32, 1, 128, 16, "bf16"),        # G = 32: two 16-head passes per kv head
     ([64, 65, 63, 128], 8, 2, 64, 8, "bf16"),    # stage-boundary lengths, d 64
+    # 60 requests of 1..400 tokens: many segments per CTA and many split groups
+    ([int(x) for x in np.random.default_rng(78).integers(1, 401, size=60)], 32, 8, 128, 16, "bf16"),
+    ([int(x) for x in np.random.default_rng(79).integers(1, 401, size=40)], 16, 1, 64, 8, "bf16"),
 ]
 
 
