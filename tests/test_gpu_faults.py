@@ -100,3 +100,46 @@ def test_clean_run_leaves_no_flag(pkv):
     pkv.paged_attention_decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens,
                                w.bs, w.scale)
     assert pkv.get_device_error() == 0
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+def test_bad_block_tokens_do_not_take_part(pkv, dtype):
+    """A table entry outside the pool: that block's tokens are left out of the
+    request's softmax (the others are unaffected) and PKV_DEVERR_BAD_BLOCK is
+    raised.  Expected values: numpy brute force over the rows that remain."""
+    from oracle import brute
+    bs = 16
+    w = workloads.make_paged([100, 64, 50], Hq=8, Hkv=2, d=128, bs=bs, dtype=dtype, seed=3,
+                             append_last=False)
+    bt = w.block_tables.copy()
+    bt[1, 2] = w.num_blocks + 7  # request 1's third block (tokens 32..47) is out of range
+    dw = DevWorkload(w)
+    out = pkv.paged_attention_decode(dw.q, dw.k_cache, dw.v_cache, to_dev(bt), dw.seq_lens, bs,
+                                     w.scale, out_dtype=torch.float32, k_scale=dw.k_scale,
+                                     v_scale=dw.v_scale)
+    assert pkv.get_device_error() & pkv.DEVERR["BAD_BLOCK"]
+    got = to_host_f64(out)
+    G = w.Hq // w.Hkv
+
+    def rows(cache, scale_arr, b, h, tokens):
+        r = np.stack([cache[w.block_tables[b, t // bs], h, t % bs] for t in tokens])
+        if dtype == "fp8":
+            return workloads_e4m3(r) * float(scale_arr[h])
+        return brute.bf16_bits_to_f64(r)
+
+    q = brute.bf16_bits_to_f64(w.q)
+    for b in range(3):
+        L = int(w.seq_lens[b])
+        keep = [t for t in range(L) if not (b == 1 and 32 <= t < 48)]
+        for hq in range(w.Hq):
+            h = hq // G
+            ref = brute.attention_numpy(q[b, hq], rows(w.k_cache, w.k_scale, b, h, keep),
+                                        rows(w.v_cache, w.v_scale, b, h, keep), w.scale)
+            assert np.max(np.abs(got[b, hq] - ref)) <= 2e-3, (b, hq)
+
+
+def workloads_e4m3(codes: np.ndarray) -> np.ndarray:
+    """e4m3 codes -> float64 through torch's float8_e4m3fn (pinned against the
+    oracle's code table in the oracle tests)."""
+    t = torch.from_numpy(np.ascontiguousarray(codes)).view(torch.float8_e4m3fn)
+    return t.to(torch.float64).numpy()
