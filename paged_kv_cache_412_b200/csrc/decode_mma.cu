@@ -227,8 +227,13 @@ struct Producer {
                     const int boff = t0 - (j << p.log2_bs) > 0 ? t0 - (j << p.log2_bs) : 0;
                     const int grow = (phys * p.num_kv_heads + kvh) * p.block_size + boff;
                     if constexpr (F8) {
-                        tma_load_2d(sk + srow * D, tmk, 0, grow, &full[stage], policy);
-                        tma_load_2d(sv + srow * D, tmv, 0, grow, &full[stage], policy);
+                        // a block's code rows of one kv head are one contiguous run:
+                        // plain bulk copies (no tensor map, rows land unswizzled)
+                        const size_t goff = (size_t)grow * D;
+                        bulk_load(sk + srow * D, static_cast<const uint8_t*>(p.k_cache) + goff,
+                                  (uint32_t)(rb * D), &full[stage], policy);
+                        bulk_load(sv + srow * D, static_cast<const uint8_t*>(p.v_cache) + goff,
+                                  (uint32_t)(rb * D), &full[stage], policy);
                     } else {
 #pragma unroll
                         for (int h = 0; h < C::NHALF; ++h) {
@@ -628,10 +633,7 @@ __device__ __forceinline__ void convert(const DecodeParams& p, SegIter<kCH>& it,
                 const int part = idx / (RPW * C16);
                 const int rest = idx % (RPW * C16);
                 const int row = v * RPW + rest / C16, c16 = rest % C16;
-                // the code row is stored swizzled: 16-byte group c16 of row r
-                // sits at c16 ^ (r % 8) (128-byte rows) or ^ (r / 2 % 4) (64-byte rows)
-                const int sw = D == 128 ? (row & 7) : ((row >> 1) & 3);
-                raw[i] = *reinterpret_cast<const uint4*>((part ? sv : sk) + row * D + ((c16 ^ sw) << 4));
+                raw[i] = *reinterpret_cast<const uint4*>((part ? sv : sk) + row * D + c16 * 16);
             }
 #pragma unroll
             for (int i = 0; i < PER_LANE; ++i) {
