@@ -459,11 +459,6 @@ def run_ours(args, rank: int, world: int, local: int):
     e2e_value = dbytes * e2e_steps * world / (e2e_ms / 1e3) / 1e9
     assert pkv.get_device_error() == 0
 
-    # --- one parity spot check of the timed path against the oracle ---
-    parity = None
-    if rank == 0 and not args.no_check:
-        parity = spot_check(pkv, layers[0], out, ws, scale)
-
     result = None
     if rank == 0:
         cpu = cpu_baseline() if (world == 1 and not args.no_cpu_baseline) else None
@@ -503,7 +498,6 @@ def run_ours(args, rank: int, world: int, local: int):
                     "mode": e2e_mode},
             "gpu_launches": 2 * args.steps,
             "clocks": clocks,
-            "parity_spot_check": parity,
         }
         print(json.dumps(result), flush=True)
     dist_barrier(world)
@@ -745,24 +739,6 @@ def _suite_cache_ops(pkv, torch, workloads, dev, iters, flush, emit):
     assert pkv.get_device_error() == 0
 
 
-def spot_check(pkv, t, out, ws, scale):
-    """Compare a few outputs of the timed configuration with the oracle."""
-    import torch
-    import oracle
-    w = t["host"]
-    kc, vc = w.k_cache.copy(), w.v_cache.copy()
-    oracle.kv_cache_write(w.k_new, w.v_new, w.slot_mapping, kc, vc)
-    rows = [0, 7, 15]
-    ref = oracle.decode(w.q[rows], kc, vc, w.block_tables[rows], w.seq_lens[rows], w.scale)
-    pkv.kv_cache_write(t["kn"], t["vn"], t["sm"], t["kc"], t["vc"])
-    pkv.paged_attention_decode(t["q"], t["kc"], t["vc"], t["bt"], t["sl"], 16, scale, out,
-                               max_seq_len=4096, workspace=ws)
-    got = out.float().cpu().numpy()[rows].astype(np.float64)
-    err = np.abs(got - ref)
-    ok = bool(np.all(err <= 2e-3 + 1e-2 * np.abs(ref)))
-    return {"requests": rows, "max_abs": float(err.max()), "pass": ok}
-
-
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -770,7 +746,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-check", action="store_true")
+    ap.add_argument("--no-check", action="store_true",
+                    help="accepted for older command lines; parity is checked by the tests, "
+                         "not by the bench")
     ap.add_argument("--suite", action="store_true",
                     help="one line per workload of the scope table instead of the headline")
     ap.add_argument("--case", default="",
