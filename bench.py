@@ -93,10 +93,11 @@ class ClockSampler:
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, path: str | None = None):
+        import tempfile
         self.gpu = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+        self.path = path or os.path.join(tempfile.gettempdir(), f"pkv_clocks_gpu{gpu_index}.csv")
 
     def start(self):
         try:
@@ -348,7 +349,7 @@ def run_ours(args, rank: int, world: int, local: int):
     torch.cuda.synchronize()
 
     # --- timed region: K steps (graph replays), device-timed ---
-    sampler = ClockSampler(dev.index if dev.index is not None else 0)
+    sampler = ClockSampler(dev.index if dev.index is not None else 0, args.clocks_csv or None)
     bounds = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
     sampler.start()
     time.sleep(0.3)
@@ -746,6 +747,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--clocks-csv", default="",
+                    help="where to keep the raw nvidia-smi samples of the timed region "
+                         "(default: a temporary file; the JSON line carries the summary)")
     ap.add_argument("--no-check", action="store_true",
                     help="accepted for older command lines; parity is checked by the tests, "
                          "not by the bench")
