@@ -634,11 +634,12 @@ def run_suite(args):
                 decode_case(f"decode long_ctx 2 x 131072 bs {bs} partition {P or 'auto'}", wl,
                             partition_size=P)
             del wl
-    if want("simt"):
-        # block size 4: the CUDA-core path (the tensor-core one needs blocks of >= 8)
+    if want("small_blocks"):
+        # block size 4: tensor-core decode fed by per-lane row copies (blocks of
+        # fewer than 8 rows cannot be 128-byte-swizzled TMA boxes)
         w = workloads.make_paged([4096] * 16, Hq=32, Hkv=8, d=128, bs=4, dtype="bf16",
                                  seed=1002, poison=False, name="gqa_4k_bs4")
-        decode_case("decode 4k batch, block 4 (CUDA-core path)", w)
+        decode_case("decode 4k batch, block 4 (row copies)", w)
     if want("prefix"):
         _suite_prefix(pkv, torch, workloads, dev, iters, flush, emit)
     if want("cache_ops"):
@@ -763,7 +764,7 @@ def main():
                     help="one line per workload of the scope table instead of the headline")
     ap.add_argument("--case", default="",
                     help="with --suite: only the sections whose name contains this "
-                         "(gqa_4k, fp8, mixed, long_ctx, simt, prefix, cache_ops)")
+                         "(gqa_4k, fp8, mixed, long_ctx, small_blocks, prefix, cache_ops)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -281,7 +281,7 @@ pkv_status decode_entry(const void* q, const void* k_cache, const void* v_cache,
             if (!pa->prefix_of || !pa->prefix_lens || !aligned(pa->prefix_of, 4) ||
                 !aligned(pa->prefix_lens, 4))
                 return PKV_ERR_INVALID_ARG;
-            if (!(q_dtype == PKV_BF16 && kv_dtype == PKV_BF16) ||
+            if (!(q_dtype == PKV_BF16 && kv_dtype == PKV_BF16) || block_size < 8 ||
                 !decode_mma_supported(head_dim, block_size, q_dtype, kv_dtype))
                 return PKV_ERR_UNSUPPORTED;
             pfx_tiles = prefix_row_tiles(pa->max_members, num_q_heads / num_kv_heads);
@@ -344,6 +344,7 @@ pkv_status decode_entry(const void* q, const void* k_cache, const void* v_cache,
     // splits of a shared prefix) is combined in parallel instead of by one
     // warp of the decode kernel (which would stall that warp's CTA).
     p.defer_merge = (mma && (partition_size > 0 || use_prefix)) ? 1 : 0;
+    p.row_copy = (mma && block_size < 8) ? 1 : 0;
     p.rec_cap = (long long)pl.records;
     p.out_dtype = out_dtype;
     p.scale_log2 = scale * 1.4426950408889634f;

@@ -202,6 +202,53 @@ struct Producer {
             unsigned char* sk = smem + stage * C::STAGE_BYTES;
             unsigned char* sv = sk + C::KV_BYTES;
             unsigned char* sq = sv + C::KV_BYTES;
+            if constexpr (!F8) {
+                if (p.row_copy) {
+                    // Blocks of 2 or 4 rows: each lane copies whole token rows
+                    // (tokens lane and lane + 32) in 16-byte pieces to their
+                    // swizzled places, and the q rows with the segment's first
+                    // stage; the stage completes when all 32 lanes' copies have.
+                    if (lane == 0) {
+                        st_ntok[stage] = ntok;
+                        st_bad[stage] = bad;
+                        if (bad) raise_error(p.err, PKV_DEVERR_BAD_BLOCK);
+                    }
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        const int t = lane + 32 * r;
+                        const int j = (t0 + min(t, ntok - 1)) >> p.log2_bs;
+                        const int phys = __shfl_sync(FULL_MASK, tab, j - wbase);
+                        if (t < ntok && phys >= 0 && phys < p.num_blocks) {
+                            const int off = (t0 + t) & (p.block_size - 1);
+                            const size_t row =
+                                ((size_t)phys * p.num_kv_heads + kvh) * p.block_size + off;
+                            const unsigned char* gk =
+                                static_cast<const unsigned char*>(p.k_cache) + row * D * 2;
+                            const unsigned char* gvr =
+                                static_cast<const unsigned char*>(p.v_cache) + row * D * 2;
+#pragma unroll
+                            for (int c16 = 0; c16 < D / 8; ++c16) {
+                                const int so = (c16 >> 3) * C::HALF_BYTES + t * 128 +
+                                               (((c16 & 7) ^ (t & 7)) << 4);
+                                cp_async16(sk + so, gk + c16 * 16);
+                                cp_async16(sv + so, gvr + c16 * 16);
+                            }
+                        }
+                    }
+                    if (c - sg.c0 < C::QCH) {
+                        const unsigned char* gq = reinterpret_cast<const unsigned char*>(
+                            static_cast<const __nv_bfloat16*>(p.q) +
+                            ((size_t)cur.b * p.num_q_heads + hq0) * D);
+                        for (int i = lane; i < gv * D * 2 / 16; i += 32)
+                            cp_async16(sq + i * 16, gq + i * 16);
+                    }
+                    __threadfence_block();  // the chunk's meta before the arrival
+                    cp_async_mbar_arrive(&full[stage]);
+                    ++issued;
+                    last_n = n;
+                    continue;
+                }
+            }
             if (lane == 0) {
                 st_ntok[stage] = ntok;
                 st_bad[stage] = bad;
@@ -1007,7 +1054,8 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
     if (threadIdx.x == 0) {
         ctrl[0] = 0;
         for (int s = 0; s < C::NSTAGE; ++s) {
-            mbar_init(&full[s], 1);
+            // row copies: every producer lane arrives once its copies have landed
+            mbar_init(&full[s], (!F8 && p.row_copy) ? 32 : 1);
             mbar_init(&empty[s], F8 ? C::NCV : 1);  // released by the converters (fp8)
         }
         for (int s = 0; s < S::NSLOT; ++s) {
@@ -1276,8 +1324,12 @@ bool encode_cache_map(CUtensorMap* map, const void* base, long long rows, int he
 }
 
 bool decode_mma_supported(int head_dim, int block_size, pkv_dtype q_dtype, pkv_dtype kv_dtype) {
+    // blocks of >= 8 rows: TMA boxes; bf16 blocks of 2 or 4 rows: per-lane row copies
+    // (a 64-token chunk then spans 32 or 16 blocks, within one table window)
+    const bool rows_ok = block_size >= 8 ||
+                         (kv_dtype == PKV_BF16 && (block_size == 2 || block_size == 4));
     return q_dtype == PKV_BF16 && (kv_dtype == PKV_BF16 || kv_dtype == PKV_FP8_E4M3) &&
-           (head_dim == 64 || head_dim == 128) && block_size >= 8;
+           (head_dim == 64 || head_dim == 128) && rows_ok;
 }
 
 pkv_status launch_decode_mma(const DecodeParams& p, int head_dim, int group_pad, bool fp8,

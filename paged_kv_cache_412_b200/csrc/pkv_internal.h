@@ -80,6 +80,8 @@ struct DecodeParams {
     int fixed_units;  // 0 = automatic
     int defer_merge;  // 1: parts of a split group only publish records (+ meta);
                       // a separate merge kernel combines them
+    int row_copy;     // 1: blocks of 2 or 4 rows -- the producer copies token rows
+                      // with per-lane 16-byte async copies instead of TMA boxes
     long long rec_cap;  // records the workspace holds
     int out_dtype;
     float scale_log2;  // softmax scale * log2(e)
