@@ -116,9 +116,12 @@ struct Smem {
 
 // ---- producer ------------------------------------------------------------------
 
-template <int D, int NT, bool F8>
+// RC: blocks of 2 or 4 rows (bf16), copied row by row instead of by TMA boxes;
+// a separate instance so the boxed producer carries no trace of it.
+template <int D, int NT, bool F8, bool RC>
 struct Producer {
     using C = MmaCfg<D, NT, F8>;
+    static_assert(!(RC && F8), "row copies serve bf16 caches only");
 
     const DecodeParams& p;
     const CUtensorMap* tmk;
@@ -202,52 +205,50 @@ struct Producer {
             unsigned char* sk = smem + stage * C::STAGE_BYTES;
             unsigned char* sv = sk + C::KV_BYTES;
             unsigned char* sq = sv + C::KV_BYTES;
-            if constexpr (!F8) {
-                if (p.row_copy) {
-                    // Blocks of 2 or 4 rows: each lane copies whole token rows
-                    // (tokens lane and lane + 32) in 16-byte pieces to their
-                    // swizzled places, and the q rows with the segment's first
-                    // stage; the stage completes when all 32 lanes' copies have.
-                    if (lane == 0) {
-                        st_ntok[stage] = ntok;
-                        st_bad[stage] = bad;
-                        if (bad) raise_error(p.err, PKV_DEVERR_BAD_BLOCK);
-                    }
+            if constexpr (RC) {
+                // Blocks of 2 or 4 rows: each lane copies whole token rows
+                // (tokens lane and lane + 32) in 16-byte pieces to their
+                // swizzled places, and the q rows with the segment's first
+                // stage; the stage completes when all 32 lanes' copies have.
+                if (lane == 0) {
+                    st_ntok[stage] = ntok;
+                    st_bad[stage] = bad;
+                    if (bad) raise_error(p.err, PKV_DEVERR_BAD_BLOCK);
+                }
 #pragma unroll
-                    for (int r = 0; r < 2; ++r) {
-                        const int t = lane + 32 * r;
-                        const int j = (t0 + min(t, ntok - 1)) >> p.log2_bs;
-                        const int phys = __shfl_sync(FULL_MASK, tab, j - wbase);
-                        if (t < ntok && phys >= 0 && phys < p.num_blocks) {
-                            const int off = (t0 + t) & (p.block_size - 1);
-                            const size_t row =
-                                ((size_t)phys * p.num_kv_heads + kvh) * p.block_size + off;
-                            const unsigned char* gk =
-                                static_cast<const unsigned char*>(p.k_cache) + row * D * 2;
-                            const unsigned char* gvr =
-                                static_cast<const unsigned char*>(p.v_cache) + row * D * 2;
+                for (int r = 0; r < 2; ++r) {
+                    const int t = lane + 32 * r;
+                    const int j = (t0 + min(t, ntok - 1)) >> p.log2_bs;
+                    const int phys = __shfl_sync(FULL_MASK, tab, j - wbase);
+                    if (t < ntok && phys >= 0 && phys < p.num_blocks) {
+                        const int off = (t0 + t) & (p.block_size - 1);
+                        const size_t row =
+                            ((size_t)phys * p.num_kv_heads + kvh) * p.block_size + off;
+                        const unsigned char* gk =
+                            static_cast<const unsigned char*>(p.k_cache) + row * D * 2;
+                        const unsigned char* gvr =
+                            static_cast<const unsigned char*>(p.v_cache) + row * D * 2;
 #pragma unroll
-                            for (int c16 = 0; c16 < D / 8; ++c16) {
-                                const int so = (c16 >> 3) * C::HALF_BYTES + t * 128 +
-                                               (((c16 & 7) ^ (t & 7)) << 4);
-                                cp_async16(sk + so, gk + c16 * 16);
-                                cp_async16(sv + so, gvr + c16 * 16);
-                            }
+                        for (int c16 = 0; c16 < D / 8; ++c16) {
+                            const int so = (c16 >> 3) * C::HALF_BYTES + t * 128 +
+                                           (((c16 & 7) ^ (t & 7)) << 4);
+                            cp_async16(sk + so, gk + c16 * 16);
+                            cp_async16(sv + so, gvr + c16 * 16);
                         }
                     }
-                    if (c - sg.c0 < C::QCH) {
-                        const unsigned char* gq = reinterpret_cast<const unsigned char*>(
-                            static_cast<const __nv_bfloat16*>(p.q) +
-                            ((size_t)cur.b * p.num_q_heads + hq0) * D);
-                        for (int i = lane; i < gv * D * 2 / 16; i += 32)
-                            cp_async16(sq + i * 16, gq + i * 16);
-                    }
-                    __threadfence_block();  // the chunk's meta before the arrival
-                    cp_async_mbar_arrive(&full[stage]);
-                    ++issued;
-                    last_n = n;
-                    continue;
                 }
+                if (c - sg.c0 < C::QCH) {
+                    const unsigned char* gq = reinterpret_cast<const unsigned char*>(
+                        static_cast<const __nv_bfloat16*>(p.q) +
+                        ((size_t)cur.b * p.num_q_heads + hq0) * D);
+                    for (int i = lane; i < gv * D * 2 / 16; i += 32)
+                        cp_async16(sq + i * 16, gq + i * 16);
+                }
+                __threadfence_block();  // the chunk's meta before the arrival
+                cp_async_mbar_arrive(&full[stage]);
+                ++issued;
+                last_n = n;
+                continue;
             }
             if (lane == 0) {
                 st_ntok[stage] = ntok;
@@ -1029,7 +1030,7 @@ __device__ __forceinline__ long long total_chunks_warp(const DecodeParams& p, in
     return t * p.num_hg;
 }
 
-template <int D, int NT, bool F8>
+template <int D, int NT, bool F8, bool RC>
 __global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
     decode_mma_kernel(const __grid_constant__ DecodeParams p,
                                                              const __grid_constant__ CUtensorMap tmk,
@@ -1055,7 +1056,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
         ctrl[0] = 0;
         for (int s = 0; s < C::NSTAGE; ++s) {
             // row copies: every producer lane arrives once its copies have landed
-            mbar_init(&full[s], (!F8 && p.row_copy) ? 32 : 1);
+            mbar_init(&full[s], RC ? 32 : 1);
             mbar_init(&empty[s], F8 ? C::NCV : 1);  // released by the converters (fp8)
         }
         for (int s = 0; s < S::NSLOT; ++s) {
@@ -1095,7 +1096,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
 
     // warps: producers | consumers | epilogue | converters (fp8)
     if (warp < C::NPROD) {
-        Producer<D, NT, F8> pr{p, &tmk, &tmv, smem, full, empty, st_ntok, st_bad, ctrl, lane,
+        Producer<D, NT, F8, RC> pr{p, &tmk, &tmv, smem, full, empty, st_ntok, st_bad, ctrl, lane,
                            l2_policy_evict_first()};
         pr.me = warp;
         pr.run(it);
@@ -1239,7 +1240,7 @@ __global__ void __launch_bounds__(32 * kMergeWarps)
 
 // ---- host side ---------------------------------------------------------------
 
-template <int D, int NT, bool F8>
+template <int D, int NT, bool F8, bool RC>
 pkv_status launch_impl(const DecodeParams& p, cudaStream_t stream, int* grid_out) {
     using C = MmaCfg<D, NT, F8>;
     using S = Smem<D, NT, F8>;
@@ -1247,7 +1248,7 @@ pkv_status launch_impl(const DecodeParams& p, cudaStream_t stream, int* grid_out
     if (!di) return PKV_ERR_CUDA;
     static std::mutex mu;
     static int occupancy[64] = {0};
-    auto kern = decode_mma_kernel<D, NT, F8>;
+    auto kern = decode_mma_kernel<D, NT, F8, RC>;
     {
         std::lock_guard<std::mutex> lock(mu);
         if (di->device >= 64) return PKV_ERR_UNSUPPORTED;
@@ -1336,15 +1337,21 @@ pkv_status launch_decode_mma(const DecodeParams& p, int head_dim, int group_pad,
                              cudaStream_t stream, int* grid_out) {
     const int nt = group_pad > 8 ? 2 : 1;
     if (fp8) {
-        if (head_dim == 128) return nt == 1 ? launch_impl<128, 1, true>(p, stream, grid_out)
-                                            : launch_impl<128, 2, true>(p, stream, grid_out);
-        if (head_dim == 64) return nt == 1 ? launch_impl<64, 1, true>(p, stream, grid_out)
-                                           : launch_impl<64, 2, true>(p, stream, grid_out);
+        if (p.row_copy) return PKV_ERR_UNSUPPORTED;
+        if (head_dim == 128) return nt == 1 ? launch_impl<128, 1, true, false>(p, stream, grid_out)
+                                            : launch_impl<128, 2, true, false>(p, stream, grid_out);
+        if (head_dim == 64) return nt == 1 ? launch_impl<64, 1, true, false>(p, stream, grid_out)
+                                           : launch_impl<64, 2, true, false>(p, stream, grid_out);
+    } else if (p.row_copy) {
+        if (head_dim == 128) return nt == 1 ? launch_impl<128, 1, false, true>(p, stream, grid_out)
+                                            : launch_impl<128, 2, false, true>(p, stream, grid_out);
+        if (head_dim == 64) return nt == 1 ? launch_impl<64, 1, false, true>(p, stream, grid_out)
+                                           : launch_impl<64, 2, false, true>(p, stream, grid_out);
     } else {
-        if (head_dim == 128) return nt == 1 ? launch_impl<128, 1, false>(p, stream, grid_out)
-                                            : launch_impl<128, 2, false>(p, stream, grid_out);
-        if (head_dim == 64) return nt == 1 ? launch_impl<64, 1, false>(p, stream, grid_out)
-                                           : launch_impl<64, 2, false>(p, stream, grid_out);
+        if (head_dim == 128) return nt == 1 ? launch_impl<128, 1, false, false>(p, stream, grid_out)
+                                            : launch_impl<128, 2, false, false>(p, stream, grid_out);
+        if (head_dim == 64) return nt == 1 ? launch_impl<64, 1, false, false>(p, stream, grid_out)
+                                           : launch_impl<64, 2, false, false>(p, stream, grid_out);
     }
     return PKV_ERR_UNSUPPORTED;
 }
