@@ -1117,42 +1117,50 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
 
 constexpr int kMergeWarps = 4;  // warps that share one output row
 
-// One CTA per output row (request b, query head): it merges the row over the
-// parts of its own pass (records of the decode kernel) and the splits of its
-// group's shared prefix pass.  The CTA finds the common max M first; then
-// warp w takes records w, w + 4, ... eight at a time (each record row read as
-// one coalesced run of float4 / float2, lane = head_dim/32 dims), and the
-// warps' sums meet in shared memory.
-//   out = vscale * sum_r 2^(m_r - M) acc_r / sum_r 2^(m_r - M) l_r.
-template <int D, int GP>
+// Merges output rows (request b, query head) over the parts of the row's own
+// pass (records of the decode kernel) and the splits of its group's shared
+// prefix pass.  RPC rows per CTA: with RPC == kMergeWarps each warp merges one
+// row (many short rows: the grid fits one wave); with RPC == 1 the CTA's warps
+// share one row, warp w taking records w, w + 4, ... (few long rows).  A warp
+// reads its records eight at a time (each record row one coalesced run of
+// float4 / float2, lane = head_dim/32 dims) and keeps a running max, sum and
+// accumulator; the warps of a row meet in shared memory.
+//   out = vscale * sum_r 2^(m_r - M) acc_r / sum_r 2^(m_r - M) l_r,  M = max_r m_r.
+template <int D, int GP, int RPC>
 __global__ void __launch_bounds__(32 * kMergeWarps)
     decode_mma_merge_kernel(const __grid_constant__ DecodeParams p) {
     constexpr int PER = D / 32;  // dims per lane
     constexpr int NB = 8;        // records in flight per warp
-    __shared__ float red_acc[kMergeWarps][D];
+    constexpr int WPR = kMergeWarps / RPC;  // warps per row
+    static_assert(RPC == 1 || RPC == kMergeWarps, "a row per CTA or a row per warp");
+    __shared__ float red_acc[WPR > 1 ? kMergeWarps : 1][D];
     __shared__ float red_m[kMergeWarps], red_s[kMergeWarps];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int b = (int)(blockIdx.x / p.num_q_heads), hq = (int)(blockIdx.x % p.num_q_heads);
+    const int wr = warp % WPR;  // this warp's rank among its row's warps
+    const long long row = (long long)blockIdx.x * RPC + warp / WPR;
+    const bool live = row < (long long)p.num_seqs * p.num_q_heads;
+    const int b = live ? (int)(row / p.num_q_heads) : 0;
+    const int hq = live ? (int)(row % p.num_q_heads) : 0;
     const int kvh = hq / p.group, jg = hq % p.group;
     const int hg = kvh * p.num_sub + jg / GP, h = jg % GP;
     const size_t bg = (size_t)b * p.num_hg + hg;
-    const int L = clamp_len(p, b, false);
-    const int T = seq_begin(p, b, L);
+    const int L = live ? clamp_len(p, b, false) : 0;
+    const int T = live ? seq_begin(p, b, L) : 0;
     const int ns = T > 0 ? prefix_num_splits(prefix_tokens_of(p, b), p.pfx_splits) : 0;
     griddep_wait();  // the records and meta of the kernels before
-    // every condition below is the same in all threads of the CTA
+    // every condition below is the same in all threads of the row's warps
     int u0 = 0, nseg = 0;
     if (L > T) {
         u0 = p.meta[2 * bg];
         nseg = p.meta[2 * bg + 1];
         if (nseg == 0) return;  // did not fit the workspace (flagged by the decode kernel)
         if (u0 < 0 || (long long)bg + u0 + nseg > p.rec_cap) {  // never for a word this call wrote
-            if (threadIdx.x == 0) raise_error(p.err, PKV_DEVERR_BAD_SEQ_LEN);
+            if (lane == 0 && wr == 0) raise_error(p.err, PKV_DEVERR_BAD_SEQ_LEN);
             return;
         }
     }
     const int n = nseg + ns;
-    if (n == 0) return;  // an empty request: the decode kernel wrote zeros
+    if (n == 0) return;  // an empty request (or no row): the decode kernel wrote zeros
     const size_t rec0 = bg + u0;
     // record r < nseg: own part r; r >= nseg: split r - nseg of the shared pass
     auto ml_of = [&](int r) -> const float* {
@@ -1176,65 +1184,77 @@ __global__ void __launch_bounds__(32 * kMergeWarps)
             v[1] = t.y;
         }
     };
-    // the common max
-    float m = -INFINITY;
-    for (int r = threadIdx.x; r < n; r += 32 * kMergeWarps) m = fmaxf(m, ml_of(r)[0]);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL_MASK, m, off));
-    if (lane == 0) red_m[warp] = m;
-    __syncthreads();
-    float M = red_m[0];
-#pragma unroll
-    for (int w = 1; w < kMergeWarps; ++w) M = fmaxf(M, red_m[w]);
-    const float mref = M == -INFINITY ? 0.f : M;
-    // this warp's records
-    float A[PER], S = 0.f;
+    // this warp's records, NB at a time (the last batch predicated)
+    float A[PER], S = 0.f, mw = -INFINITY;
 #pragma unroll
     for (int i = 0; i < PER; ++i) A[i] = 0.f;
-    int r = warp;
-    for (; r + kMergeWarps * (NB - 1) < n; r += kMergeWarps * NB) {
+    for (int r0 = wr; r0 < n; r0 += WPR * NB) {
         float v[NB][PER], mm[NB], ll[NB];
 #pragma unroll
         for (int q = 0; q < NB; ++q) {
-            const float* ml = ml_of(r + kMergeWarps * q);
-            mm[q] = ml[0];
-            ll[q] = ml[1];
-            load_row(acc_of(r + kMergeWarps * q), v[q]);
+            const int r = r0 + WPR * q;
+            if (r < n) {
+                const float* ml = ml_of(r);
+                mm[q] = ml[0];
+                ll[q] = ml[1];
+                load_row(acc_of(r), v[q]);
+            } else {
+                mm[q] = -INFINITY;
+                ll[q] = 0.f;
+#pragma unroll
+                for (int i = 0; i < PER; ++i) v[q][i] = 0.f;
+            }
         }
+        float mb = mw;
+#pragma unroll
+        for (int q = 0; q < NB; ++q) mb = fmaxf(mb, mm[q]);
+        const float ref = mb == -INFINITY ? 0.f : mb;
+        const float c = exp2f(mw - ref);  // 0 while nothing is held
+        S *= c;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) A[i] *= c;
 #pragma unroll
         for (int q = 0; q < NB; ++q) {
-            const float wq = exp2f(mm[q] - mref);
+            const float wq = exp2f(mm[q] - ref);
             S = fmaf(ll[q], wq, S);
 #pragma unroll
             for (int i = 0; i < PER; ++i) A[i] = fmaf(v[q][i], wq, A[i]);
         }
+        mw = mb;
     }
-    for (; r < n; r += kMergeWarps) {
-        const float* ml = ml_of(r);
-        const float wq = exp2f(ml[0] - mref);
-        S = fmaf(ml[1], wq, S);
-        float v[PER];
-        load_row(acc_of(r), v);
-#pragma unroll
-        for (int i = 0; i < PER; ++i) A[i] = fmaf(v[i], wq, A[i]);
-    }
-#pragma unroll
-    for (int i = 0; i < PER; ++i) red_acc[warp][lane * PER + i] = A[i];
-    if (lane == 0) red_s[warp] = S;
-    __syncthreads();
-    if (warp != 0) return;
-    float St = 0.f;
-#pragma unroll
-    for (int w = 0; w < kMergeWarps; ++w) St += red_s[w];
     const float vsc = p.v_scale ? __ldg(p.v_scale + kvh) : 1.f;
-    const float inv = St > 0.f ? vsc / St : 0.f;
     const size_t orow = ((size_t)b * p.num_q_heads + hq) * D + lane * PER;
+    if constexpr (WPR == 1) {
+        const float inv = S > 0.f ? vsc / S : 0.f;
 #pragma unroll
-    for (int i = 0; i < PER; ++i) {
-        float t = 0.f;
+        for (int i = 0; i < PER; ++i) store_out(p.out, orow + i, A[i] * inv, p.out_dtype);
+    } else {
 #pragma unroll
-        for (int w = 0; w < kMergeWarps; ++w) t += red_acc[w][lane * PER + i];
-        store_out(p.out, orow + i, t * inv, p.out_dtype);
+        for (int i = 0; i < PER; ++i) red_acc[warp][lane * PER + i] = A[i];
+        if (lane == 0) {
+            red_m[warp] = mw;
+            red_s[warp] = S;
+        }
+        __syncthreads();
+        if (warp != 0) return;
+        float M = red_m[0];
+#pragma unroll
+        for (int w = 1; w < kMergeWarps; ++w) M = fmaxf(M, red_m[w]);
+        const float ref = M == -INFINITY ? 0.f : M;
+        float cw[kMergeWarps], St = 0.f;
+#pragma unroll
+        for (int w = 0; w < kMergeWarps; ++w) {
+            cw[w] = exp2f(red_m[w] - ref);
+            St = fmaf(red_s[w], cw[w], St);
+        }
+        const float inv = St > 0.f ? vsc / St : 0.f;
+#pragma unroll
+        for (int i = 0; i < PER; ++i) {
+            float t = 0.f;
+#pragma unroll
+            for (int w = 0; w < kMergeWarps; ++w) t = fmaf(red_acc[w][lane * PER + i], cw[w], t);
+            store_out(p.out, orow + i, t * inv, p.out_dtype);
+        }
     }
 }
 
@@ -1277,11 +1297,17 @@ pkv_status launch_impl(const DecodeParams& p, cudaStream_t stream, int* grid_out
     if (cudaLaunchKernelEx(&L.cfg, kern, p, tmk, tmv) != cudaSuccess) return PKV_ERR_CUDA;
     if (p.defer_merge) {
         constexpr int GP = MmaCfg<D, NT, F8>::GP;
-        const long long mgrid = (long long)p.num_seqs * p.num_q_heads;  // one CTA per output row
+        // many rows: one warp per row (a single wave of CTAs); few rows, which
+        // may each hold many parts: the CTA's warps share a row
+        const long long rows = (long long)p.num_seqs * p.num_q_heads;
+        const bool per_warp = rows >= 4LL * di->num_sms;
+        const long long mgrid = per_warp ? (rows + kMergeWarps - 1) / kMergeWarps : rows;
         if (mgrid > 0x7fffffffLL) return PKV_ERR_UNSUPPORTED;
         PdlLaunch M(dim3((unsigned)mgrid), dim3(32 * kMergeWarps), 0, stream);
-        if (cudaLaunchKernelEx(&M.cfg, decode_mma_merge_kernel<D, GP>, p) != cudaSuccess)
-            return PKV_ERR_CUDA;
+        const cudaError_t e =
+            per_warp ? cudaLaunchKernelEx(&M.cfg, decode_mma_merge_kernel<D, GP, kMergeWarps>, p)
+                     : cudaLaunchKernelEx(&M.cfg, decode_mma_merge_kernel<D, GP, 1>, p);
+        if (e != cudaSuccess) return PKV_ERR_CUDA;
     }
     if (grid_out) *grid_out = grid;
     return PKV_OK;
