@@ -194,6 +194,17 @@ def test_workload_mixed(pkv):
     _full_check(pkv, w, sample=sample)
 
 
+@pytest.mark.parametrize("P", [256, 1024])
+def test_workload_mixed_fixed_partitions(pkv, P):
+    """Fixed partitions over many rows (256 requests x 32 query heads): the
+    separate merge runs one warp per row, rows of up to 32 parts."""
+    w = workloads.mixed()
+    rng = np.random.default_rng(1)
+    sample = sorted(set(rng.choice(w.B, size=24, replace=False).tolist()) |
+                    {int(np.argmax(w.seq_lens)), int(np.argmin(w.seq_lens))})
+    _full_check(pkv, w, sample=sample, partition_size=P, out_f32=False)
+
+
 def test_workload_prefix(pkv):
     w = workloads.prefix_shared()
     _full_check(pkv, w)
