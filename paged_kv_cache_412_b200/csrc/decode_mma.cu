@@ -634,6 +634,24 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
 
 // ---- converters (fp8 caches) ----------------------------------------------------
 
+// Row and 16-code group of item `rest` (0 .. RPW*C16-1) of converter v.  With
+// 8 groups per row (two 64-column halves of f16) a quarter-warp takes two
+// adjacent rows and complementary halves: its 16-byte code loads cover eight
+// distinct bank groups, and so do its swizzled f16 stores (the rows' XOR keys
+// differ in the low bit).  One row per quarter-warp would store both halves
+// to the same four bank groups.
+template <int C16, int RPW>
+__device__ __forceinline__ void code_group(int rest, int v, int& row, int& c16) {
+    if constexpr (C16 == 8) {
+        const int rs = (rest >> 2) & 1;
+        row = v * RPW + (rest >> 4) * 2 + rs;
+        c16 = (rest & 3) + 4 * (rs ^ ((rest >> 3) & 1));
+    } else {
+        row = v * RPW + rest / C16;
+        c16 = rest % C16;
+    }
+}
+
 // Converter v (0 .. NCV-1) widens rows v*16 .. v*16+15 of every fp8 stage's K
 // and V (exactly, e4m3 -> f16) into the swizzled staging slot of the consumer
 // that takes the chunk; tokens that do not take part (past the end, or in a
@@ -679,16 +697,16 @@ __device__ __forceinline__ void convert(const DecodeParams& p, SegIter<kCH>& it,
             for (int i = 0; i < PER_LANE; ++i) {
                 const int idx = lane + 32 * i;
                 const int part = idx / (RPW * C16);
-                const int rest = idx % (RPW * C16);
-                const int row = v * RPW + rest / C16, c16 = rest % C16;
+                int row, c16;
+                code_group<C16, RPW>(idx % (RPW * C16), v, row, c16);
                 raw[i] = *reinterpret_cast<const uint4*>((part ? sv : sk) + row * D + c16 * 16);
             }
 #pragma unroll
             for (int i = 0; i < PER_LANE; ++i) {
                 const int idx = lane + 32 * i;
                 const int part = idx / (RPW * C16);
-                const int rest = idx % (RPW * C16);
-                const int row = v * RPW + rest / C16, c16 = rest % C16;
+                int row, c16;
+                code_group<C16, RPW>(idx % (RPW * C16), v, row, c16);
                 bool valid = whole;
                 if (!whole) {
                     const int jrel = ((c * kCH + row) >> p.log2_bs) - ((c * kCH) >> p.log2_bs);
