@@ -135,3 +135,73 @@ def test_get_device_error_needs_output_pointer(lib):
     f = lib.pkv_get_device_error
     f.argtypes = [V, V]
     assert f(None, None) == 1
+
+
+def _write_fp8(lib, **kw):
+    a = dict(k=DUMMY, v=DUMMY, slots=DUMMY, kc=DUMMY, vc=DUMMY, ks=DUMMY, vs=DUMMY, T=4, Hkv=2,
+             d=128, bs=16, NB=8)
+    a.update(kw)
+    f = lib.pkv_kv_cache_write_fp8
+    i32 = ctypes.c_int32
+    f.argtypes = [V, V, V, V, V, V, V, i32, i32, i32, i32, i32, V]
+    return f(a["k"], a["v"], a["slots"], a["kc"], a["vc"], a["ks"], a["vs"], a["T"], a["Hkv"],
+             a["d"], a["bs"], a["NB"], None)
+
+
+def test_fp8_write_rejects_bad_args(lib):
+    assert _write_fp8(lib, T=-1) == 1
+    assert _write_fp8(lib, NB=0) == 1
+    assert _write_fp8(lib, d=96) == 2           # unsupported head_dim
+    assert _write_fp8(lib, T=0) == 0            # nothing to do
+    assert _write_fp8(lib, ks=None) == 1        # the per-head scales are required
+    assert _write_fp8(lib, vs=None) == 1
+    assert _write_fp8(lib, k=V(0x10008)) == 1   # misaligned input rows
+
+
+def _prefix(lib, **kw):
+    a = dict(q=DUMMY, kc=DUMMY, vc=DUMMY, bt=DUMMY, sl=DUMMY, bs=16, scale=0.125, out=DUMMY,
+             B=2, Hq=8, Hkv=2, d=128, maxb=4, NB=8, maxL=64, qdt=1, kvdt=1, odt=1, po=DUMMY,
+             pl=DUMMY, npfx=1, maxm=2, maxpl=64, ws=DUMMY, wsb=1 << 20)
+    a.update(kw)
+    f = lib.pkv_paged_attention_decode_prefix
+    i32 = ctypes.c_int32
+    f.argtypes = [V, V, V, V, V, i32, ctypes.c_float, V, i32, i32, i32, i32, i32, i32, i32,
+                  ctypes.c_int, ctypes.c_int, ctypes.c_int, V, V, i32, i32, i32, V,
+                  ctypes.c_size_t, V]
+    return f(a["q"], a["kc"], a["vc"], a["bt"], a["sl"], a["bs"], a["scale"], a["out"], a["B"],
+             a["Hq"], a["Hkv"], a["d"], a["maxb"], a["NB"], a["maxL"], a["qdt"], a["kvdt"],
+             a["odt"], a["po"], a["pl"], a["npfx"], a["maxm"], a["maxpl"], a["ws"], a["wsb"],
+             None)
+
+
+def test_prefix_decode_rejects_bad_args(lib):
+    # the checks the prefix-aware call shares with the plain decode (made
+    # before any device is touched)
+    assert _prefix(lib, Hq=6, Hkv=4) == 1
+    assert _prefix(lib, bs=24) == 1
+    assert _prefix(lib, d=80) == 2
+    assert _prefix(lib, odt=2) == 2
+    assert _prefix(lib, q=None) == 1
+    assert _prefix(lib, out=V(0x10001)) == 1
+    assert _prefix(lib, B=0) == 0
+
+
+def _swap(lib, **kw):
+    a = dict(sk=DUMMY, sv=DUMMY, dk=DUMMY, dv=DUMMY, bm=DUMMY, n=3, sNB=8, dNB=8, Hkv=2, d=64,
+             bs=16, dt=1)
+    a.update(kw)
+    f = lib.pkv_swap_blocks
+    i32 = ctypes.c_int32
+    f.argtypes = [V, V, V, V, V, i32, i32, i32, i32, i32, i32, ctypes.c_int, V]
+    return f(a["sk"], a["sv"], a["dk"], a["dv"], a["bm"], a["n"], a["sNB"], a["dNB"], a["Hkv"],
+             a["d"], a["bs"], a["dt"], None)
+
+
+def test_swap_rejects_bad_args(lib):
+    assert _swap(lib, n=-1) == 1
+    assert _swap(lib, sNB=0) == 1
+    assert _swap(lib, dt=7) == 1                # unknown dtype
+    assert _swap(lib, d=96) == 2
+    assert _swap(lib, n=0) == 0                 # nothing to do
+    assert _swap(lib, bm=None) == 1
+    assert _swap(lib, dk=None) == 1
