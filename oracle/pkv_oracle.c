@@ -79,10 +79,17 @@ static double e4m3_bits_to_double(uint8_t b) {
     int m = b & 0x7;
     double v;
     if (e == 0xF && m == 0x7) return NAN;
+    int bias = 7, sub_exp = -6;
+#if ORACLE_MUTANT == 11
+    bias = 8; /* planted: exponent bias of e5m2-like formats */
+#endif
+#if ORACLE_MUTANT == 12
+    sub_exp = -7; /* planted: subnormals one binade too low */
+#endif
     if (e == 0)
-        v = ldexp((double)m / 8.0, -6);
+        v = ldexp((double)m / 8.0, sub_exp);
     else
-        v = ldexp(1.0 + (double)m / 8.0, e - 7);
+        v = ldexp(1.0 + (double)m / 8.0, e - bias);
     return sign ? -v : v;
 }
 
@@ -355,7 +362,9 @@ int oracle_decode_partitioned(const void* q, int q_dtype, const void* k_cache,
                     double mn = m > bm ? m : bm;
                     double alpha = (m == -INFINITY) ? 0.0 : exp(m - mn);
                     l *= alpha;
+#if ORACLE_MUTANT != 14 /* planted (14): the running sum is not rescaled */
                     for (int k = 0; k < d; ++k) acc[k] *= alpha;
+#endif
                     for (int t = tb; t < te; ++t) {
                         double sc = 0.0;
                         for (int k = 0; k < d; ++k) sc += qv[k] * Kc[(size_t)t * d + k];
@@ -379,7 +388,11 @@ int oracle_decode_partitioned(const void* q, int q_dtype, const void* k_cache,
             for (int k = 0; k < d; ++k) tot[k] = 0.0;
             for (int p = 0; p < nparts; ++p) {
                 double f = exp(pm[p] - M);
+#if ORACLE_MUTANT == 15
+                Z += pl[p]; /* planted: the normaliser merged without its weight */
+#else
                 Z += f * pl[p];
+#endif
                 for (int k = 0; k < d; ++k) tot[k] += f * pacc[(size_t)p * d + k];
             }
             for (int k = 0; k < d; ++k) o[k] = tot[k] / Z;
@@ -481,6 +494,9 @@ int oracle_swap_blocks(const void* src_k, const void* src_v, void* dst_k, void* 
     size_t blk = (size_t)Hkv * bs * d * elem_size;
     for (int i = 0; i < n; ++i) {
         int64_t s = block_mapping[2 * i], t = block_mapping[2 * i + 1];
+#if ORACLE_MUTANT == 13
+        int64_t tmp = s; s = t; t = tmp; /* planted: pair read backwards */
+#endif
         if (s < 0 || t < 0 || s >= src_blocks || t >= dst_blocks) {
             ++bad;
             continue;
@@ -514,13 +530,20 @@ void oracle_quantize_e4m3(const float* x, int n, float scale, uint8_t* out) {
         double a = fabs(y);
         if (a >= 448.0) {
             out[i] = (uint8_t)(sign | 0x7E);
+#if ORACLE_MUTANT == 10
+            out[i] = (uint8_t)(sign | 0x7F); /* planted: saturates to the NaN code */
+#endif
             continue;
         }
         int best = 0;
         double bestd = INFINITY;
         for (int c = 0; c <= 0x7E; ++c) {
             double dv = fabs(a - e4m3_bits_to_double((uint8_t)c));
-            if (dv < bestd || (dv == bestd && (c & 1) == 0)) {
+            int tie_to = 0;
+#if ORACLE_MUTANT == 9
+            tie_to = 1; /* planted: ties go to the odd code */
+#endif
+            if (dv < bestd || (dv == bestd && (c & 1) == tie_to)) {
                 bestd = dv;
                 best = c;
             }

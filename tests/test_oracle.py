@@ -483,6 +483,30 @@ def _pin_suite(lib):
     oracle.copy_blocks(a, a.copy(), np.array([[1, 3]], np.int64), lib=lib)
     if not np.array_equal(a[3], a0[1]):
         fails.append("copy")
+    # the split-sequence restatement (partitions of 16 tokens over 8-token
+    # blocks, so a partition's running max grows inside it) equals brute force
+    try:
+        got = oracle.decode_partitioned(q, kc, vc, bt, sl, 0.25, 16, lib=lib)
+        if not np.allclose(got, brute_all(q, Kc, Vc, 0.25), rtol=0, atol=1e-12):
+            fails.append("partitioned")
+    except oracle.OracleError:
+        fails.append("partitioned-error")
+    # swap between pools of 3 and 2 blocks: dst[0] = src[1]
+    src = np.arange(3 * 2 * 2 * 2, dtype=np.float32).reshape(3, 2, 2, 2)
+    dst = np.zeros((2, 2, 2, 2), np.float32)
+    dst_v = dst.copy()
+    oracle.swap_blocks(src, src + 100, dst, dst_v, np.array([[1, 0]], np.int64), lib=lib)
+    if not (np.array_equal(dst[0], src[1]) and np.array_equal(dst_v[0], src[1] + 100)
+            and not dst[1].any()):
+        fails.append("swap")
+    # e4m3 codes fixed by the format (bias 7, 3 mantissa bits, subnormals below
+    # 2^-6, largest finite 448) and round-to-nearest-even: 1, the two ties
+    # next to it, saturation both ways, the smallest subnormal and a subnormal tie
+    x = np.array([1.0, 1.0625, 1.1875, 1000.0, -1000.0, 2.0 ** -9, 1.5 * 2.0 ** -9],
+                 np.float32)
+    want = np.array([0x38, 0x38, 0x3A, 0x7E, 0xFE, 0x01, 0x02], np.uint8)
+    if not np.array_equal(oracle.quantize_e4m3(x, 1.0, lib=lib), want):
+        fails.append("e4m3")
     return fails
 
 
@@ -490,7 +514,7 @@ def test_pins_pass_on_the_real_oracle():
     assert _pin_suite(oracle.load()) == []
 
 
-@pytest.mark.parametrize("mutant", [1, 2, 3, 4, 5, 6, 7, 8])
+@pytest.mark.parametrize("mutant", list(range(1, 16)))
 def test_planted_mistake_is_caught(mutant):
     with tempfile.TemporaryDirectory() as td:
         path = oracle.build(mutant=mutant, out_path=os.path.join(td, f"m{mutant}.so"))
