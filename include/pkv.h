@@ -177,7 +177,9 @@ pkv_status pkv_decode_workspace_init(void* workspace, size_t workspace_bytes,
  *                 block_tables must not be written by the kernel immediately
  *                 before this call if that kernel releases its dependents early
  *                 (griddepcontrol.launch_dependents); host copies and ordinary
- *                 kernels are fine, and so is pkv_kv_cache_write.
+ *                 kernels are fine, and so is pkv_kv_cache_write.  With
+ *                 partition_size > 0 on the bf16/fp8 path a merge kernel
+ *                 follows on the same stream.
  *   workspace     device scratch of at least pkv_decode_workspace_bytes(...)
  *                 bytes, 256-byte aligned, zeroed once by
  *                 pkv_decode_workspace_init.  Calls that overlap in time need
@@ -242,9 +244,10 @@ size_t pkv_decode_prefix_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
  *   Other arguments as pkv_paged_attention_decode (partition_size automatic).
  *   Supported: q and caches PKV_BF16, head_dim 64 or 128, block_size >= 8;
  *   other configurations return PKV_ERR_UNSUPPORTED.
- *   Ordering: two kernels on `stream`, the shared pass first; both read
- *   seq_lens, block_tables, prefix_of and prefix_lens before waiting for the
- *   previous kernel, with the same rule as pkv_paged_attention_decode.
+ *   Ordering: three kernels on `stream`: the shared pass, each request's own
+ *   pass, and the merge of the two; the first two read seq_lens,
+ *   block_tables, prefix_of and prefix_lens before waiting for the previous
+ *   kernel, with the same rule as pkv_paged_attention_decode.
  *   Device checks: a group id >= num_prefixes, a prefix length that is not a
  *   multiple of block_size or exceeds max_prefix_len (it is clamped and
  *   rounded down), and a group with more than max_prefix_members requests
