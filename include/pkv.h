@@ -71,7 +71,8 @@ typedef enum pkv_dtype {
 #define PKV_DEVERR_BAD_SLOT 0x1u       /* write: slot >= num_blocks*block_size      */
 #define PKV_DEVERR_BAD_BLOCK 0x2u      /* decode: table entry outside [0,num_blocks) */
 #define PKV_DEVERR_BAD_SEQ_LEN 0x4u    /* decode: seq_len < 0 or > max_blocks*bs    */
-#define PKV_DEVERR_BAD_PAIR 0x8u       /* copy/swap: block id out of range          */
+#define PKV_DEVERR_BAD_PAIR 0x8u       /* copy/swap: block id out of range; copy:
+                                          a dst repeated or also a src            */
 #define PKV_DEVERR_TIMEOUT 0x10u       /* a bounded in-kernel wait gave up          */
 #define PKV_DEVERR_PREFIX 0x20u        /* prefix decode: bad group id, length or size */
 
@@ -311,8 +312,11 @@ size_t pkv_decode_noalloc_scratch_bytes(void);
  * v_cache[dst] = v_cache[src] (all kv heads, all slots), bit-exact.
  *
  *   block_mapping [num_pairs, 2] int64 (src, dst).  dst ids must be distinct
- *                 and no dst may also be a src in the same call.  Out-of-range
- *                 ids: pair skipped, PKV_DEVERR_BAD_PAIR.
+ *                 and no dst may also be a src in the same call (then the
+ *                 copies touch disjoint blocks and their order is immaterial);
+ *                 the device checks this and raises PKV_DEVERR_BAD_PAIR for a
+ *                 call that breaks it, whose result is then unspecified.
+ *                 Out-of-range ids: pair skipped, PKV_DEVERR_BAD_PAIR.
  *   elem_bytes of dtype: 4 (F32), 2 (BF16), 1 (FP8_E4M3).
  */
 pkv_status pkv_copy_blocks(void* k_cache, void* v_cache, const int64_t* block_mapping,

@@ -29,7 +29,7 @@ __all__ = [
     "PkvError", "LIB_PATH", "lib", "kv_cache_write", "paged_attention_decode", "copy_blocks",
     "decode_workspace_bytes", "new_workspace", "get_device_error", "status_string", "DEVERR",
     "paged_attention_decode_noalloc", "BlockAllocator", "waste_compare", "swap_blocks",
-    "kv_cache_write_fp8",
+    "kv_cache_write_fp8", "workspace_init",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpkv.so")
@@ -184,6 +184,16 @@ def new_workspace(nbytes: int, device: torch.device | None = None) -> torch.Tens
         _check("pkv_decode_workspace_init",
                _get_lib().pkv_decode_workspace_init(_ptr(buf), buf.numel(), _stream(dev)))
     return buf
+
+
+def workspace_init(workspace: torch.Tensor) -> None:
+    """Zero a decode workspace on the current stream (pkv_decode_workspace_init):
+    once after allocating it, and again after a call reported TIMEOUT."""
+    dev = _need_cuda(workspace)
+    with torch.cuda.device(dev):
+        _check("pkv_decode_workspace_init",
+               _get_lib().pkv_decode_workspace_init(
+                   _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(dev)))
 
 
 def _workspace(dev: torch.device, nbytes: int) -> torch.Tensor:
@@ -393,12 +403,15 @@ def paged_attention_decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cac
                                    block_size: int | None = None, scale: float | None = None,
                                    out: torch.Tensor | None = None, *,
                                    max_seq_len: int | None = None, partition_size: int = 0,
-                                   out_dtype: torch.dtype | None = None) -> torch.Tensor:
+                                   out_dtype: torch.dtype | None = None,
+                                   k_scale: torch.Tensor | None = None,
+                                   v_scale: torch.Tensor | None = None) -> torch.Tensor:
     """The same decode through ``pkv_paged_attention_decode_noalloc``: no
     workspace argument, the library's fixed device scratch array is used.
 
     For callers that may not allocate device memory (see the C header).  Calls
     on one device share that array and must not overlap on the GPU.
+    ``k_scale`` / ``v_scale`` as in :func:`paged_attention_decode` (fp8 caches).
     """
     global _noalloc_declared
     L = _get_lib()
@@ -411,7 +424,7 @@ def paged_attention_decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cac
         L.pkv_decode_noalloc_scratch_bytes.argtypes = []
         L.pkv_decode_noalloc_scratch_bytes.restype = sz
         _noalloc_declared = True
-    dev = _need_cuda(q, k_cache, v_cache, block_tables, seq_lens, out)
+    dev = _need_cuda(q, k_cache, v_cache, block_tables, seq_lens, out, k_scale, v_scale)
     if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32:
         raise TypeError("block_tables and seq_lens must be int32")
     B, Hq, d = q.shape
@@ -431,8 +444,8 @@ def paged_attention_decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cac
         st = L.pkv_paged_attention_decode_noalloc(
             _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(seq_lens), bs,
             float(scale), _ptr(out), B, Hq, Hkv, d, max_blocks, NB, int(max_seq_len),
-            _dtype_code(q), _dtype_code(k_cache), _dtype_code(out), None, None,
-            int(partition_size), _stream(dev))
+            _dtype_code(q), _dtype_code(k_cache), _dtype_code(out), _ptr(k_scale),
+            _ptr(v_scale), int(partition_size), _stream(dev))
     _check("pkv_paged_attention_decode_noalloc", st)
     return out
 

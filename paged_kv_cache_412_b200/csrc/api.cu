@@ -227,23 +227,14 @@ pkv_status pkv_decode_workspace_init(void* workspace, size_t workspace_bytes,
 }  // extern "C"
 
 namespace pkv {
-namespace {
 
-// Shared-prefix arguments of pkv_paged_attention_decode_prefix.
-struct PrefixArgs {
-    const int32_t* prefix_of;
-    const int32_t* prefix_lens;
-    int num_prefixes, max_members, max_prefix_len;
-};
-
-pkv_status decode_entry(const void* q, const void* k_cache, const void* v_cache,
-                        const int32_t* block_tables, const int32_t* seq_lens, int32_t block_size,
-                        float scale, void* out, int32_t num_seqs, int32_t num_q_heads,
-                        int32_t num_kv_heads, int32_t head_dim, int32_t max_blocks_per_seq,
-                        int32_t num_blocks, int32_t max_seq_len, pkv_dtype q_dtype,
-                        pkv_dtype kv_dtype, pkv_dtype out_dtype, const float* k_scale,
-                        const float* v_scale, int32_t partition_size, void* workspace,
-                        size_t workspace_bytes, pkv_stream_t stream, const PrefixArgs* pa) {
+pkv_status check_decode_args(const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* block_tables, const int32_t* seq_lens,
+                             int32_t block_size, float scale, const void* out, int32_t num_seqs,
+                             int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                             int32_t max_blocks_per_seq, int32_t num_blocks, int32_t max_seq_len,
+                             pkv_dtype q_dtype, pkv_dtype kv_dtype, pkv_dtype out_dtype,
+                             const float* k_scale, const float* v_scale, int32_t partition_size) {
     if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || head_dim <= 0 ||
         max_blocks_per_seq <= 0 || num_blocks <= 0 || max_seq_len < 0 || partition_size < 0)
         return PKV_ERR_INVALID_ARG;
@@ -268,6 +259,41 @@ pkv_status decode_entry(const void* q, const void* k_cache, const void* v_cache,
     if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) ||
         !aligned(block_tables, 4) || !aligned(seq_lens, 4) || !aligned(out, elem_size(out_dtype)))
         return PKV_ERR_INVALID_ARG;
+    return PKV_OK;
+}
+
+namespace {
+
+// Test-only fault of the next decode call on this host thread (DecodeFault).
+struct PendingFault {
+    int mode = kFaultNone;
+    int arg = 0;
+    unsigned long long wait_ns = 0;
+};
+thread_local PendingFault t_fault;
+
+// Shared-prefix arguments of pkv_paged_attention_decode_prefix.
+struct PrefixArgs {
+    const int32_t* prefix_of;
+    const int32_t* prefix_lens;
+    int num_prefixes, max_members, max_prefix_len;
+};
+
+pkv_status decode_entry(const void* q, const void* k_cache, const void* v_cache,
+                        const int32_t* block_tables, const int32_t* seq_lens, int32_t block_size,
+                        float scale, void* out, int32_t num_seqs, int32_t num_q_heads,
+                        int32_t num_kv_heads, int32_t head_dim, int32_t max_blocks_per_seq,
+                        int32_t num_blocks, int32_t max_seq_len, pkv_dtype q_dtype,
+                        pkv_dtype kv_dtype, pkv_dtype out_dtype, const float* k_scale,
+                        const float* v_scale, int32_t partition_size, void* workspace,
+                        size_t workspace_bytes, pkv_stream_t stream, const PrefixArgs* pa) {
+    {
+        const pkv_status cs = check_decode_args(
+            q, k_cache, v_cache, block_tables, seq_lens, block_size, scale, out, num_seqs,
+            num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, num_blocks, max_seq_len,
+            q_dtype, kv_dtype, out_dtype, k_scale, v_scale, partition_size);
+        if (cs != PKV_OK || num_seqs == 0) return cs;
+    }
     const DeviceInfo* di0 = current_device_info();
     if (!di0) return PKV_ERR_CUDA;
     const bool use_prefix = pa && pa->num_prefixes > 0;
@@ -293,7 +319,7 @@ pkv_status decode_entry(const void* q, const void* k_cache, const void* v_cache,
     DecodePlan pl;
     if (!make_decode_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len,
                           partition_size, &pl, pfx_bytes))
-        return PKV_ERR_CUDA;
+        return PKV_ERR_INVALID_ARG;  // the device was queried above: the sizes are at fault
     if (!workspace || workspace_bytes < pl.bytes || !aligned(workspace, 256))
         return PKV_ERR_WORKSPACE;
     if ((long long)num_blocks * num_kv_heads * block_size > 0x7fffffffLL)
@@ -348,6 +374,13 @@ pkv_status decode_entry(const void* q, const void* k_cache, const void* v_cache,
     p.rec_cap = (long long)pl.records;
     p.out_dtype = out_dtype;
     p.scale_log2 = scale * 1.4426950408889634f;
+    p.wait_ns = kWaitLimitNs;
+    if (t_fault.mode != kFaultNone) {  // consumed by this call
+        p.fault_mode = t_fault.mode;
+        p.fault_arg = t_fault.arg;
+        p.wait_ns = t_fault.wait_ns;
+        t_fault = PendingFault{};
+    }
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
     if (use_prefix) {
         const size_t rows = (size_t)pfx_splits * num_seqs * num_q_heads;
@@ -543,3 +576,18 @@ pkv_status pkv_get_device_error(pkv_stream_t stream, uint32_t* flags) {
 }
 
 }  // extern "C"
+
+// Not declared in the public header: arms a test-only fault (pkv::DecodeFault)
+// for the next decode call made by the calling host thread, with every
+// in-kernel wait of that call bounded by wait_ns instead of the default 2 s.
+// Used by the failure-detection tests to make a bounded wait run out.
+extern "C" pkv_status pkv_internal_decode_fault(int32_t mode, int32_t arg,
+                                                unsigned long long wait_ns) {
+    if (mode < pkv::kFaultNone || mode > pkv::kFaultSkipStage || arg < 0 || wait_ns == 0 ||
+        wait_ns > pkv::kWaitLimitNs)
+        return PKV_ERR_INVALID_ARG;
+    pkv::t_fault.mode = mode;
+    pkv::t_fault.arg = arg;
+    pkv::t_fault.wait_ns = wait_ns;
+    return PKV_OK;
+}

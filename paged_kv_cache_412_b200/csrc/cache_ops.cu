@@ -121,10 +121,27 @@ __global__ void kv_cache_write_fp8_kernel(const uint4* __restrict__ k, const uin
     }
 }
 
+// Copy-on-write contract of one call, checked for pair i by one CTA: its
+// destination is no other pair's destination and no pair's source (its own
+// included).  Under it the pairs' copies touch disjoint blocks, so their order
+// does not matter; a call that breaks it has an unspecified result and raises
+// PKV_DEVERR_BAD_PAIR.  Block-uniform; every thread must call it.
+__device__ __forceinline__ void check_cow_contract(const int64_t* __restrict__ pairs,
+                                                   int num_pairs, int i, int64_t dst,
+                                                   unsigned* err) {
+    bool clash = false;
+    for (int j = threadIdx.x; j < num_pairs; j += blockDim.x) {
+        const int64_t sj = __ldg(pairs + 2 * j), dj = __ldg(pairs + 2 * j + 1);
+        clash |= (j != i && dj == dst) || sj == dst;
+    }
+    if (__syncthreads_or(clash) && threadIdx.x == 0) raise_error(err, PKV_DEVERR_BAD_PAIR);
+}
+
 // grid.x = pair, grid.y = 0 (K) / 1 (V), grid.z = slice of the block.
 __global__ void copy_blocks_kernel(uint4* __restrict__ kc, uint4* __restrict__ vc,
-                                   const int64_t* __restrict__ pairs, long long vecs_per_block,
-                                   int slice_vecs, int num_blocks, unsigned* err) {
+                                   const int64_t* __restrict__ pairs, int num_pairs,
+                                   long long vecs_per_block, int slice_vecs, int num_blocks,
+                                   unsigned* err) {
     const int64_t src = __ldg(pairs + 2 * blockIdx.x);
     const int64_t dst = __ldg(pairs + 2 * blockIdx.x + 1);
     if (src < 0 || dst < 0 || src >= num_blocks || dst >= num_blocks) {
@@ -132,6 +149,8 @@ __global__ void copy_blocks_kernel(uint4* __restrict__ kc, uint4* __restrict__ v
             raise_error(err, PKV_DEVERR_BAD_PAIR);
         return;
     }
+    if (blockIdx.y == 0 && blockIdx.z == 0)
+        check_cow_contract(pairs, num_pairs, blockIdx.x, dst, err);
     uint4* base = blockIdx.y == 0 ? kc : vc;
     const uint4* s = base + src * vecs_per_block;
     uint4* d = base + dst * vecs_per_block;
@@ -254,8 +273,8 @@ pkv_status launch_copy_blocks(void* k_cache, void* v_cache, const int64_t* pairs
     if (slices > 65535 || num_pairs > 2147483647) return PKV_ERR_UNSUPPORTED;
     dim3 grid(num_pairs, 2, (unsigned)slices);
     copy_blocks_kernel<<<grid, threads, 0, stream>>>(static_cast<uint4*>(k_cache),
-                                                      static_cast<uint4*>(v_cache), pairs, vecs,
-                                                      slice, num_blocks, err);
+                                                      static_cast<uint4*>(v_cache), pairs,
+                                                      num_pairs, vecs, slice, num_blocks, err);
     return cudaGetLastError() == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 

@@ -180,7 +180,7 @@ struct Producer {
             const int stage = (int)(n % C::NSTAGE);
             const uint32_t phase = (n / C::NSTAGE) & 1u;
             int ok = 1;
-            if (lane == 0) ok = !ctrl[0] && mbar_wait(&empty[stage], phase ^ 1u);
+            if (lane == 0) ok = !ctrl[0] && mbar_wait(&empty[stage], phase ^ 1u, p.wait_ns);
             ok = __shfl_sync(FULL_MASK, ok, 0);
             if (!ok) {
                 if (lane == 0) {
@@ -193,6 +193,13 @@ struct Producer {
                 // K/V and q may come from the previous kernel in the stream.
                 griddep_wait();
                 waited = true;
+            }
+            if (p.fault_mode == kFaultSkipStage && blockIdx.x == 0 && (int)n == p.fault_arg) {
+                // test-only fault: this stage is never filled, so its
+                // consumer's bounded wait runs out (nothing is in flight)
+                ++issued;
+                last_n = n;
+                continue;
             }
             uint32_t nvalid = 0, bad = 0;
             for (int j = ja; j <= jb; ++j) {
@@ -324,7 +331,7 @@ struct Producer {
             const int k_max = min(issued, C::NSTAGE / C::NPROD);
             for (int k = 0; k < k_max; ++k) {
                 const unsigned nn = last_n - (unsigned)(k * C::NPROD);
-                mbar_wait(&full[nn % C::NSTAGE], (nn / C::NSTAGE) & 1u);
+                mbar_wait(&full[nn % C::NSTAGE], (nn / C::NSTAGE) & 1u, p.wait_ns);
             }
         }
     }
@@ -407,7 +414,7 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                 const bool mine = (int)(n_chunk % C::NCONS) == me;
                 ++n_chunk;
                 if (!mine) continue;
-                if (ctrl[0] || !mbar_wait(&sfull[me], sphase)) {
+                if (ctrl[0] || !mbar_wait(&sfull[me], sphase, p.wait_ns)) {
                     if (lane == 0 && !ctrl[0]) {
                         ctrl[0] = 1;
                         raise_error(p.err, PKV_DEVERR_TIMEOUT);
@@ -418,7 +425,7 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                 bad = sl_bad[me];
                 sk = smem + S::OFF_STG + me * C::SLOT_BYTES;
             } else {
-                if (ctrl[0] || !mbar_wait(&full[ring.stage], ring.phase)) {
+                if (ctrl[0] || !mbar_wait(&full[ring.stage], ring.phase, p.wait_ns)) {
                     if (lane == 0 && !ctrl[0]) {
                         ctrl[0] = 1;
                         raise_error(p.err, PKV_DEVERR_TIMEOUT);
@@ -605,7 +612,7 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
         // (an fp8 consumer that took no chunk of the segment hands over the
         // empty state)
         const int slot = me * S::NDUMP + dring.stage;
-        if (!mbar_wait(&dempty[slot], dring.phase ^ 1u)) {
+        if (!mbar_wait(&dempty[slot], dring.phase ^ 1u, p.wait_ns)) {
             if (lane == 0) {
                 ctrl[0] = 1;
                 raise_error(p.err, PKV_DEVERR_TIMEOUT);
@@ -677,8 +684,8 @@ __device__ __forceinline__ void convert(const DecodeParams& p, SegIter<kCH>& it,
         for (int c = sg.c0; c < sg.c1; ++c, ++n_chunk) {
             const int slot = (int)(n_chunk % C::NCONS);
             const uint32_t sph = (n_chunk / C::NCONS) & 1u;
-            if (ctrl[0] || !mbar_wait(&full[ring.stage], ring.phase) ||
-                !mbar_wait(&sempty[slot], sph ^ 1u)) {
+            if (ctrl[0] || !mbar_wait(&full[ring.stage], ring.phase, p.wait_ns) ||
+                !mbar_wait(&sempty[slot], sph ^ 1u, p.wait_ns)) {
                 if (lane == 0 && !ctrl[0]) {
                     ctrl[0] = 1;
                     raise_error(p.err, PKV_DEVERR_TIMEOUT);
@@ -811,7 +818,7 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
 #pragma unroll
         for (int k = 0; k < C::NCONS; ++k) {
             const int slot = k * S::NDUMP + dring.stage;
-            if (ctrl[0] || !mbar_wait(&dfull[slot], dring.phase)) {
+            if (ctrl[0] || !mbar_wait(&dfull[slot], dring.phase, p.wait_ns)) {
                 if (lane == 0 && !ctrl[0]) {
                     ctrl[0] = 1;
                     raise_error(p.err, PKV_DEVERR_TIMEOUT);
@@ -931,10 +938,12 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
         if (lane == 0) {
             const uint64_t t0 = global_timer_ns();
             for (long long uu = si.u_first; uu <= si.u_last && ok; ++uu) {
-                if (uu == si.u) continue;
+                // (the test-only fault waits for the merger's own flag too,
+                // which nothing sets)
+                if (uu == si.u && p.fault_mode != kFaultMergeFlag) continue;
                 volatile unsigned* f = p.ready + si.bg + uu;
                 for (uint32_t it = 0; *f == 0u; ++it) {
-                    if ((it & 63u) == 63u && global_timer_ns() - t0 > kWaitLimitNs) {
+                    if ((it & 63u) == 63u && global_timer_ns() - t0 > p.wait_ns) {
                         ok = 0;
                         break;
                     }

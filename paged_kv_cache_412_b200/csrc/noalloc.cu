@@ -65,15 +65,20 @@ extern "C" pkv_status pkv_paged_attention_decode_noalloc(
     pkv_stream_t stream) {
     using namespace pkv;
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    // Sizes the workspace planner rejects are passed on so the decode call
-    // reports the precise argument error; nothing is launched for them.
+    // Every argument check comes before the scratch array is touched, so a
+    // rejected call puts no work on the stream (nor on a graph being captured).
+    const pkv_status cs = check_decode_args(
+        q, k_cache, v_cache, block_tables, seq_lens, block_size, scale, out, num_seqs,
+        num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, num_blocks, max_seq_len, q_dtype,
+        kv_dtype, out_dtype, k_scale, v_scale, partition_size);
+    if (cs != PKV_OK || num_seqs == 0) return cs;
     DecodePlan pl;
-    const bool planned = num_seqs > 0 && max_blocks_per_seq > 0 && num_blocks > 0 &&
-                         make_decode_plan(num_seqs, num_q_heads, num_kv_heads, head_dim,
-                                          block_size, max_seq_len, partition_size, &pl);
-    if (planned && pl.bytes > kScratchBytes) return PKV_ERR_WORKSPACE;  // beyond the fixed maximum
+    if (!make_decode_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, max_seq_len,
+                          partition_size, &pl))
+        return current_device_info() ? PKV_ERR_INVALID_ARG : PKV_ERR_CUDA;
+    if (pl.bytes > kScratchBytes) return PKV_ERR_WORKSPACE;  // beyond the fixed maximum
     void* ws = nullptr;
-    if (planned) {
+    {
         const pkv_status s = scratch_address(st, &ws);
         if (s != PKV_OK) return s;
         // The array keeps the previous call's contents; the arrival counters
@@ -89,5 +94,5 @@ extern "C" pkv_status pkv_paged_attention_decode_noalloc(
                                       scale, out, num_seqs, num_q_heads, num_kv_heads, head_dim,
                                       max_blocks_per_seq, num_blocks, max_seq_len, q_dtype,
                                       kv_dtype, out_dtype, k_scale, v_scale, partition_size, ws,
-                                      planned ? kScratchBytes : 0, stream);
+                                      kScratchBytes, stream);
 }

@@ -93,7 +93,33 @@ struct DecodeParams {
     const float* pfx_acc;        // [pfx_splits][num_seqs][num_q_heads][head_dim]
     const float* pfx_ml;         // [pfx_splits][num_seqs][num_q_heads][2]
     int num_prefixes, max_prefix_len, pfx_splits;
+    // Bound of every in-kernel wait (ns of global time), and a test-only fault
+    // (DecodeFault) that makes one wait run out; 0 = none.
+    unsigned long long wait_ns;
+    int fault_mode, fault_arg;
 };
+
+// Test-only faults of the tensor-core decode, set for the next decode call of
+// the calling host thread by pkv_internal_decode_fault (exported, not part of
+// the public header).  Each one makes a bounded wait run out so the give-up
+// path (PKV_DEVERR_TIMEOUT, workspace re-initialisation) can be exercised
+// without faulting the GPU:
+//   kFaultMergeFlag: the merger of a split group also waits for its own
+//     ready flag, which nothing sets;
+//   kFaultSkipStage: CTA 0's producer never arrives on the full barrier of its
+//     chunk fault_arg (no copy is issued for it), so that stage never fills.
+enum DecodeFault { kFaultNone = 0, kFaultMergeFlag = 1, kFaultSkipStage = 2 };
+
+// Host argument checks of a decode call (everything but the workspace):
+// null pointers, sizes, dtypes, head_dim, alignment.  PKV_OK if the call may
+// proceed.
+pkv_status check_decode_args(const void* q, const void* k_cache, const void* v_cache,
+                             const int32_t* block_tables, const int32_t* seq_lens,
+                             int32_t block_size, float scale, const void* out, int32_t num_seqs,
+                             int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                             int32_t max_blocks_per_seq, int32_t num_blocks, int32_t max_seq_len,
+                             pkv_dtype q_dtype, pkv_dtype kv_dtype, pkv_dtype out_dtype,
+                             const float* k_scale, const float* v_scale, int32_t partition_size);
 
 // Kernel arguments of the shared pass of pkv_paged_attention_decode_prefix.
 // CTA x handles split (x % splits) of row tile ((x / splits) % row_tiles) of

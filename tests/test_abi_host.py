@@ -205,3 +205,41 @@ def test_swap_rejects_bad_args(lib):
     assert _swap(lib, n=0) == 0                 # nothing to do
     assert _swap(lib, bm=None) == 1
     assert _swap(lib, dk=None) == 1
+
+
+def _decode_noalloc(lib, **kw):
+    a = dict(q=DUMMY, kc=DUMMY, vc=DUMMY, bt=DUMMY, sl=DUMMY, bs=16, scale=0.125, out=DUMMY,
+             B=2, Hq=8, Hkv=2, d=128, maxb=4, NB=8, maxL=64, qdt=1, kvdt=1, odt=1, ks=None,
+             vs=None, P=0)
+    a.update(kw)
+    f = lib.pkv_paged_attention_decode_noalloc
+    i32 = ctypes.c_int32
+    f.argtypes = [V, V, V, V, V, i32, ctypes.c_float, V, i32, i32, i32, i32, i32, i32, i32,
+                  ctypes.c_int, ctypes.c_int, ctypes.c_int, V, V, i32, V]
+    return f(a["q"], a["kc"], a["vc"], a["bt"], a["sl"], a["bs"], a["scale"], a["out"], a["B"],
+             a["Hq"], a["Hkv"], a["d"], a["maxb"], a["NB"], a["maxL"], a["qdt"], a["kvdt"],
+             a["odt"], a["ks"], a["vs"], a["P"], None)
+
+
+def test_noalloc_decode_checks_arguments_before_its_scratch(lib):
+    """Every argument error is reported as such, on the host, before the
+    scratch array is looked up or cleared (no device is touched)."""
+    assert _decode_noalloc(lib, Hq=6, Hkv=4) == 1
+    assert _decode_noalloc(lib, d=96) == 2
+    assert _decode_noalloc(lib, out=None) == 1
+    assert _decode_noalloc(lib, kvdt=2) == 1     # fp8 cache without scales
+    assert _decode_noalloc(lib, scale=float("inf")) == 1
+    assert _decode_noalloc(lib, B=0) == 0        # empty batch: nothing to do
+
+
+def test_internal_fault_setter_rejects_bad_modes(lib):
+    """The test-only fault setter (exported, not in the public header) accepts
+    only its known modes and a wait bound in (0, 2 s]."""
+    f = lib.pkv_internal_decode_fault
+    f.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_ulonglong]
+    f.restype = ctypes.c_int
+    assert f(7, 0, 1000000) == 1
+    assert f(1, -1, 1000000) == 1
+    assert f(1, 0, 0) == 1
+    assert f(1, 0, 3_000_000_000) == 1
+    assert f(0, 0, 1000000) == 0  # disarm

@@ -143,3 +143,77 @@ def workloads_e4m3(codes: np.ndarray) -> np.ndarray:
     oracle's code table in the oracle tests)."""
     t = torch.from_numpy(np.ascontiguousarray(codes)).view(torch.float8_e4m3fn)
     return t.to(torch.float64).numpy()
+
+
+# ---- bounded waits that run out (the fault is armed on the host) -------------
+#
+# The pages' own failure case is running out of blocks mid-generation
+# ("PagedAttention: Optimizing KV Cache Utilization in Large Language Models",
+# "Conclusion").  In the kernels the failure to guard against is a wait that
+# never ends.  Every in-kernel wait is bounded; these tests arm a test-only
+# fault for ONE decode call (pkv_internal_decode_fault, exported but not in the
+# public header) that makes one wait run out after a few milliseconds: the
+# call must raise PKV_DEVERR_TIMEOUT and return, the context must stay usable,
+# and after pkv_decode_workspace_init the same decode must match the oracle.
+
+FAULT_MERGE_FLAG, FAULT_SKIP_STAGE = 1, 2
+
+
+def _arm(pkv, mode, arg=0, wait_ns=5_000_000):
+    import ctypes
+    f = pkv._get_lib().pkv_internal_decode_fault
+    f.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_ulonglong]
+    f.restype = ctypes.c_int
+    assert f(mode, arg, wait_ns) == 0
+
+
+@pytest.mark.parametrize("mode,arg", [(FAULT_MERGE_FLAG, 0), (FAULT_SKIP_STAGE, 1)],
+                         ids=["merger-ready-flag", "stage-full-barrier"])
+def test_wait_runs_out_then_workspace_recovers(pkv, mode, arg):
+    # long requests: every (request, kv head) is split over several units, so
+    # mergers exist, and CTA 0 streams more than two stages
+    w = workloads.make_paged([4096, 3000, 1, 2500], Hq=32, Hkv=8, d=128, bs=16, dtype="bf16",
+                             seed=61)
+    dw = DevWorkload(w)
+    pkv.kv_cache_write(dw.k_new, dw.v_new, dw.slot_mapping, dw.k_cache, dw.v_cache)
+    L = int(w.seq_lens.max())
+    ws = pkv.new_workspace(pkv.decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.d, w.bs, L, 0))
+    out = torch.empty((w.B, w.Hq, w.d), dtype=torch.float32, device="cuda")
+    assert pkv.get_device_error() == 0
+    _arm(pkv, mode, arg)
+    pkv.paged_attention_decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.bs,
+                               w.scale, out, max_seq_len=L, workspace=ws)
+    flags = pkv.get_device_error()  # synchronises: the call has returned
+    assert flags & pkv.DEVERR["TIMEOUT"], hex(flags)
+    # the context is usable; a TIMEOUT leaves the workspace's counters and
+    # flags in an unknown state, so re-initialise it, then decode again
+    pkv.workspace_init(ws)
+    pkv.paged_attention_decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.bs,
+                               w.scale, out, max_seq_len=L, workspace=ws)
+    assert pkv.get_device_error() == 0
+    kc, vc = host_step(w)
+    ref = oracle.decode(w.q, kc, vc, w.block_tables, w.seq_lens, w.scale)
+    assert_decode_close(to_host_f64(out), ref, "bf16", "f32", what="decode after recovery")
+    # the fault was consumed by the one call: the next call is clean too
+    pkv.paged_attention_decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables, dw.seq_lens, w.bs,
+                               w.scale, out, max_seq_len=L, workspace=ws)
+    assert pkv.get_device_error() == 0
+
+
+def test_copy_contract_violation_is_flagged(pkv):
+    """copy_blocks pairs must name distinct destinations, none of them also a
+    source; a call that breaks it raises PKV_DEVERR_BAD_PAIR (its result is
+    unspecified, so only the flag is checked), and a valid call does not."""
+    w = workloads.make_paged([40, 40], Hq=4, Hkv=2, d=64, bs=16, dtype="bf16", seed=9,
+                             extra_blocks=8, append_last=False)
+    dw = DevWorkload(w)
+    free = [b for b in range(w.num_blocks) if b not in set(w.block_tables[w.block_tables >= 0])]
+    a, b = int(w.block_tables[0, 0]), int(w.block_tables[1, 0])
+    for pairs in ([[a, free[0]], [b, free[0]]],      # destination repeated
+                  [[a, free[0]], [free[0], free[1]]],  # a destination is also a source
+                  [[a, a]]):                          # a block copied onto itself
+        pkv.copy_blocks(dw.k_cache, dw.v_cache, to_dev(np.array(pairs, np.int64)))
+        assert pkv.get_device_error() & pkv.DEVERR["BAD_PAIR"], pairs
+    pkv.copy_blocks(dw.k_cache, dw.v_cache,
+                    to_dev(np.array([[a, free[0]], [b, free[1]]], np.int64)))
+    assert pkv.get_device_error() == 0

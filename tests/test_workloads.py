@@ -116,3 +116,13 @@ def test_prefix_groups_share_blocks_and_fill_every_token():
             assert blk >= 0
             assert not np.any(kc[blk, :, t % w.bs] == workloads.BF16_NAN)
             assert not np.any(vc[blk, :, t % w.bs] == workloads.BF16_NAN)
+
+
+def test_e4m3_codes_cover_every_binade_and_never_nan():
+    """The fp8 history draws every exponent field 0..15 (subnormals up to the
+    binade of 448) with both signs, and never a NaN code (S.1111.111)."""
+    codes = workloads.e4m3_codes(np.random.default_rng(5), (64, 1024))
+    assert not np.any((codes & 0x7F) == 0x7F)
+    assert set(np.unique((codes >> 3) & 0xF).tolist()) == set(range(16))
+    assert set(np.unique(codes >> 7).tolist()) == {0, 1}
+    assert np.any(codes == 0x7E) and np.any(codes == 0xFE)  # +-448

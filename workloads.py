@@ -35,6 +35,8 @@ stray read or write shows up) and 0 otherwise (timed runs).
 from __future__ import annotations
 
 import math
+import os
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
 
 import numpy as np
@@ -43,11 +45,38 @@ BF16_NAN = np.uint16(0x7FC0)
 E4M3_NAN = np.uint8(0x7F)
 
 
+_CHUNK = 1 << 22  # values per chunk of the threaded fills below
+_THREADS = max(1, min(16, os.cpu_count() or 1))
+
+
+def _chunked(n: int, fn) -> None:
+    """Run fn(lo, hi) over [0, n) in chunks of _CHUNK on a thread pool (the
+    numpy kernels used release the GIL); deterministic whatever the pool size."""
+    spans = [(lo, min(lo + _CHUNK, n)) for lo in range(0, n, _CHUNK)]
+    if len(spans) <= 1:
+        for lo, hi in spans:
+            fn(lo, hi)
+        return
+    with ThreadPoolExecutor(_THREADS) as ex:
+        list(ex.map(lambda sp: fn(*sp), spans))
+
+
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
-    """Round-to-nearest-even fp32 -> bf16, returned as uint16 bit patterns."""
-    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32).astype(np.uint64)
-    rounded = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
-    return rounded.astype(np.uint16)
+    """Round-to-nearest-even fp32 -> bf16, returned as uint16 bit patterns
+    (finite inputs; 32-bit integer arithmetic cannot overflow for them)."""
+    u = np.ascontiguousarray(x, dtype=np.float32).reshape(-1).view(np.uint32)
+    out = np.empty(u.shape, dtype=np.uint16)
+
+    def conv(lo, hi):
+        v = u[lo:hi]
+        r = (v >> 16) & 1
+        r += 0x7FFF
+        r += v
+        r >>= 16
+        out[lo:hi] = r
+
+    _chunked(u.size, conv)
+    return out.reshape(np.shape(x))
 
 
 def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
@@ -88,17 +117,41 @@ class Workload:
 
 
 def _normal(rng: np.random.Generator, shape, dtype: str) -> np.ndarray:
-    x = rng.standard_normal(size=shape, dtype=np.float32)
+    """N(0, 1) fp32 values (bf16 bit patterns for bf16).  Chunk i of the
+    flattened array is drawn from its own generator, seeded from one draw of
+    ``rng`` and i, so the result depends on the seed alone."""
+    n = int(np.prod(shape))
+    x = np.empty(n, dtype=np.float32)
+    base = int(rng.integers(0, 2**63 - 1))
+
+    def fill(lo, hi):
+        g = np.random.default_rng([base, lo // _CHUNK])
+        g.standard_normal(size=hi - lo, dtype=np.float32, out=x[lo:hi])
+
+    _chunked(n, fill)
+    x = x.reshape(shape)
     return x if dtype == "f32" else f32_to_bf16_bits(x)
 
 
 def e4m3_codes(rng: np.random.Generator, shape) -> np.ndarray:
-    """Random fp8 e4m3 codes (uint8): random sign, exponent field 0..10 (so
-    magnitudes up to 15, subnormals included), random mantissa; never NaN."""
+    """Random fp8 e4m3 codes (uint8): random sign, exponent field 0..15 (every
+    binade, subnormals and the top one up to 448 included), random mantissa;
+    the two NaN codes (S.1111.111) are redrawn as the largest finite magnitude
+    of the same sign, so a code is never NaN."""
     sign = rng.integers(0, 2, size=shape, dtype=np.uint8) << 7
-    exp = rng.integers(0, 11, size=shape, dtype=np.uint8) << 3
+    exp = rng.integers(0, 16, size=shape, dtype=np.uint8) << 3
     man = rng.integers(0, 8, size=shape, dtype=np.uint8)
-    return (sign | exp | man).astype(np.uint8)
+    codes = (sign | exp | man).astype(np.uint8)
+    nan = (codes & 0x7F) == 0x7F
+    codes[nan] ^= 1  # 0x7F -> 0x7E (448), 0xFF -> 0xFE (-448)
+    return codes
+
+
+def e4m3_scales(rng: np.random.Generator, num_kv_heads: int) -> np.ndarray:
+    """Per-kv-head dequantisation scales U(0.01, 0.1): with codes over the whole
+    e4m3 range the stored values reach +-44.8, and an N(0,1) token appended at
+    the smallest scale saturates only beyond |x| = 4.48."""
+    return rng.uniform(0.01, 0.1, size=num_kv_heads).astype(np.float32)
 
 
 def _cache_values(rng, shape, dtype: str) -> np.ndarray:
@@ -114,13 +167,17 @@ def _empty_cache(shape, dtype: str, poison: bool) -> np.ndarray:
     return np.full(shape, BF16_NAN if poison else 0, dtype=np.uint16)
 
 
-def _fill_history(rng, k_cache, v_cache, table_row, n_tokens, bs, dtype):
-    """Write n_tokens random K/V rows at logical positions 0..n_tokens-1."""
+def _fill_history(rng, k_cache, v_cache, table_row, n_tokens, bs, dtype, kv=None):
+    """Write n_tokens random K/V rows at logical positions 0..n_tokens-1
+    (``kv``: the rows, [n_tokens, Hkv, d] each, if already drawn)."""
     Hkv, d = k_cache.shape[1], k_cache.shape[3]
     if n_tokens <= 0:
         return
-    kh = _cache_values(rng, (n_tokens, Hkv, d), dtype)
-    vh = _cache_values(rng, (n_tokens, Hkv, d), dtype)
+    if kv is None:
+        kh = _cache_values(rng, (n_tokens, Hkv, d), dtype)
+        vh = _cache_values(rng, (n_tokens, Hkv, d), dtype)
+    else:
+        kh, vh = kv
     nfull = n_tokens // bs
     if nfull:
         blocks = np.asarray(table_row[:nfull], dtype=np.int64)
@@ -161,8 +218,17 @@ def make_paged(seq_lens, *, Hq: int, Hkv: int, d: int, bs: int, dtype: str, seed
     k_cache = _empty_cache((NB, Hkv, bs, d), dtype, poison)
     v_cache = _empty_cache((NB, Hkv, bs, d), dtype, poison)
     hist = [int(L) - 1 if (append_last and L > 0) else int(L) for L in seq_lens]
+    # every request's history rows in one draw (threaded), then laid out
+    total = int(sum(hist))
+    kh = _cache_values(rng, (total, Hkv, d), dtype)
+    vh = _cache_values(rng, (total, Hkv, d), dtype)
+    at = 0
     for b in range(B):
-        _fill_history(rng, k_cache, v_cache, tables[b], hist[b], bs, dtype)
+        n = hist[b]
+        _fill_history(rng, k_cache, v_cache, tables[b], n, bs, dtype,
+                      kv=(kh[at:at + n], vh[at:at + n]))
+        at += n
+    del kh, vh
     new_rows = [b for b in range(B) if append_last and seq_lens[b] > 0]
     T = len(new_rows)
     k_new = _normal(rng, (T, Hkv, d), qdt)
@@ -175,8 +241,8 @@ def make_paged(seq_lens, *, Hq: int, Hkv: int, d: int, bs: int, dtype: str, seed
         scale = 1.0 / math.sqrt(d)
     ks = vs = None
     if dtype == "fp8":  # per-kv-head dequantisation scales
-        ks = rng.uniform(0.05, 0.5, size=Hkv).astype(np.float32)
-        vs = rng.uniform(0.05, 0.5, size=Hkv).astype(np.float32)
+        ks = e4m3_scales(rng, Hkv)
+        vs = e4m3_scales(rng, Hkv)
     return Workload(name=name, B=B, Hq=Hq, Hkv=Hkv, d=d, bs=bs, num_blocks=NB,
                     dtype=dtype, scale=float(scale), q=q, k_cache=k_cache,
                     v_cache=v_cache, block_tables=tables, seq_lens=seq_lens,
@@ -344,8 +410,8 @@ def prefix_groups(groups, singles: int = 0, *, seed: int = 1007, suffix_lo: int 
     q = _normal(rng, (B, Hq, d), qdt)
     ks = vs = None
     if dtype == "fp8":
-        ks = rng.uniform(0.05, 0.5, size=Hkv).astype(np.float32)
-        vs = rng.uniform(0.05, 0.5, size=Hkv).astype(np.float32)
+        ks = e4m3_scales(rng, Hkv)
+        vs = e4m3_scales(rng, Hkv)
     return Workload(name="prefix_groups", B=B, Hq=Hq, Hkv=Hkv, d=d, bs=bs, num_blocks=NB,
                     dtype=dtype, scale=1.0 / math.sqrt(d), q=q, k_cache=k_cache,
                     v_cache=v_cache, block_tables=tables,
