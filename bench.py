@@ -39,6 +39,8 @@ METRIC = "paged decode attention KV GB/s (fraction of HBM peak) and tokens/s at 
 UNIT = "GB/s"
 WORKLOAD = "gqa_4k: batch 16 x 4096 tokens, 32 q / 8 KV heads, head_dim 128, block 16, bf16"
 FALLBACK_HBM_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0  # the B200's ~8 TB/s HBM3e figure, for the nominal fraction
+ROOFLINE_LAUNCHES = 2000  # decode-only launches timed for the roofline, whatever --steps
 N_LAYERS = 4
 DECODE_SRC = os.path.join(ROOT, "paged_kv_cache_412_b200", "csrc", "decode_mma.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_gqa_4k_traffic.txt")
@@ -149,11 +151,30 @@ def replica_seed(rank: int, layer: int) -> int:
     return 1002 + 100 * rank + layer
 
 
+def relaunch_under_torchrun(n_gpus: int, argv: list[str]) -> int:
+    """``--gpus N`` (N > 1) run without torchrun: start N ranks of this script
+    under torch.distributed.run on 127.0.0.1 and return their exit status."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+           f"--nproc-per-node={n_gpus}", "--master-addr=127.0.0.1", f"--master-port={port}",
+           os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
 def dist_setup(n_gpus: int):
+    """Rank, world size and local rank of this process.  The world must be the
+    requested --gpus: a mismatch is an error, never a silent single replica."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_gpus:
+        raise SystemExit(f"bench.py: --gpus {n_gpus} but WORLD_SIZE is {world}; launch one "
+                         f"process per GPU (torchrun --nproc-per-node {n_gpus}), or run "
+                         f"without torchrun and let bench.py start the ranks")
     if world > 1:
         import datetime
         import torch.distributed as dist
@@ -193,6 +214,20 @@ def dist_done(world: int):
 # CPU baseline: the oracle, as it stands, on a bounded sample
 # ---------------------------------------------------------------------------
 
+_ALL_CORES = None
+
+
+def oracle_all_cores(lib) -> int:
+    """The oracle's thread count with nothing set (all host cores, or
+    OMP_NUM_THREADS), read once: a single-thread timing sets the OpenMP
+    default of this thread to 1, so every call passes its count explicitly."""
+    global _ALL_CORES
+    if _ALL_CORES is None:
+        import oracle
+        _ALL_CORES = oracle.max_threads(lib)
+    return _ALL_CORES
+
+
 def cpu_baseline(budget_s: float = 12.0, per_call_cap_s: float | None = None) -> dict:
     """Time the oracle (write + decode) on whole requests of the same workload
     until about ``budget_s`` seconds of CPU work; report KV GB/s by the same
@@ -201,7 +236,7 @@ def cpu_baseline(budget_s: float = 12.0, per_call_cap_s: float | None = None) ->
     import workloads
     w = workloads.gqa_4k(poison=False, seed=2002, batch=4)
     lib = oracle.load()
-    threads = oracle.max_threads(lib)
+    threads = oracle_all_cores(lib)
     total_bytes = 0
     calls = 0
     reqs = 0
@@ -212,7 +247,8 @@ def cpu_baseline(budget_s: float = 12.0, per_call_cap_s: float | None = None) ->
         kc, vc = w.k_cache, w.v_cache
         t0 = time.perf_counter()
         oracle.kv_cache_write(w.k_new[sl], w.v_new[sl], w.slot_mapping[sl], kc, vc, lib=lib)
-        oracle.decode(w.q[sl], kc, vc, w.block_tables[sl], w.seq_lens[sl], w.scale, lib=lib)
+        oracle.decode(w.q[sl], kc, vc, w.block_tables[sl], w.seq_lens[sl], w.scale,
+                      nthreads=threads, lib=lib)
         t_all += time.perf_counter() - t0
         total_bytes += decode_bytes(1, 4096, 32, 8, 128)
         calls += 1
@@ -220,11 +256,15 @@ def cpu_baseline(budget_s: float = 12.0, per_call_cap_s: float | None = None) ->
         if per_call_cap_s is not None and t_all > per_call_cap_s:
             break
     gbs = total_bytes / t_all / 1e9
+    one = _oracle_rate(w, 1, 3.0, lib, per_head=True)
     return {"value": round(gbs, 4), "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"{reqs} whole requests of the 4k workload (4096 tokens x 32 q / 8 KV "
                       f"heads each), fp64 C oracle with OpenMP over (request, head), "
                       f"{t_all:.1f} s of CPU time",
-            "seconds": round(t_all, 3)}
+            "seconds": round(t_all, 3),
+            "single_thread": {"value": one["GBps"], "unit": UNIT, "cores": 1,
+                              "sample": f"{one['sample']} of the 4k workload (one kv head's "
+                                        f"4 query heads x 4096 tokens each)"}}
 
 
 def run_reference(args, rank: int, world: int):
@@ -235,7 +275,7 @@ def run_reference(args, rank: int, world: int):
     import workloads
     w = workloads.gqa_4k(poison=False, seed=2002, batch=4)
     lib = oracle.load()
-    threads = oracle.max_threads(lib)
+    threads = oracle_all_cores(lib)
     budget_total = 150.0
     per_step = max(budget_total / max(args.steps + args.warmup, 1), 0.0)
     # calibrate the sample: whole requests if affordable, else the first
@@ -355,11 +395,13 @@ def run_ours(args, rank: int, world: int, local: int):
     time.sleep(0.3)
     dist_barrier(world)
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("timed steps")
     bounds[0].record()
     for i in range(args.steps):
         step_graphs[i % N_LAYERS].replay()
         bounds[i + 1].record()
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
     dist_barrier(world)
     clocks = sampler.stop()
     ms_total = bounds[0].elapsed_time(bounds[-1])
@@ -368,15 +410,18 @@ def run_ours(args, rank: int, world: int, local: int):
     ms_step = ms_total_max / args.steps
 
     # --- the decode kernel alone, events around every launch (roofline) ---
-    n_dec = max(args.warmup, min(args.steps, 2000))
+    # a fixed number of launches, whatever --steps is
+    n_dec = ROOFLINE_LAUNCHES
     dev_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(n_dec)]
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("roofline: decode-only graph replays")
     for i in range(n_dec):
         dev_ev[i][0].record()
         dec_graphs[i % N_LAYERS].replay()
         dev_ev[i][1].record()
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
     decode_ms = [a.elapsed_time(b) for a, b in dev_ev]
     del step_graphs, dec_graphs
 
@@ -452,14 +497,49 @@ def run_ours(args, rank: int, world: int, local: int):
     dist_barrier(world)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push("e2e: graph per step")
     e0.record()
     for i in range(e2e_steps):
         e2e_step(i)
     e1.record()
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
     e2e_ms = dist_max(e0.elapsed_time(e1), world)
     e2e_value = dbytes * e2e_steps * world / (e2e_ms / 1e3) / 1e9
     assert pkv.get_device_error() == 0
+
+    # The same step with the three C-ABI calls issued eagerly every step: each
+    # call's host validation, planning, tensor-map encoding and launch is inside
+    # the timed region.  host_us_per_step is the host time of those calls.
+    def eager_step(li):
+        e2e_body(li)
+        torch.cuda.current_stream().synchronize()
+    for i in range(5):
+        eager_step(i)
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    host_s = 0.0
+    torch.cuda.nvtx.range_push("e2e: eager calls")
+    e0.record()
+    for i in range(e2e_steps):
+        h0 = time.perf_counter()
+        e2e_body(i)
+        host_s += time.perf_counter() - h0
+        torch.cuda.current_stream().synchronize()
+    e1.record()
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
+    eager_ms = dist_max(e0.elapsed_time(e1), world)
+    eager_value = dbytes * e2e_steps * world / (eager_ms / 1e3) / 1e9
+    assert pkv.get_device_error() == 0
+    del e2e_graphs
+
+    configs = None
+    if world == 1 and not args.no_configs:
+        layers.clear()  # free the four layer pools before the per-workload section
+        torch.cuda.empty_cache()
+        configs = run_configs(pkv, torch, dev, peak, peak_kind,
+                              with_oracle=not args.no_cpu_baseline)
 
     result = None
     if rank == 0:
@@ -480,6 +560,8 @@ def run_ours(args, rank: int, world: int, local: int):
             "tokens_per_s": round(B * world * args.steps / (ms_total_max / 1e3), 1),
             "context_tokens_per_s": round(B * L * world * args.steps / (ms_total_max / 1e3), 1),
             "fraction_of_hbm_peak": round(value / peak, 4),
+            "fraction_of_nominal_peak": round(value / NOMINAL_HBM_GBS, 4),
+            "nominal_peak_gbs": NOMINAL_HBM_GBS,
             "step_ms_median": round(statistics.median(step_ms), 5),
             "decode_ms_avg": round(dec_avg_ms, 5), "decode_ms_median": round(dec_med_ms, 5),
             "decode_launches_timed": n_dec,
@@ -498,8 +580,18 @@ def run_ours(args, rank: int, world: int, local: int):
                     "note": "pinned host inputs copied in and output copied out every step, "
                             "with a stream synchronize per step",
                     "mode": e2e_mode},
+            "e2e_eager": {"value": round(eager_value, 2), "unit": UNIT,
+                          "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                          "steps": e2e_steps, "ms_per_step": round(eager_ms / e2e_steps, 5),
+                          "host_us_per_step": round(host_s / e2e_steps * 1e6, 2),
+                          "note": "the same step with copy_blocks, kv_cache_write and the "
+                                  "decode called eagerly through the binding every step "
+                                  "(host validation, planning, tensor-map encoding and "
+                                  "launches inside the timed region); host_us_per_step = "
+                                  "host time of the copy-in, three calls and copy-out"},
             "gpu_launches": 2 * args.steps,
             "clocks": clocks,
+            "configs": configs,
         }
         print(json.dumps(result), flush=True)
     dist_barrier(world)
@@ -646,6 +738,213 @@ def run_suite(args):
         _suite_cache_ops(pkv, torch, workloads, dev, iters, flush, emit)
 
 
+# ---------------------------------------------------------------------------
+# per-workload section of the headline line: every workload of the scope
+# table, each timed on the GPU and with the oracle timed beside it
+# ---------------------------------------------------------------------------
+
+def _oracle_rate(w, nthreads: int, budget_s: float, lib, per_head: bool) -> dict:
+    """KV GB/s of the oracle on a bounded sample of workload ``w``: whole
+    requests (all heads; ``per_head`` False), or one kv head's query group of a
+    request at a time (``per_head`` True, for the single-thread figure), taken
+    in order until about ``budget_s`` seconds of oracle time.  Bytes are counted
+    by the same formula as the GPU (K+V once per kv head + q + out)."""
+    import oracle
+    G = w.Hq // w.Hkv
+    e_kv = w.elem_bytes
+    e_q = 4 if w.dtype == "f32" else 2
+    ks = None if w.k_scale is None else w.k_scale
+    vs = None if w.v_scale is None else w.v_scale
+    t_all, nbytes, units = 0.0, 0, 0
+    sliced = {}
+    order = [b for b in range(w.B) if int(w.seq_lens[b]) > 0]
+    heads = range(w.Hkv) if per_head else [None]
+    # in order, starting over while the budget lasts (a tiny workload is
+    # repeated until the sample is long enough to time)
+    order = [order[i % len(order)] for i in range(len(order) * 10_000)] if order else []
+    for b in order:
+        L = int(w.seq_lens[b])
+        for g in heads:
+            if g is None:
+                q, kc, vc, hk, kss, vss = w.q[b:b + 1], w.k_cache, w.v_cache, w.Hkv, ks, vs
+            else:
+                if g not in sliced:
+                    sliced[g] = (np.ascontiguousarray(w.k_cache[:, g:g + 1]),
+                                 np.ascontiguousarray(w.v_cache[:, g:g + 1]))
+                kc, vc = sliced[g]
+                q = np.ascontiguousarray(w.q[b:b + 1, g * G:(g + 1) * G])
+                hk = 1
+                kss = None if ks is None else ks[g:g + 1]
+                vss = None if vs is None else vs[g:g + 1]
+            t0 = time.perf_counter()
+            oracle.decode(q, kc, vc, w.block_tables[b:b + 1], w.seq_lens[b:b + 1], w.scale,
+                          k_scale=kss, v_scale=vss, nthreads=nthreads, lib=lib)
+            t_all += time.perf_counter() - t0
+            nbytes += 2 * L * hk * w.d * e_kv + q.shape[1] * w.d * (e_q + e_q)
+            units += 1
+            if t_all >= budget_s:
+                break
+        if t_all >= budget_s:
+            break
+    what = "kv-head groups" if per_head else "whole requests"
+    return {"GBps": round(nbytes / t_all / 1e9, 4), "threads": nthreads,
+            "sample": f"{units} {what}, {t_all:.2f} s"}
+
+
+def run_configs(pkv, torch, dev, peak, peak_kind, with_oracle=True, iters=200,
+                oracle_budget_s=0.8) -> list:
+    """One compact entry per workload: mean decode time over ``iters`` launches
+    (each after a 256 MB L2 flush, CUDA events around each), KV GB/s by the
+    decode byte model, the fraction of the HBM peak, and the oracle's KV GB/s on
+    a bounded sample of the same workload on all host cores and on one thread.
+    """
+    import oracle
+    import workloads
+    flush = _L2Flush(dev)
+    lib = oracle.load() if with_oracle else None
+    allc = oracle_all_cores(lib) if with_oracle else 0
+    entries = []
+
+    def oracle_pair(w):
+        if not with_oracle:
+            return None
+        return {"all_cores": _oracle_rate(w, allc, oracle_budget_s, lib, per_head=False),
+                "single_thread": _oracle_rate(w, 1, oracle_budget_s, lib, per_head=True)}
+
+    def nbytes_of(w):
+        e_q = 4 if w.dtype == "f32" else 2
+        return (2 * int(w.seq_lens.astype(np.int64).sum()) * w.Hkv * w.d * w.elem_bytes
+                + w.B * w.Hq * w.d * 2 * e_q)
+
+    def entry(name, w, ms, nbytes, extra=None, oracle_w=None):
+        mean, med = ms
+        gbs = nbytes / (mean / 1e3) / 1e9
+        e = {"workload": name, "us_mean": round(mean * 1e3, 2), "us_median": round(med * 1e3, 2),
+             "GBps": round(gbs, 1), "frac_of_peak": round(gbs / peak, 4), "bytes": int(nbytes),
+             "tokens_per_s": round(w.B / (mean / 1e3), 1)}
+        e.update(extra or {})
+        e["oracle"] = oracle_pair(oracle_w if oracle_w is not None else w)
+        entries.append(e)
+        print(json.dumps({"config_line": e}), file=sys.stderr, flush=True)
+
+    def decode_fn(t, w, out, ws, partition_size=0):
+        L = int(w.seq_lens.max())
+        return lambda: pkv.paged_attention_decode(
+            t["q"], t["kc"], t["vc"], t["bt"], t["sl"], w.bs, w.scale, out, max_seq_len=L,
+            workspace=ws, partition_size=partition_size, k_scale=t["ks"], v_scale=t["vs"])
+
+    def setup(w, partition_size=0):
+        t = _dev_workload(w, dev)
+        L = int(w.seq_lens.max())
+        odt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+        out = torch.empty((w.B, w.Hq, w.d), dtype=odt, device=dev)
+        ws = pkv.new_workspace(pkv.decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.d, w.bs, L,
+                                                          partition_size), dev)
+        return t, out, ws
+
+    def write_fn(t, w):
+        if w.dtype == "fp8":
+            return lambda: pkv.kv_cache_write_fp8(t["kn"], t["vn"], t["sm"], t["kc"], t["vc"],
+                                                  t["ks"], t["vs"])
+        return lambda: pkv.kv_cache_write(t["kn"], t["vn"], t["sm"], t["kc"], t["vc"])
+
+    torch.cuda.nvtx.range_push("per-workload section")
+    # config 1: tiny fp32 (latency-bound; correctness workload)
+    w = workloads.tiny_f32(poison=False)
+    t, out, ws = setup(w)
+    dec = decode_fn(t, w, out, ws)
+    wr = write_fn(t, w)
+    ms = _time_graph(lambda: (wr(), dec()), iters, flush)
+    entry("tiny_f32: 4 requests [1,17,100,200], 4 q / 2 KV heads, d 64, bs 16, fp32 "
+          "(append + decode)", w, ms, nbytes_of(w), {"kv_dtype": "f32"})
+    del t, out, ws
+
+    # config 2: the 4k batch, permuted pool and identity tables (indirection cost)
+    for name, perm in (("gqa_4k permuted pool", True), ("gqa_4k identity tables", False)):
+        w = workloads.make_paged([4096] * 16, Hq=32, Hkv=8, d=128, bs=16, dtype="bf16",
+                                 seed=1002, poison=False, permute=perm, name=name)
+        t, out, ws = setup(w)
+        ms = _time_graph(decode_fn(t, w, out, ws), iters, flush)
+        entry(f"{name}: 16 x 4096, 32 q / 8 KV heads, d 128, bs 16, bf16 (decode)", w, ms,
+              nbytes_of(w), {"kv_dtype": "bf16"})
+        del t, out, ws
+
+    # the same batch with an fp8 (e4m3) cache
+    w = workloads.gqa_4k_fp8(poison=False)
+    t, out, ws = setup(w)
+    ms = _time_graph(decode_fn(t, w, out, ws), iters, flush)
+    entry("gqa_4k_fp8: 16 x 4096, e4m3 cache with per-kv-head scales (decode; bytes of codes)",
+          w, ms, nbytes_of(w), {"kv_dtype": "fp8_e4m3"})
+    del t, out, ws
+
+    # config 3: mixed lengths, append + decode
+    w = workloads.mixed(poison=False)
+    t, out, ws = setup(w)
+    dec, wr = decode_fn(t, w, out, ws), write_fn(t, w)
+    ms_dec = _time_graph(dec, iters, flush)
+    ms_step = _time_graph(lambda: (wr(), dec()), iters, flush)
+    entry("mixed: 256 requests, log-uniform 16..8192 tokens (decode)", w, ms_dec, nbytes_of(w),
+          {"kv_dtype": "bf16", "step_us_mean": round(ms_step[0] * 1e3, 2),
+           "step": "kv_cache_write (256 tokens) + decode",
+           "context_tokens": int(w.seq_lens.astype(np.int64).sum())})
+    del t, out, ws, w
+    torch.cuda.empty_cache()
+
+    # config 4: shared prefix, per-request decode and prefix-aware decode
+    w = workloads.prefix_shared(poison=False)
+    t, out, ws = setup(w)
+    L = int(w.seq_lens.max())
+    plen = (w.info["prefix_tokens"] // w.bs) * w.bs
+    pfx_of = torch.zeros(w.B, dtype=torch.int32, device=dev)
+    pfx_len = torch.tensor([plen], dtype=torch.int32, device=dev)
+    ws_p = pkv.new_workspace(pkv.decode_prefix_workspace_bytes(
+        w.B, w.Hq, w.Hkv, w.d, w.bs, L, 1, w.B, w.info["prefix_tokens"]), dev)
+    dec = decode_fn(t, w, out, ws)
+
+    def dec_p():
+        pkv.paged_attention_decode_prefix(t["q"], t["kc"], t["vc"], t["bt"], t["sl"], pfx_of,
+                                          pfx_len, w.bs, w.scale, out, max_seq_len=L,
+                                          max_prefix_members=w.B,
+                                          max_prefix_len=w.info["prefix_tokens"], workspace=ws_p)
+
+    def fork_append():
+        pkv.copy_blocks(t["kc"], t["vc"], t["pairs"])
+        pkv.kv_cache_write(t["kn"], t["vn"], t["sm"], t["kc"], t["vc"])
+    logical = nbytes_of(w)
+    unique_tok = w.info["prefix_tokens"] + sum(w.info["suffix"])
+    unique = 2 * unique_tok * w.Hkv * w.d * 2 + w.B * w.Hq * w.d * 4
+    ms_a = _time_graph(dec, iters, flush)
+    ms_b = _time_graph(dec_p, iters, flush)
+    ms_sa = _time_graph(lambda: (fork_append(), dec()), iters, flush)
+    ms_sb = _time_graph(lambda: (fork_append(), dec_p()), iters, flush)
+    common = {"kv_dtype": "bf16", "bytes_kind": "logical (prefix counted once per request)",
+              "unique_bytes": unique}
+    entry("prefix: 64 requests sharing a 2040-token prefix, per-request decode", w, ms_a,
+          logical, dict(common, unique_GBps=round(unique / (ms_a[0] / 1e3) / 1e9, 1),
+                        step_us_mean=round(ms_sa[0] * 1e3, 2),
+                        step="copy_blocks (64 forks) + kv_cache_write (suffixes) + decode"))
+    entry("prefix: the same, prefix-aware decode (shared blocks read once per group)", w, ms_b,
+          logical, dict(common, unique_GBps=round(unique / (ms_b[0] / 1e3) / 1e9, 1),
+                        step_us_mean=round(ms_sb[0] * 1e3, 2),
+                        step="copy_blocks (64 forks) + kv_cache_write (suffixes) + "
+                             "paged_attention_decode_prefix"))
+    del t, out, ws, ws_p, w
+    torch.cuda.empty_cache()
+
+    # config 5: long context, block sizes 8 / 16 / 32, automatic split
+    for bs in (8, 16, 32):
+        w = workloads.long_ctx(bs=bs, poison=False)
+        t, out, ws = setup(w)
+        ms = _time_graph(decode_fn(t, w, out, ws), max(50, iters // 4), flush)
+        entry(f"long_ctx: 2 x 131072 tokens, 64 q / 8 KV heads, d 128, bs {bs}, automatic "
+              f"split (decode)", w, ms, nbytes_of(w), {"kv_dtype": "bf16", "block_size": bs})
+        del t, out, ws, w
+        torch.cuda.empty_cache()
+    torch.cuda.nvtx.range_pop()
+    assert pkv.get_device_error() == 0
+    return entries
+
+
 def _suite_prefix(pkv, torch, workloads, dev, iters, flush, emit):
 
     # shared prefix: the step (fork copy + suffix append + decode)
@@ -754,12 +1053,18 @@ def main():
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-workload section (every workload of the scope table, "
+                         "each with the oracle timed beside it)")
     ap.add_argument("--clocks-csv", default="",
                     help="where to keep the raw nvidia-smi samples of the timed region "
                          "(default: a temporary file; the JSON line carries the summary)")
     ap.add_argument("--no-check", action="store_true",
                     help="accepted for older command lines; parity is checked by the tests, "
                          "not by the bench")
+    ap.add_argument("--plumbing-only", action="store_true",
+                    help="set up the ranks, pass the barriers and the max-over-ranks "
+                         "exchange, print n_gpus, and stop (no GPU work; runs on CPU)")
     ap.add_argument("--suite", action="store_true",
                     help="one line per workload of the scope table instead of the headline")
     ap.add_argument("--case", default="",
@@ -777,7 +1082,22 @@ def main():
     if args.suite:
         run_suite(args)
         return
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(relaunch_under_torchrun(args.gpus, sys.argv[1:]))
     rank, world, local = dist_setup(args.gpus)
+    if args.plumbing_only:
+        # the rank set-up, barriers and max-over-ranks exchange alone (no GPU
+        # work): what the multi-rank launch does before and after timing
+        try:
+            dist_barrier(world)
+            top = dist_max(float(rank), world)
+            if rank == 0:
+                print(json.dumps({"plumbing_only": True, "n_gpus": world, "max_rank": top}),
+                      flush=True)
+            dist_barrier(world)
+        finally:
+            dist_done(world)
+        return
     try:
         run_ours(args, rank, world, local)
     finally:
