@@ -57,9 +57,10 @@ constexpr int cmin(int a, int b) { return a < b ? a : b; }
 constexpr int cmax(int a, int b) { return a > b ? a : b; }
 
 // F8 = false: bf16 cache, tiles land swizzled and feed bf16 MMAs directly.
-// F8 = true : fp8 (e4m3) cache, tiles land as plain rows of head_dim bytes and
-//             the consumer widens them (exactly) to f16 in a swizzled staging
-//             tile before f16 MMAs; q is widened to f16 likewise.
+// F8 = true : fp8 (e4m3) cache, tiles land as rows of head_dim one-byte codes
+//             (TMA boxes with the swizzle of their width) and every consumer
+//             widens what it loads from them to f16 in registers (exact), for
+//             f16 MMAs; q is widened to f16 likewise.
 template <int D, int NT, bool F8>
 struct MmaCfg {
     static constexpr int NHALF = D / 64;            // 128-byte column halves of a 16-bit row
@@ -67,29 +68,34 @@ struct MmaCfg {
     static constexpr int HALF_BYTES = kCH * 128;    // one swizzled half region (16-bit data)
     static constexpr int KV_BYTES = F8 ? kCH * D : NHALF * HALF_BYTES;  // K (or V) of a stage
     static constexpr int GP = 8 * NT;               // query heads per head group (padded)
-    static constexpr int Q_BYTES = GP * D * 2;      // the group's q rows (first stages of a segment)
-    // K | V | q, rounded to the 1 KB the 128-byte swizzle pattern repeats on
-    static constexpr int STAGE_BYTES = (2 * KV_BYTES + Q_BYTES + 1023) / 1024 * 1024;
-    // bf16: one tensor-core consumer reads the TMA stages directly (two CTAs
-    // per SM).  fp8: NCONS consumers own one f16 staging slot each and take
-    // the CTA's chunks in turn (chunk n -> consumer n % NCONS), and NCV
-    // converter warps widen every fp8 stage into the slot of the consumer that
-    // takes it (one CTA per SM).  Each barrier then has one waiter stepping
-    // through its phases in order.
-    static constexpr int NCONS = F8 ? (NT == 1 ? 3 : 2) : 1;
-    static constexpr int NCV = F8 ? 4 : 0;
+    static constexpr int Q_BYTES = GP * D * 2;      // the group's q rows (first stage of a segment)
+    // bf16: K | V | q, rounded to the 1 KB the 128-byte swizzle pattern repeats
+    // on.  fp8: K | V only (8 or 4 KB each, whole swizzle periods); each
+    // consumer reads the group's q from global memory.
+    static constexpr int STAGE_BYTES = F8 ? 2 * KV_BYTES : (2 * KV_BYTES + Q_BYTES + 1023) / 1024 * 1024;
+    // bf16: one tensor-core consumer reads the TMA stages (two CTAs per SM).
+    // fp8: one CTA per SM whose NCONS consumers take the CTA's chunks in turn
+    // (chunk n -> consumer n % NCONS, stage n % NSTAGE; NSTAGE is a multiple of
+    // NCONS, so a stage always serves the same consumer and each barrier has
+    // one waiter stepping through its phases in order).  Widening codes costs
+    // instructions the bf16 path does not have; four consumers put one on
+    // every SM sub-partition.
+    static constexpr int NCONS = F8 ? 4 : 1;
     // producer warps: a TMA issue holds the issuing warp ~0.1 us, and one fp8
     // producer per SM cannot issue fast enough; two take alternate chunks
-    // (stage n % NSTAGE belongs to producer n % NPROD).  The 16-head fp8
-    // config keeps one (its consumers need all the registers).
-    static constexpr int NPROD = (F8 && NT == 1) ? 2 : 1;
-    static constexpr int THREADS = 32 * (NPROD + NCONS + NCV + 1);  // + the epilogue
-    static constexpr int QCH = NCONS;  // a segment's first QCH chunks carry the group's q
-    static constexpr int SLOT_BYTES = F8 ? (2 * NHALF * HALF_BYTES + Q_BYTES + 1023) / 1024 * 1024 : 0;
-    static constexpr int STG_BYTES = NCONS * SLOT_BYTES;   // f16 K | V | q per consumer
-    // fp8 (one CTA per SM): six stages keep ~100 KB of codes in flight per SM
-    static constexpr int NSTAGE = F8 ? 6 : cmax(2, cmin(8, kRingBudget / STAGE_BYTES));
-    static_assert(NSTAGE % NPROD == 0, "each stage belongs to one producer");
+    // (stage n % NSTAGE belongs to producer n % NPROD).
+    static constexpr int NPROD = F8 ? 2 : 1;
+    static constexpr int THREADS = 32 * (NPROD + NCONS + 1);  // + the epilogue
+    // consumer -> epilogue hand-off: per lane, the accumulators and (m, l)
+    static constexpr int DUMP_BYTES = (KS * NT * 4 + NT * 4) * 32 * 4;
+    // fp8: as many stages as the shared memory holds beside the hand-off
+    // slots (up to 24), a multiple of NCONS and NPROD: ~190 KB of codes in
+    // flight per SM, as much as the two bf16 CTAs of an SM keep
+    static constexpr int F8_RING = 227 * 1024 - NCONS * DUMP_BYTES - 4096;
+    static constexpr int NSTAGE = F8 ? cmin(24, F8_RING / STAGE_BYTES) / 4 * 4
+                                     : cmax(2, cmin(8, kRingBudget / STAGE_BYTES));
+    static_assert(NSTAGE % NPROD == 0 && NSTAGE % NCONS == 0 && NSTAGE >= 2,
+                  "each stage belongs to one producer and one consumer");
 };
 
 // ---- shared-memory layout ------------------------------------------------------
@@ -102,17 +108,39 @@ struct Smem {
     static constexpr int NSLOT = C::NCONS * NDUMP;
     static constexpr int DUMP_ACC = C::KS * NT * 4;       // acc registers per lane
     static constexpr int DUMP_ML = NT * 4;                // m[2], l[2] per n-tile per lane
-    static constexpr int DUMP_BYTES = (DUMP_ACC + DUMP_ML) * 32 * 4;
-    static constexpr int OFF_STG = C::NSTAGE * C::STAGE_BYTES;
-    static constexpr int OFF_DUMP = OFF_STG + C::STG_BYTES;
+    static constexpr int DUMP_BYTES = C::DUMP_BYTES;
+    static constexpr int OFF_DUMP = C::NSTAGE * C::STAGE_BYTES;
     static constexpr int OFF_BAR = OFF_DUMP + NSLOT * DUMP_BYTES;
-    // full/empty per stage, dfull/dempty per dump slot, sfull/sempty per staging slot
-    static constexpr int OFF_META = OFF_BAR + (2 * C::NSTAGE + 2 * NSLOT + 2 * C::NCONS) * 8;
-    // ntok/bad per stage, then per staging slot
-    static constexpr int OFF_CTRL = OFF_META + 2 * (C::NSTAGE + C::NCONS) * 4;
+    // full/empty per stage, dfull/dempty per dump slot
+    static constexpr int OFF_META = OFF_BAR + (2 * C::NSTAGE + 2 * NSLOT) * 8;
+    // ntok/bad per stage
+    static constexpr int OFF_CTRL = OFF_META + 2 * C::NSTAGE * 4;
     static constexpr int BYTES = OFF_CTRL + 16 + 1024;   // + alignment slack
     static_assert(BYTES <= 227 * 1024, "within the opt-in shared memory of one CTA");
 };
+
+// Head-dim index of accumulator element (dt, lane group grp, upper half hi) of
+// P.V.  bf16: the natural m16n8 rows, 16 dt + grp + 8 hi.  fp8: the consumer
+// loads V with ldmatrix on byte pairs, so lane group grp of m-tile dt holds
+// dims 16 dt + 4 (grp / 2) + grp % 2 (+ 2 for the upper half).
+template <bool F8>
+__device__ __forceinline__ int dcol(int dt, int grp, int hi) {
+    if constexpr (F8)
+        return dt * 16 + 4 * (grp >> 1) + (grp & 1) + 2 * hi;
+    else
+        return dt * 16 + grp + 8 * hi;
+}
+
+// fp8 stage rows are D bytes landed by TMA with the swizzle of their width:
+// 16-byte chunk c of row r sits at chunk c ^ f8_swz(r) (128-byte rows: r mod 8;
+// 64-byte rows: (r / 2) mod 4).  Stage regions start on the pattern's period.
+template <int D>
+__device__ __forceinline__ int f8_swz(int row) {
+    if constexpr (D == 128)
+        return row & 7;
+    else
+        return (row >> 1) & 3;
+}
 
 // ---- producer ------------------------------------------------------------------
 
@@ -244,7 +272,7 @@ struct Producer {
                         }
                     }
                 }
-                if (c - sg.c0 < C::QCH) {
+                if (c == sg.c0) {
                     const unsigned char* gq = reinterpret_cast<const unsigned char*>(
                         static_cast<const __nv_bfloat16*>(p.q) +
                         ((size_t)cur.b * p.num_q_heads + hq0) * D);
@@ -261,10 +289,10 @@ struct Producer {
                 st_ntok[stage] = ntok;
                 st_bad[stage] = bad;
                 if (bad) raise_error(p.err, PKV_DEVERR_BAD_BLOCK);
-                const uint32_t qbytes = c - sg.c0 < C::QCH ? (uint32_t)gv * D * 2u : 0u;
+                const uint32_t qbytes = (!F8 && c == sg.c0) ? (uint32_t)gv * D * 2u : 0u;
                 const uint32_t row_bytes = F8 ? (uint32_t)D : (uint32_t)C::NHALF * 128u;
                 mbar_arrive_expect_tx(&full[stage], nvalid * 2u * rb * row_bytes + qbytes);
-                if (qbytes)  // the group's q rows ride with the segment's first stage(s)
+                if (qbytes)  // the group's q rows ride with the segment's first stage
                     bulk_load(sq, static_cast<const __nv_bfloat16*>(p.q) +
                                       ((size_t)cur.b * p.num_q_heads + hq0) * D,
                               qbytes, &full[stage], policy);
@@ -282,13 +310,11 @@ struct Producer {
                     const int boff = t0 - (j << p.log2_bs) > 0 ? t0 - (j << p.log2_bs) : 0;
                     const int grow = (phys * p.num_kv_heads + kvh) * p.block_size + boff;
                     if constexpr (F8) {
-                        // a block's code rows of one kv head are one contiguous run:
-                        // plain bulk copies (no tensor map, rows land unswizzled)
-                        const size_t goff = (size_t)grow * D;
-                        bulk_load(sk + srow * D, static_cast<const uint8_t*>(p.k_cache) + goff,
-                                  (uint32_t)(rb * D), &full[stage], policy);
-                        bulk_load(sv + srow * D, static_cast<const uint8_t*>(p.v_cache) + goff,
-                                  (uint32_t)(rb * D), &full[stage], policy);
+                        // whole code rows (D bytes) with the swizzle of their
+                        // width, so the consumers' ldmatrix reads are free of
+                        // bank conflicts
+                        tma_load_2d(sk + srow * D, tmk, 0, grow, &full[stage], policy);
+                        tma_load_2d(sv + srow * D, tmv, 0, grow, &full[stage], policy);
                     } else {
 #pragma unroll
                         for (int h = 0; h < C::NHALF; ++h) {
@@ -362,17 +388,24 @@ __device__ __forceinline__ SegInfo seg_info(const DecodeParams& p, const Segment
 
 // ---- consumer (tensor-core math) ----------------------------------------------
 
-// Consumer `me` (0 .. NCONS-1).  bf16: reads every TMA stage in turn.  fp8:
-// takes the CTA's chunks n with n % NCONS == me from its own f16 staging slot
-// (sfull/sempty), where the converter warps put K, V and, for a segment's
-// first chunks, q.
+// Consumer `me` (0 .. NCONS-1).  bf16: reads every TMA stage in turn, K and V
+// as 16-bit swizzled tiles, the group's q from the segment's first stage.
+// fp8: takes the CTA's chunks n with n % NCONS == me (stage n % NSTAGE) and
+// widens the e4m3 codes in registers: ldmatrix on byte pairs gives lane
+// (grp, tig) four consecutive codes of one token row, which one cvt per pair
+// turns into two f16x2 words.
+//   q.K^T: the four codes 4 tig .. 4 tig + 3 of a 16-code block serve as the A
+//     fragment's k = 2 tig, 2 tig + 1 and 2 tig + 8, 2 tig + 9, a fixed
+//     permutation of the head dim inside each block; q is loaded with the same
+//     permutation (dims 4 tig .. 4 tig + 3), so the dot products are unchanged.
+//   P.V: the widened words are 8 x 8 tiles with tokens as rows; movmatrix.trans
+//     makes them A fragments of V^T with tokens as k, and the head-dim rows
+//     come out permuted as dcol<true> describes.
 template <int D, int NT, bool F8>
 __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                                         unsigned char* smem, uint64_t* full, uint64_t* empty,
-                                        uint64_t* dfull, uint64_t* dempty, uint64_t* sfull,
-                                        uint64_t* sempty, const int* st_ntok,
-                                        const unsigned* st_bad, const int* sl_ntok,
-                                        const unsigned* sl_bad, volatile int* ctrl, int lane,
+                                        uint64_t* dfull, uint64_t* dempty, const int* st_ntok,
+                                        const unsigned* st_bad, volatile int* ctrl, int lane,
                                         int me) {
     using C = MmaCfg<D, NT, F8>;
     using S = Smem<D, NT, F8>;
@@ -380,11 +413,11 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
     const int grp = lane >> 2, tig = lane & 3;
     const int mi = lane >> 3, r8 = lane & 7;
     // ldmatrix row/chunk components that depend only on the lane
-    const int k_row = r8 + 8 * (mi & 1), k_cx = mi >> 1;  // K (A operand)
-    const int v_row = r8 + 8 * (mi >> 1), v_cx = mi & 1;  // V^T (A operand, transposed load)
+    const int k_row = r8 + 8 * (mi & 1), k_cx = mi >> 1;  // K (A operand); fp8: K and V
+    const int v_row = r8 + 8 * (mi >> 1), v_cx = mi & 1;  // bf16 V^T (transposed load)
     Ring ring, dring;
-    uint32_t sphase = 0;   // fp8: phase of this consumer's staging slot
     unsigned n_chunk = 0;  // fp8: chunks of the CTA so far
+    bool waited = false;   // fp8: q is read from global memory
 
     while (it.valid) {
         const Segment sg = it.current();
@@ -406,58 +439,73 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
         }
 
         bool have_q = false;
-        for (int c = sg.c0; c < sg.c1; ++c) {
-            int ntok;
-            unsigned bad;
-            unsigned char* sk;
-            if constexpr (F8) {
-                const bool mine = (int)(n_chunk % C::NCONS) == me;
-                ++n_chunk;
-                if (!mine) continue;
-                if (ctrl[0] || !mbar_wait(&sfull[me], sphase, p.wait_ns)) {
-                    if (lane == 0 && !ctrl[0]) {
-                        ctrl[0] = 1;
-                        raise_error(p.err, PKV_DEVERR_TIMEOUT);
-                    }
-                    return;
+        if constexpr (F8) {
+            // Q^T B-fragments in the permuted order: head nt*8+grp, dims
+            // 16 ks + 4 tig, +1 (b0) and 16 ks + 4 tig + 2, +3 (b1), bf16 -> f16.
+            // Only a consumer with a chunk of this segment needs them.
+            bool any = false;
+            for (unsigned n = n_chunk; n < n_chunk + (unsigned)(sg.c1 - sg.c0); ++n)
+                any |= (int)(n % C::NCONS) == me;
+            if (any) {
+                if (!waited) {
+                    griddep_wait();  // q may come from the previous kernel
+                    waited = true;
                 }
-                ntok = sl_ntok[me];
-                bad = sl_bad[me];
-                sk = smem + S::OFF_STG + me * C::SLOT_BYTES;
-            } else {
-                if (ctrl[0] || !mbar_wait(&full[ring.stage], ring.phase, p.wait_ns)) {
-                    if (lane == 0 && !ctrl[0]) {
-                        ctrl[0] = 1;
-                        raise_error(p.err, PKV_DEVERR_TIMEOUT);
-                    }
-                    return;
-                }
-                ntok = st_ntok[ring.stage];
-                bad = st_bad[ring.stage];
-                sk = smem + ring.stage * C::STAGE_BYTES;
-            }
-            const bool whole = ntok == kCH && bad == 0;
-            // 16-bit K | V | q (a bf16 stage, or an fp8 chunk's f16 staging slot)
-            unsigned char* sv = sk + C::NHALF * C::HALF_BYTES;
-
-            if (!have_q) {
-                // This consumer's first chunk of the segment carries the group's q.
-                // Q^T B-fragments: head nt*8+grp, dims ks*16 + 2*tig (+1) and +8 (+9).
-                have_q = true;
-                const uint32_t* sq = reinterpret_cast<const uint32_t*>(sv + C::NHALF * C::HALF_BYTES);
+                const __nv_bfloat16* gq =
+                    static_cast<const __nv_bfloat16*>(p.q) + ((size_t)si.b * p.num_q_heads + si.hq0) * D;
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     const int h = nt * 8 + grp;
 #pragma unroll
                     for (int ks = 0; ks < C::KS; ++ks) {
-                        uint32_t w0 = h < si.gv ? sq[h * (D / 2) + ks * 8 + tig] : 0u;
-                        uint32_t w1 = h < si.gv ? sq[h * (D / 2) + ks * 8 + 4 + tig] : 0u;
-                        if constexpr (F8) {
-                            w0 = bf16x2_to_f16x2(w0);
-                            w1 = bf16x2_to_f16x2(w1);
-                        }
-                        qb[nt][ks][0] = w0;
-                        qb[nt][ks][1] = w1;
+                        uint2 w = make_uint2(0u, 0u);
+                        if (h < si.gv)
+                            w = __ldg(reinterpret_cast<const uint2*>(gq + (size_t)h * D + ks * 16 + 4 * tig));
+                        qb[nt][ks][0] = bf16x2_to_f16x2(w.x);
+                        qb[nt][ks][1] = bf16x2_to_f16x2(w.y);
+                    }
+                }
+                have_q = true;
+            }
+        }
+
+        for (int c = sg.c0; c < sg.c1; ++c) {
+            int stage;
+            uint32_t phase;
+            if constexpr (F8) {
+                const unsigned n = n_chunk++;
+                if ((int)(n % C::NCONS) != me) continue;
+                stage = (int)(n % C::NSTAGE);
+                phase = (n / C::NSTAGE) & 1u;
+            } else {
+                stage = ring.stage;
+                phase = ring.phase;
+            }
+            if (ctrl[0] || !mbar_wait(&full[stage], phase, p.wait_ns)) {
+                if (lane == 0 && !ctrl[0]) {
+                    ctrl[0] = 1;
+                    raise_error(p.err, PKV_DEVERR_TIMEOUT);
+                }
+                return;
+            }
+            const int ntok = st_ntok[stage];
+            const unsigned bad = st_bad[stage];
+            unsigned char* sk = smem + stage * C::STAGE_BYTES;
+            unsigned char* sv = sk + C::KV_BYTES;
+            const bool whole = ntok == kCH && bad == 0;
+
+            if (!F8 && !have_q) {
+                // The segment's first chunk carries the group's q.
+                // Q^T B-fragments: head nt*8+grp, dims ks*16 + 2*tig (+1) and +8 (+9).
+                have_q = true;
+                const uint32_t* sq = reinterpret_cast<const uint32_t*>(sv + C::KV_BYTES);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    const int h = nt * 8 + grp;
+#pragma unroll
+                    for (int ks = 0; ks < C::KS; ++ks) {
+                        qb[nt][ks][0] = h < si.gv ? sq[h * (D / 2) + ks * 8 + tig] : 0u;
+                        qb[nt][ks][1] = h < si.gv ? sq[h * (D / 2) + ks * 8 + 4 + tig] : 0u;
                     }
                 }
             }
@@ -488,16 +536,39 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                     for (int i = 0; i < 4; ++i) s[mt][nt][i] = 0.f;
+            if constexpr (F8) {
+                // one ldmatrix.x4 = 16 token rows x 32 codes = two k-steps
 #pragma unroll
-            for (int ks = 0; ks < C::KS; ++ks) {
-                const int half = ks >> 2;
-                const int chunk = (2 * (ks & 3) + k_cx) ^ r8;
+                for (int j = 0; j < C::KS / 2; ++j) {
 #pragma unroll
-                for (int mt = 0; mt < kMT; ++mt) {
-                    uint32_t a[4];
-                    ldsm_x4(skb + half * C::HALF_BYTES + (mt * 16 + k_row) * 128 + (chunk << 4), a);
+                    for (int mt = 0; mt < kMT; ++mt) {
+                        const int row = mt * 16 + k_row;
+                        uint32_t r[4];
+                        ldsm_x4(skb + row * D + (((2 * j + k_cx) ^ f8_swz<D>(row)) << 4), r);
+                        uint32_t a[2][4];
+                        e4m3x4_to_f16(r[0], a[0][0], a[0][2]);
+                        e4m3x4_to_f16(r[1], a[0][1], a[0][3]);
+                        e4m3x4_to_f16(r[2], a[1][0], a[1][2]);
+                        e4m3x4_to_f16(r[3], a[1][1], a[1][3]);
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) mma16<F8>(s[mt][nt], a, qb[nt][ks][0], qb[nt][ks][1]);
+                        for (int h = 0; h < 2; ++h)
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt)
+                                mma_f16(s[mt][nt], a[h], qb[nt][2 * j + h][0], qb[nt][2 * j + h][1]);
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int ks = 0; ks < C::KS; ++ks) {
+                    const int half = ks >> 2;
+                    const int chunk = (2 * (ks & 3) + k_cx) ^ r8;
+#pragma unroll
+                    for (int mt = 0; mt < kMT; ++mt) {
+                        uint32_t a[4];
+                        ldsm_x4(skb + half * C::HALF_BYTES + (mt * 16 + k_row) * 128 + (chunk << 4), a);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) mma_bf16(s[mt][nt], a, qb[nt][ks][0], qb[nt][ks][1]);
+                    }
                 }
             }
 
@@ -563,7 +634,7 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                     }
             }
 
-            // ---- O^T += V^T . P^T, P split into bf16 hi + lo ----
+            // ---- O^T += V^T . P^T, P split into 16-bit hi + lo ----
 #pragma unroll
             for (int mt = 0; mt < kMT; ++mt) {
                 uint32_t bh[NT][2], bl[NT][2];
@@ -583,29 +654,59 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                         }
                     }
                 }
+                if constexpr (F8) {
+                    // this lane's token rows of the tile: grp (ldmatrix matrices
+                    // 0, 2) and grp + 8 (matrices 1, 3); a row that does not take
+                    // part is zeroed in registers (0-weight x NaN stays out)
+                    bool ok_lo = true, ok_hi = true;
+                    if (!whole) {
+                        const int r0 = mt * 16 + grp, r1 = r0 + 8;
+                        const int j0 = ((c * kCH + r0) >> p.log2_bs) - ((c * kCH) >> p.log2_bs);
+                        const int j1 = ((c * kCH + r1) >> p.log2_bs) - ((c * kCH) >> p.log2_bs);
+                        ok_lo = r0 < ntok && !((bad >> j0) & 1u);
+                        ok_hi = r1 < ntok && !((bad >> j1) & 1u);
+                    }
 #pragma unroll
-                for (int dt = 0; dt < C::KS; ++dt) {
-                    const int half = dt >> 2;
-                    const int chunk = (2 * (dt & 3) + v_cx) ^ r8;
-                    uint32_t a[4];
-                    ldsm_x4_t(svb + half * C::HALF_BYTES + (mt * 16 + v_row) * 128 + (chunk << 4), a);
+                    for (int j = 0; j < C::KS / 2; ++j) {
+                        const int row = mt * 16 + k_row;
+                        uint32_t r[4];
+                        ldsm_x4(svb + row * D + (((2 * j + k_cx) ^ f8_swz<D>(row)) << 4), r);
+                        if (!ok_lo) r[0] = r[2] = 0u;
+                        if (!ok_hi) r[1] = r[3] = 0u;
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        mma16<F8>(acc[dt][nt], a, bh[nt][0], bh[nt][1]);
-                        mma16<F8>(acc[dt][nt], a, bl[nt][0], bl[nt][1]);
+                        for (int h = 0; h < 2; ++h) {
+                            // m-tile dt = 2j + h: rows 0-7 the low code pairs, 8-15 the high
+                            uint32_t xl, xh, yl, yh;
+                            e4m3x4_to_f16(r[2 * h], xl, xh);      // tokens 0-7 of the tile
+                            e4m3x4_to_f16(r[2 * h + 1], yl, yh);  // tokens 8-15
+                            const uint32_t a[4] = {movmatrix_t(xl), movmatrix_t(xh), movmatrix_t(yl),
+                                                   movmatrix_t(yh)};
+#pragma unroll
+                            for (int nt = 0; nt < NT; ++nt) {
+                                mma_f16(acc[2 * j + h][nt], a, bh[nt][0], bh[nt][1]);
+                                mma_f16(acc[2 * j + h][nt], a, bl[nt][0], bl[nt][1]);
+                            }
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int dt = 0; dt < C::KS; ++dt) {
+                        const int half = dt >> 2;
+                        const int chunk = (2 * (dt & 3) + v_cx) ^ r8;
+                        uint32_t a[4];
+                        ldsm_x4_t(svb + half * C::HALF_BYTES + (mt * 16 + v_row) * 128 + (chunk << 4), a);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            mma_bf16(acc[dt][nt], a, bh[nt][0], bh[nt][1]);
+                            mma_bf16(acc[dt][nt], a, bl[nt][0], bl[nt][1]);
+                        }
                     }
                 }
             }
-            if constexpr (!F8) {
-                if (!whole) fence_proxy_async_smem();  // our zero-fill before the next TMA write
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[ring.stage]);
-                ring.advance(C::NSTAGE);
-            } else {
-                __syncwarp();  // slot reads done before the converters refill it
-                if (lane == 0) mbar_arrive(&sempty[me]);
-                sphase ^= 1u;
-            }
+            if (!F8 && !whole) fence_proxy_async_smem();  // our zero-fill before the next TMA write
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+            if constexpr (!F8) ring.advance(C::NSTAGE);
         }
 
         // ---- hand the segment's state to the epilogue warp ----
@@ -639,120 +740,6 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
     }
 }
 
-// ---- converters (fp8 caches) ----------------------------------------------------
-
-// Row and 16-code group of item `rest` (0 .. RPW*C16-1) of converter v.  With
-// 8 groups per row (two 64-column halves of f16) a quarter-warp takes two
-// adjacent rows and complementary halves: its 16-byte code loads cover eight
-// distinct bank groups, and so do its swizzled f16 stores (the rows' XOR keys
-// differ in the low bit).  One row per quarter-warp would store both halves
-// to the same four bank groups.
-template <int C16, int RPW>
-__device__ __forceinline__ void code_group(int rest, int v, int& row, int& c16) {
-    if constexpr (C16 == 8) {
-        const int rs = (rest >> 2) & 1;
-        row = v * RPW + (rest >> 4) * 2 + rs;
-        c16 = (rest & 3) + 4 * (rs ^ ((rest >> 3) & 1));
-    } else {
-        row = v * RPW + rest / C16;
-        c16 = rest % C16;
-    }
-}
-
-// Converter v (0 .. NCV-1) widens rows v*16 .. v*16+15 of every fp8 stage's K
-// and V (exactly, e4m3 -> f16) into the swizzled staging slot of the consumer
-// that takes the chunk; tokens that do not take part (past the end, or in a
-// block the table got wrong) become zero rows.  Converter 0 also copies the
-// group's q rows and the chunk's token count / bad-block mask into the slot.
-template <int D, int NT>
-__device__ __forceinline__ void convert(const DecodeParams& p, SegIter<kCH>& it,
-                                        unsigned char* smem, uint64_t* full, uint64_t* empty,
-                                        uint64_t* sfull, uint64_t* sempty, const int* st_ntok,
-                                        const unsigned* st_bad, int* sl_ntok, unsigned* sl_bad,
-                                        volatile int* ctrl, int lane, int v) {
-    using C = MmaCfg<D, NT, true>;
-    using S = Smem<D, NT, true>;
-    constexpr int RPW = kCH / C::NCV;              // rows of K (and of V) per converter
-    constexpr int C16 = D / 16;                    // 16-code groups per row
-    constexpr int PER_LANE = 2 * RPW * C16 / 32;
-    static_assert(2 * RPW * C16 % 32 == 0, "whole lanes");
-    Ring ring;
-    unsigned n_chunk = 0;
-    while (it.valid) {
-        const Segment sg = it.current();
-        it.advance(p, lane);
-        for (int c = sg.c0; c < sg.c1; ++c, ++n_chunk) {
-            const int slot = (int)(n_chunk % C::NCONS);
-            const uint32_t sph = (n_chunk / C::NCONS) & 1u;
-            if (ctrl[0] || !mbar_wait(&full[ring.stage], ring.phase, p.wait_ns) ||
-                !mbar_wait(&sempty[slot], sph ^ 1u, p.wait_ns)) {
-                if (lane == 0 && !ctrl[0]) {
-                    ctrl[0] = 1;
-                    raise_error(p.err, PKV_DEVERR_TIMEOUT);
-                }
-                return;
-            }
-            const int ntok = st_ntok[ring.stage];
-            const unsigned bad = st_bad[ring.stage];
-            const bool whole = ntok == kCH && bad == 0;
-            const unsigned char* sk = smem + ring.stage * C::STAGE_BYTES;  // e4m3 rows of D bytes
-            const unsigned char* sv = sk + C::KV_BYTES;
-            unsigned char* dst0 = smem + S::OFF_STG + slot * C::SLOT_BYTES;
-            // all of this lane's code groups in flight first, then widen them
-            uint4 raw[PER_LANE];
-#pragma unroll
-            for (int i = 0; i < PER_LANE; ++i) {
-                const int idx = lane + 32 * i;
-                const int part = idx / (RPW * C16);
-                int row, c16;
-                code_group<C16, RPW>(idx % (RPW * C16), v, row, c16);
-                raw[i] = *reinterpret_cast<const uint4*>((part ? sv : sk) + row * D + c16 * 16);
-            }
-#pragma unroll
-            for (int i = 0; i < PER_LANE; ++i) {
-                const int idx = lane + 32 * i;
-                const int part = idx / (RPW * C16);
-                int row, c16;
-                code_group<C16, RPW>(idx % (RPW * C16), v, row, c16);
-                bool valid = whole;
-                if (!whole) {
-                    const int jrel = ((c * kCH + row) >> p.log2_bs) - ((c * kCH) >> p.log2_bs);
-                    valid = row < ntok && !((bad >> jrel) & 1u);
-                }
-                uint4 o0 = make_uint4(0, 0, 0, 0), o1 = make_uint4(0, 0, 0, 0);
-                if (valid) {
-                    e4m3x4_to_f16(raw[i].x, o0.x, o0.y);
-                    e4m3x4_to_f16(raw[i].y, o0.z, o0.w);
-                    e4m3x4_to_f16(raw[i].z, o1.x, o1.y);
-                    e4m3x4_to_f16(raw[i].w, o1.z, o1.w);
-                }
-                const int half = (c16 * 16) >> 6, cc = ((c16 * 16) & 63) >> 3;
-                unsigned char* dst = dst0 + part * C::NHALF * C::HALF_BYTES +
-                                     half * C::HALF_BYTES + row * 128;
-                *reinterpret_cast<uint4*>(dst + ((cc ^ (row & 7)) << 4)) = o0;
-                *reinterpret_cast<uint4*>(dst + (((cc + 1) ^ (row & 7)) << 4)) = o1;
-            }
-            if (v == 0) {
-                if (c - sg.c0 < C::QCH) {
-                    const uint4* qs = reinterpret_cast<const uint4*>(sv + C::KV_BYTES);
-                    uint4* qd = reinterpret_cast<uint4*>(dst0 + 2 * C::NHALF * C::HALF_BYTES);
-                    for (int i = lane; i < C::Q_BYTES / 16; i += 32) qd[i] = qs[i];
-                }
-                if (lane == 0) {
-                    sl_ntok[slot] = ntok;
-                    sl_bad[slot] = bad;
-                }
-            }
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&empty[ring.stage]);
-                mbar_arrive(&sfull[slot]);
-            }
-            ring.advance(C::NSTAGE);
-        }
-    }
-}
-
 // ---- shared-prefix results ------------------------------------------------------
 
 // Tokens of request b's prefix group that the shared pass covered (0: none).
@@ -765,7 +752,7 @@ __device__ __forceinline__ int prefix_tokens_of(const DecodeParams& p, int b) {
 }
 
 // A part's partial result (unnormalised acc, max m, sum l) as record `rec`.
-template <int D, int NT>
+template <int D, int NT, bool F8>
 __device__ __forceinline__ void write_record(const DecodeParams& p, size_t rec, int tig, int grp,
                                              const float (&acc)[D / 16][NT][4],
                                              const float (&m)[NT][2], const float (&l)[NT][2]) {
@@ -778,8 +765,8 @@ __device__ __forceinline__ void write_record(const DecodeParams& p, size_t rec, 
             float* ra = p.rec_acc + (rec * GP + h) * D;
 #pragma unroll
             for (int dt = 0; dt < D / 16; ++dt) {
-                ra[dt * 16 + grp] = acc[dt][nt][j];
-                ra[dt * 16 + grp + 8] = acc[dt][nt][j + 2];
+                ra[dcol<F8>(dt, grp, 0)] = acc[dt][nt][j];
+                ra[dcol<F8>(dt, grp, 1)] = acc[dt][nt][j + 2];
             }
             if (grp == 0) {
                 p.rec_ml[(rec * GP + h) * 2] = m[nt][j];
@@ -893,7 +880,7 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
                 p.meta[2 * si.bg + 1] = fits ? si.nseg : 0;
                 if (!fits) raise_error(p.err, PKV_DEVERR_BAD_SEQ_LEN);
             }
-            if (fits) write_record<D, NT>(p, si.bg + si.u, tig, grp, acc, m, l);
+            if (fits) write_record<D, NT, F8>(p, si.bg + si.u, tig, grp, acc, m, l);
             continue;
         }
         if (si.nseg == 1) {
@@ -907,8 +894,9 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
                     const size_t orow = ((size_t)si.b * p.num_q_heads + si.hq0 + h) * D;
 #pragma unroll
                     for (int dt = 0; dt < C::KS; ++dt) {
-                        store_out(p.out, orow + dt * 16 + grp, acc[dt][nt][j] * inv, p.out_dtype);
-                        store_out(p.out, orow + dt * 16 + grp + 8, acc[dt][nt][j + 2] * inv,
+                        store_out(p.out, orow + dcol<F8>(dt, grp, 0), acc[dt][nt][j] * inv,
+                                  p.out_dtype);
+                        store_out(p.out, orow + dcol<F8>(dt, grp, 1), acc[dt][nt][j + 2] * inv,
                                   p.out_dtype);
                     }
                 }
@@ -926,7 +914,7 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
         arrived = __shfl_sync(FULL_MASK, arrived, 0);
         const size_t rec = si.bg + si.u;
         if (arrived != (unsigned)(si.nseg - 1)) {
-            write_record<D, NT>(p, rec, tig, grp, acc, m, l);
+            write_record<D, NT, F8>(p, rec, tig, grp, acc, m, l);
             __threadfence();
             __syncwarp();
             if (lane == 0) atomicExch(p.ready + rec, 1u);
@@ -989,8 +977,8 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
                         const float* ra = p.rec_acc + rr * D;
 #pragma unroll
                         for (int dt = 0; dt < C::KS; ++dt) {
-                            ar[k][dt][nt][j] = ld_cg(ra + dt * 16 + grp);
-                            ar[k][dt][nt][j + 2] = ld_cg(ra + dt * 16 + grp + 8);
+                            ar[k][dt][nt][j] = ld_cg(ra + dcol<F8>(dt, grp, 0));
+                            ar[k][dt][nt][j + 2] = ld_cg(ra + dcol<F8>(dt, grp, 1));
                         }
                     }
             }
@@ -1024,8 +1012,9 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
                 const size_t orow = ((size_t)si.b * p.num_q_heads + si.hq0 + h) * D;
 #pragma unroll
                 for (int dt = 0; dt < C::KS; ++dt) {
-                    store_out(p.out, orow + dt * 16 + grp, A[dt][nt][j] * inv, p.out_dtype);
-                    store_out(p.out, orow + dt * 16 + grp + 8, A[dt][nt][j + 2] * inv, p.out_dtype);
+                    store_out(p.out, orow + dcol<F8>(dt, grp, 0), A[dt][nt][j] * inv, p.out_dtype);
+                    store_out(p.out, orow + dcol<F8>(dt, grp, 1), A[dt][nt][j + 2] * inv,
+                              p.out_dtype);
                 }
             }
         __syncwarp();
@@ -1070,12 +1059,8 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
     uint64_t* empty = full + C::NSTAGE;
     uint64_t* dfull = empty + C::NSTAGE;
     uint64_t* dempty = dfull + S::NSLOT;
-    uint64_t* sfull = dempty + S::NSLOT;  // fp8 staging slots
-    uint64_t* sempty = sfull + C::NCONS;
     int* st_ntok = reinterpret_cast<int*>(smem + S::OFF_META);
     unsigned* st_bad = reinterpret_cast<unsigned*>(st_ntok + C::NSTAGE);
-    int* sl_ntok = reinterpret_cast<int*>(st_bad + C::NSTAGE);
-    unsigned* sl_bad = reinterpret_cast<unsigned*>(sl_ntok + C::NCONS);
     volatile int* ctrl = reinterpret_cast<volatile int*>(smem + S::OFF_CTRL);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -1084,15 +1069,11 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
         for (int s = 0; s < C::NSTAGE; ++s) {
             // row copies: every producer lane arrives once its copies have landed
             mbar_init(&full[s], RC ? 32 : 1);
-            mbar_init(&empty[s], F8 ? C::NCV : 1);  // released by the converters (fp8)
+            mbar_init(&empty[s], 1);  // released by the stage's one consumer
         }
         for (int s = 0; s < S::NSLOT; ++s) {
             mbar_init(&dfull[s], 1);
             mbar_init(&dempty[s], 1);
-        }
-        for (int s = 0; s < C::NCONS; ++s) {
-            mbar_init(&sfull[s], C::NCV);
-            mbar_init(&sempty[s], 1);
         }
         fence_mbar_init();
         prefetch_tensormap(&tmk);
@@ -1121,7 +1102,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
     SegIter<kCH> it;
     it.init(p, total, W, lane, L_first, T_first);
 
-    // warps: producers | consumers | epilogue | converters (fp8)
+    // warps: producers | consumers | epilogue
     if (warp < C::NPROD) {
         Producer<D, NT, F8, RC> pr{p, &tmk, &tmv, smem, full, empty, st_ntok, st_bad, ctrl, lane,
                            l2_policy_evict_first()};
@@ -1129,14 +1110,10 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
         pr.run(it);
         if (!pr.waited) griddep_wait();
     } else if (warp < C::NPROD + C::NCONS) {
-        consume<D, NT, F8>(p, it, smem, full, empty, dfull, dempty, sfull, sempty, st_ntok, st_bad,
-                           sl_ntok, sl_bad, ctrl, lane, warp - C::NPROD);
-    } else if (warp == C::NPROD + C::NCONS) {
-        epilogue<D, NT, F8>(p, it, smem, dfull, dempty, ctrl, lane);
+        consume<D, NT, F8>(p, it, smem, full, empty, dfull, dempty, st_ntok, st_bad, ctrl, lane,
+                           warp - C::NPROD);
     } else {
-        if constexpr (C::NCV > 0)
-            convert<D, NT>(p, it, smem, full, empty, sfull, sempty, st_ntok, st_bad, sl_ntok,
-                           sl_bad, ctrl, lane, warp - C::NPROD - C::NCONS - 1);
+        epilogue<D, NT, F8>(p, it, smem, dfull, dempty, ctrl, lane);
     }
 }
 

@@ -1,30 +1,37 @@
-// decode_prefix.cu -- the shared pass of prefix-aware paged decode.
+// decode_prefix.cu -- the shared pass of prefix-aware paged decode, on the
+// 5th-generation tensor cores (tcgen05, accumulators in tensor memory).
 //
 // Requests forked from one prompt share the physical blocks of its prefix
 // ("KV Cache Management", "The Bonus: Zero-Copy Sharing"; "KV Cache
 // Optimization and PagedAttention", intro: shared blocks are computed and
 // stored once).  Decoding them one request at a time still reads those blocks
-// once per request.  This pass reads each prefix tile once per 64 (member,
+// once per request.  This pass reads each prefix tile once per 128 (member,
 // query head) rows instead, which turns the group's decode over the prefix
 // into a dense contraction with the rows as the MMA M dimension:
-//   S[64 x 64]  = Q[64 x d] . K_chunk^T       (q rows of 16 members x 4 heads)
-//   O[64 x d]  += P[64 x 64] . V_chunk
-// Each consumer warp owns 16 rows and runs the FlashAttention-2 register
-// layout (Q as A fragments in registers, K via ldmatrix as the B operand, the
-// S accumulator re-packed in registers as the A operand of P.V, V via
-// ldmatrix.trans), online softmax in base 2 with P split into bf16 hi + lo.
+//   S[128 x 64] = Q[128 x d] . K_chunk^T     (tcgen05.mma, both operands K-major)
+//   O[128 x d] += P[128 x 64] . V_chunk      (P K-major, V MN-major)
+// S (two buffers) and O live in tensor memory: 64 + 64 + d columns of fp32
+// over 128 lanes, one lane per row.  One thread of the MMA warp issues the
+// MMAs; four softmax warps (one per 32-lane quarter of tensor memory, one row
+// per thread) read S with tcgen05.ld, mask it, run the online softmax in base
+// 2 and write P, split into bf16 hi + lo, to shared memory in the 128-byte
+// swizzled K-major layout the P.V MMA reads.  The running maximum is raised
+// lazily: O (in tensor memory) is rescaled only when a row's maximum grows by
+// more than 8 (a factor 256), so the weights stay below 2^8 and the result is
+// exact whatever maximum is used, as long as O and the row sum l use the same.
 //
-// The pass leaves, per (split, request, query head), the partial state
-// (max m in log2 units, sum l, unnormalised acc) of the attention over that
-// split's prefix tokens; the per-request decode pass starts after the prefix
-// and merges these states into its own:
+// The pass leaves, per (split, request, query head), the partial state (max m
+// in log2 units, sum l, unnormalised acc) of the attention over that split's
+// prefix tokens; the per-request decode pass starts after the prefix and
+// merges these states into its own:
 //   out = (A + sum_s 2^(m_s - M) acc_s) / (S + sum_s 2^(m_s - M) l_s).
-// A member shorter than the prefix has its rows masked past its own length.
+// A member shorter than the prefix has its row masked past its own length.
 //
-// Data movement as in the per-request decode kernel: one producer warp reads
-// the block table of the group's longest member and issues TMA tensor copies
+// Data movement as in the per-request decode kernel: a producer warp reads the
+// block table of the group's longest member and issues TMA tensor copies
 // (128-byte swizzle, no multicast) of each block's K and V rows of one kv head
-// into a 3-stage ring; the four consumer warps all read every stage.
+// into a 3-stage ring; the stage is released by the MMA completion of the
+// P.V product that reads it (tcgen05.commit on the stage's empty barrier).
 #include <cuda.h>
 
 #include <algorithm>
@@ -32,39 +39,53 @@
 
 #include "decode_common.cuh"
 #include "mma_ptx.cuh"
+#include "umma_ptx.cuh"
 
 namespace pkv {
 namespace {
 
-constexpr int kCW = 4;                     // consumer warps, 16 rows each
-constexpr int kThreadsP = 32 * (1 + kCW);  // + the producer warp
 constexpr int kStagesP = 3;
-static_assert(kCW * 16 == kPrefixRows, "one row tile per CTA");
+constexpr int kSoftWarps = 4;                       // one row per thread
+constexpr int kThreadsP = 32 * (2 + kSoftWarps);    // producer, MMA, softmax
+constexpr int kTmemCols = 256;                      // S x2 (64 each) + O (<= 128)
+constexpr int kSCol = 0, kOCol = 128;               // tensor-memory columns
+static_assert(kSoftWarps * 32 == kPrefixRows, "one tile row per softmax thread");
 
 template <int D>
 struct PCfg {
     static constexpr int NHALF = D / 64;               // 128-byte halves of a bf16 row
     static constexpr int KS = D / 16;                  // k-steps of Q.K^T
-    static constexpr int DT = D / 8;                   // 8-wide output tiles
-    static constexpr int HALF_BYTES = kPrefixCH * 128;
+    static constexpr int HALF_BYTES = kPrefixCH * 128; // one 64-column half of a K or V tile
     static constexpr int KV_BYTES = NHALF * HALF_BYTES;
     static constexpr int STAGE_BYTES = 2 * KV_BYTES;   // K | V, whole KB
-    static constexpr int OFF_BAR = kStagesP * STAGE_BYTES;
-    static constexpr int OFF_META = OFF_BAR + 2 * kStagesP * 8;
+    static constexpr int QHALF = kPrefixRows * 128;    // one 64-column half of the Q tile
+    static constexpr int P_BYTES = kPrefixRows * 128;  // 128 rows x 64 tokens of bf16
+    static constexpr int OFF_Q = kStagesP * STAGE_BYTES;
+    static constexpr int OFF_P = OFF_Q + NHALF * QHALF;  // [2 buffers][hi, lo]
+    static constexpr int OFF_BAR = OFF_P + 4 * P_BYTES;
+    // full, empty per stage; s_full, s_free, p_full, pv_done per buffer; q_ready; drain
+    static constexpr int NBAR = 2 * kStagesP + 4 * 2 + 2;
+    static constexpr int OFF_META = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ROWS = OFF_META + 2 * kStagesP * 4;
     static constexpr int OFF_CTRL = OFF_ROWS + 3 * kPrefixRows * 4;
     static constexpr int BYTES = OFF_CTRL + 32 + 1024;  // + alignment slack
+    static_assert(BYTES <= 227 * 1024, "within the opt-in shared memory of one CTA");
 };
 
-// smem address of the 16-byte chunk holding (row, col) of a swizzled tile
-// region (rows of 128 bytes per 64-column half; chunk index XOR row % 8)
-__device__ __forceinline__ uint32_t swz(uint32_t base, int row, int col, int half_bytes) {
-    const int half = col >> 6, cc = (col & 63) >> 3;
-    return base + half * half_bytes + row * 128 + ((cc ^ (row & 7)) << 4);
-}
+// Instruction descriptors: S = Q.K^T (M 128, N 64, B K-major) and
+// O += P.V (M 128, N d, B MN-major).
+template <int D>
+struct PIdesc {
+    static constexpr uint32_t S = idesc_bf16_f32(kPrefixRows, kPrefixCH, false);
+    static constexpr uint32_t PV = idesc_bf16_f32(kPrefixRows, D, true);
+};
+
+// Byte offset of the 16-byte chunk `c` (8 bf16) of row `r` in a 128-byte
+// swizzled region (chunk index XOR row % 8).
+__device__ __forceinline__ uint32_t sw128(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
 
 template <int D>
-__global__ void __launch_bounds__(kThreadsP, 2)
+__global__ void __launch_bounds__(kThreadsP, 1)
     prefix_kernel(const __grid_constant__ PrefixParams p, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv) {
     using C = PCfg<D>;
@@ -72,12 +93,19 @@ __global__ void __launch_bounds__(kThreadsP, 2)
     unsigned char* smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* empty = full + kStagesP;
+    uint64_t* s_full = empty + kStagesP;  // S buffer b holds a chunk's scores
+    uint64_t* s_free = s_full + 2;        // the softmax warps have read S buffer b
+    uint64_t* p_full = s_free + 2;        // P buffer b (and any O rescale) is ready
+    uint64_t* pv_done = p_full + 2;       // the P.V MMAs reading P buffer b completed
+    uint64_t* q_ready = pv_done + 2;      // the Q tile is in shared memory
+    uint64_t* drain = q_ready + 1;        // every MMA this CTA issued has completed
     int* st_ntok = reinterpret_cast<int*>(smem + C::OFF_META);
     unsigned* st_bad = reinterpret_cast<unsigned*>(st_ntok + kStagesP);
     int* row_b = reinterpret_cast<int*>(smem + C::OFF_ROWS);
     int* row_h = row_b + kPrefixRows;
     int* row_L = row_h + kPrefixRows;
     volatile int* ctrl = reinterpret_cast<volatile int*>(smem + C::OFF_CTRL);
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_CTRL + 16);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     int x = blockIdx.x;
@@ -107,11 +135,23 @@ __global__ void __launch_bounds__(kThreadsP, 2)
         ctrl[0] = 0;
         for (int s = 0; s < kStagesP; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], kCW);
+            mbar_init(&empty[s], 1);  // the MMA completion of the chunk's P.V
         }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&s_full[b], 1);
+            mbar_init(&s_free[b], kSoftWarps);
+            mbar_init(&p_full[b], kSoftWarps * 32);
+            mbar_init(&pv_done[b], 1);
+        }
+        mbar_init(q_ready, kSoftWarps * 32);
+        mbar_init(drain, 1);
         fence_mbar_init();
         prefetch_tensormap(&tmk);
         prefetch_tensormap(&tmv);
+    }
+    if (warp == 1) {  // this warp owns the tensor memory: allocates and frees it
+        tmem_alloc(tmem_slot, kTmemCols);
+        tmem_relinquish();
     }
     // Members of group g in request order; rank r holds rows r*G .. r*G+G-1.
     // The table source is the longest member (the first of equal ones).
@@ -163,15 +203,15 @@ __global__ void __launch_bounds__(kThreadsP, 2)
             if (leader && count > p.max_members) raise_error(p.err, PKV_DEVERR_PREFIX);
         }
     }
+    tc_fence_before();
     __syncthreads();
+    tc_fence_after();
     griddep_launch_dependents();
-    if (!ctrl[3]) {
-        griddep_wait();
-        return;
-    }
+    const uint32_t tmem = *tmem_slot;
     const int b_src = ctrl[1];
     const int tl = ctrl[2];
-    const int c_end = min(c1, chunks_of<kPrefixCH>(tl));
+    const int c_end = ctrl[3] ? min(c1, chunks_of<kPrefixCH>(tl)) : c0;
+    const int n_local = max(c_end - c0, 0);  // chunks this CTA streams
 
     if (warp == 0) {
         // ---- producer ----
@@ -267,203 +307,252 @@ __global__ void __launch_bounds__(kThreadsP, 2)
         return;
     }
 
-    // ---- consumers: warp w owns rows 16w .. 16w+15 of the tile ----
-    const int w = warp - 1;
-    const int grp = lane >> 2, tig = lane & 3;
-    const int rA = w * 16 + grp, rB = rA + 8;
-    const int bA = row_b[rA], bB = row_b[rB];
-    const int hA = row_h[rA], hB = row_h[rB];
-    const int LA = row_L[rA], LB = row_L[rB];
-    griddep_wait();  // q may come from the previous kernel
-
-    // Q as A fragments: a0 = (row grp, k 2tig..+1), a1 = (row grp+8, ...),
-    // a2 = (row grp, k 8+2tig..), a3 = (row grp+8, k 8+2tig..) per 16-wide k-step
-    uint32_t qa[C::KS][4];
-    {
-        const uint32_t* qA = reinterpret_cast<const uint32_t*>(
-            static_cast<const __nv_bfloat16*>(p.q) + ((size_t)max(bA, 0) * p.num_q_heads + hA) * D);
-        const uint32_t* qB = reinterpret_cast<const uint32_t*>(
-            static_cast<const __nv_bfloat16*>(p.q) + ((size_t)max(bB, 0) * p.num_q_heads + hB) * D);
+    if (warp == 1) {
+        // ---- MMA issue (one thread) ----
+        if (lane == 0 && n_local > 0) {
+            const uint32_t qb = smem_addr(smem + C::OFF_Q);
+            const uint32_t pb = smem_addr(smem + C::OFF_P);
+            const uint32_t sb = smem_addr(smem);
+            bool ok = mbar_wait(q_ready, 0);
+            tc_fence_after();
+            // S_i = Q . K_i^T into S buffer i % 2, once that buffer was read
+            auto issue_s = [&](int i) -> bool {
+                const int st = i % kStagesP, b = i & 1;
+                if (!mbar_wait(&full[st], (i / kStagesP) & 1u) ||
+                    !mbar_wait(&s_free[b], ((i >> 1) & 1u) ^ 1u))
+                    return false;
+                tc_fence_after();
+                const uint32_t kb = sb + st * C::STAGE_BYTES;
 #pragma unroll
-        for (int ks = 0; ks < C::KS; ++ks) {
-            qa[ks][0] = bA >= 0 ? __ldg(qA + ks * 8 + tig) : 0u;
-            qa[ks][1] = bB >= 0 ? __ldg(qB + ks * 8 + tig) : 0u;
-            qa[ks][2] = bA >= 0 ? __ldg(qA + ks * 8 + 4 + tig) : 0u;
-            qa[ks][3] = bB >= 0 ? __ldg(qB + ks * 8 + 4 + tig) : 0u;
+                for (int ks = 0; ks < C::KS; ++ks) {
+                    const uint32_t off = (ks & 3) * 32;  // k-step inside the 128-byte atom
+                    const uint64_t a = smem_desc_sw128(qb + (ks >> 2) * C::QHALF + off, 16, 1024);
+                    const uint64_t bd = smem_desc_sw128(kb + (ks >> 2) * C::HALF_BYTES + off, 16, 1024);
+                    umma_bf16(tmem + kSCol + b * kPrefixCH, a, bd, PIdesc<D>::S, ks > 0 ? 1u : 0u);
+                }
+                umma_commit(&s_full[b]);
+                return true;
+            };
+            if (ok) ok = issue_s(0);
+            for (int i = 0; i < n_local && ok; ++i) {
+                const int st = i % kStagesP, b = i & 1;
+                if (i + 1 < n_local && !issue_s(i + 1)) {  // overlaps the softmax of chunk i
+                    ok = false;
+                    break;
+                }
+                if (ctrl[0] || !mbar_wait(&p_full[b], (i >> 1) & 1u)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t vb = sb + st * C::STAGE_BYTES + C::KV_BYTES;
+#pragma unroll
+                for (int part = 0; part < 2; ++part) {  // P hi, then P lo
+                    const uint32_t pa = pb + (2 * b + part) * C::P_BYTES;
+#pragma unroll
+                    for (int kt = 0; kt < kPrefixCH / 16; ++kt) {
+                        const uint64_t a = smem_desc_sw128(pa + kt * 32, 16, 1024);
+                        const uint64_t bd = smem_desc_sw128(vb + kt * 16 * 128, C::HALF_BYTES, 1024);
+                        const uint32_t acc = (i == 0 && part == 0 && kt == 0) ? 0u : 1u;
+                        umma_bf16(tmem + kOCol, a, bd, PIdesc<D>::PV, acc);
+                    }
+                }
+                umma_commit(&empty[st]);   // the K/V stage may be refilled
+                umma_commit(&pv_done[b]);  // P buffer b may be rewritten; O is current
+            }
+            if (!ok) {
+                if (!ctrl[0]) raise_error(p.err, PKV_DEVERR_TIMEOUT);
+                ctrl[0] = 1;
+            }
+            // nothing may still write tensor memory when it is freed: a commit
+            // tracks every MMA issued before it (bounded wait)
+            umma_commit(drain);
+            mbar_wait(drain, 0u);
         }
-    }
-    float o[C::DT][4];
+        __syncwarp();
+    } else {
+        // ---- softmax warps: thread t of warp w owns tile row 32 (w % 4) + t ----
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const uint32_t trow = tmem + ((uint32_t)(quarter * 32) << 16);  // this warp's lanes
+        const int b_r = row_b[r], h_r = row_h[r], L_r = row_L[r];
+        griddep_wait();  // q may come from the previous kernel
+        {
+            // the row's q, bf16, into the swizzled K-major Q tile
+            unsigned char* qs = smem + C::OFF_Q;
+            const uint4* gq = reinterpret_cast<const uint4*>(
+                static_cast<const __nv_bfloat16*>(p.q) + ((size_t)max(b_r, 0) * p.num_q_heads + h_r) * D);
 #pragma unroll
-    for (int dt = 0; dt < C::DT; ++dt)
+            for (int c = 0; c < D / 8; ++c) {
+                const uint4 v = b_r >= 0 ? __ldg(gq + c) : make_uint4(0, 0, 0, 0);
+                *reinterpret_cast<uint4*>(qs + (c >> 3) * C::QHALF + sw128(r, c & 7)) = v;
+            }
+            fence_proxy_async_smem();  // generic writes -> the tensor cores' reads
+            mbar_arrive(q_ready);
+        }
+        const float sl2 = p.scale_log2;
+        float m_used = -INFINITY, l = 0.f;
+        for (int i = 0; i < n_local; ++i) {
+            const int st = i % kStagesP, b = i & 1, c = c0 + i;
+            // the stage's token count (written before its copies), then the
+            // scores.  Every decision before a tcgen05.ld/st is taken by the
+            // whole warp (those instructions need all 32 lanes).
+            bool ok = !ctrl[0] && mbar_wait(&full[st], (i / kStagesP) & 1u) &&
+                      mbar_wait(&s_full[b], (i >> 1) & 1u);
+            if (!__all_sync(FULL_MASK, ok)) {
+                if (lane == 0 && !ctrl[0]) {
+                    ctrl[0] = 1;
+                    raise_error(p.err, PKV_DEVERR_TIMEOUT);
+                }
+                break;
+            }
+            tc_fence_after();
+            float s[kPrefixCH];
+            {
+                uint32_t u[32];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) o[dt][i] = 0.f;
-    float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
-    const float sl2 = p.scale_log2;
-    // lane-dependent parts of the ldmatrix row addresses
-    const int kq = lane >> 3, kr = lane & 7;
+                for (int half = 0; half < 2; ++half) {
+                    tmem_ld32(trow + kSCol + b * kPrefixCH + half * 32, u);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) s[half * 32 + j] = __uint_as_float(u[j]);
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_free[b]);
 
-    Ring ring;
-    for (int c = c0; c < c_end; ++c) {
-        if (ctrl[0] || !mbar_wait(&full[ring.stage], ring.phase)) {
-            if (lane == 0 && !ctrl[0]) {
+            const int ntok = st_ntok[st];
+            const unsigned bad = st_bad[st];
+            const bool whole = ntok == kPrefixCH && bad == 0;
+            const int tbase = c * kPrefixCH;
+            float mx = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < kPrefixCH; ++j) {
+                bool ok = tbase + j < L_r;
+                if (!whole) {
+                    const int jrel = ((tbase + j) >> p.log2_bs) - (tbase >> p.log2_bs);
+                    ok = ok && j < ntok && !((bad >> jrel) & 1u);
+                }
+                s[j] = ok ? s[j] * sl2 : -INFINITY;
+                mx = fmaxf(mx, s[j]);
+            }
+            // lazy maximum: raise it (and rescale O, l) only past a factor 2^8
+            const bool raise = mx > m_used + 8.f;
+            const float m_new = raise ? mx : m_used;
+            if (__any_sync(FULL_MASK, raise) && i > 0) {
+                const float alpha = raise ? exp2f(m_used - m_new) : 1.f;  // 0 from -inf
+                // O must hold the previous chunk's P.V before it is rescaled
+                if (!__all_sync(FULL_MASK, mbar_wait(&pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1u))) {
+                    if (lane == 0 && !ctrl[0]) {
+                        ctrl[0] = 1;
+                        raise_error(p.err, PKV_DEVERR_TIMEOUT);
+                    }
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll 1
+                for (int q = 0; q < D / 32; ++q) {
+                    uint32_t u[32];
+                    tmem_ld32(trow + kOCol + q * 32, u);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) u[j] = __float_as_uint(__uint_as_float(u[j]) * alpha);
+                    tmem_st32(trow + kOCol + q * 32, u);
+                }
+                tmem_wait_st();
+                l *= alpha;
+            }
+            m_used = m_new;
+            const float ref = m_used == -INFINITY ? 0.f : m_used;
+            // P buffer b was last read by the P.V MMAs of chunk i - 2
+            if (!__all_sync(FULL_MASK, mbar_wait(&pv_done[b], ((i >> 1) & 1u) ^ 1u))) {
+                if (lane == 0 && !ctrl[0]) {
+                    ctrl[0] = 1;
+                    raise_error(p.err, PKV_DEVERR_TIMEOUT);
+                }
+                break;
+            }
+            unsigned char* ph = smem + C::OFF_P + (2 * b) * C::P_BYTES;
+            unsigned char* pl = ph + C::P_BYTES;
+#pragma unroll
+            for (int c8 = 0; c8 < kPrefixCH / 8; ++c8) {
+                uint32_t wh[4], wl[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float p0 = exp2f(s[c8 * 8 + 2 * e] - ref);
+                    const float p1 = exp2f(s[c8 * 8 + 2 * e + 1] - ref);
+                    l += p0 + p1;
+                    const float h0 = bf16_round(p0), h1 = bf16_round(p1);
+                    wh[e] = pack_bf16(h0, h1);
+                    wl[e] = pack_bf16(p0 - h0, p1 - h1);
+                }
+                *reinterpret_cast<uint4*>(ph + sw128(r, c8)) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+                *reinterpret_cast<uint4*>(pl + sw128(r, c8)) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+            }
+            if (!whole) {
+                // V rows of tokens that do not take part (past the chunk's end or
+                // in a bad block) hold stale or poisoned data: zero them so that
+                // 0-weight x NaN cannot reach O
+                unsigned char* sv = smem + st * C::STAGE_BYTES + C::KV_BYTES;
+                for (int idx = r; idx < kPrefixCH * C::NHALF * 8; idx += kPrefixRows) {
+                    const int row = idx / (C::NHALF * 8), rest = idx % (C::NHALF * 8);
+                    const int jrel = ((tbase + row) >> p.log2_bs) - (tbase >> p.log2_bs);
+                    if (row >= ntok || ((bad >> jrel) & 1u))
+                        *reinterpret_cast<uint4*>(sv + (rest >> 3) * C::HALF_BYTES + row * 128 +
+                                                  (rest & 7) * 16) = make_uint4(0, 0, 0, 0);
+                }
+            }
+            fence_proxy_async_smem();  // P (and zeroed V rows) -> the tensor cores' reads
+            tc_fence_before();
+            mbar_arrive(&p_full[b]);
+        }
+        // the partial state of this split for row r (an empty state when the
+        // split holds no token that any member attends to)
+        if (n_local == 0 && b_r >= 0) {
+            const size_t row = ((size_t)sp * p.num_seqs + b_r) * p.num_q_heads + h_r;
+            float4* ra = reinterpret_cast<float4*>(p.pfx_acc + row * D);
+            for (int j = 0; j < D / 4; ++j) ra[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+            p.pfx_ml[row * 2] = -INFINITY;
+            p.pfx_ml[row * 2 + 1] = 0.f;
+        }
+        if (__all_sync(FULL_MASK, n_local > 0 && !ctrl[0])) {
+            const int last = n_local - 1;
+            if (__all_sync(FULL_MASK, mbar_wait(&pv_done[last & 1], (last >> 1) & 1u))) {
+                tc_fence_after();
+                float* ra = b_r >= 0 ? p.pfx_acc + (((size_t)sp * p.num_seqs + b_r) * p.num_q_heads + h_r) * D
+                                     : nullptr;
+#pragma unroll 1
+                for (int q = 0; q < D / 32; ++q) {
+                    uint32_t u[32];
+                    tmem_ld32(trow + kOCol + q * 32, u);
+                    tmem_wait_ld();
+                    if (ra) {
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4)
+                            *reinterpret_cast<float4*>(ra + q * 32 + j) =
+                                make_float4(__uint_as_float(u[j]), __uint_as_float(u[j + 1]),
+                                            __uint_as_float(u[j + 2]), __uint_as_float(u[j + 3]));
+                    }
+                }
+                if (ra) {
+                    const size_t row = ((size_t)sp * p.num_seqs + b_r) * p.num_q_heads + h_r;
+                    p.pfx_ml[row * 2] = m_used;
+                    p.pfx_ml[row * 2 + 1] = l;
+                }
+            } else if (lane == 0 && !ctrl[0]) {
                 ctrl[0] = 1;
                 raise_error(p.err, PKV_DEVERR_TIMEOUT);
             }
-            return;
         }
-        const int ntok = st_ntok[ring.stage];
-        const unsigned bad = st_bad[ring.stage];
-        const bool whole = ntok == kPrefixCH && bad == 0;
-        const uint32_t skb = smem_addr(smem + ring.stage * C::STAGE_BYTES);
-        const uint32_t svb = skb + C::KV_BYTES;
-        const int tbase = c * kPrefixCH;
-
-        // Two halves of 32 tokens, each a full online-softmax step: fewer
-        // live score registers keep two CTAs per SM within the register file.
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-            // S = Q . K^T over 4 token tiles of 8; K rows (tokens) as the B operand
-            float sc[4][4];
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                const int trow = (hf * 4 + nt) * 8;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) sc[nt][i] = 0.f;
-#pragma unroll
-                for (int k2 = 0; k2 < C::KS / 2; ++k2) {
-                    uint32_t r[4];
-                    ldsm_x4(swz(skb, trow + kr, k2 * 32 + kq * 8, C::HALF_BYTES), r);
-                    mma_bf16(sc[nt], qa[2 * k2], r[0], r[1]);
-                    mma_bf16(sc[nt], qa[2 * k2 + 1], r[2], r[3]);
-                }
-            }
-            // mask (chunk tail, bad blocks, each row's own length), scale to
-            // log2 units, running max per row (the 4 lanes of a quad share a row)
-            float mxA = -INFINITY, mxB = -INFINITY;
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int tok = (hf * 4 + nt) * 8 + 2 * tig + (e & 1);
-                    bool ok = whole;
-                    if (!whole) {
-                        const int jrel = ((tbase + tok) >> p.log2_bs) - (tbase >> p.log2_bs);
-                        ok = tok < ntok && !((bad >> jrel) & 1u);
-                    }
-                    ok = ok && tbase + tok < (e < 2 ? LA : LB);
-                    const float v = ok ? sc[nt][e] * sl2 : -INFINITY;
-                    sc[nt][e] = v;
-                    if (e < 2)
-                        mxA = fmaxf(mxA, v);
-                    else
-                        mxB = fmaxf(mxB, v);
-                }
-            mxA = fmaxf(mxA, __shfl_xor_sync(FULL_MASK, mxA, 1));
-            mxA = fmaxf(mxA, __shfl_xor_sync(FULL_MASK, mxA, 2));
-            mxB = fmaxf(mxB, __shfl_xor_sync(FULL_MASK, mxB, 1));
-            mxB = fmaxf(mxB, __shfl_xor_sync(FULL_MASK, mxB, 2));
-            const float nA = fmaxf(mA, mxA), nB = fmaxf(mB, mxB);
-            const float refA = nA == -INFINITY ? 0.f : nA, refB = nB == -INFINITY ? 0.f : nB;
-            const float alA = exp2f(mA - refA), alB = exp2f(mB - refB);
-            mA = nA;
-            mB = nB;
-            lA *= alA;
-            lB *= alB;
-#pragma unroll
-            for (int dt = 0; dt < C::DT; ++dt) {
-                o[dt][0] *= alA;
-                o[dt][1] *= alA;
-                o[dt][2] *= alB;
-                o[dt][3] *= alB;
-            }
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                sc[nt][0] = exp2f(sc[nt][0] - refA);
-                sc[nt][1] = exp2f(sc[nt][1] - refA);
-                sc[nt][2] = exp2f(sc[nt][2] - refB);
-                sc[nt][3] = exp2f(sc[nt][3] - refB);
-                lA += sc[nt][0] + sc[nt][1];
-                lB += sc[nt][2] + sc[nt][3];
-            }
-
-            // O += P . V over 2 k-steps of 16 tokens; P from the S accumulator
-            // (token tiles 2kt, 2kt+1 of this half), split into bf16 hi + lo
-#pragma unroll
-            for (int kt = 0; kt < 2; ++kt) {
-                const int t16 = hf * 32 + kt * 16;  // first token of the k-step
-                uint32_t ph[4], pl[4];
-                {
-                    const float* s0 = sc[2 * kt];
-                    const float* s1 = sc[2 * kt + 1];
-                    ph[0] = pack_bf16(s0[0], s0[1]);
-                    ph[1] = pack_bf16(s0[2], s0[3]);
-                    ph[2] = pack_bf16(s1[0], s1[1]);
-                    ph[3] = pack_bf16(s1[2], s1[3]);
-                    pl[0] = pack_bf16(s0[0] - bf16_round(s0[0]), s0[1] - bf16_round(s0[1]));
-                    pl[1] = pack_bf16(s0[2] - bf16_round(s0[2]), s0[3] - bf16_round(s0[3]));
-                    pl[2] = pack_bf16(s1[0] - bf16_round(s1[0]), s1[1] - bf16_round(s1[1]));
-                    pl[3] = pack_bf16(s1[2] - bf16_round(s1[2]), s1[3] - bf16_round(s1[3]));
-                }
-                // V tokens this lane's B fragments carry: t16 + 2tig (+1), and + 8
-                uint32_t keep0 = 0xffffffffu, keep1 = 0xffffffffu;
-                if (!whole) {
-                    auto valid = [&](int tok) {
-                        const int jrel = ((tbase + tok) >> p.log2_bs) - (tbase >> p.log2_bs);
-                        return tok < ntok && !((bad >> jrel) & 1u);
-                    };
-                    const int t = t16 + 2 * tig;
-                    keep0 = (valid(t) ? 0x0000ffffu : 0u) | (valid(t + 1) ? 0xffff0000u : 0u);
-                    keep1 = (valid(t + 8) ? 0x0000ffffu : 0u) | (valid(t + 9) ? 0xffff0000u : 0u);
-                }
-#pragma unroll
-                for (int d2 = 0; d2 < C::DT / 2; ++d2) {
-                    uint32_t r[4];
-                    ldsm_x4_t(swz(svb, t16 + kr + 8 * (kq & 1), d2 * 16 + 8 * (kq >> 1),
-                                  C::HALF_BYTES),
-                              r);
-                    r[0] &= keep0;
-                    r[1] &= keep1;
-                    r[2] &= keep0;
-                    r[3] &= keep1;
-                    mma_bf16(o[2 * d2], ph, r[0], r[1]);
-                    mma_bf16(o[2 * d2], pl, r[0], r[1]);
-                    mma_bf16(o[2 * d2 + 1], ph, r[2], r[3]);
-                    mma_bf16(o[2 * d2 + 1], pl, r[2], r[3]);
-                }
-            }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[ring.stage]);
-        ring.advance(kStagesP);
+        tc_fence_before();
     }
-
-    // the row sums: add the quad's partials
-    lA += __shfl_xor_sync(FULL_MASK, lA, 1);
-    lA += __shfl_xor_sync(FULL_MASK, lA, 2);
-    lB += __shfl_xor_sync(FULL_MASK, lB, 1);
-    lB += __shfl_xor_sync(FULL_MASK, lB, 2);
-    // partial state of this split for rows A and B
-    if (bA >= 0) {
-        const size_t row = ((size_t)sp * p.num_seqs + bA) * p.num_q_heads + hA;
-        if (tig == 0) {
-            p.pfx_ml[row * 2] = mA;
-            p.pfx_ml[row * 2 + 1] = lA;
-        }
-        float* ra = p.pfx_acc + row * D;
-#pragma unroll
-        for (int dt = 0; dt < C::DT; ++dt)
-            *reinterpret_cast<float2*>(ra + dt * 8 + 2 * tig) = make_float2(o[dt][0], o[dt][1]);
-    }
-    if (bB >= 0) {
-        const size_t row = ((size_t)sp * p.num_seqs + bB) * p.num_q_heads + hB;
-        if (tig == 0) {
-            p.pfx_ml[row * 2] = mB;
-            p.pfx_ml[row * 2 + 1] = lB;
-        }
-        float* ra = p.pfx_acc + row * D;
-#pragma unroll
-        for (int dt = 0; dt < C::DT; ++dt)
-            *reinterpret_cast<float2*>(ra + dt * 8 + 2 * tig) = make_float2(o[dt][2], o[dt][3]);
+    // The MMA warp (its MMAs drained) and the softmax warps (their tensor-memory
+    // loads and stores complete) meet before the tensor memory is freed.
+    named_bar_sync(1, 32 * (1 + kSoftWarps));
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, kTmemCols);
     }
 }
 

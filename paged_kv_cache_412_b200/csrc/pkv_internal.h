@@ -142,7 +142,7 @@ struct PrefixParams {
 };
 
 // Rows of (member, query head) pairs one CTA of the shared pass covers.
-constexpr int kPrefixRows = 64;
+constexpr int kPrefixRows = 128;
 
 pkv_status launch_decode_prefix(const PrefixParams& p, const void* k_cache, const void* v_cache,
                                 int head_dim, cudaStream_t stream);
