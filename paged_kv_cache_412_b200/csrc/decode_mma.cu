@@ -73,6 +73,10 @@ struct MmaCfg {
     // on.  fp8: K | V only (8 or 4 KB each, whole swizzle periods); each
     // consumer reads the group's q from global memory.
     static constexpr int STAGE_BYTES = F8 ? 2 * KV_BYTES : (2 * KV_BYTES + Q_BYTES + 1023) / 1024 * 1024;
+    // row-copy stages (bf16 blocks of 2 or 4 rows): K | V regions of up to 32
+    // skewed blocks (rc_block_bytes), inside the same stage size
+    static constexpr int RC_KV_BYTES = kCH * D * 2 + 32 * 16;
+    static_assert(F8 || 2 * RC_KV_BYTES <= STAGE_BYTES, "row-copy regions fit a stage");
     // bf16: one tensor-core consumer reads the TMA stages (two CTAs per SM).
     // fp8: one CTA per SM whose NCONS consumers take the CTA's chunks in turn
     // (chunk n -> consumer n % NCONS, stage n % NSTAGE; NSTAGE is a multiple of
@@ -140,6 +144,26 @@ __device__ __forceinline__ int f8_swz(int row) {
         return row & 7;
     else
         return (row >> 1) & 3;
+}
+
+// Row-copy stages (bf16, blocks of 2 or 4 rows): block j of the chunk holds
+// its rows contiguously at j * rc_block_bytes, one 16-byte bank group further
+// than a dense packing would put it, so rows of eight consecutive blocks fall
+// in eight distinct bank groups.  K and V regions of 32 blocks of 2 rows (the
+// larger case) fit inside a bf16 stage.
+template <int D>
+__device__ __forceinline__ int rc_block_bytes(int block_size) {
+    return block_size * D * 2 + 16;
+}
+
+// Token (within the 64-token chunk) behind MMA row i of token tile mt in
+// row-copy stages: a tile is one in-block row (mt % block_size) of 16
+// consecutive blocks, so each 8-row ldmatrix tile reads eight different
+// blocks.  q.K^T and P.V use the same mapping, so the token order inside the
+// chunk is immaterial.
+__device__ __forceinline__ int rc_token(int mt, int i, int log2_bs) {
+    const int bs = 1 << log2_bs;
+    return bs * (16 * (mt >> log2_bs) + i) + (mt & (bs - 1));
 }
 
 // ---- producer ------------------------------------------------------------------
@@ -241,46 +265,34 @@ struct Producer {
             unsigned char* sv = sk + C::KV_BYTES;
             unsigned char* sq = sv + C::KV_BYTES;
             if constexpr (RC) {
-                // Blocks of 2 or 4 rows: each lane copies whole token rows
-                // (tokens lane and lane + 32) in 16-byte pieces to their
-                // swizzled places, and the q rows with the segment's first
-                // stage; the stage completes when all 32 lanes' copies have.
+                // Blocks of 2 or 4 rows: a block's rows of one kv head are one
+                // contiguous run of block_size * D bf16, fetched with one bulk
+                // copy per (block, K or V) -- 32 or 64 per chunk, one or two
+                // per lane -- into the skewed layout of rc_block_bytes().  The
+                // consumer reads q from global memory.
+                const uint32_t run = (uint32_t)p.block_size * D * 2u;
                 if (lane == 0) {
                     st_ntok[stage] = ntok;
                     st_bad[stage] = bad;
                     if (bad) raise_error(p.err, PKV_DEVERR_BAD_BLOCK);
+                    mbar_arrive_expect_tx(&full[stage], nvalid * 2u * run);
                 }
+                __syncwarp();  // the expect-tx above comes first
 #pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    const int t = lane + 32 * r;
-                    const int j = (t0 + min(t, ntok - 1)) >> p.log2_bs;
-                    const int phys = __shfl_sync(FULL_MASK, tab, j - wbase);
-                    if (t < ntok && phys >= 0 && phys < p.num_blocks) {
-                        const int off = (t0 + t) & (p.block_size - 1);
-                        const size_t row =
-                            ((size_t)phys * p.num_kv_heads + kvh) * p.block_size + off;
-                        const unsigned char* gk =
-                            static_cast<const unsigned char*>(p.k_cache) + row * D * 2;
-                        const unsigned char* gvr =
-                            static_cast<const unsigned char*>(p.v_cache) + row * D * 2;
-#pragma unroll
-                        for (int c16 = 0; c16 < D / 8; ++c16) {
-                            const int so = (c16 >> 3) * C::HALF_BYTES + t * 128 +
-                                           (((c16 & 7) ^ (t & 7)) << 4);
-                            cp_async16(sk + so, gk + c16 * 16);
-                            cp_async16(sv + so, gvr + c16 * 16);
-                        }
+                for (int it = 0; it < 2; ++it) {
+                    const int cp = lane + 32 * it;  // copy cp: block cp / 2, K (even) or V
+                    const int jrel = cp >> 1;
+                    const int phys = __shfl_sync(FULL_MASK, tab, min(ja + jrel, jb) - wbase);
+                    if (ja + jrel <= jb && phys >= 0 && phys < p.num_blocks) {
+                        const size_t goff =
+                            ((size_t)phys * p.num_kv_heads + kvh) * p.block_size * D * 2;
+                        const unsigned char* src =
+                            static_cast<const unsigned char*>((cp & 1) ? p.v_cache : p.k_cache) + goff;
+                        bulk_load(sk + ((cp & 1) ? C::RC_KV_BYTES : 0) +
+                                      jrel * rc_block_bytes<D>(p.block_size),
+                                  src, run, &full[stage], policy);
                     }
                 }
-                if (c == sg.c0) {
-                    const unsigned char* gq = reinterpret_cast<const unsigned char*>(
-                        static_cast<const __nv_bfloat16*>(p.q) +
-                        ((size_t)cur.b * p.num_q_heads + hq0) * D);
-                    for (int i = lane; i < gv * D * 2 / 16; i += 32)
-                        cp_async16(sq + i * 16, gq + i * 16);
-                }
-                __threadfence_block();  // the chunk's meta before the arrival
-                cp_async_mbar_arrive(&full[stage]);
                 ++issued;
                 last_n = n;
                 continue;
@@ -401,7 +413,7 @@ __device__ __forceinline__ SegInfo seg_info(const DecodeParams& p, const Segment
 //   P.V: the widened words are 8 x 8 tiles with tokens as rows; movmatrix.trans
 //     makes them A fragments of V^T with tokens as k, and the head-dim rows
 //     come out permuted as dcol<true> describes.
-template <int D, int NT, bool F8>
+template <int D, int NT, bool F8, bool RC>
 __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                                         unsigned char* smem, uint64_t* full, uint64_t* empty,
                                         uint64_t* dfull, uint64_t* dempty, const int* st_ntok,
@@ -439,13 +451,16 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
         }
 
         bool have_q = false;
-        if constexpr (F8) {
-            // Q^T B-fragments in the permuted order: head nt*8+grp, dims
-            // 16 ks + 4 tig, +1 (b0) and 16 ks + 4 tig + 2, +3 (b1), bf16 -> f16.
+        if constexpr (F8 || RC) {
+            // Q^T B-fragments straight from global memory, head nt*8+grp.
+            // fp8: the permuted order, dims 16 ks + 4 tig, +1 (b0) and
+            // 16 ks + 4 tig + 2, +3 (b1), widened bf16 -> f16.  Row copies: the
+            // natural order, dims 16 ks + 2 tig, +1 (b0) and + 8, + 9 (b1).
             // Only a consumer with a chunk of this segment needs them.
-            bool any = false;
-            for (unsigned n = n_chunk; n < n_chunk + (unsigned)(sg.c1 - sg.c0); ++n)
-                any |= (int)(n % C::NCONS) == me;
+            bool any = !F8;
+            if constexpr (F8)
+                for (unsigned n = n_chunk; n < n_chunk + (unsigned)(sg.c1 - sg.c0); ++n)
+                    any |= (int)(n % C::NCONS) == me;
             if (any) {
                 if (!waited) {
                     griddep_wait();  // q may come from the previous kernel
@@ -458,11 +473,17 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                     const int h = nt * 8 + grp;
 #pragma unroll
                     for (int ks = 0; ks < C::KS; ++ks) {
-                        uint2 w = make_uint2(0u, 0u);
-                        if (h < si.gv)
-                            w = __ldg(reinterpret_cast<const uint2*>(gq + (size_t)h * D + ks * 16 + 4 * tig));
-                        qb[nt][ks][0] = bf16x2_to_f16x2(w.x);
-                        qb[nt][ks][1] = bf16x2_to_f16x2(w.y);
+                        if constexpr (F8) {
+                            uint2 w = make_uint2(0u, 0u);
+                            if (h < si.gv)
+                                w = __ldg(reinterpret_cast<const uint2*>(gq + (size_t)h * D + ks * 16 + 4 * tig));
+                            qb[nt][ks][0] = bf16x2_to_f16x2(w.x);
+                            qb[nt][ks][1] = bf16x2_to_f16x2(w.y);
+                        } else {
+                            const uint32_t* q32 = reinterpret_cast<const uint32_t*>(gq + (size_t)h * D);
+                            qb[nt][ks][0] = h < si.gv ? __ldg(q32 + ks * 8 + tig) : 0u;
+                            qb[nt][ks][1] = h < si.gv ? __ldg(q32 + ks * 8 + 4 + tig) : 0u;
+                        }
                     }
                 }
                 have_q = true;
@@ -494,7 +515,7 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
             unsigned char* sv = sk + C::KV_BYTES;
             const bool whole = ntok == kCH && bad == 0;
 
-            if (!F8 && !have_q) {
+            if (!F8 && !RC && !have_q) {
                 // The segment's first chunk carries the group's q.
                 // Q^T B-fragments: head nt*8+grp, dims ks*16 + 2*tig (+1) and +8 (+9).
                 have_q = true;
@@ -512,7 +533,7 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
 
             const uint32_t skb = smem_addr(sk), svb = smem_addr(sv);
 
-            if (!F8 && !whole) {
+            if (!F8 && !RC && !whole) {
                 // Rows of tokens that do not take part (past the end, or in a
                 // block the table got wrong) may hold stale or poisoned data:
                 // zero their V rows so 0-weight x NaN cannot reach the sum.
@@ -557,6 +578,21 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                                 mma_f16(s[mt][nt], a[h], qb[nt][2 * j + h][0], qb[nt][2 * j + h][1]);
                     }
                 }
+            } else if constexpr (RC) {
+                // rows of tile mt: token rc_token(mt, row), unswizzled in its block
+#pragma unroll
+                for (int mt = 0; mt < kMT; ++mt) {
+                    const int tok = rc_token(mt, k_row, p.log2_bs);
+                    const uint32_t rb = skb + (tok >> p.log2_bs) * rc_block_bytes<D>(p.block_size) +
+                                        (tok & (p.block_size - 1)) * D * 2;
+#pragma unroll
+                    for (int ks = 0; ks < C::KS; ++ks) {
+                        uint32_t a[4];
+                        ldsm_x4(rb + ((2 * ks + k_cx) << 4), a);
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) mma_bf16(s[mt][nt], a, qb[nt][ks][0], qb[nt][ks][1]);
+                    }
+                }
             } else {
 #pragma unroll
                 for (int ks = 0; ks < C::KS; ++ks) {
@@ -584,7 +620,7 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                 if (!whole) {
 #pragma unroll
                     for (int hi = 0; hi < 2; ++hi) {
-                        const int row = mt * 16 + grp + 8 * hi;
+                        const int row = RC ? rc_token(mt, grp + 8 * hi, p.log2_bs) : mt * 16 + grp + 8 * hi;
                         const int jrel = ((c * kCH + row) >> p.log2_bs) - ((c * kCH) >> p.log2_bs);
                         const bool valid = row < ntok && !((bad >> jrel) & 1u);
                         if (!valid) {
@@ -688,6 +724,39 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                             }
                         }
                     }
+                } else if constexpr (RC) {
+                    // V^T by ldmatrix.trans over the rows of tile mt (tokens
+                    // rc_token(mt, k)); a token that does not take part is
+                    // zeroed in registers (k = 2 tig, 2 tig + 1 in a0/a1 and
+                    // k + 8 in a2/a3)
+                    const int tok = rc_token(mt, v_row, p.log2_bs);
+                    const uint32_t rb = svb + (tok >> p.log2_bs) * rc_block_bytes<D>(p.block_size) +
+                                        (tok & (p.block_size - 1)) * D * 2;
+                    uint32_t keep0 = 0xffffffffu, keep1 = 0xffffffffu;
+                    if (!whole) {
+                        auto valid = [&](int k) {
+                            const int t = rc_token(mt, k, p.log2_bs);
+                            const int jrel = ((c * kCH + t) >> p.log2_bs) - ((c * kCH) >> p.log2_bs);
+                            return t < ntok && !((bad >> jrel) & 1u);
+                        };
+                        keep0 = (valid(2 * tig) ? 0x0000ffffu : 0u) | (valid(2 * tig + 1) ? 0xffff0000u : 0u);
+                        keep1 = (valid(2 * tig + 8) ? 0x0000ffffu : 0u) |
+                                (valid(2 * tig + 9) ? 0xffff0000u : 0u);
+                    }
+#pragma unroll
+                    for (int dt = 0; dt < C::KS; ++dt) {
+                        uint32_t a[4];
+                        ldsm_x4_t(rb + ((2 * dt + v_cx) << 4), a);
+                        a[0] &= keep0;
+                        a[1] &= keep0;
+                        a[2] &= keep1;
+                        a[3] &= keep1;
+#pragma unroll
+                        for (int nt = 0; nt < NT; ++nt) {
+                            mma_bf16(acc[dt][nt], a, bh[nt][0], bh[nt][1]);
+                            mma_bf16(acc[dt][nt], a, bl[nt][0], bl[nt][1]);
+                        }
+                    }
                 } else {
 #pragma unroll
                     for (int dt = 0; dt < C::KS; ++dt) {
@@ -703,7 +772,7 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                     }
                 }
             }
-            if (!F8 && !whole) fence_proxy_async_smem();  // our zero-fill before the next TMA write
+            if (!F8 && !RC && !whole) fence_proxy_async_smem();  // our zero-fill before the next TMA write
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
             if constexpr (!F8) ring.advance(C::NSTAGE);
@@ -1110,7 +1179,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
         pr.run(it);
         if (!pr.waited) griddep_wait();
     } else if (warp < C::NPROD + C::NCONS) {
-        consume<D, NT, F8>(p, it, smem, full, empty, dfull, dempty, st_ntok, st_bad, ctrl, lane,
+        consume<D, NT, F8, RC>(p, it, smem, full, empty, dfull, dempty, st_ntok, st_bad, ctrl, lane,
                            warp - C::NPROD);
     } else {
         epilogue<D, NT, F8>(p, it, smem, dfull, dempty, ctrl, lane);
