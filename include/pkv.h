@@ -137,9 +137,9 @@ size_t pkv_decode_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,
 /*
  * pkv_decode_workspace_init -- zero a decode workspace (asynchronous on
  * `stream`).  Call once after allocating a workspace, before its first decode.
- * Decode calls leave the workspace ready for the next call (the per-group
- * arrival counters they use return to zero), so re-initialising is needed only
- * if a call reported PKV_DEVERR_TIMEOUT.
+ * Decode calls leave the workspace ready for the next call (the ready flags
+ * of the partial results they use return to zero), so re-initialising is
+ * needed only if a call reported PKV_DEVERR_TIMEOUT.
  */
 pkv_status pkv_decode_workspace_init(void* workspace, size_t workspace_bytes,
                                      pkv_stream_t stream);

@@ -128,11 +128,10 @@ bool make_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_
     pl.off_meta = pl.off_ml + up(ml_bytes);
     pl.off_extra = pl.off_meta + up(meta_bytes);
     pl.rec_bytes = pl.off_extra + up(extra_bytes);
-    // smallest B with counter region(B) + records <= B and room for every counter
-    const size_t sync_words = std::max(pl.n_bg_max, pl.records);
-    size_t b = up(pl.rec_bytes + 2 * sync_words * sizeof(uint32_t));
-    while (counter_region_bytes(b) + pl.rec_bytes > b ||
-           ready_flags_offset(b) < sync_words * sizeof(uint32_t))
+    // smallest B with sync region(B) + records <= B and a flag for every record
+    size_t b = up(pl.rec_bytes + pl.records * sizeof(uint32_t));
+    while (sync_region_bytes(b) + pl.rec_bytes > b ||
+           sync_region_bytes(b) < pl.records * sizeof(uint32_t))
         b += 256;
     pl.bytes = b;
     *plan = pl;
@@ -344,12 +343,10 @@ pkv_status decode_entry(const void* q, const void* k_cache, const void* v_cache,
     p.out = out;
     p.k_scale = k_scale;
     p.v_scale = v_scale;
-    const size_t cnt_region = counter_region_bytes(workspace_bytes);
-    if (cnt_region + pl.rec_bytes > workspace_bytes ||
-        ready_flags_offset(workspace_bytes) < std::max(pl.n_bg_max, pl.records) * sizeof(uint32_t))
+    const size_t cnt_region = sync_region_bytes(workspace_bytes);
+    if (cnt_region + pl.rec_bytes > workspace_bytes || cnt_region < pl.records * sizeof(uint32_t))
         return PKV_ERR_WORKSPACE;
-    p.counters = reinterpret_cast<unsigned*>(ws);
-    p.ready = reinterpret_cast<unsigned*>(ws + ready_flags_offset(workspace_bytes));
+    p.ready = reinterpret_cast<unsigned*>(ws);
     p.rec_acc = reinterpret_cast<float*>(ws + cnt_region);
     p.rec_ml = reinterpret_cast<float*>(ws + cnt_region + pl.off_ml);
     p.meta = reinterpret_cast<int32_t*>(ws + cnt_region + pl.off_meta);

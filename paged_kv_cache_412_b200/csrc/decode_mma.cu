@@ -975,14 +975,14 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
             if (lane == 0) raise_error(p.err, PKV_DEVERR_BAD_SEQ_LEN);
             continue;
         }
-        // Arrive first.  Only a part that is not the last of its group to
-        // finish publishes its partial result (record, then a ready flag); the
-        // last one keeps its own in registers and merges the others'.
-        unsigned arrived = 0;
-        if (lane == 0) arrived = atomicAdd(p.counters + si.bg, 1u);
-        arrived = __shfl_sync(FULL_MASK, arrived, 0);
+        // The group's first unit merges.  A unit processes its chunks in
+        // list order, so the head of a group that runs on into later units is
+        // the last segment of its unit (nothing waits behind the merge), while
+        // the tail of a group is the first segment of its unit (published
+        // early).  The other parts publish their partial results (record,
+        // then a ready flag); the merger keeps its own in registers.
         const size_t rec = si.bg + si.u;
-        if (arrived != (unsigned)(si.nseg - 1)) {
+        if (si.u != si.u_first) {
             write_record<D, NT, F8>(p, rec, tig, grp, acc, m, l);
             __threadfence();
             __syncwarp();
@@ -990,7 +990,7 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
             continue;
         }
 
-        // Last part: wait (bounded) until every other part's record is out.
+        // Merger: wait (bounded) until every other part's record is out.
         int ok = 1;
         if (lane == 0) {
             const uint64_t t0 = global_timer_ns();
@@ -1089,7 +1089,6 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
         __syncwarp();
         if (lane == 0)  // ready for the next call
             for (long long uu = si.u_first; uu <= si.u_last; ++uu) p.ready[si.bg + uu] = 0u;
-        if (lane == 0) p.counters[si.bg] = 0u;  // ready for the next call
     }
 }
 

@@ -26,11 +26,12 @@ const DeviceInfo* current_device_info();
 // tensor-core one groups up to 16 query heads per kv-head pass, the CUDA-core
 // one up to 8), so one size fits whichever path the call takes.
 //
-// Layout of a workspace of B bytes: arrival counters first, in a region whose
-// size depends only on B (counter_region_bytes(B)), then the partial records.
-// A given buffer therefore always keeps its counters in the same words, which
-// every call returns to zero; records are always written before they are read
-// in the same call and need no clearing, whatever the sizes of the next call.
+// Layout of a workspace of B bytes: the records' ready flags first, in a
+// region whose size depends only on B (sync_region_bytes(B)), then the partial
+// records.  A given buffer therefore always keeps its flags in the same words,
+// which every call returns to zero; records are always written before they are
+// read in the same call and need no clearing, whatever the sizes of the next
+// call.
 struct DecodePlan {
     int rec_gp;        // floats per record row = largest query-head group of either path
     size_t n_bg_max;   // (request, head group) pairs, largest over the paths
@@ -43,14 +44,10 @@ struct DecodePlan {
 };
 
 // Bytes at the start of a B-byte workspace reserved for the merge's
-// synchronisation words: per-group arrival counters in its first half, one
-// ready flag per partial record in its second half.  Both return to zero at
-// the end of every call.
-inline size_t counter_region_bytes(size_t workspace_bytes) {
-    return (workspace_bytes / 128 + 255) / 256 * 256;
-}
-inline size_t ready_flags_offset(size_t workspace_bytes) {
-    return counter_region_bytes(workspace_bytes) / 2;
+// synchronisation words: one ready flag per partial record, which returns to
+// zero at the end of every call.
+inline size_t sync_region_bytes(size_t workspace_bytes) {
+    return (workspace_bytes / 256 + 255) / 256 * 256;
 }
 
 // Fill a plan for these sizes on the current device (false if invalid).
@@ -72,8 +69,7 @@ struct DecodeParams {
     float* rec_acc;   // [records][group_pad][head_dim]
     float* rec_ml;    // [records][group_pad][2]  (running max in log2 units, sum)
     int32_t* meta;    // [num_seqs * num_hg][2]   (first unit, number of units)
-    unsigned* counters;  // [num_seqs * num_hg] arrivals per split group (zero between calls)
-    unsigned* ready;     // [records] 1 once a partial record is written (zero between calls)
+    unsigned* ready;  // [records] 1 once a partial record is written (zero between calls)
     unsigned* err;
     int num_seqs, num_q_heads, num_kv_heads, group, num_sub, num_hg;
     int block_size, log2_bs, max_blocks, num_blocks;
