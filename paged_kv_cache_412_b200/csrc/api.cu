@@ -361,6 +361,7 @@ pkv_status decode_entry(const void* q, const void* k_cache, const void* v_cache,
     p.log2_bs = log2_int(block_size);
     p.max_blocks = max_blocks_per_seq;
     p.num_blocks = num_blocks;
+    p.max_len_hint = max_seq_len;
     p.fixed_units = partition_size > 0 ? std::max(1, partition_size / (mma ? 64 : 32)) : 0;
     // Fixed partitions and prefix groups on the tensor-core path: merge in a
     // separate kernel, so a group split into many parts (or folded with many

@@ -344,11 +344,20 @@ struct Producer {
         return true;
     }
 
-    __device__ void run(SegIter<kCH>& it) {
+    // spec_b / spec_j / spec_tab: a table window of request spec_b starting
+    // at block spec_j, loaded before the plan was known (spec_b < 0: none);
+    // used if the CTA's first segment starts there.
+    __device__ void run(SegIter<kCH>& it, int spec_b, int spec_j, int spec_tab) {
         int tab_first = -1;
         if (it.valid) {
             const Segment sg = it.current();
-            tab_first = load_window(sg.cur, first_block(sg.cur, sg.c0, p.log2_bs));
+            const int j0 = first_block(sg.cur, sg.c0, p.log2_bs);
+            if (sg.cur.b == spec_b && j0 == spec_j) {
+                const int nblk = (sg.cur.L + p.block_size - 1) >> p.log2_bs;
+                tab_first = j0 + lane < nblk ? spec_tab : -1;
+            } else {
+                tab_first = load_window(sg.cur, j0);
+            }
         }
         while (it.valid) {
             const Segment sg = it.current();
@@ -1154,6 +1163,24 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
     // guarantees are not produced by the kernel right before this one; so it
     // overlaps that kernel's tail.  Each role waits on the grid dependency
     // before touching K/V, q, out or the workspace.
+    // The producer first guesses its first table window from the largest
+    // length the caller announced (exact for a batch of equal lengths) and
+    // starts loading it, so that load overlaps the seq_lens round trip.
+    int spec_b = -1, spec_j = -1, spec_tab = -1;
+    if (warp < C::NPROD && !p.prefix_of && p.fixed_units == 0 && p.max_len_hint > 0) {
+        const int Lg = min(p.max_len_hint, p.max_blocks * p.block_size);
+        const long long nchg = chunks_of<kCH>(Lg);
+        const long long totg = nchg * p.num_hg * p.num_seqs;
+        const long long Wg = (totg + gridDim.x - 1) / gridDim.x;
+        const long long s0 = (long long)blockIdx.x * Wg;
+        if (s0 < totg) {
+            spec_b = (int)(s0 / (nchg * p.num_hg));
+            spec_j = (int)((s0 % nchg) * kCH) >> p.log2_bs;
+            const int nblkg = (Lg + p.block_size - 1) >> p.log2_bs;
+            if (spec_j + lane < nblkg)
+                spec_tab = __ldg(p.block_tables + (size_t)spec_b * p.max_blocks + spec_j + lane);
+        }
+    }
     int L_first = 0, T_first = 0;
     const long long total =
         total_chunks_warp(p, lane, blockIdx.x == 0 && warp == 0, &L_first, &T_first);
@@ -1175,7 +1202,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
         Producer<D, NT, F8, RC> pr{p, &tmk, &tmv, smem, full, empty, st_ntok, st_bad, ctrl, lane,
                            l2_policy_evict_first()};
         pr.me = warp;
-        pr.run(it);
+        pr.run(it, spec_b, spec_j, spec_tab);
         if (!pr.waited) griddep_wait();
     } else if (warp < C::NPROD + C::NCONS) {
         consume<D, NT, F8, RC>(p, it, smem, full, empty, dfull, dempty, st_ntok, st_bad, ctrl, lane,

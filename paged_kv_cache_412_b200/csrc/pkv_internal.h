@@ -74,6 +74,7 @@ struct DecodeParams {
     int num_seqs, num_q_heads, num_kv_heads, group, num_sub, num_hg;
     int block_size, log2_bs, max_blocks, num_blocks;
     int fixed_units;  // 0 = automatic
+    int max_len_hint;  // the caller's bound of seq_lens (a guess of the first table window)
     int defer_merge;  // 1: parts of a split group only publish records (+ meta);
                       // a separate merge kernel combines them
     int row_copy;     // 1: blocks of 2 or 4 rows -- the producer copies token rows
