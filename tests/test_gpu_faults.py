@@ -102,17 +102,17 @@ def test_clean_run_leaves_no_flag(pkv):
     assert pkv.get_device_error() == 0
 
 
-@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
-def test_bad_block_tokens_do_not_take_part(pkv, dtype):
+@pytest.mark.parametrize("dtype,bs", [("bf16", 16), ("fp8", 16), ("bf16", 4), ("bf16", 2)])
+def test_bad_block_tokens_do_not_take_part(pkv, dtype, bs):
     """A table entry outside the pool: that block's tokens are left out of the
     request's softmax (the others are unaffected) and PKV_DEVERR_BAD_BLOCK is
     raised.  Expected values: numpy brute force over the rows that remain."""
     from oracle import brute
-    bs = 16
     w = workloads.make_paged([100, 64, 50], Hq=8, Hkv=2, d=128, bs=bs, dtype=dtype, seed=3,
                              append_last=False)
     bt = w.block_tables.copy()
-    bt[1, 2] = w.num_blocks + 7  # request 1's third block (tokens 32..47) is out of range
+    bad_blk = 32 // bs  # request 1's block holding token 32 (tokens 32 .. 32 + bs - 1)
+    bt[1, bad_blk] = w.num_blocks + 7
     dw = DevWorkload(w)
     out = pkv.paged_attention_decode(dw.q, dw.k_cache, dw.v_cache, to_dev(bt), dw.seq_lens, bs,
                                      w.scale, out_dtype=torch.float32, k_scale=dw.k_scale,
@@ -130,7 +130,7 @@ def test_bad_block_tokens_do_not_take_part(pkv, dtype):
     q = brute.bf16_bits_to_f64(w.q)
     for b in range(3):
         L = int(w.seq_lens[b])
-        keep = [t for t in range(L) if not (b == 1 and 32 <= t < 48)]
+        keep = [t for t in range(L) if not (b == 1 and 32 <= t < 32 + bs)]
         for hq in range(w.Hq):
             h = hq // G
             ref = brute.attention_numpy(q[b, hq], rows(w.k_cache, w.k_scale, b, h, keep),

@@ -68,6 +68,9 @@ SMALL = [
     ([90, 45], 16, 1, 128, 16, "bf16"),          # G = 16 (two head groups per kv head)
     ([70, 200, 5], 6, 3, 64, 1, "f32"),          # block size 1
     ([70, 200, 5], 10, 2, 128, 4, "bf16"),       # G = 5
+    ([70, 200, 5, 64], 8, 2, 128, 2, "bf16"),    # block size 2 (bulk copies of 2-row runs)
+    ([130, 1, 64], 16, 1, 64, 4, "bf16"),        # block size 4, d 64, G = 16
+    ([257, 33, 4096], 32, 8, 128, 2, "bf16"),    # block size 2, split groups
     ([300, 129], 8, 2, 128, 64, "bf16"),         # block larger than a stage
     ([513, 20], 8, 4, 64, 256, "f32"),           # block size 256
     ([0, 40, 0, 1], 4, 2, 128, 16, "bf16"),      # empty requests

@@ -61,7 +61,8 @@ CASES = [
     (32, 16, 8, 64, [(6, 512), (2, 96)], 2, 1),
     (128, 32, 8, 128, [(5, 384), (3, 128)], 1, 1),
     (16, 32, 2, 128, [(6, 320), (2, 64)], 1, 1),   # 16 query heads per kv head
-    (16, 24, 8, 64, [(23, 192), (5, 48)], 2, 2),   # 3 query heads per kv head, 2 row tiles
+    (16, 24, 8, 64, [(23, 192), (5, 48)], 2, 2),   # 3 query heads per kv head
+    (16, 64, 8, 128, [(40, 448), (3, 32)], 1, 2),  # 320 rows: three 128-row tiles, the last partial
 ]
 
 
