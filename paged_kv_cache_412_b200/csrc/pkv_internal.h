@@ -36,6 +36,7 @@ struct DecodePlan {
     int rec_gp;        // floats per record row = largest query-head group of either path
     size_t n_bg_max;   // (request, head group) pairs, largest over the paths
     size_t units_max;  // upper bound of split units
+    size_t dyn_base;   // first record of the dynamic tails (one per group after it)
     size_t records;    // partial-result records
     size_t rec_bytes;  // records + their (max, sum) pairs + per-group meta
     size_t off_ml, off_meta;  // offsets inside the record region
@@ -44,10 +45,18 @@ struct DecodePlan {
 };
 
 // Bytes at the start of a B-byte workspace reserved for the merge's
-// synchronisation words: one ready flag per partial record, which returns to
-// zero at the end of every call.
+// synchronisation words, all of which return to zero at the end of every call:
+// one ready flag per partial record in its first half, per-group arrival
+// counters in its second half, and the two ticket words of the dynamic tails
+// in its last 8 bytes.
 inline size_t sync_region_bytes(size_t workspace_bytes) {
-    return (workspace_bytes / 256 + 255) / 256 * 256;
+    return (workspace_bytes / 128 + 255) / 256 * 256;
+}
+inline size_t sync_counters_offset(size_t workspace_bytes) {
+    return sync_region_bytes(workspace_bytes) / 2;
+}
+inline size_t sync_tickets_offset(size_t workspace_bytes) {
+    return sync_region_bytes(workspace_bytes) - 8;
 }
 
 // Fill a plan for these sizes on the current device (false if invalid).
@@ -77,8 +86,16 @@ struct DecodeParams {
     int max_len_hint;  // the caller's bound of seq_lens (a guess of the first table window)
     int defer_merge;  // 1: parts of a split group only publish records (+ meta);
                       // a separate merge kernel combines them
-    int row_copy;     // 1: blocks of 2 or 4 rows -- the producer copies token rows
-                      // with per-lane 16-byte async copies instead of TMA boxes
+    int row_copy;     // 1: blocks of 2 or 4 rows -- one bulk copy per (block, K or V)
+                      // into a skewed stage layout instead of TMA boxes
+    // Dynamic tails (automatic split only; 0 = off): the last tail_chunks
+    // chunks of every (request, head group) are left out of the static split
+    // and handed out one group at a time, by an atomic ticket, to the CTAs that
+    // finish their static unit first.  Their records start at dyn_rec_base + bg.
+    int tail_chunks;
+    long long dyn_rec_base;
+    unsigned* counters;  // [num_seqs * num_hg] arrivals per split group (zero between calls)
+    unsigned* tickets;   // [2]: next tail ticket, CTAs done fetching (zero between calls)
     long long rec_cap;  // records the workspace holds
     int out_dtype;
     float scale_log2;  // softmax scale * log2(e)
