@@ -295,6 +295,9 @@ struct SegIter {
         ++qk;
         if (lane == 0) {
             if (fetcher) {
+                // the ticket words are workspace: the previous kernel in the
+                // stream may still be using this workspace
+                griddep_wait();
                 if (failed || !mbar_wait(&q.empty[slot], ph ^ 1u, p.wait_ns)) {
                     failed = true;
                 } else {
