@@ -1476,12 +1476,40 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
+namespace {
+
+// The last few views encoded, so that a caller decoding the same caches call
+// after call (every layer of a serving loop) pays for encoding once.
+struct MapCacheEntry {
+    const void* base = nullptr;
+    long long rows = 0;
+    int head_dim = 0, box_rows = 0;
+    bool fp8 = false;
+    CUtensorMap map;
+};
+constexpr int kMapCache = 16;
+std::mutex g_map_mu;
+MapCacheEntry g_map_cache[kMapCache];
+int g_map_next = 0;
+
+}  // namespace
+
 // 2-D view of a cache: rows = num_blocks*Hkv*block_size, columns = head_dim
 // bf16; boxes of 64 columns x min(block_size, 64) rows, 128-byte swizzle.
 // fp8: rows of head_dim one-byte codes, whole-row boxes with the swizzle of
-// their width (128 bytes at head_dim 128, 64 at 64); the converters undo it.
+// their width (128 bytes at head_dim 128, 64 at 64), which the consumers'
+// reads apply.
 bool encode_cache_map(CUtensorMap* map, const void* base, long long rows, int head_dim,
                       int box_rows, bool fp8) {
+    {
+        std::lock_guard<std::mutex> lock(g_map_mu);
+        for (const MapCacheEntry& e : g_map_cache)
+            if (e.base == base && e.rows == rows && e.head_dim == head_dim &&
+                e.box_rows == box_rows && e.fp8 == fp8) {
+                *map = e.map;
+                return true;
+            }
+    }
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint64_t gdim[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
@@ -1494,7 +1522,17 @@ bool encode_cache_map(CUtensorMap* map, const void* base, long long rows, int he
                            (fp8 && head_dim == 64) ? CU_TENSOR_MAP_SWIZZLE_64B
                                                    : CU_TENSOR_MAP_SWIZZLE_128B,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    if (r != CUDA_SUCCESS) return false;
+    std::lock_guard<std::mutex> lock(g_map_mu);
+    MapCacheEntry& e = g_map_cache[g_map_next];
+    g_map_next = (g_map_next + 1) % kMapCache;
+    e.base = base;
+    e.rows = rows;
+    e.head_dim = head_dim;
+    e.box_rows = box_rows;
+    e.fp8 = fp8;
+    e.map = *map;
+    return true;
 }
 
 bool decode_mma_supported(int head_dim, int block_size, pkv_dtype q_dtype, pkv_dtype kv_dtype) {
