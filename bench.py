@@ -613,6 +613,15 @@ class _L2Flush:
         self.buf.zero_()
 
 
+def _device_clean():
+    """Fail fast (before any timed launch) if the library's device error word
+    is set: a call that reported an error is not worth timing."""
+    import paged_kv_cache_412_b200 as pkv
+    flags = pkv.get_device_error()
+    if flags:
+        raise RuntimeError(f"device error word 0x{flags:x} before timing")
+
+
 def _time_graph(fn, iters, flush, warm=5):
     """Mean / median device time (ms) of ``fn`` captured in a CUDA graph, L2
     flushed before each launch, CUDA events around each launch."""
@@ -620,6 +629,7 @@ def _time_graph(fn, iters, flush, warm=5):
     for _ in range(2):
         fn()
     torch.cuda.synchronize()
+    _device_clean()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         fn()

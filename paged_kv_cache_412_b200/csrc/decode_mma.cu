@@ -1183,8 +1183,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
     if (threadIdx.x == 0) {
         ctrl[0] = 0;
         for (int s = 0; s < C::NSTAGE; ++s) {
-            // row copies: every producer lane arrives once its copies have landed
-            mbar_init(&full[s], RC ? 32 : 1);
+            mbar_init(&full[s], 1);  // the producer's expect-tx arrival
             mbar_init(&empty[s], 1);  // released by the stage's one consumer
         }
         for (int s = 0; s < S::NSLOT; ++s) {
