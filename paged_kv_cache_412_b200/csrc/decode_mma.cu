@@ -82,9 +82,11 @@ struct MmaCfg {
     // (chunk n -> consumer n % NCONS, stage n % NSTAGE; NSTAGE is a multiple of
     // NCONS, so a stage always serves the same consumer and each barrier has
     // one waiter stepping through its phases in order).  Widening codes costs
-    // instructions the bf16 path does not have; four consumers put one on
-    // every SM sub-partition.
-    static constexpr int NCONS = F8 ? 4 : 1;
+    // instructions and latency the bf16 path does not have, and one consumer
+    // warp cannot hide its own ldmatrix -> cvt -> mma chains: six consumers
+    // (two on each of two SM sub-partitions) overlap them; the 16-head
+    // configuration keeps four (its consumers need all the registers).
+    static constexpr int NCONS = F8 ? (NT == 1 ? 6 : 4) : 1;
     // producer warps: a TMA issue holds the issuing warp ~0.1 us, and one fp8
     // producer per SM cannot issue fast enough; two take alternate chunks
     // (stage n % NSTAGE belongs to producer n % NPROD).
@@ -93,10 +95,11 @@ struct MmaCfg {
     // consumer -> epilogue hand-off: per lane, the accumulators and (m, l)
     static constexpr int DUMP_BYTES = (KS * NT * 4 + NT * 4) * 32 * 4;
     // fp8: as many stages as the shared memory holds beside the hand-off
-    // slots (up to 24), a multiple of NCONS and NPROD: ~190 KB of codes in
-    // flight per SM, as much as the two bf16 CTAs of an SM keep
+    // slots (up to 24), a multiple of NCONS and NPROD: 192 KB of codes in
+    // flight per SM at head_dim 128, as much as the two bf16 CTAs of an SM keep
     static constexpr int F8_RING = 227 * 1024 - NCONS * DUMP_BYTES - 4096;
-    static constexpr int NSTAGE = F8 ? cmin(24, F8_RING / STAGE_BYTES) / 4 * 4
+    static constexpr int STAGE_STEP = F8 ? (NCONS % 2 == 0 ? NCONS : 2 * NCONS) : 1;  // lcm(NCONS, 2)
+    static constexpr int NSTAGE = F8 ? cmin(24, F8_RING / STAGE_BYTES) / STAGE_STEP * STAGE_STEP
                                      : cmax(2, cmin(8, kRingBudget / STAGE_BYTES));
     static_assert(NSTAGE % NPROD == 0 && NSTAGE % NCONS == 0 && NSTAGE >= 2,
                   "each stage belongs to one producer and one consumer");
