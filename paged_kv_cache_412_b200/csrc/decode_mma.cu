@@ -885,12 +885,40 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
     Ring dring;
     griddep_wait();  // `out` and the workspace may be in use by the previous kernel
     // Requests with no token at all: all-zero rows (softmax of an empty set).
-    // (A request whose shared prefix covers all of it has no token of its own
-    // pass either; the merge kernel writes it from the shared pass's results.)
+    // A request whose shared prefix covers all of it has no token of its own
+    // pass either: unless a separate merge kernel follows, its rows are the
+    // merge of the shared pass's splits alone.
     for (int b = blockIdx.x; b < p.num_seqs; b += gridDim.x) {
-        if (clamp_len(p, b, false) != 0) continue;
-        for (int i = lane; i < p.num_q_heads * D; i += 32)
-            store_out(p.out, (size_t)b * p.num_q_heads * D + i, 0.f, p.out_dtype);
+        const int L = clamp_len(p, b, false);
+        if (L == 0) {
+            for (int i = lane; i < p.num_q_heads * D; i += 32)
+                store_out(p.out, (size_t)b * p.num_q_heads * D + i, 0.f, p.out_dtype);
+        } else if (!p.defer_merge && seq_begin(p, b, L) == L) {
+            const int ns = prefix_num_splits(prefix_tokens_of(p, b), p.pfx_splits);
+            for (int hq = 0; hq < p.num_q_heads; ++hq) {
+                const size_t row = (size_t)b * p.num_q_heads + hq;
+                float M = -INFINITY, Sum = 0.f, Acc[D / 32];
+#pragma unroll
+                for (int i = 0; i < D / 32; ++i) Acc[i] = 0.f;
+                for (int sp = 0; sp < ns; ++sp) {
+                    const size_t rr = (size_t)sp * p.num_seqs * p.num_q_heads + row;
+                    const float ms = ld_cg(p.pfx_ml + rr * 2), ls = ld_cg(p.pfx_ml + rr * 2 + 1);
+                    const float Mn = fmaxf(M, ms);
+                    const float ref = Mn == -INFINITY ? 0.f : Mn;
+                    const float fa = exp2f(M - ref), fb = exp2f(ms - ref);
+                    Sum = Sum * fa + ls * fb;
+#pragma unroll
+                    for (int i = 0; i < D / 32; ++i)
+                        Acc[i] = Acc[i] * fa + ld_cg(p.pfx_acc + rr * D + lane + 32 * i) * fb;
+                    M = Mn;
+                }
+                const float vsc = F8 ? __ldg(p.v_scale + hq / p.group) : 1.f;
+                const float inv = Sum > 0.f ? vsc / Sum : 0.f;
+#pragma unroll
+                for (int i = 0; i < D / 32; ++i)
+                    store_out(p.out, row * D + lane + 32 * i, Acc[i] * inv, p.out_dtype);
+            }
+        }
     }
     while (it.valid) {
         const Segment sg = it.current();
@@ -980,77 +1008,11 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
             if (fits) write_record<D, NT, F8>(p, si.bg + si.u, tig, grp, acc, m, l);
             continue;
         }
-        if (si.nseg == 1) {
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int j = 0; j < 2; ++j) {
-                    const int h = nt * 8 + 2 * tig + j;
-                    if (h >= si.gv) continue;
-                    const float inv = l[nt][j] > 0.f ? vsc / l[nt][j] : 0.f;
-                    const size_t orow = ((size_t)si.b * p.num_q_heads + si.hq0 + h) * D;
-#pragma unroll
-                    for (int dt = 0; dt < C::KS; ++dt) {
-                        store_out(p.out, orow + dcol<F8>(dt, grp, 0), acc[dt][nt][j] * inv,
-                                  p.out_dtype);
-                        store_out(p.out, orow + dcol<F8>(dt, grp, 1), acc[dt][nt][j + 2] * inv,
-                                  p.out_dtype);
-                    }
-                }
-            continue;
-        }
-        // Parts of the group: its static units' records bg + u_first + k
-        // (k < n_static), then its tail's record dyn_rec_base + bg.
-        auto rec_of = [&](int k) -> size_t {
-            return k < si.n_static ? si.bg + (size_t)(si.u_first + k)
-                                   : (size_t)p.dyn_rec_base + si.bg;
-        };
-        const int own = si.dyn ? si.n_static : (int)(si.u - si.u_first);
-        if (rec_of(si.n_static > 0 ? si.n_static - 1 : 0) >= (size_t)p.rec_cap ||
-            rec_of(si.nseg - 1) >= (size_t)p.rec_cap) {
-            if (lane == 0) raise_error(p.err, PKV_DEVERR_BAD_SEQ_LEN);
-            continue;
-        }
-        // Arrive first.  Only a part that is not the last of its group to
-        // finish publishes its partial result (record, then a ready flag); the
-        // last one keeps its own in registers and merges the others'.  (The
-        // tails are taken dynamically, so no part can know in advance which
-        // one finishes last.)
-        unsigned arrived = 0;
-        if (lane == 0) arrived = atomicAdd(p.counters + si.bg, 1u);
-        arrived = __shfl_sync(FULL_MASK, arrived, 0);
-        if (arrived != (unsigned)(si.nseg - 1)) {
-            write_record<D, NT, F8>(p, rec_of(own), tig, grp, acc, m, l);
-            __threadfence();
-            __syncwarp();
-            if (lane == 0) atomicExch(p.ready + rec_of(own), 1u);
-            continue;
-        }
-
-        // Last part: wait (bounded) until every other part's record is out.
-        int ok = 1;
-        if (lane == 0) {
-            const uint64_t t0 = global_timer_ns();
-            for (int k = 0; k < si.nseg && ok; ++k) {
-                // (the test-only fault waits for the merger's own flag too,
-                // which nothing sets)
-                if (k == own && p.fault_mode != kFaultMergeFlag) continue;
-                volatile unsigned* f = p.ready + rec_of(k);
-                for (uint32_t it = 0; *f == 0u; ++it) {
-                    if ((it & 63u) == 63u && global_timer_ns() - t0 > p.wait_ns) {
-                        ok = 0;
-                        break;
-                    }
-                }
-            }
-            if (!ok) raise_error(p.err, PKV_DEVERR_TIMEOUT);
-        }
-        ok = __shfl_sync(FULL_MASK, ok, 0);
-        if (!ok) continue;
-        __threadfence();
-        // Online merge, records in order: M = max m, S = sum 2^(m-M) l,
-        // A = sum 2^(m-M) acc, out = A / S.  The other records are fetched two
-        // at a time with every load of the pair in flight before any math.
+        // Splits of the shared prefix pass whose records fold into this
+        // request's output (prefix groups only).
+        const int n_pfx =
+            sg.cur.t0 > 0 ? prefix_num_splits(prefix_tokens_of(p, si.b), p.pfx_splits) : 0;
+        // The row state: this part's own, then everything merged into it.
         float Mc[NT][2], Sc[NT][2], A[C::KS][NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
@@ -1065,23 +1027,93 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) A[dt][nt][i] = acc[dt][nt][i];
-        for (int k0 = 0; k0 < si.nseg; k0 += 2) {
+        // Parts of the group: its static units' records bg + u_first + k
+        // (k < n_static), then its tail's record dyn_rec_base + bg.
+        auto rec_of = [&](int k) -> size_t {
+            return k < si.n_static ? si.bg + (size_t)(si.u_first + k)
+                                   : (size_t)p.dyn_rec_base + si.bg;
+        };
+        const int own = si.dyn ? si.n_static : (int)(si.u - si.u_first);
+        if (si.nseg > 1) {
+            if (rec_of(si.n_static > 0 ? si.n_static - 1 : 0) >= (size_t)p.rec_cap ||
+                rec_of(si.nseg - 1) >= (size_t)p.rec_cap) {
+                if (lane == 0) raise_error(p.err, PKV_DEVERR_BAD_SEQ_LEN);
+                continue;
+            }
+            // Arrive first.  Only a part that is not the last of its group to
+            // finish publishes its partial result (record, then a ready flag);
+            // the last one keeps its own in registers and merges the others'.
+            // (The tails are taken dynamically, so no part can know in advance
+            // which one finishes last.)
+            unsigned arrived = 0;
+            if (lane == 0) arrived = atomicAdd(p.counters + si.bg, 1u);
+            arrived = __shfl_sync(FULL_MASK, arrived, 0);
+            if (arrived != (unsigned)(si.nseg - 1)) {
+                write_record<D, NT, F8>(p, rec_of(own), tig, grp, acc, m, l);
+                __threadfence();
+                __syncwarp();
+                if (lane == 0) atomicExch(p.ready + rec_of(own), 1u);
+                continue;
+            }
+
+            // Last part: wait (bounded) until every other part's record is out.
+            int ok = 1;
+            if (lane == 0) {
+                const uint64_t t0 = global_timer_ns();
+                for (int k = 0; k < si.nseg && ok; ++k) {
+                    // (the test-only fault waits for the merger's own flag too,
+                    // which nothing sets)
+                    if (k == own && p.fault_mode != kFaultMergeFlag) continue;
+                    volatile unsigned* f = p.ready + rec_of(k);
+                    for (uint32_t it = 0; *f == 0u; ++it) {
+                        if ((it & 63u) == 63u && global_timer_ns() - t0 > p.wait_ns) {
+                            ok = 0;
+                            break;
+                        }
+                    }
+                }
+                if (!ok) raise_error(p.err, PKV_DEVERR_TIMEOUT);
+            }
+            ok = __shfl_sync(FULL_MASK, ok, 0);
+            if (!ok) continue;
+            __threadfence();
+        }
+        // Online merge of the other parts' records, then of the shared pass's
+        // splits, in order: M = max m, S = sum 2^(m-M) l, A = sum 2^(m-M) acc,
+        // out = A / S.  Records are fetched two at a time with every load of
+        // the pair in flight before any math.
+        const int n_other = (si.nseg > 1 ? si.nseg : 1) + n_pfx;  // slot 0.. with own skipped
+        for (int k0 = 0; k0 < n_other; k0 += 2) {
             float mr[2][NT][2], lr[2][NT][2], ar[2][C::KS][NT][4];
             bool use[2];
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
                 const int kk = k0 + k;
-                use[k] = kk < si.nseg && kk != own;
+                const int n_own = si.nseg > 1 ? si.nseg : 1;
+                use[k] = kk < n_other && (kk >= n_own || (si.nseg > 1 && kk != own));
                 if (!use[k]) continue;
-                const size_t rk = rec_of(kk);
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
-                        const size_t rr = rk * GP + nt * 8 + 2 * tig + j;
-                        mr[k][nt][j] = ld_cg(p.rec_ml + rr * 2);
-                        lr[k][nt][j] = ld_cg(p.rec_ml + rr * 2 + 1);
-                        const float* ra = p.rec_acc + rr * D;
+                        const int h = nt * 8 + 2 * tig + j;
+                        const float* mlp;
+                        const float* ra;
+                        if (kk < n_own) {
+                            const size_t rr = rec_of(kk) * GP + h;
+                            mlp = p.rec_ml + rr * 2;
+                            ra = p.rec_acc + rr * D;
+                        } else {
+                            // split kk - n_own of the shared pass; padding
+                            // heads of the group read row hq0 instead (unused)
+                            const size_t rr =
+                                ((size_t)(kk - n_own) * p.num_seqs + si.b) * p.num_q_heads +
+                                si.hq0 + (h < si.gv ? h : 0);
+                            mlp = p.pfx_ml + rr * 2;
+                            ra = p.pfx_acc + rr * D;
+                        }
+                        mr[k][nt][j] = ld_cg(mlp);
+                        lr[k][nt][j] = ld_cg(mlp + 1);
 #pragma unroll
                         for (int dt = 0; dt < C::KS; ++dt) {
                             ar[k][dt][nt][j] = ld_cg(ra + dcol<F8>(dt, grp, 0));
@@ -1124,10 +1156,12 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
                               p.out_dtype);
                 }
             }
-        __syncwarp();
-        if (lane == 0) {  // ready for the next call
-            for (int k = 0; k < si.nseg; ++k) p.ready[rec_of(k)] = 0u;
-            p.counters[si.bg] = 0u;
+        if (si.nseg > 1) {
+            __syncwarp();
+            if (lane == 0) {  // ready for the next call
+                for (int k = 0; k < si.nseg; ++k) p.ready[rec_of(k)] = 0u;
+                p.counters[si.bg] = 0u;
+            }
         }
     }
 }
