@@ -19,7 +19,6 @@ namespace {
 constexpr int kMaxDevices = 64;
 constexpr int kChunkTokens = 32;  // tokens per decode pipeline stage
 constexpr int kMaxCtasPerSm = 4;  // cap of resident decode CTAs per SM
-constexpr int kTailChunks = 2;    // chunks of each group handed out dynamically
 
 bool is_pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
@@ -120,8 +119,7 @@ bool make_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_
         }
     }
     pl.units_max = units;
-    pl.dyn_base = pl.n_bg_max + units;
-    pl.records = pl.dyn_base + pl.n_bg_max;  // + one dynamic-tail record per group
+    pl.records = pl.n_bg_max + units;
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
     const size_t acc_bytes = pl.records * pl.rec_gp * head_dim * sizeof(float);
     const size_t ml_bytes = pl.records * pl.rec_gp * 2 * sizeof(float);
@@ -131,11 +129,11 @@ bool make_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_
     pl.off_extra = pl.off_meta + up(meta_bytes);
     pl.rec_bytes = pl.off_extra + up(extra_bytes);
     // smallest B with sync region(B) + records <= B, a flag for every record
-    // and a counter for every group beside the ticket words
+    // and a counter for every group
     size_t b = up(pl.rec_bytes + 2 * pl.records * sizeof(uint32_t));
     while (sync_region_bytes(b) + pl.rec_bytes > b ||
            sync_counters_offset(b) < pl.records * sizeof(uint32_t) ||
-           sync_tickets_offset(b) - sync_counters_offset(b) < pl.n_bg_max * sizeof(uint32_t))
+           sync_region_bytes(b) - sync_counters_offset(b) < pl.n_bg_max * sizeof(uint32_t))
         b += 256;
     pl.bytes = b;
     *plan = pl;
@@ -350,13 +348,10 @@ pkv_status decode_entry(const void* q, const void* k_cache, const void* v_cache,
     const size_t cnt_region = sync_region_bytes(workspace_bytes);
     if (cnt_region + pl.rec_bytes > workspace_bytes ||
         sync_counters_offset(workspace_bytes) < pl.records * sizeof(uint32_t) ||
-        sync_tickets_offset(workspace_bytes) - sync_counters_offset(workspace_bytes) <
-            pl.n_bg_max * sizeof(uint32_t))
+        cnt_region - sync_counters_offset(workspace_bytes) < pl.n_bg_max * sizeof(uint32_t))
         return PKV_ERR_WORKSPACE;
     p.ready = reinterpret_cast<unsigned*>(ws);
     p.counters = reinterpret_cast<unsigned*>(ws + sync_counters_offset(workspace_bytes));
-    p.tickets = reinterpret_cast<unsigned*>(ws + sync_tickets_offset(workspace_bytes));
-    p.dyn_rec_base = (long long)pl.dyn_base;
     p.rec_acc = reinterpret_cast<float*>(ws + cnt_region);
     p.rec_ml = reinterpret_cast<float*>(ws + cnt_region + pl.off_ml);
     p.meta = reinterpret_cast<int32_t*>(ws + cnt_region + pl.off_meta);
@@ -380,8 +375,6 @@ pkv_status decode_entry(const void* q, const void* k_cache, const void* v_cache,
     // the shared pass's splits (a few records per row).
     p.defer_merge = (mma && partition_size > 0) ? 1 : 0;
     p.row_copy = (mma && block_size < 8) ? 1 : 0;
-    // dynamic tails: the tensor-core path with the automatic split
-    p.tail_chunks = (mma && !p.defer_merge) ? kTailChunks : 0;
     p.rec_cap = (long long)pl.records;
     p.out_dtype = out_dtype;
     p.scale_log2 = scale * 1.4426950408889634f;

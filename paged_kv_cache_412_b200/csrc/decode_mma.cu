@@ -118,10 +118,10 @@ struct Smem {
     static constexpr int DUMP_BYTES = C::DUMP_BYTES;
     static constexpr int OFF_DUMP = C::NSTAGE * C::STAGE_BYTES;
     static constexpr int OFF_BAR = OFF_DUMP + NSLOT * DUMP_BYTES;
-    // full/empty per stage, dfull/dempty per dump slot, full/empty per tail-queue slot
-    static constexpr int OFF_META = OFF_BAR + (2 * C::NSTAGE + 2 * NSLOT + 2 * kTailQueue) * 8;
-    // ntok/bad per stage, tail-queue tickets
-    static constexpr int OFF_CTRL = OFF_META + (2 * C::NSTAGE + kTailQueue) * 4;
+    // full/empty per stage, dfull/dempty per dump slot
+    static constexpr int OFF_META = OFF_BAR + (2 * C::NSTAGE + 2 * NSLOT) * 8;
+    // ntok/bad per stage
+    static constexpr int OFF_CTRL = OFF_META + 2 * C::NSTAGE * 4;
     static constexpr int BYTES = OFF_CTRL + 16 + 1024;   // + alignment slack
     static_assert(BYTES <= 227 * 1024, "within the opt-in shared memory of one CTA");
 };
@@ -389,34 +389,19 @@ struct Producer {
 
 // Per-segment facts every role derives the same way.
 struct SegInfo {
-    long long u, u_first, u_last;  // the group's static units u_first .. u_last
-    int n_static;                  // number of them (0: the group is all tail)
-    int nseg;                      // parts of the group: static units + its tail
-    bool dyn;                      // this segment is the group's dynamic tail
+    long long u, u_first, u_last;  // the group's units u_first .. u_last
+    int nseg;                      // parts of the group (units)
     int hq0, gv, b, kvh;
     size_t bg;
 };
 
-// need_parts: also work out the group's static units for a tail segment
-// (a warp-cooperative scan; only the epilogue needs them).
 template <int GP>
-__device__ __forceinline__ SegInfo seg_info(const DecodeParams& p, const Segment& sg, long long W,
-                                            bool need_parts = false, int lane = 0) {
+__device__ __forceinline__ SegInfo seg_info(const DecodeParams& p, const Segment& sg, long long W) {
     SegInfo si;
     si.u = sg.u;
-    si.dyn = sg.dyn_t >= 0;
-    const int n = sg.cur.L - sg.cur.t0;
-    const int nch_s = list_chunks<kCH>(p, n);  // the group's chunks in the static list
-    long long gs = sg.gstart;
-    if (si.dyn) gs = (need_parts && nch_s > 0) ? static_start<kCH>(p, sg.cur.b, sg.cur.hg, nch_s, lane) : 0;
-    si.n_static = 0;
-    si.u_first = si.u_last = 0;
-    if (nch_s > 0) {
-        si.u_first = gs / W;
-        si.u_last = (gs + nch_s - 1) / W;
-        si.n_static = (int)(si.u_last - si.u_first + 1);
-    }
-    si.nseg = si.n_static + ((p.tail_chunks > 0 && chunks_of<kCH>(n) > 0) ? 1 : 0);
+    si.u_first = sg.gstart / W;
+    si.u_last = (sg.gstart + sg.cur.nch - 1) / W;
+    si.nseg = (int)(si.u_last - si.u_first + 1);
     const int kvh = sg.cur.hg / p.num_sub, sub = sg.cur.hg % p.num_sub;
     si.hq0 = kvh * p.group + sub * GP;
     si.gv = min(GP, p.group - sub * GP);
@@ -540,7 +525,7 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
             const int ntok = st_ntok[stage];
             const unsigned bad = st_bad[stage];
             unsigned char* sk = smem + stage * C::STAGE_BYTES;
-            unsigned char* sv = sk + C::KV_BYTES;
+            unsigned char* sv = sk + (RC ? C::RC_KV_BYTES : C::KV_BYTES);
             const bool whole = ntok == kCH && bad == 0;
 
             if (!F8 && !RC && !have_q) {
@@ -923,7 +908,7 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
     while (it.valid) {
         const Segment sg = it.current();
         it.advance(p, lane);
-        const SegInfo si = seg_info<GP>(p, sg, it.W, true, lane);
+        const SegInfo si = seg_info<GP>(p, sg, it.W);
         const float vsc = F8 ? __ldg(p.v_scale + si.kvh) : 1.f;  // V dequantisation scale
         // the segment's state: one consumer's, or the merge of NCONS consumers'
         float acc[C::KS][NT][4], m[NT][2], l[NT][2];
@@ -1027,24 +1012,17 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int i = 0; i < 4; ++i) A[dt][nt][i] = acc[dt][nt][i];
-        // Parts of the group: its static units' records bg + u_first + k
-        // (k < n_static), then its tail's record dyn_rec_base + bg.
-        auto rec_of = [&](int k) -> size_t {
-            return k < si.n_static ? si.bg + (size_t)(si.u_first + k)
-                                   : (size_t)p.dyn_rec_base + si.bg;
-        };
-        const int own = si.dyn ? si.n_static : (int)(si.u - si.u_first);
+        // Parts of the group: the records bg + u of its units u_first .. u_last.
+        auto rec_of = [&](int k) -> size_t { return si.bg + (size_t)(si.u_first + k); };
+        const int own = (int)(si.u - si.u_first);
         if (si.nseg > 1) {
-            if (rec_of(si.n_static > 0 ? si.n_static - 1 : 0) >= (size_t)p.rec_cap ||
-                rec_of(si.nseg - 1) >= (size_t)p.rec_cap) {
+            if (rec_of(si.nseg - 1) >= (size_t)p.rec_cap) {
                 if (lane == 0) raise_error(p.err, PKV_DEVERR_BAD_SEQ_LEN);
                 continue;
             }
             // Arrive first.  Only a part that is not the last of its group to
             // finish publishes its partial result (record, then a ready flag);
             // the last one keeps its own in registers and merges the others'.
-            // (The tails are taken dynamically, so no part can know in advance
-            // which one finishes last.)
             unsigned arrived = 0;
             if (lane == 0) arrived = atomicAdd(p.counters + si.bg, 1u);
             arrived = __shfl_sync(FULL_MASK, arrived, 0);
@@ -1166,14 +1144,12 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
     }
 }
 
-// Chunk count of the static list, computed by one warp (same value in every
-// warp and CTA), and the number of dynamic tails (one per non-empty request and
-// head group when they are on).  *L_first / *T_first receive this lane's
-// length of request `lane` and the first token of its pass (or 0).
+// Total chunk count, computed by one warp (same value in every warp and CTA).
+// *L_first / *T_first receive this lane's length of request `lane` and the
+// first token of its pass (or 0).
 __device__ __forceinline__ long long total_chunks_warp(const DecodeParams& p, int lane, bool flag,
-                                                       int* L_first, int* T_first,
-                                                       long long* n_tails) {
-    long long t = 0, nonempty = 0;
+                                                       int* L_first, int* T_first) {
+    long long t = 0;
     *L_first = 0;
     *T_first = 0;
     for (int b = lane; b < p.num_seqs; b += 32) {
@@ -1183,15 +1159,10 @@ __device__ __forceinline__ long long total_chunks_warp(const DecodeParams& p, in
             *L_first = L;
             *T_first = T;
         }
-        t += list_chunks<kCH>(p, L - T);
-        nonempty += chunks_of<kCH>(L - T) > 0 ? 1 : 0;
+        t += chunks_of<kCH>(L - T);
     }
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        t += __shfl_xor_sync(FULL_MASK, t, off);
-        nonempty += __shfl_xor_sync(FULL_MASK, nonempty, off);
-    }
-    *n_tails = p.tail_chunks > 0 ? nonempty * p.num_hg : 0;
+    for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(FULL_MASK, t, off);
     return t * p.num_hg;
 }
 
@@ -1208,12 +1179,8 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
     uint64_t* empty = full + C::NSTAGE;
     uint64_t* dfull = empty + C::NSTAGE;
     uint64_t* dempty = dfull + S::NSLOT;
-    TailQueue tq;
-    tq.full = dempty + S::NSLOT;
-    tq.empty = tq.full + kTailQueue;
     int* st_ntok = reinterpret_cast<int*>(smem + S::OFF_META);
     unsigned* st_bad = reinterpret_cast<unsigned*>(st_ntok + C::NSTAGE);
-    tq.val = reinterpret_cast<int*>(st_bad + C::NSTAGE);
     volatile int* ctrl = reinterpret_cast<volatile int*>(smem + S::OFF_CTRL);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -1226,11 +1193,6 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
         for (int s = 0; s < S::NSLOT; ++s) {
             mbar_init(&dfull[s], 1);
             mbar_init(&dempty[s], 1);
-        }
-        // tail tickets: warp 0 publishes, every other warp reads
-        for (int s = 0; s < kTailQueue; ++s) {
-            mbar_init(&tq.full[s], 1);
-            mbar_init(&tq.empty[s], C::THREADS / 32 - 1);
         }
         fence_mbar_init();
         prefetch_tensormap(&tmk);
@@ -1249,7 +1211,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
     int spec_b = -1, spec_j = -1, spec_tab = -1;
     if (warp < C::NPROD && !p.prefix_of && p.fixed_units == 0 && p.max_len_hint > 0) {
         const int Lg = min(p.max_len_hint, p.max_blocks * p.block_size);
-        const long long nchg = list_chunks<kCH>(p, Lg);  // static chunks per group
+        const long long nchg = chunks_of<kCH>(Lg);
         const long long totg = nchg * p.num_hg * p.num_seqs;
         const long long Wg = (totg + gridDim.x - 1) / gridDim.x;
         const long long s0 = (long long)blockIdx.x * Wg;
@@ -1262,10 +1224,9 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
         }
     }
     int L_first = 0, T_first = 0;
-    long long n_tails = 0;
     const long long total =
-        total_chunks_warp(p, lane, blockIdx.x == 0 && warp == 0, &L_first, &T_first, &n_tails);
-    if (total == 0 && n_tails == 0) {
+        total_chunks_warp(p, lane, blockIdx.x == 0 && warp == 0, &L_first, &T_first);
+    if (total == 0) {
         if (warp == C::NPROD + C::NCONS) {
             SegIter<kCH> none;
             none.valid = false;
@@ -1276,9 +1237,6 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
     long long W = p.fixed_units > 0 ? p.fixed_units : (total + gridDim.x - 1) / gridDim.x;
     if (W < 1) W = 1;
     SegIter<kCH> it;
-    it.n_tails = n_tails;
-    it.q = tq;
-    it.fetcher = warp == 0;
     it.init(p, total, W, lane, L_first, T_first);
 
     // warps: producers | consumers | epilogue

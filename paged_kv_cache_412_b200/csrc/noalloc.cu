@@ -82,13 +82,12 @@ extern "C" pkv_status pkv_paged_attention_decode_noalloc(
         const pkv_status s = scratch_address(st, &ws);
         if (s != PKV_OK) return s;
         // The array keeps the previous call's contents; the record-ready
-        // flags, arrival counters and ticket words this call can use must
-        // start at zero, so clear them (no allocation: memset nodes).
+        // flags and arrival counters this call can use must start at zero, so
+        // clear them (no allocation: memset nodes).
         unsigned char* base = static_cast<unsigned char*>(ws);
         if (cudaMemsetAsync(base, 0, pl.records * sizeof(uint32_t), st) != cudaSuccess ||
             cudaMemsetAsync(base + sync_counters_offset(kScratchBytes), 0,
-                            pl.n_bg_max * sizeof(uint32_t), st) != cudaSuccess ||
-            cudaMemsetAsync(base + sync_tickets_offset(kScratchBytes), 0, 8, st) != cudaSuccess)
+                            pl.n_bg_max * sizeof(uint32_t), st) != cudaSuccess)
             return PKV_ERR_CUDA;
     }
     return pkv_paged_attention_decode(q, k_cache, v_cache, block_tables, seq_lens, block_size,

@@ -36,7 +36,6 @@ struct DecodePlan {
     int rec_gp;        // floats per record row = largest query-head group of either path
     size_t n_bg_max;   // (request, head group) pairs, largest over the paths
     size_t units_max;  // upper bound of split units
-    size_t dyn_base;   // first record of the dynamic tails (one per group after it)
     size_t records;    // partial-result records
     size_t rec_bytes;  // records + their (max, sum) pairs + per-group meta
     size_t off_ml, off_meta;  // offsets inside the record region
@@ -47,16 +46,12 @@ struct DecodePlan {
 // Bytes at the start of a B-byte workspace reserved for the merge's
 // synchronisation words, all of which return to zero at the end of every call:
 // one ready flag per partial record in its first half, per-group arrival
-// counters in its second half, and the two ticket words of the dynamic tails
-// in its last 8 bytes.
+// counters in its second half.
 inline size_t sync_region_bytes(size_t workspace_bytes) {
     return (workspace_bytes / 128 + 255) / 256 * 256;
 }
 inline size_t sync_counters_offset(size_t workspace_bytes) {
     return sync_region_bytes(workspace_bytes) / 2;
-}
-inline size_t sync_tickets_offset(size_t workspace_bytes) {
-    return sync_region_bytes(workspace_bytes) - 8;
 }
 
 // Fill a plan for these sizes on the current device (false if invalid).
@@ -88,14 +83,7 @@ struct DecodeParams {
                       // a separate merge kernel combines them
     int row_copy;     // 1: blocks of 2 or 4 rows -- one bulk copy per (block, K or V)
                       // into a skewed stage layout instead of TMA boxes
-    // Dynamic tails (automatic split only; 0 = off): the last tail_chunks
-    // chunks of every (request, head group) are left out of the static split
-    // and handed out one group at a time, by an atomic ticket, to the CTAs that
-    // finish their static unit first.  Their records start at dyn_rec_base + bg.
-    int tail_chunks;
-    long long dyn_rec_base;
     unsigned* counters;  // [num_seqs * num_hg] arrivals per split group (zero between calls)
-    unsigned* tickets;   // [2]: next tail ticket, CTAs done fetching (zero between calls)
     long long rec_cap;  // records the workspace holds
     int out_dtype;
     float scale_log2;  // softmax scale * log2(e)
