@@ -238,9 +238,10 @@ def paged_attention_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torc
         max_seq_len = max_blocks * bs
     if out is None:
         out = torch.empty((B, Hq, d), dtype=out_dtype or q.dtype, device=dev)
-    need = decode_workspace_bytes(B, Hq, Hkv, d, bs, max_seq_len, partition_size)
     with torch.cuda.device(dev):
-        ws = workspace if workspace is not None else _workspace(dev, need)
+        # a caller's workspace is checked by the library itself
+        ws = workspace if workspace is not None else _workspace(
+            dev, decode_workspace_bytes(B, Hq, Hkv, d, bs, max_seq_len, partition_size))
         st = _get_lib().pkv_paged_attention_decode(
             _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables), _ptr(seq_lens),
             bs, float(scale), _ptr(out), B, Hq, Hkv, d, max_blocks, NB, int(max_seq_len),
