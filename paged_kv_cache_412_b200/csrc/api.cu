@@ -368,12 +368,11 @@ pkv_status decode_entry(const void* q, const void* k_cache, const void* v_cache,
     p.num_blocks = num_blocks;
     p.max_len_hint = max_seq_len;
     p.fixed_units = partition_size > 0 ? std::max(1, partition_size / (mma ? 64 : 32)) : 0;
-    // Fixed partitions on the tensor-core path: merge in a separate kernel,
-    // so a group split into many parts is combined in parallel instead of by
-    // one warp of the decode kernel (which would stall that warp's CTA).
-    // Prefix groups merge in-kernel: a split group's last part also folds in
-    // the shared pass's splits (a few records per row).
-    p.defer_merge = (mma && partition_size > 0) ? 1 : 0;
+    // Fixed partitions and prefix groups on the tensor-core path: merge in a
+    // separate kernel, so a group split into many parts (or folded with many
+    // splits of a shared prefix) is combined in parallel instead of by one
+    // warp of the decode kernel (which would stall that warp's CTA).
+    p.defer_merge = (mma && (partition_size > 0 || use_prefix)) ? 1 : 0;
     p.row_copy = (mma && block_size < 8) ? 1 : 0;
     p.rec_cap = (long long)pl.records;
     p.out_dtype = out_dtype;

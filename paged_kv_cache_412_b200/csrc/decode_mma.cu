@@ -870,40 +870,12 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
     Ring dring;
     griddep_wait();  // `out` and the workspace may be in use by the previous kernel
     // Requests with no token at all: all-zero rows (softmax of an empty set).
-    // A request whose shared prefix covers all of it has no token of its own
-    // pass either: unless a separate merge kernel follows, its rows are the
-    // merge of the shared pass's splits alone.
+    // (A request whose shared prefix covers all of it has no token of its own
+    // pass either; the merge kernel writes it from the shared pass's results.)
     for (int b = blockIdx.x; b < p.num_seqs; b += gridDim.x) {
-        const int L = clamp_len(p, b, false);
-        if (L == 0) {
-            for (int i = lane; i < p.num_q_heads * D; i += 32)
-                store_out(p.out, (size_t)b * p.num_q_heads * D + i, 0.f, p.out_dtype);
-        } else if (!p.defer_merge && seq_begin(p, b, L) == L) {
-            const int ns = prefix_num_splits(prefix_tokens_of(p, b), p.pfx_splits);
-            for (int hq = 0; hq < p.num_q_heads; ++hq) {
-                const size_t row = (size_t)b * p.num_q_heads + hq;
-                float M = -INFINITY, Sum = 0.f, Acc[D / 32];
-#pragma unroll
-                for (int i = 0; i < D / 32; ++i) Acc[i] = 0.f;
-                for (int sp = 0; sp < ns; ++sp) {
-                    const size_t rr = (size_t)sp * p.num_seqs * p.num_q_heads + row;
-                    const float ms = ld_cg(p.pfx_ml + rr * 2), ls = ld_cg(p.pfx_ml + rr * 2 + 1);
-                    const float Mn = fmaxf(M, ms);
-                    const float ref = Mn == -INFINITY ? 0.f : Mn;
-                    const float fa = exp2f(M - ref), fb = exp2f(ms - ref);
-                    Sum = Sum * fa + ls * fb;
-#pragma unroll
-                    for (int i = 0; i < D / 32; ++i)
-                        Acc[i] = Acc[i] * fa + ld_cg(p.pfx_acc + rr * D + lane + 32 * i) * fb;
-                    M = Mn;
-                }
-                const float vsc = F8 ? __ldg(p.v_scale + hq / p.group) : 1.f;
-                const float inv = Sum > 0.f ? vsc / Sum : 0.f;
-#pragma unroll
-                for (int i = 0; i < D / 32; ++i)
-                    store_out(p.out, row * D + lane + 32 * i, Acc[i] * inv, p.out_dtype);
-            }
-        }
+        if (clamp_len(p, b, false) != 0) continue;
+        for (int i = lane; i < p.num_q_heads * D; i += 32)
+            store_out(p.out, (size_t)b * p.num_q_heads * D + i, 0.f, p.out_dtype);
     }
     while (it.valid) {
         const Segment sg = it.current();
@@ -993,10 +965,6 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
             if (fits) write_record<D, NT, F8>(p, si.bg + si.u, tig, grp, acc, m, l);
             continue;
         }
-        // Splits of the shared prefix pass whose records fold into this
-        // request's output (prefix groups only).
-        const int n_pfx =
-            sg.cur.t0 > 0 ? prefix_num_splits(prefix_tokens_of(p, si.b), p.pfx_splits) : 0;
         // The row state: this part's own, then everything merged into it.
         float Mc[NT][2], Sc[NT][2], A[C::KS][NT][4];
 #pragma unroll
@@ -1056,40 +1024,25 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
             if (!ok) continue;
             __threadfence();
         }
-        // Online merge of the other parts' records, then of the shared pass's
-        // splits, in order: M = max m, S = sum 2^(m-M) l, A = sum 2^(m-M) acc,
-        // out = A / S.  Records are fetched two at a time with every load of
-        // the pair in flight before any math.
-        const int n_other = (si.nseg > 1 ? si.nseg : 1) + n_pfx;  // slot 0.. with own skipped
-        for (int k0 = 0; k0 < n_other; k0 += 2) {
+        // Online merge of the other parts' records, in order: M = max m,
+        // S = sum 2^(m-M) l, A = sum 2^(m-M) acc, out = A / S.  Records are
+        // fetched two at a time with every load of the pair in flight before
+        // any math.
+        for (int k0 = 0; si.nseg > 1 && k0 < si.nseg; k0 += 2) {
             float mr[2][NT][2], lr[2][NT][2], ar[2][C::KS][NT][4];
             bool use[2];
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
                 const int kk = k0 + k;
-                const int n_own = si.nseg > 1 ? si.nseg : 1;
-                use[k] = kk < n_other && (kk >= n_own || (si.nseg > 1 && kk != own));
+                use[k] = kk < si.nseg && kk != own;
                 if (!use[k]) continue;
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                     for (int j = 0; j < 2; ++j) {
-                        const int h = nt * 8 + 2 * tig + j;
-                        const float* mlp;
-                        const float* ra;
-                        if (kk < n_own) {
-                            const size_t rr = rec_of(kk) * GP + h;
-                            mlp = p.rec_ml + rr * 2;
-                            ra = p.rec_acc + rr * D;
-                        } else {
-                            // split kk - n_own of the shared pass; padding
-                            // heads of the group read row hq0 instead (unused)
-                            const size_t rr =
-                                ((size_t)(kk - n_own) * p.num_seqs + si.b) * p.num_q_heads +
-                                si.hq0 + (h < si.gv ? h : 0);
-                            mlp = p.pfx_ml + rr * 2;
-                            ra = p.pfx_acc + rr * D;
-                        }
+                        const size_t rr = rec_of(kk) * GP + nt * 8 + 2 * tig + j;
+                        const float* mlp = p.rec_ml + rr * 2;
+                        const float* ra = p.rec_acc + rr * D;
                         mr[k][nt][j] = ld_cg(mlp);
                         lr[k][nt][j] = ld_cg(mlp + 1);
 #pragma unroll
