@@ -87,10 +87,12 @@ struct MmaCfg {
     // (two on each of two SM sub-partitions) overlap them; the 16-head
     // configuration keeps four (its consumers need all the registers).
     static constexpr int NCONS = F8 ? (NT == 1 ? 6 : 4) : 1;
-    // producer warps: a TMA issue holds the issuing warp ~0.1 us, and one fp8
-    // producer per SM cannot issue fast enough; two take alternate chunks
-    // (stage n % NSTAGE belongs to producer n % NPROD).
-    static constexpr int NPROD = F8 ? 2 : 1;
+    // producer warps: a TMA issue holds the issuing warp ~0.11 us, so one
+    // warp issues at most ~9 boxes per us however its lanes share them.  An
+    // fp8 chunk is 8 boxes of 2 KB; four producers take chunks in turn (stage
+    // n % NSTAGE belongs to producer n % NPROD), enough to keep 12 stages in
+    // flight.  The 16-head configuration keeps two (registers).
+    static constexpr int NPROD = F8 ? (NT == 1 ? 4 : 2) : 1;
     static constexpr int THREADS = 32 * (NPROD + NCONS + 1);  // + the epilogue
     // consumer -> epilogue hand-off: per lane, the accumulators and (m, l)
     static constexpr int DUMP_BYTES = (KS * NT * 4 + NT * 4) * 32 * 4;
@@ -98,7 +100,7 @@ struct MmaCfg {
     // slots (up to 24), a multiple of NCONS and NPROD: 192 KB of codes in
     // flight per SM at head_dim 128, as much as the two bf16 CTAs of an SM keep
     static constexpr int F8_RING = 227 * 1024 - NCONS * DUMP_BYTES - 4096;
-    static constexpr int STAGE_STEP = F8 ? (NCONS % 2 == 0 ? NCONS : 2 * NCONS) : 1;  // lcm(NCONS, 2)
+    static constexpr int STAGE_STEP = F8 ? (NCONS == 6 ? 12 : 4) : 1;  // lcm(NCONS, NPROD)
     static constexpr int NSTAGE = F8 ? cmin(24, F8_RING / STAGE_BYTES) / STAGE_STEP * STAGE_STEP
                                      : cmax(2, cmin(8, kRingBudget / STAGE_BYTES));
     static_assert(NSTAGE % NPROD == 0 && NSTAGE % NCONS == 0 && NSTAGE >= 2,
@@ -167,6 +169,17 @@ __device__ __forceinline__ int rc_block_bytes(int block_size) {
 __device__ __forceinline__ int rc_token(int mt, int i, int log2_bs) {
     const int bs = 1 << log2_bs;
     return bs * (16 * (mt >> log2_bs) + i) + (mt & (bs - 1));
+}
+
+// bf16 stages hold each block's rows as one TMA box of [half][rb rows][128 B]
+// (rb = min(block_size, 64), both 64-column halves of a 128-dim row in one
+// box), blocks one after another: byte offset of 64-column half `half` of
+// stage row t (t < 64).  The 128-byte swizzle is keyed on t % 8, since every
+// box starts on a 1 KB boundary.
+template <int NHALF>
+__device__ __forceinline__ int bf16_row_off(int t, int half, int log2_rb) {
+    const int rb = 1 << log2_rb;
+    return (t >> log2_rb) * (rb * NHALF * 128) + half * (rb * 128) + (t & (rb - 1)) * 128;
 }
 
 // ---- producer ------------------------------------------------------------------
@@ -330,14 +343,14 @@ struct Producer {
                         // bank conflicts
                         tma_load_2d(sk + srow * D, tmk, 0, grow, &full[stage], policy);
                         tma_load_2d(sv + srow * D, tmv, 0, grow, &full[stage], policy);
+                    } else if constexpr (C::NHALF == 2) {
+                        // one 3-D box per block holds both 64-column halves of
+                        // its rb rows ([half][row][128 B]): half the TMA issues
+                        tma_load_3d(sk + srow * 256, tmk, 0, grow, 0, &full[stage], policy);
+                        tma_load_3d(sv + srow * 256, tmv, 0, grow, 0, &full[stage], policy);
                     } else {
-#pragma unroll
-                        for (int h = 0; h < C::NHALF; ++h) {
-                            tma_load_2d(sk + h * C::HALF_BYTES + srow * 128, tmk, h * 64, grow,
-                                        &full[stage], policy);
-                            tma_load_2d(sv + h * C::HALF_BYTES + srow * 128, tmv, h * 64, grow,
-                                        &full[stage], policy);
-                        }
+                        tma_load_2d(sk + srow * 128, tmk, 0, grow, &full[stage], policy);
+                        tma_load_2d(sv + srow * 128, tmv, 0, grow, &full[stage], policy);
                     }
                 }
             }
@@ -443,6 +456,14 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
     Ring ring, dring;
     unsigned n_chunk = 0;  // fp8: chunks of the CTA so far
     bool waited = false;   // fp8: q is read from global memory
+    // bf16 stages: byte offsets of this lane's ldmatrix rows per token tile
+    const int log2_rb = min(p.log2_bs, 6);
+    int k_off[kMT], v_off[kMT];
+#pragma unroll
+    for (int mt = 0; mt < kMT; ++mt) {
+        k_off[mt] = bf16_row_off<C::NHALF>(mt * 16 + k_row, 0, log2_rb);
+        v_off[mt] = bf16_row_off<C::NHALF>(mt * 16 + v_row, 0, log2_rb);
+    }
 
     while (it.valid) {
         const Segment sg = it.current();
@@ -556,7 +577,7 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                     const int jrel = ((c * kCH + row) >> p.log2_bs) - ((c * kCH) >> p.log2_bs);
                     const bool valid = row < ntok && !((bad >> jrel) & 1u);
                     if (!valid)
-                        *reinterpret_cast<uint4*>(sv + (rest >> 3) * C::HALF_BYTES + row * 128 +
+                        *reinterpret_cast<uint4*>(sv + bf16_row_off<C::NHALF>(row, rest >> 3, log2_rb) +
                                                   (rest & 7) * 16) = make_uint4(0, 0, 0, 0);
                 }
                 __syncwarp();
@@ -614,7 +635,7 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
 #pragma unroll
                     for (int mt = 0; mt < kMT; ++mt) {
                         uint32_t a[4];
-                        ldsm_x4(skb + half * C::HALF_BYTES + (mt * 16 + k_row) * 128 + (chunk << 4), a);
+                        ldsm_x4(skb + k_off[mt] + half * (128 << log2_rb) + (chunk << 4), a);
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) mma_bf16(s[mt][nt], a, qb[nt][ks][0], qb[nt][ks][1]);
                     }
@@ -776,7 +797,7 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                         const int half = dt >> 2;
                         const int chunk = (2 * (dt & 3) + v_cx) ^ r8;
                         uint32_t a[4];
-                        ldsm_x4_t(svb + half * C::HALF_BYTES + (mt * 16 + v_row) * 128 + (chunk << 4), a);
+                        ldsm_x4_t(svb + v_off[mt] + half * (128 << log2_rb) + (chunk << 4), a);
 #pragma unroll
                         for (int nt = 0; nt < NT; ++nt) {
                             mma_bf16(acc[dt][nt], a, bh[nt][0], bh[nt][1]);
@@ -1382,8 +1403,8 @@ pkv_status launch_impl(const DecodeParams& p, cudaStream_t stream, int* grid_out
     const long long rows = (long long)p.num_blocks * p.num_kv_heads * p.block_size;
     const int box_rows = std::min(p.block_size, kCH);
     CUtensorMap tmk, tmv;
-    if (!encode_cache_map(&tmk, p.k_cache, rows, D, box_rows, F8) ||
-        !encode_cache_map(&tmv, p.v_cache, rows, D, box_rows, F8))
+    if (!encode_cache_map(&tmk, p.k_cache, rows, D, box_rows, F8, !F8 && !RC) ||
+        !encode_cache_map(&tmv, p.v_cache, rows, D, box_rows, F8, !F8 && !RC))
         return PKV_ERR_CUDA;
     const int grid = di->num_sms * std::min(occupancy[di->device], 4);
 
@@ -1431,7 +1452,7 @@ struct MapCacheEntry {
     const void* base = nullptr;
     long long rows = 0;
     int head_dim = 0, box_rows = 0;
-    bool fp8 = false;
+    bool fp8 = false, both_halves = false;
     CUtensorMap map;
 };
 constexpr int kMapCache = 16;
@@ -1443,29 +1464,33 @@ int g_map_next = 0;
 
 // 2-D view of a cache: rows = num_blocks*Hkv*block_size, columns = head_dim
 // bf16; boxes of 64 columns x min(block_size, 64) rows, 128-byte swizzle.
-// fp8: rows of head_dim one-byte codes, whole-row boxes with the swizzle of
-// their width (128 bytes at head_dim 128, 64 at 64), which the consumers'
-// reads apply.
+// both_halves (bf16, head_dim 128): a 3-D view (64 columns, rows, 2 halves
+// 128 bytes apart) whose boxes hold both halves of box_rows rows, landing as
+// [half][row][128 B].  fp8: rows of head_dim one-byte codes, whole-row boxes
+// with the swizzle of their width (128 bytes at head_dim 128, 64 at 64),
+// which the consumers' reads apply.
 bool encode_cache_map(CUtensorMap* map, const void* base, long long rows, int head_dim,
-                      int box_rows, bool fp8) {
+                      int box_rows, bool fp8, bool both_halves) {
+    both_halves = both_halves && !fp8 && head_dim == 128;
     {
         std::lock_guard<std::mutex> lock(g_map_mu);
         for (const MapCacheEntry& e : g_map_cache)
             if (e.base == base && e.rows == rows && e.head_dim == head_dim &&
-                e.box_rows == box_rows && e.fp8 == fp8) {
+                e.box_rows == box_rows && e.fp8 == fp8 && e.both_halves == both_halves) {
                 *map = e.map;
                 return true;
             }
     }
     auto enc = tensor_map_encoder();
     if (!enc) return false;
-    cuuint64_t gdim[2] = {(cuuint64_t)head_dim, (cuuint64_t)rows};
-    cuuint64_t gstride[1] = {(cuuint64_t)head_dim * (fp8 ? 1 : 2)};
-    cuuint32_t box[2] = {fp8 ? (cuuint32_t)head_dim : 64u, (cuuint32_t)box_rows};
-    cuuint32_t estride[2] = {1u, 1u};
+    const cuuint64_t row_bytes = (cuuint64_t)head_dim * (fp8 ? 1 : 2);
+    cuuint64_t gdim[3] = {(cuuint64_t)(both_halves ? 64 : head_dim), (cuuint64_t)rows, 2};
+    cuuint64_t gstride[2] = {row_bytes, 128};
+    cuuint32_t box[3] = {fp8 ? (cuuint32_t)head_dim : 64u, (cuuint32_t)box_rows, 2u};
+    cuuint32_t estride[3] = {1u, 1u, 1u};
     const CUresult r = enc(map, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                           2, const_cast<void*>(base), gdim, gstride, box, estride,
-                           CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           both_halves ? 3 : 2, const_cast<void*>(base), gdim, gstride, box,
+                           estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
                            (fp8 && head_dim == 64) ? CU_TENSOR_MAP_SWIZZLE_64B
                                                    : CU_TENSOR_MAP_SWIZZLE_128B,
                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -1478,6 +1503,7 @@ bool encode_cache_map(CUtensorMap* map, const void* base, long long rows, int he
     e.head_dim = head_dim;
     e.box_rows = box_rows;
     e.fp8 = fp8;
+    e.both_halves = both_halves;
     e.map = *map;
     return true;
 }

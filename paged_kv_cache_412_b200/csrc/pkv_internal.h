@@ -157,12 +157,13 @@ bool decode_mma_supported(int head_dim, int block_size, pkv_dtype q_dtype, pkv_d
 pkv_status launch_decode_mma(const DecodeParams& p, int head_dim, int group_pad, bool fp8,
                              cudaStream_t stream, int* grid_out);
 
-// 2-D TMA view of a cache [num_blocks, Hkv, block_size, head_dim] as
-// rows x head_dim: bf16 boxes of 64 columns x box_rows rows with the 128-byte
-// swizzle; fp8 boxes of whole rows without swizzle.  False if the driver
-// entry point is missing or the encoder rejects the view.
+// TMA view of a cache [num_blocks, Hkv, block_size, head_dim] as rows x
+// head_dim: bf16 boxes of 64 columns x box_rows rows with the 128-byte
+// swizzle (both_halves at head_dim 128: 3-D boxes holding both 64-column
+// halves); fp8 boxes of whole rows with the swizzle of their width.  False if
+// the driver entry point is missing or the encoder rejects the view.
 bool encode_cache_map(CUtensorMap* map, const void* base, long long rows, int head_dim,
-                      int box_rows, bool fp8);
+                      int box_rows, bool fp8, bool both_halves = false);
 
 // Launch config with programmatic dependent launch: the kernel may start while
 // the previous kernel in the stream drains; it waits (griddepcontrol.wait)
