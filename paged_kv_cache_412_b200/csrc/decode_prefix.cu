@@ -164,13 +164,12 @@ __global__ void __launch_bounds__(kThreadsP, 1)
         __syncwarp();
         const int r_lo = rt * kPrefixRows;
         int count = 0, best_L = -1, best_b = 0x7fffffff;
-        for (int b0 = 0; b0 < p.num_seqs; b0 += 32) {
+        auto scan = [&](int b0, int gb, int L) {
             const int b = b0 + lane;
-            const bool mem = b < p.num_seqs && __ldg(p.prefix_of + b) == g;
+            const bool mem = b < p.num_seqs && gb == g;
             const unsigned bal = __ballot_sync(FULL_MASK, mem);
             if (mem) {
                 const int rank = count + __popc(bal & ((1u << lane) - 1u));
-                int L = __ldg(p.seq_lens + b);
                 L = L < 0 ? 0 : (L > cap ? cap : L);  // the decode pass flags it
                 if (L > best_L) {
                     best_L = L;
@@ -186,6 +185,24 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                 }
             }
             count += __popc(bal);
+        };
+        // The first 128 requests' group ids and lengths are loaded together
+        // (one round trip), the rest as the scan reaches them.
+        constexpr int kAhead = 4;
+        int gb[kAhead], lb[kAhead];
+#pragma unroll
+        for (int k = 0; k < kAhead; ++k) {
+            const int b = 32 * k + lane;
+            gb[k] = b < p.num_seqs ? __ldg(p.prefix_of + b) : -1;
+            lb[k] = b < p.num_seqs ? __ldg(p.seq_lens + b) : 0;
+        }
+#pragma unroll
+        for (int k = 0; k < kAhead; ++k)
+            if (32 * k < p.num_seqs) scan(32 * k, gb[k], lb[k]);
+        for (int b0 = 32 * kAhead; b0 < p.num_seqs; b0 += 32) {
+            const int b = b0 + lane;
+            scan(b0, b < p.num_seqs ? __ldg(p.prefix_of + b) : -1,
+                 b < p.num_seqs ? __ldg(p.seq_lens + b) : 0);
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
@@ -409,13 +426,15 @@ __global__ void __launch_bounds__(kThreadsP, 1)
             tc_fence_after();
             float s[kPrefixCH];
             {
-                uint32_t u[32];
+                // both 32-column halves in flight before one wait
+                uint32_t u0[32], u1[32];
+                tmem_ld32(trow + kSCol + b * kPrefixCH, u0);
+                tmem_ld32(trow + kSCol + b * kPrefixCH + 32, u1);
+                tmem_wait_ld();
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    tmem_ld32(trow + kSCol + b * kPrefixCH + half * 32, u);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) s[half * 32 + j] = __uint_as_float(u[j]);
+                for (int j = 0; j < 32; ++j) {
+                    s[j] = __uint_as_float(u0[j]);
+                    s[32 + j] = __uint_as_float(u1[j]);
                 }
             }
             tc_fence_before();
