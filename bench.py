@@ -592,6 +592,7 @@ def run_ours(args, rank: int, world: int, local: int):
             "gpu_launches": 2 * args.steps,
             "clocks": clocks,
             "configs": configs,
+            "configs_l2": _L2Flush.DESCRIPTION if configs else None,
         }
         print(json.dumps(result), flush=True)
     dist_barrier(world)
@@ -603,14 +604,24 @@ def run_ours(args, rank: int, world: int, local: int):
 # ---------------------------------------------------------------------------
 
 class _L2Flush:
-    """Writes a buffer twice the size of L2 between timed launches."""
+    """Between timed launches: writes a buffer twice the size of L2, then reads
+    a second one of the same size.  The write evicts whatever the timed launch
+    touched; the read makes the L2 write those dirty lines back before the
+    launch starts, so the launch neither finds its data in L2 nor pays for the
+    flush's own write-backs."""
+
+    DESCRIPTION = "flushed (256 MB write, then 256 MB read of another buffer) before every timed launch"
 
     def __init__(self, dev):
         import torch
         self.buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        self.clean = torch.zeros(64 << 20, dtype=torch.float32, device=dev)
+        self.acc = torch.zeros((), dtype=torch.float32, device=dev)
 
     def __call__(self):
+        import torch
         self.buf.zero_()
+        torch.sum(self.clean, dim=0, out=self.acc)
 
 
 def _device_clean():
@@ -688,7 +699,7 @@ def run_suite(args):
                 "frac_of_hbm_peak": round(gbs / peak, 4), "peak": peak,
                 "peak_kind": f"{peak_kind} HBM copy bandwidth", "us_mean": round(mean * 1e3, 2),
                 "us_median": round(med * 1e3, 2), "bytes": int(nbytes), "launches_timed": iters,
-                "l2": "flushed (256 MB write) before every timed launch"}
+                "l2": _L2Flush.DESCRIPTION}
         line.update(extra)
         print(json.dumps(line), flush=True)
 
@@ -804,7 +815,7 @@ def _oracle_rate(w, nthreads: int, budget_s: float, lib, per_head: bool) -> dict
 def run_configs(pkv, torch, dev, peak, peak_kind, with_oracle=True, iters=200,
                 oracle_budget_s=0.8) -> list:
     """One compact entry per workload: mean decode time over ``iters`` launches
-    (each after a 256 MB L2 flush, CUDA events around each), KV GB/s by the
+    (each after the L2 flush of _L2Flush, CUDA events around each), KV GB/s by the
     decode byte model, the fraction of the HBM peak, and the oracle's KV GB/s on
     a bounded sample of the same workload on all host cores and on one thread.
     """

@@ -39,15 +39,15 @@ int elem_size(pkv_dtype t) {
     }
 }
 
-// Splits of the shared prefix pass: enough (group, kv head, row tile, split)
-// CTAs for about one per SM (the pass holds one CTA per SM), at most one per
-// 64-token chunk of the longest prefix.
+// Splits of the shared prefix pass: as many (group, kv head, row tile, split)
+// CTAs as fit one wave (the pass holds one CTA per SM; a partial second wave
+// would double the pass), at most one per 64-token chunk of the longest prefix.
 int prefix_splits_for(int num_sms, int num_prefixes, int num_kv_heads, int row_tiles,
                       int max_prefix_len) {
     const long long base = (long long)num_prefixes * num_kv_heads * row_tiles;
     const long long nch = (max_prefix_len + 63) / 64;
     if (base <= 0 || nch <= 0) return 1;
-    long long s = ((long long)num_sms + base - 1) / base;
+    long long s = (long long)num_sms / base;
     s = std::min(s, nch);
     s = std::min(s, 64LL);
     return (int)std::max(s, 1LL);

@@ -119,7 +119,11 @@ struct Smem {
     static constexpr int DUMP_ML = NT * 4;                // m[2], l[2] per n-tile per lane
     static constexpr int DUMP_BYTES = C::DUMP_BYTES;
     static constexpr int OFF_DUMP = C::NSTAGE * C::STAGE_BYTES;
-    static constexpr int OFF_BAR = OFF_DUMP + NSLOT * DUMP_BYTES;
+    // fp8, 8-head groups: one partial record (acc rows, then m/l pairs) the
+    // epilogue prefetches for a split group's merge
+    static constexpr int PF_BYTES = (F8 && NT == 1) ? C::GP * D * 4 + C::GP * 2 * 4 : 0;
+    static constexpr int OFF_PF = OFF_DUMP + NSLOT * DUMP_BYTES;
+    static constexpr int OFF_BAR = OFF_PF + PF_BYTES;
     // full/empty per stage, dfull/dempty per dump slot
     static constexpr int OFF_META = OFF_BAR + (2 * C::NSTAGE + 2 * NSLOT) * 8;
     // ntok/bad per stage
@@ -898,21 +902,106 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
         for (int i = lane; i < p.num_q_heads * D; i += 32)
             store_out(p.out, (size_t)b * p.num_q_heads * D + i, 0.f, p.out_dtype);
     }
+    // A partial record (acc rows of GP heads, then their m/l pairs) as this
+    // lane's fragment: from global memory (through L2), or from the
+    // prefetch buffer in shared memory.
+    auto load_frag = [&](const float* acc_rows, const float* ml_rows, bool global,
+                         float (&mr)[NT][2], float (&lr)[NT][2], float (&ar)[C::KS][NT][4]) {
+        auto ld = [&](const float* q) { return global ? ld_cg(q) : *q; };
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                const int h = nt * 8 + 2 * tig + j;
+                const float* mlp = ml_rows + h * 2;
+                const float* ra = acc_rows + h * D;
+                mr[nt][j] = ld(mlp);
+                lr[nt][j] = ld(mlp + 1);
+#pragma unroll
+                for (int dt = 0; dt < C::KS; ++dt) {
+                    ar[dt][nt][j] = ld(ra + dcol<F8>(dt, grp, 0));
+                    ar[dt][nt][j + 2] = ld(ra + dcol<F8>(dt, grp, 1));
+                }
+            }
+    };
+    auto load_rec = [&](size_t rec, float (&mr)[NT][2], float (&lr)[NT][2],
+                        float (&ar)[C::KS][NT][4]) {
+        load_frag(p.rec_acc + rec * GP * D, p.rec_ml + rec * GP * 2, true, mr, lr, ar);
+    };
+    // The epilogue warp is idle while the consumers stream a segment.  For a
+    // group split over several units it watches, meanwhile, the ready flags of
+    // the group's other parts (in merge order): a part that has seen all of
+    // them is the last to finish without asking.  It also fetches the first
+    // published record, so the merge's inputs are at hand: bf16 into
+    // registers, fp8 (no registers to spare) into a shared-memory buffer with
+    // asynchronous copies.  16-head groups neither watch nor prefetch.
+    constexpr bool kWatch = NT == 1;
+    constexpr bool kPrefetch = NT == 1 && !F8;
+    constexpr bool kPrefetchSmem = S::PF_BYTES > 0;
+    float* pf_acc = reinterpret_cast<float*>(smem + S::OFF_PF);
+    float* pf_ml = pf_acc + GP * D;
+
     while (it.valid) {
         const Segment sg = it.current();
         it.advance(p, lane);
         const SegInfo si = seg_info<GP>(p, sg, it.W);
         const float vsc = F8 ? __ldg(p.v_scale + si.kvh) : 1.f;  // V dequantisation scale
+        // Parts of the group: the records bg + u of its units u_first .. u_last.
+        auto rec_of = [&](int k) -> size_t { return si.bg + (size_t)(si.u_first + k); };
+        const int own = (int)(si.u - si.u_first);
+        const bool split = !p.defer_merge && si.nseg > 1 && rec_of(si.nseg - 1) < (size_t)p.rec_cap;
+        // next other part (ascending, skipping our own) whose flag has not been seen
+        auto next_other = [&](int k) {
+            ++k;
+            if (k == own) ++k;
+            return k;
+        };
+        int watch = split ? next_other(-1) : si.nseg;
+        int pf_k = -1;  // the part whose record sits in pm / pl / pa
+        float pm[NT][2], pl[NT][2], pa[C::KS][NT][4];
+
         // the segment's state: one consumer's, or the merge of NCONS consumers'
         float acc[C::KS][NT][4], m[NT][2], l[NT][2];
 #pragma unroll
         for (int k = 0; k < C::NCONS; ++k) {
             const int slot = k * S::NDUMP + dring.stage;
+            if constexpr (kWatch) {
+                // Watch the flags until the hand-over is there: lane 0's flag
+                // load is in flight while the warp tests the barrier.  Bounded
+                // by the wait below, which also reports a hang.
+                const uint64_t t0 = global_timer_ns();
+                while (watch < si.nseg && !ctrl[0]) {
+                    if (__any_sync(FULL_MASK, mbar_try_wait(&dfull[slot], dring.phase))) break;
+                    unsigned f = 0u;
+                    if (lane == 0) f = ld_acquire_u32(p.ready + rec_of(watch));
+                    f = __shfl_sync(FULL_MASK, f, 0);
+                    if (f) {
+                        __syncwarp();  // lane 0's acquire orders the warp's reads of the record
+                        if (pf_k < 0 && kPrefetch) {
+                            load_rec(rec_of(watch), pm, pl, pa);
+                            pf_k = watch;
+                        } else if (pf_k < 0 && kPrefetchSmem) {
+                            // the whole record, 16 bytes per copy, into the
+                            // buffer (free once an earlier prefetch whose
+                            // record went unused has landed)
+                            cp_async_wait_all();
+                            const float* ga = p.rec_acc + rec_of(watch) * GP * D;
+                            const float* gm = p.rec_ml + rec_of(watch) * GP * 2;
+                            for (int i = lane; i < GP * D / 4; i += 32) cp_async_cg16(pf_acc + 4 * i, ga + 4 * i);
+                            if (lane < GP * 2 / 4) cp_async_cg16(pf_ml + 4 * lane, gm + 4 * lane);
+                            pf_k = watch;
+                        }
+                        watch = next_other(watch);
+                    }
+                    if (global_timer_ns() - t0 > p.wait_ns) break;
+                }
+            }
             if (ctrl[0] || !mbar_wait(&dfull[slot], dring.phase, p.wait_ns)) {
                 if (lane == 0 && !ctrl[0]) {
                     ctrl[0] = 1;
                     raise_error(p.err, PKV_DEVERR_TIMEOUT);
                 }
+                if constexpr (kPrefetchSmem) cp_async_wait_all();  // nothing lands after exit
                 return;
             }
             const float* dump =
@@ -986,53 +1075,43 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
             if (fits) write_record<D, NT, F8>(p, si.bg + si.u, tig, grp, acc, m, l);
             continue;
         }
-        // The row state: this part's own, then everything merged into it.
-        float Mc[NT][2], Sc[NT][2], A[C::KS][NT][4];
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-            for (int j = 0; j < 2; ++j) {
-                Mc[nt][j] = m[nt][j];
-                Sc[nt][j] = l[nt][j];
-            }
-#pragma unroll
-        for (int dt = 0; dt < C::KS; ++dt)
-#pragma unroll
-            for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                for (int i = 0; i < 4; ++i) A[dt][nt][i] = acc[dt][nt][i];
-        // Parts of the group: the records bg + u of its units u_first .. u_last.
-        auto rec_of = [&](int k) -> size_t { return si.bg + (size_t)(si.u_first + k); };
-        const int own = (int)(si.u - si.u_first);
-        if (si.nseg > 1) {
-            if (rec_of(si.nseg - 1) >= (size_t)p.rec_cap) {
-                if (lane == 0) raise_error(p.err, PKV_DEVERR_BAD_SEQ_LEN);
-                continue;
-            }
-            // Arrive first.  Only a part that is not the last of its group to
-            // finish publishes its partial result (record, then a ready flag);
-            // the last one keeps its own in registers and merges the others'.
+        if (si.nseg > 1 && !split) {
+            if (lane == 0) raise_error(p.err, PKV_DEVERR_BAD_SEQ_LEN);
+            continue;
+        }
+        if (split && watch < si.nseg) {
+            // Not every other part is known to be out: arrive.  A part that
+            // is not the last of its group to finish publishes its partial
+            // result (record, then a release of its ready flag); the last one
+            // keeps its own in registers and merges the others'.  (When every
+            // other flag was seen, every other part has arrived and published:
+            // this part is the last without asking.)
             unsigned arrived = 0;
             if (lane == 0) arrived = atomicAdd(p.counters + si.bg, 1u);
             arrived = __shfl_sync(FULL_MASK, arrived, 0);
             if (arrived != (unsigned)(si.nseg - 1)) {
                 write_record<D, NT, F8>(p, rec_of(own), tig, grp, acc, m, l);
-                __threadfence();
                 __syncwarp();
-                if (lane == 0) atomicExch(p.ready + rec_of(own), 1u);
+                if (lane == 0) st_release_u32(p.ready + rec_of(own), 1u);
                 continue;
             }
 
-            // Last part: wait (bounded) until every other part's record is out.
+            // Last part: wait (bounded) until the remaining parts' records are out.
             int ok = 1;
             if (lane == 0) {
                 const uint64_t t0 = global_timer_ns();
-                for (int k = 0; k < si.nseg && ok; ++k) {
-                    // (the test-only fault waits for the merger's own flag too,
-                    // which nothing sets)
-                    if (k == own && p.fault_mode != kFaultMergeFlag) continue;
-                    volatile unsigned* f = p.ready + rec_of(k);
-                    for (uint32_t it = 0; *f == 0u; ++it) {
+                for (int k = watch; k < si.nseg && ok; k = next_other(k)) {
+                    for (uint32_t it = 0; ld_acquire_u32(p.ready + rec_of(k)) == 0u; ++it) {
+                        if ((it & 63u) == 63u && global_timer_ns() - t0 > p.wait_ns) {
+                            ok = 0;
+                            break;
+                        }
+                    }
+                }
+                // (the test-only fault waits for the merger's own flag too,
+                // which nothing sets)
+                if (ok && p.fault_mode == kFaultMergeFlag) {
+                    for (uint32_t it = 0; ld_acquire_u32(p.ready + rec_of(own)) == 0u; ++it) {
                         if ((it & 63u) == 63u && global_timer_ns() - t0 > p.wait_ns) {
                             ok = 0;
                             break;
@@ -1043,55 +1122,52 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
             }
             ok = __shfl_sync(FULL_MASK, ok, 0);
             if (!ok) continue;
-            __threadfence();
+            __syncwarp();  // lane 0's acquires order the warp's reads of the records
         }
-        // Online merge of the other parts' records, in order: M = max m,
-        // S = sum 2^(m-M) l, A = sum 2^(m-M) acc, out = A / S.  Records are
-        // fetched two at a time with every load of the pair in flight before
-        // any math.
-        for (int k0 = 0; si.nseg > 1 && k0 < si.nseg; k0 += 2) {
-            float mr[2][NT][2], lr[2][NT][2], ar[2][C::KS][NT][4];
-            bool use[2];
+        // The row state: this part's own, then the other parts merged into it
+        // in ascending order (the prefetched one, when there is one, is the
+        // first of them): M = max m, S = sum 2^(m-M) l, A = sum 2^(m-M) acc,
+        // out = A / S.  The others are fetched two at a time (8-head groups)
+        // with every load of the pair in flight before any math.
+        auto merge_in = [&](const float (&mr)[NT][2], const float (&lr)[NT][2],
+                            const float (&ar)[C::KS][NT][4]) {
 #pragma unroll
-            for (int k = 0; k < 2; ++k) {
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const float M = fmaxf(m[nt][j], mr[nt][j]);
+                    const float mref = M == -INFINITY ? 0.f : M;
+                    const float fa = exp2f(m[nt][j] - mref), fb = exp2f(mr[nt][j] - mref);
+                    l[nt][j] = l[nt][j] * fa + lr[nt][j] * fb;
+#pragma unroll
+                    for (int dt = 0; dt < C::KS; ++dt) {
+                        acc[dt][nt][j] = acc[dt][nt][j] * fa + ar[dt][nt][j] * fb;
+                        acc[dt][nt][j + 2] = acc[dt][nt][j + 2] * fa + ar[dt][nt][j + 2] * fb;
+                    }
+                    m[nt][j] = M;
+                }
+        };
+        if (kPrefetch && split && pf_k >= 0) merge_in(pm, pl, pa);
+        if (kPrefetchSmem && split && pf_k >= 0) {
+            cp_async_wait_all();
+            __syncwarp();  // every lane's copies have landed
+            float mr[NT][2], lr[NT][2], ar[C::KS][NT][4];
+            load_frag(pf_acc, pf_ml, false, mr, lr, ar);
+            merge_in(mr, lr, ar);
+        }
+        constexpr int kPair = NT == 1 ? 2 : 1;  // records in flight at once
+        for (int k0 = 0; split && k0 < si.nseg; k0 += kPair) {
+            float mr[kPair][NT][2], lr[kPair][NT][2], ar[kPair][C::KS][NT][4];
+            bool use[kPair];
+#pragma unroll
+            for (int k = 0; k < kPair; ++k) {
                 const int kk = k0 + k;
-                use[k] = kk < si.nseg && kk != own;
-                if (!use[k]) continue;
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        const size_t rr = rec_of(kk) * GP + nt * 8 + 2 * tig + j;
-                        const float* mlp = p.rec_ml + rr * 2;
-                        const float* ra = p.rec_acc + rr * D;
-                        mr[k][nt][j] = ld_cg(mlp);
-                        lr[k][nt][j] = ld_cg(mlp + 1);
-#pragma unroll
-                        for (int dt = 0; dt < C::KS; ++dt) {
-                            ar[k][dt][nt][j] = ld_cg(ra + dcol<F8>(dt, grp, 0));
-                            ar[k][dt][nt][j + 2] = ld_cg(ra + dcol<F8>(dt, grp, 1));
-                        }
-                    }
+                use[k] = kk < si.nseg && kk != own && kk != pf_k;
+                if (use[k]) load_rec(rec_of(kk), mr[k], lr[k], ar[k]);
             }
 #pragma unroll
-            for (int k = 0; k < 2; ++k) {
-                if (!use[k]) continue;
-#pragma unroll
-                for (int nt = 0; nt < NT; ++nt)
-#pragma unroll
-                    for (int j = 0; j < 2; ++j) {
-                        const float M = fmaxf(Mc[nt][j], mr[k][nt][j]);
-                        const float mref = M == -INFINITY ? 0.f : M;
-                        const float fa = exp2f(Mc[nt][j] - mref), fb = exp2f(mr[k][nt][j] - mref);
-                        Sc[nt][j] = Sc[nt][j] * fa + lr[k][nt][j] * fb;
-#pragma unroll
-                        for (int dt = 0; dt < C::KS; ++dt) {
-                            A[dt][nt][j] = A[dt][nt][j] * fa + ar[k][dt][nt][j] * fb;
-                            A[dt][nt][j + 2] = A[dt][nt][j + 2] * fa + ar[k][dt][nt][j + 2] * fb;
-                        }
-                        Mc[nt][j] = M;
-                    }
-            }
+            for (int k = 0; k < kPair; ++k)
+                if (use[k]) merge_in(mr[k], lr[k], ar[k]);
         }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)
@@ -1099,16 +1175,16 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
             for (int j = 0; j < 2; ++j) {
                 const int h = nt * 8 + 2 * tig + j;
                 if (h >= si.gv) continue;
-                const float inv = Sc[nt][j] > 0.f ? vsc / Sc[nt][j] : 0.f;
+                const float inv = l[nt][j] > 0.f ? vsc / l[nt][j] : 0.f;
                 const size_t orow = ((size_t)si.b * p.num_q_heads + si.hq0 + h) * D;
 #pragma unroll
                 for (int dt = 0; dt < C::KS; ++dt) {
-                    store_out(p.out, orow + dcol<F8>(dt, grp, 0), A[dt][nt][j] * inv, p.out_dtype);
-                    store_out(p.out, orow + dcol<F8>(dt, grp, 1), A[dt][nt][j + 2] * inv,
+                    store_out(p.out, orow + dcol<F8>(dt, grp, 0), acc[dt][nt][j] * inv, p.out_dtype);
+                    store_out(p.out, orow + dcol<F8>(dt, grp, 1), acc[dt][nt][j + 2] * inv,
                               p.out_dtype);
                 }
             }
-        if (si.nseg > 1) {
+        if (split) {
             __syncwarp();
             if (lane == 0) {  // ready for the next call
                 for (int k = 0; k < si.nseg; ++k) p.ready[rec_of(k)] = 0u;
@@ -1116,6 +1192,7 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
             }
         }
     }
+    if constexpr (kPrefetchSmem) cp_async_wait_all();  // an unused prefetch lands before exit
 }
 
 // Total chunk count, computed by one warp (same value in every warp and CTA).

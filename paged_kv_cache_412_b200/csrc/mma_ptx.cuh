@@ -120,4 +120,16 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 
 __device__ __forceinline__ float ld_cg(const float* p) { return __ldcg(p); }
 
+// 16-byte global -> shared copy through L2 (no L1), asynchronous to the
+// issuing thread; complete with cp_async_wait_all().
+__device__ __forceinline__ void cp_async_cg16(void* dst_smem, const void* src_gmem) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst_smem)),
+                 "l"(src_gmem)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 }  // namespace pkv

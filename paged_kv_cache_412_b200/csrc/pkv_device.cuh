@@ -78,6 +78,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
     return false;
 }
 
+// ---- flags between CTAs ------------------------------------------------------
+
+// Acquire load of a flag at GPU scope: what its releasing writer wrote before
+// the release is visible to this thread (and, after a warp barrier, to the
+// rest of the warp) once the value is seen.
+__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
+    unsigned v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Release store of a flag at GPU scope: the writes this thread, and the
+// threads synchronised with it by a barrier before, made are visible to an
+// acquirer that reads the value.
+__device__ __forceinline__ void st_release_u32(unsigned* p, unsigned v) {
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
 // ---- bulk copies (TMA, non-tensor, no multicast) ---------------------------
 
 // L2 policy for data read exactly once (streamed K/V tiles).
