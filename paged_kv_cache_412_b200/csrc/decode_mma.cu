@@ -22,18 +22,20 @@
 // into the B-operand layout with movmatrix.trans.  P is split into bf16 hi + lo
 // parts (two MMAs) so the weights keep ~16 mantissa bits.
 //
-// Data movement: a producer warp walks the block table (32 entries per
+// Data movement: producer warps walk the block table (32 entries per
 // coalesced load, next window prefetched, next segment's first window too) and
-// issues TMA tensor copies (2-D tensor map over the cache rows, 128-byte
+// issue TMA tensor copies (2-D or 3-D tensor map over the cache rows, 128-byte
 // swizzle, no multicast) of each physical block's K and V rows into a ring of
 // shared-memory stages with mbarrier completion, one lane per block.
-// bf16: one consumer warp does the math (no cross-warp reduction), two CTAs
-// share an SM.  fp8: one CTA per SM with two producers, four converter warps
-// that widen each stage to f16 and three consumers taking the chunks in turn.
-// An epilogue warp normalises; a request's (head group) split over several
-// units is merged in-kernel by the last unit to finish (per-group arrival
-// counter in the workspace, reset by the merger), or -- fixed partitions and
-// prefix groups -- by a separate merge kernel:
+// Consumer warps do the math, taking the CTA's 64-token chunks in turn, and
+// hand their running state to an epilogue warp: bf16 one CTA per SM with one
+// producer and two consumers (16-head groups: one consumer, two CTAs per SM);
+// fp8 one CTA per SM with four producers and six consumers that widen the
+// codes to f16 in registers.  The epilogue normalises; a (request, head group)
+// split over several units is merged in-kernel by the last unit to finish
+// (per-group arrival counter and ready flags in the workspace, reset by the
+// merger), or -- fixed partitions and prefix groups -- by a separate merge
+// kernel:
 //   out = sum_u 2^(m_u - M) acc_u / sum_u 2^(m_u - M) l_u.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -55,13 +57,15 @@ constexpr int kRingBudget = 104448;  // 3 stages of K+V+q at head_dim 128
 
 constexpr int cmin(int a, int b) { return a < b ? a : b; }
 constexpr int cmax(int a, int b) { return a > b ? a : b; }
+constexpr int cgcd(int a, int b) { return b == 0 ? a : cgcd(b, a % b); }
+constexpr int clcm(int a, int b) { return a / cgcd(a, b) * b; }
 
 // F8 = false: bf16 cache, tiles land swizzled and feed bf16 MMAs directly.
 // F8 = true : fp8 (e4m3) cache, tiles land as rows of head_dim one-byte codes
 //             (TMA boxes with the swizzle of their width) and every consumer
 //             widens what it loads from them to f16 in registers (exact), for
 //             f16 MMAs; q is widened to f16 likewise.
-template <int D, int NT, bool F8>
+template <int D, int NT, bool F8, bool RC = false>
 struct MmaCfg {
     static constexpr int NHALF = D / 64;            // 128-byte column halves of a 16-bit row
     static constexpr int KS = D / 16;               // k-steps of q.K^T, m-tiles of P.V
@@ -69,49 +73,64 @@ struct MmaCfg {
     static constexpr int KV_BYTES = F8 ? kCH * D : NHALF * HALF_BYTES;  // K (or V) of a stage
     static constexpr int GP = 8 * NT;               // query heads per head group (padded)
     static constexpr int Q_BYTES = GP * D * 2;      // the group's q rows (first stage of a segment)
-    // bf16: K | V | q, rounded to the 1 KB the 128-byte swizzle pattern repeats
-    // on.  fp8: K | V only (8 or 4 KB each, whole swizzle periods); each
-    // consumer reads the group's q from global memory.
-    static constexpr int STAGE_BYTES = F8 ? 2 * KV_BYTES : (2 * KV_BYTES + Q_BYTES + 1023) / 1024 * 1024;
+    // Consumers.  bf16, 16-head groups: one tensor-core consumer reads every
+    // stage (two CTAs per SM).  Otherwise one CTA per SM whose NCONS consumers
+    // take the CTA's chunks in turn (chunk n -> consumer n % NCONS, stage
+    // n % NSTAGE; NSTAGE is a multiple of NCONS, so a stage always serves the
+    // same consumer and each barrier has one waiter stepping through its
+    // phases in order):
+    //   bf16, 8-head groups, TMA boxes: two consumers.  One CTA per SM halves the units
+    //     of a call, so a unit (56 chunks of the 4k batch) is nearly as long
+    //     as a (request, kv head) group (64): most groups split into two
+    //     parts, one of which finishes early and is prefetched by the other's
+    //     merge -- with two CTAs per SM a group's middle parts end with the
+    //     kernel and the last merges wait for them.  (Row copies keep two
+    //     CTAs per SM with one consumer: their producer issues 64 copies per
+    //     chunk, and one producer per SM cannot keep up.)
+    //   fp8: widening codes costs instructions and latency the bf16 path does
+    //     not have, and one consumer warp cannot hide its own ldmatrix -> cvt
+    //     -> mma chains: six consumers (two on each of two SM sub-partitions)
+    //     overlap them; the 16-head configuration keeps four (its consumers
+    //     need all the registers).
+    static constexpr int NCONS = F8 ? (NT == 1 ? 6 : 4) : (NT == 1 && !RC ? 2 : 1);
+    // bf16 with one consumer: K | V | q, rounded to the 1 KB the 128-byte
+    // swizzle pattern repeats on (the segment's first stage carries q).
+    // Otherwise each consumer reads the group's q from global memory: fp8
+    // K | V only (8 or 4 KB each, whole swizzle periods); bf16 K | V, or the
+    // row-copy regions if larger.
+    static constexpr bool Q_IN_STAGE = !F8 && NCONS == 1;
     // row-copy stages (bf16 blocks of 2 or 4 rows): K | V regions of up to 32
     // skewed blocks (rc_block_bytes), inside the same stage size
     static constexpr int RC_KV_BYTES = kCH * D * 2 + 32 * 16;
+    static constexpr int STAGE_BYTES =
+        F8 ? 2 * KV_BYTES
+           : (cmax(2 * KV_BYTES + (Q_IN_STAGE ? Q_BYTES : 0), 2 * RC_KV_BYTES) + 1023) / 1024 * 1024;
     static_assert(F8 || 2 * RC_KV_BYTES <= STAGE_BYTES, "row-copy regions fit a stage");
-    // bf16: one tensor-core consumer reads the TMA stages (two CTAs per SM).
-    // fp8: one CTA per SM whose NCONS consumers take the CTA's chunks in turn
-    // (chunk n -> consumer n % NCONS, stage n % NSTAGE; NSTAGE is a multiple of
-    // NCONS, so a stage always serves the same consumer and each barrier has
-    // one waiter stepping through its phases in order).  Widening codes costs
-    // instructions and latency the bf16 path does not have, and one consumer
-    // warp cannot hide its own ldmatrix -> cvt -> mma chains: six consumers
-    // (two on each of two SM sub-partitions) overlap them; the 16-head
-    // configuration keeps four (its consumers need all the registers).
-    static constexpr int NCONS = F8 ? (NT == 1 ? 6 : 4) : 1;
     // producer warps: a TMA issue holds the issuing warp ~0.11 us, so one
     // warp issues at most ~9 boxes per us however its lanes share them.  An
     // fp8 chunk is 8 boxes of 2 KB; four producers take chunks in turn (stage
     // n % NSTAGE belongs to producer n % NPROD), enough to keep 12 stages in
-    // flight.  The 16-head configuration keeps two (registers).
+    // flight.  The 16-head configuration keeps two (registers).  bf16: one.
     static constexpr int NPROD = F8 ? (NT == 1 ? 4 : 2) : 1;
     static constexpr int THREADS = 32 * (NPROD + NCONS + 1);  // + the epilogue
     // consumer -> epilogue hand-off: per lane, the accumulators and (m, l)
     static constexpr int DUMP_BYTES = (KS * NT * 4 + NT * 4) * 32 * 4;
-    // fp8: as many stages as the shared memory holds beside the hand-off
-    // slots (up to 24), a multiple of NCONS and NPROD: 192 KB of codes in
-    // flight per SM at head_dim 128, as much as the two bf16 CTAs of an SM keep
-    static constexpr int F8_RING = 227 * 1024 - NCONS * DUMP_BYTES - 4096;
-    static constexpr int STAGE_STEP = F8 ? (NCONS == 6 ? 12 : 4) : 1;  // lcm(NCONS, NPROD)
-    static constexpr int NSTAGE = F8 ? cmin(24, F8_RING / STAGE_BYTES) / STAGE_STEP * STAGE_STEP
-                                     : cmax(2, cmin(8, kRingBudget / STAGE_BYTES));
+    // One CTA per SM: as many stages as the shared memory holds beside the
+    // hand-off slots (up to 24), a multiple of NCONS and NPROD: 192 KB or
+    // more in flight per SM at head_dim 128.
+    static constexpr int RING = 227 * 1024 - NCONS * DUMP_BYTES - 4096;
+    static constexpr int STAGE_STEP = clcm(NCONS, NPROD);
+    static constexpr int NSTAGE = NCONS == 1 ? cmax(2, cmin(8, kRingBudget / STAGE_BYTES))
+                                             : cmin(24, RING / STAGE_BYTES) / STAGE_STEP * STAGE_STEP;
     static_assert(NSTAGE % NPROD == 0 && NSTAGE % NCONS == 0 && NSTAGE >= 2,
                   "each stage belongs to one producer and one consumer");
 };
 
 // ---- shared-memory layout ------------------------------------------------------
 
-template <int D, int NT, bool F8>
+template <int D, int NT, bool F8, bool RC = false>
 struct Smem {
-    using C = MmaCfg<D, NT, F8>;
+    using C = MmaCfg<D, NT, F8, RC>;
     // consumer -> epilogue hand-off slots per consumer
     static constexpr int NDUMP = C::NCONS == 1 ? 2 : 1;
     static constexpr int NSLOT = C::NCONS * NDUMP;
@@ -192,7 +211,7 @@ __device__ __forceinline__ int bf16_row_off(int t, int half, int log2_rb) {
 // a separate instance so the boxed producer carries no trace of it.
 template <int D, int NT, bool F8, bool RC>
 struct Producer {
-    using C = MmaCfg<D, NT, F8>;
+    using C = MmaCfg<D, NT, F8, RC>;
     static_assert(!(RC && F8), "row copies serve bf16 caches only");
 
     const DecodeParams& p;
@@ -321,7 +340,7 @@ struct Producer {
                 st_ntok[stage] = ntok;
                 st_bad[stage] = bad;
                 if (bad) raise_error(p.err, PKV_DEVERR_BAD_BLOCK);
-                const uint32_t qbytes = (!F8 && c == sg.c0) ? (uint32_t)gv * D * 2u : 0u;
+                const uint32_t qbytes = (C::Q_IN_STAGE && c == sg.c0) ? (uint32_t)gv * D * 2u : 0u;
                 const uint32_t row_bytes = F8 ? (uint32_t)D : (uint32_t)C::NHALF * 128u;
                 mbar_arrive_expect_tx(&full[stage], nvalid * 2u * rb * row_bytes + qbytes);
                 if (qbytes)  // the group's q rows ride with the segment's first stage
@@ -430,9 +449,9 @@ __device__ __forceinline__ SegInfo seg_info(const DecodeParams& p, const Segment
 
 // ---- consumer (tensor-core math) ----------------------------------------------
 
-// Consumer `me` (0 .. NCONS-1).  bf16: reads every TMA stage in turn, K and V
-// as 16-bit swizzled tiles, the group's q from the segment's first stage.
-// fp8: takes the CTA's chunks n with n % NCONS == me (stage n % NSTAGE) and
+// Consumer `me` (0 .. NCONS-1): takes the CTA's chunks n with n % NCONS == me
+// (stage n % NSTAGE).  bf16: K and V as 16-bit swizzled tiles; the group's q
+// from the segment's first stage (one consumer) or from global memory.  fp8:
 // widens the e4m3 codes in registers: ldmatrix on byte pairs gives lane
 // (grp, tig) four consecutive codes of one token row, which one cvt per pair
 // turns into two f16x2 words.
@@ -449,8 +468,8 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                                         uint64_t* dfull, uint64_t* dempty, const int* st_ntok,
                                         const unsigned* st_bad, volatile int* ctrl, int lane,
                                         int me) {
-    using C = MmaCfg<D, NT, F8>;
-    using S = Smem<D, NT, F8>;
+    using C = MmaCfg<D, NT, F8, RC>;
+    using S = Smem<D, NT, F8, RC>;
     constexpr int GP = C::GP;
     const int grp = lane >> 2, tig = lane & 3;
     const int mi = lane >> 3, r8 = lane & 7;
@@ -458,8 +477,8 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
     const int k_row = r8 + 8 * (mi & 1), k_cx = mi >> 1;  // K (A operand); fp8: K and V
     const int v_row = r8 + 8 * (mi >> 1), v_cx = mi & 1;  // bf16 V^T (transposed load)
     Ring ring, dring;
-    unsigned n_chunk = 0;  // fp8: chunks of the CTA so far
-    bool waited = false;   // fp8: q is read from global memory
+    unsigned n_chunk = 0;  // several consumers: chunks of the CTA so far
+    bool waited = false;   // q read from global memory: after the grid dependency
     // bf16 stages: byte offsets of this lane's ldmatrix rows per token tile
     const int log2_rb = min(p.log2_bs, 6);
     int k_off[kMT], v_off[kMT];
@@ -489,14 +508,14 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
         }
 
         bool have_q = false;
-        if constexpr (F8 || RC) {
+        if constexpr (!C::Q_IN_STAGE || RC) {
             // Q^T B-fragments straight from global memory, head nt*8+grp.
             // fp8: the permuted order, dims 16 ks + 4 tig, +1 (b0) and
-            // 16 ks + 4 tig + 2, +3 (b1), widened bf16 -> f16.  Row copies: the
+            // 16 ks + 4 tig + 2, +3 (b1), widened bf16 -> f16.  bf16: the
             // natural order, dims 16 ks + 2 tig, +1 (b0) and + 8, + 9 (b1).
             // Only a consumer with a chunk of this segment needs them.
-            bool any = !F8;
-            if constexpr (F8)
+            bool any = C::NCONS == 1;
+            if constexpr (C::NCONS > 1)
                 for (unsigned n = n_chunk; n < n_chunk + (unsigned)(sg.c1 - sg.c0); ++n)
                     any |= (int)(n % C::NCONS) == me;
             if (any) {
@@ -531,7 +550,7 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
         for (int c = sg.c0; c < sg.c1; ++c) {
             int stage;
             uint32_t phase;
-            if constexpr (F8) {
+            if constexpr (C::NCONS > 1) {
                 const unsigned n = n_chunk++;
                 if ((int)(n % C::NCONS) != me) continue;
                 stage = (int)(n % C::NSTAGE);
@@ -553,7 +572,7 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
             unsigned char* sv = sk + (RC ? C::RC_KV_BYTES : C::KV_BYTES);
             const bool whole = ntok == kCH && bad == 0;
 
-            if (!F8 && !RC && !have_q) {
+            if (C::Q_IN_STAGE && !RC && !have_q) {
                 // The segment's first chunk carries the group's q.
                 // Q^T B-fragments: head nt*8+grp, dims ks*16 + 2*tig (+1) and +8 (+9).
                 have_q = true;
@@ -813,11 +832,11 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
             if (!F8 && !RC && !whole) fence_proxy_async_smem();  // our zero-fill before the next TMA write
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[stage]);
-            if constexpr (!F8) ring.advance(C::NSTAGE);
+            if constexpr (C::NCONS == 1) ring.advance(C::NSTAGE);
         }
 
         // ---- hand the segment's state to the epilogue warp ----
-        // (an fp8 consumer that took no chunk of the segment hands over the
+        // (a consumer that took no chunk of the segment hands over the
         // empty state)
         const int slot = me * S::NDUMP + dring.stage;
         if (!mbar_wait(&dempty[slot], dring.phase ^ 1u, p.wait_ns)) {
@@ -884,12 +903,12 @@ __device__ __forceinline__ void write_record(const DecodeParams& p, size_t rec, 
 
 // ---- epilogue: normalise, or write a partial record and merge the group ----
 
-template <int D, int NT, bool F8>
+template <int D, int NT, bool F8, bool RC>
 __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it,
                                          unsigned char* smem, uint64_t* dfull, uint64_t* dempty,
                                          volatile int* ctrl, int lane) {
-    using C = MmaCfg<D, NT, F8>;
-    using S = Smem<D, NT, F8>;
+    using C = MmaCfg<D, NT, F8, RC>;
+    using S = Smem<D, NT, F8, RC>;
     constexpr int GP = C::GP;
     const int grp = lane >> 2, tig = lane & 3;
     Ring dring;
@@ -1218,12 +1237,12 @@ __device__ __forceinline__ long long total_chunks_warp(const DecodeParams& p, in
 }
 
 template <int D, int NT, bool F8, bool RC>
-__global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
+__global__ void __launch_bounds__(MmaCfg<D, NT, F8, RC>::THREADS)
     decode_mma_kernel(const __grid_constant__ DecodeParams p,
                                                              const __grid_constant__ CUtensorMap tmk,
                                                              const __grid_constant__ CUtensorMap tmv) {
-    using C = MmaCfg<D, NT, F8>;
-    using S = Smem<D, NT, F8>;
+    using C = MmaCfg<D, NT, F8, RC>;
+    using S = Smem<D, NT, F8, RC>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
@@ -1281,7 +1300,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
         if (warp == C::NPROD + C::NCONS) {
             SegIter<kCH> none;
             none.valid = false;
-            epilogue<D, NT, F8>(p, none, smem, dfull, dempty, ctrl, lane);
+            epilogue<D, NT, F8, RC>(p, none, smem, dfull, dempty, ctrl, lane);
         }
         return;
     }
@@ -1301,7 +1320,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8>::THREADS)
         consume<D, NT, F8, RC>(p, it, smem, full, empty, dfull, dempty, st_ntok, st_bad, ctrl, lane,
                            warp - C::NPROD);
     } else {
-        epilogue<D, NT, F8>(p, it, smem, dfull, dempty, ctrl, lane);
+        epilogue<D, NT, F8, RC>(p, it, smem, dfull, dempty, ctrl, lane);
     }
 }
 
@@ -1454,8 +1473,8 @@ __global__ void __launch_bounds__(32 * kMergeWarps)
 
 template <int D, int NT, bool F8, bool RC>
 pkv_status launch_impl(const DecodeParams& p, cudaStream_t stream, int* grid_out) {
-    using C = MmaCfg<D, NT, F8>;
-    using S = Smem<D, NT, F8>;
+    using C = MmaCfg<D, NT, F8, RC>;
+    using S = Smem<D, NT, F8, RC>;
     const DeviceInfo* di = current_device_info();
     if (!di) return PKV_ERR_CUDA;
     static std::mutex mu;
