@@ -41,6 +41,8 @@ WORKLOAD = "gqa_4k: batch 16 x 4096 tokens, 32 q / 8 KV heads, head_dim 128, blo
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0  # the B200's ~8 TB/s HBM3e figure, for the nominal fraction
 ROOFLINE_LAUNCHES = 2000  # decode-only launches timed for the roofline, whatever --steps
+DEC_RUN = 20               # back-to-back decode launches per timed graph (roofline)
+ISOLATED_LAUNCHES = 200    # single decode launches timed on their own (latency)
 N_LAYERS = 4
 DECODE_SRC = os.path.join(ROOT, "paged_kv_cache_412_b200", "csrc", "decode_mma.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_gqa_4k_traffic.txt")
@@ -376,54 +378,84 @@ def run_ours(args, rank: int, world: int, local: int):
     torch.cuda.synchronize()
     assert pkv.get_device_error() == 0
 
-    # one CUDA graph per layer pool: the whole step, and the decode alone
-    def capture(t, with_write):
+    # A decode iteration of a model runs the step once per layer, back to
+    # back: one CUDA graph holds a sweep over the N_LAYERS layer pools (a step
+    # per layer), so consecutive kernels overlap through programmatic
+    # dependent launch as they would in the serving loop; a second graph holds
+    # the first K % N_LAYERS steps of a sweep.
+    def capture(steps, with_write):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            step_body(t, with_write)
+            for li in range(steps):
+                step_body(layers[li % N_LAYERS], with_write)
         return g
-    step_graphs = [capture(t, True) for t in layers]
-    dec_graphs = [capture(t, False) for t in layers]
-    for i in range(args.warmup):
-        step_graphs[i % N_LAYERS].replay()
+    sweep = capture(N_LAYERS, True)
+    n_sweeps, rest = divmod(args.steps, N_LAYERS)
+    part = capture(rest, True) if rest else None
+    for _ in range(max(1, -(-args.warmup // N_LAYERS))):
+        sweep.replay()
     torch.cuda.synchronize()
 
     # --- timed region: K steps (graph replays), device-timed ---
     sampler = ClockSampler(dev.index if dev.index is not None else 0, args.clocks_csv or None)
-    bounds = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+    bounds = [torch.cuda.Event(enable_timing=True) for _ in range(n_sweeps + 2)]
     sampler.start()
     time.sleep(0.3)
     dist_barrier(world)
     torch.cuda.synchronize()
     torch.cuda.nvtx.range_push("timed steps")
     bounds[0].record()
-    for i in range(args.steps):
-        step_graphs[i % N_LAYERS].replay()
+    for i in range(n_sweeps):
+        sweep.replay()
         bounds[i + 1].record()
+    if part is not None:
+        part.replay()
+    bounds[n_sweeps + 1].record()
     torch.cuda.synchronize()
     torch.cuda.nvtx.range_pop()
     dist_barrier(world)
     clocks = sampler.stop()
     ms_total = bounds[0].elapsed_time(bounds[-1])
-    step_ms = [bounds[i].elapsed_time(bounds[i + 1]) for i in range(args.steps)]
+    # per-step time of each full sweep (the partial sweep only counts in the total)
+    step_ms = [bounds[i].elapsed_time(bounds[i + 1]) / N_LAYERS for i in range(n_sweeps)] or \
+              [ms_total / args.steps]
     ms_total_max = dist_max(ms_total, world)
     ms_step = ms_total_max / args.steps
+    del sweep, part
 
-    # --- the decode kernel alone, events around every launch (roofline) ---
-    # a fixed number of launches, whatever --steps is
-    n_dec = ROOFLINE_LAUNCHES
-    dev_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-              for _ in range(n_dec)]
+    # --- the decode kernel alone (roofline), a fixed number of launches ---
+    # Throughput: graphs of DEC_RUN back-to-back decode launches over the layer
+    # pools, events around each graph; the launch duration is the graph's time
+    # over DEC_RUN.  Latency of one launch on its own (events around a graph
+    # of one launch) is reported beside it.
+    dec_run = capture(DEC_RUN, False)
+    dec_one = [capture(1, False) for _ in range(1)]
+    n_runs = -(-ROOFLINE_LAUNCHES // DEC_RUN)
+    n_dec = n_runs * DEC_RUN
+    for _ in range(3):
+        dec_run.replay()
     torch.cuda.synchronize()
-    torch.cuda.nvtx.range_push("roofline: decode-only graph replays")
-    for i in range(n_dec):
-        dev_ev[i][0].record()
-        dec_graphs[i % N_LAYERS].replay()
-        dev_ev[i][1].record()
+    dev_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(n_runs)]
+    torch.cuda.nvtx.range_push("roofline: back-to-back decode launches")
+    for a, b in dev_ev:
+        a.record()
+        dec_run.replay()
+        b.record()
     torch.cuda.synchronize()
     torch.cuda.nvtx.range_pop()
-    decode_ms = [a.elapsed_time(b) for a, b in dev_ev]
-    del step_graphs, dec_graphs
+    decode_ms = [a.elapsed_time(b) / DEC_RUN for a, b in dev_ev]
+    iso_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(ISOLATED_LAUNCHES)]
+    torch.cuda.nvtx.range_push("decode launches on their own")
+    for a, b in iso_ev:
+        a.record()
+        dec_one[0].replay()
+        b.record()
+    torch.cuda.synchronize()
+    torch.cuda.nvtx.range_pop()
+    iso_ms = statistics.fmean(a.elapsed_time(b) for a, b in iso_ev)
+    del dec_run, dec_one
 
     dbytes = decode_bytes(B, L, Hq, Hkv, d)
     wbytes = write_bytes(B, Hkv, d)
@@ -556,7 +588,9 @@ def run_ours(args, rank: int, world: int, local: int):
                              f"{2 * B * L * Hkv * d * 2 / 1e6:.0f} MB K+V rotated per step",
                        "parallelism": f"replica x{world}" if world > 1 else "single GPU",
                        "step": "copy_blocks (0 pairs) + kv_cache_write (16 tokens) + "
-                               "paged_attention_decode, one CUDA graph per layer pool"},
+                               "paged_attention_decode; the steps of a sweep over the "
+                               f"{N_LAYERS} layer pools captured in one CUDA graph and "
+                               "replayed back to back"},
             "tokens_per_s": round(B * world * args.steps / (ms_total_max / 1e3), 1),
             "context_tokens_per_s": round(B * L * world * args.steps / (ms_total_max / 1e3), 1),
             "fraction_of_hbm_peak": round(value / peak, 4),
@@ -565,13 +599,19 @@ def run_ours(args, rank: int, world: int, local: int):
             "step_ms_median": round(statistics.median(step_ms), 5),
             "decode_ms_avg": round(dec_avg_ms, 5), "decode_ms_median": round(dec_med_ms, 5),
             "decode_launches_timed": n_dec,
+            "decode_isolated": {"ms_avg": round(iso_ms, 5), "launches": ISOLATED_LAUNCHES,
+                                "GBps": round(dbytes / (iso_ms / 1e3) / 1e9, 2),
+                                "note": "one decode launch on its own between events (its "
+                                        "launch latency, planning and ramp not overlapped "
+                                        "with a previous kernel)"},
             "bytes_per_step": {"decode_algorithmic": dbytes, "write": wbytes},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "traffic": traffic_per_launch(),
                          "kernel": "decode_mma_kernel (split decode with in-kernel merge)",
-                         "duration": "mean of CUDA-event intervals around each decode launch "
-                                     "(decode-only graph replays after the timed steps)",
+                         "duration": f"per-launch mean of graphs of {DEC_RUN} back-to-back "
+                                     "decode launches over the layer pools (events around "
+                                     "each graph), after the timed steps",
                          "peak_kind": f"{peak_kind} HBM copy bandwidth"},
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,

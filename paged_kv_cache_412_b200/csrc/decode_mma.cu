@@ -65,7 +65,7 @@ constexpr int clcm(int a, int b) { return a / cgcd(a, b) * b; }
 //             (TMA boxes with the swizzle of their width) and every consumer
 //             widens what it loads from them to f16 in registers (exact), for
 //             f16 MMAs; q is widened to f16 likewise.
-template <int D, int NT, bool F8, bool RC = false>
+template <int D, int NT, bool F8, bool SOLO = false>
 struct MmaCfg {
     static constexpr int NHALF = D / 64;            // 128-byte column halves of a 16-bit row
     static constexpr int KS = D / 16;               // k-steps of q.K^T, m-tiles of P.V
@@ -84,21 +84,24 @@ struct MmaCfg {
     //     as a (request, kv head) group (64): most groups split into two
     //     parts, one of which finishes early and is prefetched by the other's
     //     merge -- with two CTAs per SM a group's middle parts end with the
-    //     kernel and the last merges wait for them.  (Row copies keep two
-    //     CTAs per SM with one consumer: their producer issues 64 copies per
-    //     chunk, and one producer per SM cannot keep up.)
+    //     kernel and the last merges wait for them.  SOLO keeps two CTAs
+    //     per SM with one consumer each: row copies (their producer issues 64
+    //     copies per chunk; one producer per SM cannot keep up) and calls of
+    //     many (request, head group) pairs, where few groups split and two
+    //     epilogue warps per SM share the many short segments.
     //   fp8: widening codes costs instructions and latency the bf16 path does
     //     not have, and one consumer warp cannot hide its own ldmatrix -> cvt
     //     -> mma chains: six consumers (two on each of two SM sub-partitions)
     //     overlap them; the 16-head configuration keeps four (its consumers
     //     need all the registers).
-    static constexpr int NCONS = F8 ? (NT == 1 ? 6 : 4) : (NT == 1 && !RC ? 2 : 1);
-    // bf16 with one consumer: K | V | q, rounded to the 1 KB the 128-byte
-    // swizzle pattern repeats on (the segment's first stage carries q).
-    // Otherwise each consumer reads the group's q from global memory: fp8
-    // K | V only (8 or 4 KB each, whole swizzle periods); bf16 K | V, or the
-    // row-copy regions if larger.
-    static constexpr bool Q_IN_STAGE = !F8 && NCONS == 1;
+    static constexpr int NCONS = F8 ? (NT == 1 ? 6 : 4) : (NT == 1 && !SOLO ? 2 : 1);
+    // bf16: K | V | q, rounded to the 1 KB the 128-byte swizzle pattern
+    // repeats on, or the row-copy regions if larger; the first NCONS stages
+    // of a segment -- each consumer's first chunk of it -- carry the group's q
+    // (row copies: the consumer reads it from global memory).  fp8: K | V only
+    // (8 or 4 KB each, whole swizzle periods); each consumer reads the group's
+    // q from global memory.
+    static constexpr bool Q_IN_STAGE = !F8;
     // row-copy stages (bf16 blocks of 2 or 4 rows): K | V regions of up to 32
     // skewed blocks (rc_block_bytes), inside the same stage size
     static constexpr int RC_KV_BYTES = kCH * D * 2 + 32 * 16;
@@ -110,15 +113,20 @@ struct MmaCfg {
     // warp issues at most ~9 boxes per us however its lanes share them.  An
     // fp8 chunk is 8 boxes of 2 KB; four producers take chunks in turn (stage
     // n % NSTAGE belongs to producer n % NPROD), enough to keep 12 stages in
-    // flight.  The 16-head configuration keeps two (registers).  bf16: one.
-    static constexpr int NPROD = F8 ? (NT == 1 ? 4 : 2) : 1;
+    // flight.  The 16-head configuration keeps two (registers).  bf16 with one
+    // CTA per SM: two (a chunk of 8-row blocks is 16 boxes); two CTAs: one each.
+    static constexpr int NPROD = F8 ? (NT == 1 ? 4 : 2) : (NCONS > 1 ? 2 : 1);
     static constexpr int THREADS = 32 * (NPROD + NCONS + 1);  // + the epilogue
-    // consumer -> epilogue hand-off: per lane, the accumulators and (m, l)
+    // consumer -> epilogue hand-off: per lane, the accumulators and (m, l);
+    // NDUMP slots per consumer (two, so a consumer can hand over a short
+    // segment while the epilogue still merges the previous one, where the
+    // shared memory allows)
     static constexpr int DUMP_BYTES = (KS * NT * 4 + NT * 4) * 32 * 4;
+    static constexpr int NDUMP = NCONS <= 2 ? 2 : 1;
     // One CTA per SM: as many stages as the shared memory holds beside the
     // hand-off slots (up to 24), a multiple of NCONS and NPROD: 192 KB or
     // more in flight per SM at head_dim 128.
-    static constexpr int RING = 227 * 1024 - NCONS * DUMP_BYTES - 4096;
+    static constexpr int RING = 227 * 1024 - NCONS * NDUMP * DUMP_BYTES - 4096;
     static constexpr int STAGE_STEP = clcm(NCONS, NPROD);
     static constexpr int NSTAGE = NCONS == 1 ? cmax(2, cmin(8, kRingBudget / STAGE_BYTES))
                                              : cmin(24, RING / STAGE_BYTES) / STAGE_STEP * STAGE_STEP;
@@ -128,11 +136,11 @@ struct MmaCfg {
 
 // ---- shared-memory layout ------------------------------------------------------
 
-template <int D, int NT, bool F8, bool RC = false>
+template <int D, int NT, bool F8, bool SOLO = false>
 struct Smem {
-    using C = MmaCfg<D, NT, F8, RC>;
+    using C = MmaCfg<D, NT, F8, SOLO>;
     // consumer -> epilogue hand-off slots per consumer
-    static constexpr int NDUMP = C::NCONS == 1 ? 2 : 1;
+    static constexpr int NDUMP = C::NDUMP;
     static constexpr int NSLOT = C::NCONS * NDUMP;
     static constexpr int DUMP_ACC = C::KS * NT * 4;       // acc registers per lane
     static constexpr int DUMP_ML = NT * 4;                // m[2], l[2] per n-tile per lane
@@ -209,9 +217,9 @@ __device__ __forceinline__ int bf16_row_off(int t, int half, int log2_rb) {
 
 // RC: blocks of 2 or 4 rows (bf16), copied row by row instead of by TMA boxes;
 // a separate instance so the boxed producer carries no trace of it.
-template <int D, int NT, bool F8, bool RC>
+template <int D, int NT, bool F8, bool RC, bool SOLO>
 struct Producer {
-    using C = MmaCfg<D, NT, F8, RC>;
+    using C = MmaCfg<D, NT, F8, SOLO>;
     static_assert(!(RC && F8), "row copies serve bf16 caches only");
 
     const DecodeParams& p;
@@ -340,10 +348,12 @@ struct Producer {
                 st_ntok[stage] = ntok;
                 st_bad[stage] = bad;
                 if (bad) raise_error(p.err, PKV_DEVERR_BAD_BLOCK);
-                const uint32_t qbytes = (C::Q_IN_STAGE && c == sg.c0) ? (uint32_t)gv * D * 2u : 0u;
+                // each consumer's first chunk of the segment carries q
+                const uint32_t qbytes =
+                    (C::Q_IN_STAGE && c - sg.c0 < C::NCONS) ? (uint32_t)gv * D * 2u : 0u;
                 const uint32_t row_bytes = F8 ? (uint32_t)D : (uint32_t)C::NHALF * 128u;
                 mbar_arrive_expect_tx(&full[stage], nvalid * 2u * rb * row_bytes + qbytes);
-                if (qbytes)  // the group's q rows ride with the segment's first stage
+                if (qbytes)  // the group's q rows ride with the stage
                     bulk_load(sq, static_cast<const __nv_bfloat16*>(p.q) +
                                       ((size_t)cur.b * p.num_q_heads + hq0) * D,
                               qbytes, &full[stage], policy);
@@ -462,14 +472,14 @@ __device__ __forceinline__ SegInfo seg_info(const DecodeParams& p, const Segment
 //   P.V: the widened words are 8 x 8 tiles with tokens as rows; movmatrix.trans
 //     makes them A fragments of V^T with tokens as k, and the head-dim rows
 //     come out permuted as dcol<true> describes.
-template <int D, int NT, bool F8, bool RC>
+template <int D, int NT, bool F8, bool RC, bool SOLO>
 __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                                         unsigned char* smem, uint64_t* full, uint64_t* empty,
                                         uint64_t* dfull, uint64_t* dempty, const int* st_ntok,
                                         const unsigned* st_bad, volatile int* ctrl, int lane,
                                         int me) {
-    using C = MmaCfg<D, NT, F8, RC>;
-    using S = Smem<D, NT, F8, RC>;
+    using C = MmaCfg<D, NT, F8, SOLO>;
+    using S = Smem<D, NT, F8, SOLO>;
     constexpr int GP = C::GP;
     const int grp = lane >> 2, tig = lane & 3;
     const int mi = lane >> 3, r8 = lane & 7;
@@ -573,7 +583,7 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
             const bool whole = ntok == kCH && bad == 0;
 
             if (C::Q_IN_STAGE && !RC && !have_q) {
-                // The segment's first chunk carries the group's q.
+                // This consumer's first chunk of the segment carries the group's q.
                 // Q^T B-fragments: head nt*8+grp, dims ks*16 + 2*tig (+1) and +8 (+9).
                 have_q = true;
                 const uint32_t* sq = reinterpret_cast<const uint32_t*>(sv + C::KV_BYTES);
@@ -903,12 +913,12 @@ __device__ __forceinline__ void write_record(const DecodeParams& p, size_t rec, 
 
 // ---- epilogue: normalise, or write a partial record and merge the group ----
 
-template <int D, int NT, bool F8, bool RC>
+template <int D, int NT, bool F8, bool RC, bool SOLO>
 __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it,
                                          unsigned char* smem, uint64_t* dfull, uint64_t* dempty,
                                          volatile int* ctrl, int lane) {
-    using C = MmaCfg<D, NT, F8, RC>;
-    using S = Smem<D, NT, F8, RC>;
+    using C = MmaCfg<D, NT, F8, SOLO>;
+    using S = Smem<D, NT, F8, SOLO>;
     constexpr int GP = C::GP;
     const int grp = lane >> 2, tig = lane & 3;
     Ring dring;
@@ -1236,13 +1246,13 @@ __device__ __forceinline__ long long total_chunks_warp(const DecodeParams& p, in
     return t * p.num_hg;
 }
 
-template <int D, int NT, bool F8, bool RC>
-__global__ void __launch_bounds__(MmaCfg<D, NT, F8, RC>::THREADS)
+template <int D, int NT, bool F8, bool RC, bool SOLO>
+__global__ void __launch_bounds__(MmaCfg<D, NT, F8, SOLO>::THREADS)
     decode_mma_kernel(const __grid_constant__ DecodeParams p,
                                                              const __grid_constant__ CUtensorMap tmk,
                                                              const __grid_constant__ CUtensorMap tmv) {
-    using C = MmaCfg<D, NT, F8, RC>;
-    using S = Smem<D, NT, F8, RC>;
+    using C = MmaCfg<D, NT, F8, SOLO>;
+    using S = Smem<D, NT, F8, SOLO>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
@@ -1300,7 +1310,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8, RC>::THREADS)
         if (warp == C::NPROD + C::NCONS) {
             SegIter<kCH> none;
             none.valid = false;
-            epilogue<D, NT, F8, RC>(p, none, smem, dfull, dempty, ctrl, lane);
+            epilogue<D, NT, F8, RC, SOLO>(p, none, smem, dfull, dempty, ctrl, lane);
         }
         return;
     }
@@ -1311,16 +1321,16 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8, RC>::THREADS)
 
     // warps: producers | consumers | epilogue
     if (warp < C::NPROD) {
-        Producer<D, NT, F8, RC> pr{p, &tmk, &tmv, smem, full, empty, st_ntok, st_bad, ctrl, lane,
+        Producer<D, NT, F8, RC, SOLO> pr{p, &tmk, &tmv, smem, full, empty, st_ntok, st_bad, ctrl, lane,
                            l2_policy_evict_first()};
         pr.me = warp;
         pr.run(it, spec_b, spec_j, spec_tab);
         if (!pr.waited) griddep_wait();
     } else if (warp < C::NPROD + C::NCONS) {
-        consume<D, NT, F8, RC>(p, it, smem, full, empty, dfull, dempty, st_ntok, st_bad, ctrl, lane,
+        consume<D, NT, F8, RC, SOLO>(p, it, smem, full, empty, dfull, dempty, st_ntok, st_bad, ctrl, lane,
                            warp - C::NPROD);
     } else {
-        epilogue<D, NT, F8, RC>(p, it, smem, dfull, dempty, ctrl, lane);
+        epilogue<D, NT, F8, RC, SOLO>(p, it, smem, dfull, dempty, ctrl, lane);
     }
 }
 
@@ -1471,15 +1481,15 @@ __global__ void __launch_bounds__(32 * kMergeWarps)
 
 // ---- host side ---------------------------------------------------------------
 
-template <int D, int NT, bool F8, bool RC>
+template <int D, int NT, bool F8, bool RC, bool SOLO>
 pkv_status launch_impl(const DecodeParams& p, cudaStream_t stream, int* grid_out) {
-    using C = MmaCfg<D, NT, F8, RC>;
-    using S = Smem<D, NT, F8, RC>;
+    using C = MmaCfg<D, NT, F8, SOLO>;
+    using S = Smem<D, NT, F8, SOLO>;
     const DeviceInfo* di = current_device_info();
     if (!di) return PKV_ERR_CUDA;
     static std::mutex mu;
     static int occupancy[64] = {0};
-    auto kern = decode_mma_kernel<D, NT, F8, RC>;
+    auto kern = decode_mma_kernel<D, NT, F8, RC, SOLO>;
     {
         std::lock_guard<std::mutex> lock(mu);
         if (di->device >= 64) return PKV_ERR_UNSUPPORTED;
@@ -1616,22 +1626,33 @@ bool decode_mma_supported(int head_dim, int block_size, pkv_dtype q_dtype, pkv_d
 pkv_status launch_decode_mma(const DecodeParams& p, int head_dim, int group_pad, bool fp8,
                              cudaStream_t stream, int* grid_out) {
     const int nt = group_pad > 8 ? 2 : 1;
+    // bf16 with TMA boxes, 8-head groups: one CTA per SM with two consumers,
+    // unless the call has at least four (request, head group) pairs per SM --
+    // then few of them split, and two CTAs per SM (one consumer and one
+    // epilogue warp each) share the many short segments better.
+    const DeviceInfo* di = current_device_info();
+    if (!di) return PKV_ERR_CUDA;
+    const bool many = (long long)p.num_seqs * p.num_hg >= 4LL * di->num_sms;
     if (fp8) {
         if (p.row_copy) return PKV_ERR_UNSUPPORTED;
-        if (head_dim == 128) return nt == 1 ? launch_impl<128, 1, true, false>(p, stream, grid_out)
-                                            : launch_impl<128, 2, true, false>(p, stream, grid_out);
-        if (head_dim == 64) return nt == 1 ? launch_impl<64, 1, true, false>(p, stream, grid_out)
-                                           : launch_impl<64, 2, true, false>(p, stream, grid_out);
+        if (head_dim == 128) return nt == 1 ? launch_impl<128, 1, true, false, false>(p, stream, grid_out)
+                                            : launch_impl<128, 2, true, false, false>(p, stream, grid_out);
+        if (head_dim == 64) return nt == 1 ? launch_impl<64, 1, true, false, false>(p, stream, grid_out)
+                                           : launch_impl<64, 2, true, false, false>(p, stream, grid_out);
     } else if (p.row_copy) {
-        if (head_dim == 128) return nt == 1 ? launch_impl<128, 1, false, true>(p, stream, grid_out)
-                                            : launch_impl<128, 2, false, true>(p, stream, grid_out);
-        if (head_dim == 64) return nt == 1 ? launch_impl<64, 1, false, true>(p, stream, grid_out)
-                                           : launch_impl<64, 2, false, true>(p, stream, grid_out);
+        if (head_dim == 128) return nt == 1 ? launch_impl<128, 1, false, true, true>(p, stream, grid_out)
+                                            : launch_impl<128, 2, false, true, true>(p, stream, grid_out);
+        if (head_dim == 64) return nt == 1 ? launch_impl<64, 1, false, true, true>(p, stream, grid_out)
+                                           : launch_impl<64, 2, false, true, true>(p, stream, grid_out);
     } else {
-        if (head_dim == 128) return nt == 1 ? launch_impl<128, 1, false, false>(p, stream, grid_out)
-                                            : launch_impl<128, 2, false, false>(p, stream, grid_out);
-        if (head_dim == 64) return nt == 1 ? launch_impl<64, 1, false, false>(p, stream, grid_out)
-                                           : launch_impl<64, 2, false, false>(p, stream, grid_out);
+        if (head_dim == 128)
+            return nt == 2 ? launch_impl<128, 2, false, false, true>(p, stream, grid_out)
+                   : many  ? launch_impl<128, 1, false, false, true>(p, stream, grid_out)
+                           : launch_impl<128, 1, false, false, false>(p, stream, grid_out);
+        if (head_dim == 64)
+            return nt == 2 ? launch_impl<64, 2, false, false, true>(p, stream, grid_out)
+                   : many  ? launch_impl<64, 1, false, false, true>(p, stream, grid_out)
+                           : launch_impl<64, 1, false, false, false>(p, stream, grid_out);
     }
     return PKV_ERR_UNSUPPORTED;
 }
