@@ -701,6 +701,36 @@ def _time_graph(fn, iters, flush, warm=5):
     return statistics.fmean(ms), statistics.median(ms)
 
 
+B2B_RUN = 20    # launches per graph, back-to-back timing of the suite
+B2B_POOLS = 4   # copies of the caches the launches rotate over
+
+
+def _time_back_to_back(fn, run, reps):
+    """Median per-launch time (ms) of graphs of ``run`` launches fn(0) .. fn(run-1)
+    issued back to back, CUDA events around each graph."""
+    import torch
+    for i in range(2):
+        fn(i)
+    torch.cuda.synchronize()
+    _device_clean()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for i in range(run):
+            fn(i)
+    for _ in range(2):
+        g.replay()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(reps)]
+    for a, b in ev:
+        a.record()
+        g.replay()
+        b.record()
+    torch.cuda.synchronize()
+    del g
+    return statistics.median(a.elapsed_time(b) / run for a, b in ev)
+
+
 def _dev_workload(w, dev):
     import torch
 
@@ -750,19 +780,30 @@ def run_suite(args):
         ws = pkv.new_workspace(pkv.decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.d, w.bs, L,
                                                           partition_size), dev)
 
-        def fn():
-            pkv.paged_attention_decode(t["q"], t["kc"], t["vc"], t["bt"], t["sl"], w.bs,
+        def fn(kc=t["kc"], vc=t["vc"]):
+            pkv.paged_attention_decode(t["q"], kc, vc, t["bt"], t["sl"], w.bs,
                                        w.scale, out, max_seq_len=L, workspace=ws,
                                        partition_size=partition_size, k_scale=t["ks"],
                                        v_scale=t["vs"])
         ms = _time_graph(fn, iters, flush)
+        assert pkv.get_device_error() == 0
+        # back to back: graphs of B2B_RUN launches over B2B_POOLS copies of the
+        # caches (more than L2 holds), events around each graph
+        pools = [(t["kc"], t["vc"])] + [(t["kc"].clone(), t["vc"].clone())
+                                        for _ in range(B2B_POOLS - 1)]
+        b2b = _time_back_to_back(lambda i: fn(*pools[i % B2B_POOLS]), B2B_RUN, 10)
+        del pools
         assert pkv.get_device_error() == 0
         e_kv = 1 if fp8 else 2
         nbytes = (2 * int(w.seq_lens.astype(np.int64).sum()) * w.Hkv * w.d * e_kv
                   + w.B * w.Hq * w.d * 4)
         info = {"B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "block_size": w.bs,
                 "kv_dtype": "fp8_e4m3" if fp8 else "bf16", "partition_size": partition_size,
-                "context_tokens": int(w.seq_lens.astype(np.int64).sum())}
+                "context_tokens": int(w.seq_lens.astype(np.int64).sum()),
+                "us_back_to_back": round(b2b * 1e3, 2),
+                "GBps_back_to_back": round(nbytes / (b2b / 1e3) / 1e9, 1),
+                "back_to_back": f"graphs of {B2B_RUN} launches over {B2B_POOLS} copies of "
+                                "the caches, median per launch"}
         info.update(extra or {})
         emit(name, ms, nbytes, info)
         del t, ws, out
