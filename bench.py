@@ -829,11 +829,14 @@ def run_suite(args):
                             partition_size=P)
             del wl
     if want("small_blocks"):
-        # block size 4: tensor-core decode fed by per-lane row copies (blocks of
-        # fewer than 8 rows cannot be 128-byte-swizzled TMA boxes)
-        w = workloads.make_paged([4096] * 16, Hq=32, Hkv=8, d=128, bs=4, dtype="bf16",
-                                 seed=1002, poison=False, name="gqa_4k_bs4")
-        decode_case("decode 4k batch, block 4 (row copies)", w)
+        # block sizes 4 and 2: tensor-core decode fed by one bulk copy per
+        # (block, K or V) (blocks of fewer than 8 rows cannot be
+        # 128-byte-swizzled TMA boxes)
+        for bs in (4, 2):
+            w = workloads.make_paged([4096] * 16, Hq=32, Hkv=8, d=128, bs=bs, dtype="bf16",
+                                     seed=1002, poison=False, name=f"gqa_4k_bs{bs}")
+            decode_case(f"decode 4k batch, block {bs} (row copies)", w)
+            del w
     if want("prefix"):
         _suite_prefix(pkv, torch, workloads, dev, iters, flush, emit)
     if want("cache_ops"):

@@ -65,7 +65,7 @@ constexpr int clcm(int a, int b) { return a / cgcd(a, b) * b; }
 //             (TMA boxes with the swizzle of their width) and every consumer
 //             widens what it loads from them to f16 in registers (exact), for
 //             f16 MMAs; q is widened to f16 likewise.
-template <int D, int NT, bool F8, bool SOLO = false>
+template <int D, int NT, bool F8, bool SOLO = false, bool RC = false>
 struct MmaCfg {
     static constexpr int NHALF = D / 64;            // 128-byte column halves of a 16-bit row
     static constexpr int KS = D / 16;               // k-steps of q.K^T, m-tiles of P.V
@@ -85,10 +85,9 @@ struct MmaCfg {
     //     parts, one of which finishes early and is prefetched by the other's
     //     merge -- with two CTAs per SM a group's middle parts end with the
     //     kernel and the last merges wait for them.  SOLO keeps two CTAs
-    //     per SM with one consumer each: row copies (their producer issues 64
-    //     copies per chunk; one producer per SM cannot keep up) and calls of
-    //     many (request, head group) pairs, where few groups split and two
-    //     epilogue warps per SM share the many short segments.
+    //     per SM with one consumer each, for calls of many (request, head
+    //     group) pairs, where few groups split and two epilogue warps per SM
+    //     share the many short segments.
     //   fp8: widening codes costs instructions and latency the bf16 path does
     //     not have, and one consumer warp cannot hide its own ldmatrix -> cvt
     //     -> mma chains: six consumers (two on each of two SM sub-partitions)
@@ -114,8 +113,9 @@ struct MmaCfg {
     // fp8 chunk is 8 boxes of 2 KB; four producers take chunks in turn (stage
     // n % NSTAGE belongs to producer n % NPROD), enough to keep 12 stages in
     // flight.  The 16-head configuration keeps two (registers).  bf16 with one
-    // CTA per SM: two (a chunk of 8-row blocks is 16 boxes); two CTAs: one each.
-    static constexpr int NPROD = F8 ? (NT == 1 ? 4 : 2) : (NCONS > 1 ? 2 : 1);
+    // CTA per SM: two (a chunk of 8-row blocks is 16 boxes), three for row
+    // copies (32 or 64 bulk copies per chunk); two CTAs: one each.
+    static constexpr int NPROD = F8 ? (NT == 1 ? 4 : 2) : (NCONS > 1 ? (RC ? 3 : 2) : 1);
     static constexpr int THREADS = 32 * (NPROD + NCONS + 1);  // + the epilogue
     // consumer -> epilogue hand-off: per lane, the accumulators and (m, l);
     // NDUMP slots per consumer (two, so a consumer can hand over a short
@@ -136,9 +136,9 @@ struct MmaCfg {
 
 // ---- shared-memory layout ------------------------------------------------------
 
-template <int D, int NT, bool F8, bool SOLO = false>
+template <int D, int NT, bool F8, bool SOLO = false, bool RC = false>
 struct Smem {
-    using C = MmaCfg<D, NT, F8, SOLO>;
+    using C = MmaCfg<D, NT, F8, SOLO, RC>;
     // consumer -> epilogue hand-off slots per consumer
     static constexpr int NDUMP = C::NDUMP;
     static constexpr int NSLOT = C::NCONS * NDUMP;
@@ -219,7 +219,7 @@ __device__ __forceinline__ int bf16_row_off(int t, int half, int log2_rb) {
 // a separate instance so the boxed producer carries no trace of it.
 template <int D, int NT, bool F8, bool RC, bool SOLO>
 struct Producer {
-    using C = MmaCfg<D, NT, F8, SOLO>;
+    using C = MmaCfg<D, NT, F8, SOLO, RC>;
     static_assert(!(RC && F8), "row copies serve bf16 caches only");
 
     const DecodeParams& p;
@@ -478,8 +478,8 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                                         uint64_t* dfull, uint64_t* dempty, const int* st_ntok,
                                         const unsigned* st_bad, volatile int* ctrl, int lane,
                                         int me) {
-    using C = MmaCfg<D, NT, F8, SOLO>;
-    using S = Smem<D, NT, F8, SOLO>;
+    using C = MmaCfg<D, NT, F8, SOLO, RC>;
+    using S = Smem<D, NT, F8, SOLO, RC>;
     constexpr int GP = C::GP;
     const int grp = lane >> 2, tig = lane & 3;
     const int mi = lane >> 3, r8 = lane & 7;
@@ -917,8 +917,8 @@ template <int D, int NT, bool F8, bool RC, bool SOLO>
 __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it,
                                          unsigned char* smem, uint64_t* dfull, uint64_t* dempty,
                                          volatile int* ctrl, int lane) {
-    using C = MmaCfg<D, NT, F8, SOLO>;
-    using S = Smem<D, NT, F8, SOLO>;
+    using C = MmaCfg<D, NT, F8, SOLO, RC>;
+    using S = Smem<D, NT, F8, SOLO, RC>;
     constexpr int GP = C::GP;
     const int grp = lane >> 2, tig = lane & 3;
     Ring dring;
@@ -1247,12 +1247,12 @@ __device__ __forceinline__ long long total_chunks_warp(const DecodeParams& p, in
 }
 
 template <int D, int NT, bool F8, bool RC, bool SOLO>
-__global__ void __launch_bounds__(MmaCfg<D, NT, F8, SOLO>::THREADS)
+__global__ void __launch_bounds__(MmaCfg<D, NT, F8, SOLO, RC>::THREADS)
     decode_mma_kernel(const __grid_constant__ DecodeParams p,
                                                              const __grid_constant__ CUtensorMap tmk,
                                                              const __grid_constant__ CUtensorMap tmv) {
-    using C = MmaCfg<D, NT, F8, SOLO>;
-    using S = Smem<D, NT, F8, SOLO>;
+    using C = MmaCfg<D, NT, F8, SOLO, RC>;
+    using S = Smem<D, NT, F8, SOLO, RC>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char* smem = smem_raw + ((1024 - (smem_addr(smem_raw) & 1023)) & 1023);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
@@ -1483,8 +1483,8 @@ __global__ void __launch_bounds__(32 * kMergeWarps)
 
 template <int D, int NT, bool F8, bool RC, bool SOLO>
 pkv_status launch_impl(const DecodeParams& p, cudaStream_t stream, int* grid_out) {
-    using C = MmaCfg<D, NT, F8, SOLO>;
-    using S = Smem<D, NT, F8, SOLO>;
+    using C = MmaCfg<D, NT, F8, SOLO, RC>;
+    using S = Smem<D, NT, F8, SOLO, RC>;
     const DeviceInfo* di = current_device_info();
     if (!di) return PKV_ERR_CUDA;
     static std::mutex mu;
@@ -1626,8 +1626,8 @@ bool decode_mma_supported(int head_dim, int block_size, pkv_dtype q_dtype, pkv_d
 pkv_status launch_decode_mma(const DecodeParams& p, int head_dim, int group_pad, bool fp8,
                              cudaStream_t stream, int* grid_out) {
     const int nt = group_pad > 8 ? 2 : 1;
-    // bf16 with TMA boxes, 8-head groups: one CTA per SM with two consumers,
-    // unless the call has at least four (request, head group) pairs per SM --
+    // bf16, 8-head groups: one CTA per SM with two consumers, unless the call
+    // has at least four (request, head group) pairs per SM --
     // then few of them split, and two CTAs per SM (one consumer and one
     // epilogue warp each) share the many short segments better.
     const DeviceInfo* di = current_device_info();
@@ -1640,10 +1640,14 @@ pkv_status launch_decode_mma(const DecodeParams& p, int head_dim, int group_pad,
         if (head_dim == 64) return nt == 1 ? launch_impl<64, 1, true, false, false>(p, stream, grid_out)
                                            : launch_impl<64, 2, true, false, false>(p, stream, grid_out);
     } else if (p.row_copy) {
-        if (head_dim == 128) return nt == 1 ? launch_impl<128, 1, false, true, true>(p, stream, grid_out)
-                                            : launch_impl<128, 2, false, true, true>(p, stream, grid_out);
-        if (head_dim == 64) return nt == 1 ? launch_impl<64, 1, false, true, true>(p, stream, grid_out)
-                                           : launch_impl<64, 2, false, true, true>(p, stream, grid_out);
+        if (head_dim == 128)
+            return nt == 2 ? launch_impl<128, 2, false, true, true>(p, stream, grid_out)
+                   : many  ? launch_impl<128, 1, false, true, true>(p, stream, grid_out)
+                           : launch_impl<128, 1, false, true, false>(p, stream, grid_out);
+        if (head_dim == 64)
+            return nt == 2 ? launch_impl<64, 2, false, true, true>(p, stream, grid_out)
+                   : many  ? launch_impl<64, 1, false, true, true>(p, stream, grid_out)
+                           : launch_impl<64, 1, false, true, false>(p, stream, grid_out);
     } else {
         if (head_dim == 128)
             return nt == 2 ? launch_impl<128, 2, false, false, true>(p, stream, grid_out)
