@@ -81,6 +81,11 @@ SMALL = [
     # 60 requests of 1..400 tokens: many segments per CTA and many split groups
     ([int(x) for x in np.random.default_rng(78).integers(1, 401, size=60)], 32, 8, 128, 16, "bf16"),
     ([int(x) for x in np.random.default_rng(79).integers(1, 401, size=40)], 16, 1, 64, 8, "bf16"),
+    # 100 requests x 8 kv heads: more (request, head group) pairs than four per SM,
+    # so the bf16 decode takes its two-CTAs-per-SM layout (TMA boxes and row copies)
+    ([int(x) for x in np.random.default_rng(80).integers(1, 300, size=100)], 32, 8, 128, 8, "bf16"),
+    ([int(x) for x in np.random.default_rng(81).integers(1, 300, size=100)], 32, 8, 128, 4, "bf16"),
+    ([int(x) for x in np.random.default_rng(82).integers(1, 200, size=100)], 16, 8, 64, 2, "bf16"),
 ]
 
 
