@@ -40,9 +40,10 @@ UNIT = "GB/s"
 WORKLOAD = "gqa_4k: batch 16 x 4096 tokens, 32 q / 8 KV heads, head_dim 128, block 16, bf16"
 FALLBACK_HBM_GBS = 6650.0
 NOMINAL_HBM_GBS = 8000.0  # the B200's ~8 TB/s HBM3e figure, for the nominal fraction
-ROOFLINE_LAUNCHES = 2000  # decode-only launches timed for the roofline, whatever --steps
-DEC_RUN = 20               # back-to-back decode launches per timed graph (roofline)
-ISOLATED_LAUNCHES = 200    # single decode launches timed on their own (latency)
+ROOFLINE_LAUNCHES = 2000  # decode-append launches timed for the roofline, whatever --steps
+DEC_RUN = 20               # back-to-back decode-append launches per timed graph (roofline)
+ISOLATED_LAUNCHES = 200    # single decode-append launches timed on their own (latency)
+SEPARATE_SWEEPS = 50       # sweeps timed for the step with the append as its own launch
 N_LAYERS = 4
 DECODE_SRC = os.path.join(ROOT, "paged_kv_cache_412_b200", "csrc", "decode_mma.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_gqa_4k_traffic.txt")
@@ -365,9 +366,18 @@ def run_ours(args, rank: int, world: int, local: int):
     no_pairs = torch.empty((0, 2), dtype=torch.int64, device=dev)
     scale = 1.0 / math.sqrt(d)
 
-    def step_body(t, with_write=True):
+    # Every request appends one token, so the step's new rows are one per
+    # request ([B, Hkv, d]) and the append rides in the decode launch
+    # (paged_attention_decode_append); ``fused=False`` is the same step with
+    # the append as its own kv_cache_write launch.
+    def step_body(t, with_write=True, fused=True):
         if with_write:
             pkv.copy_blocks(t["kc"], t["vc"], no_pairs)  # no shared block to fork here
+            if fused:
+                pkv.paged_attention_decode_append(t["q"], t["kn"], t["vn"], t["kc"], t["vc"],
+                                                  t["bt"], t["sl"], bs, scale, out,
+                                                  max_seq_len=L, workspace=ws)
+                return
             pkv.kv_cache_write(t["kn"], t["vn"], t["sm"], t["kc"], t["vc"])
         pkv.paged_attention_decode(t["q"], t["kc"], t["vc"], t["bt"], t["sl"], bs, scale, out,
                                    max_seq_len=L, workspace=ws)
@@ -375,6 +385,7 @@ def run_ours(args, rank: int, world: int, local: int):
     # eager warm-up (first calls set up per-device state outside any capture)
     for i in range(args.warmup):
         step_body(layers[i % N_LAYERS])
+    step_body(layers[0], fused=False)
     torch.cuda.synchronize()
     assert pkv.get_device_error() == 0
 
@@ -383,11 +394,11 @@ def run_ours(args, rank: int, world: int, local: int):
     # per layer), so consecutive kernels overlap through programmatic
     # dependent launch as they would in the serving loop; a second graph holds
     # the first K % N_LAYERS steps of a sweep.
-    def capture(steps, with_write):
+    def capture(steps, with_write, fused=True):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             for li in range(steps):
-                step_body(layers[li % N_LAYERS], with_write)
+                step_body(layers[li % N_LAYERS], with_write, fused)
         return g
     sweep = capture(N_LAYERS, True)
     n_sweeps, rest = divmod(args.steps, N_LAYERS)
@@ -423,13 +434,30 @@ def run_ours(args, rank: int, world: int, local: int):
     ms_step = ms_total_max / args.steps
     del sweep, part
 
+    # The same step with the append as its own launch (kv_cache_write, then
+    # the decode): sweeps of N_LAYERS steps, events around each sweep.
+    sep = capture(N_LAYERS, True, fused=False)
+    for _ in range(3):
+        sep.replay()
+    torch.cuda.synchronize()
+    sep_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(SEPARATE_SWEEPS)]
+    for a, b in sep_ev:
+        a.record()
+        sep.replay()
+        b.record()
+    torch.cuda.synchronize()
+    sep_ms = statistics.median(a.elapsed_time(b) / N_LAYERS for a, b in sep_ev)
+    del sep
+    assert pkv.get_device_error() == 0
+
     # --- the decode kernel alone (roofline), a fixed number of launches ---
     # Throughput: graphs of DEC_RUN back-to-back decode launches over the layer
     # pools, events around each graph; the launch duration is the graph's time
     # over DEC_RUN.  Latency of one launch on its own (events around a graph
     # of one launch) is reported beside it.
-    dec_run = capture(DEC_RUN, False)
-    dec_one = [capture(1, False) for _ in range(1)]
+    dec_run = capture(DEC_RUN, True)
+    dec_one = [capture(1, True) for _ in range(1)]
     n_runs = -(-ROOFLINE_LAUNCHES // DEC_RUN)
     n_dec = n_runs * DEC_RUN
     for _ in range(3):
@@ -437,7 +465,7 @@ def run_ours(args, rank: int, world: int, local: int):
     torch.cuda.synchronize()
     dev_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(n_runs)]
-    torch.cuda.nvtx.range_push("roofline: back-to-back decode launches")
+    torch.cuda.nvtx.range_push("roofline: back-to-back decode-append launches")
     for a, b in dev_ev:
         a.record()
         dec_run.replay()
@@ -456,6 +484,18 @@ def run_ours(args, rank: int, world: int, local: int):
     torch.cuda.nvtx.range_pop()
     iso_ms = statistics.fmean(a.elapsed_time(b) for a, b in iso_ev)
     del dec_run, dec_one
+    # the decode alone (no append), for comparison
+    dec_only = capture(DEC_RUN, False)
+    for _ in range(3):
+        dec_only.replay()
+    torch.cuda.synchronize()
+    for a, b in dev_ev:
+        a.record()
+        dec_only.replay()
+        b.record()
+    torch.cuda.synchronize()
+    dec_only_ms = statistics.fmean(a.elapsed_time(b) / DEC_RUN for a, b in dev_ev)
+    del dec_only
 
     dbytes = decode_bytes(B, L, Hq, Hkv, d)
     wbytes = write_bytes(B, Hkv, d)
@@ -463,7 +503,9 @@ def run_ours(args, rank: int, world: int, local: int):
     dec_avg_ms = statistics.fmean(decode_ms)
     dec_med_ms = statistics.median(decode_ms)
     peak, peak_kind = measured_peak()
-    achieved = dbytes / (dec_avg_ms / 1e3) / 1e9
+    # the fused launch moves the decode's bytes and the append's (k_new and
+    # v_new read, the same bytes written to the cache)
+    achieved = (dbytes + wbytes) / (dec_avg_ms / 1e3) / 1e9
 
     # --- e2e: host inputs -> device, the step, result -> host, per step ---
     t0l = layers[0]
@@ -474,8 +516,7 @@ def run_ours(args, rank: int, world: int, local: int):
     parts = [("q", hw.q.view(np.int16), torch.bfloat16),
              ("kn", hw.k_new.view(np.int16), torch.bfloat16),
              ("vn", hw.v_new.view(np.int16), torch.bfloat16),
-             ("sm", hw.slot_mapping, torch.int64), ("bt", hw.block_tables, torch.int32),
-             ("sl", hw.seq_lens, torch.int32)]
+             ("bt", hw.block_tables, torch.int32), ("sl", hw.seq_lens, torch.int32)]
     offs, total = {}, 0
     for name, arr, _ in parts:
         offs[name] = total
@@ -495,16 +536,16 @@ def run_ours(args, rank: int, world: int, local: int):
         t = layers[li % N_LAYERS]
         d_in.copy_(h_in, non_blocking=True)
         pkv.copy_blocks(t["kc"], t["vc"], no_pairs)
-        pkv.kv_cache_write(views["kn"], views["vn"], views["sm"], t["kc"], t["vc"])
-        pkv.paged_attention_decode(views["q"], t["kc"], t["vc"], views["bt"], views["sl"], bs,
-                                   scale, out, max_seq_len=L, workspace=ws)
+        pkv.paged_attention_decode_append(views["q"], views["kn"], views["vn"], t["kc"],
+                                          t["vc"], views["bt"], views["sl"], bs, scale, out,
+                                          max_seq_len=L, workspace=ws)
         h_out.copy_(out.view(torch.int16), non_blocking=True)
 
     # A serving loop captures its decode step once and replays it: one graph per
     # layer pool holding the host->device copies, the three calls and the
     # device->host copy; every step is a replay plus a stream synchronize.
     e2e_mode = ("CUDA graph per step (one copy in of the staged inputs, copy_blocks, "
-                "kv_cache_write, decode, copy out)")
+                "decode with the fused append, copy out)")
     try:
         e2e_graphs = []
         for li in range(N_LAYERS):
@@ -540,7 +581,7 @@ def run_ours(args, rank: int, world: int, local: int):
     e2e_value = dbytes * e2e_steps * world / (e2e_ms / 1e3) / 1e9
     assert pkv.get_device_error() == 0
 
-    # The same step with the three C-ABI calls issued eagerly every step: each
+    # The same step with the two C-ABI calls issued eagerly every step: each
     # call's host validation, planning, tensor-map encoding and launch is inside
     # the timed region.  host_us_per_step is the host time of those calls.
     def eager_step(li):
@@ -587,31 +628,40 @@ def run_ours(args, rank: int, world: int, local: int):
                        "l2": f"inputs larger than L2: {N_LAYERS} layer pools of "
                              f"{2 * B * L * Hkv * d * 2 / 1e6:.0f} MB K+V rotated per step",
                        "parallelism": f"replica x{world}" if world > 1 else "single GPU",
-                       "step": "copy_blocks (0 pairs) + kv_cache_write (16 tokens) + "
-                               "paged_attention_decode; the steps of a sweep over the "
-                               f"{N_LAYERS} layer pools captured in one CUDA graph and "
-                               "replayed back to back"},
+                       "step": "copy_blocks (0 pairs) + paged_attention_decode_append "
+                               "(the 16 new tokens appended inside the decode launch); the "
+                               f"steps of a sweep over the {N_LAYERS} layer pools captured "
+                               "in one CUDA graph and replayed back to back"},
             "tokens_per_s": round(B * world * args.steps / (ms_total_max / 1e3), 1),
             "context_tokens_per_s": round(B * L * world * args.steps / (ms_total_max / 1e3), 1),
             "fraction_of_hbm_peak": round(value / peak, 4),
             "fraction_of_nominal_peak": round(value / NOMINAL_HBM_GBS, 4),
             "nominal_peak_gbs": NOMINAL_HBM_GBS,
             "step_ms_median": round(statistics.median(step_ms), 5),
+            "step_separate_calls": {
+                "ms_median": round(sep_ms, 5),
+                "GBps": round(dbytes / (sep_ms / 1e3) / 1e9, 2),
+                "note": "the same step with the append as its own launch (copy_blocks + "
+                        "kv_cache_write + paged_attention_decode), median over "
+                        f"{SEPARATE_SWEEPS} sweeps of the layer pools"},
             "decode_ms_avg": round(dec_avg_ms, 5), "decode_ms_median": round(dec_med_ms, 5),
             "decode_launches_timed": n_dec,
+            "decode_only_ms_avg": round(dec_only_ms, 5),
             "decode_isolated": {"ms_avg": round(iso_ms, 5), "launches": ISOLATED_LAUNCHES,
                                 "GBps": round(dbytes / (iso_ms / 1e3) / 1e9, 2),
-                                "note": "one decode launch on its own between events (its "
+                                "note": "one decode-append launch on its own between events (its "
                                         "launch latency, planning and ramp not overlapped "
                                         "with a previous kernel)"},
-            "bytes_per_step": {"decode_algorithmic": dbytes, "write": wbytes},
+            "bytes_per_step": {"decode_algorithmic": dbytes, "append": wbytes},
             "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peak,
                          "unit": "GB/s", "frac": round(achieved / peak, 4),
                          "traffic": traffic_per_launch(),
-                         "kernel": "decode_mma_kernel (split decode with in-kernel merge)",
+                         "kernel": "decode_mma_kernel (split decode with in-kernel merge "
+                                   "and the fused append)",
+                         "bytes": "decode_algorithmic + append",
                          "duration": f"per-launch mean of graphs of {DEC_RUN} back-to-back "
-                                     "decode launches over the layer pools (events around "
-                                     "each graph), after the timed steps",
+                                     "decode-append launches over the layer pools (events "
+                                     "around each graph), after the timed steps",
                          "peak_kind": f"{peak_kind} HBM copy bandwidth"},
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_value, 2), "unit": UNIT, "h2d_bytes_per_step": h2d,
@@ -624,12 +674,12 @@ def run_ours(args, rank: int, world: int, local: int):
                           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                           "steps": e2e_steps, "ms_per_step": round(eager_ms / e2e_steps, 5),
                           "host_us_per_step": round(host_s / e2e_steps * 1e6, 2),
-                          "note": "the same step with copy_blocks, kv_cache_write and the "
-                                  "decode called eagerly through the binding every step "
+                          "note": "the same step with copy_blocks and the decode-append "
+                                  "called eagerly through the binding every step "
                                   "(host validation, planning, tensor-map encoding and "
                                   "launches inside the timed region); host_us_per_step = "
-                                  "host time of the copy-in, three calls and copy-out"},
-            "gpu_launches": 2 * args.steps,
+                                  "host time of the copy-in, two calls and copy-out"},
+            "gpu_launches": args.steps,
             "clocks": clocks,
             "configs": configs,
             "configs_l2": _L2Flush.DESCRIPTION if configs else None,
@@ -773,7 +823,7 @@ def run_suite(args):
         line.update(extra)
         print(json.dumps(line), flush=True)
 
-    def decode_case(name, w, partition_size=0, extra=None, fp8=False):
+    def decode_case(name, w, partition_size=0, extra=None, fp8=False, append=False):
         t = _dev_workload(w, dev)
         L = int(w.seq_lens.max())
         out = torch.empty((w.B, w.Hq, w.d), dtype=torch.bfloat16, device=dev)
@@ -781,6 +831,11 @@ def run_suite(args):
                                                           partition_size), dev)
 
         def fn(kc=t["kc"], vc=t["vc"]):
+            if append:  # every request appends one token: one new row per request
+                pkv.paged_attention_decode_append(t["q"], t["kn"], t["vn"], kc, vc, t["bt"],
+                                                  t["sl"], w.bs, w.scale, out, max_seq_len=L,
+                                                  workspace=ws, partition_size=partition_size)
+                return
             pkv.paged_attention_decode(t["q"], kc, vc, t["bt"], t["sl"], w.bs,
                                        w.scale, out, max_seq_len=L, workspace=ws,
                                        partition_size=partition_size, k_scale=t["ks"],
@@ -797,6 +852,8 @@ def run_suite(args):
         e_kv = 1 if fp8 else 2
         nbytes = (2 * int(w.seq_lens.astype(np.int64).sum()) * w.Hkv * w.d * e_kv
                   + w.B * w.Hq * w.d * 4)
+        if append:
+            nbytes += write_bytes(w.B, w.Hkv, w.d)
         info = {"B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "block_size": w.bs,
                 "kv_dtype": "fp8_e4m3" if fp8 else "bf16", "partition_size": partition_size,
                 "context_tokens": int(w.seq_lens.astype(np.int64).sum()),
@@ -816,6 +873,9 @@ def run_suite(args):
         w = workloads.make_paged([4096] * 16, Hq=32, Hkv=8, d=128, bs=16, dtype="bf16",
                                  seed=1002, poison=False, permute=False, name="gqa_4k_identity")
         decode_case("decode gqa_4k identity tables", w)
+    if want("append"):
+        decode_case("decode gqa_4k with the fused append (paged_attention_decode_append)",
+                    workloads.gqa_4k(poison=False), append=True)
     if want("fp8"):
         decode_case("decode gqa_4k fp8 e4m3 cache", workloads.gqa_4k_fp8(poison=False), fp8=True)
     if want("mixed"):
@@ -900,8 +960,10 @@ def run_configs(pkv, torch, dev, peak, peak_kind, with_oracle=True, iters=200,
                 oracle_budget_s=0.8) -> list:
     """One compact entry per workload: mean decode time over ``iters`` launches
     (each after the L2 flush of _L2Flush, CUDA events around each), KV GB/s by the
-    decode byte model, the fraction of the HBM peak, and the oracle's KV GB/s on
-    a bounded sample of the same workload on all host cores and on one thread.
+    decode byte model, the fraction of the HBM peak, the same for launches issued
+    back to back (``us_back_to_back``: graphs of B2B_RUN launches over B2B_POOLS
+    copies of the caches, median per launch), and the oracle's KV GB/s on a
+    bounded sample of the same workload on all host cores and on one thread.
     """
     import oracle
     import workloads
@@ -921,12 +983,16 @@ def run_configs(pkv, torch, dev, peak, peak_kind, with_oracle=True, iters=200,
         return (2 * int(w.seq_lens.astype(np.int64).sum()) * w.Hkv * w.d * w.elem_bytes
                 + w.B * w.Hq * w.d * 2 * e_q)
 
-    def entry(name, w, ms, nbytes, extra=None, oracle_w=None):
+    def entry(name, w, ms, nbytes, extra=None, oracle_w=None, b2b_ms=None):
         mean, med = ms
         gbs = nbytes / (mean / 1e3) / 1e9
         e = {"workload": name, "us_mean": round(mean * 1e3, 2), "us_median": round(med * 1e3, 2),
              "GBps": round(gbs, 1), "frac_of_peak": round(gbs / peak, 4), "bytes": int(nbytes),
              "tokens_per_s": round(w.B / (mean / 1e3), 1)}
+        if b2b_ms is not None:
+            g2 = nbytes / (b2b_ms / 1e3) / 1e9
+            e.update({"us_back_to_back": round(b2b_ms * 1e3, 2), "GBps_back_to_back": round(g2, 1),
+                      "frac_back_to_back": round(g2 / peak, 4)})
         e.update(extra or {})
         e["oracle"] = oracle_pair(oracle_w if oracle_w is not None else w)
         entries.append(e)
@@ -934,9 +1000,20 @@ def run_configs(pkv, torch, dev, peak, peak_kind, with_oracle=True, iters=200,
 
     def decode_fn(t, w, out, ws, partition_size=0):
         L = int(w.seq_lens.max())
-        return lambda: pkv.paged_attention_decode(
-            t["q"], t["kc"], t["vc"], t["bt"], t["sl"], w.bs, w.scale, out, max_seq_len=L,
+        return lambda kc=t["kc"], vc=t["vc"]: pkv.paged_attention_decode(
+            t["q"], kc, vc, t["bt"], t["sl"], w.bs, w.scale, out, max_seq_len=L,
             workspace=ws, partition_size=partition_size, k_scale=t["ks"], v_scale=t["vs"])
+
+    def b2b(t, fn):
+        """Median per-launch time (ms) of graphs of B2B_RUN launches of fn(kc, vc)
+        back to back over B2B_POOLS copies of the caches (more than L2 holds)."""
+        pools = [(t["kc"], t["vc"])] + [(t["kc"].clone(), t["vc"].clone())
+                                        for _ in range(B2B_POOLS - 1)]
+        ms = _time_back_to_back(lambda i: fn(*pools[i % B2B_POOLS]), B2B_RUN, 10)
+        del pools
+        torch.cuda.empty_cache()
+        assert pkv.get_device_error() == 0
+        return ms
 
     def setup(w, partition_size=0):
         t = _dev_workload(w, dev)
@@ -971,7 +1048,7 @@ def run_configs(pkv, torch, dev, peak, peak_kind, with_oracle=True, iters=200,
         t, out, ws = setup(w)
         ms = _time_graph(decode_fn(t, w, out, ws), iters, flush)
         entry(f"{name}: 16 x 4096, 32 q / 8 KV heads, d 128, bs 16, bf16 (decode)", w, ms,
-              nbytes_of(w), {"kv_dtype": "bf16"})
+              nbytes_of(w), {"kv_dtype": "bf16"}, b2b_ms=b2b(t, decode_fn(t, w, out, ws)))
         del t, out, ws
 
     # the same batch with an fp8 (e4m3) cache
@@ -979,19 +1056,25 @@ def run_configs(pkv, torch, dev, peak, peak_kind, with_oracle=True, iters=200,
     t, out, ws = setup(w)
     ms = _time_graph(decode_fn(t, w, out, ws), iters, flush)
     entry("gqa_4k_fp8: 16 x 4096, e4m3 cache with per-kv-head scales (decode; bytes of codes)",
-          w, ms, nbytes_of(w), {"kv_dtype": "fp8_e4m3"})
+          w, ms, nbytes_of(w), {"kv_dtype": "fp8_e4m3"}, b2b_ms=b2b(t, decode_fn(t, w, out, ws)))
     del t, out, ws
 
     # config 3: mixed lengths, append + decode
     w = workloads.mixed(poison=False)
     t, out, ws = setup(w)
-    dec, wr = decode_fn(t, w, out, ws), write_fn(t, w)
+    dec = decode_fn(t, w, out, ws)
+    Lm = int(w.seq_lens.max())
+
+    def dec_append():  # every request appends one token, inside the decode launch
+        pkv.paged_attention_decode_append(t["q"], t["kn"], t["vn"], t["kc"], t["vc"], t["bt"],
+                                          t["sl"], w.bs, w.scale, out, max_seq_len=Lm,
+                                          workspace=ws)
     ms_dec = _time_graph(dec, iters, flush)
-    ms_step = _time_graph(lambda: (wr(), dec()), iters, flush)
+    ms_step = _time_graph(dec_append, iters, flush)
     entry("mixed: 256 requests, log-uniform 16..8192 tokens (decode)", w, ms_dec, nbytes_of(w),
           {"kv_dtype": "bf16", "step_us_mean": round(ms_step[0] * 1e3, 2),
-           "step": "kv_cache_write (256 tokens) + decode",
-           "context_tokens": int(w.seq_lens.astype(np.int64).sum())})
+           "step": "paged_attention_decode_append (256 new tokens appended in the decode launch)",
+           "context_tokens": int(w.seq_lens.astype(np.int64).sum())}, b2b_ms=b2b(t, dec))
     del t, out, ws, w
     torch.cuda.empty_cache()
 
@@ -1006,8 +1089,8 @@ def run_configs(pkv, torch, dev, peak, peak_kind, with_oracle=True, iters=200,
         w.B, w.Hq, w.Hkv, w.d, w.bs, L, 1, w.B, w.info["prefix_tokens"]), dev)
     dec = decode_fn(t, w, out, ws)
 
-    def dec_p():
-        pkv.paged_attention_decode_prefix(t["q"], t["kc"], t["vc"], t["bt"], t["sl"], pfx_of,
+    def dec_p(kc=t["kc"], vc=t["vc"]):
+        pkv.paged_attention_decode_prefix(t["q"], kc, vc, t["bt"], t["sl"], pfx_of,
                                           pfx_len, w.bs, w.scale, out, max_seq_len=L,
                                           max_prefix_members=w.B,
                                           max_prefix_len=w.info["prefix_tokens"], workspace=ws_p)
@@ -1020,6 +1103,7 @@ def run_configs(pkv, torch, dev, peak, peak_kind, with_oracle=True, iters=200,
     unique = 2 * unique_tok * w.Hkv * w.d * 2 + w.B * w.Hq * w.d * 4
     ms_a = _time_graph(dec, iters, flush)
     ms_b = _time_graph(dec_p, iters, flush)
+    b2b_a, b2b_b = b2b(t, dec), b2b(t, dec_p)
     ms_sa = _time_graph(lambda: (fork_append(), dec()), iters, flush)
     ms_sb = _time_graph(lambda: (fork_append(), dec_p()), iters, flush)
     common = {"kv_dtype": "bf16", "bytes_kind": "logical (prefix counted once per request)",
@@ -1027,12 +1111,13 @@ def run_configs(pkv, torch, dev, peak, peak_kind, with_oracle=True, iters=200,
     entry("prefix: 64 requests sharing a 2040-token prefix, per-request decode", w, ms_a,
           logical, dict(common, unique_GBps=round(unique / (ms_a[0] / 1e3) / 1e9, 1),
                         step_us_mean=round(ms_sa[0] * 1e3, 2),
-                        step="copy_blocks (64 forks) + kv_cache_write (suffixes) + decode"))
+                        step="copy_blocks (64 forks) + kv_cache_write (suffixes) + decode"),
+          b2b_ms=b2b_a)
     entry("prefix: the same, prefix-aware decode (shared blocks read once per group)", w, ms_b,
           logical, dict(common, unique_GBps=round(unique / (ms_b[0] / 1e3) / 1e9, 1),
                         step_us_mean=round(ms_sb[0] * 1e3, 2),
                         step="copy_blocks (64 forks) + kv_cache_write (suffixes) + "
-                             "paged_attention_decode_prefix"))
+                             "paged_attention_decode_prefix"), b2b_ms=b2b_b)
     del t, out, ws, ws_p, w
     torch.cuda.empty_cache()
 
@@ -1042,7 +1127,8 @@ def run_configs(pkv, torch, dev, peak, peak_kind, with_oracle=True, iters=200,
         t, out, ws = setup(w)
         ms = _time_graph(decode_fn(t, w, out, ws), max(50, iters // 4), flush)
         entry(f"long_ctx: 2 x 131072 tokens, 64 q / 8 KV heads, d 128, bs {bs}, automatic "
-              f"split (decode)", w, ms, nbytes_of(w), {"kv_dtype": "bf16", "block_size": bs})
+              f"split (decode)", w, ms, nbytes_of(w), {"kv_dtype": "bf16", "block_size": bs},
+              b2b_ms=b2b(t, decode_fn(t, w, out, ws)))
         del t, out, ws, w
         torch.cuda.empty_cache()
     torch.cuda.nvtx.range_pop()

@@ -6,6 +6,8 @@
  *   - pkv_paged_attention_decode  single-query decode attention over a cache
  *                                 held in fixed-size physical blocks reached
  *                                 through a per-request block table;
+ *   - pkv_paged_attention_decode_append  the append of each request's new
+ *                                 token fused into the decode;
  *   - pkv_copy_blocks             copy-on-write copy of shared blocks;
  *   - pkv_paged_attention_decode_prefix  the same decode with the blocks a
  *                                 group of requests shares read once per group.
@@ -202,6 +204,34 @@ pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache,
                                       const float* v_scale, int32_t partition_size,
                                       void* workspace, size_t workspace_bytes,
                                       pkv_stream_t stream);
+
+/*
+ * pkv_paged_attention_decode_append -- each request's new token appended to
+ * the cache, then pkv_paged_attention_decode, in one kernel.
+ *
+ * [PAMEM] "The Mechanics of PagedAttention": the new token's K and V go to the
+ * slot its block table names; "The Math: Block Attention Calculation": the
+ * decode.  Request b's new token is the last of its seq_lens[b] tokens: K row
+ * k_new[b] and V row v_new[b] are written at position L-1 (L = seq_lens[b]) as
+ * the table names it -- physical block block_tables[b][(L-1)/block_size], row
+ * (L-1) % block_size -- the same bytes pkv_kv_cache_write writes for that
+ * slot; the decode then runs exactly as pkv_paged_attention_decode (same
+ * arguments, same result).  The row is written by the CTA that fetches its
+ * block for the decode, just before fetching it, so the append needs no launch
+ * and no wait of its own.
+ *   k_new, v_new  [num_seqs, num_kv_heads, head_dim] bf16, 16-byte aligned.
+ *   Other arguments as pkv_paged_attention_decode.  bf16 q and caches on the
+ *   tensor-core path (block_size >= 2, not 1) only: other configurations
+ *   return PKV_ERR_UNSUPPORTED (use pkv_kv_cache_write + the decode).  A
+ *   request with seq_lens[b] == 0 appends nothing; an out-of-range table entry
+ *   skips the copy and flags PKV_DEVERR_BAD_BLOCK, as the decode does.
+ */
+pkv_status pkv_paged_attention_decode_append(
+    const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+    const int32_t* block_tables, const int32_t* seq_lens, int32_t block_size, float scale,
+    void* out, int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t max_blocks_per_seq, int32_t num_blocks, int32_t max_seq_len, pkv_dtype out_dtype,
+    int32_t partition_size, void* workspace, size_t workspace_bytes, pkv_stream_t stream);
 
 /*
  * pkv_decode_prefix_workspace_bytes -- workspace bytes of

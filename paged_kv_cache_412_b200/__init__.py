@@ -29,7 +29,7 @@ __all__ = [
     "PkvError", "LIB_PATH", "lib", "kv_cache_write", "paged_attention_decode", "copy_blocks",
     "decode_workspace_bytes", "new_workspace", "get_device_error", "status_string", "DEVERR",
     "paged_attention_decode_noalloc", "BlockAllocator", "waste_compare", "swap_blocks",
-    "kv_cache_write_fp8", "workspace_init",
+    "kv_cache_write_fp8", "workspace_init", "paged_attention_decode_append",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libpkv.so")
@@ -71,6 +71,10 @@ def _load() -> ctypes.CDLL:
                                              i32, i32, i32, i32, ctypes.c_int, ctypes.c_int,
                                              ctypes.c_int, vp, vp, i32, vp, sz, vp]
     L.pkv_paged_attention_decode.restype = ctypes.c_int
+    L.pkv_paged_attention_decode_append.argtypes = [vp, vp, vp, vp, vp, vp, vp, i32, f32, vp,
+                                                    i32, i32, i32, i32, i32, i32, i32,
+                                                    ctypes.c_int, i32, vp, sz, vp]
+    L.pkv_paged_attention_decode_append.restype = ctypes.c_int
     L.pkv_decode_prefix_workspace_bytes.argtypes = [i32] * 9
     L.pkv_decode_prefix_workspace_bytes.restype = sz
     L.pkv_paged_attention_decode_prefix.argtypes = [vp, vp, vp, vp, vp, i32, f32, vp, i32, i32,
@@ -249,6 +253,54 @@ def paged_attention_decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torc
             _ptr(v_scale), int(partition_size), _ptr(ws), ws.numel() * ws.element_size(),
             _stream(dev))
     _check("pkv_paged_attention_decode", st)
+    return out
+
+
+def paged_attention_decode_append(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                                  k_cache: torch.Tensor, v_cache: torch.Tensor,
+                                  block_tables: torch.Tensor, seq_lens: torch.Tensor,
+                                  block_size: int | None = None, scale: float | None = None,
+                                  out: torch.Tensor | None = None, *,
+                                  max_seq_len: int | None = None, partition_size: int = 0,
+                                  out_dtype: torch.dtype | None = None,
+                                  workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Append each request's new token, then paged_attention_decode, in one kernel.
+
+    k_new, v_new [B, Hkv, d] bf16: the K and V rows of request b's token at
+    position seq_lens[b] - 1, written to the slot its block table names (the
+    bytes kv_cache_write writes there) before the decode reads that block.
+    bf16 q and caches, head_dim 64 or 128, block_size >= 2.
+    """
+    dev = _need_cuda(q, k_new, v_new, k_cache, v_cache, block_tables, seq_lens, out, workspace)
+    if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32:
+        raise TypeError("block_tables and seq_lens must be int32")
+    for name, t in (("q", q), ("k_new", k_new), ("v_new", v_new), ("k_cache", k_cache),
+                    ("v_cache", v_cache)):
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bfloat16")
+    B, Hq, d = q.shape
+    NB, Hkv, bs, d2 = k_cache.shape
+    if block_size is None:
+        block_size = bs
+    if (block_size != bs or d2 != d or v_cache.shape != k_cache.shape
+            or tuple(k_new.shape) != (B, Hkv, d) or v_new.shape != k_new.shape):
+        raise ValueError("shape mismatch")
+    if scale is None:
+        scale = d ** -0.5
+    max_blocks = block_tables.shape[1]
+    if max_seq_len is None:
+        max_seq_len = max_blocks * bs
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=out_dtype or q.dtype, device=dev)
+    with torch.cuda.device(dev):
+        ws = workspace if workspace is not None else _workspace(
+            dev, decode_workspace_bytes(B, Hq, Hkv, d, bs, max_seq_len, partition_size))
+        st = _get_lib().pkv_paged_attention_decode_append(
+            _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_cache), _ptr(v_cache), _ptr(block_tables),
+            _ptr(seq_lens), bs, float(scale), _ptr(out), B, Hq, Hkv, d, max_blocks, NB,
+            int(max_seq_len), _dtype_code(out), int(partition_size), _ptr(ws),
+            ws.numel() * ws.element_size(), _stream(dev))
+    _check("pkv_paged_attention_decode_append", st)
     return out
 
 

@@ -287,13 +287,21 @@ pkv_status decode_entry(const void* q, const void* k_cache, const void* v_cache,
                         int32_t num_blocks, int32_t max_seq_len, pkv_dtype q_dtype,
                         pkv_dtype kv_dtype, pkv_dtype out_dtype, const float* k_scale,
                         const float* v_scale, int32_t partition_size, void* workspace,
-                        size_t workspace_bytes, pkv_stream_t stream, const PrefixArgs* pa) {
+                        size_t workspace_bytes, pkv_stream_t stream, const PrefixArgs* pa,
+                        const void* k_new = nullptr, const void* v_new = nullptr) {
     {
         const pkv_status cs = check_decode_args(
             q, k_cache, v_cache, block_tables, seq_lens, block_size, scale, out, num_seqs,
             num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq, num_blocks, max_seq_len,
             q_dtype, kv_dtype, out_dtype, k_scale, v_scale, partition_size);
         if (cs != PKV_OK || num_seqs == 0) return cs;
+    }
+    if (k_new || v_new) {  // fused append: bf16 caches on the tensor-core path
+        if (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16))
+            return PKV_ERR_INVALID_ARG;
+        if (!decode_mma_supported(head_dim, block_size, q_dtype, kv_dtype) ||
+            kv_dtype != PKV_BF16 || (pa && pa->num_prefixes > 0))
+            return PKV_ERR_UNSUPPORTED;
     }
     const DeviceInfo* di0 = current_device_info();
     if (!di0) return PKV_ERR_CUDA;
@@ -378,6 +386,8 @@ pkv_status decode_entry(const void* q, const void* k_cache, const void* v_cache,
     p.out_dtype = out_dtype;
     p.scale_log2 = scale * 1.4426950408889634f;
     p.wait_ns = kWaitLimitNs;
+    p.k_new = k_new;
+    p.v_new = v_new;
     if (t_fault.mode != kFaultNone) {  // consumed by this call
         p.fault_mode = t_fault.mode;
         p.fault_arg = t_fault.arg;
@@ -448,6 +458,19 @@ pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache, const 
                         num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
                         num_blocks, max_seq_len, q_dtype, kv_dtype, out_dtype, k_scale, v_scale,
                         partition_size, workspace, workspace_bytes, stream, nullptr);
+}
+
+pkv_status pkv_paged_attention_decode_append(
+    const void* q, const void* k_new, const void* v_new, void* k_cache, void* v_cache,
+    const int32_t* block_tables, const int32_t* seq_lens, int32_t block_size, float scale,
+    void* out, int32_t num_seqs, int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+    int32_t max_blocks_per_seq, int32_t num_blocks, int32_t max_seq_len, pkv_dtype out_dtype,
+    int32_t partition_size, void* workspace, size_t workspace_bytes, pkv_stream_t stream) {
+    if (num_seqs > 0 && (!k_new || !v_new)) return PKV_ERR_INVALID_ARG;
+    return decode_entry(q, k_cache, v_cache, block_tables, seq_lens, block_size, scale, out,
+                        num_seqs, num_q_heads, num_kv_heads, head_dim, max_blocks_per_seq,
+                        num_blocks, max_seq_len, PKV_BF16, PKV_BF16, out_dtype, nullptr, nullptr,
+                        partition_size, workspace, workspace_bytes, stream, nullptr, k_new, v_new);
 }
 
 size_t pkv_decode_prefix_workspace_bytes(int32_t num_seqs, int32_t num_q_heads,

@@ -308,6 +308,31 @@ struct Producer {
                 else
                     ++nvalid;
             }
+            if (!F8 && p.k_new && c == cur.nch - 1) {
+                // Fused append: the request's new token (its last, position
+                // L - 1) is in this chunk.  Its K and V rows of this kv head
+                // go to their slot before the chunk's copies are issued (one
+                // 16-byte vector per lane, K on lanes 0 .., V on lanes 16 ..);
+                // the proxy fence orders these generic writes before the
+                // copy engine's reads of the block.
+                const int t = cur.L - 1;
+                const int phys = __shfl_sync(FULL_MASK, tab, (t >> p.log2_bs) - wbase);
+                constexpr int VEC = D * 2 / 16;  // 16-byte vectors per row
+                const int v = lane & 15;
+                if (phys >= 0 && phys < p.num_blocks && v < VEC) {
+                    const size_t src = ((size_t)cur.b * p.num_kv_heads + kvh) * D;
+                    const size_t dst =
+                        ((size_t)phys * p.num_kv_heads + kvh) * p.block_size * D +
+                        (size_t)(t & (p.block_size - 1)) * D;
+                    const uint4* from = reinterpret_cast<const uint4*>(
+                        static_cast<const __nv_bfloat16*>(lane < 16 ? p.k_new : p.v_new) + src);
+                    uint4* to = reinterpret_cast<uint4*>(
+                        static_cast<__nv_bfloat16*>(const_cast<void*>(lane < 16 ? p.k_cache : p.v_cache)) + dst);
+                    to[v] = __ldg(from + v);
+                    fence_proxy_async_global();
+                }
+                __syncwarp();
+            }
             unsigned char* sk = smem + stage * C::STAGE_BYTES;
             unsigned char* sv = sk + C::KV_BYTES;
             unsigned char* sq = sv + C::KV_BYTES;
@@ -887,28 +912,38 @@ __device__ __forceinline__ int prefix_tokens_of(const DecodeParams& p, int b) {
                          p.log2_bs, p.err, false);
 }
 
-// A part's partial result (unnormalised acc, max m, sum l) as record `rec`.
+// A part's partial result (unnormalised acc, max m, sum l) in the record
+// layout: acc rows of the 8*NT heads at `acc_rows`, their (m, l) pairs at
+// `ml_rows` (global memory, or shared memory).
 template <int D, int NT, bool F8>
-__device__ __forceinline__ void write_record(const DecodeParams& p, size_t rec, int tig, int grp,
-                                             const float (&acc)[D / 16][NT][4],
-                                             const float (&m)[NT][2], const float (&l)[NT][2]) {
-    constexpr int GP = 8 * NT;
+__device__ __forceinline__ void store_frag(float* acc_rows, float* ml_rows, int tig, int grp,
+                                           const float (&acc)[D / 16][NT][4],
+                                           const float (&m)[NT][2], const float (&l)[NT][2]) {
 #pragma unroll
     for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
             const int h = nt * 8 + 2 * tig + j;
-            float* ra = p.rec_acc + (rec * GP + h) * D;
+            float* ra = acc_rows + h * D;
 #pragma unroll
             for (int dt = 0; dt < D / 16; ++dt) {
                 ra[dcol<F8>(dt, grp, 0)] = acc[dt][nt][j];
                 ra[dcol<F8>(dt, grp, 1)] = acc[dt][nt][j + 2];
             }
             if (grp == 0) {
-                p.rec_ml[(rec * GP + h) * 2] = m[nt][j];
-                p.rec_ml[(rec * GP + h) * 2 + 1] = l[nt][j];
+                ml_rows[h * 2] = m[nt][j];
+                ml_rows[h * 2 + 1] = l[nt][j];
             }
         }
+}
+
+// ... as record `rec` of the workspace.
+template <int D, int NT, bool F8>
+__device__ __forceinline__ void write_record(const DecodeParams& p, size_t rec, int tig, int grp,
+                                             const float (&acc)[D / 16][NT][4],
+                                             const float (&m)[NT][2], const float (&l)[NT][2]) {
+    constexpr int GP = 8 * NT;
+    store_frag<D, NT, F8>(p.rec_acc + rec * GP * D, p.rec_ml + rec * GP * 2, tig, grp, acc, m, l);
 }
 
 // ---- epilogue: normalise, or write a partial record and merge the group ----
@@ -1153,50 +1188,92 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
             if (!ok) continue;
             __syncwarp();  // lane 0's acquires order the warp's reads of the records
         }
-        // The row state: this part's own, then the other parts merged into it
-        // in ascending order (the prefetched one, when there is one, is the
-        // first of them): M = max m, S = sum 2^(m-M) l, A = sum 2^(m-M) acc,
-        // out = A / S.  The others are fetched two at a time (8-head groups)
-        // with every load of the pair in flight before any math.
-        auto merge_in = [&](const float (&mr)[NT][2], const float (&lr)[NT][2],
-                            const float (&ar)[C::KS][NT][4]) {
+        // The row state: the group's parts merged in ascending part order
+        // 0, 1, .., nseg - 1 whichever part finishes last, so the result does
+        // not depend on timing.  Two states (m, l, acc) merge as M = max m,
+        // l = 2^(m0-M) l0 + 2^(m1-M) l1, acc likewise, with separately
+        // rounded products and one add, so the merge is symmetric in its
+        // operands.  Parts below this one are folded into a prefix first (the
+        // prefetched record, when there is one, is the lowest other part),
+        // the prefix is merged with this part's state, and the parts above it
+        // follow in order, fetched two at a time (8-head groups) with every
+        // load of the pair in flight before any math.
+        auto merge2 = [&](float (&m0)[NT][2], float (&l0)[NT][2], float (&a0)[C::KS][NT][4],
+                          const float (&mr)[NT][2], const float (&lr)[NT][2],
+                          const float (&ar)[C::KS][NT][4]) {
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
-                    const float M = fmaxf(m[nt][j], mr[nt][j]);
+                    const float M = fmaxf(m0[nt][j], mr[nt][j]);
                     const float mref = M == -INFINITY ? 0.f : M;
-                    const float fa = exp2f(m[nt][j] - mref), fb = exp2f(mr[nt][j] - mref);
-                    l[nt][j] = l[nt][j] * fa + lr[nt][j] * fb;
+                    const float fa = exp2f(m0[nt][j] - mref), fb = exp2f(mr[nt][j] - mref);
+                    l0[nt][j] = __fadd_rn(__fmul_rn(l0[nt][j], fa), __fmul_rn(lr[nt][j], fb));
 #pragma unroll
                     for (int dt = 0; dt < C::KS; ++dt) {
-                        acc[dt][nt][j] = acc[dt][nt][j] * fa + ar[dt][nt][j] * fb;
-                        acc[dt][nt][j + 2] = acc[dt][nt][j + 2] * fa + ar[dt][nt][j + 2] * fb;
+                        a0[dt][nt][j] =
+                            __fadd_rn(__fmul_rn(a0[dt][nt][j], fa), __fmul_rn(ar[dt][nt][j], fb));
+                        a0[dt][nt][j + 2] = __fadd_rn(__fmul_rn(a0[dt][nt][j + 2], fa),
+                                                      __fmul_rn(ar[dt][nt][j + 2], fb));
                     }
-                    m[nt][j] = M;
+                    m0[nt][j] = M;
                 }
         };
-        if (kPrefetch && split && pf_k >= 0) merge_in(pm, pl, pa);
-        if (kPrefetchSmem && split && pf_k >= 0) {
+        if (split && own > 0) {
+            if constexpr (kPrefetch) {
+                // bf16, 8-head groups: the prefix (parts 0 .. own-1) in the
+                // prefetch registers, where part 0 may be already
+                if (pf_k != 0) load_rec(rec_of(0), pm, pl, pa);
+                for (int k = 1; k < own; ++k) {
+                    float mr[NT][2], lr[NT][2], ar[C::KS][NT][4];
+                    load_rec(rec_of(k), mr, lr, ar);
+                    merge2(pm, pl, pa, mr, lr, ar);
+                }
+                merge2(m, l, acc, pm, pl, pa);
+            } else {
+                // No registers for a second state (fp8, 16-head groups): this
+                // part's state goes out as its record too, the fold starts
+                // from part 0 (fp8: from the shared-memory prefetch buffer
+                // when it is there) and reads this part's record back in its
+                // turn
+                write_record<D, NT, F8>(p, rec_of(own), tig, grp, acc, m, l);
+                __syncwarp();  // the m / l words are written by other lanes
+                if (kPrefetchSmem && pf_k == 0) {
+                    cp_async_wait_all();
+                    __syncwarp();  // every lane's copies have landed
+                    load_frag(pf_acc, pf_ml, false, m, l, acc);
+                } else {
+                    load_rec(rec_of(0), m, l, acc);
+                }
+                for (int k = 1; k <= own; ++k) {
+                    float mr[NT][2], lr[NT][2], ar[C::KS][NT][4];
+                    load_rec(rec_of(k), mr, lr, ar);
+                    merge2(m, l, acc, mr, lr, ar);
+                }
+            }
+        }
+        // parts above this one (own == 0: the prefetched record is part 1)
+        if (kPrefetch && split && pf_k > own) merge2(m, l, acc, pm, pl, pa);
+        if (kPrefetchSmem && split && pf_k > own) {
             cp_async_wait_all();
             __syncwarp();  // every lane's copies have landed
             float mr[NT][2], lr[NT][2], ar[C::KS][NT][4];
             load_frag(pf_acc, pf_ml, false, mr, lr, ar);
-            merge_in(mr, lr, ar);
+            merge2(m, l, acc, mr, lr, ar);
         }
         constexpr int kPair = NT == 1 ? 2 : 1;  // records in flight at once
-        for (int k0 = 0; split && k0 < si.nseg; k0 += kPair) {
+        for (int k0 = own + 1; split && k0 < si.nseg; k0 += kPair) {
             float mr[kPair][NT][2], lr[kPair][NT][2], ar[kPair][C::KS][NT][4];
             bool use[kPair];
 #pragma unroll
             for (int k = 0; k < kPair; ++k) {
                 const int kk = k0 + k;
-                use[k] = kk < si.nseg && kk != own && kk != pf_k;
+                use[k] = kk < si.nseg && kk != pf_k;
                 if (use[k]) load_rec(rec_of(kk), mr[k], lr[k], ar[k]);
             }
 #pragma unroll
             for (int k = 0; k < kPair; ++k)
-                if (use[k]) merge_in(mr[k], lr[k], ar[k]);
+                if (use[k]) merge2(m, l, acc, mr[k], lr[k], ar[k]);
         }
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt)

@@ -118,6 +118,12 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// This thread's generic-proxy writes to global memory before the async proxy's
+// (bulk / tensor copies') later accesses.
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 __device__ __forceinline__ float ld_cg(const float* p) { return __ldcg(p); }
 
 // 16-byte global -> shared copy through L2 (no L1), asynchronous to the

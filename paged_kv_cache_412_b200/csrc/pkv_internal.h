@@ -99,6 +99,11 @@ struct DecodeParams {
     // (DecodeFault) that makes one wait run out; 0 = none.
     unsigned long long wait_ns;
     int fault_mode, fault_arg;
+    // Fused append (pkv_paged_attention_decode_append): request b's new K/V rows
+    // [num_seqs][num_kv_heads][head_dim] bf16, written at position seq_lens[b]-1
+    // before the decode reads that block; nullptr: no append.
+    const void* k_new;
+    const void* v_new;
 };
 
 // Test-only faults of the tensor-core decode, set for the next decode call of

@@ -34,7 +34,8 @@ def lib():
 def test_header_declares_the_hot_path_calls():
     names = _declared_functions()
     for n in ("pkv_kv_cache_write", "pkv_paged_attention_decode", "pkv_copy_blocks",
-              "pkv_decode_workspace_bytes", "pkv_get_device_error", "pkv_status_string"):
+              "pkv_paged_attention_decode_append", "pkv_decode_workspace_bytes",
+              "pkv_get_device_error", "pkv_status_string"):
         assert n in names
 
 
@@ -111,6 +112,31 @@ def test_decode_rejects_bad_args(lib):
     assert _decode(lib, B=0) == 0               # empty batch: nothing to do
     assert _decode(lib, q=None) == 1
     assert _decode(lib, maxb=0) == 1
+
+
+def _decode_append(lib, **kw):
+    a = dict(q=DUMMY, kn=V(0x20000), vn=V(0x30000), kc=DUMMY, vc=DUMMY, bt=DUMMY, sl=DUMMY,
+             bs=16, scale=0.125, out=DUMMY, B=2, Hq=8, Hkv=2, d=128, maxb=4, NB=8, maxL=64,
+             odt=1, P=0, ws=DUMMY, wsb=1 << 20)
+    a.update(kw)
+    f = lib.pkv_paged_attention_decode_append
+    i32 = ctypes.c_int32
+    f.argtypes = [V, V, V, V, V, V, V, i32, ctypes.c_float, V, i32, i32, i32, i32, i32, i32, i32,
+                  ctypes.c_int, i32, V, ctypes.c_size_t, V]
+    return f(a["q"], a["kn"], a["vn"], a["kc"], a["vc"], a["bt"], a["sl"], a["bs"], a["scale"],
+             a["out"], a["B"], a["Hq"], a["Hkv"], a["d"], a["maxb"], a["NB"], a["maxL"], a["odt"],
+             a["P"], a["ws"], a["wsb"], None)
+
+
+def test_decode_append_rejects_bad_args(lib):
+    """Checked on the host before any device call (so no GPU is needed)."""
+    assert _decode_append(lib, kn=None) == 1          # a request has no new K row
+    assert _decode_append(lib, vn=None) == 1
+    assert _decode_append(lib, kn=V(0x20002)) == 1    # not on a 16-byte boundary
+    assert _decode_append(lib, bs=1) == 2             # no tensor-core path for 1-row blocks
+    assert _decode_append(lib, d=256) == 2
+    assert _decode_append(lib, Hq=6, Hkv=4) == 1      # the decode's own checks still apply
+    assert _decode_append(lib, B=0, kn=None, vn=None) == 0  # empty batch: nothing to do
 
 
 def _copy(lib, **kw):

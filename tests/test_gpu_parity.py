@@ -136,6 +136,31 @@ def test_deterministic_repeat(pkv):
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
 
 
+@pytest.mark.parametrize("dtype,Hq,Hkv", [("bf16", 8, 2), ("bf16", 16, 1), ("fp8", 8, 2)],
+                         ids=["bf16_G4", "bf16_G16", "fp8_G4"])
+def test_split_merge_is_deterministic(pkv, dtype, Hq, Hkv):
+    """Long requests over few (request, kv head) groups: every group is split
+    over many units and merged in-kernel by whichever part finishes last; the
+    parts are merged in a fixed order, so repeated calls give bit-identical
+    fp32 outputs (and agree with the oracle)."""
+    w = workloads.make_paged([30000, 20001], Hq=Hq, Hkv=Hkv, d=128, bs=16, dtype=dtype,
+                             seed=31, append_last=False)
+    dw = DevWorkload(w)
+    outs = []
+    for _ in range(4):
+        o = pkv.paged_attention_decode(dw.q, dw.k_cache, dw.v_cache, dw.block_tables,
+                                       dw.seq_lens, w.bs, w.scale, out_dtype=torch.float32,
+                                       k_scale=dw.k_scale, v_scale=dw.v_scale)
+        torch.cuda.synchronize()
+        outs.append(o)
+    assert pkv.get_device_error() == 0
+    for o in outs[1:]:
+        assert torch.equal(outs[0].view(torch.int32), o.view(torch.int32))
+    ref = oracle.decode(w.q, w.k_cache, w.v_cache, w.block_tables, w.seq_lens, w.scale,
+                        k_scale=w.k_scale, v_scale=w.v_scale)
+    assert_decode_close(to_host_f64(outs[0]), ref, "bf16", "f32", what=f"{dtype} split merge")
+
+
 def test_identity_and_permuted_tables_agree(pkv):
     lens = [700, 300]
     w1 = workloads.make_paged(lens, Hq=8, Hkv=2, d=128, bs=16, dtype="bf16", seed=3,
