@@ -216,11 +216,14 @@ __device__ __forceinline__ int bf16_row_off(int t, int half, int log2_rb) {
 // ---- producer ------------------------------------------------------------------
 
 // RC: blocks of 2 or 4 rows (bf16), copied row by row instead of by TMA boxes;
-// a separate instance so the boxed producer carries no trace of it.
-template <int D, int NT, bool F8, bool RC, bool SOLO>
+// a separate instance so the boxed producer carries no trace of it.  APP: the
+// fused append (bf16), likewise a separate instance: a plain decode's chunk
+// loop carries no trace of it.
+template <int D, int NT, bool F8, bool RC, bool SOLO, bool APP>
 struct Producer {
     using C = MmaCfg<D, NT, F8, SOLO, RC>;
     static_assert(!(RC && F8), "row copies serve bf16 caches only");
+    static_assert(!(APP && F8), "the fused append serves bf16 caches only");
 
     const DecodeParams& p;
     const CUtensorMap* tmk;
@@ -247,6 +250,31 @@ struct Producer {
 
     static __device__ __forceinline__ int first_block(const Cursor& cur, int c0, int log2_bs) {
         return (cur.t0 + c0 * kCH) >> log2_bs;
+    }
+
+    // Fused append: the request's new token (its last, position L - 1) is in
+    // the chunk about to be issued.  Its K and V rows of this kv head go to
+    // their slot before the chunk's copies are issued (one 16-byte vector per
+    // lane, K on lanes 0 .., V on lanes 16 ..); the proxy fence orders these
+    // generic writes before the copy engine's reads of the block.
+    __device__ __forceinline__ void append_rows(const Cursor& cur, int kvh, int tab, int wbase) {
+        const int t = cur.L - 1;
+        const int phys = __shfl_sync(FULL_MASK, tab, (t >> p.log2_bs) - wbase);
+        constexpr int VEC = D * 2 / 16;  // 16-byte vectors per row
+        const int v = lane & 15;
+        if (phys >= 0 && phys < p.num_blocks && v < VEC) {
+            const size_t src = ((size_t)cur.b * p.num_kv_heads + kvh) * D;
+            const size_t dst = ((size_t)phys * p.num_kv_heads + kvh) * p.block_size * D +
+                               (size_t)(t & (p.block_size - 1)) * D;
+            const uint4* from = reinterpret_cast<const uint4*>(
+                static_cast<const __nv_bfloat16*>(lane < 16 ? p.k_new : p.v_new) + src);
+            uint4* to = reinterpret_cast<uint4*>(
+                static_cast<__nv_bfloat16*>(const_cast<void*>(lane < 16 ? p.k_cache : p.v_cache)) +
+                dst);
+            to[v] = __ldg(from + v);
+            fence_proxy_async_global();
+        }
+        __syncwarp();
     }
 
     // Returns false when the CTA must stop (a wait gave up).
@@ -308,30 +336,8 @@ struct Producer {
                 else
                     ++nvalid;
             }
-            if (!F8 && p.k_new && c == cur.nch - 1) {
-                // Fused append: the request's new token (its last, position
-                // L - 1) is in this chunk.  Its K and V rows of this kv head
-                // go to their slot before the chunk's copies are issued (one
-                // 16-byte vector per lane, K on lanes 0 .., V on lanes 16 ..);
-                // the proxy fence orders these generic writes before the
-                // copy engine's reads of the block.
-                const int t = cur.L - 1;
-                const int phys = __shfl_sync(FULL_MASK, tab, (t >> p.log2_bs) - wbase);
-                constexpr int VEC = D * 2 / 16;  // 16-byte vectors per row
-                const int v = lane & 15;
-                if (phys >= 0 && phys < p.num_blocks && v < VEC) {
-                    const size_t src = ((size_t)cur.b * p.num_kv_heads + kvh) * D;
-                    const size_t dst =
-                        ((size_t)phys * p.num_kv_heads + kvh) * p.block_size * D +
-                        (size_t)(t & (p.block_size - 1)) * D;
-                    const uint4* from = reinterpret_cast<const uint4*>(
-                        static_cast<const __nv_bfloat16*>(lane < 16 ? p.k_new : p.v_new) + src);
-                    uint4* to = reinterpret_cast<uint4*>(
-                        static_cast<__nv_bfloat16*>(const_cast<void*>(lane < 16 ? p.k_cache : p.v_cache)) + dst);
-                    to[v] = __ldg(from + v);
-                    fence_proxy_async_global();
-                }
-                __syncwarp();
+            if constexpr (APP) {
+                if (c == cur.nch - 1) append_rows(cur, kvh, tab, wbase);
             }
             unsigned char* sk = smem + stage * C::STAGE_BYTES;
             unsigned char* sv = sk + C::KV_BYTES;
@@ -1193,11 +1199,8 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
         // not depend on timing.  Two states (m, l, acc) merge as M = max m,
         // l = 2^(m0-M) l0 + 2^(m1-M) l1, acc likewise, with separately
         // rounded products and one add, so the merge is symmetric in its
-        // operands.  Parts below this one are folded into a prefix first (the
-        // prefetched record, when there is one, is the lowest other part),
-        // the prefix is merged with this part's state, and the parts above it
-        // follow in order, fetched two at a time (8-head groups) with every
-        // load of the pair in flight before any math.
+        // operands.  Records are fetched two at a time (8-head groups) with
+        // every load of the pair in flight before any math.
         auto merge2 = [&](float (&m0)[NT][2], float (&l0)[NT][2], float (&a0)[C::KS][NT][4],
                           const float (&mr)[NT][2], const float (&lr)[NT][2],
                           const float (&ar)[C::KS][NT][4]) {
@@ -1219,7 +1222,12 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
                     m0[nt][j] = M;
                 }
         };
-        if (split && own > 0) {
+        // With a symmetric merge, this part's state, then the lowest other
+        // part, then the rest in ascending order is the ascending order when
+        // this part is part 0 or 1.  A later part first folds the parts below
+        // it into a prefix.
+        int k_from = 0;  // the first part the loop below considers
+        if (split && own >= 2) {
             if constexpr (kPrefetch) {
                 // bf16, 8-head groups: the prefix (parts 0 .. own-1) in the
                 // prefetch registers, where part 0 may be already
@@ -1251,24 +1259,26 @@ __device__ __forceinline__ void epilogue(const DecodeParams& p, SegIter<kCH>& it
                     merge2(m, l, acc, mr, lr, ar);
                 }
             }
-        }
-        // parts above this one (own == 0: the prefetched record is part 1)
-        if (kPrefetch && split && pf_k > own) merge2(m, l, acc, pm, pl, pa);
-        if (kPrefetchSmem && split && pf_k > own) {
-            cp_async_wait_all();
-            __syncwarp();  // every lane's copies have landed
-            float mr[NT][2], lr[NT][2], ar[C::KS][NT][4];
-            load_frag(pf_acc, pf_ml, false, mr, lr, ar);
-            merge2(m, l, acc, mr, lr, ar);
+            k_from = own + 1;
+        } else {
+            // the prefetched record is the lowest other part
+            if (kPrefetch && split && pf_k >= 0) merge2(m, l, acc, pm, pl, pa);
+            if (kPrefetchSmem && split && pf_k >= 0) {
+                cp_async_wait_all();
+                __syncwarp();  // every lane's copies have landed
+                float mr[NT][2], lr[NT][2], ar[C::KS][NT][4];
+                load_frag(pf_acc, pf_ml, false, mr, lr, ar);
+                merge2(m, l, acc, mr, lr, ar);
+            }
         }
         constexpr int kPair = NT == 1 ? 2 : 1;  // records in flight at once
-        for (int k0 = own + 1; split && k0 < si.nseg; k0 += kPair) {
+        for (int k0 = k_from; split && k0 < si.nseg; k0 += kPair) {
             float mr[kPair][NT][2], lr[kPair][NT][2], ar[kPair][C::KS][NT][4];
             bool use[kPair];
 #pragma unroll
             for (int k = 0; k < kPair; ++k) {
                 const int kk = k0 + k;
-                use[k] = kk < si.nseg && kk != pf_k;
+                use[k] = kk < si.nseg && kk != own && kk != pf_k;
                 if (use[k]) load_rec(rec_of(kk), mr[k], lr[k], ar[k]);
             }
 #pragma unroll
@@ -1323,7 +1333,7 @@ __device__ __forceinline__ long long total_chunks_warp(const DecodeParams& p, in
     return t * p.num_hg;
 }
 
-template <int D, int NT, bool F8, bool RC, bool SOLO>
+template <int D, int NT, bool F8, bool RC, bool SOLO, bool APP>
 __global__ void __launch_bounds__(MmaCfg<D, NT, F8, SOLO, RC>::THREADS)
     decode_mma_kernel(const __grid_constant__ DecodeParams p,
                                                              const __grid_constant__ CUtensorMap tmk,
@@ -1398,7 +1408,7 @@ __global__ void __launch_bounds__(MmaCfg<D, NT, F8, SOLO, RC>::THREADS)
 
     // warps: producers | consumers | epilogue
     if (warp < C::NPROD) {
-        Producer<D, NT, F8, RC, SOLO> pr{p, &tmk, &tmv, smem, full, empty, st_ntok, st_bad, ctrl, lane,
+        Producer<D, NT, F8, RC, SOLO, APP> pr{p, &tmk, &tmv, smem, full, empty, st_ntok, st_bad, ctrl, lane,
                            l2_policy_evict_first()};
         pr.me = warp;
         pr.run(it, spec_b, spec_j, spec_tab);
@@ -1558,7 +1568,7 @@ __global__ void __launch_bounds__(32 * kMergeWarps)
 
 // ---- host side ---------------------------------------------------------------
 
-template <int D, int NT, bool F8, bool RC, bool SOLO>
+template <int D, int NT, bool F8, bool RC, bool SOLO, bool APP = false>
 pkv_status launch_impl(const DecodeParams& p, cudaStream_t stream, int* grid_out) {
     using C = MmaCfg<D, NT, F8, SOLO, RC>;
     using S = Smem<D, NT, F8, SOLO, RC>;
@@ -1566,7 +1576,7 @@ pkv_status launch_impl(const DecodeParams& p, cudaStream_t stream, int* grid_out
     if (!di) return PKV_ERR_CUDA;
     static std::mutex mu;
     static int occupancy[64] = {0};
-    auto kern = decode_mma_kernel<D, NT, F8, RC, SOLO>;
+    auto kern = decode_mma_kernel<D, NT, F8, RC, SOLO, APP>;
     {
         std::lock_guard<std::mutex> lock(mu);
         if (di->device >= 64) return PKV_ERR_UNSUPPORTED;
@@ -1700,6 +1710,33 @@ bool decode_mma_supported(int head_dim, int block_size, pkv_dtype q_dtype, pkv_d
            (head_dim == 64 || head_dim == 128) && rows_ok;
 }
 
+// bf16 caches: TMA boxes or row copies, one CTA per SM or two (SOLO), with or
+// without the fused append.
+template <bool APP>
+pkv_status launch_bf16(const DecodeParams& p, int head_dim, int nt, bool many, cudaStream_t stream,
+                       int* grid_out) {
+    if (p.row_copy) {
+        if (head_dim == 128)
+            return nt == 2 ? launch_impl<128, 2, false, true, true, APP>(p, stream, grid_out)
+                   : many  ? launch_impl<128, 1, false, true, true, APP>(p, stream, grid_out)
+                           : launch_impl<128, 1, false, true, false, APP>(p, stream, grid_out);
+        if (head_dim == 64)
+            return nt == 2 ? launch_impl<64, 2, false, true, true, APP>(p, stream, grid_out)
+                   : many  ? launch_impl<64, 1, false, true, true, APP>(p, stream, grid_out)
+                           : launch_impl<64, 1, false, true, false, APP>(p, stream, grid_out);
+    } else {
+        if (head_dim == 128)
+            return nt == 2 ? launch_impl<128, 2, false, false, true, APP>(p, stream, grid_out)
+                   : many  ? launch_impl<128, 1, false, false, true, APP>(p, stream, grid_out)
+                           : launch_impl<128, 1, false, false, false, APP>(p, stream, grid_out);
+        if (head_dim == 64)
+            return nt == 2 ? launch_impl<64, 2, false, false, true, APP>(p, stream, grid_out)
+                   : many  ? launch_impl<64, 1, false, false, true, APP>(p, stream, grid_out)
+                           : launch_impl<64, 1, false, false, false, APP>(p, stream, grid_out);
+    }
+    return PKV_ERR_UNSUPPORTED;
+}
+
 pkv_status launch_decode_mma(const DecodeParams& p, int head_dim, int group_pad, bool fp8,
                              cudaStream_t stream, int* grid_out) {
     const int nt = group_pad > 8 ? 2 : 1;
@@ -1716,24 +1753,10 @@ pkv_status launch_decode_mma(const DecodeParams& p, int head_dim, int group_pad,
                                             : launch_impl<128, 2, true, false, false>(p, stream, grid_out);
         if (head_dim == 64) return nt == 1 ? launch_impl<64, 1, true, false, false>(p, stream, grid_out)
                                            : launch_impl<64, 2, true, false, false>(p, stream, grid_out);
-    } else if (p.row_copy) {
-        if (head_dim == 128)
-            return nt == 2 ? launch_impl<128, 2, false, true, true>(p, stream, grid_out)
-                   : many  ? launch_impl<128, 1, false, true, true>(p, stream, grid_out)
-                           : launch_impl<128, 1, false, true, false>(p, stream, grid_out);
-        if (head_dim == 64)
-            return nt == 2 ? launch_impl<64, 2, false, true, true>(p, stream, grid_out)
-                   : many  ? launch_impl<64, 1, false, true, true>(p, stream, grid_out)
-                           : launch_impl<64, 1, false, true, false>(p, stream, grid_out);
+    } else if (p.k_new) {
+        return launch_bf16<true>(p, head_dim, nt, many, stream, grid_out);
     } else {
-        if (head_dim == 128)
-            return nt == 2 ? launch_impl<128, 2, false, false, true>(p, stream, grid_out)
-                   : many  ? launch_impl<128, 1, false, false, true>(p, stream, grid_out)
-                           : launch_impl<128, 1, false, false, false>(p, stream, grid_out);
-        if (head_dim == 64)
-            return nt == 2 ? launch_impl<64, 2, false, false, true>(p, stream, grid_out)
-                   : many  ? launch_impl<64, 1, false, false, true>(p, stream, grid_out)
-                           : launch_impl<64, 1, false, false, false>(p, stream, grid_out);
+        return launch_bf16<false>(p, head_dim, nt, many, stream, grid_out);
     }
     return PKV_ERR_UNSUPPORTED;
 }
