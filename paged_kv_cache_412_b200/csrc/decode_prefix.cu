@@ -445,8 +445,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
             const unsigned bad = st_bad[st];
             const bool whole = ntok == kPrefixCH && bad == 0;
             const int tbase = c * kPrefixCH;
-            // four independent maximum chains (fmaxf is exact in any order)
-            float mxs[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+            float mx = -INFINITY;
 #pragma unroll
             for (int j = 0; j < kPrefixCH; ++j) {
                 bool ok = tbase + j < L_r;
@@ -455,9 +454,8 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                     ok = ok && j < ntok && !((bad >> jrel) & 1u);
                 }
                 s[j] = ok ? s[j] * sl2 : -INFINITY;
-                mxs[j & 3] = fmaxf(mxs[j & 3], s[j]);
+                mx = fmaxf(mx, s[j]);
             }
-            const float mx = fmaxf(fmaxf(mxs[0], mxs[1]), fmaxf(mxs[2], mxs[3]));
             // lazy maximum: raise it (and rescale O, l) only past a factor 2^8
             const bool raise = mx > m_used + 8.f;
             const float m_new = raise ? mx : m_used;
@@ -501,15 +499,12 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                 uint32_t wh[4], wl[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    // P = hi + lo, both rounded to bf16 on the integer units (the
-                    // conversion pipe is the one the exponentials use)
                     const float p0 = exp2f(s[c8 * 8 + 2 * e] - ref);
                     const float p1 = exp2f(s[c8 * 8 + 2 * e + 1] - ref);
                     l += p0 + p1;
-                    const uint32_t h0 = bf16_rne_bits(p0), h1 = bf16_rne_bits(p1);
-                    wh[e] = pack_bf16_bits(h0, h1);
-                    wl[e] = pack_bf16_bits(bf16_rne_bits(p0 - __uint_as_float(h0)),
-                                           bf16_rne_bits(p1 - __uint_as_float(h1)));
+                    const float h0 = bf16_round(p0), h1 = bf16_round(p1);
+                    wh[e] = pack_bf16(h0, h1);
+                    wl[e] = pack_bf16(p0 - h0, p1 - h1);
                 }
                 *reinterpret_cast<uint4*>(ph + sw128(r, c8)) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
                 *reinterpret_cast<uint4*>(pl + sw128(r, c8)) = make_uint4(wl[0], wl[1], wl[2], wl[3]);

@@ -114,20 +114,6 @@ __device__ __forceinline__ float bf16_round(float x) {
     return __bfloat162float(__float2bfloat16_rn(x));
 }
 
-// x rounded to the nearest bf16 (ties to even), as the bit pattern of that
-// bf16 in the high half of a 32-bit word (the low half zero), computed on the
-// integer units instead of the conversion pipe.  Finite x only (for which it
-// equals cvt.rn.bf16.f32).
-__device__ __forceinline__ uint32_t bf16_rne_bits(float x) {
-    const uint32_t u = __float_as_uint(x);
-    return (u + 0x7FFFu + ((u >> 16) & 1u)) & 0xFFFF0000u;
-}
-
-// Two such words packed as bf16x2 (a in the low half), as pack_bf16 packs.
-__device__ __forceinline__ uint32_t pack_bf16_bits(uint32_t a, uint32_t b) {
-    return __byte_perm(a, b, 0x7632);
-}
-
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
