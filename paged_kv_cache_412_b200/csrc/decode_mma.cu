@@ -749,8 +749,8 @@ __device__ __forceinline__ void consume(const DecodeParams& p, SegIter<kCH>& it,
                     float ps = 0.f;
 #pragma unroll
                     for (int mt = 0; mt < kMT; ++mt) {
-                        s[mt][nt][j] = exp2f(s[mt][nt][j] - mref);
-                        s[mt][nt][j + 2] = exp2f(s[mt][nt][j + 2] - mref);
+                        s[mt][nt][j] = ex2_ftz(s[mt][nt][j] - mref);
+                        s[mt][nt][j + 2] = ex2_ftz(s[mt][nt][j + 2] - mref);
                         ps += s[mt][nt][j] + s[mt][nt][j + 2];
                     }
                     l[nt][j] = fmaf(l[nt][j], alpha[nt][j], ps);

@@ -499,8 +499,8 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                 uint32_t wh[4], wl[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    const float p0 = exp2f(s[c8 * 8 + 2 * e] - ref);
-                    const float p1 = exp2f(s[c8 * 8 + 2 * e + 1] - ref);
+                    const float p0 = ex2_ftz(s[c8 * 8 + 2 * e] - ref);
+                    const float p1 = ex2_ftz(s[c8 * 8 + 2 * e + 1] - ref);
                     l += p0 + p1;
                     const float h0 = bf16_round(p0), h1 = bf16_round(p1);
                     wh[e] = pack_bf16(h0, h1);

@@ -188,7 +188,13 @@ __device__ __forceinline__ void store_out(void* out, size_t idx, float v, int ou
         static_cast<__nv_bfloat16*>(out)[idx] = __float2bfloat16_rn(v);
 }
 
-// 2^x for the softmax (scores are kept in the log2 domain).
-__device__ __forceinline__ float exp2_approx(float x) { return exp2f(x); }
+// 2^x for softmax weights (scores are kept in the log2 domain): the hardware
+// exponential alone (ex2.approx.ftz: about 2 ulp; results below 2^-126 flush
+// to 0, weights that small vanish beside the row maximum's 1; 2^-inf = 0).
+__device__ __forceinline__ float ex2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 }  // namespace pkv
