@@ -7,7 +7,8 @@
  *                                 held in fixed-size physical blocks reached
  *                                 through a per-request block table;
  *   - pkv_paged_attention_decode_append  the append of each request's new
- *                                 token fused into the decode;
+ *                                 token and the decode, in one launch where
+ *                                 the decode's layout allows;
  *   - pkv_copy_blocks             copy-on-write copy of shared blocks;
  *   - pkv_paged_attention_decode_prefix  the same decode with the blocks a
  *                                 group of requests shares read once per group.
@@ -207,7 +208,7 @@ pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache,
 
 /*
  * pkv_paged_attention_decode_append -- each request's new token appended to
- * the cache, then pkv_paged_attention_decode, in one kernel.
+ * the cache, then pkv_paged_attention_decode.
  *
  * [PAMEM] "The Mechanics of PagedAttention": the new token's K and V go to the
  * slot its block table names; "The Math: Block Attention Calculation": the
@@ -216,9 +217,12 @@ pkv_status pkv_paged_attention_decode(const void* q, const void* k_cache,
  * the table names it -- physical block block_tables[b][(L-1)/block_size], row
  * (L-1) % block_size -- the same bytes pkv_kv_cache_write writes for that
  * slot; the decode then runs exactly as pkv_paged_attention_decode (same
- * arguments, same result).  The row is written by the CTA that fetches its
- * block for the decode, just before fetching it, so the append needs no launch
- * and no wait of its own.
+ * arguments, same result).  When the decode runs one CTA per SM (groups of at
+ * most 8 query heads per kv head and fewer than 4 (request, kv head) pairs per
+ * SM), the row is written inside the decode launch, by the CTA that fetches
+ * its block, just before fetching it: one launch.  Otherwise (many short
+ * groups, where that CTA's single producer would be held up) a small append
+ * kernel runs first and the decode overlaps its start: two launches.
  *   k_new, v_new  [num_seqs, num_kv_heads, head_dim] bf16, 16-byte aligned.
  *   Other arguments as pkv_paged_attention_decode.  bf16 q and caches on the
  *   tensor-core path (block_size >= 2, not 1) only: other configurations

@@ -264,12 +264,14 @@ def paged_attention_decode_append(q: torch.Tensor, k_new: torch.Tensor, v_new: t
                                   max_seq_len: int | None = None, partition_size: int = 0,
                                   out_dtype: torch.dtype | None = None,
                                   workspace: torch.Tensor | None = None) -> torch.Tensor:
-    """Append each request's new token, then paged_attention_decode, in one kernel.
+    """Append each request's new token, then paged_attention_decode.
 
     k_new, v_new [B, Hkv, d] bf16: the K and V rows of request b's token at
     position seq_lens[b] - 1, written to the slot its block table names (the
-    bytes kv_cache_write writes there) before the decode reads that block.
-    bf16 q and caches, head_dim 64 or 128, block_size >= 2.
+    bytes kv_cache_write writes there) before the decode reads that block --
+    inside the decode launch when the decode runs one CTA per SM, else by a
+    small kernel launched first.  bf16 q and caches, head_dim 64 or 128,
+    block_size >= 2.
     """
     dev = _need_cuda(q, k_new, v_new, k_cache, v_cache, block_tables, seq_lens, out, workspace)
     if block_tables.dtype != torch.int32 or seq_lens.dtype != torch.int32:

@@ -434,6 +434,18 @@ pkv_status decode_entry(const void* q, const void* k_cache, const void* v_cache,
         const pkv_status ps = launch_decode_prefix(pp, k_cache, v_cache, head_dim, st);
         if (ps != PKV_OK) return ps;
     }
+    if (k_new && !decode_mma_fuses_append(p, group_pad)) {
+        // Many (request, head group) pairs or 16-head groups: one producer per
+        // CTA, which the append would hold up; the append runs first as its
+        // own kernel (the decode overlaps its start through programmatic
+        // dependent launch).
+        p.k_new = p.v_new = nullptr;
+        const pkv_status as = launch_append_by_table(
+            k_new, v_new, block_tables, seq_lens, const_cast<void*>(k_cache),
+            const_cast<void*>(v_cache), num_seqs, num_kv_heads, head_dim, block_size, p.log2_bs,
+            max_blocks_per_seq, num_blocks, st);
+        if (as != PKV_OK) return as;
+    }
     if (mma)
         return launch_decode_mma(p, head_dim, group_pad, kv_dtype == PKV_FP8_E4M3, st, nullptr);
     return launch_decode_simt(p, head_dim, kv_dtype, group_pad, st, nullptr);

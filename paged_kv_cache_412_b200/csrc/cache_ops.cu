@@ -67,6 +67,39 @@ __global__ void kv_cache_write_kernel(const uint4* __restrict__ k, const uint4* 
     }
 }
 
+// Append of each request's new token through its block table (the decode
+// step: request b's token is its last, position L - 1, L = seq_lens[b]
+// clamped to the table's capacity as the decode clamps it): one thread per
+// 16-byte vector of a (request, kv head) row, K and V together.  A request of
+// length 0 appends nothing; an entry outside the pool is skipped (the decode
+// that reads the block flags it).
+__global__ void append_by_table_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
+                                       const int32_t* __restrict__ block_tables,
+                                       const int32_t* __restrict__ seq_lens,
+                                       uint4* __restrict__ kc, uint4* __restrict__ vc,
+                                       long long total_vecs, int vecs_per_row, int num_kv_heads,
+                                       int block_size, int log2_bs, int max_blocks,
+                                       int num_blocks) {
+    griddep_wait();  // the previous kernel may read this cache or write the new rows
+    griddep_launch_dependents();
+    const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= total_vecs) return;
+    const long long row = i / vecs_per_row;  // b * Hkv + h
+    const int vec = (int)(i - row * vecs_per_row);
+    const int b = (int)(row / num_kv_heads);
+    const int h = (int)(row - (long long)b * num_kv_heads);
+    const int L = min(__ldg(seq_lens + b), max_blocks * block_size);
+    if (L <= 0) return;
+    const int t = L - 1;
+    const int phys = __ldg(block_tables + (size_t)b * max_blocks + (t >> log2_bs));
+    if (phys < 0 || phys >= num_blocks) return;
+    const size_t dst =
+        (((size_t)phys * num_kv_heads + h) * block_size + (t & (block_size - 1))) * vecs_per_row + vec;
+    const uint4 kv = __ldg(k + i), vv = __ldg(v + i);
+    kc[dst] = kv;
+    vc[dst] = vv;
+}
+
 // fp8 append: one thread per 16 output bytes (16 elements) of one (token, kv
 // head) row, K and V together.  code = e4m3(x / scale[h]): the quotient is the
 // correctly rounded fp32 division, the conversion rounds to nearest even and
@@ -237,6 +270,25 @@ pkv_status launch_kv_cache_write(const void* k, const void* v, const int64_t* sl
         &L.cfg, kv_cache_write_kernel, static_cast<const uint4*>(k), static_cast<const uint4*>(v),
         slots, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), total, vecs_per_row,
         num_kv_heads, block_size, num_blocks, err);
+    return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
+}
+
+pkv_status launch_append_by_table(const void* k, const void* v, const int32_t* block_tables,
+                                  const int32_t* seq_lens, void* k_cache, void* v_cache,
+                                  int num_seqs, int num_kv_heads, int head_dim, int block_size,
+                                  int log2_bs, int max_blocks, int num_blocks,
+                                  cudaStream_t stream) {
+    const int vecs_per_row = head_dim * 2 / 16;  // bf16 rows
+    const long long total = (long long)num_seqs * num_kv_heads * vecs_per_row;
+    if (total == 0) return PKV_OK;
+    const int threads = 256;
+    const long long grid = (total + threads - 1) / threads;
+    if (grid > 0x7fffffffLL) return PKV_ERR_UNSUPPORTED;
+    PdlLaunch L(dim3((unsigned)grid), dim3(threads), 0, stream);
+    const cudaError_t e = cudaLaunchKernelEx(
+        &L.cfg, append_by_table_kernel, static_cast<const uint4*>(k), static_cast<const uint4*>(v),
+        block_tables, seq_lens, static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache), total,
+        vecs_per_row, num_kv_heads, block_size, log2_bs, max_blocks, num_blocks);
     return e == cudaSuccess ? PKV_OK : PKV_ERR_CUDA;
 }
 

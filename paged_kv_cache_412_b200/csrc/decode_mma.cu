@@ -217,8 +217,8 @@ __device__ __forceinline__ int bf16_row_off(int t, int half, int log2_rb) {
 
 // RC: blocks of 2 or 4 rows (bf16), copied row by row instead of by TMA boxes;
 // a separate instance so the boxed producer carries no trace of it.  APP: the
-// fused append (bf16), likewise a separate instance: a plain decode's chunk
-// loop carries no trace of it.
+// fused append (bf16, one CTA per SM), likewise a separate instance: a plain
+// decode's chunk loop carries no trace of it.
 template <int D, int NT, bool F8, bool RC, bool SOLO, bool APP>
 struct Producer {
     using C = MmaCfg<D, NT, F8, SOLO, RC>;
@@ -252,26 +252,31 @@ struct Producer {
         return (cur.t0 + c0 * kCH) >> log2_bs;
     }
 
-    // Fused append: the request's new token (its last, position L - 1) is in
-    // the chunk about to be issued.  Its K and V rows of this kv head go to
-    // their slot before the chunk's copies are issued (one 16-byte vector per
-    // lane, K on lanes 0 .., V on lanes 16 ..); the proxy fence orders these
-    // generic writes before the copy engine's reads of the block.
-    __device__ __forceinline__ void append_rows(const Cursor& cur, int kvh, int tab, int wbase) {
+    // Fused append.  The new token of request cur.b (its last, position
+    // L - 1): this lane's 16-byte vector of its K (lanes 0 ..) or V (lanes
+    // 16 ..) row of kv head kvh, loaded when the segment that holds it starts,
+    // so the load is in flight while the segment's earlier chunks are issued.
+    static constexpr int kAppVec = D * 2 / 16;  // 16-byte vectors per row
+    __device__ __forceinline__ uint4 append_load(int b, int kvh) const {
+        const size_t src = ((size_t)b * p.num_kv_heads + kvh) * D;
+        const uint4* from = reinterpret_cast<const uint4*>(
+            static_cast<const __nv_bfloat16*>(lane < 16 ? p.k_new : p.v_new) + src);
+        return (lane & 15) < kAppVec ? __ldg(from + (lane & 15)) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    // ... then stored to its slot just before the copies of the chunk that
+    // holds it are issued; the proxy fence orders these generic writes before
+    // the copy engine's reads of the block.
+    __device__ __forceinline__ void append_store(const Cursor& cur, int kvh, int tab, int wbase,
+                                                 uint4 row) {
         const int t = cur.L - 1;
         const int phys = __shfl_sync(FULL_MASK, tab, (t >> p.log2_bs) - wbase);
-        constexpr int VEC = D * 2 / 16;  // 16-byte vectors per row
-        const int v = lane & 15;
-        if (phys >= 0 && phys < p.num_blocks && v < VEC) {
-            const size_t src = ((size_t)cur.b * p.num_kv_heads + kvh) * D;
+        if (phys >= 0 && phys < p.num_blocks && (lane & 15) < kAppVec) {
             const size_t dst = ((size_t)phys * p.num_kv_heads + kvh) * p.block_size * D +
                                (size_t)(t & (p.block_size - 1)) * D;
-            const uint4* from = reinterpret_cast<const uint4*>(
-                static_cast<const __nv_bfloat16*>(lane < 16 ? p.k_new : p.v_new) + src);
             uint4* to = reinterpret_cast<uint4*>(
                 static_cast<__nv_bfloat16*>(const_cast<void*>(lane < 16 ? p.k_cache : p.v_cache)) +
                 dst);
-            to[v] = __ldg(from + v);
+            to[lane & 15] = row;
             fence_proxy_async_global();
         }
         __syncwarp();
@@ -292,6 +297,17 @@ struct Producer {
         int wbase = first_block(cur, sg.c0, p.log2_bs);
         int tab = tab_first;
         int tab_next = (wbase + 32 < nblk) ? load_window(cur, wbase + 32) : -1;
+        uint4 app_row = make_uint4(0u, 0u, 0u, 0u);
+        if constexpr (APP) {
+            if (!waited) {
+                griddep_wait();  // the new rows may come from the previous kernel
+                waited = true;
+            }
+            // this producer issues the group's last chunk (the new token's)
+            const unsigned n_last = n_chunk + (unsigned)(sg.c1 - 1 - sg.c0);
+            if (sg.c1 == cur.nch && (C::NPROD == 1 || (int)(n_last % C::NPROD) == me))
+                app_row = append_load(cur.b, kvh);
+        }
         for (int c = sg.c0; c < sg.c1; ++c) {
             const int t0 = cur.t0 + c * kCH;
             const int ntok = min(kCH, cur.L - t0);
@@ -337,7 +353,7 @@ struct Producer {
                     ++nvalid;
             }
             if constexpr (APP) {
-                if (c == cur.nch - 1) append_rows(cur, kvh, tab, wbase);
+                if (c == cur.nch - 1) append_store(cur, kvh, tab, wbase, app_row);
             }
             unsigned char* sk = smem + stage * C::STAGE_BYTES;
             unsigned char* sv = sk + C::KV_BYTES;
@@ -1715,6 +1731,17 @@ bool decode_mma_supported(int head_dim, int block_size, pkv_dtype q_dtype, pkv_d
 template <bool APP>
 pkv_status launch_bf16(const DecodeParams& p, int head_dim, int nt, bool many, cudaStream_t stream,
                        int* grid_out) {
+    if constexpr (APP) {
+        // the append rides only in the one-CTA-per-SM layout (decode_mma_fuses_append)
+        if (nt == 2 || many) return PKV_ERR_UNSUPPORTED;
+        if (head_dim == 128)
+            return p.row_copy ? launch_impl<128, 1, false, true, false, true>(p, stream, grid_out)
+                              : launch_impl<128, 1, false, false, false, true>(p, stream, grid_out);
+        if (head_dim == 64)
+            return p.row_copy ? launch_impl<64, 1, false, true, false, true>(p, stream, grid_out)
+                              : launch_impl<64, 1, false, false, false, true>(p, stream, grid_out);
+        return PKV_ERR_UNSUPPORTED;
+    }
     if (p.row_copy) {
         if (head_dim == 128)
             return nt == 2 ? launch_impl<128, 2, false, true, true, APP>(p, stream, grid_out)
@@ -1737,6 +1764,18 @@ pkv_status launch_bf16(const DecodeParams& p, int head_dim, int nt, bool many, c
     return PKV_ERR_UNSUPPORTED;
 }
 
+// Many (request, head group) pairs: at least four per SM.  Then two CTAs per
+// SM (one consumer and one epilogue warp each) share the many short segments
+// better than one CTA with two consumers.
+static bool many_groups(const DecodeParams& p, int num_sms) {
+    return (long long)p.num_seqs * p.num_hg >= 4LL * num_sms;
+}
+
+bool decode_mma_fuses_append(const DecodeParams& p, int group_pad) {
+    const DeviceInfo* di = current_device_info();
+    return di && group_pad <= 8 && !many_groups(p, di->num_sms);
+}
+
 pkv_status launch_decode_mma(const DecodeParams& p, int head_dim, int group_pad, bool fp8,
                              cudaStream_t stream, int* grid_out) {
     const int nt = group_pad > 8 ? 2 : 1;
@@ -1746,7 +1785,7 @@ pkv_status launch_decode_mma(const DecodeParams& p, int head_dim, int group_pad,
     // epilogue warp each) share the many short segments better.
     const DeviceInfo* di = current_device_info();
     if (!di) return PKV_ERR_CUDA;
-    const bool many = (long long)p.num_seqs * p.num_hg >= 4LL * di->num_sms;
+    const bool many = many_groups(p, di->num_sms);
     if (fp8) {
         if (p.row_copy) return PKV_ERR_UNSUPPORTED;
         if (head_dim == 128) return nt == 1 ? launch_impl<128, 1, true, false, false>(p, stream, grid_out)

@@ -193,6 +193,18 @@ pkv_status launch_kv_cache_write(const void* k, const void* v, const int64_t* sl
                                  int head_dim, int block_size, int num_blocks, int elem_bytes,
                                  unsigned* err, cudaStream_t stream);
 
+// Each request's new token (position seq_lens[b] - 1) appended through its
+// block table: bf16 rows k[b], v[b] of [num_seqs, num_kv_heads, head_dim].
+pkv_status launch_append_by_table(const void* k, const void* v, const int32_t* block_tables,
+                                  const int32_t* seq_lens, void* k_cache, void* v_cache,
+                                  int num_seqs, int num_kv_heads, int head_dim, int block_size,
+                                  int log2_bs, int max_blocks, int num_blocks,
+                                  cudaStream_t stream);
+
+// Whether the tensor-core decode of this call appends inside its own launch
+// (the one-CTA-per-SM layout); otherwise the append runs as its own kernel.
+bool decode_mma_fuses_append(const DecodeParams& p, int group_pad);
+
 pkv_status launch_kv_cache_write_fp8(const void* k, const void* v, const int64_t* slots,
                                      void* k_cache, void* v_cache, const float* k_scale,
                                      const float* v_scale, int num_tokens, int num_kv_heads,
