@@ -182,10 +182,13 @@ def test_fused_append_in_cuda_graph(pkv):
     assert pkv.get_device_error() == 0
 
 
-def test_new_token_in_bad_block_is_skipped_and_flagged(pkv):
+@pytest.mark.parametrize("Hq,Hkv", [(8, 2), (16, 1)], ids=["in_launch", "append_kernel"])
+def test_new_token_in_bad_block_is_skipped_and_flagged(pkv, Hq, Hkv):
     """The new token's table entry outside the pool: nothing is written
-    anywhere (the caches stay as they were) and PKV_DEVERR_BAD_BLOCK is set."""
-    w = workloads.make_paged([100, 40], Hq=8, Hkv=2, d=128, bs=16, dtype="bf16", seed=21)
+    anywhere (the caches stay as they were) and PKV_DEVERR_BAD_BLOCK is set.
+    8-head groups append inside the decode launch; 16-head groups through the
+    separate append kernel."""
+    w = workloads.make_paged([100, 40], Hq=Hq, Hkv=Hkv, d=128, bs=16, dtype="bf16", seed=21)
     bt = w.block_tables.copy()
     bt[1, (40 - 1) // 16] = w.num_blocks + 5
     dw = DevWorkload(w)
