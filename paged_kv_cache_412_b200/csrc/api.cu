@@ -47,7 +47,7 @@ int prefix_splits_for(int num_sms, int num_prefixes, int num_kv_heads, int row_t
     const long long base = (long long)num_prefixes * num_kv_heads * row_tiles;
     const long long nch = (max_prefix_len + 63) / 64;
     if (base <= 0 || nch <= 0) return 1;
-    long long s = (long long)num_sms / base;
+    long long s = (long long)num_sms * kPrefixCtasPerSm / base;
     s = std::min(s, nch);
     s = std::min(s, 64LL);
     return (int)std::max(s, 1LL);

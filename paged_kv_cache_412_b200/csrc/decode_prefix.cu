@@ -14,8 +14,11 @@
 // over 128 lanes, one lane per row.  One thread of the MMA warp issues the
 // MMAs; four softmax warps (one per 32-lane quarter of tensor memory, one row
 // per thread) read S with tcgen05.ld, mask it, run the online softmax in base
-// 2 and write P, split into bf16 hi + lo, to shared memory in the 128-byte
-// swizzled K-major layout the P.V MMA reads.  The running maximum is raised
+// 2 and write P, split into bf16 hi + lo, back into the S buffer it came from
+// (hi in its first 32 columns, lo in the next 32, two bf16 per column), where
+// the P.V MMA reads it as its A operand (no shared-memory P, no store and
+// proxy fence per chunk); the MMAs of one thread execute in order, so the next
+// S into that buffer follows the P.V that reads it.  The running maximum is raised
 // lazily: O (in tensor memory) is rescaled only when a row's maximum grows by
 // more than 8 (a factor 256), so the weights stay below 2^8 and the result is
 // exact whatever maximum is used, as long as O and the row sum l use the same.
@@ -59,17 +62,15 @@ struct PCfg {
     static constexpr int KV_BYTES = NHALF * HALF_BYTES;
     static constexpr int STAGE_BYTES = 2 * KV_BYTES;   // K | V, whole KB
     static constexpr int QHALF = kPrefixRows * 128;    // one 64-column half of the Q tile
-    static constexpr int P_BYTES = kPrefixRows * 128;  // 128 rows x 64 tokens of bf16
     static constexpr int OFF_Q = kStagesP * STAGE_BYTES;
-    static constexpr int OFF_P = OFF_Q + NHALF * QHALF;  // [2 buffers][hi, lo]
-    static constexpr int OFF_BAR = OFF_P + 4 * P_BYTES;
+    static constexpr int OFF_BAR = OFF_Q + NHALF * QHALF;
     // full, empty per stage; s_full, s_free, p_full, pv_done per buffer; q_ready; drain
     static constexpr int NBAR = 2 * kStagesP + 4 * 2 + 2;
     static constexpr int OFF_META = OFF_BAR + NBAR * 8;
     static constexpr int OFF_ROWS = OFF_META + 2 * kStagesP * 4;
     static constexpr int OFF_CTRL = OFF_ROWS + 3 * kPrefixRows * 4;
     static constexpr int BYTES = OFF_CTRL + 32 + 1024;  // + alignment slack
-    static_assert(BYTES <= 227 * 1024, "within the opt-in shared memory of one CTA");
+    static_assert(BYTES * kPrefixCtasPerSm <= 227 * 1024, "kPrefixCtasPerSm CTAs per SM");
 };
 
 // Instruction descriptors: S = Q.K^T (M 128, N 64, B K-major) and
@@ -85,7 +86,7 @@ struct PIdesc {
 __device__ __forceinline__ uint32_t sw128(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
 
 template <int D>
-__global__ void __launch_bounds__(kThreadsP, 1)
+__global__ void __launch_bounds__(kThreadsP, kPrefixCtasPerSm)
     prefix_kernel(const __grid_constant__ PrefixParams p, const __grid_constant__ CUtensorMap tmk,
                   const __grid_constant__ CUtensorMap tmv) {
     using C = PCfg<D>;
@@ -95,8 +96,8 @@ __global__ void __launch_bounds__(kThreadsP, 1)
     uint64_t* empty = full + kStagesP;
     uint64_t* s_full = empty + kStagesP;  // S buffer b holds a chunk's scores
     uint64_t* s_free = s_full + 2;        // the softmax warps have read S buffer b
-    uint64_t* p_full = s_free + 2;        // P buffer b (and any O rescale) is ready
-    uint64_t* pv_done = p_full + 2;       // the P.V MMAs reading P buffer b completed
+    uint64_t* p_full = s_free + 2;        // P in S buffer b (and any O rescale) is ready
+    uint64_t* pv_done = p_full + 2;       // the P.V MMAs reading S buffer b's P completed
     uint64_t* q_ready = pv_done + 2;      // the Q tile is in shared memory
     uint64_t* drain = q_ready + 1;        // every MMA this CTA issued has completed
     int* st_ntok = reinterpret_cast<int*>(smem + C::OFF_META);
@@ -328,7 +329,6 @@ __global__ void __launch_bounds__(kThreadsP, 1)
         // ---- MMA issue (one thread) ----
         if (lane == 0 && n_local > 0) {
             const uint32_t qb = smem_addr(smem + C::OFF_Q);
-            const uint32_t pb = smem_addr(smem + C::OFF_P);
             const uint32_t sb = smem_addr(smem);
             bool ok = mbar_wait(q_ready, 0);
             tc_fence_after();
@@ -365,13 +365,14 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                 const uint32_t vb = sb + st * C::STAGE_BYTES + C::KV_BYTES;
 #pragma unroll
                 for (int part = 0; part < 2; ++part) {  // P hi, then P lo
-                    const uint32_t pa = pb + (2 * b + part) * C::P_BYTES;
+                    // P of chunk i: columns [32 part, 32 part + 32) of S buffer b,
+                    // 16 tokens (8 columns) per MMA
+                    const uint32_t pa = tmem + kSCol + b * kPrefixCH + part * (kPrefixCH / 2);
 #pragma unroll
                     for (int kt = 0; kt < kPrefixCH / 16; ++kt) {
-                        const uint64_t a = smem_desc_sw128(pa + kt * 32, 16, 1024);
                         const uint64_t bd = smem_desc_sw128(vb + kt * 16 * 128, C::HALF_BYTES, 1024);
                         const uint32_t acc = (i == 0 && part == 0 && kt == 0) ? 0u : 1u;
-                        umma_bf16(tmem + kOCol, a, bd, PIdesc<D>::PV, acc);
+                        umma_bf16_ts(tmem + kOCol, pa + kt * 8, bd, PIdesc<D>::PV, acc);
                     }
                 }
                 umma_commit(&empty[st]);   // the K/V stage may be refilled
@@ -484,31 +485,25 @@ __global__ void __launch_bounds__(kThreadsP, 1)
             }
             m_used = m_new;
             const float ref = m_used == -INFINITY ? 0.f : m_used;
-            // P buffer b was last read by the P.V MMAs of chunk i - 2
-            if (!__all_sync(FULL_MASK, mbar_wait(&pv_done[b], ((i >> 1) & 1u) ^ 1u))) {
-                if (lane == 0 && !ctrl[0]) {
-                    ctrl[0] = 1;
-                    raise_error(p.err, PKV_DEVERR_TIMEOUT);
-                }
-                break;
-            }
-            unsigned char* ph = smem + C::OFF_P + (2 * b) * C::P_BYTES;
-            unsigned char* pl = ph + C::P_BYTES;
+            // P into S buffer b (its scores are in registers): hi in columns
+            // [0, 32), lo in [32, 64), two tokens per column, 32 tokens at a time
+            const uint32_t pcol = trow + kSCol + b * kPrefixCH;
 #pragma unroll
-            for (int c8 = 0; c8 < kPrefixCH / 8; ++c8) {
-                uint32_t wh[4], wl[4];
+            for (int hq = 0; hq < 2; ++hq) {
+                uint32_t wh[16], wl[16];
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float p0 = ex2_ftz(s[c8 * 8 + 2 * e] - ref);
-                    const float p1 = ex2_ftz(s[c8 * 8 + 2 * e + 1] - ref);
+                for (int e = 0; e < 16; ++e) {
+                    const float p0 = ex2_ftz(s[hq * 32 + 2 * e] - ref);
+                    const float p1 = ex2_ftz(s[hq * 32 + 2 * e + 1] - ref);
                     l += p0 + p1;
                     const float h0 = bf16_round(p0), h1 = bf16_round(p1);
                     wh[e] = pack_bf16(h0, h1);
                     wl[e] = pack_bf16(p0 - h0, p1 - h1);
                 }
-                *reinterpret_cast<uint4*>(ph + sw128(r, c8)) = make_uint4(wh[0], wh[1], wh[2], wh[3]);
-                *reinterpret_cast<uint4*>(pl + sw128(r, c8)) = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+                tmem_st16(pcol + hq * 16, wh);
+                tmem_st16(pcol + kPrefixCH / 2 + hq * 16, wl);
             }
+            tmem_wait_st();
             if (!whole) {
                 // V rows of tokens that do not take part (past the chunk's end or
                 // in a bad block) hold stale or poisoned data: zero them so that
@@ -522,7 +517,7 @@ __global__ void __launch_bounds__(kThreadsP, 1)
                                                   (rest & 7) * 16) = make_uint4(0, 0, 0, 0);
                 }
             }
-            fence_proxy_async_smem();  // P (and zeroed V rows) -> the tensor cores' reads
+            if (!whole) fence_proxy_async_smem();  // zeroed V rows -> the tensor cores' reads
             tc_fence_before();
             mbar_arrive(&p_full[b]);
         }

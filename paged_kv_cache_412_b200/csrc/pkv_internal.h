@@ -150,6 +150,11 @@ struct PrefixParams {
 
 // Rows of (member, query head) pairs one CTA of the shared pass covers.
 constexpr int kPrefixRows = 128;
+// CTAs of the shared pass resident per SM; the launch sizes its splits for one
+// wave of that many.  (Two fit -- 256 tensor-memory columns and under half the
+// shared memory each -- but doubled the partial records to merge and shared one
+// SM's issue slots between two softmax chains: slower.)
+constexpr int kPrefixCtasPerSm = 1;
 
 pkv_status launch_decode_prefix(const PrefixParams& p, const void* k_cache, const void* v_cache,
                                 int head_dim, cudaStream_t stream);
