@@ -5,10 +5,12 @@ One step = one pass of the hot path over one batch of the 4k-token decode
 workload (batch 16 x 4096 tokens, 32 q / 8 KV heads, head_dim 128, block 16,
 bf16): copy-on-write block copy (none are due in this workload: no block is
 shared), the KV-cache append of the batch's 16 new tokens, then paged decode
-attention over all 4096 tokens of every request.  Inputs are synthetic
-(seeded N(0,1) values, randomly permuted block pool) and resident in HBM
-before the timed region.  Each step uses the next of 4 layer pools (268 MB of
-K+V each, 1.07 GB in all), so every step reads KV that is not in the 126 MB L2.
+attention over all 4096 tokens of every request (the append inside the decode
+launch).  Inputs are synthetic (seeded N(0,1) values, randomly permuted block
+pool) and resident in HBM before the timed region.  Each step uses the next
+of 4 layer pools (268 MB of K+V each, 1.07 GB in all), so every step reads KV
+that is not in the 126 MB L2; the 32 steps of a 32-layer model's decode
+iteration form one CUDA graph.
 
 Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle (the
 only other implementation of the path) on a bounded sample instead.
@@ -43,8 +45,9 @@ NOMINAL_HBM_GBS = 8000.0  # the B200's ~8 TB/s HBM3e figure, for the nominal fra
 ROOFLINE_LAUNCHES = 2000  # decode-append launches timed for the roofline, whatever --steps
 DEC_RUN = 20               # back-to-back decode-append launches per timed graph (roofline)
 ISOLATED_LAUNCHES = 200    # single decode-append launches timed on their own (latency)
-SEPARATE_SWEEPS = 50       # sweeps timed for the step with the append as its own launch
-N_LAYERS = 4
+SEPARATE_SWEEPS = 10       # iterations timed for the step with the append as its own launch
+N_LAYERS = 4               # distinct K/V pools (1.07 GB together: every step reads HBM)
+STEPS_PER_GRAPH = 32       # steps of one decode iteration of a 32-layer model, one CUDA graph
 DECODE_SRC = os.path.join(ROOT, "paged_kv_cache_412_b200", "csrc", "decode_mma.cu")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_gqa_4k_traffic.txt")
 
@@ -390,21 +393,24 @@ def run_ours(args, rank: int, world: int, local: int):
     assert pkv.get_device_error() == 0
 
     # A decode iteration of a model runs the step once per layer, back to
-    # back: one CUDA graph holds a sweep over the N_LAYERS layer pools (a step
-    # per layer), so consecutive kernels overlap through programmatic
-    # dependent launch as they would in the serving loop; a second graph holds
-    # the first K % N_LAYERS steps of a sweep.
+    # back: one CUDA graph holds the STEPS_PER_GRAPH steps of an iteration of
+    # a 32-layer model (layer l reads pool l % N_LAYERS, which the three other
+    # pools have evicted from L2 since its last visit), so consecutive kernels
+    # overlap through programmatic dependent launch as they would in the
+    # serving loop; a second graph holds the first K % STEPS_PER_GRAPH steps.
     def capture(steps, with_write, fused=True):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
             for li in range(steps):
                 step_body(layers[li % N_LAYERS], with_write, fused)
         return g
-    sweep = capture(N_LAYERS, True)
-    n_sweeps, rest = divmod(args.steps, N_LAYERS)
+    sweep = capture(STEPS_PER_GRAPH, True)
+    n_sweeps, rest = divmod(args.steps, STEPS_PER_GRAPH)
     part = capture(rest, True) if rest else None
-    for _ in range(max(1, -(-args.warmup // N_LAYERS))):
+    for _ in range(max(1, -(-args.warmup // STEPS_PER_GRAPH))):
         sweep.replay()
+    if part is not None:  # a graph's first launch also uploads it: not inside the timing
+        part.replay()
     torch.cuda.synchronize()
 
     # --- timed region: K steps (graph replays), device-timed ---
@@ -428,15 +434,15 @@ def run_ours(args, rank: int, world: int, local: int):
     clocks = sampler.stop()
     ms_total = bounds[0].elapsed_time(bounds[-1])
     # per-step time of each full sweep (the partial sweep only counts in the total)
-    step_ms = [bounds[i].elapsed_time(bounds[i + 1]) / N_LAYERS for i in range(n_sweeps)] or \
+    step_ms = [bounds[i].elapsed_time(bounds[i + 1]) / STEPS_PER_GRAPH for i in range(n_sweeps)] or \
               [ms_total / args.steps]
     ms_total_max = dist_max(ms_total, world)
     ms_step = ms_total_max / args.steps
     del sweep, part
 
     # The same step with the append as its own launch (kv_cache_write, then
-    # the decode): sweeps of N_LAYERS steps, events around each sweep.
-    sep = capture(N_LAYERS, True, fused=False)
+    # the decode): graphs of STEPS_PER_GRAPH steps, events around each.
+    sep = capture(STEPS_PER_GRAPH, True, fused=False)
     for _ in range(3):
         sep.replay()
     torch.cuda.synchronize()
@@ -447,7 +453,7 @@ def run_ours(args, rank: int, world: int, local: int):
         sep.replay()
         b.record()
     torch.cuda.synchronize()
-    sep_ms = statistics.median(a.elapsed_time(b) / N_LAYERS for a, b in sep_ev)
+    sep_ms = statistics.median(a.elapsed_time(b) / STEPS_PER_GRAPH for a, b in sep_ev)
     del sep
     assert pkv.get_device_error() == 0
 
@@ -624,14 +630,15 @@ def run_ours(args, rank: int, world: int, local: int):
             "data": "synthetic",
             "config": {"workload": WORKLOAD, "global_batch": B * world, "seq_len": L,
                        "num_q_heads": Hq, "num_kv_heads": Hkv, "head_dim": d, "block_size": bs,
-                       "layers_rotated": N_LAYERS,
+                       "layers_rotated": N_LAYERS, "steps_per_graph": STEPS_PER_GRAPH,
                        "l2": f"inputs larger than L2: {N_LAYERS} layer pools of "
                              f"{2 * B * L * Hkv * d * 2 / 1e6:.0f} MB K+V rotated per step",
                        "parallelism": f"replica x{world}" if world > 1 else "single GPU",
                        "step": "copy_blocks (0 pairs) + paged_attention_decode_append "
                                "(the 16 new tokens appended inside the decode launch); the "
-                               f"steps of a sweep over the {N_LAYERS} layer pools captured "
-                               "in one CUDA graph and replayed back to back"},
+                               f"{STEPS_PER_GRAPH} steps of a 32-layer model's decode "
+                               "iteration (layer l on pool l mod "
+                               f"{N_LAYERS}) captured in one CUDA graph, replayed back to back"},
             "tokens_per_s": round(B * world * args.steps / (ms_total_max / 1e3), 1),
             "context_tokens_per_s": round(B * L * world * args.steps / (ms_total_max / 1e3), 1),
             "fraction_of_hbm_peak": round(value / peak, 4),
@@ -643,7 +650,7 @@ def run_ours(args, rank: int, world: int, local: int):
                 "GBps": round(dbytes / (sep_ms / 1e3) / 1e9, 2),
                 "note": "the same step with the append as its own launch (copy_blocks + "
                         "kv_cache_write + paged_attention_decode), median over "
-                        f"{SEPARATE_SWEEPS} sweeps of the layer pools"},
+                        f"{SEPARATE_SWEEPS} graphs of {STEPS_PER_GRAPH} steps"},
             "decode_ms_avg": round(dec_avg_ms, 5), "decode_ms_median": round(dec_med_ms, 5),
             "decode_launches_timed": n_dec,
             "decode_only_ms_avg": round(dec_only_ms, 5),
