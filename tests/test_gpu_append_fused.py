@@ -145,10 +145,12 @@ def test_length_one_returns_new_v_row(pkv):
             np.testing.assert_array_equal(got[b, h], vnew[b, h // 4])
 
 
-def test_fused_append_in_cuda_graph(pkv):
+@pytest.mark.parametrize("Hq,Hkv", [(32, 8), (32, 2)], ids=["in_launch", "append_kernel"])
+def test_fused_append_in_cuda_graph(pkv, Hq, Hkv):
     """Captured once, replayed twice: the append writes the same rows again
-    and the output is unchanged."""
-    w = workloads.make_paged([300, 17, 1000], Hq=32, Hkv=8, d=128, bs=16, dtype="bf16", seed=11)
+    and the output is unchanged.  8-head groups append inside the decode
+    launch; 16-head groups through the append kernel launched before it."""
+    w = workloads.make_paged([300, 17, 1000], Hq=Hq, Hkv=Hkv, d=128, bs=16, dtype="bf16", seed=11)
     kc_ref, vc_ref = host_step(w)
     ref = oracle.decode(w.q, kc_ref, vc_ref, w.block_tables, w.seq_lens, w.scale)
     dw = DevWorkload(w)
