@@ -88,12 +88,17 @@ struct MmaCfg {
     //     per SM with one consumer each, for calls of many (request, head
     //     group) pairs, where few groups split and two epilogue warps per SM
     //     share the many short segments.
+    //   bf16, 8-head groups, row copies (blocks of 2 or 4 rows): three
+    //     consumers -- each tile's rows come from several blocks (per-row
+    //     addresses) and q from global memory, work two consumers left
+    //     exposed (block size 4: 60.1 -> 53.3 us back to back); the TMA
+    //     path is better with two.
     //   fp8: widening codes costs instructions and latency the bf16 path does
     //     not have, and one consumer warp cannot hide its own ldmatrix -> cvt
     //     -> mma chains: six consumers (two on each of two SM sub-partitions)
     //     overlap them; the 16-head configuration keeps four (its consumers
     //     need all the registers).
-    static constexpr int NCONS = F8 ? (NT == 1 ? 6 : 4) : (NT == 1 && !SOLO ? 2 : 1);
+    static constexpr int NCONS = F8 ? (NT == 1 ? 6 : 4) : (NT == 1 && !SOLO ? (RC ? 3 : 2) : 1);
     // bf16: K | V | q, rounded to the 1 KB the 128-byte swizzle pattern
     // repeats on, or the row-copy regions if larger; the first NCONS stages
     // of a segment -- each consumer's first chunk of it -- carry the group's q
