@@ -73,6 +73,8 @@ CASES = [
     ([70, 200, 5], 10, 2, 128, 4),                # row copies of 4-row blocks
     ([70, 200, 5, 64], 8, 2, 128, 2),             # row copies of 2-row blocks
     ([130, 1, 64], 16, 1, 64, 4),                 # d 64, G = 16, block size 4
+    ([130, 1, 64, 700], 8, 2, 64, 4),             # d 64, G = 4, block size 4, in launch
+    ([257, 33, 900], 16, 2, 64, 2),               # d 64, G = 8, block size 2, in launch
     ([300, 129], 8, 2, 128, 64),
     ([700, 129], 32, 8, 128, 128),                # block larger than a chunk
     ([513, 20, 300], 8, 4, 64, 256),

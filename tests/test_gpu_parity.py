@@ -70,6 +70,8 @@ SMALL = [
     ([70, 200, 5], 10, 2, 128, 4, "bf16"),       # G = 5
     ([70, 200, 5, 64], 8, 2, 128, 2, "bf16"),    # block size 2 (bulk copies of 2-row runs)
     ([130, 1, 64], 16, 1, 64, 4, "bf16"),        # block size 4, d 64, G = 16
+    ([130, 1, 64, 700], 8, 2, 64, 4, "bf16"),    # block size 4, d 64, G = 4 (one CTA per SM)
+    ([257, 33, 900], 16, 2, 64, 2, "bf16"),      # block size 2, d 64, G = 8 (one CTA per SM)
     ([257, 33, 4096], 32, 8, 128, 2, "bf16"),    # block size 2, split groups
     ([300, 129], 8, 2, 128, 64, "bf16"),         # block larger than a stage
     ([513, 20], 8, 4, 64, 256, "f32"),           # block size 256
